@@ -1,0 +1,199 @@
+/*
+ * mk.h -- C-ABI of libmk: batch-1 (and small-batch) transformer decoding on
+ * one B200 (sm_100a), each decode step run as ONE persistent megakernel.
+ *
+ * The method ("LLMs in einen MegaKernel kompilieren, um Low-Latency-Inferenz
+ * zu ermöglichen", de.news.hada.io/topic?id=21563, sections "Part 1.
+ * Compiler" and "Part 2. Laufzeit"; "MPK: A Compiler and Runtime for
+ * Mega-Kernelizing Tensor Programs", gist.science/hi/paper/2512.22219,
+ * sections 1-4): the operators of a decode step are cut into SM-sized tasks
+ * linked by event counters instead of kernel boundaries; one kernel with one
+ * CTA per SM runs every task; a finished task bumps an event counter, and a
+ * task whose event reached its threshold may run.  Here a host-side builder
+ * makes the task graph once at mk_create; each CTA gets an ahead-of-time task
+ * queue; inside each CTA a scheduler warp waits on the events, a producer warp
+ * streams bf16 weights with bulk copies (TMA) into a shared-memory ring that
+ * runs ahead across task and layer boundaries, and worker warps compute.
+ *
+ * The model: embedding table, then transformer blocks (pre-norm RMSNorm,
+ * fused QKV projection with optional bias, rotate-half RoPE, KV-cache append,
+ * grouped-query attention, O projection + residual, RMSNorm, SwiGLU FFN +
+ * residual), final RMSNorm, LM head, greedy argmax ("Crear desde cero un
+ * motor de inferencia para LLM usando C++ y CUDA", es.news.hada.io/topic?id=
+ * 18295, §1 and §1.1; "LLM高速化勉強会資料" slides 4-6, 9, 28).
+ *
+ * Conventions for every entry point:
+ *   - Return 0 on success or a negative MK_ERR_* code.  Argument errors are
+ *     found on the host before anything is enqueued.  Device-side errors
+ *     (a wait that timed out, a token id out of range) are reported by
+ *     mk_status; after one the context is poisoned and every later call
+ *     returns MK_ERR_POISONED.  mk_last_error gives a one-line reason.
+ *   - "_dev" pointers are CUDA device pointers, "_host" pointers host memory.
+ *   - Work is enqueued on the stream given to mk_create and the call returns
+ *     without synchronising (except mk_status, mk_decode_step_host and
+ *     mk_create, which synchronise that stream).  Results are valid after a
+ *     stream synchronisation.
+ *   - One context is not thread-safe; different contexts are independent.
+ */
+#ifndef MK_H
+#define MK_H
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MK_OK 0
+#define MK_ERR_INVALID_ARG -1  /* bad pointer, size or configuration */
+#define MK_ERR_OOM -2          /* device allocation failed */
+#define MK_ERR_CUDA -3         /* a CUDA runtime call failed */
+#define MK_ERR_TIMEOUT -4      /* a device-side event wait ran out of time */
+#define MK_ERR_POS_RANGE -5    /* position outside [0, max_seq) */
+#define MK_ERR_NOT_RESIDENT -6 /* one CTA per SM cannot be co-resident */
+#define MK_ERR_POISONED -7     /* an earlier device error; destroy the context */
+#define MK_ERR_TOKEN_RANGE -8  /* a token id outside [0, vocab) reached the device */
+#define MK_ERR_UNSUPPORTED -9  /* valid request this build does not implement */
+
+/* Execution modes of a decode step. */
+#define MK_MODE_MEGAKERNEL 0   /* one persistent launch per step (the product) */
+#define MK_MODE_PER_OP 1       /* the same task bodies, one launch per operator */
+#define MK_MODE_PER_OP_GRAPH 2 /* MK_MODE_PER_OP captured once and replayed as a CUDA graph */
+
+/* Decoder shape.  Sizes in elements.  Limits of this build: head_dim 64 or
+ * 128; hidden and ffn multiples of 8 and at most 16384; n_q_heads a multiple
+ * of n_kv_heads; max_batch 1..8. */
+typedef struct {
+  int n_layers, hidden, n_q_heads, n_kv_heads, head_dim, ffn, vocab;
+  float rms_eps;
+  double rope_theta;
+  int qkv_bias;        /* 1: q/k/v projections carry a bias (Qwen2 family) */
+  int tied_embeddings; /* 1: the LM head is the embedding table */
+  int max_seq;         /* positions per request: 0 .. max_seq-1 */
+  int max_batch;       /* requests decoded together per step */
+} mk_config;
+
+/* bf16 device pointers in the natural layout, [out_features][in_features]
+ * row-major: wq [n_q_heads*head_dim][hidden], wk/wv [n_kv_heads*head_dim]
+ * [hidden], wo [hidden][n_q_heads*head_dim], w_gate/w_up [ffn][hidden],
+ * w_down [hidden][ffn], norms [hidden], biases [out_features] (NULL without
+ * qkv_bias).  mk_create copies and re-packs everything into memory it owns;
+ * the caller may free these afterwards. */
+typedef struct {
+  const void *attn_norm, *wq, *wk, *wv, *bq, *bk, *bv, *wo;
+  const void *ffn_norm, *w_gate, *w_up, *w_down;
+} mk_layer_weights;
+
+typedef struct {
+  const void* embed;              /* [vocab][hidden] */
+  const mk_layer_weights* layers; /* host array of n_layers entries */
+  const void* final_norm;         /* [hidden] */
+  const void* lm_head;            /* [vocab][hidden]; NULL when tied */
+} mk_weights;
+
+/* Optional knobs (pass NULL for defaults). */
+typedef struct {
+  int num_ctas;      /* 0: one CTA per SM of the device */
+  int attn_splits;   /* 0: automatic split-KV factor per KV head */
+  int timeout_ms;    /* device-side wait limit per event (0: 1000 ms) */
+  int mode;          /* MK_MODE_* used by mk_decode_step and mk_prefill */
+} mk_options;
+
+typedef struct mk_ctx mk_ctx;
+
+/* Builds the task graph, packs the weights, allocates the KV cache and the
+ * activation scratch, uploads the RoPE table and checks that one CTA per SM
+ * can be co-resident.  `stream` is a cudaStream_t (NULL: the legacy default
+ * stream).  On success *out owns ~(weights + KV cache) of device memory. */
+int mk_create(const mk_config* cfg, const mk_weights* w, const mk_options* opt, void* stream,
+              mk_ctx** out);
+
+/* Prefill ("LLM高速化勉強会資料" slide 9; "Crear desde cero ..." §1.1): runs
+ * the prompt of each request through the model and fills its KV cache at
+ * positions 0..len-1.  Requests are packed as one flat token sequence
+ * ("LLM高速化勉強会資料" slides 14-16): request r owns tokens
+ * [offsets_host[r], offsets_host[r+1]) of tokens_dev; 1 <= len <= max_seq.
+ * Writes the last position's logits (n_req x vocab fp32, may be NULL) and
+ * greedy next ids (n_req int32, may be NULL). */
+int mk_prefill(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t* offsets_host, int n_req,
+               float* last_logits_dev, int32_t* next_ids_dev);
+
+/* One decode step: request r feeds tokens_dev[r] at position pos_host[r]
+ * (positions 0..pos-1 must be in its KV cache), appends its K/V at pos, and
+ * writes logits_dev[r*vocab ..] (may be NULL) and next_ids_dev[r] (may be
+ * NULL).  n_req <= max_batch. */
+int mk_decode_step(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t* pos_host, int n_req,
+                   float* logits_dev, int32_t* next_ids_dev);
+
+/* mk_decode_step from and to HOST memory: copies the tokens in, runs the
+ * step, copies the next ids out and synchronises the stream. */
+int mk_decode_step_host(mk_ctx* ctx, const int32_t* tokens_host, const int32_t* pos_host,
+                        int n_req, int32_t* next_ids_host);
+
+/* Copies the final residual stream of the last step (before the final norm),
+ * n_req x hidden fp32, to hidden_dev (enqueued on the context's stream). */
+int mk_copy_hidden(mk_ctx* ctx, float* hidden_dev, int n_req);
+
+/* Device pointer of the bf16 K (which=0) or V (which=1) cache of one request,
+ * layer and KV head: max_seq x head_dim elements, row-major. */
+int mk_kv_pointer(mk_ctx* ctx, int req, int layer, int kv_head, int which, void** out_dev);
+
+/* Copies positions [0, n) of one K (which=0) or V (which=1) cache head, bf16
+ * n x head_dim, to dst_dev (enqueued on the context's stream). */
+int mk_copy_kv(mk_ctx* ctx, int req, int layer, int kv_head, int which, int n, void* dst_dev);
+
+/* Selects the execution mode of later steps (MK_MODE_*). */
+int mk_set_mode(mk_ctx* ctx, int mode);
+
+/* Synchronises the stream and reports the device status: 0, MK_ERR_TIMEOUT,
+ * MK_ERR_TOKEN_RANGE or MK_ERR_CUDA.  Poisons the context on error. */
+int mk_status(mk_ctx* ctx);
+
+const char* mk_last_error(const mk_ctx* ctx);
+void mk_destroy(mk_ctx* ctx);
+
+/* ---------------------------------------------------------------------
+ * Introspection of the task graph (host only, no GPU needed).
+ * mk_plan_build makes the same graph mk_create would for `num_ctas` CTAs.
+ */
+typedef struct {
+  int num_ctas, n_tasks, n_events, n_stages;
+  int attn_splits, n_lm_tasks, ring_slots, slot_bytes;
+  int smem_bytes, threads_per_cta;
+  long long weight_bytes_per_step; /* bf16 weight bytes one step streams */
+} mk_plan_info;
+
+/* One task as the builder laid it out (a copy, for tests and tools). */
+typedef struct {
+  int kind;        /* 0 QKV, 1 ATTN, 2 OPROJ, 3 GATEUP, 4 DOWN, 5 LMHEAD */
+  int layer;
+  int row0, row1;  /* GEMV: packed output rows; ATTN: kv group, split */
+  int req;         /* ATTN: batch slot */
+  int wait_event;  /* -1: none */
+  int wait_count;  /* signals per step the event must reach */
+  int signal_event0, n_signal; /* events bumped on completion */
+  int cta;         /* CTA whose queue holds the task */
+  int stage;       /* operator stage for the per-operator mode */
+} mk_plan_task;
+
+typedef struct mk_plan mk_plan;
+int mk_plan_build(const mk_config* cfg, const mk_options* opt, int num_ctas, mk_plan** out);
+int mk_plan_get_info(const mk_plan* p, mk_plan_info* info);
+/* Copies min(cap, n_tasks) tasks; returns the number copied. */
+int mk_plan_get_tasks(const mk_plan* p, mk_plan_task* out, int cap);
+/* Queue of one CTA in the megakernel mode (task indices in run order). */
+int mk_plan_get_queue(const mk_plan* p, int cta, int* out, int cap);
+/* Signals per step each event receives. */
+int mk_plan_get_event_counts(const mk_plan* p, int* out, int cap);
+void mk_plan_destroy(mk_plan* p);
+
+/* Packed-row layout of the fused QKV matrix: the source of packed row r as
+ * (which: 0 q, 1 k, 2 v; head; dim).  Rows are grouped per KV head (its G
+ * query heads, then its K head, then its V head); inside a q or k head the
+ * RoPE partners (i, i + head_dim/2) sit on adjacent rows. */
+int mk_qkv_row_source(const mk_config* cfg, int packed_row, int* which, int* head, int* dim);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -1,0 +1,514 @@
+// api.cu -- the C-ABI of libmk (declared in include/mk.h).
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "../../include/mk.h"
+#include "mk_internal.h"
+#include "plan.h"
+
+namespace mk {
+size_t step_kernel_smem_bytes();
+const void* step_kernel_ptr();
+cudaError_t launch_pack_qkv(uint16_t*, const uint16_t*, const uint16_t*, const uint16_t*, int, int,
+                            int, int, cudaStream_t);
+cudaError_t launch_pack_qkv_bias(uint16_t*, const uint16_t*, const uint16_t*, const uint16_t*, int,
+                                 int, int, cudaStream_t);
+cudaError_t launch_pack_gateup(uint16_t*, const uint16_t*, const uint16_t*, int, int, cudaStream_t);
+cudaError_t launch_step(const KernelArgs& args, int grid, bool cooperative, cudaStream_t st);
+}  // namespace mk
+
+using namespace mk;
+
+static thread_local std::string g_create_error;
+
+struct mk_ctx {
+  mk_config cfg{};
+  mk_options opt{};
+  cudaStream_t stream = nullptr;
+  int device = 0;
+  Plan plan;
+  ModelDev md{};
+  std::vector<void*> allocs;
+  Task* d_tasks = nullptr;
+  int32_t* d_queue = nullptr;
+  int32_t* d_queue_off = nullptr;
+  StepParams* d_sp = nullptr;
+  int32_t* d_tokens = nullptr;   // staging for mk_decode_step_host
+  int32_t* d_ids = nullptr;
+  int32_t* h_pinned = nullptr;   // pinned staging: tokens in, ids out
+  int mode = MK_MODE_MEGAKERNEL;
+  bool poisoned = false;
+  std::string err;
+  cudaGraphExec_t graph = nullptr;
+  cudaGraph_t graph_src = nullptr;
+  size_t kv_bytes = 0;
+};
+
+static int fail(mk_ctx* c, int code, const std::string& msg) {
+  if (c) c->err = msg; else g_create_error = msg;
+  return code;
+}
+
+#define CK(call)                                                                 \
+  do {                                                                           \
+    cudaError_t e_ = (call);                                                     \
+    if (e_ != cudaSuccess)                                                       \
+      return fail(ctx, MK_ERR_CUDA, std::string(#call) + ": " + cudaGetErrorString(e_)); \
+  } while (0)
+
+template <class T>
+static int dalloc(mk_ctx* ctx, T** p, size_t bytes) {
+  void* v = nullptr;
+  cudaError_t e = cudaMalloc(&v, bytes ? bytes : 16);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(ctx, MK_ERR_OOM, "cudaMalloc(" + std::to_string(bytes) + "): " + cudaGetErrorString(e));
+  }
+  ctx->allocs.push_back(v);
+  *p = static_cast<T*>(v);
+  return MK_OK;
+}
+
+static void release(mk_ctx* ctx) {
+  if (!ctx) return;
+  if (ctx->graph) cudaGraphExecDestroy(ctx->graph);
+  if (ctx->graph_src) cudaGraphDestroy(ctx->graph_src);
+  for (void* p : ctx->allocs) cudaFree(p);
+  if (ctx->h_pinned) cudaFreeHost(ctx->h_pinned);
+  ctx->allocs.clear();
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static void fill_args(mk_ctx* ctx, KernelArgs& a, int set, const StepParams* sp_val,
+                      const StepParams* sp_ptr, bool no_wait) {
+  a.m = ctx->md;
+  a.tasks = ctx->d_tasks;
+  a.queue = ctx->d_queue;
+  a.queue_off = ctx->d_queue_off + ctx->plan.set_offset(set);
+  if (sp_val) a.sp_val = *sp_val; else memset(&a.sp_val, 0, sizeof(a.sp_val));
+  a.sp_ptr = sp_ptr;
+  a.no_wait = no_wait ? 1 : 0;
+}
+
+// Enqueues one decode step in the context's mode.
+static int enqueue_step(mk_ctx* ctx, const StepParams& sp) {
+  const int P = ctx->plan.num_ctas;
+  KernelArgs a;
+  if (ctx->mode == MK_MODE_MEGAKERNEL) {
+    fill_args(ctx, a, 0, &sp, nullptr, false);
+    CK(launch_step(a, P, true, ctx->stream));
+  } else if (ctx->mode == MK_MODE_PER_OP) {
+    for (int s = 0; s < ctx->plan.n_stages; ++s) {
+      fill_args(ctx, a, 1 + s, &sp, nullptr, true);
+      CK(launch_step(a, P, false, ctx->stream));
+    }
+  } else {
+    CK(cudaMemcpyAsync(ctx->d_sp, &sp, sizeof(StepParams), cudaMemcpyHostToDevice, ctx->stream));
+    if (!ctx->graph) {
+      cudaStream_t cs;
+      CK(cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking));
+      cudaError_t e = cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal);
+      for (int s = 0; e == cudaSuccess && s < ctx->plan.n_stages; ++s) {
+        fill_args(ctx, a, 1 + s, nullptr, ctx->d_sp, true);
+        e = launch_step(a, P, false, cs);
+      }
+      cudaGraph_t g = nullptr;
+      cudaError_t e2 = cudaStreamEndCapture(cs, &g);
+      cudaStreamDestroy(cs);
+      if (e != cudaSuccess || e2 != cudaSuccess)
+        return fail(ctx, MK_ERR_CUDA, std::string("graph capture: ") +
+                                          cudaGetErrorString(e != cudaSuccess ? e : e2));
+      ctx->graph_src = g;
+      CK(cudaGraphInstantiate(&ctx->graph, g, 0));
+    }
+    CK(cudaGraphLaunch(ctx->graph, ctx->stream));
+  }
+  return MK_OK;
+}
+
+static void host_rope_table(int max_seq, int d, double theta, std::vector<float>& c,
+                            std::vector<float>& s) {
+  const int half = d / 2;
+  c.resize((size_t)max_seq * half);
+  s.resize((size_t)max_seq * half);
+  for (int p = 0; p < max_seq; ++p)
+    for (int i = 0; i < half; ++i) {
+      const double freq = std::pow(theta, -2.0 * (double)i / (double)d);
+      const double ang = (double)p * freq;
+      c[(size_t)p * half + i] = (float)std::cos(ang);
+      s[(size_t)p * half + i] = (float)std::sin(ang);
+    }
+}
+
+extern "C" int mk_create(const mk_config* cfg, const mk_weights* w, const mk_options* opt,
+                         void* stream, mk_ctx** out) {
+  g_create_error.clear();
+  mk_ctx* ctx = nullptr;
+  if (!cfg || !w || !out) return fail(nullptr, MK_ERR_INVALID_ARG, "null argument");
+  *out = nullptr;
+  std::string verr = validate_config(*cfg);
+  if (!verr.empty()) return fail(nullptr, MK_ERR_INVALID_ARG, verr);
+  if (cfg->max_batch != 1)
+    return fail(nullptr, MK_ERR_UNSUPPORTED, "this build decodes one request per step (max_batch 1)");
+  if (!w->embed || !w->layers || !w->final_norm || (!cfg->tied_embeddings && !w->lm_head))
+    return fail(nullptr, MK_ERR_INVALID_ARG, "missing weight pointer");
+  for (int l = 0; l < cfg->n_layers; ++l) {
+    const mk_layer_weights& L = w->layers[l];
+    const void* need[] = {L.attn_norm, L.wq, L.wk, L.wv, L.wo, L.ffn_norm, L.w_gate, L.w_up, L.w_down};
+    for (const void* p : need)
+      if (!p || !aligned16(p)) return fail(nullptr, MK_ERR_INVALID_ARG, "layer weight null or not 16-byte aligned");
+    if (cfg->qkv_bias && (!L.bq || !L.bk || !L.bv))
+      return fail(nullptr, MK_ERR_INVALID_ARG, "qkv_bias set but a bias pointer is null");
+  }
+  const int G = cfg->n_q_heads / cfg->n_kv_heads;
+  const bool g_ok = cfg->head_dim == 128 ? (G == 1 || G == 2 || G == 4)
+                                         : (G == 1 || G == 2 || G == 4 || G == 7 || G == 8);
+  if (!g_ok) return fail(nullptr, MK_ERR_UNSUPPORTED, "unsupported query heads per KV head");
+
+  ctx = new mk_ctx();
+  ctx->cfg = *cfg;
+  if (opt) ctx->opt = *opt;
+  ctx->stream = static_cast<cudaStream_t>(stream);
+  ctx->mode = ctx->opt.mode;
+  int rc = MK_OK;
+  auto bail = [&](int code) {
+    std::string m = ctx->err;
+    release(ctx);
+    delete ctx;
+    g_create_error = m;
+    return code;
+  };
+#define CKC(call)                                                                          \
+  do {                                                                                     \
+    cudaError_t e_ = (call);                                                               \
+    if (e_ != cudaSuccess) {                                                               \
+      ctx->err = std::string(#call) + ": " + cudaGetErrorString(e_);                       \
+      return bail(MK_ERR_CUDA);                                                            \
+    }                                                                                      \
+  } while (0)
+  CKC(cudaGetDevice(&ctx->device));
+  int sms = 0, smem_optin = 0;
+  CKC(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, ctx->device));
+  CKC(cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, ctx->device));
+  const size_t smem = step_kernel_smem_bytes();
+  if ((size_t)smem_optin < smem) {
+    ctx->err = "device offers " + std::to_string(smem_optin) + " B shared memory per block, need " +
+               std::to_string(smem);
+    return bail(MK_ERR_NOT_RESIDENT);
+  }
+  CKC(cudaFuncSetAttribute(step_kernel_ptr(), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  int per_sm = 0;
+  CKC(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, step_kernel_ptr(), kThreads, smem));
+  if (per_sm < 1) {
+    ctx->err = "one CTA of the step kernel does not fit on an SM";
+    return bail(MK_ERR_NOT_RESIDENT);
+  }
+  int P = ctx->opt.num_ctas > 0 ? ctx->opt.num_ctas : sms;
+  if (P > sms * per_sm) {
+    ctx->err = "num_ctas exceeds the co-resident limit";
+    return bail(MK_ERR_NOT_RESIDENT);
+  }
+  std::string perr = build_plan(*cfg, P, ctx->opt.attn_splits, &ctx->plan);
+  if (!perr.empty()) {
+    ctx->err = perr;
+    return bail(MK_ERR_INVALID_ARG);
+  }
+  const Plan& plan = ctx->plan;
+  const int L = cfg->n_layers, H = cfg->hidden, nq = cfg->n_q_heads, nkv = cfg->n_kv_heads;
+  const int d = cfg->head_dim, F = cfg->ffn, V = cfg->vocab, B = cfg->max_batch;
+  const int qkvR = qkv_rows(nq, nkv, d), qd = nq * d, S = plan.attn_splits;
+  cudaStream_t st = ctx->stream;
+
+  // ---- packed weights, one allocation
+  auto al = [](size_t b) { return (b + 255) & ~(size_t)255; };
+  const size_t sz_qkv = (size_t)qkvR * H * 2, sz_o = (size_t)H * qd * 2;
+  const size_t sz_gu = (size_t)2 * F * H * 2, sz_dn = (size_t)H * F * 2;
+  const size_t per_layer = al(sz_qkv) + al(sz_o) + al(sz_gu) + al(sz_dn);
+  const size_t sz_emb = (size_t)V * H * 2;
+  size_t total = per_layer * L + al(sz_emb) + (cfg->tied_embeddings ? 0 : al(sz_emb)) +
+                 2 * al((size_t)L * H * 2) + al((size_t)H * 2) +
+                 (cfg->qkv_bias ? al((size_t)L * qkvR * 2) : 0);
+  uint8_t* wbuf = nullptr;
+  if ((rc = dalloc(ctx, &wbuf, total))) return bail(rc);
+  uint8_t* cur = wbuf;
+  auto take = [&](size_t b) { uint8_t* p = cur; cur += al(b); return p; };
+  std::vector<const uint16_t*> w_qkv(L), w_o(L), w_gu(L), w_dn(L);
+  for (int l = 0; l < L; ++l) {
+    const mk_layer_weights& Lw = w->layers[l];
+    uint16_t* pq = (uint16_t*)take(sz_qkv);
+    uint16_t* po = (uint16_t*)take(sz_o);
+    uint16_t* pg = (uint16_t*)take(sz_gu);
+    uint16_t* pd = (uint16_t*)take(sz_dn);
+    CKC(launch_pack_qkv(pq, (const uint16_t*)Lw.wq, (const uint16_t*)Lw.wk, (const uint16_t*)Lw.wv, H,
+                        G, d, qkvR, st));
+    CKC(cudaMemcpyAsync(po, Lw.wo, sz_o, cudaMemcpyDeviceToDevice, st));
+    CKC(launch_pack_gateup(pg, (const uint16_t*)Lw.w_gate, (const uint16_t*)Lw.w_up, H, F, st));
+    CKC(cudaMemcpyAsync(pd, Lw.w_down, sz_dn, cudaMemcpyDeviceToDevice, st));
+    w_qkv[l] = pq; w_o[l] = po; w_gu[l] = pg; w_dn[l] = pd;
+  }
+  uint16_t* emb = (uint16_t*)take(sz_emb);
+  CKC(cudaMemcpyAsync(emb, w->embed, sz_emb, cudaMemcpyDeviceToDevice, st));
+  uint16_t* lm = emb;
+  if (!cfg->tied_embeddings) {
+    lm = (uint16_t*)take(sz_emb);
+    CKC(cudaMemcpyAsync(lm, w->lm_head, sz_emb, cudaMemcpyDeviceToDevice, st));
+  }
+  uint16_t* an = (uint16_t*)take((size_t)L * H * 2);
+  uint16_t* fn = (uint16_t*)take((size_t)L * H * 2);
+  uint16_t* finaln = (uint16_t*)take((size_t)H * 2);
+  for (int l = 0; l < L; ++l) {
+    CKC(cudaMemcpyAsync(an + (size_t)l * H, w->layers[l].attn_norm, (size_t)H * 2, cudaMemcpyDeviceToDevice, st));
+    CKC(cudaMemcpyAsync(fn + (size_t)l * H, w->layers[l].ffn_norm, (size_t)H * 2, cudaMemcpyDeviceToDevice, st));
+  }
+  CKC(cudaMemcpyAsync(finaln, w->final_norm, (size_t)H * 2, cudaMemcpyDeviceToDevice, st));
+  uint16_t* bq = nullptr;
+  if (cfg->qkv_bias) {
+    bq = (uint16_t*)take((size_t)L * qkvR * 2);
+    for (int l = 0; l < L; ++l)
+      CKC(launch_pack_qkv_bias(bq + (size_t)l * qkvR, (const uint16_t*)w->layers[l].bq,
+                               (const uint16_t*)w->layers[l].bk, (const uint16_t*)w->layers[l].bv, G, d,
+                               qkvR, st));
+  }
+  if ((size_t)(cur - wbuf) > total) {
+    ctx->err = "internal: weight buffer overflow";
+    return bail(MK_ERR_INVALID_ARG);
+  }
+
+  // ---- RoPE table, KV cache, activations, sync words
+  std::vector<float> hc, hs;
+  host_rope_table(cfg->max_seq, d, cfg->rope_theta, hc, hs);
+  float *rc_d = nullptr, *rs_d = nullptr;
+  if ((rc = dalloc(ctx, &rc_d, hc.size() * 4))) return bail(rc);
+  if ((rc = dalloc(ctx, &rs_d, hs.size() * 4))) return bail(rc);
+  CKC(cudaMemcpyAsync(rc_d, hc.data(), hc.size() * 4, cudaMemcpyHostToDevice, st));
+  CKC(cudaMemcpyAsync(rs_d, hs.data(), hs.size() * 4, cudaMemcpyHostToDevice, st));
+  ctx->kv_bytes = (size_t)B * L * nkv * cfg->max_seq * d * 2;
+  uint16_t *kc = nullptr, *vc = nullptr;
+  if ((rc = dalloc(ctx, &kc, ctx->kv_bytes))) return bail(rc);
+  if ((rc = dalloc(ctx, &vc, ctx->kv_bytes))) return bail(rc);
+  CKC(cudaMemsetAsync(kc, 0, ctx->kv_bytes, st));
+  CKC(cudaMemsetAsync(vc, 0, ctx->kv_bytes, st));
+  float *x = nullptr, *q = nullptr, *att = nullptr, *act = nullptr, *part = nullptr;
+  unsigned long long* am = nullptr;
+  if ((rc = dalloc(ctx, &x, (size_t)B * H * 4))) return bail(rc);
+  if ((rc = dalloc(ctx, &q, (size_t)B * qd * 4))) return bail(rc);
+  if ((rc = dalloc(ctx, &att, (size_t)B * qd * 4))) return bail(rc);
+  if ((rc = dalloc(ctx, &act, (size_t)B * F * 4))) return bail(rc);
+  if ((rc = dalloc(ctx, &part, (size_t)B * nkv * S * G * (d + 2) * 4))) return bail(rc);
+  if ((rc = dalloc(ctx, &am, (size_t)B * plan.n_lm_tasks * 8))) return bail(rc);
+  CKC(cudaMemsetAsync(x, 0, (size_t)B * H * 4, st));
+  uint32_t *events = nullptr, *tickets = nullptr, *epoch = nullptr;
+  int32_t* status = nullptr;
+  if ((rc = dalloc(ctx, &events, (size_t)plan.n_events * 4))) return bail(rc);
+  if ((rc = dalloc(ctx, &tickets, (size_t)plan.n_tickets * 4))) return bail(rc);
+  if ((rc = dalloc(ctx, &epoch, 16))) return bail(rc);
+  if ((rc = dalloc(ctx, &status, 16))) return bail(rc);
+  CKC(cudaMemsetAsync(events, 0, (size_t)plan.n_events * 4, st));
+  CKC(cudaMemsetAsync(tickets, 0, (size_t)plan.n_tickets * 4, st));
+  CKC(cudaMemsetAsync(epoch, 0, 16, st));
+  CKC(cudaMemsetAsync(status, 0, 16, st));
+
+  // ---- task graph upload (weight pointers patched per kind and layer)
+  std::vector<Task> tasks = plan.tasks;
+  for (Task& t : tasks) {
+    switch (t.kind) {
+      case T_QKV: t.w = w_qkv[t.layer]; break;
+      case T_OPROJ: t.w = w_o[t.layer]; break;
+      case T_GATEUP: t.w = w_gu[t.layer]; break;
+      case T_DOWN: t.w = w_dn[t.layer]; break;
+      case T_LMHEAD: t.w = lm; break;
+      default: t.w = nullptr; break;
+    }
+  }
+  if ((rc = dalloc(ctx, &ctx->d_tasks, tasks.size() * sizeof(Task)))) return bail(rc);
+  if ((rc = dalloc(ctx, &ctx->d_queue, plan.queue.size() * 4))) return bail(rc);
+  if ((rc = dalloc(ctx, &ctx->d_queue_off, plan.queue_off.size() * 4))) return bail(rc);
+  CKC(cudaMemcpyAsync(ctx->d_tasks, tasks.data(), tasks.size() * sizeof(Task), cudaMemcpyHostToDevice, st));
+  CKC(cudaMemcpyAsync(ctx->d_queue, plan.queue.data(), plan.queue.size() * 4, cudaMemcpyHostToDevice, st));
+  CKC(cudaMemcpyAsync(ctx->d_queue_off, plan.queue_off.data(), plan.queue_off.size() * 4,
+                      cudaMemcpyHostToDevice, st));
+  if ((rc = dalloc(ctx, &ctx->d_sp, sizeof(StepParams)))) return bail(rc);
+  if ((rc = dalloc(ctx, &ctx->d_tokens, kMaxBatch * 4))) return bail(rc);
+  if ((rc = dalloc(ctx, &ctx->d_ids, kMaxBatch * 4))) return bail(rc);
+  CKC(cudaMallocHost(&ctx->h_pinned, 2 * kMaxBatch * 4));
+
+  ModelDev& m = ctx->md;
+  m.n_layers = L; m.hidden = H; m.n_q = nq; m.n_kv = nkv; m.head_dim = d; m.ffn = F; m.vocab = V;
+  m.group = G; m.max_seq = cfg->max_seq; m.max_batch = B; m.attn_splits = S;
+  m.qkv_bias = cfg->qkv_bias ? 1 : 0;
+  m.rms_eps = cfg->rms_eps;
+  m.attn_scale = (float)(1.0 / std::sqrt((double)d));
+  m.n_lm_tasks = plan.n_lm_tasks;
+  m.timeout_ms = ctx->opt.timeout_ms > 0 ? ctx->opt.timeout_ms : 1000;
+  m.embed = emb; m.lm_head = lm; m.final_norm = finaln; m.attn_norm = an; m.ffn_norm = fn;
+  m.bqkv = bq; m.rope_cos = rc_d; m.rope_sin = rs_d; m.kcache = kc; m.vcache = vc;
+  m.x = x; m.q = q; m.attn = att; m.act = act; m.part = part; m.am = am;
+  m.events = events; m.tickets = tickets; m.epoch = epoch; m.status = status;
+  m.status_info = status + 1;
+  CKC(cudaStreamSynchronize(st));
+  CKC(cudaGetLastError());
+  *out = ctx;
+  return MK_OK;
+#undef CKC
+}
+
+static int check_ctx(mk_ctx* ctx) {
+  if (!ctx) return MK_ERR_INVALID_ARG;
+  if (ctx->poisoned) return fail(ctx, MK_ERR_POISONED, "context poisoned by an earlier device error");
+  return MK_OK;
+}
+
+static int check_step_args(mk_ctx* ctx, const int32_t* pos_host, int n_req) {
+  if (n_req < 1 || n_req > ctx->cfg.max_batch) return fail(ctx, MK_ERR_INVALID_ARG, "n_req out of range");
+  if (!pos_host) return fail(ctx, MK_ERR_INVALID_ARG, "pos_host is null");
+  for (int r = 0; r < n_req; ++r)
+    if (pos_host[r] < 0 || pos_host[r] >= ctx->cfg.max_seq)
+      return fail(ctx, MK_ERR_POS_RANGE, "position " + std::to_string(pos_host[r]) + " outside [0, max_seq)");
+  return MK_OK;
+}
+
+extern "C" int mk_decode_step(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t* pos_host,
+                              int n_req, float* logits_dev, int32_t* next_ids_dev) {
+  int rc = check_ctx(ctx);
+  if (rc) return rc;
+  if (!tokens_dev) return fail(ctx, MK_ERR_INVALID_ARG, "tokens_dev is null");
+  if ((rc = check_step_args(ctx, pos_host, n_req))) return rc;
+  StepParams sp{};
+  sp.n_req = n_req;
+  for (int r = 0; r < n_req; ++r) {
+    sp.pos[r] = pos_host[r];
+    sp.kv_slot[r] = r;
+  }
+  sp.tokens = tokens_dev;
+  sp.logits = logits_dev;
+  sp.next_ids = next_ids_dev;
+  sp.want_logits = logits_dev != nullptr;
+  return enqueue_step(ctx, sp);
+}
+
+extern "C" int mk_decode_step_host(mk_ctx* ctx, const int32_t* tokens_host, const int32_t* pos_host,
+                                   int n_req, int32_t* next_ids_host) {
+  int rc = check_ctx(ctx);
+  if (rc) return rc;
+  if (!tokens_host || !next_ids_host) return fail(ctx, MK_ERR_INVALID_ARG, "null host buffer");
+  if ((rc = check_step_args(ctx, pos_host, n_req))) return rc;
+  memcpy(ctx->h_pinned, tokens_host, (size_t)n_req * 4);
+  CK(cudaMemcpyAsync(ctx->d_tokens, ctx->h_pinned, (size_t)n_req * 4, cudaMemcpyHostToDevice, ctx->stream));
+  if ((rc = mk_decode_step(ctx, ctx->d_tokens, pos_host, n_req, nullptr, ctx->d_ids))) return rc;
+  CK(cudaMemcpyAsync(ctx->h_pinned + kMaxBatch, ctx->d_ids, (size_t)n_req * 4, cudaMemcpyDeviceToHost,
+                     ctx->stream));
+  CK(cudaStreamSynchronize(ctx->stream));
+  memcpy(next_ids_host, ctx->h_pinned + kMaxBatch, (size_t)n_req * 4);
+  return MK_OK;
+}
+
+extern "C" int mk_prefill(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t* offsets_host,
+                          int n_req, float* last_logits_dev, int32_t* next_ids_dev) {
+  int rc = check_ctx(ctx);
+  if (rc) return rc;
+  if (!tokens_dev || !offsets_host) return fail(ctx, MK_ERR_INVALID_ARG, "null argument");
+  if (n_req < 1 || n_req > ctx->cfg.max_batch) return fail(ctx, MK_ERR_INVALID_ARG, "n_req out of range");
+  for (int r = 0; r < n_req; ++r) {
+    const int len = offsets_host[r + 1] - offsets_host[r];
+    if (offsets_host[r] < 0 || len < 1 || len > ctx->cfg.max_seq)
+      return fail(ctx, MK_ERR_POS_RANGE, "prompt length outside [1, max_seq]");
+  }
+  // Each prompt position runs through the same step as decoding: position t
+  // appends its K/V and attends over 0..t.  Only the last position's logits
+  // and id are kept.
+  for (int r = 0; r < n_req; ++r) {
+    const int len = offsets_host[r + 1] - offsets_host[r];
+    for (int t = 0; t < len; ++t) {
+      StepParams sp{};
+      sp.n_req = 1;
+      sp.pos[0] = t;
+      sp.kv_slot[0] = r;
+      sp.tokens = tokens_dev + offsets_host[r] + t;
+      const bool last = t == len - 1;
+      sp.logits = last && last_logits_dev ? last_logits_dev + (size_t)r * ctx->cfg.vocab : nullptr;
+      sp.next_ids = last && next_ids_dev ? next_ids_dev + r : nullptr;
+      sp.want_logits = sp.logits != nullptr;
+      if ((rc = enqueue_step(ctx, sp))) return rc;
+    }
+  }
+  return MK_OK;
+}
+
+extern "C" int mk_copy_hidden(mk_ctx* ctx, float* hidden_dev, int n_req) {
+  int rc = check_ctx(ctx);
+  if (rc) return rc;
+  if (!hidden_dev || n_req < 1 || n_req > ctx->cfg.max_batch) return fail(ctx, MK_ERR_INVALID_ARG, "bad argument");
+  CK(cudaMemcpyAsync(hidden_dev, ctx->md.x, (size_t)n_req * ctx->cfg.hidden * 4, cudaMemcpyDeviceToDevice,
+                     ctx->stream));
+  return MK_OK;
+}
+
+extern "C" int mk_kv_pointer(mk_ctx* ctx, int req, int layer, int kv_head, int which, void** out_dev) {
+  if (!ctx || !out_dev) return MK_ERR_INVALID_ARG;
+  const mk_config& c = ctx->cfg;
+  if (req < 0 || req >= c.max_batch || layer < 0 || layer >= c.n_layers || kv_head < 0 ||
+      kv_head >= c.n_kv_heads || which < 0 || which > 1)
+    return fail(ctx, MK_ERR_INVALID_ARG, "bad KV index");
+  const size_t off = (((size_t)req * c.n_layers + layer) * c.n_kv_heads + kv_head) * (size_t)c.max_seq * c.head_dim;
+  *out_dev = (which ? ctx->md.vcache : ctx->md.kcache) + off;
+  return MK_OK;
+}
+
+extern "C" int mk_copy_kv(mk_ctx* ctx, int req, int layer, int kv_head, int which, int n, void* dst_dev) {
+  int rc = check_ctx(ctx);
+  if (rc) return rc;
+  void* src = nullptr;
+  if ((rc = mk_kv_pointer(ctx, req, layer, kv_head, which, &src))) return rc;
+  if (!dst_dev || n < 0 || n > ctx->cfg.max_seq) return fail(ctx, MK_ERR_INVALID_ARG, "bad copy size");
+  CK(cudaMemcpyAsync(dst_dev, src, (size_t)n * ctx->cfg.head_dim * 2, cudaMemcpyDeviceToDevice, ctx->stream));
+  return MK_OK;
+}
+
+extern "C" int mk_set_mode(mk_ctx* ctx, int mode) {
+  if (!ctx) return MK_ERR_INVALID_ARG;
+  if (mode < MK_MODE_MEGAKERNEL || mode > MK_MODE_PER_OP_GRAPH) return fail(ctx, MK_ERR_INVALID_ARG, "bad mode");
+  ctx->mode = mode;
+  return MK_OK;
+}
+
+extern "C" int mk_status(mk_ctx* ctx) {
+  if (!ctx) return MK_ERR_INVALID_ARG;
+  if (ctx->poisoned) return MK_ERR_POISONED;
+  cudaError_t e = cudaStreamSynchronize(ctx->stream);
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    ctx->poisoned = true;
+    return fail(ctx, MK_ERR_CUDA, std::string("device error: ") + cudaGetErrorString(e));
+  }
+  int32_t st[2] = {0, 0};
+  e = cudaMemcpy(st, ctx->md.status, sizeof st, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) {
+    ctx->poisoned = true;
+    return fail(ctx, MK_ERR_CUDA, std::string("status read: ") + cudaGetErrorString(e));
+  }
+  if (st[0] != 0) {
+    ctx->poisoned = true;
+    const char* what = st[0] == MK_ERR_TIMEOUT ? "event wait timed out at task "
+                       : st[0] == MK_ERR_TOKEN_RANGE ? "token id out of range: "
+                                                     : "device error, detail ";
+    return fail(ctx, st[0], std::string(what) + std::to_string(st[1]));
+  }
+  return MK_OK;
+}
+
+extern "C" const char* mk_last_error(const mk_ctx* ctx) {
+  return ctx ? ctx->err.c_str() : g_create_error.c_str();
+}
+
+extern "C" void mk_destroy(mk_ctx* ctx) {
+  if (!ctx) return;
+  cudaStreamSynchronize(ctx->stream);
+  release(ctx);
+  delete ctx;
+}

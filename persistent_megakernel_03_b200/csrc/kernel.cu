@@ -1,0 +1,927 @@
+// kernel.cu -- the persistent decode-step kernel for sm_100a.
+//
+// One CTA per SM runs an ahead-of-time queue of tasks ("LLMs in einen
+// MegaKernel kompilieren ...", "Part 2. Laufzeit": each worker SM loops
+// fetch task -> execute -> notify event).  Inside a CTA the roles are split
+// by warp:
+//   warp 0  producer : walks the queue ahead of the workers and streams every
+//                      task's bf16 weight rows (or old K/V rows) with bulk
+//                      copies into a ring of shared-memory slots.  It never
+//                      waits on events, so the next task's -- and the next
+//                      layer's -- weights are already on chip while the
+//                      current dependency resolves ("MPK ..." §4: a task
+//                      releases its shared-memory pages so the next task can
+//                      prefetch early).
+//   warp 1  scheduler: waits (gpu-scope acquire, bounded by %globaltimer) until
+//                      the event of the next task reached its threshold, then
+//                      releases the workers ("Ereignisbasierte Ausführung").
+//   warps 2-17 workers: compute each task from the ring: fp32 activations,
+//                      bf16 weights widened in registers, 128-bit shared-memory
+//                      loads, warp-shuffle reductions ("Crear desde cero ..."
+//                      §3.2: threads cooperate on rows and reduce by warp);
+//                      epilogues fuse bias, RoPE, the KV append, residual adds,
+//                      SwiGLU and the argmax ("Crear desde cero ..." §3.3).
+// A finished task bumps its event counters with a gpu-scope release.
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "../../include/mk.h"
+#include "mk_internal.h"
+#include "ptx.cuh"
+
+namespace mk {
+
+struct __align__(128) Smem {
+  uint8_t ring[kRingSlots][kSlotBytes];
+  float scratch[kScratchBytes / 4];
+  float ybuf[kYBufFloats];
+  float red[64];
+  unsigned long long red64[kWorkerWarps];
+  uint64_t full[kRingSlots];
+  uint64_t empty[kRingSlots];
+  uint64_t ready;
+  uint64_t done;
+  uint32_t epoch;
+  int32_t abort_flag;
+  int32_t consumed_seq;
+  int32_t flag;
+};
+
+constexpr uint32_t kWorkerBarrier = 1;
+
+__device__ __forceinline__ void worker_sync() { named_barrier_sync(kWorkerBarrier, kWorkerThreads); }
+
+__device__ __forceinline__ bool aborting(Smem& s) { return *(volatile int32_t*)&s.abort_flag != 0; }
+
+__device__ __forceinline__ const StepParams& step_params(const KernelArgs& a) {
+  return a.sp_ptr ? *a.sp_ptr : a.sp_val;
+}
+
+__device__ __forceinline__ float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
+__device__ __forceinline__ float bf16_to_float(uint16_t h) {
+  return __uint_as_float(static_cast<uint32_t>(h) << 16);
+}
+__device__ __forceinline__ uint16_t float_to_bf16_rne(float f) {
+  __nv_bfloat16 b = __float2bfloat16_rn(f);
+  return *reinterpret_cast<uint16_t*>(&b);
+}
+
+__device__ __forceinline__ float dot8(const uint4 w, const float (&x)[8], float acc) {
+  acc = fmaf(bf_lo(w.x), x[0], acc);
+  acc = fmaf(bf_hi(w.x), x[1], acc);
+  acc = fmaf(bf_lo(w.y), x[2], acc);
+  acc = fmaf(bf_hi(w.y), x[3], acc);
+  acc = fmaf(bf_lo(w.z), x[4], acc);
+  acc = fmaf(bf_hi(w.z), x[5], acc);
+  acc = fmaf(bf_lo(w.w), x[6], acc);
+  acc = fmaf(bf_hi(w.w), x[7], acc);
+  return acc;
+}
+
+__device__ __forceinline__ void set_error(const ModelDev& m, int code, int info) {
+  if (atomicCAS(m.status, 0, code) == 0) m.status_info[0] = info;
+}
+
+// Codes stored in status_info when a shared-memory barrier wait times out
+// (event waits store the task index instead).
+constexpr int kWaitFull = -1, kWaitReady = -2, kWaitDone = -3, kWaitEmpty = -4;
+
+__device__ __forceinline__ bool aborting(Smem& s);
+
+// Bounded mbarrier wait.  True once the phase with `parity` completed; false
+// when this CTA is aborting or the wait exceeded the context's limit (which
+// records MK_ERR_TIMEOUT and starts the abort).  Every wait in the kernel is
+// bounded, so a broken invariant ends the launch with an error, not a hang.
+// The limit is twice the event-wait limit: a barrier may legitimately wait
+// behind an event wait, and a stalled event should be reported as such.
+__device__ __noinline__ bool wait_bounded(Smem& s, uint64_t* bar, uint32_t parity,
+                                          const ModelDev& m, int where) {
+  const uint64_t limit = 2ull * (uint64_t)(m.timeout_ms > 0 ? m.timeout_ms : 1000) * 1000000ull;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (aborting(s)) return false;
+    if (globaltimer_ns() - t0 > limit) {
+      set_error(m, MK_ERR_TIMEOUT, where);
+      *(volatile int32_t*)&s.abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+// Orderable key: larger value first, then lower index.
+__device__ __forceinline__ unsigned long long argmax_key(float v, int idx) {
+  uint32_t u = __float_as_uint(v);
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return (static_cast<unsigned long long>(u) << 32) | (0xffffffffu - static_cast<uint32_t>(idx));
+}
+
+// ------------------------------------------------------ chunk enumeration
+// The producer and the workers walk the same chunk list for every task.
+
+struct AttnRange {
+  int k0, k1, old_end;  // keys [k0, k1); [k0, old_end) come through the ring
+  bool active;
+};
+
+__device__ __forceinline__ AttnRange attn_range(const Task& t, const StepParams& sp,
+                                                const ModelDev& m) {
+  AttnRange r{0, 0, 0, false};
+  if (t.req >= sp.n_req) return r;
+  const int pos = sp.pos[t.req];
+  const int n = pos + 1, S = m.attn_splits;
+  const int chunk = (n + S - 1) / S;
+  r.k0 = min(n, t.row1 * chunk);
+  r.k1 = min(n, r.k0 + chunk);
+  r.old_end = min(r.k1, pos);
+  if (r.old_end < r.k0) r.old_end = r.k0;
+  r.active = true;
+  return r;
+}
+
+__device__ __forceinline__ size_t kv_offset(const ModelDev& m, int slot, int layer, int g,
+                                            int key) {
+  return ((((size_t)slot * m.n_layers + layer) * m.n_kv + g) * (size_t)m.max_seq + key) *
+         (size_t)m.head_dim;
+}
+
+// ---------------------------------------------------------------- producer
+
+__device__ __forceinline__ bool producer_acquire_slot(Smem& s, uint32_t seq, const ModelDev& m) {
+  const int slot = seq % kRingSlots;
+  const uint32_t ph = (seq / kRingSlots) & 1u;
+  if (!wait_bounded(s, &s.empty[slot], ph ^ 1u, m, kWaitEmpty)) return false;
+  return !aborting(s);
+}
+
+__device__ void producer(const KernelArgs& a, Smem& s, int q0, int q1) {
+  const ModelDev& m = a.m;
+  const StepParams& sp = step_params(a);
+  const uint64_t pol_w = l2_policy_evict_first();
+  const uint64_t pol_kv = l2_policy_evict_normal();
+  uint32_t seq = 0;
+  bool ok = true;
+  for (int qi = q0; qi < q1 && ok; ++qi) {
+    const Task& t = a.tasks[a.queue[qi]];
+    if (t.kind == T_ATTN) {
+      const AttnRange r = attn_range(t, sp, m);
+      if (!r.active) continue;
+      const int kpc = attn_keys_per_chunk(m.head_dim);
+      const int slotkv = sp.kv_slot[t.req];
+      for (int k = r.k0; k < r.old_end && ok; k += kpc) {
+        const int nk = min(kpc, r.old_end - k);
+        const uint32_t bytes = (uint32_t)nk * m.head_dim * 2;
+        if (!(ok = producer_acquire_slot(s, seq, m))) break;
+        const int slot = seq % kRingSlots;
+        const size_t off = kv_offset(m, slotkv, t.layer, t.row0, k);
+        mbar_arrive_expect_tx(&s.full[slot], 2 * bytes);
+        bulk_g2s(s.ring[slot], m.kcache + off, bytes, &s.full[slot], pol_kv);
+        bulk_g2s(s.ring[slot] + kSlotBytes / 2, m.vcache + off, bytes, &s.full[slot], pol_kv);
+        ++seq;
+      }
+    } else {
+      const int K = t.K;
+      for (int r = t.row0; r < t.row1 && ok; r += t.chunk_rows) {
+        const int nr = min(t.chunk_rows, t.row1 - r);
+        const uint32_t bytes = (uint32_t)nr * K * 2;
+        if (!(ok = producer_acquire_slot(s, seq, m))) break;
+        const int slot = seq % kRingSlots;
+        mbar_arrive_expect_tx(&s.full[slot], bytes);
+        bulk_g2s(s.ring[slot], t.w + (size_t)r * K, bytes, &s.full[slot], pol_w);
+        ++seq;
+      }
+    }
+  }
+  // Before this warp may retire, every copy it issued must have landed: if
+  // the workers stop early (abort) nobody else waits for them, and a bulk copy
+  // must never write into shared memory of a CTA that has exited.  Only the
+  // last kRingSlots copies can still be in flight (older slots were reused).
+  // The wait is bounded: the sources are valid device memory.
+  const uint32_t first = seq > kRingSlots ? seq - kRingSlots : 0;
+  for (uint32_t q = first; q < seq; ++q) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(&s.full[q % kRingSlots], (q / kRingSlots) & 1u)) {
+      if (globaltimer_ns() - t0 > 200000000ull) break;
+    }
+  }
+}
+
+// --------------------------------------------------------------- scheduler
+
+__device__ void scheduler(const KernelArgs& a, Smem& s, int q0, int q1) {
+  const ModelDev& m = a.m;
+  const uint32_t epoch = s.epoch;
+  const uint64_t limit = (uint64_t)(m.timeout_ms > 0 ? m.timeout_ms : 1000) * 1000000ull;
+  int i = 0;
+  for (int qi = q0; qi < q1; ++qi, ++i) {
+    const int tid = a.queue[qi];
+    const Task& t = a.tasks[tid];
+    bool abort = false;
+    if (t.wait_ev >= 0 && !a.no_wait) {
+      const uint32_t target = t.wait_count * (epoch + 1u);
+      const uint32_t* ev = m.events + t.wait_ev;
+      const uint64_t t0 = globaltimer_ns();
+      uint32_t spins = 0;
+      while ((int32_t)(ld_acquire_gpu(ev) - target) < 0) {
+        if ((++spins & 63u) == 0) {
+          if (ld_relaxed_gpu_s32(m.status) != 0 || aborting(s)) { abort = true; break; }
+          if (globaltimer_ns() - t0 > limit) {
+            set_error(m, MK_ERR_TIMEOUT, tid);
+            abort = true;
+            break;
+          }
+        }
+      }
+    }
+    if (abort) {
+      *(volatile int32_t*)&s.abort_flag = 1;
+      __threadfence_block();
+      mbar_arrive(&s.ready);
+      return;
+    }
+    mbar_arrive(&s.ready);
+    if (!wait_bounded(s, &s.done, i & 1, m, kWaitDone)) return;
+  }
+}
+
+// ------------------------------------------------------------ worker: GEMV
+
+template <int NR>
+__device__ __forceinline__ float warp_reduce_rows(float (&v)[NR], int lane) {
+  if constexpr (NR == 4) {
+    const bool b4 = lane & 16;
+    float a0 = b4 ? v[2] : v[0], a1 = b4 ? v[3] : v[1];
+    float s0 = b4 ? v[0] : v[2], s1 = b4 ? v[1] : v[3];
+    a0 += __shfl_xor_sync(0xffffffffu, s0, 16);
+    a1 += __shfl_xor_sync(0xffffffffu, s1, 16);
+    const bool b3 = lane & 8;
+    float k = b3 ? a1 : a0, snd = b3 ? a0 : a1;
+    k += __shfl_xor_sync(0xffffffffu, snd, 8);
+    k += __shfl_xor_sync(0xffffffffu, k, 4);
+    k += __shfl_xor_sync(0xffffffffu, k, 2);
+    k += __shfl_xor_sync(0xffffffffu, k, 1);
+    return k;  // row lane >> 3
+  } else if constexpr (NR == 2) {
+    const bool b4 = lane & 16;
+    float k = b4 ? v[1] : v[0], snd = b4 ? v[0] : v[1];
+    k += __shfl_xor_sync(0xffffffffu, snd, 16);
+    k += __shfl_xor_sync(0xffffffffu, k, 8);
+    k += __shfl_xor_sync(0xffffffffu, k, 4);
+    k += __shfl_xor_sync(0xffffffffu, k, 2);
+    k += __shfl_xor_sync(0xffffffffu, k, 1);
+    return k;  // row lane >> 4
+  } else {
+    float k = v[0];
+    k += __shfl_xor_sync(0xffffffffu, k, 16);
+    k += __shfl_xor_sync(0xffffffffu, k, 8);
+    k += __shfl_xor_sync(0xffffffffu, k, 4);
+    k += __shfl_xor_sync(0xffffffffu, k, 2);
+    k += __shfl_xor_sync(0xffffffffu, k, 1);
+    return k;
+  }
+}
+
+// Sum over the 512 worker threads; every worker gets the result.
+__device__ __forceinline__ float worker_sum(Smem& s, float v, int wtid) {
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if ((wtid & 31) == 0) s.red[wtid >> 5] = v;
+  worker_sync();
+  float t = 0.f;
+#pragma unroll
+  for (int w = 0; w < kWorkerWarps; ++w) t += s.red[w];
+  worker_sync();
+  return t;
+}
+
+// Waits for ring chunk `seq`.  Once the CTA is aborting the workers no longer
+// wait: they run the rest of the current task on whatever the slot holds
+// (every access stays in bounds), meet the task's barriers, and stop.
+__device__ __forceinline__ void wait_full(Smem& s, uint32_t seq, const ModelDev& m) {
+  const int slot = seq % kRingSlots;
+  const uint32_t ph = (seq / kRingSlots) & 1u;
+  if (mbar_try_wait(&s.full[slot], ph)) return;
+  wait_bounded(s, &s.full[slot], ph, m, kWaitFull);
+}
+
+// Loads this thread's input columns (fp32 or the bf16 embedding row), applies
+// RMSNorm when the task's operator has one, and leaves the result in xr.
+template <int CPT>
+__device__ __forceinline__ void gemv_load_input(const KernelArgs& a, Smem& s, const Task& t,
+                                                int wtid, int ct, int rl, float (&xr)[CPT][8]) {
+  const ModelDev& m = a.m;
+  const StepParams& sp = step_params(a);
+  const int K = t.K, C = K >> 3;
+  const float* src32 = nullptr;
+  const uint16_t* src16 = nullptr;
+  const uint16_t* normw = nullptr;
+  switch (t.kind) {
+    case T_QKV:
+      normw = m.attn_norm + (size_t)t.layer * m.hidden;
+      if (t.layer == 0) {
+        int tok = sp.tokens[0];
+        if (tok < 0 || tok >= m.vocab) {
+          if (wtid == 0) set_error(m, MK_ERR_TOKEN_RANGE, tok);
+          tok = 0;
+        }
+        src16 = m.embed + (size_t)tok * m.hidden;
+      } else {
+        src32 = m.x;
+      }
+      break;
+    case T_OPROJ: src32 = m.attn; break;
+    case T_GATEUP: src32 = m.x; normw = m.ffn_norm + (size_t)t.layer * m.hidden; break;
+    case T_DOWN: src32 = m.act; break;
+    default: src32 = m.x; normw = m.final_norm; break;  // LM head
+  }
+  const int TPR = t.tpr;
+#pragma unroll
+  for (int c = 0; c < CPT; ++c) {
+    const int cc = ct + c * TPR;
+    if (cc < C) {
+      if (src16) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(src16) + cc);
+        xr[c][0] = bf_lo(v.x); xr[c][1] = bf_hi(v.x); xr[c][2] = bf_lo(v.y); xr[c][3] = bf_hi(v.y);
+        xr[c][4] = bf_lo(v.z); xr[c][5] = bf_hi(v.z); xr[c][6] = bf_lo(v.w); xr[c][7] = bf_hi(v.w);
+      } else {
+        const float4 u = __ldcg(reinterpret_cast<const float4*>(src32) + 2 * cc);
+        const float4 w = __ldcg(reinterpret_cast<const float4*>(src32) + 2 * cc + 1);
+        xr[c][0] = u.x; xr[c][1] = u.y; xr[c][2] = u.z; xr[c][3] = u.w;
+        xr[c][4] = w.x; xr[c][5] = w.y; xr[c][6] = w.z; xr[c][7] = w.w;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) xr[c][e] = 0.f;
+    }
+  }
+  if (normw) {
+    float ss = 0.f;
+    if (rl == 0) {
+#pragma unroll
+      for (int c = 0; c < CPT; ++c)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ss = fmaf(xr[c][e], xr[c][e], ss);
+    }
+    ss = worker_sum(s, ss, wtid);
+    const float r = 1.0f / sqrtf(ss / (float)K + m.rms_eps);
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) {
+      const int cc = ct + c * TPR;
+      if (cc < C) {
+        const uint4 wv = __ldg(reinterpret_cast<const uint4*>(normw) + cc);
+        const float wn[8] = {bf_lo(wv.x), bf_hi(wv.x), bf_lo(wv.y), bf_hi(wv.y),
+                             bf_lo(wv.z), bf_hi(wv.z), bf_lo(wv.w), bf_hi(wv.w)};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) xr[c][e] = (xr[c][e] * r) * wn[e];
+      }
+    }
+  }
+}
+
+// Streams the task's rows through the ring and leaves y[row] in s.ybuf.
+template <int CPT, int NR>
+__device__ void gemv_stream(const KernelArgs& a, Smem& s, const Task& t, uint32_t& seq, int wtid) {
+  const int TPR = t.tpr;
+  const int rl = wtid / TPR, ct = wtid % TPR;
+  const int wpr = TPR >> 5, wir = ct >> 5;
+  const int lane = wtid & 31;
+  const int K = t.K, C = K >> 3;
+  const size_t row_bytes = (size_t)K * 2;
+  const int nrows = t.row1 - t.row0;
+  float xr[CPT][8];
+  gemv_load_input<CPT>(a, s, t, wtid, ct, rl, xr);
+  constexpr int kShift = NR == 4 ? 3 : (NR == 2 ? 4 : 5);
+  for (int r = 0; r < nrows; r += t.chunk_rows) {
+    const int rows_here = min(t.chunk_rows, nrows - r);
+    const int slot = seq % kRingSlots;
+    wait_full(s, seq, a.m);
+    const uint8_t* base = s.ring[slot];
+    float acc[NR];
+#pragma unroll
+    for (int j = 0; j < NR; ++j) {
+      acc[j] = 0.f;
+      const int lr = rl * NR + j;
+      if (lr < rows_here) {
+        const uint8_t* row = base + (size_t)lr * row_bytes;
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) {
+          const int cc = ct + c * TPR;
+          if (cc < C) acc[j] = dot8(*reinterpret_cast<const uint4*>(row + (size_t)cc * 16), xr[c], acc[j]);
+        }
+      }
+    }
+    const float v = warp_reduce_rows<NR>(acc, lane);
+    const int jj = lane >> kShift;
+    if ((lane & ((1 << kShift) - 1)) == 0) {
+      const int lr = rl * NR + jj;
+      if (lr < rows_here) s.scratch[wir * nrows + r + lr] = v;
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.empty[slot]);
+    ++seq;
+  }
+  worker_sync();
+  for (int i = wtid; i < nrows; i += kWorkerThreads) {
+    float y = 0.f;
+    for (int w = 0; w < wpr; ++w) y += s.scratch[w * nrows + i];
+    s.ybuf[i] = y;
+  }
+  worker_sync();
+}
+
+template <int CPT>
+__device__ void gemv_dispatch_nr(const KernelArgs& a, Smem& s, const Task& t, uint32_t& seq,
+                                 int wtid) {
+  const int nr = t.chunk_rows / (kWorkerThreads / t.tpr);
+  if (nr >= 4) gemv_stream<CPT, 4>(a, s, t, seq, wtid);
+  else if (nr == 2) gemv_stream<CPT, 2>(a, s, t, seq, wtid);
+  else gemv_stream<CPT, 1>(a, s, t, seq, wtid);
+}
+
+__device__ void gemv_core(const KernelArgs& a, Smem& s, const Task& t, uint32_t& seq, int wtid) {
+  const int cpt = (t.K / 8 + t.tpr - 1) / t.tpr;
+  switch (cpt) {
+    case 1: gemv_dispatch_nr<1>(a, s, t, seq, wtid); break;
+    case 2: gemv_dispatch_nr<2>(a, s, t, seq, wtid); break;
+    case 3: gemv_dispatch_nr<3>(a, s, t, seq, wtid); break;
+    default: gemv_dispatch_nr<4>(a, s, t, seq, wtid); break;
+  }
+}
+
+// Signals the task's events (after every worker's writes) and frees the
+// scheduler for the next task.
+__device__ __forceinline__ void finish_task(const KernelArgs& a, Smem& s, const Task& t,
+                                            int wtid, bool signal) {
+  worker_sync();
+  if (wtid == 0) {
+    if (signal && t.n_sig > 0) {
+      __threadfence();
+      for (int e = 0; e < t.n_sig; ++e) red_release_gpu_add(a.m.events + t.sig_ev0 + e, 1u);
+    }
+    mbar_arrive(&s.done);
+  }
+}
+
+__device__ void epilogue_qkv(const KernelArgs& a, Smem& s, const Task& t, int wtid) {
+  const ModelDev& m = a.m;
+  const StepParams& sp = step_params(a);
+  const int d = m.head_dim, G = m.group, half = d >> 1;
+  const int pos = sp.pos[0], slot = sp.kv_slot[0];
+  const int qkvR = qkv_rows(m.n_q, m.n_kv, d);
+  const int npairs = (t.row1 - t.row0) >> 1;
+  for (int pi = wtid; pi < npairs; pi += kWorkerThreads) {
+    const int r = t.row0 + 2 * pi;
+    float y0 = s.ybuf[2 * pi], y1 = s.ybuf[2 * pi + 1];
+    if (m.qkv_bias) {
+      const uint16_t* b = m.bqkv + (size_t)t.layer * qkvR;
+      y0 = y0 + bf16_to_float(b[r]);
+      y1 = y1 + bf16_to_float(b[r + 1]);
+    }
+    int which, head, dim0, w1, h1, dim1;
+    qkv_source(r, G, d, &which, &head, &dim0);
+    qkv_source(r + 1, G, d, &w1, &h1, &dim1);
+    if (which < 2) {
+      const float c = m.rope_cos[(size_t)pos * half + dim0];
+      const float sn = m.rope_sin[(size_t)pos * half + dim0];
+      const float o0 = y0 * c - y1 * sn;
+      const float o1 = y0 * sn + y1 * c;
+      y0 = o0;
+      y1 = o1;
+    }
+    if (which == 0) {
+      float* q = m.q + (size_t)head * d;
+      q[dim0] = y0;
+      q[dim1] = y1;
+    } else {
+      uint16_t* cache = which == 1 ? m.kcache : m.vcache;
+      const size_t off = kv_offset(m, slot, t.layer, head, pos);
+      cache[off + dim0] = float_to_bf16_rne(y0);
+      cache[off + dim1] = float_to_bf16_rne(y1);
+    }
+  }
+}
+
+__device__ void epilogue_residual(const KernelArgs& a, Smem& s, const Task& t, int wtid) {
+  const ModelDev& m = a.m;
+  const StepParams& sp = step_params(a);
+  const int nrows = t.row1 - t.row0;
+  const bool from_embed = t.kind == T_OPROJ && t.layer == 0;
+  int tok = 0;
+  if (from_embed) {
+    tok = sp.tokens[0];
+    if (tok < 0 || tok >= m.vocab) tok = 0;
+  }
+  for (int i = wtid; i < nrows; i += kWorkerThreads) {
+    const int row = t.row0 + i;
+    const float old = from_embed ? bf16_to_float(m.embed[(size_t)tok * m.hidden + row])
+                                 : __ldcg(m.x + row);
+    m.x[row] = old + s.ybuf[i];
+  }
+}
+
+__device__ void epilogue_swiglu(const KernelArgs& a, Smem& s, const Task& t, int wtid) {
+  const ModelDev& m = a.m;
+  const int npairs = (t.row1 - t.row0) >> 1;
+  for (int pi = wtid; pi < npairs; pi += kWorkerThreads) {
+    const float g = s.ybuf[2 * pi], u = s.ybuf[2 * pi + 1];
+    const float silu = g / (1.0f + expf(-g));
+    m.act[(t.row0 >> 1) + pi] = silu * u;
+  }
+}
+
+__device__ void epilogue_lmhead(const KernelArgs& a, Smem& s, const Task& t, int wtid) {
+  const ModelDev& m = a.m;
+  const StepParams& sp = step_params(a);
+  const int nrows = t.row1 - t.row0;
+  unsigned long long best = 0ull;
+  for (int i = wtid; i < nrows; i += kWorkerThreads) {
+    const float y = s.ybuf[i];
+    if (sp.logits) sp.logits[t.row0 + i] = y;
+    const unsigned long long k = argmax_key(y, t.row0 + i);
+    best = k > best ? k : best;
+  }
+  for (int o = 16; o; o >>= 1) {
+    const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
+    best = other > best ? other : best;
+  }
+  if ((wtid & 31) == 0) s.red64[wtid >> 5] = best;
+  worker_sync();
+  if (wtid == 0) {
+    unsigned long long b = 0ull;
+    for (int w = 0; w < kWorkerWarps; ++w) b = s.red64[w] > b ? s.red64[w] : b;
+    m.am[t.aux] = b;
+    __threadfence();
+    const uint32_t old = atom_add_acq_rel_gpu(m.tickets + m.max_batch * m.n_layers * m.n_kv, 1u);
+    s.flag = (old == (uint32_t)m.n_lm_tasks * (s.epoch + 1u) - 1u) ? 1 : 0;
+  }
+  worker_sync();
+  if (s.flag) {
+    // Last LM task of the step: reduce every task's candidate.
+    unsigned long long b = 0ull;
+    for (int i = wtid; i < m.n_lm_tasks; i += kWorkerThreads) {
+      const unsigned long long v = __ldcg(m.am + i);
+      b = v > b ? v : b;
+    }
+    for (int o = 16; o; o >>= 1) {
+      const unsigned long long other = __shfl_xor_sync(0xffffffffu, b, o);
+      b = other > b ? other : b;
+    }
+    if ((wtid & 31) == 0) s.red64[wtid >> 5] = b;
+    worker_sync();
+    if (wtid == 0) {
+      unsigned long long g = 0ull;
+      for (int w = 0; w < kWorkerWarps; ++w) g = s.red64[w] > g ? s.red64[w] : g;
+      const int id = (int)(0xffffffffu - (uint32_t)(g & 0xffffffffull));
+      if (sp.next_ids) sp.next_ids[0] = id;
+      __threadfence();
+      red_release_gpu_add(m.epoch, 1u);
+    }
+  }
+}
+
+// ------------------------------------------------------- worker: attention
+
+template <int DPL>
+__device__ __forceinline__ void load_kv_row(const uint16_t* p, float (&v)[DPL]) {
+  if constexpr (DPL == 4) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    v[0] = bf_lo(u.x); v[1] = bf_hi(u.x); v[2] = bf_lo(u.y); v[3] = bf_hi(u.y);
+  } else {
+    const uint32_t u = *reinterpret_cast<const uint32_t*>(p);
+    v[0] = bf_lo(u); v[1] = bf_hi(u);
+  }
+}
+
+template <int DPL>
+__device__ __forceinline__ void load_kv_row_global(const uint16_t* p, float (&v)[DPL]) {
+  if constexpr (DPL == 4) {
+    const uint2 u = __ldcg(reinterpret_cast<const uint2*>(p));
+    v[0] = bf_lo(u.x); v[1] = bf_hi(u.x); v[2] = bf_lo(u.y); v[3] = bf_hi(u.y);
+  } else {
+    const uint32_t u = __ldcg(reinterpret_cast<const unsigned int*>(p));
+    v[0] = bf_lo(u); v[1] = bf_hi(u);
+  }
+}
+
+template <int DPL, int G>
+struct AttnState {
+  float q[G][DPL];
+  float o[G][DPL];
+  float mx[G];
+  float l[G];
+};
+
+// Online softmax update with one key ("Hạt nhân là gì ...": running maximum
+// and running sum, earlier partial results rescaled).
+template <int DPL, int G>
+__device__ __forceinline__ void attn_key(AttnState<DPL, G>& st, const float (&k)[DPL],
+                                         const float (&v)[DPL]) {
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    float p = 0.f;
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) p = fmaf(st.q[h][i], k[i], p);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
+    const float mn = fmaxf(st.mx[h], p);
+    const float c = __expf(st.mx[h] - mn);
+    const float e = __expf(p - mn);
+    st.l[h] = fmaf(st.l[h], c, e);
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) st.o[h][i] = fmaf(st.o[h][i], c, e * v[i]);
+    st.mx[h] = mn;
+  }
+}
+
+template <int DPL, int G>
+__device__ void attn_task(const KernelArgs& a, Smem& s, const Task& t, uint32_t& seq, int wtid) {
+  const ModelDev& m = a.m;
+  const StepParams& sp = step_params(a);
+  const int d = m.head_dim, S = m.attn_splits;
+  const int warp = wtid >> 5, lane = wtid & 31;
+  const int g = t.row0, split = t.row1, b = t.req;
+  const AttnRange r = attn_range(t, sp, m);
+  if (r.active) {
+    AttnState<DPL, G> st;
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) {
+        st.q[h][i] = __ldcg(m.q + (size_t)(g * G + h) * d + lane * DPL + i) * m.attn_scale;
+        st.o[h][i] = 0.f;
+      }
+      st.mx[h] = -INFINITY;
+      st.l[h] = 0.f;
+    }
+    const int kpc = attn_keys_per_chunk(d);
+    for (int k = r.k0; k < r.old_end; k += kpc) {
+      const int nk = min(kpc, r.old_end - k);
+      const int slot = seq % kRingSlots;
+      wait_full(s, seq, m);
+      const uint16_t* kb = reinterpret_cast<const uint16_t*>(s.ring[slot]);
+      const uint16_t* vb = reinterpret_cast<const uint16_t*>(s.ring[slot] + kSlotBytes / 2);
+      for (int j = warp; j < nk; j += kWorkerWarps) {
+        float kv[DPL], vv[DPL];
+        load_kv_row<DPL>(kb + (size_t)j * d + lane * DPL, kv);
+        load_kv_row<DPL>(vb + (size_t)j * d + lane * DPL, vv);
+        attn_key<DPL, G>(st, kv, vv);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.empty[slot]);
+      ++seq;
+    }
+    // The newest key (written by this step's QKV tasks) is read from memory.
+    const int pos = sp.pos[b];
+    if (pos >= r.k0 && pos < r.k1 && warp == (kWorkerWarps - 1)) {
+      const size_t off = kv_offset(m, sp.kv_slot[b], t.layer, g, pos);
+      float kv[DPL], vv[DPL];
+      load_kv_row_global<DPL>(m.kcache + off + lane * DPL, kv);
+      load_kv_row_global<DPL>(m.vcache + off + lane * DPL, vv);
+      attn_key<DPL, G>(st, kv, vv);
+    }
+    // Tree merge of the 16 warps' (max, sum, output) through shared memory.
+    float* buf = s.scratch;
+    const int stride_w = G * (d + 2);
+    for (int half = kWorkerWarps / 2; half >= 1; half >>= 1) {
+      if (warp >= half && warp < 2 * half) {
+        float* dst = buf + (warp - half) * stride_w;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+#pragma unroll
+          for (int i = 0; i < DPL; ++i) dst[h * (d + 2) + lane * DPL + i] = st.o[h][i];
+          if (lane == 0) {
+            dst[h * (d + 2) + d] = st.mx[h];
+            dst[h * (d + 2) + d + 1] = st.l[h];
+          }
+        }
+      }
+      worker_sync();
+      if (warp < half) {
+        const float* src = buf + warp * stride_w;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float m2 = src[h * (d + 2) + d], l2 = src[h * (d + 2) + d + 1];
+          if (m2 != -INFINITY) {
+            if (st.mx[h] == -INFINITY) {
+              st.mx[h] = m2;
+              st.l[h] = l2;
+#pragma unroll
+              for (int i = 0; i < DPL; ++i) st.o[h][i] = src[h * (d + 2) + lane * DPL + i];
+            } else {
+              const float mn = fmaxf(st.mx[h], m2);
+              const float c1 = __expf(st.mx[h] - mn), c2 = __expf(m2 - mn);
+              st.l[h] = st.l[h] * c1 + l2 * c2;
+#pragma unroll
+              for (int i = 0; i < DPL; ++i)
+                st.o[h][i] = st.o[h][i] * c1 + src[h * (d + 2) + lane * DPL + i] * c2;
+              st.mx[h] = mn;
+            }
+          }
+        }
+      }
+      worker_sync();
+    }
+    if (warp == 0) {
+      float* part = m.part + ((size_t)(b * m.n_kv + g) * S + split) * G * (d + 2);
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) part[h * (d + 2) + lane * DPL + i] = st.o[h][i];
+        if (lane == 0) {
+          part[h * (d + 2) + d] = st.mx[h];
+          part[h * (d + 2) + d + 1] = st.l[h];
+        }
+      }
+    }
+  }
+  // Ticket: the last split of this (slot, group) merges all splits.
+  worker_sync();
+  if (wtid == 0) {
+    __threadfence();
+    const uint32_t old = atom_add_acq_rel_gpu(m.tickets + t.aux, 1u);
+    s.flag = (old == (uint32_t)S * (s.epoch + 1u) - 1u) ? 1 : 0;
+  }
+  worker_sync();
+  if (s.flag) {
+    if (r.active) {
+      const float* part = m.part + (size_t)(b * m.n_kv + g) * S * G * (d + 2);
+      for (int idx = wtid; idx < G * d; idx += kWorkerThreads) {
+        const int h = idx / d, i = idx - h * d;
+        float M = -INFINITY;
+        for (int sp_i = 0; sp_i < S; ++sp_i)
+          M = fmaxf(M, __ldcg(part + ((size_t)sp_i * G + h) * (d + 2) + d));
+        float num = 0.f, den = 0.f;
+        for (int sp_i = 0; sp_i < S; ++sp_i) {
+          const float* ps = part + ((size_t)sp_i * G + h) * (d + 2);
+          const float ls = __ldcg(ps + d + 1);
+          if (ls == 0.f) continue;
+          const float c = __expf(__ldcg(ps + d) - M);
+          num = fmaf(c, __ldcg(ps + i), num);
+          den = fmaf(c, ls, den);
+        }
+        m.attn[(size_t)(g * G + h) * d + i] = num / den;
+      }
+    }
+    worker_sync();
+    if (wtid == 0) {
+      __threadfence();
+      red_release_gpu_add(m.events + t.sig_ev0, 1u);
+    }
+  }
+}
+
+__device__ void attn_dispatch(const KernelArgs& a, Smem& s, const Task& t, uint32_t& seq, int wtid) {
+  const int G = a.m.group;
+  if (a.m.head_dim == 128) {
+    switch (G) {
+      case 1: attn_task<4, 1>(a, s, t, seq, wtid); break;
+      case 2: attn_task<4, 2>(a, s, t, seq, wtid); break;
+      case 4: attn_task<4, 4>(a, s, t, seq, wtid); break;
+      default: if (wtid == 0) set_error(a.m, MK_ERR_UNSUPPORTED, G); break;
+    }
+  } else {
+    switch (G) {
+      case 1: attn_task<2, 1>(a, s, t, seq, wtid); break;
+      case 2: attn_task<2, 2>(a, s, t, seq, wtid); break;
+      case 4: attn_task<2, 4>(a, s, t, seq, wtid); break;
+      case 7: attn_task<2, 7>(a, s, t, seq, wtid); break;
+      case 8: attn_task<2, 8>(a, s, t, seq, wtid); break;
+      default: if (wtid == 0) set_error(a.m, MK_ERR_UNSUPPORTED, G); break;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ worker
+
+__device__ void worker(const KernelArgs& a, Smem& s, int q0, int q1) {
+  const int wtid = threadIdx.x - kFirstWorkerWarp * 32;
+  uint32_t seq = 0;
+  int i = 0;
+  for (int qi = q0; qi < q1; ++qi, ++i) {
+    const Task t = a.tasks[a.queue[qi]];
+    const bool go = wait_bounded(s, &s.ready, i & 1, a.m, kWaitReady);
+    // all workers agree: the flag was published before the ready arrival
+    worker_sync();
+    if (!go || aborting(s)) break;
+    switch (t.kind) {
+      case T_ATTN:
+        attn_dispatch(a, s, t, seq, wtid);
+        finish_task(a, s, t, wtid, false);
+        break;
+      case T_LMHEAD:
+        gemv_core(a, s, t, seq, wtid);
+        epilogue_lmhead(a, s, t, wtid);
+        finish_task(a, s, t, wtid, false);
+        break;
+      default:
+        gemv_core(a, s, t, seq, wtid);
+        if (t.kind == T_QKV) epilogue_qkv(a, s, t, wtid);
+        else if (t.kind == T_GATEUP) epilogue_swiglu(a, s, t, wtid);
+        else epilogue_residual(a, s, t, wtid);
+        finish_task(a, s, t, wtid, true);
+        break;
+    }
+  }
+}
+
+__global__ void __maxnreg__(112) mk_step_kernel(const __grid_constant__ KernelArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  Smem& s = *reinterpret_cast<Smem*>(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int q0 = a.queue_off[blockIdx.x], q1 = a.queue_off[blockIdx.x + 1];
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kRingSlots; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.empty[i], kWorkerWarps);
+    }
+    mbar_init(&s.ready, 1);
+    mbar_init(&s.done, 1);
+    s.abort_flag = 0;
+    s.consumed_seq = 0;
+    s.flag = 0;
+    s.epoch = *reinterpret_cast<volatile uint32_t*>(a.m.epoch);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (q0 == q1) return;
+  if (warp == kProducerWarp) {
+    if (lane == 0) producer(a, s, q0, q1);
+  } else if (warp == kSchedulerWarp) {
+    if (lane == 0) scheduler(a, s, q0, q1);
+  } else {
+    worker(a, s, q0, q1);
+  }
+}
+
+// ------------------------------------------------------------ weight packing
+
+// Fused QKV: packed row r <- wq / wk / wv row given by qkv_source.
+__global__ void pack_qkv_kernel(uint16_t* dst, const uint16_t* wq, const uint16_t* wk,
+                                const uint16_t* wv, int H, int G, int d, int rows) {
+  const int r = blockIdx.x;
+  if (r >= rows) return;
+  int which, head, dim;
+  qkv_source(r, G, d, &which, &head, &dim);
+  const uint16_t* src = which == 0 ? wq : (which == 1 ? wk : wv);
+  const uint4* s4 = reinterpret_cast<const uint4*>(src + ((size_t)head * d + dim) * H);
+  uint4* d4 = reinterpret_cast<uint4*>(dst + (size_t)r * H);
+  for (int i = threadIdx.x; i < H / 8; i += blockDim.x) d4[i] = s4[i];
+}
+
+__global__ void pack_qkv_bias_kernel(uint16_t* dst, const uint16_t* bq, const uint16_t* bk,
+                                     const uint16_t* bv, int G, int d, int rows) {
+  const int r = blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= rows) return;
+  int which, head, dim;
+  qkv_source(r, G, d, &which, &head, &dim);
+  const uint16_t* src = which == 0 ? bq : (which == 1 ? bk : bv);
+  dst[r] = src[(size_t)head * d + dim];
+}
+
+// gate/up interleaved: packed row 2j = gate row j, 2j + 1 = up row j.
+__global__ void pack_gateup_kernel(uint16_t* dst, const uint16_t* wg, const uint16_t* wu, int H,
+                                   int F) {
+  const int r = blockIdx.x;
+  if (r >= 2 * F) return;
+  const uint16_t* src = ((r & 1) ? wu : wg) + (size_t)(r >> 1) * H;
+  const uint4* s4 = reinterpret_cast<const uint4*>(src);
+  uint4* d4 = reinterpret_cast<uint4*>(dst + (size_t)r * H);
+  for (int i = threadIdx.x; i < H / 8; i += blockDim.x) d4[i] = s4[i];
+}
+
+}  // namespace mk
+
+// Host-visible launch helpers (called from api.cu).
+namespace mk {
+size_t step_kernel_smem_bytes() { return sizeof(Smem); }
+const void* step_kernel_ptr() { return reinterpret_cast<const void*>(&mk_step_kernel); }
+
+cudaError_t launch_pack_qkv(uint16_t* dst, const uint16_t* wq, const uint16_t* wk,
+                            const uint16_t* wv, int H, int G, int d, int rows, cudaStream_t st) {
+  pack_qkv_kernel<<<rows, 128, 0, st>>>(dst, wq, wk, wv, H, G, d, rows);
+  return cudaGetLastError();
+}
+cudaError_t launch_pack_qkv_bias(uint16_t* dst, const uint16_t* bq, const uint16_t* bk,
+                                 const uint16_t* bv, int G, int d, int rows, cudaStream_t st) {
+  pack_qkv_bias_kernel<<<(rows + 255) / 256, 256, 0, st>>>(dst, bq, bk, bv, G, d, rows);
+  return cudaGetLastError();
+}
+cudaError_t launch_pack_gateup(uint16_t* dst, const uint16_t* wg, const uint16_t* wu, int H, int F,
+                               cudaStream_t st) {
+  pack_gateup_kernel<<<2 * F, 128, 0, st>>>(dst, wg, wu, H, F);
+  return cudaGetLastError();
+}
+cudaError_t launch_step(const KernelArgs& args, int grid, bool cooperative, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = sizeof(Smem);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = cooperative ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, mk_step_kernel, args);
+}
+}  // namespace mk

@@ -1,0 +1,113 @@
+"""Teacher-forced comparison of the CUDA path with the oracle.
+
+The oracle runs the prompt and then greedy decoding on CPU; its tokens are
+fed to the CUDA path step by step ("teacher forcing"), and at every step the
+two sides' logits, final residual stream and greedy ids are compared.
+
+Acceptance (bf16 weights, fp32 accumulation): logits max-abs <= 3e-2,
+residual-stream relative L2 <= 1e-2, identical greedy id wherever the
+oracle's top-1/top-2 margin is >= 0.1.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+from typing import List
+
+import numpy as np
+
+LOGITS_ATOL = 3e-2
+HIDDEN_REL_L2 = 1e-2
+MARGIN = 0.1
+
+
+@dataclass
+class OracleTrace:
+    prompt: List[int]
+    feed: List[int]                 # token fed at each decode step
+    logits: List[np.ndarray] = field(default_factory=list)   # [0] = prefill's last position
+    hidden: List[np.ndarray] = field(default_factory=list)
+    ids: List[int] = field(default_factory=list)
+
+
+def oracle_trace(model, w_cpu, prompt, steps: int, max_seq: int, kv_bf16: bool = True):
+    import oracle
+    om = oracle.OracleModel(model, w_cpu, kv_bf16=kv_bf16)
+    st = om.new_state(max_seq)
+    tr = OracleTrace(prompt=list(prompt), feed=[])
+    for p, t in enumerate(prompt):
+        nid, lg, hid = om.decode(st, int(t), p, want_logits=(p == len(prompt) - 1))
+    tr.logits.append(lg)
+    tr.hidden.append(hid)
+    tr.ids.append(nid)
+    for s in range(steps):
+        tok = tr.ids[-1]
+        tr.feed.append(tok)
+        nid, lg, hid = om.decode(st, tok, len(prompt) + s)
+        tr.logits.append(lg)
+        tr.hidden.append(hid)
+        tr.ids.append(nid)
+    return tr, om, st
+
+
+def margin(lg: np.ndarray) -> float:
+    top2 = np.partition(lg, -2)[-2:]
+    return float(top2[1] - top2[0])
+
+
+@dataclass
+class StepReport:
+    step: int
+    logits_err: float
+    hidden_rel: float
+    id_ok: bool
+    margin: float
+
+
+def compare(tr: OracleTrace, got_logits, got_hidden, got_ids) -> List[StepReport]:
+    out = []
+    for s, (lg, hid, nid) in enumerate(zip(tr.logits, tr.hidden, tr.ids)):
+        e = float(np.abs(got_logits[s] - lg).max())
+        rel = float("nan")
+        if got_hidden[s] is not None:
+            rel = float(np.linalg.norm(got_hidden[s] - hid) / np.linalg.norm(hid))
+        m = margin(lg)
+        ok = (m < MARGIN) or (int(got_ids[s]) == int(nid))
+        out.append(StepReport(s, e, rel, ok, m))
+    return out
+
+
+def assert_within(reports: List[StepReport]):
+    bad = [r for r in reports if not (r.logits_err <= LOGITS_ATOL and
+                                       (np.isnan(r.hidden_rel) or r.hidden_rel <= HIDDEN_REL_L2)
+                                       and r.id_ok)]
+    assert not bad, "\n".join(str(r) for r in bad[:10])
+
+
+def run_gpu(dec, model, tr: OracleTrace, want_hidden: bool = True):
+    """Prefill + teacher-forced decode through the C-ABI; returns per-step
+    (logits, hidden, id) as host arrays.  Step 0 is the prefill's last
+    position (no residual readback: the prefill's hidden is the same kernel)."""
+    import torch
+    V, H = model.vocab, model.hidden
+    P = len(tr.prompt)
+    logits = torch.empty(V, device="cuda", dtype=torch.float32)
+    ids = torch.empty(1, device="cuda", dtype=torch.int32)
+    hidden = torch.empty(H, device="cuda", dtype=torch.float32)
+    toks = torch.tensor(tr.prompt, dtype=torch.int32, device="cuda")
+    dec.prefill(toks, [0, P], logits, ids)
+    dec.copy_hidden(hidden)
+    torch.cuda.synchronize()
+    gl, gh, gi = [logits.cpu().numpy().copy()], [hidden.cpu().numpy().copy()], [int(ids.item())]
+    tok = torch.empty(1, device="cuda", dtype=torch.int32)
+    for s, t in enumerate(tr.feed):
+        tok.fill_(int(t))
+        dec.decode(tok, [P + s], logits, ids)
+        if want_hidden:
+            dec.copy_hidden(hidden)
+        torch.cuda.synchronize()
+        gl.append(logits.cpu().numpy().copy())
+        gh.append(hidden.cpu().numpy().copy() if want_hidden else None)
+        gi.append(int(ids.item()))
+    rc = dec.status()
+    assert rc == 0, f"device status {rc}: {dec.last_error()}"
+    return gl, gh, gi
