@@ -1,0 +1,371 @@
+"""Decode-step benchmark: one JSON line per run.
+
+Workload: Llama-3-8B-shaped decoder (32 layers, hidden 4096, 32 q / 8 KV
+heads, head_dim 128, SwiGLU 14336, vocab 128256), bf16 random-init weights
+N(0, 0.02), batch 1, 39-token random prompt, then greedy decoding.  A "step"
+is one decode step: one token through the whole model (one persistent
+kernel launch).  W untimed warm-up steps, then exactly K timed steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+--impl reference times the CPU oracle (the only reference this method has)
+on the host's cores on a bounded sample of the same workload.
+Multi-GPU (under torchrun): independent replicas, one request per GPU, no
+collective on the data path; time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode ms/token (batch 1, Llama-3-8B-shape) & achieved HBM GB/s vs 8 TB/s peak"
+NOMINAL_HBM = 8000.0   # GB/s, the metric's denominator
+PROMPT = 39
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(n_gpus):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v, world):
+    if world <= 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def oracle_sample(model, w_cpu, n_steps: int, budget_s: float):
+    """Times the oracle's decode step (positions 0..) on host cores."""
+    import oracle
+    om = oracle.OracleModel(model, w_cpu)
+    st = om.new_state(n_steps + 1)
+    tok = 1
+    times = []
+    t_all = time.perf_counter()
+    for p in range(n_steps):
+        t0 = time.perf_counter()
+        tok, _, _ = om.decode(st, tok, p, want_logits=False)
+        times.append(time.perf_counter() - t0)
+        if time.perf_counter() - t_all > budget_s and len(times) >= 2:
+            break
+    return times, oracle.num_threads()
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import torch
+
+    from persistent_megakernel_03_b200 import synth
+    model = synth.LLAMA8B
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    w = synth.make_model(model, 0, device=dev)
+    w_cpu = {k: v.cpu() for k, v in w.items()}
+    del w
+    budget = float(os.environ.get("MK_REF_BUDGET_S", "60"))
+    n = max(2, min(args.warmup + args.steps, 64))
+    times, cores = oracle_sample(model, w_cpu, n, budget)
+    warm = min(1, len(times) - 1)
+    timed = times[warm:]
+    ms = 1e3 * sum(timed) / len(timed)
+    sample = (f"{len(timed)} oracle decode steps of the Llama-3-8B shape at positions "
+              f"{warm}..{len(times) - 1} (after {warm} untimed), bf16 weights widened to fp32 "
+              f"on the fly, {cores} OpenMP threads")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": ms, "unit": "ms/token",
+        "n_gpus": args.gpus, "steps": len(timed), "warmup": warm, "ms_per_step": ms,
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": "llama-3-8b-shape decode, batch 1, 39-token random prompt, "
+                               "greedy decode", "sample": "bounded oracle sample"},
+        "cpu_baseline": {"value": ms, "unit": "ms/token", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": ms, "unit": "ms/token", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def load_traffic():
+    """DRAM traffic per launch from the committed ncu summary, when it was
+    taken on the current kernel sources."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "megakernel_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    h = hashlib.sha256()
+    for name in ("kernel.cu", "mk_internal.h", "ptx.cuh"):
+        with open(os.path.join(ROOT, "persistent_megakernel_03_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    if rec.get("source_sha256") != h.hexdigest():
+        return None
+    return rec.get("traffic_bytes_per_launch_full")
+
+
+def run_mk(args):
+    import numpy as np
+    import torch
+
+    from persistent_megakernel_03_b200 import binding, roofline, synth
+
+    rank, world, local = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    model = synth.LLAMA8B
+    W, K = args.warmup, args.steps
+    max_seq = PROMPT + W + K + 1
+    w = synth.make_model(model, 0, device="cuda")
+    stream = torch.cuda.current_stream()
+    dec = binding.Decoder(model, w, max_seq, stream=stream)
+    prompt = synth.make_prompt(PROMPT, model.vocab).cuda()
+    ids = [torch.zeros(1, dtype=torch.int32, device="cuda") for _ in range(2)]
+
+    def prefill():
+        dec.prefill(prompt, [0, PROMPT], None, ids[0])
+
+    def run_steps(first_pos, n, evs=None):
+        for k in range(n):
+            dec.decode(ids[k % 2], [first_pos + k], None, ids[(k + 1) % 2])
+            if evs is not None:
+                evs[k + 1].record(stream)
+
+    # ---- device-timed region (megakernel)
+    prefill()
+    run_steps(PROMPT, W)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+    torch.cuda.synchronize()
+    barrier(world)
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize()
+        evs[0].record(stream)
+        run_steps(PROMPT + W, K, evs)
+        torch.cuda.synchronize()
+    barrier(world)
+    rc = dec.status()
+    if rc != 0:
+        raise RuntimeError(f"device status {rc}: {dec.last_error()}")
+    per_step = [evs[k].elapsed_time(evs[k + 1]) for k in range(K)]
+    total_ms = evs[0].elapsed_time(evs[K])
+    total_ms = max_over_ranks(total_ms, world)
+    value = total_ms / (K * world)
+    positions = list(range(PROMPT + W, PROMPT + W + K))
+    bytes_mean = sum(roofline.step_bytes(model, [p]) for p in positions) / K
+    avg_launch_s = (sum(per_step) / K) * 1e-3
+    achieved = bytes_mean / avg_launch_s / 1e9
+    peak, peak_src = measured_peaks()
+
+    # ---- read-stream probe: practical read ceiling on this GPU
+    probe_buf = torch.empty(4 * 2**30, dtype=torch.uint8, device="cuda")
+    sink = torch.zeros(1, dtype=torch.int64, device="cuda")
+    for _ in range(3):
+        binding.read_probe(probe_buf, sink)
+    pe = [torch.cuda.Event(enable_timing=True) for _ in range(11)]
+    pe[0].record(stream)
+    for i in range(10):
+        binding.read_probe(probe_buf, sink)
+        pe[i + 1].record(stream)
+    torch.cuda.synchronize()
+    probe_gbs = max(probe_buf.numel() / (pe[i].elapsed_time(pe[i + 1]) * 1e-3) / 1e9
+                    for i in range(10))
+    del probe_buf
+
+    # ---- baselines: the same task bodies, one launch per operator
+    baselines = {}
+    nb = min(K, 64)
+    for name, mode in (("per_op", binding.MODE_PER_OP), ("per_op_graph", binding.MODE_PER_OP_GRAPH)):
+        dec.set_mode(mode)
+        prefill()
+        run_steps(PROMPT, min(W, 4))
+        bev = [torch.cuda.Event(enable_timing=True) for _ in range(nb + 1)]
+        torch.cuda.synchronize()
+        bev[0].record(stream)
+        run_steps(PROMPT + min(W, 4), nb, bev)
+        torch.cuda.synchronize()
+        steps_ms = [bev[k].elapsed_time(bev[k + 1]) for k in range(nb)]
+        baselines[name] = {"ms_per_token": statistics.median(steps_ms), "steps": nb,
+                           "launches_per_step": dec_stage_count(dec)}
+    dec.set_mode(binding.MODE_MEGAKERNEL)
+    rc = dec.status()
+    if rc != 0:
+        raise RuntimeError(f"device status {rc}: {dec.last_error()}")
+
+    # ---- end to end through the host entry point (token in, id out, per step)
+    prefill()
+    torch.cuda.synchronize()
+    tok = int(ids[0].item())
+    for k in range(W):
+        tok = dec.decode_host([tok], [PROMPT + k])[0]
+    barrier(world)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for k in range(K):
+        tok = dec.decode_host([tok], [PROMPT + W + k])[0]
+    t1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(t0.elapsed_time(t1), world) / (K * world)
+
+    clocks = clk.summary()
+    line = {
+        "metric": METRIC, "value": value, "unit": "ms/token", "n_gpus": world, "steps": K,
+        "warmup": W, "ms_per_step": total_ms / K, "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "weights": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "llama-3-8b-shape decode, batch 1, 39-token random prompt, "
+                               f"greedy decode steps {PROMPT + W}..{PROMPT + W + K - 1} timed",
+                   "l2": "inputs larger than L2 (15.0 GB of weights streamed per step)",
+                   "parallelism": f"replicas x{world}"},
+        "tok_per_s": 1e3 / value,
+        "step_ms": {"median": statistics.median(per_step),
+                    "p10": float(np.percentile(per_step, 10)),
+                    "p90": float(np.percentile(per_step, 90))},
+        "achieved_gbs": achieved, "frac_of_8tbs": achieved / NOMINAL_HBM,
+        "read_probe_gbs": probe_gbs, "frac_of_read_probe": achieved / probe_gbs,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": peak_src,
+                     "traffic": load_traffic(),
+                     "bytes_per_launch": bytes_mean},
+        "baselines": baselines,
+        "clocks": clocks,
+        "e2e": {"value": e2e_ms, "unit": "ms/token", "h2d_bytes_per_step": 4,
+                "d2h_bytes_per_step": 4},
+        "gpu_launches": K,
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        del w
+        dec.close()
+        torch.cuda.empty_cache()
+        w2 = synth.make_model(model, 0, device="cuda")
+        w_cpu = {k: v.cpu() for k, v in w2.items()}
+        del w2
+        times, cores = oracle_sample(model, w_cpu, 4, 25.0)
+        timed = times[1:] if len(times) > 1 else times
+        cms = 1e3 * sum(timed) / len(timed)
+        line["cpu_baseline"] = {
+            "value": cms, "unit": "ms/token", "cores": cores, "kind": "oracle",
+            "sample": f"{len(timed)} oracle decode steps of the same Llama-3-8B-shape model "
+                      f"at positions {len(times) - len(timed)}..{len(times) - 1}, fp32 with "
+                      f"bf16 weights widened on the fly"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def dec_stage_count(dec) -> int:
+    return 5 * dec.model.n_layers + 1
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=504)
+    ap.add_argument("--warmup", type=int, default=8)
+    ap.add_argument("--impl", default="mk", choices=["mk", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_mk(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -152,6 +152,13 @@ int mk_status(mk_ctx* ctx);
 const char* mk_last_error(const mk_ctx* ctx);
 void mk_destroy(mk_ctx* ctx);
 
+/* Read-only HBM stream probe: every byte of src_dev[0, bytes) is loaded
+ * once with 128-bit loads by a grid of (SMs x 4) CTAs; a value derived from
+ * the data is written to sink_dev[0] so nothing is elided.  bytes must be a
+ * multiple of 16 and src_dev 16-byte aligned.  Enqueued on `stream`.  Used to
+ * measure the practical read ceiling the decode step is compared with. */
+int mk_read_probe(const void* src_dev, size_t bytes, unsigned long long* sink_dev, void* stream);
+
 /* ---------------------------------------------------------------------
  * Introspection of the task graph (host only, no GPU needed).
  * mk_plan_build makes the same graph mk_create would for `num_ctas` CTAs.

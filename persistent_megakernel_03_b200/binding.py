@@ -25,7 +25,7 @@ EXPORTS = ("mk_create", "mk_prefill", "mk_decode_step", "mk_decode_step_host", "
            "mk_kv_pointer", "mk_copy_kv", "mk_set_mode", "mk_status", "mk_last_error",
            "mk_destroy", "mk_plan_build", "mk_plan_get_info", "mk_plan_get_tasks",
            "mk_plan_get_queue", "mk_plan_get_event_counts", "mk_plan_destroy",
-           "mk_qkv_row_source")
+           "mk_qkv_row_source", "mk_read_probe")
 
 
 class MkError(RuntimeError):
@@ -111,6 +111,7 @@ def lib(build_if_missing: bool = True):
     L.mk_plan_destroy.argtypes = [vp]
     L.mk_plan_destroy.restype = None
     L.mk_qkv_row_source.argtypes = [C.POINTER(Config), i, ip, ip, ip]
+    L.mk_read_probe.argtypes = [vp, C.c_size_t, vp, vp]
     _lib = L
     return L
 
@@ -262,3 +263,11 @@ class Decoder:
 
     def last_error(self) -> str:
         return lib().mk_last_error(self.h).decode(errors="replace")
+
+
+def read_probe(src_dev, sink_dev, stream=None):
+    """Enqueues one read-only pass over ``src_dev`` (a contiguous CUDA tensor)."""
+    import torch
+    st = stream if stream is not None else torch.cuda.current_stream()
+    nbytes = src_dev.numel() * src_dev.element_size()
+    _check(lib().mk_read_probe(src_dev.data_ptr(), nbytes, sink_dev.data_ptr(), st.cuda_stream))

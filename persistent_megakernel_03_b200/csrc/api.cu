@@ -20,6 +20,8 @@ cudaError_t launch_pack_qkv_bias(uint16_t*, const uint16_t*, const uint16_t*, co
                                  int, int, cudaStream_t);
 cudaError_t launch_pack_gateup(uint16_t*, const uint16_t*, const uint16_t*, int, int, cudaStream_t);
 cudaError_t launch_step(const KernelArgs& args, int grid, bool cooperative, cudaStream_t st);
+cudaError_t launch_read_probe(const void* src, size_t bytes, unsigned long long* sink, int sms,
+                              cudaStream_t st);
 }  // namespace mk
 
 using namespace mk;
@@ -511,4 +513,17 @@ extern "C" void mk_destroy(mk_ctx* ctx) {
   cudaStreamSynchronize(ctx->stream);
   release(ctx);
   delete ctx;
+}
+
+extern "C" int mk_read_probe(const void* src_dev, size_t bytes, unsigned long long* sink_dev,
+                             void* stream) {
+  if (!src_dev || !sink_dev || bytes == 0 || bytes % 16 || !aligned16(src_dev))
+    return fail(nullptr, MK_ERR_INVALID_ARG, "read probe: bad buffer");
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return fail(nullptr, MK_ERR_CUDA, "read probe: no device");
+  cudaError_t e = launch_read_probe(src_dev, bytes, sink_dev, sms, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(nullptr, MK_ERR_CUDA, cudaGetErrorString(e));
+  return MK_OK;
 }
