@@ -205,11 +205,13 @@ def run_mk(args):
     rank, world, local = dist_setup(args.gpus)
     torch.cuda.set_device(local)
     model = synth.LLAMA8B
+    if args.layers:
+        model = model.with_layers(args.layers)
     W, K = args.warmup, args.steps
     max_seq = PROMPT + W + K + 1
     w = synth.make_model(model, 0, device="cuda")
     stream = torch.cuda.current_stream()
-    dec = binding.Decoder(model, w, max_seq, stream=stream)
+    dec = binding.Decoder(model, w, max_seq, stream=stream, l2_prefetch=args.l2_prefetch)
     prompt = synth.make_prompt(PROMPT, model.vocab).cuda()
     ids = [torch.zeros(1, dtype=torch.int32, device="cuda") for _ in range(2)]
 
@@ -299,6 +301,23 @@ def run_mk(args):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(t0.elapsed_time(t1), world) / (K * world)
 
+    trace_summary = None
+    if args.trace:
+        # a few more steps with the per-task timeline on (not part of the timing)
+        from persistent_megakernel_03_b200 import trace as mktrace
+        plan = binding.Plan(model, max_seq, dec_num_ctas())
+        tbuf = torch.zeros((plan.info.n_tasks, 8), dtype=torch.int64, device="cuda")
+        prefill()
+        run_steps(PROMPT, W)
+        dec.set_trace(tbuf)
+        run_steps(PROMPT + W, 1)
+        torch.cuda.synchronize()
+        dec.set_trace(None)
+        rows = tbuf.cpu().numpy().astype("uint64").tolist()
+        trace_summary = mktrace.summarize(rows, plan.tasks())
+        with open(args.trace, "w") as f:
+            json.dump(trace_summary, f, indent=1)
+
     clocks = clk.summary()
     line = {
         "metric": METRIC, "value": value, "unit": "ms/token", "n_gpus": world, "steps": K,
@@ -325,6 +344,12 @@ def run_mk(args):
                 "d2h_bytes_per_step": 4},
         "gpu_launches": K,
     }
+    if args.layers:
+        line["config"]["workload"] += f" [profiling case: {args.layers} layers]"
+    if args.l2_prefetch:
+        line["config"]["l2_prefetch_chunks"] = args.l2_prefetch
+    if trace_summary:
+        line["trace"] = {k: trace_summary[k] for k in ("step_us", "mean_cta_busy_frac")}
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         del w
         dec.close()
@@ -351,6 +376,11 @@ def dec_stage_count(dec) -> int:
     return 5 * dec.model.n_layers + 1
 
 
+def dec_num_ctas() -> int:
+    import torch
+    return torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -358,6 +388,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--impl", default="mk", choices=["mk", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--trace", default=None, help="write a per-task timeline summary here")
+    ap.add_argument("--l2-prefetch", type=int, default=0,
+                    help="ring chunks prefetched into L2 beyond the ring (0: library default)")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="profiling aid: a shallower model of the same widths (not a bench line)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

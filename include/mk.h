@@ -97,6 +97,9 @@ typedef struct {
   int attn_splits;   /* 0: automatic split-KV factor per KV head */
   int timeout_ms;    /* device-side wait limit per event (0: 1000 ms) */
   int mode;          /* MK_MODE_* used by mk_decode_step and mk_prefill */
+  int l2_prefetch;   /* when a CTA's next task must wait for its event, the number
+                        of 32 KB weight chunks past its shared-memory ring it
+                        prefetches into L2 meanwhile; 0: default (off), < 0: off */
 } mk_options;
 
 typedef struct mk_ctx mk_ctx;
@@ -141,6 +144,14 @@ int mk_kv_pointer(mk_ctx* ctx, int req, int layer, int kv_head, int which, void*
 /* Copies positions [0, n) of one K (which=0) or V (which=1) cache head, bf16
  * n x head_dim, to dst_dev (enqueued on the context's stream). */
 int mk_copy_kv(mk_ctx* ctx, int req, int layer, int kv_head, int which, int n, void* dst_dev);
+
+/* Per-task timeline of later megakernel steps (diagnostics).  trace_dev
+ * holds 8 uint64 per entry of the megakernel's task queues (mk_plan_info
+ * n_tasks entries), %globaltimer ns: 0 the task's event was satisfied,
+ * 1 workers started, 2 input loaded, 3 first ring chunk ready, 4 last chunk
+ * consumed, 5 epilogue done, 6 finished; 7 holds (cta << 32 | task).
+ * NULL turns tracing off.  The buffer must outlive the traced steps. */
+int mk_set_trace(mk_ctx* ctx, unsigned long long* trace_dev);
 
 /* Selects the execution mode of later steps (MK_MODE_*). */
 int mk_set_mode(mk_ctx* ctx, int mode);

@@ -12,7 +12,8 @@ import os
 from typing import Dict, List, Optional, Sequence
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libmk.so")
+# MK_LIBRARY selects another build of the library (A/B comparisons of builds).
+LIB_PATH = os.environ.get("MK_LIBRARY") or os.path.join(HERE, "libmk.so")
 
 MK_OK = 0
 ERRORS = {-1: "MK_ERR_INVALID_ARG", -2: "MK_ERR_OOM", -3: "MK_ERR_CUDA", -4: "MK_ERR_TIMEOUT",
@@ -25,7 +26,7 @@ EXPORTS = ("mk_create", "mk_prefill", "mk_decode_step", "mk_decode_step_host", "
            "mk_kv_pointer", "mk_copy_kv", "mk_set_mode", "mk_status", "mk_last_error",
            "mk_destroy", "mk_plan_build", "mk_plan_get_info", "mk_plan_get_tasks",
            "mk_plan_get_queue", "mk_plan_get_event_counts", "mk_plan_destroy",
-           "mk_qkv_row_source", "mk_read_probe")
+           "mk_qkv_row_source", "mk_read_probe", "mk_set_trace")
 
 
 class MkError(RuntimeError):
@@ -57,7 +58,7 @@ class Weights(C.Structure):
 
 class Options(C.Structure):
     _fields_ = [("num_ctas", C.c_int), ("attn_splits", C.c_int), ("timeout_ms", C.c_int),
-                ("mode", C.c_int)]
+                ("mode", C.c_int), ("l2_prefetch", C.c_int)]
 
 
 class PlanInfo(C.Structure):
@@ -82,7 +83,7 @@ def lib(build_if_missing: bool = True):
     global _lib
     if _lib is not None:
         return _lib
-    if not os.path.exists(LIB_PATH) and build_if_missing:
+    if not os.path.exists(LIB_PATH) and build_if_missing and not os.environ.get("MK_LIBRARY"):
         from . import build as _build
         _build.build()
     if not os.path.exists(LIB_PATH):
@@ -112,6 +113,7 @@ def lib(build_if_missing: bool = True):
     L.mk_plan_destroy.restype = None
     L.mk_qkv_row_source.argtypes = [C.POINTER(Config), i, ip, ip, ip]
     L.mk_read_probe.argtypes = [vp, C.c_size_t, vp, vp]
+    L.mk_set_trace.argtypes = [vp, vp]
     _lib = L
     return L
 
@@ -143,7 +145,7 @@ class Plan:
         L = lib()
         self.h = C.c_void_p()
         cfg = make_config(model, max_seq, max_batch)
-        opt = Options(num_ctas, attn_splits, 0, 0)
+        opt = Options(num_ctas, attn_splits, 0, 0, 0)
         rc = L.mk_plan_build(C.byref(cfg), C.byref(opt), int(num_ctas), C.byref(self.h))
         if rc != MK_OK:
             raise MkError(rc, "mk_plan_build rejected the configuration")
@@ -190,7 +192,8 @@ class Decoder:
 
     def __init__(self, model, weights: Dict[str, "torch.Tensor"], max_seq: int,
                  max_batch: int = 1, num_ctas: int = 0, attn_splits: int = 0,
-                 timeout_ms: int = 0, mode: int = MODE_MEGAKERNEL, stream=None):
+                 timeout_ms: int = 0, mode: int = MODE_MEGAKERNEL, stream=None,
+                 l2_prefetch: int = 0):
         import torch
         L = lib()
         self.model = model
@@ -212,7 +215,7 @@ class Decoder:
         w = Weights(ptr("embed"), layers, ptr("final_norm"),
                     None if model.tied_embeddings else ptr("lm_head"))
         cfg = make_config(model, max_seq, max_batch)
-        opt = Options(num_ctas, attn_splits, timeout_ms, mode)
+        opt = Options(num_ctas, attn_splits, timeout_ms, mode, l2_prefetch)
         self.h = C.c_void_p()
         rc = L.mk_create(C.byref(cfg), C.byref(w), C.byref(opt), self.stream.cuda_stream,
                          C.byref(self.h))
@@ -256,6 +259,12 @@ class Decoder:
 
     def copy_kv(self, req: int, layer: int, kv_head: int, which: int, n: int, dst_dev):
         _check(lib().mk_copy_kv(self.h, req, layer, kv_head, which, n, dst_dev.data_ptr()),
+               self.h)
+
+    def set_trace(self, trace_dev=None):
+        """Per-task timeline of later megakernel steps into ``trace_dev``
+        (int64 CUDA tensor, 8 words per task); None turns it off."""
+        _check(lib().mk_set_trace(self.h, None if trace_dev is None else trace_dev.data_ptr()),
                self.h)
 
     def status(self) -> int:

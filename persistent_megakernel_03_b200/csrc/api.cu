@@ -302,8 +302,8 @@ extern "C" int mk_create(const mk_config* cfg, const mk_weights* w, const mk_opt
   if ((rc = dalloc(ctx, &q, (size_t)B * qd * 4))) return bail(rc);
   if ((rc = dalloc(ctx, &att, (size_t)B * qd * 4))) return bail(rc);
   if ((rc = dalloc(ctx, &act, (size_t)B * F * 4))) return bail(rc);
-  if ((rc = dalloc(ctx, &part, (size_t)B * nkv * S * G * (d + 2) * 4))) return bail(rc);
-  if ((rc = dalloc(ctx, &am, (size_t)B * plan.n_lm_tasks * 8))) return bail(rc);
+  if ((rc = dalloc(ctx, &part, (size_t)B * nkv * S * G * attn_part_stride(d) * 4))) return bail(rc);
+  if ((rc = dalloc(ctx, &am, (size_t)B * plan.n_lm_slots * 8))) return bail(rc);
   CKC(cudaMemsetAsync(x, 0, (size_t)B * H * 4, st));
   uint32_t *events = nullptr, *tickets = nullptr, *epoch = nullptr;
   int32_t* status = nullptr;
@@ -346,8 +346,11 @@ extern "C" int mk_create(const mk_config* cfg, const mk_weights* w, const mk_opt
   m.qkv_bias = cfg->qkv_bias ? 1 : 0;
   m.rms_eps = cfg->rms_eps;
   m.attn_scale = (float)(1.0 / std::sqrt((double)d));
-  m.n_lm_tasks = plan.n_lm_tasks;
+  m.n_lm_slots = plan.n_lm_slots;
   m.timeout_ms = ctx->opt.timeout_ms > 0 ? ctx->opt.timeout_ms : 1000;
+  m.l2_prefetch_chunks = ctx->opt.l2_prefetch == 0 ? kDefaultL2Prefetch
+                                                  : (ctx->opt.l2_prefetch < 0 ? 0 : ctx->opt.l2_prefetch);
+  m.trace = nullptr;
   m.embed = emb; m.lm_head = lm; m.final_norm = finaln; m.attn_norm = an; m.ffn_norm = fn;
   m.bqkv = bq; m.rope_cos = rc_d; m.rope_sin = rs_d; m.kcache = kc; m.vcache = vc;
   m.x = x; m.q = q; m.attn = att; m.act = act; m.part = part; m.am = am;
@@ -469,6 +472,12 @@ extern "C" int mk_copy_kv(mk_ctx* ctx, int req, int layer, int kv_head, int whic
   if ((rc = mk_kv_pointer(ctx, req, layer, kv_head, which, &src))) return rc;
   if (!dst_dev || n < 0 || n > ctx->cfg.max_seq) return fail(ctx, MK_ERR_INVALID_ARG, "bad copy size");
   CK(cudaMemcpyAsync(dst_dev, src, (size_t)n * ctx->cfg.head_dim * 2, cudaMemcpyDeviceToDevice, ctx->stream));
+  return MK_OK;
+}
+
+extern "C" int mk_set_trace(mk_ctx* ctx, unsigned long long* trace_dev) {
+  if (!ctx) return MK_ERR_INVALID_ARG;
+  ctx->md.trace = trace_dev;
   return MK_OK;
 }
 

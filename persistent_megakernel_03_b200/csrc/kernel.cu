@@ -43,8 +43,9 @@ struct __align__(128) Smem {
   uint64_t done;
   uint32_t epoch;
   int32_t abort_flag;
-  int32_t consumed_seq;
   int32_t flag;
+  int32_t cur_qi;              // queue entry the workers are running (trace)
+  unsigned long long lm_best;  // running argmax over this CTA's LM-head tasks
 };
 
 constexpr uint32_t kWorkerBarrier = 1;
@@ -57,6 +58,15 @@ __device__ __forceinline__ const StepParams& step_params(const KernelArgs& a) {
   return a.sp_ptr ? *a.sp_ptr : a.sp_val;
 }
 
+// Per-task timeline (diagnostics, off unless a trace buffer is set): word k of
+// the running queue entry.  0 event satisfied, 1 workers start, 2 input
+// loaded, 3 first chunk ready, 4 last chunk consumed, 5 epilogue done, 6 end,
+// 7 cta << 32 | task.
+constexpr int kTraceWords = 8;
+__device__ __forceinline__ void trace_mark(const KernelArgs& a, Smem& s, int wtid, int k) {
+  if (a.m.trace && wtid == 0) a.m.trace[(size_t)s.cur_qi * kTraceWords + k] = globaltimer_ns();
+}
+
 __device__ __forceinline__ float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
 __device__ __forceinline__ float bf16_to_float(uint16_t h) {
@@ -67,15 +77,13 @@ __device__ __forceinline__ uint16_t float_to_bf16_rne(float f) {
   return *reinterpret_cast<uint16_t*>(&b);
 }
 
-__device__ __forceinline__ float dot8(const uint4 w, const float (&x)[8], float acc) {
-  acc = fmaf(bf_lo(w.x), x[0], acc);
-  acc = fmaf(bf_hi(w.x), x[1], acc);
-  acc = fmaf(bf_lo(w.y), x[2], acc);
-  acc = fmaf(bf_hi(w.y), x[3], acc);
-  acc = fmaf(bf_lo(w.z), x[4], acc);
-  acc = fmaf(bf_hi(w.z), x[5], acc);
-  acc = fmaf(bf_lo(w.w), x[6], acc);
-  acc = fmaf(bf_hi(w.w), x[7], acc);
+// Eight bf16 weights times eight fp32 inputs into a pair of fp32 partial sums
+// (even and odd columns) with the packed fp32x2 FMA of sm_100.
+__device__ __forceinline__ float2 dot8(const uint4 w, const float2 (&x)[4], float2 acc) {
+  acc = __ffma2_rn(make_float2(bf_lo(w.x), bf_hi(w.x)), x[0], acc);
+  acc = __ffma2_rn(make_float2(bf_lo(w.y), bf_hi(w.y)), x[1], acc);
+  acc = __ffma2_rn(make_float2(bf_lo(w.z), bf_hi(w.z)), x[2], acc);
+  acc = __ffma2_rn(make_float2(bf_lo(w.w), bf_hi(w.w)), x[3], acc);
   return acc;
 }
 
@@ -148,6 +156,7 @@ __device__ __forceinline__ size_t kv_offset(const ModelDev& m, int slot, int lay
 
 // ---------------------------------------------------------------- producer
 
+
 __device__ __forceinline__ bool producer_acquire_slot(Smem& s, uint32_t seq, const ModelDev& m) {
   const int slot = seq % kRingSlots;
   const uint32_t ph = (seq / kRingSlots) & 1u;
@@ -155,43 +164,77 @@ __device__ __forceinline__ bool producer_acquire_slot(Smem& s, uint32_t seq, con
   return !aborting(s);
 }
 
-__device__ void producer(const KernelArgs& a, Smem& s, int q0, int q1) {
+// One ring chunk: up to two 1-D bulk copies into the same slot (weights: one
+// copy of whole rows; attention: K rows into the first half, V rows into the
+// second half).
+struct Chunk {
+  const void* src0;
+  const void* src1;
+  uint32_t bytes0, bytes1;
+  bool kv;
+};
+
+// Walks the chunks of a CTA's queue in the order the workers consume them.
+struct ChunkCursor {
+  int qi, q1;
+  int off;  // next row (GEMV) or key (ATTN) inside task qi
+
+  __device__ __forceinline__ bool next(const KernelArgs& a, const StepParams& sp, Chunk& c) {
+    const ModelDev& m = a.m;
+    while (qi < q1) {
+      const Task& t = a.tasks[a.queue[qi]];
+      if (t.kind == T_ATTN) {
+        const AttnRange r = attn_range(t, sp, m);
+        if (r.active) {
+          const int k = off < 0 ? r.k0 : off;
+          if (k < r.old_end) {
+            const int nk = min(attn_keys_per_chunk(m.head_dim), r.old_end - k);
+            const size_t o = kv_offset(m, sp.kv_slot[t.req], t.layer, t.row0, k);
+            c.src0 = m.kcache + o;
+            c.src1 = m.vcache + o;
+            c.bytes0 = c.bytes1 = (uint32_t)nk * m.head_dim * 2;
+            c.kv = true;
+            off = k + nk;
+            return true;
+          }
+        }
+      } else {
+        const int r = off < 0 ? t.row0 : off;
+        if (r < t.row1) {
+          const int nr = min(t.chunk_rows, t.row1 - r);
+          c.src0 = t.w + (size_t)r * t.K;
+          c.src1 = nullptr;
+          c.bytes0 = (uint32_t)nr * t.K * 2;
+          c.bytes1 = 0;
+          c.kv = false;
+          off = r + nr;
+          return true;
+        }
+      }
+      ++qi;
+      off = -1;
+    }
+    return false;
+  }
+};
+
+// Streams every chunk of the CTA's queue into the ring, in the workers'
+// consumption order, as fast as slots free up.
+__device__ __forceinline__ void producer(const KernelArgs& a, Smem& s, int q0, int q1) {
   const ModelDev& m = a.m;
   const StepParams& sp = step_params(a);
   const uint64_t pol_w = l2_policy_evict_first();
-  const uint64_t pol_kv = l2_policy_evict_normal();
+  const uint64_t pol_keep = l2_policy_evict_normal();
+  ChunkCursor cc{q0, q1, -1};
+  Chunk c;
   uint32_t seq = 0;
-  bool ok = true;
-  for (int qi = q0; qi < q1 && ok; ++qi) {
-    const Task& t = a.tasks[a.queue[qi]];
-    if (t.kind == T_ATTN) {
-      const AttnRange r = attn_range(t, sp, m);
-      if (!r.active) continue;
-      const int kpc = attn_keys_per_chunk(m.head_dim);
-      const int slotkv = sp.kv_slot[t.req];
-      for (int k = r.k0; k < r.old_end && ok; k += kpc) {
-        const int nk = min(kpc, r.old_end - k);
-        const uint32_t bytes = (uint32_t)nk * m.head_dim * 2;
-        if (!(ok = producer_acquire_slot(s, seq, m))) break;
-        const int slot = seq % kRingSlots;
-        const size_t off = kv_offset(m, slotkv, t.layer, t.row0, k);
-        mbar_arrive_expect_tx(&s.full[slot], 2 * bytes);
-        bulk_g2s(s.ring[slot], m.kcache + off, bytes, &s.full[slot], pol_kv);
-        bulk_g2s(s.ring[slot] + kSlotBytes / 2, m.vcache + off, bytes, &s.full[slot], pol_kv);
-        ++seq;
-      }
-    } else {
-      const int K = t.K;
-      for (int r = t.row0; r < t.row1 && ok; r += t.chunk_rows) {
-        const int nr = min(t.chunk_rows, t.row1 - r);
-        const uint32_t bytes = (uint32_t)nr * K * 2;
-        if (!(ok = producer_acquire_slot(s, seq, m))) break;
-        const int slot = seq % kRingSlots;
-        mbar_arrive_expect_tx(&s.full[slot], bytes);
-        bulk_g2s(s.ring[slot], t.w + (size_t)r * K, bytes, &s.full[slot], pol_w);
-        ++seq;
-      }
-    }
+  while (cc.next(a, sp, c)) {
+    if (!producer_acquire_slot(s, seq, m)) break;
+    const int slot = seq % kRingSlots;
+    mbar_arrive_expect_tx(&s.full[slot], c.bytes0 + c.bytes1);
+    bulk_g2s(s.ring[slot], c.src0, c.bytes0, &s.full[slot], c.kv ? pol_keep : pol_w);
+    if (c.src1) bulk_g2s(s.ring[slot] + kSlotBytes / 2, c.src1, c.bytes1, &s.full[slot], pol_keep);
+    ++seq;
   }
   // Before this warp may retire, every copy it issued must have landed: if
   // the workers stop early (abort) nobody else waits for them, and a bulk copy
@@ -209,8 +252,10 @@ __device__ void producer(const KernelArgs& a, Smem& s, int q0, int q1) {
 
 // --------------------------------------------------------------- scheduler
 
-__device__ void scheduler(const KernelArgs& a, Smem& s, int q0, int q1) {
+__device__ __forceinline__ void scheduler(const KernelArgs& a, Smem& s, int q0, int q1) {
   const ModelDev& m = a.m;
+  const StepParams& sp = step_params(a);
+  const uint64_t pol_keep = l2_policy_evict_normal();
   const uint32_t epoch = s.epoch;
   const uint64_t limit = (uint64_t)(m.timeout_ms > 0 ? m.timeout_ms : 1000) * 1000000ull;
   int i = 0;
@@ -221,6 +266,19 @@ __device__ void scheduler(const KernelArgs& a, Smem& s, int q0, int q1) {
     if (t.wait_ev >= 0 && !a.no_wait) {
       const uint32_t target = t.wait_count * (epoch + 1u);
       const uint32_t* ev = m.events + t.wait_ev;
+      if (m.l2_prefetch_chunks > 0 && (int32_t)(ld_acquire_gpu(ev) - target) < 0) {
+        // The workers are about to stall on this event, and the ring holds
+        // (or is receiving) the first kRingSlots chunks from here on: prefetch
+        // the next l2_prefetch_chunks chunks into L2 so HBM keeps streaming
+        // through the wait and their copies hit in L2.
+        ChunkCursor pc{qi, q1, -1};
+        Chunk pf;
+        for (int n = 0; n < kRingSlots + m.l2_prefetch_chunks && pc.next(a, sp, pf); ++n) {
+          if (n < kRingSlots) continue;
+          bulk_prefetch_l2(pf.src0, pf.bytes0, pol_keep);
+          if (pf.src1) bulk_prefetch_l2(pf.src1, pf.bytes1, pol_keep);
+        }
+      }
       const uint64_t t0 = globaltimer_ns();
       uint32_t spins = 0;
       while ((int32_t)(ld_acquire_gpu(ev) - target) < 0) {
@@ -240,6 +298,7 @@ __device__ void scheduler(const KernelArgs& a, Smem& s, int q0, int q1) {
       mbar_arrive(&s.ready);
       return;
     }
+    if (m.trace) m.trace[(size_t)qi * kTraceWords] = globaltimer_ns();
     mbar_arrive(&s.ready);
     if (!wait_bounded(s, &s.done, i & 1, m, kWaitDone)) return;
   }
@@ -282,18 +341,6 @@ __device__ __forceinline__ float warp_reduce_rows(float (&v)[NR], int lane) {
   }
 }
 
-// Sum over the 512 worker threads; every worker gets the result.
-__device__ __forceinline__ float worker_sum(Smem& s, float v, int wtid) {
-  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  if ((wtid & 31) == 0) s.red[wtid >> 5] = v;
-  worker_sync();
-  float t = 0.f;
-#pragma unroll
-  for (int w = 0; w < kWorkerWarps; ++w) t += s.red[w];
-  worker_sync();
-  return t;
-}
-
 // Waits for ring chunk `seq`.  Once the CTA is aborting the workers no longer
 // wait: they run the rest of the current task on whatever the slot holds
 // (every access stays in bounds), meet the task's barriers, and stop.
@@ -304,11 +351,65 @@ __device__ __forceinline__ void wait_full(Smem& s, uint32_t seq, const ModelDev&
   wait_bounded(s, &s.full[slot], ph, m, kWaitFull);
 }
 
-// Loads this thread's input columns (fp32 or the bf16 embedding row), applies
-// RMSNorm when the task's operator has one, and leaves the result in xr.
+// Attention output for input columns [8cc, 8cc + 8) of the O projection,
+// merged from the split partials in one pass with a running maximum (online
+// softmax, "Hạt nhân là gì ...": each split's sum and output are rescaled to
+// the common maximum); four splits' loads are in flight at a time.
+struct Cols8 {
+  float2 v[4];
+};
+
+__device__ __forceinline__ Cols8 merge_attn_columns(const ModelDev& m, int cc) {
+  const int d = m.head_dim, G = m.group, S = m.attn_splits, PS = attn_part_stride(d);
+  const int col = cc * 8, h = col / d, i0 = col - h * d;
+  const float* base = m.part + ((size_t)(h / G) * S * G + (h % G)) * PS;
+  const size_t sstride = (size_t)G * PS;
+  float M = -INFINITY, den = 0.f;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int s0 = 0; s0 < S; s0 += 4) {
+    float2 ml[4];
+    float4 oa[4], ob[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (s0 + j < S) {
+        const float* ps = base + (size_t)(s0 + j) * sstride;
+        ml[j] = __ldcg(reinterpret_cast<const float2*>(ps + d));
+        oa[j] = __ldcg(reinterpret_cast<const float4*>(ps + i0));
+        ob[j] = __ldcg(reinterpret_cast<const float4*>(ps + i0) + 1);
+      } else {
+        ml[j] = make_float2(-INFINITY, 0.f);
+        oa[j] = ob[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (ml[j].y == 0.f) continue;  // empty split
+      const float mn = fmaxf(M, ml[j].x);
+      const float co = __expf(M - mn), cn = __expf(ml[j].x - mn);
+      den = fmaf(den, co, ml[j].y * cn);
+      const float o[8] = {oa[j].x, oa[j].y, oa[j].z, oa[j].w, ob[j].x, ob[j].y, ob[j].z, ob[j].w};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = fmaf(acc[e], co, cn * o[e]);
+      M = mn;
+    }
+  }
+  const float inv = 1.0f / den;
+  Cols8 r;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) r.v[e] = make_float2(acc[2 * e] * inv, acc[2 * e + 1] * inv);
+  return r;
+}
+
+// Loads this thread's input columns into xr (fp32, or the bf16 embedding
+// row).  For the O projection the input is the attention output, merged from
+// the split partials (merge_attn_columns).  For operators
+// that start with RMSNorm, xr = x * w_norm and the returned value is this
+// thread's share of sum(x^2); the 1/rms factor is applied to the dot products
+// afterwards (W (x * w * r) = r * W (x * w)), so the first ring chunk is not
+// held back by a block-wide reduction.
 template <int CPT>
-__device__ __forceinline__ void gemv_load_input(const KernelArgs& a, Smem& s, const Task& t,
-                                                int wtid, int ct, int rl, float (&xr)[CPT][8]) {
+__device__ __forceinline__ float gemv_load_input(const KernelArgs& a, const Task& t, int wtid,
+                                                 int ct, int rl, float2 (&x2)[CPT][4]) {
   const ModelDev& m = a.m;
   const StepParams& sp = step_params(a);
   const int K = t.K, C = K >> 3;
@@ -329,58 +430,60 @@ __device__ __forceinline__ void gemv_load_input(const KernelArgs& a, Smem& s, co
         src32 = m.x;
       }
       break;
-    case T_OPROJ: src32 = m.attn; break;
+    case T_OPROJ: break;
     case T_GATEUP: src32 = m.x; normw = m.ffn_norm + (size_t)t.layer * m.hidden; break;
     case T_DOWN: src32 = m.act; break;
     default: src32 = m.x; normw = m.final_norm; break;  // LM head
   }
   const int TPR = t.tpr;
+  float ss = 0.f;
 #pragma unroll
   for (int c = 0; c < CPT; ++c) {
     const int cc = ct + c * TPR;
-    if (cc < C) {
-      if (src16) {
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(src16) + cc);
-        xr[c][0] = bf_lo(v.x); xr[c][1] = bf_hi(v.x); xr[c][2] = bf_lo(v.y); xr[c][3] = bf_hi(v.y);
-        xr[c][4] = bf_lo(v.z); xr[c][5] = bf_hi(v.z); xr[c][6] = bf_lo(v.w); xr[c][7] = bf_hi(v.w);
-      } else {
-        const float4 u = __ldcg(reinterpret_cast<const float4*>(src32) + 2 * cc);
-        const float4 w = __ldcg(reinterpret_cast<const float4*>(src32) + 2 * cc + 1);
-        xr[c][0] = u.x; xr[c][1] = u.y; xr[c][2] = u.z; xr[c][3] = u.w;
-        xr[c][4] = w.x; xr[c][5] = w.y; xr[c][6] = w.z; xr[c][7] = w.w;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) x2[c][e] = make_float2(0.f, 0.f);
+    if (cc >= C) continue;
+    if (t.kind == T_OPROJ) {
+      // n_q * head_dim <= 8192 (checked at create) keeps CPT <= 2 here.
+      if constexpr (CPT <= 2) {
+        const Cols8 v = merge_attn_columns(m, cc);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x2[c][e] = v.v[e];
       }
+    } else if (src16) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(src16) + cc);
+      x2[c][0] = make_float2(bf_lo(v.x), bf_hi(v.x));
+      x2[c][1] = make_float2(bf_lo(v.y), bf_hi(v.y));
+      x2[c][2] = make_float2(bf_lo(v.z), bf_hi(v.z));
+      x2[c][3] = make_float2(bf_lo(v.w), bf_hi(v.w));
     } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) xr[c][e] = 0.f;
+      const float4 u = __ldcg(reinterpret_cast<const float4*>(src32) + 2 * cc);
+      const float4 w = __ldcg(reinterpret_cast<const float4*>(src32) + 2 * cc + 1);
+      x2[c][0] = make_float2(u.x, u.y);
+      x2[c][1] = make_float2(u.z, u.w);
+      x2[c][2] = make_float2(w.x, w.y);
+      x2[c][3] = make_float2(w.z, w.w);
     }
-  }
-  if (normw) {
-    float ss = 0.f;
-    if (rl == 0) {
+    if (normw) {
+      const uint4 wv = __ldg(reinterpret_cast<const uint4*>(normw) + cc);
+      const float2 wn[4] = {make_float2(bf_lo(wv.x), bf_hi(wv.x)), make_float2(bf_lo(wv.y), bf_hi(wv.y)),
+                            make_float2(bf_lo(wv.z), bf_hi(wv.z)), make_float2(bf_lo(wv.w), bf_hi(wv.w))};
 #pragma unroll
-      for (int c = 0; c < CPT; ++c)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) ss = fmaf(xr[c][e], xr[c][e], ss);
-    }
-    ss = worker_sum(s, ss, wtid);
-    const float r = 1.0f / sqrtf(ss / (float)K + m.rms_eps);
-#pragma unroll
-    for (int c = 0; c < CPT; ++c) {
-      const int cc = ct + c * TPR;
-      if (cc < C) {
-        const uint4 wv = __ldg(reinterpret_cast<const uint4*>(normw) + cc);
-        const float wn[8] = {bf_lo(wv.x), bf_hi(wv.x), bf_lo(wv.y), bf_hi(wv.y),
-                             bf_lo(wv.z), bf_hi(wv.z), bf_lo(wv.w), bf_hi(wv.w)};
-#pragma unroll
-        for (int e = 0; e < 8; ++e) xr[c][e] = (xr[c][e] * r) * wn[e];
+      for (int e = 0; e < 4; ++e) {
+        if (rl == 0) {
+          ss = fmaf(x2[c][e].x, x2[c][e].x, ss);
+          ss = fmaf(x2[c][e].y, x2[c][e].y, ss);
+        }
+        x2[c][e] = make_float2(x2[c][e].x * wn[e].x, x2[c][e].y * wn[e].y);
       }
     }
   }
+  return ss;
 }
 
 // Streams the task's rows through the ring and leaves y[row] in s.ybuf.
 template <int CPT, int NR>
-__device__ void gemv_stream(const KernelArgs& a, Smem& s, const Task& t, uint32_t& seq, int wtid) {
+__device__ __forceinline__ void gemv_stream(const KernelArgs& a, Smem& s, const Task& t, uint32_t& seq, int wtid) {
   const int TPR = t.tpr;
   const int rl = wtid / TPR, ct = wtid % TPR;
   const int wpr = TPR >> 5, wir = ct >> 5;
@@ -388,27 +491,36 @@ __device__ void gemv_stream(const KernelArgs& a, Smem& s, const Task& t, uint32_
   const int K = t.K, C = K >> 3;
   const size_t row_bytes = (size_t)K * 2;
   const int nrows = t.row1 - t.row0;
-  float xr[CPT][8];
-  gemv_load_input<CPT>(a, s, t, wtid, ct, rl, xr);
+  float2 x2[CPT][4];
+  float ss = gemv_load_input<CPT>(a, t, wtid, ct, rl, x2);
+  trace_mark(a, s, wtid, 2);
+  const bool has_norm = t.kind == T_QKV || t.kind == T_GATEUP || t.kind == T_LMHEAD;
+  if (has_norm) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (lane == 0) s.red[wtid >> 5] = ss;  // read after the barrier that ends the stream
+  }
   constexpr int kShift = NR == 4 ? 3 : (NR == 2 ? 4 : 5);
   for (int r = 0; r < nrows; r += t.chunk_rows) {
     const int rows_here = min(t.chunk_rows, nrows - r);
     const int slot = seq % kRingSlots;
     wait_full(s, seq, a.m);
+    if (r == 0) trace_mark(a, s, wtid, 3);
     const uint8_t* base = s.ring[slot];
     float acc[NR];
 #pragma unroll
     for (int j = 0; j < NR; ++j) {
-      acc[j] = 0.f;
+      float2 a2 = make_float2(0.f, 0.f);
       const int lr = rl * NR + j;
       if (lr < rows_here) {
         const uint8_t* row = base + (size_t)lr * row_bytes;
 #pragma unroll
         for (int c = 0; c < CPT; ++c) {
           const int cc = ct + c * TPR;
-          if (cc < C) acc[j] = dot8(*reinterpret_cast<const uint4*>(row + (size_t)cc * 16), xr[c], acc[j]);
+          if (cc < C) a2 = dot8(*reinterpret_cast<const uint4*>(row + (size_t)cc * 16), x2[c], a2);
         }
       }
+      acc[j] = a2.x + a2.y;
     }
     const float v = warp_reduce_rows<NR>(acc, lane);
     const int jj = lane >> kShift;
@@ -420,17 +532,25 @@ __device__ void gemv_stream(const KernelArgs& a, Smem& s, const Task& t, uint32_
     if (lane == 0) mbar_arrive(&s.empty[slot]);
     ++seq;
   }
+  trace_mark(a, s, wtid, 4);
   worker_sync();
+  float r = 1.0f;
+  if (has_norm) {
+    float tot = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWorkerWarps; ++w) tot += s.red[w];
+    r = 1.0f / sqrtf(tot / (float)K + a.m.rms_eps);
+  }
   for (int i = wtid; i < nrows; i += kWorkerThreads) {
     float y = 0.f;
     for (int w = 0; w < wpr; ++w) y += s.scratch[w * nrows + i];
-    s.ybuf[i] = y;
+    s.ybuf[i] = has_norm ? y * r : y;
   }
   worker_sync();
 }
 
 template <int CPT>
-__device__ void gemv_dispatch_nr(const KernelArgs& a, Smem& s, const Task& t, uint32_t& seq,
+__device__ __forceinline__ void gemv_dispatch_nr(const KernelArgs& a, Smem& s, const Task& t, uint32_t& seq,
                                  int wtid) {
   const int nr = t.chunk_rows / (kWorkerThreads / t.tpr);
   if (nr >= 4) gemv_stream<CPT, 4>(a, s, t, seq, wtid);
@@ -438,7 +558,7 @@ __device__ void gemv_dispatch_nr(const KernelArgs& a, Smem& s, const Task& t, ui
   else gemv_stream<CPT, 1>(a, s, t, seq, wtid);
 }
 
-__device__ void gemv_core(const KernelArgs& a, Smem& s, const Task& t, uint32_t& seq, int wtid) {
+__device__ __forceinline__ void gemv_core(const KernelArgs& a, Smem& s, const Task& t, uint32_t& seq, int wtid) {
   const int cpt = (t.K / 8 + t.tpr - 1) / t.tpr;
   switch (cpt) {
     case 1: gemv_dispatch_nr<1>(a, s, t, seq, wtid); break;
@@ -452,6 +572,7 @@ __device__ void gemv_core(const KernelArgs& a, Smem& s, const Task& t, uint32_t&
 // scheduler for the next task.
 __device__ __forceinline__ void finish_task(const KernelArgs& a, Smem& s, const Task& t,
                                             int wtid, bool signal) {
+  trace_mark(a, s, wtid, 5);
   worker_sync();
   if (wtid == 0) {
     if (signal && t.n_sig > 0) {
@@ -462,7 +583,7 @@ __device__ __forceinline__ void finish_task(const KernelArgs& a, Smem& s, const 
   }
 }
 
-__device__ void epilogue_qkv(const KernelArgs& a, Smem& s, const Task& t, int wtid) {
+__device__ __forceinline__ void epilogue_qkv(const KernelArgs& a, Smem& s, const Task& t, int wtid) {
   const ModelDev& m = a.m;
   const StepParams& sp = step_params(a);
   const int d = m.head_dim, G = m.group, half = d >> 1;
@@ -501,7 +622,7 @@ __device__ void epilogue_qkv(const KernelArgs& a, Smem& s, const Task& t, int wt
   }
 }
 
-__device__ void epilogue_residual(const KernelArgs& a, Smem& s, const Task& t, int wtid) {
+__device__ __forceinline__ void epilogue_residual(const KernelArgs& a, Smem& s, const Task& t, int wtid) {
   const ModelDev& m = a.m;
   const StepParams& sp = step_params(a);
   const int nrows = t.row1 - t.row0;
@@ -519,7 +640,7 @@ __device__ void epilogue_residual(const KernelArgs& a, Smem& s, const Task& t, i
   }
 }
 
-__device__ void epilogue_swiglu(const KernelArgs& a, Smem& s, const Task& t, int wtid) {
+__device__ __forceinline__ void epilogue_swiglu(const KernelArgs& a, Smem& s, const Task& t, int wtid) {
   const ModelDev& m = a.m;
   const int npairs = (t.row1 - t.row0) >> 1;
   for (int pi = wtid; pi < npairs; pi += kWorkerThreads) {
@@ -529,7 +650,7 @@ __device__ void epilogue_swiglu(const KernelArgs& a, Smem& s, const Task& t, int
   }
 }
 
-__device__ void epilogue_lmhead(const KernelArgs& a, Smem& s, const Task& t, int wtid) {
+__device__ __forceinline__ void epilogue_lmhead(const KernelArgs& a, Smem& s, const Task& t, int wtid) {
   const ModelDev& m = a.m;
   const StepParams& sp = step_params(a);
   const int nrows = t.row1 - t.row0;
@@ -547,18 +668,22 @@ __device__ void epilogue_lmhead(const KernelArgs& a, Smem& s, const Task& t, int
   if ((wtid & 31) == 0) s.red64[wtid >> 5] = best;
   worker_sync();
   if (wtid == 0) {
-    unsigned long long b = 0ull;
+    unsigned long long b = (t.req & 1) ? 0ull : s.lm_best;
     for (int w = 0; w < kWorkerWarps; ++w) b = s.red64[w] > b ? s.red64[w] : b;
-    m.am[t.aux] = b;
-    __threadfence();
-    const uint32_t old = atom_add_acq_rel_gpu(m.tickets + m.max_batch * m.n_layers * m.n_kv, 1u);
-    s.flag = (old == (uint32_t)m.n_lm_tasks * (s.epoch + 1u) - 1u) ? 1 : 0;
+    s.lm_best = b;
+    s.flag = 0;
+    if (t.req & 2) {  // the CTA's last LM task publishes its candidate
+      m.am[t.aux] = b;
+      __threadfence();
+      const uint32_t old = atom_add_acq_rel_gpu(m.tickets, 1u);
+      s.flag = (old == (uint32_t)m.n_lm_slots * (s.epoch + 1u) - 1u) ? 1 : 0;
+    }
   }
   worker_sync();
   if (s.flag) {
-    // Last LM task of the step: reduce every task's candidate.
+    // Last CTA of the step: reduce every CTA's candidate.
     unsigned long long b = 0ull;
-    for (int i = wtid; i < m.n_lm_tasks; i += kWorkerThreads) {
+    for (int i = wtid; i < m.n_lm_slots; i += kWorkerThreads) {
       const unsigned long long v = __ldcg(m.am + i);
       b = v > b ? v : b;
     }
@@ -634,143 +759,133 @@ __device__ __forceinline__ void attn_key(AttnState<DPL, G>& st, const float (&k)
 }
 
 template <int DPL, int G>
-__device__ void attn_task(const KernelArgs& a, Smem& s, const Task& t, uint32_t& seq, int wtid) {
-  const ModelDev& m = a.m;
-  const StepParams& sp = step_params(a);
-  const int d = m.head_dim, S = m.attn_splits;
-  const int warp = wtid >> 5, lane = wtid & 31;
-  const int g = t.row0, split = t.row1, b = t.req;
-  const AttnRange r = attn_range(t, sp, m);
-  if (r.active) {
-    AttnState<DPL, G> st;
+__device__ __forceinline__ void attn_write_state(const AttnState<DPL, G>& st, float* dst, int PS,
+                                                 int d, int lane) {
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-#pragma unroll
-      for (int i = 0; i < DPL; ++i) {
-        st.q[h][i] = __ldcg(m.q + (size_t)(g * G + h) * d + lane * DPL + i) * m.attn_scale;
-        st.o[h][i] = 0.f;
-      }
-      st.mx[h] = -INFINITY;
-      st.l[h] = 0.f;
+  for (int h = 0; h < G; ++h) {
+    if constexpr (DPL == 4) {
+      *reinterpret_cast<float4*>(dst + h * PS + lane * 4) =
+          make_float4(st.o[h][0], st.o[h][1], st.o[h][2], st.o[h][3]);
+    } else {
+      *reinterpret_cast<float2*>(dst + h * PS + lane * 2) = make_float2(st.o[h][0], st.o[h][1]);
     }
-    const int kpc = attn_keys_per_chunk(d);
-    for (int k = r.k0; k < r.old_end; k += kpc) {
-      const int nk = min(kpc, r.old_end - k);
-      const int slot = seq % kRingSlots;
-      wait_full(s, seq, m);
-      const uint16_t* kb = reinterpret_cast<const uint16_t*>(s.ring[slot]);
-      const uint16_t* vb = reinterpret_cast<const uint16_t*>(s.ring[slot] + kSlotBytes / 2);
-      for (int j = warp; j < nk; j += kWorkerWarps) {
-        float kv[DPL], vv[DPL];
-        load_kv_row<DPL>(kb + (size_t)j * d + lane * DPL, kv);
-        load_kv_row<DPL>(vb + (size_t)j * d + lane * DPL, vv);
-        attn_key<DPL, G>(st, kv, vv);
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s.empty[slot]);
-      ++seq;
-    }
-    // The newest key (written by this step's QKV tasks) is read from memory.
-    const int pos = sp.pos[b];
-    if (pos >= r.k0 && pos < r.k1 && warp == (kWorkerWarps - 1)) {
-      const size_t off = kv_offset(m, sp.kv_slot[b], t.layer, g, pos);
-      float kv[DPL], vv[DPL];
-      load_kv_row_global<DPL>(m.kcache + off + lane * DPL, kv);
-      load_kv_row_global<DPL>(m.vcache + off + lane * DPL, vv);
-      attn_key<DPL, G>(st, kv, vv);
-    }
-    // Tree merge of the 16 warps' (max, sum, output) through shared memory.
-    float* buf = s.scratch;
-    const int stride_w = G * (d + 2);
-    for (int half = kWorkerWarps / 2; half >= 1; half >>= 1) {
-      if (warp >= half && warp < 2 * half) {
-        float* dst = buf + (warp - half) * stride_w;
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-#pragma unroll
-          for (int i = 0; i < DPL; ++i) dst[h * (d + 2) + lane * DPL + i] = st.o[h][i];
-          if (lane == 0) {
-            dst[h * (d + 2) + d] = st.mx[h];
-            dst[h * (d + 2) + d + 1] = st.l[h];
-          }
-        }
-      }
-      worker_sync();
-      if (warp < half) {
-        const float* src = buf + warp * stride_w;
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float m2 = src[h * (d + 2) + d], l2 = src[h * (d + 2) + d + 1];
-          if (m2 != -INFINITY) {
-            if (st.mx[h] == -INFINITY) {
-              st.mx[h] = m2;
-              st.l[h] = l2;
-#pragma unroll
-              for (int i = 0; i < DPL; ++i) st.o[h][i] = src[h * (d + 2) + lane * DPL + i];
-            } else {
-              const float mn = fmaxf(st.mx[h], m2);
-              const float c1 = __expf(st.mx[h] - mn), c2 = __expf(m2 - mn);
-              st.l[h] = st.l[h] * c1 + l2 * c2;
-#pragma unroll
-              for (int i = 0; i < DPL; ++i)
-                st.o[h][i] = st.o[h][i] * c1 + src[h * (d + 2) + lane * DPL + i] * c2;
-              st.mx[h] = mn;
-            }
-          }
-        }
-      }
-      worker_sync();
-    }
-    if (warp == 0) {
-      float* part = m.part + ((size_t)(b * m.n_kv + g) * S + split) * G * (d + 2);
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-#pragma unroll
-        for (int i = 0; i < DPL; ++i) part[h * (d + 2) + lane * DPL + i] = st.o[h][i];
-        if (lane == 0) {
-          part[h * (d + 2) + d] = st.mx[h];
-          part[h * (d + 2) + d + 1] = st.l[h];
-        }
-      }
-    }
-  }
-  // Ticket: the last split of this (slot, group) merges all splits.
-  worker_sync();
-  if (wtid == 0) {
-    __threadfence();
-    const uint32_t old = atom_add_acq_rel_gpu(m.tickets + t.aux, 1u);
-    s.flag = (old == (uint32_t)S * (s.epoch + 1u) - 1u) ? 1 : 0;
-  }
-  worker_sync();
-  if (s.flag) {
-    if (r.active) {
-      const float* part = m.part + (size_t)(b * m.n_kv + g) * S * G * (d + 2);
-      for (int idx = wtid; idx < G * d; idx += kWorkerThreads) {
-        const int h = idx / d, i = idx - h * d;
-        float M = -INFINITY;
-        for (int sp_i = 0; sp_i < S; ++sp_i)
-          M = fmaxf(M, __ldcg(part + ((size_t)sp_i * G + h) * (d + 2) + d));
-        float num = 0.f, den = 0.f;
-        for (int sp_i = 0; sp_i < S; ++sp_i) {
-          const float* ps = part + ((size_t)sp_i * G + h) * (d + 2);
-          const float ls = __ldcg(ps + d + 1);
-          if (ls == 0.f) continue;
-          const float c = __expf(__ldcg(ps + d) - M);
-          num = fmaf(c, __ldcg(ps + i), num);
-          den = fmaf(c, ls, den);
-        }
-        m.attn[(size_t)(g * G + h) * d + i] = num / den;
-      }
-    }
-    worker_sync();
-    if (wtid == 0) {
-      __threadfence();
-      red_release_gpu_add(m.events + t.sig_ev0, 1u);
+    if (lane == 0) {
+      dst[h * PS + d] = st.mx[h];
+      dst[h * PS + d + 1] = st.l[h];
     }
   }
 }
 
-__device__ void attn_dispatch(const KernelArgs& a, Smem& s, const Task& t, uint32_t& seq, int wtid) {
+template <int DPL, int G>
+__device__ __forceinline__ void attn_task(const KernelArgs& a, Smem& s, const Task& t, uint32_t& seq, int wtid) {
+  const ModelDev& m = a.m;
+  const StepParams& sp = step_params(a);
+  const int d = m.head_dim, S_all = m.attn_splits, PS = attn_part_stride(d);
+  const int warp = wtid >> 5, lane = wtid & 31;
+  const int g = t.row0, split = t.row1, b = t.req;
+  const AttnRange r = attn_range(t, sp, m);
+  if (!r.active) return;
+  AttnState<DPL, G> st;
+  // Issue every global load this task needs before touching the ring: the
+  // rotated queries of the group, and (in the split that holds it) the newest
+  // K/V row, which this step's QKV tasks wrote.
+  const int pos = sp.pos[b];
+  const bool has_new = pos >= r.k0 && pos < r.k1 && warp == kWorkerWarps - 1;
+  float kn[DPL], vn[DPL];
+  if (has_new) {
+    const size_t off = kv_offset(m, sp.kv_slot[b], t.layer, g, pos);
+    load_kv_row_global<DPL>(m.kcache + off + lane * DPL, kn);
+    load_kv_row_global<DPL>(m.vcache + off + lane * DPL, vn);
+  }
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) {
+      st.q[h][i] = __ldcg(m.q + (size_t)(g * G + h) * d + lane * DPL + i) * m.attn_scale;
+      st.o[h][i] = 0.f;
+    }
+    st.mx[h] = -INFINITY;
+    st.l[h] = 0.f;
+  }
+  trace_mark(a, s, wtid, 2);
+  const int kpc = attn_keys_per_chunk(d);
+  for (int k = r.k0; k < r.old_end; k += kpc) {
+    const int nk = min(kpc, r.old_end - k);
+    const int slot = seq % kRingSlots;
+    wait_full(s, seq, m);
+    if (k == r.k0) trace_mark(a, s, wtid, 3);
+    const uint16_t* kb = reinterpret_cast<const uint16_t*>(s.ring[slot]);
+    const uint16_t* vb = reinterpret_cast<const uint16_t*>(s.ring[slot] + kSlotBytes / 2);
+    for (int j = warp; j < nk; j += kWorkerWarps) {
+      float kv[DPL], vv[DPL];
+      load_kv_row<DPL>(kb + (size_t)j * d + lane * DPL, kv);
+      load_kv_row<DPL>(vb + (size_t)j * d + lane * DPL, vv);
+      attn_key<DPL, G>(st, kv, vv);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.empty[slot]);
+    ++seq;
+  }
+  if (has_new) attn_key<DPL, G>(st, kn, vn);
+  trace_mark(a, s, wtid, 4);
+  // Merge the 16 warps' (max, sum, output): warps 8-15 into warps 0-7, then
+  // one pass over the 8 remaining states with one output element per thread.
+  float* buf = s.scratch;
+  const int sw = G * PS;
+  constexpr int kHalf = kWorkerWarps / 2;
+  if (warp >= kHalf) attn_write_state<DPL, G>(st, buf + (warp - kHalf) * sw, PS, d, lane);
+  worker_sync();
+  if (warp < kHalf) {
+    const float* src = buf + warp * sw;
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float m2 = src[h * PS + d], l2 = src[h * PS + d + 1];
+      if (m2 == -INFINITY) continue;
+      float o2[DPL];
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) o2[i] = src[h * PS + lane * DPL + i];
+      if (st.mx[h] == -INFINITY) {
+        st.mx[h] = m2;
+        st.l[h] = l2;
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) st.o[h][i] = o2[i];
+      } else {
+        const float mn = fmaxf(st.mx[h], m2);
+        const float c1 = __expf(st.mx[h] - mn), c2 = __expf(m2 - mn);
+        st.l[h] = st.l[h] * c1 + l2 * c2;
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) st.o[h][i] = st.o[h][i] * c1 + o2[i] * c2;
+        st.mx[h] = mn;
+      }
+    }
+  }
+  worker_sync();
+  if (warp < kHalf) attn_write_state<DPL, G>(st, buf + warp * sw, PS, d, lane);
+  worker_sync();
+  // The split's partial -- output unnormalised at the split's maximum, the
+  // maximum, the sum -- for the O projection to merge.
+  float* part = m.part + ((size_t)(b * m.n_kv + g) * S_all + split) * G * PS;
+  for (int idx = wtid; idx < G * (d + 2); idx += kWorkerThreads) {
+    const int h = idx / (d + 2), i = idx - h * (d + 2);
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kHalf; ++w) M = fmaxf(M, buf[w * sw + h * PS + d]);
+    float val = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kHalf; ++w) {
+        const float mw = buf[w * sw + h * PS + d];
+        if (mw == -INFINITY) continue;
+        const float x = i < d ? buf[w * sw + h * PS + i] : buf[w * sw + h * PS + d + 1];
+        val = fmaf(__expf(mw - M), x, val);
+      }
+    }
+    // i < d: output dim i; i == d: the maximum; i == d + 1: the sum
+    part[h * PS + i] = i == d ? M : val;
+  }
+}
+
+__device__ __forceinline__ void attn_dispatch(const KernelArgs& a, Smem& s, const Task& t, uint32_t& seq, int wtid) {
   const int G = a.m.group;
   if (a.m.head_dim == 128) {
     switch (G) {
@@ -793,7 +908,7 @@ __device__ void attn_dispatch(const KernelArgs& a, Smem& s, const Task& t, uint3
 
 // ------------------------------------------------------------------ worker
 
-__device__ void worker(const KernelArgs& a, Smem& s, int q0, int q1) {
+__device__ __forceinline__ void worker(const KernelArgs& a, Smem& s, int q0, int q1) {
   const int wtid = threadIdx.x - kFirstWorkerWarp * 32;
   uint32_t seq = 0;
   int i = 0;
@@ -803,10 +918,12 @@ __device__ void worker(const KernelArgs& a, Smem& s, int q0, int q1) {
     // all workers agree: the flag was published before the ready arrival
     worker_sync();
     if (!go || aborting(s)) break;
+    if (wtid == 0) s.cur_qi = qi;  // read by this thread only (trace_mark)
+    trace_mark(a, s, wtid, 1);
     switch (t.kind) {
       case T_ATTN:
         attn_dispatch(a, s, t, seq, wtid);
-        finish_task(a, s, t, wtid, false);
+        finish_task(a, s, t, wtid, true);
         break;
       case T_LMHEAD:
         gemv_core(a, s, t, seq, wtid);
@@ -820,6 +937,11 @@ __device__ void worker(const KernelArgs& a, Smem& s, int q0, int q1) {
         else epilogue_residual(a, s, t, wtid);
         finish_task(a, s, t, wtid, true);
         break;
+    }
+    if (a.m.trace && wtid == 0) {
+      a.m.trace[(size_t)qi * kTraceWords + 6] = globaltimer_ns();
+      a.m.trace[(size_t)qi * kTraceWords + 7] =
+          ((unsigned long long)blockIdx.x << 32) | (unsigned)a.queue[qi];
     }
   }
 }
@@ -837,7 +959,6 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
     mbar_init(&s.ready, 1);
     mbar_init(&s.done, 1);
     s.abort_flag = 0;
-    s.consumed_seq = 0;
     s.flag = 0;
     s.epoch = *reinterpret_cast<volatile uint32_t*>(a.m.epoch);
     fence_barrier_init();

@@ -33,13 +33,14 @@ constexpr int kRingSlots = 6;                     // 192 KB of weights in flight
 constexpr int kScratchBytes = 20480;              // GEMV partial sums / attention merge
 constexpr int kYBufFloats = 1024;                 // reduced GEMV outputs of one task
 constexpr int kMaxTaskRowsCap = 1024;
+constexpr int kDefaultL2Prefetch = 0;             // chunks prefetched into L2 at a stall
 
 // One task.  64 bytes, read by all three warp roles of the owning CTA.
 struct Task {
   int32_t kind;
   int32_t layer;
   int32_t row0, row1;      // GEMV: packed output rows [row0, row1); ATTN: group, split
-  int32_t req;             // ATTN: batch slot
+  int32_t req;             // ATTN: batch slot; LMHEAD: bit 0 first / bit 1 last LM task of its CTA
   int32_t wait_ev;         // -1: no wait
   uint32_t wait_count;     // signals per step
   int32_t sig_ev0;         // first event bumped on completion (-1: none)
@@ -48,7 +49,7 @@ struct Task {
   int32_t tpr;             // GEMV: threads per row-lane (32..512, power of two)
   int32_t chunk_rows;      // GEMV: rows per ring chunk
   const uint16_t* w;       // GEMV: packed bf16 matrix base (row-major, K columns)
-  int32_t aux;             // LMHEAD: argmax slot index; ATTN: ticket index
+  int32_t aux;             // LMHEAD: argmax slot of the owning CTA
   int32_t stage;           // operator stage (per-operator mode)
 };
 static_assert(sizeof(Task) == 64, "Task layout");
@@ -70,7 +71,9 @@ struct ModelDev {
   int32_t n_layers, hidden, n_q, n_kv, head_dim, ffn, vocab, group;
   int32_t max_seq, max_batch, attn_splits, qkv_bias;
   float rms_eps, attn_scale;
-  int32_t n_lm_tasks, timeout_ms;
+  int32_t n_lm_slots, timeout_ms;  // CTAs holding LM-head tasks (argmax slots)
+  int32_t l2_prefetch_chunks;  // chunks past the ring prefetched into L2 when a task must wait (0: off)
+  int32_t pad0_;
   // packed weights
   const uint16_t* embed;       // [vocab][hidden]
   const uint16_t* lm_head;     // [vocab][hidden] (== embed when tied)
@@ -89,14 +92,17 @@ struct ModelDev {
   float* q;        // [batch][n_q*head_dim] rotated queries
   float* attn;     // [batch][n_q*head_dim] attention output
   float* act;      // [batch][ffn] SwiGLU output
-  float* part;     // [batch][n_kv][splits][group][head_dim + 2] split partials
-  unsigned long long* am; // [batch][n_lm_tasks] packed (value, index) argmax partials
+  float* part;     // [batch][n_kv][splits][group][attn_part_stride(d)] split partials
+  unsigned long long* am; // [batch][n_lm_slots] packed (value, index) argmax partials
   // sync
   uint32_t* events;
-  uint32_t* tickets;       // [batch][layers][n_kv] attention combine tickets, then LM tickets
+  uint32_t* tickets;       // [0]: LM-head argmax ticket
   uint32_t* epoch;         // completed steps
   int32_t* status;         // 0 ok, else an MK_ERR_* code
   int32_t* status_info;    // task index / detail of the first error
+  // optional per-task trace: 4 words per queue entry of the megakernel queue set
+  // (event satisfied, workers start, workers done [%globaltimer ns], cta << 32 | task)
+  unsigned long long* trace;
 };
 
 struct KernelArgs {
@@ -157,6 +163,18 @@ MK_HD int gemv_max_task_rows(int K) {
   int r = kScratchBytes / (4 * wpr);
   if (r > kYBufFloats) r = kYBufFloats;
   return r;
+}
+
+// Attention split partial record: o[d], then m and l, padded to 16 bytes.
+MK_HD int attn_part_stride(int d) { return d + 4; }
+
+// Attention splits actually used at a position: about one split per
+// kAttnKeysPerSplit keys, at most the graph's `splits` tasks per KV head.  A
+// short context then has few partials for the O projection to merge.
+constexpr int kAttnKeysPerSplit = 256;
+MK_HD int attn_live_splits(int n_keys, int splits) {
+  int s = (n_keys + kAttnKeysPerSplit - 1) / kAttnKeysPerSplit;
+  return s < 1 ? 1 : (s > splits ? splits : s);
 }
 
 // Attention: keys per ring chunk (K rows in the first half of a slot, V rows

@@ -14,7 +14,7 @@
 // (further cut so the per-task partial sums fit in shared memory); attention
 // is cut per (batch slot, KV head, key split).  Dependencies:
 //   ATTN(l,g)  waits until every QKV(l) task that wrote rows of group g is done
-//   OPROJ(l)   waits until every group's split partials were merged
+//   OPROJ(l)   waits for every ATTN(l) split; its prologue merges the partials
 //   GATEUP(l)  waits for all OPROJ(l)    (RMSNorm needs the whole residual)
 //   DOWN(l)    waits for all GATEUP(l)   (the GEMV needs the whole activation)
 //   QKV(l+1) and the LM head wait for all DOWN(l).
@@ -36,10 +36,11 @@ std::string validate_config(const mk_config& c) {
   if (c.n_q_heads % c.n_kv_heads) return "n_q_heads must be a multiple of n_kv_heads";
   if (c.hidden % 8 || c.ffn % 8) return "hidden and ffn must be multiples of 8";
   int qd = c.n_q_heads * c.head_dim;
-  if (c.hidden > 16384 || c.ffn > 16384 || qd > 16384) return "GEMV inputs are limited to 16384";
+  if (c.hidden > 16384 || c.ffn > 16384) return "GEMV inputs are limited to 16384";
+  if (qd > 8192) return "n_q_heads * head_dim is limited to 8192";
   int G = c.n_q_heads / c.n_kv_heads;
-  // attention merge scratch: 8 warps x G heads x (d + 2) floats
-  if (8 * G * (c.head_dim + 2) * 4 > kScratchBytes) {
+  // attention merge scratch: 8 warps x G heads x (d + 4) floats
+  if (8 * G * attn_part_stride(c.head_dim) * 4 > kScratchBytes) {
     snprintf(buf, sizeof buf, "query heads per KV head (%d) too large for head_dim %d", G,
              c.head_dim);
     return buf;
@@ -121,8 +122,8 @@ struct Builder {
     p.event_count.assign(ev.count(), 0);
     p.n_events = ev.count();
     p.attn_splits = splits;
-    p.n_tickets = B * L * nkv + 1;
-    p.lm_ticket = B * L * nkv;
+    p.n_tickets = 1;
+    p.lm_ticket = 0;
     p.n_stages = 5 * L + 1;
     for (int l = 0; l < L; ++l) {
       // QKV: rows of whole RoPE pairs; signal every group the rows touch.
@@ -145,15 +146,14 @@ struct Builder {
         t.row1 = s;
         t.req = req;
         t.wait_ev = ev.qkv(l, g);
-        t.sig_ev0 = ev.attn(l);  // bumped once per (slot, group) by the merging split
-        t.n_sig = 0;
+        t.sig_ev0 = ev.attn(l);
+        t.n_sig = 1;
         t.K = d;
-        t.aux = (req * L + l) * nkv + g;
+        t.aux = -1;
         t.stage = l * 5 + T_ATTN;
         int cta = (int)((long long)a * P / A);
         add(t, cta);
       }
-      p.event_count[ev.attn(l)] += B * nkv;  // one merge per (slot, group)
       split_rows(H, 1, gemv_max_task_rows(nq * d), [&](int cta, int r0, int r1) {
         Task t = gemv_task(T_OPROJ, l, nq * d, r0, r1);
         t.wait_ev = ev.attn(l);
@@ -176,15 +176,30 @@ struct Builder {
         add(t, cta);
       });
     }
-    int n_lm = 0;
+    // LM head: one argmax slot per CTA; its tasks keep a running best in
+    // shared memory and only the CTA's last one publishes it.
+    int n_lm = 0, n_slots = 0, last_cta = -1;
+    std::vector<int> lm_ids;
     split_rows(V, 1, gemv_max_task_rows(H), [&](int cta, int r0, int r1) {
       Task t = gemv_task(T_LMHEAD, L, H, r0, r1);
       t.layer = L - 1;
       t.wait_ev = ev.down(L - 1);
-      t.aux = n_lm++;
-      add(t, cta);
+      if (cta != last_cta) {
+        ++n_slots;
+        last_cta = cta;
+      }
+      t.aux = n_slots - 1;
+      lm_ids.push_back(add(t, cta));
+      ++n_lm;
     });
+    for (size_t i = 0; i < lm_ids.size(); ++i) {
+      Task& t = p.tasks[lm_ids[i]];
+      const bool first = i == 0 || p.tasks[lm_ids[i - 1]].aux != t.aux;
+      const bool last = i + 1 == lm_ids.size() || p.tasks[lm_ids[i + 1]].aux != t.aux;
+      t.req = (first ? 1 : 0) | (last ? 2 : 0);
+    }
     p.n_lm_tasks = n_lm;
+    p.n_lm_slots = n_slots;
     // Thresholds: every wait targets the full per-step count of its event.
     for (auto& t : p.tasks)
       if (t.wait_ev >= 0) t.wait_count = p.event_count[t.wait_ev];

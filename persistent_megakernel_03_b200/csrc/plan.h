@@ -12,6 +12,7 @@ struct Plan {
   int num_ctas = 0;
   int attn_splits = 1;
   int n_lm_tasks = 0;
+  int n_lm_slots = 0;                      // CTAs holding LM-head tasks
   int n_events = 0;
   int n_tickets = 0;
   int n_stages = 0;

@@ -77,7 +77,6 @@ def _simulate(plan, model, max_batch, rng):
     written = {}      # (kind, layer) -> set of rows
     done_kind = {}    # (kind, layer) -> count of finished tasks
     tickets = {}
-    merged = {}
     total = {}
     for t in tasks:
         total[(t["kind"], t["layer"])] = total.get((t["kind"], t["layer"]), 0) + 1
@@ -99,8 +98,9 @@ def _simulate(plan, model, max_batch, rng):
             rows = set(range(t["row0"] * per_group, (t["row0"] + 1) * per_group))
             assert rows <= written.get((QKV, l), set())
         if k == OPROJ:
-            assert merged.get(l, 0) == max_batch * nkv
-            # every QKV(l) task read x before OPROJ(l) overwrites it
+            # every split of every (slot, group) wrote its partial ...
+            assert done_kind.get((ATTN, l), 0) == total[(ATTN, l)] == max_batch * nkv * S
+            # ... and every QKV(l) task read x before OPROJ(l) overwrites it
             assert done_kind.get((QKV, l), 0) == total[(QKV, l)]
         if k == GATEUP:
             assert len(written.get((OPROJ, l), ())) == model.hidden
@@ -114,14 +114,12 @@ def _simulate(plan, model, max_batch, rng):
             rs = written.setdefault((k, l), set())
             assert not (rs & set(range(t["row0"], t["row1"]))), "row written twice"
             rs.update(range(t["row0"], t["row1"]))
-            for e in range(t["signal_event0"], t["signal_event0"] + t["n_signal"]):
-                ev[e] += 1
         else:
-            key = (t["req"], l, t["row0"])
-            tickets[key] = tickets.get(key, 0) + 1
-            if tickets[key] == S:
-                merged[l] = merged.get(l, 0) + 1
-                ev[t["signal_event0"]] += 1
+            key = (t["req"], l, t["row0"], t["row1"])
+            assert key not in tickets, "split computed twice"
+            tickets[key] = 1
+        for e in range(t["signal_event0"], t["signal_event0"] + t["n_signal"]):
+            ev[e] += 1
         done_kind[(k, l)] = done_kind.get((k, l), 0) + 1
         finished += 1
     assert ev == counts
