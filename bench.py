@@ -212,6 +212,8 @@ def run_mk(args):
     w = synth.make_model(model, 0, device="cuda")
     stream = torch.cuda.current_stream()
     dec = binding.Decoder(model, w, max_seq, stream=stream, l2_prefetch=args.l2_prefetch)
+    del w  # mk_create copied and packed the weights
+    torch.cuda.empty_cache()
     prompt = synth.make_prompt(PROMPT, model.vocab).cuda()
     ids = [torch.zeros(1, dtype=torch.int32, device="cuda") for _ in range(2)]
 
@@ -351,7 +353,6 @@ def run_mk(args):
     if trace_summary:
         line["trace"] = {k: trace_summary[k] for k in ("step_us", "mean_cta_busy_frac")}
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
-        del w
         dec.close()
         torch.cuda.empty_cache()
         w2 = synth.make_model(model, 0, device="cuda")

@@ -163,6 +163,24 @@ int mk_status(mk_ctx* ctx);
 const char* mk_last_error(const mk_ctx* ctx);
 void mk_destroy(mk_ctx* ctx);
 
+/* Split-KV grouped-query decode attention for one KV head ("Hạt nhân là gì
+ * ...": online softmax, exact up to rounding; "LLM高速化勉強会資料" slides
+ * 11-13 and 28).  q_dev: fp32 [n_q_per_kv][head_dim] query rows of the
+ * heads that share this KV head; k_dev, v_dev: bf16 [n_keys][head_dim]
+ * row-major, 8-byte aligned; out_dev: fp32 [n_q_per_kv][head_dim] =
+ * softmax(q K^T / sqrt(head_dim)) V per query head.  The keys are cut into
+ * `splits` contiguous blocks of ceil(n_keys / splits), one CTA each; the last
+ * CTA to finish merges the blocks.  workspace_dev holds the blocks' partial
+ * results and a merge ticket: mk_attention_workspace_bytes(...) bytes, 16-byte
+ * aligned, zeroed by the caller before its first use (the op leaves the
+ * ticket at zero after every call, so it can be reused on the same stream;
+ * two calls in flight at once on one workspace race).  head_dim 64 or 128;
+ * n_q_per_kv 1, 2, 4, 7 or 8.  Enqueued on `stream`. */
+size_t mk_attention_workspace_bytes(int n_q_per_kv, int head_dim, int splits);
+int mk_attention_decode(const float* q_dev, const void* k_dev, const void* v_dev, int n_keys,
+                        int n_q_per_kv, int head_dim, int splits, void* workspace_dev,
+                        float* out_dev, void* stream);
+
 /* Read-only HBM stream probe: every byte of src_dev[0, bytes) is loaded
  * once with 128-bit loads by a grid of (SMs x 4) CTAs; a value derived from
  * the data is written to sink_dev[0] so nothing is elided.  bytes must be a

@@ -26,7 +26,8 @@ EXPORTS = ("mk_create", "mk_prefill", "mk_decode_step", "mk_decode_step_host", "
            "mk_kv_pointer", "mk_copy_kv", "mk_set_mode", "mk_status", "mk_last_error",
            "mk_destroy", "mk_plan_build", "mk_plan_get_info", "mk_plan_get_tasks",
            "mk_plan_get_queue", "mk_plan_get_event_counts", "mk_plan_destroy",
-           "mk_qkv_row_source", "mk_read_probe", "mk_set_trace")
+           "mk_qkv_row_source", "mk_read_probe", "mk_set_trace",
+           "mk_attention_workspace_bytes", "mk_attention_decode")
 
 
 class MkError(RuntimeError):
@@ -114,6 +115,9 @@ def lib(build_if_missing: bool = True):
     L.mk_qkv_row_source.argtypes = [C.POINTER(Config), i, ip, ip, ip]
     L.mk_read_probe.argtypes = [vp, C.c_size_t, vp, vp]
     L.mk_set_trace.argtypes = [vp, vp]
+    L.mk_attention_workspace_bytes.argtypes = [i, i, i]
+    L.mk_attention_workspace_bytes.restype = C.c_size_t
+    L.mk_attention_decode.argtypes = [vp, vp, vp, i, i, i, i, vp, vp, vp]
     _lib = L
     return L
 
@@ -280,3 +284,18 @@ def read_probe(src_dev, sink_dev, stream=None):
     st = stream if stream is not None else torch.cuda.current_stream()
     nbytes = src_dev.numel() * src_dev.element_size()
     _check(lib().mk_read_probe(src_dev.data_ptr(), nbytes, sink_dev.data_ptr(), st.cuda_stream))
+
+
+def attention_workspace_bytes(n_q_per_kv: int, head_dim: int, splits: int) -> int:
+    return int(lib().mk_attention_workspace_bytes(n_q_per_kv, head_dim, splits))
+
+
+def attention_decode(q_dev, k_dev, v_dev, n_keys: int, splits: int, workspace_dev, out_dev,
+                     stream=None):
+    """Split-KV decode attention for one KV head (see mk_attention_decode)."""
+    import torch
+    st = stream if stream is not None else torch.cuda.current_stream()
+    G, d = q_dev.shape
+    _check(lib().mk_attention_decode(q_dev.data_ptr(), k_dev.data_ptr(), v_dev.data_ptr(),
+                                     int(n_keys), int(G), int(d), int(splits),
+                                     workspace_dev.data_ptr(), out_dev.data_ptr(), st.cuda_stream))

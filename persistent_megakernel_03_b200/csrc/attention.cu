@@ -1,0 +1,170 @@
+// attention.cu -- standalone split-KV grouped-query decode attention.
+//
+// One KV head and its G query heads against n cached keys: the keys are cut
+// into `splits` contiguous blocks, one CTA each.  Every warp of a CTA keeps an
+// online softmax (running maximum, running sum, rescaled output) over its
+// keys; the CTA merges its warps and writes its block's partial (unnormalised
+// output at the block maximum, the maximum, the sum) to the workspace; the
+// last CTA to finish merges the blocks ("Hạt nhân là gì ...": the online
+// softmax gives the exact softmax up to rounding; "LLM高速化勉強会資料" slides
+// 11-13, 28; "Crear desde cero ..." §3.4).  The same math runs inside the
+// persistent decode kernel's attention tasks (attn_math.cuh).
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include "../../include/mk.h"
+#include "attn_math.cuh"
+#include "mk_internal.h"
+
+namespace mk {
+
+constexpr int kAttnOpWarps = 8;
+constexpr int kAttnOpMaxG = 8;
+constexpr size_t kAttnTicketBytes = 256;  // the merge ticket, padded
+
+// Workspace: [ticket u32, padded to 256 B][splits][G][attn_part_stride(d)] floats.
+size_t attn_op_workspace_bytes(int G, int d, int splits) {
+  return kAttnTicketBytes + (size_t)splits * G * attn_part_stride(d) * sizeof(float);
+}
+
+template <int DPL, int G>
+__global__ void __launch_bounds__(kAttnOpWarps * 32)
+    attn_decode_kernel(const float* __restrict__ q, const uint16_t* __restrict__ K,
+                       const uint16_t* __restrict__ V, int n, float scale, int splits,
+                       uint8_t* __restrict__ ws, float* __restrict__ out) {
+  constexpr int d = DPL * 32, PS = d + 4;
+  __shared__ __align__(16) float buf[kAttnOpWarps][G][PS];
+  __shared__ int last;
+  unsigned int* ticket = reinterpret_cast<unsigned int*>(ws);
+  float* part = reinterpret_cast<float*>(ws + kAttnTicketBytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, split = blockIdx.x;
+  const int chunk = (n + splits - 1) / splits;
+  const int k0 = min(n, split * chunk), k1 = min(n, k0 + chunk);
+
+  AttnState<DPL, G> st;
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) {
+      st.q[h][i] = q[h * d + lane * DPL + i] * scale;
+      st.o[h][i] = 0.f;
+    }
+    st.mx[h] = -INFINITY;
+    st.l[h] = 0.f;
+  }
+  for (int j = k0 + warp; j < k1; j += kAttnOpWarps) {
+    float kv[DPL], vv[DPL];
+    load_kv_row_global<DPL>(K + (size_t)j * d + lane * DPL, kv);
+    load_kv_row_global<DPL>(V + (size_t)j * d + lane * DPL, vv);
+    attn_key<DPL, G>(st, kv, vv);
+  }
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) buf[warp][h][lane * DPL + i] = st.o[h][i];
+    if (lane == 0) {
+      buf[warp][h][d] = st.mx[h];
+      buf[warp][h][d + 1] = st.l[h];
+    }
+  }
+  __syncthreads();
+  // This block's partial: the warps merged at their common maximum.
+  float* mine = part + (size_t)split * G * PS;
+  for (int idx = threadIdx.x; idx < G * (d + 2); idx += blockDim.x) {
+    const int h = idx / (d + 2), i = idx - h * (d + 2);
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kAttnOpWarps; ++w) M = fmaxf(M, buf[w][h][d]);
+    float val = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kAttnOpWarps; ++w) {
+        const float mw = buf[w][h][d];
+        if (mw == -INFINITY) continue;
+        val = fmaf(__expf(mw - M), i < d ? buf[w][h][i] : buf[w][h][d + 1], val);
+      }
+    }
+    mine[h * PS + i] = i == d ? M : val;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    last = atomicAdd(ticket, 1u) == (unsigned)splits - 1u;
+  }
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  // Last block: merge every block's partial and normalise.
+  for (int idx = threadIdx.x; idx < G * d; idx += blockDim.x) {
+    const int h = idx / d, i = idx - h * d;
+    float M = -INFINITY;
+    for (int s = 0; s < splits; ++s) M = fmaxf(M, __ldcg(part + ((size_t)s * G + h) * PS + d));
+    float num = 0.f, den = 0.f;
+    for (int s = 0; s < splits; ++s) {
+      const float* ps = part + ((size_t)s * G + h) * PS;
+      const float ls = __ldcg(ps + d + 1);
+      if (ls == 0.f) continue;
+      const float c = __expf(__ldcg(ps + d) - M);
+      num = fmaf(c, __ldcg(ps + i), num);
+      den = fmaf(c, ls, den);
+    }
+    out[h * d + i] = num / den;
+  }
+  // Leave the ticket at zero for the next call on this workspace.
+  if (threadIdx.x == 0) *ticket = 0u;
+}
+
+template <int DPL>
+static cudaError_t launch_attn_g(int G, const float* q, const uint16_t* K, const uint16_t* V,
+                                 int n, float scale, int splits, uint8_t* ws, float* out,
+                                 cudaStream_t st) {
+  const dim3 grid(splits), block(kAttnOpWarps * 32);
+  switch (G) {
+    case 1: attn_decode_kernel<DPL, 1><<<grid, block, 0, st>>>(q, K, V, n, scale, splits, ws, out); break;
+    case 2: attn_decode_kernel<DPL, 2><<<grid, block, 0, st>>>(q, K, V, n, scale, splits, ws, out); break;
+    case 4: attn_decode_kernel<DPL, 4><<<grid, block, 0, st>>>(q, K, V, n, scale, splits, ws, out); break;
+    case 7: attn_decode_kernel<DPL, 7><<<grid, block, 0, st>>>(q, K, V, n, scale, splits, ws, out); break;
+    case 8: attn_decode_kernel<DPL, 8><<<grid, block, 0, st>>>(q, K, V, n, scale, splits, ws, out); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+// Checks the arguments of the attention op; returns 0 or an MK_ERR_* code.
+int attn_op_check(const float* q, const void* k, const void* v, int n, int G, int d, int splits,
+                  const float* out) {
+  if (!q || !k || !v || !out) return MK_ERR_INVALID_ARG;
+  if (n < 1 || splits < 1 || splits > 4096) return MK_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return MK_ERR_UNSUPPORTED;
+  if (!(G == 1 || G == 2 || G == 4 || G == 7 || G == 8)) return MK_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) & 7u) return MK_ERR_INVALID_ARG;
+  return MK_OK;
+}
+
+cudaError_t launch_attn_op(const float* q, const void* k, const void* v, int n, int G, int d,
+                           int splits, void* ws, float* out, cudaStream_t st) {
+  const float scale = (float)(1.0 / sqrt((double)d));
+  const uint16_t* K = static_cast<const uint16_t*>(k);
+  const uint16_t* V = static_cast<const uint16_t*>(v);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  return d == 128 ? launch_attn_g<4>(G, q, K, V, n, scale, splits, w, out, st)
+                  : launch_attn_g<2>(G, q, K, V, n, scale, splits, w, out, st);
+}
+
+}  // namespace mk
+
+extern "C" size_t mk_attention_workspace_bytes(int n_q_per_kv, int head_dim, int splits) {
+  if (n_q_per_kv < 1 || n_q_per_kv > mk::kAttnOpMaxG || head_dim < 1 || splits < 1) return 0;
+  return mk::attn_op_workspace_bytes(n_q_per_kv, head_dim, splits);
+}
+
+extern "C" int mk_attention_decode(const float* q_dev, const void* k_dev, const void* v_dev,
+                                   int n_keys, int n_q_per_kv, int head_dim, int splits,
+                                   void* workspace_dev, float* out_dev, void* stream) {
+  int rc = mk::attn_op_check(q_dev, k_dev, v_dev, n_keys, n_q_per_kv, head_dim, splits, out_dev);
+  if (rc) return rc;
+  if (!workspace_dev || (reinterpret_cast<uintptr_t>(workspace_dev) & 15u)) return MK_ERR_INVALID_ARG;
+  cudaError_t e = mk::launch_attn_op(q_dev, k_dev, v_dev, n_keys, n_q_per_kv, head_dim, splits,
+                                     workspace_dev, out_dev, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MK_OK : MK_ERR_CUDA;
+}
