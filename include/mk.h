@@ -181,6 +181,22 @@ int mk_attention_decode(const float* q_dev, const void* k_dev, const void* v_dev
                         int n_q_per_kv, int head_dim, int splits, void* workspace_dev,
                         float* out_dev, void* stream);
 
+/* mk_attention_decode without a workspace argument, for callers that cannot
+ * allocate device memory (a plugin whose host owns all device memory, a
+ * real-time loop that must not enter an allocator, code that may only use
+ * the buffers it is given).  No counterpart on the pages: this is a
+ * packaging of the op above.  The scratch is a 270,592-byte array compiled
+ * into the library, so this entry point never allocates; it serves up to 64
+ * splits for 8 query heads per KV head at head_dim 128 (larger requests
+ * return MK_ERR_INVALID_ARG, see mk_last_error(NULL)).  The first call on a
+ * device looks up the array's device address and clears its merge ticket;
+ * make that first call before any stream capture.  All calls on a device
+ * share the one array, which keeps the last call's partials: calls that
+ * overlap on the GPU (other streams, other threads) race. */
+int mk_attention_decode_noalloc(const float* q_dev, const void* k_dev, const void* v_dev,
+                                int n_keys, int n_q_per_kv, int head_dim, int splits,
+                                float* out_dev, void* stream);
+
 /* Read-only HBM stream probe: every byte of src_dev[0, bytes) is loaded
  * once with 128-bit loads by a grid of (SMs x 4) CTAs; a value derived from
  * the data is written to sink_dev[0] so nothing is elided.  bytes must be a

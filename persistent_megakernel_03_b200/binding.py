@@ -27,7 +27,8 @@ EXPORTS = ("mk_create", "mk_prefill", "mk_decode_step", "mk_decode_step_host", "
            "mk_destroy", "mk_plan_build", "mk_plan_get_info", "mk_plan_get_tasks",
            "mk_plan_get_queue", "mk_plan_get_event_counts", "mk_plan_destroy",
            "mk_qkv_row_source", "mk_read_probe", "mk_set_trace",
-           "mk_attention_workspace_bytes", "mk_attention_decode")
+           "mk_attention_workspace_bytes", "mk_attention_decode",
+           "mk_attention_decode_noalloc")
 
 
 class MkError(RuntimeError):
@@ -118,6 +119,7 @@ def lib(build_if_missing: bool = True):
     L.mk_attention_workspace_bytes.argtypes = [i, i, i]
     L.mk_attention_workspace_bytes.restype = C.c_size_t
     L.mk_attention_decode.argtypes = [vp, vp, vp, i, i, i, i, vp, vp, vp]
+    L.mk_attention_decode_noalloc.argtypes = [vp, vp, vp, i, i, i, i, vp, vp]
     _lib = L
     return L
 
@@ -299,3 +301,15 @@ def attention_decode(q_dev, k_dev, v_dev, n_keys: int, splits: int, workspace_de
     _check(lib().mk_attention_decode(q_dev.data_ptr(), k_dev.data_ptr(), v_dev.data_ptr(),
                                      int(n_keys), int(G), int(d), int(splits),
                                      workspace_dev.data_ptr(), out_dev.data_ptr(), st.cuda_stream))
+
+
+def attention_decode_noalloc(q_dev, k_dev, v_dev, n_keys: int, splits: int, out_dev,
+                             stream=None):
+    """mk_attention_decode with the library's static scratch instead of a
+    caller workspace (see mk_attention_decode_noalloc)."""
+    import torch
+    st = stream if stream is not None else torch.cuda.current_stream()
+    G, d = q_dev.shape
+    _check(lib().mk_attention_decode_noalloc(q_dev.data_ptr(), k_dev.data_ptr(),
+                                             v_dev.data_ptr(), int(n_keys), int(G), int(d),
+                                             int(splits), out_dev.data_ptr(), st.cuda_stream))

@@ -51,6 +51,10 @@ struct mk_ctx {
   size_t kv_bytes = 0;
 };
 
+namespace mk {
+void set_last_error(const char* msg) { g_create_error = msg; }
+}  // namespace mk
+
 static int fail(mk_ctx* c, int code, const std::string& msg) {
   if (c) c->err = msg; else g_create_error = msg;
   return code;

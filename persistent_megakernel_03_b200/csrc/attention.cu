@@ -12,11 +12,16 @@
 #include <cuda_runtime.h>
 #include <math.h>
 
+#include <mutex>
+#include <string>
+
 #include "../../include/mk.h"
 #include "attn_math.cuh"
 #include "mk_internal.h"
 
 namespace mk {
+
+void set_last_error(const char* msg);  // api.cu: the message mk_last_error(NULL) returns
 
 constexpr int kAttnOpWarps = 8;
 constexpr int kAttnOpMaxG = 8;
@@ -166,5 +171,70 @@ extern "C" int mk_attention_decode(const float* q_dev, const void* k_dev, const 
   if (!workspace_dev || (reinterpret_cast<uintptr_t>(workspace_dev) & 15u)) return MK_ERR_INVALID_ARG;
   cudaError_t e = mk::launch_attn_op(q_dev, k_dev, v_dev, n_keys, n_q_per_kv, head_dim, splits,
                                      workspace_dev, out_dev, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MK_OK : MK_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant.  Some callers cannot allocate device memory at all:
+// a plugin inside a host that owns every byte of device memory through its
+// own pool, a real-time loop that must never enter an allocator, or code that
+// is only allowed to touch buffers it was handed.  For them the workspace of
+// the op above lives in a fixed array compiled into this library.  Every GPU
+// that loads the library holds the array until the process exits.
+namespace mk {
+namespace {
+
+constexpr int kNoAllocMaxSplits = 64;   // key blocks
+constexpr int kNoAllocMaxG = 8;         // query heads per KV head
+constexpr int kNoAllocMaxHeadDim = 128;
+constexpr size_t kNoAllocBytes =
+    kAttnTicketBytes + (size_t)kNoAllocMaxSplits * kNoAllocMaxG * (kNoAllocMaxHeadDim + 4) * sizeof(float);
+
+// The shared scratch: 270,592 bytes per device.
+static __device__ __align__(256) uint8_t g_attn_noalloc_scratch[kNoAllocBytes];
+
+constexpr int kMaxDevices = 128;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+}  // namespace
+}  // namespace mk
+
+extern "C" int mk_attention_decode_noalloc(const float* q_dev, const void* k_dev, const void* v_dev,
+                                           int n_keys, int n_q_per_kv, int head_dim, int splits,
+                                           float* out_dev, void* stream) {
+  using namespace mk;
+  int rc = attn_op_check(q_dev, k_dev, v_dev, n_keys, n_q_per_kv, head_dim, splits, out_dev);
+  if (rc) return rc;
+  const size_t need = attn_op_workspace_bytes(n_q_per_kv, head_dim, splits);
+  if (need > kNoAllocBytes) {
+    set_last_error(("mk_attention_decode_noalloc: needs " + std::to_string(need) +
+                    " bytes of scratch, the static array holds " + std::to_string(kNoAllocBytes) +
+                    " (at most 64 splits for 8 query heads per KV head at head_dim 128)").c_str());
+    return MK_ERR_INVALID_ARG;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MK_ERR_CUDA;
+  void* scratch = nullptr;
+  {
+    // First call on this device: look up the device address of the array
+    // (the array's name in host code is only a stand-in for it) and clear
+    // the merge ticket.  Later calls reuse the address.
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_attn_noalloc_scratch) != cudaSuccess || !p) {
+        cudaGetLastError();
+        set_last_error("mk_attention_decode_noalloc: cudaGetSymbolAddress failed");
+        return MK_ERR_CUDA;
+      }
+      if (cudaMemsetAsync(p, 0, kAttnTicketBytes, st) != cudaSuccess) return MK_ERR_CUDA;
+      g_noalloc_ptr[dev] = p;
+    }
+    scratch = g_noalloc_ptr[dev];
+  }
+  cudaError_t e = launch_attn_op(q_dev, k_dev, v_dev, n_keys, n_q_per_kv, head_dim, splits,
+                                 scratch, out_dev, st);
   return e == cudaSuccess ? MK_OK : MK_ERR_CUDA;
 }
