@@ -188,7 +188,7 @@ def load_traffic():
     with open(p) as f:
         rec = json.load(f)
     h = hashlib.sha256()
-    for name in ("kernel.cu", "mk_internal.h", "ptx.cuh"):
+    for name in ("kernel.cu", "mk_internal.h", "ptx.cuh", "attn_math.cuh"):
         with open(os.path.join(ROOT, "persistent_megakernel_03_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     if rec.get("source_sha256") != h.hexdigest():
