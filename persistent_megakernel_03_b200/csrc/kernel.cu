@@ -541,8 +541,17 @@ __device__ __forceinline__ void gemv_stream(const KernelArgs& a, Smem& s, const 
     r = 1.0f / sqrtf(tot / (float)K + a.m.rms_eps);
   }
   for (int i = wtid; i < nrows; i += kWorkerThreads) {
-    float y = 0.f;
-    for (int w = 0; w < wpr; ++w) y += s.scratch[w * nrows + i];
+    // the row-lane's warp partials, four independent chains
+    float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
+    int w = 0;
+    for (; w + 4 <= wpr; w += 4) {
+      y0 += s.scratch[w * nrows + i];
+      y1 += s.scratch[(w + 1) * nrows + i];
+      y2 += s.scratch[(w + 2) * nrows + i];
+      y3 += s.scratch[(w + 3) * nrows + i];
+    }
+    for (; w < wpr; ++w) y0 += s.scratch[w * nrows + i];
+    const float y = (y0 + y1) + (y2 + y3);
     s.ybuf[i] = has_norm ? y * r : y;
   }
   worker_sync();
@@ -575,14 +584,53 @@ __device__ __forceinline__ void finish_task(const KernelArgs& a, Smem& s, const 
   worker_sync();
   if (wtid == 0) {
     if (signal && t.n_sig > 0) {
-      __threadfence();
-      for (int e = 0; e < t.n_sig; ++e) red_release_gpu_add(a.m.events + t.sig_ev0 + e, 1u);
+      // release pattern: an acq_rel fence (after the barrier, so it covers
+      // every worker's stores) then relaxed increments; measured cheaper
+      // than a sequentially consistent fence or a release reduction
+      fence_acq_rel_gpu();
+      for (int e = 0; e < t.n_sig; ++e) red_relaxed_gpu_add(a.m.events + t.sig_ev0 + e, 1u);
     }
     mbar_arrive(&s.done);
   }
 }
 
-__device__ __forceinline__ void epilogue_qkv(const KernelArgs& a, Smem& s, const Task& t, int wtid) {
+// What the epilogue of this thread's first output item needs, loaded before
+// the stream so its latency is hidden: RoPE factors and bias (QKV), the old
+// residual value (O projection, down).
+struct EpiPre {
+  float c, sn, b0, b1, res;
+};
+
+__device__ __forceinline__ EpiPre epilogue_prefetch(const KernelArgs& a, const Task& t, int wtid) {
+  const ModelDev& m = a.m;
+  const StepParams& sp = step_params(a);
+  EpiPre p{1.f, 0.f, 0.f, 0.f, 0.f};
+  const int nrows = t.row1 - t.row0;
+  if (t.kind == T_QKV) {
+    if (2 * wtid < nrows) {
+      const int r = t.row0 + 2 * wtid;
+      int which, head, dim;
+      qkv_source(r, m.group, m.head_dim, &which, &head, &dim);
+      if (which < 2) {
+        const int half = m.head_dim >> 1;
+        p.c = m.rope_cos[(size_t)sp.pos[0] * half + dim];
+        p.sn = m.rope_sin[(size_t)sp.pos[0] * half + dim];
+      }
+      if (m.qkv_bias) {
+        const uint16_t* b = m.bqkv + (size_t)t.layer * qkv_rows(m.n_q, m.n_kv, m.head_dim);
+        p.b0 = bf16_to_float(b[r]);
+        p.b1 = bf16_to_float(b[r + 1]);
+      }
+    }
+  } else if (t.kind == T_DOWN || (t.kind == T_OPROJ && t.layer > 0)) {
+    // the residual rows were written by the stage before the previous one
+    if (wtid < nrows) p.res = __ldcg(m.x + t.row0 + wtid);
+  }
+  return p;
+}
+
+__device__ __forceinline__ void epilogue_qkv(const KernelArgs& a, Smem& s, const Task& t, int wtid,
+                                             const EpiPre& pre) {
   const ModelDev& m = a.m;
   const StepParams& sp = step_params(a);
   const int d = m.head_dim, G = m.group, half = d >> 1;
@@ -592,17 +640,27 @@ __device__ __forceinline__ void epilogue_qkv(const KernelArgs& a, Smem& s, const
   for (int pi = wtid; pi < npairs; pi += kWorkerThreads) {
     const int r = t.row0 + 2 * pi;
     float y0 = s.ybuf[2 * pi], y1 = s.ybuf[2 * pi + 1];
-    if (m.qkv_bias) {
-      const uint16_t* b = m.bqkv + (size_t)t.layer * qkvR;
-      y0 = y0 + bf16_to_float(b[r]);
-      y1 = y1 + bf16_to_float(b[r + 1]);
-    }
     int which, head, dim0, w1, h1, dim1;
     qkv_source(r, G, d, &which, &head, &dim0);
     qkv_source(r + 1, G, d, &w1, &h1, &dim1);
+    float c = pre.c, sn = pre.sn, b0 = pre.b0, b1 = pre.b1;
+    if (pi != wtid) {  // items past the first load their factors here
+      c = 1.f; sn = 0.f; b0 = b1 = 0.f;
+      if (which < 2) {
+        c = m.rope_cos[(size_t)pos * half + dim0];
+        sn = m.rope_sin[(size_t)pos * half + dim0];
+      }
+      if (m.qkv_bias) {
+        const uint16_t* b = m.bqkv + (size_t)t.layer * qkvR;
+        b0 = bf16_to_float(b[r]);
+        b1 = bf16_to_float(b[r + 1]);
+      }
+    }
+    if (m.qkv_bias) {
+      y0 = y0 + b0;
+      y1 = y1 + b1;
+    }
     if (which < 2) {
-      const float c = m.rope_cos[(size_t)pos * half + dim0];
-      const float sn = m.rope_sin[(size_t)pos * half + dim0];
       const float o0 = y0 * c - y1 * sn;
       const float o1 = y0 * sn + y1 * c;
       y0 = o0;
@@ -621,7 +679,8 @@ __device__ __forceinline__ void epilogue_qkv(const KernelArgs& a, Smem& s, const
   }
 }
 
-__device__ __forceinline__ void epilogue_residual(const KernelArgs& a, Smem& s, const Task& t, int wtid) {
+__device__ __forceinline__ void epilogue_residual(const KernelArgs& a, Smem& s, const Task& t, int wtid,
+                                                  const EpiPre& pre) {
   const ModelDev& m = a.m;
   const StepParams& sp = step_params(a);
   const int nrows = t.row1 - t.row0;
@@ -634,7 +693,7 @@ __device__ __forceinline__ void epilogue_residual(const KernelArgs& a, Smem& s, 
   for (int i = wtid; i < nrows; i += kWorkerThreads) {
     const int row = t.row0 + i;
     const float old = from_embed ? bf16_to_float(m.embed[(size_t)tok * m.hidden + row])
-                                 : __ldcg(m.x + row);
+                      : (i == wtid ? pre.res : __ldcg(m.x + row));
     m.x[row] = old + s.ybuf[i];
   }
 }
@@ -877,13 +936,15 @@ __device__ __forceinline__ void worker(const KernelArgs& a, Smem& s, int q0, int
         epilogue_lmhead(a, s, t, wtid);
         finish_task(a, s, t, wtid, false);
         break;
-      default:
+      default: {
+        const EpiPre pre = epilogue_prefetch(a, t, wtid);
         gemv_core(a, s, t, seq, wtid);
-        if (t.kind == T_QKV) epilogue_qkv(a, s, t, wtid);
+        if (t.kind == T_QKV) epilogue_qkv(a, s, t, wtid, pre);
         else if (t.kind == T_GATEUP) epilogue_swiglu(a, s, t, wtid);
-        else epilogue_residual(a, s, t, wtid);
+        else epilogue_residual(a, s, t, wtid, pre);
         finish_task(a, s, t, wtid, true);
         break;
+      }
     }
     if (a.m.trace && wtid == 0) {
       a.m.trace[(size_t)qi * kTraceWords + 6] = globaltimer_ns();
