@@ -269,6 +269,15 @@ int orc_state_kv(const orc_state* s, int layer, int kv_head, int which, int n, f
   return 0;
 }
 
+int orc_state_set_kv(orc_state* s, int layer, int kv_head, int which, int n, const float* in) {
+  const orc_config* c = &s->m->c;
+  if (layer < 0 || layer >= c->n_layers || kv_head < 0 || kv_head >= c->n_kv_heads || n < 0 ||
+      n > s->max_seq || which < 0 || which > 1 || !in)
+    return -1;
+  kv_store(s, kv_index(c, s->max_seq, layer, kv_head, which, 0), in, n * c->head_dim);
+  return 0;
+}
+
 static void add_bias(float* y, const uint16_t* b, int n) {
   if (!b) return;
   for (int i = 0; i < n; ++i) y[i] = y[i] + bf16_to_f32(b[i]);

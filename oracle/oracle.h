@@ -90,6 +90,10 @@ int orc_decode(const orc_model* m, orc_state* s, int token, int pos, float* logi
 /* Cached K or V of one layer and kv head, positions [0, n): out[n*head_dim]. */
 int orc_state_kv(const orc_state* s, int layer, int kv_head, int which /*0 K, 1 V*/,
                  int n, float* out);
+/* Overwrites positions [0, n) of one layer/kv head's K or V with in[n*head_dim]
+ * (stored as the cache stores: rounded to bf16 when kv_bf16).  Lets a test
+ * continue decoding from a cache it did not build (a long context). */
+int orc_state_set_kv(orc_state* s, int layer, int kv_head, int which, int n, const float* in);
 
 /* Whole sequence without a KV cache (full recompute, causal): logits and
  * hidden of every position, out_logits[n*vocab], out_hidden[n*hidden]. */

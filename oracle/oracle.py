@@ -77,6 +77,7 @@ def _bind(L):
     L.orc_state_create.argtypes = [C.c_void_p, C.c_int]
     L.orc_state_create.restype = C.c_void_p
     L.orc_state_destroy.argtypes = [C.c_void_p]
+    L.orc_state_set_kv.argtypes = [C.c_void_p, C.c_int, C.c_int, C.c_int, C.c_int, _f32p]
     L.orc_decode.argtypes = [C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_void_p,
                              C.c_void_p]
     L.orc_decode.restype = C.c_int
@@ -293,3 +294,11 @@ class OracleState:
         if rc != 0:
             raise ValueError("bad kv query")
         return out.reshape(n, d)
+
+    def set_kv(self, layer: int, kv_head: int, which: int, values) -> None:
+        """Writes positions [0, len(values)) of one cache head (K: which 0, V: 1)."""
+        v = np.ascontiguousarray(np.asarray(values, dtype=np.float32))
+        n = v.shape[0]
+        rc = self._L.orc_state_set_kv(self.h, layer, kv_head, which, n, v.reshape(-1))
+        if rc != 0:
+            raise ValueError("bad kv write")

@@ -277,6 +277,39 @@ def test_cache_holds_rotated_bf16_keys(tiny):
     assert np.array_equal(K[0], torch.from_numpy(k).to(torch.bfloat16).float().numpy())
 
 
+def test_decode_continues_identically_from_a_copied_cache(tiny):
+    # the long-context checks hand the oracle a cache it did not build: a
+    # state whose cache was written through set_kv must decode exactly like
+    # the state that built it
+    cfg, w = tiny
+    m = oracle.OracleModel(cfg, w)
+    toks = synth.make_prompt(12, cfg.vocab, seed=4).numpy()
+    a = m.new_state(16)
+    for p, t in enumerate(toks[:-1]):
+        m.decode(a, int(t), p)
+    b = m.new_state(16)
+    n = len(toks) - 1
+    for l in range(cfg.n_layers):
+        for g in range(cfg.n_kv_heads):
+            for which in (0, 1):
+                b.set_kv(l, g, which, a.kv(l, g, which, n))
+    ra = m.decode(a, int(toks[-1]), n)
+    rb = m.decode(b, int(toks[-1]), n)
+    assert ra[0] == rb[0]
+    assert np.array_equal(ra[1], rb[1]) and np.array_equal(ra[2], rb[2])
+    # and a cache that differs in one key changes the result
+    c = m.new_state(16)
+    for l in range(cfg.n_layers):
+        for g in range(cfg.n_kv_heads):
+            for which in (0, 1):
+                kv = a.kv(l, g, which, n)
+                if (l, g, which) == (1, 0, 0):
+                    kv[3] = -kv[3]
+                c.set_kv(l, g, which, kv)
+    rc = m.decode(c, int(toks[-1]), n)
+    assert not np.array_equal(ra[1], rc[1])
+
+
 def _hf_model(cfg, w):
     transformers = pytest.importorskip("transformers")
     common = dict(hidden_size=cfg.hidden, intermediate_size=cfg.ffn,
