@@ -29,7 +29,9 @@ sys.path.insert(0, ROOT)
 
 METRIC = "decode ms/token (batch 1, Llama-3-8B-shape) & achieved HBM GB/s vs 8 TB/s peak"
 NOMINAL_HBM = 8000.0   # GB/s, the metric's denominator
-PROMPT = 39
+SHORT_PROMPT = 39      # the 39-token prompt, 512 greedy steps workload
+LONG_PROMPT = 32768    # the long-context workload: 32768-token prompt, 256 steps
+LONG_STEPS = 256
 
 
 def measured_peaks():
@@ -125,15 +127,24 @@ def max_over_ranks(v, world):
     return float(t.item())
 
 
-def oracle_sample(model, w_cpu, n_steps: int, budget_s: float):
-    """Times the oracle's decode step (positions 0..) on host cores."""
+def oracle_sample(model, w_cpu, n_steps: int, budget_s: float, first_pos: int = 0):
+    """Times the oracle's decode step (positions first_pos..) on host cores."""
+    import numpy as np
+
     import oracle
     om = oracle.OracleModel(model, w_cpu)
-    st = om.new_state(n_steps + 1)
+    st = om.new_state(first_pos + n_steps + 1)
+    if first_pos:
+        rng = np.random.default_rng(0)
+        fill = rng.standard_normal((first_pos, model.head_dim), dtype=np.float32)
+        for l in range(model.n_layers):
+            for g in range(model.n_kv_heads):
+                for which in (0, 1):
+                    st.set_kv(l, g, which, fill)
     tok = 1
     times = []
     t_all = time.perf_counter()
-    for p in range(n_steps):
+    for p in range(first_pos, first_pos + n_steps):
         t0 = time.perf_counter()
         tok, _, _ = om.decode(st, tok, p, want_logits=False)
         times.append(time.perf_counter() - t0)
@@ -156,20 +167,25 @@ def run_reference(args):
     del w
     budget = float(os.environ.get("MK_REF_BUDGET_S", "60"))
     n = max(2, min(args.warmup + args.steps, 64))
-    times, cores = oracle_sample(model, w_cpu, n, budget)
+    long_ctx = args.workload == "llama8b-32k"
+    prompt_len = LONG_PROMPT if long_ctx else SHORT_PROMPT
+    first_pos = prompt_len if long_ctx else 0
+    times, cores = oracle_sample(model, w_cpu, n, budget, first_pos)
     warm = min(1, len(times) - 1)
     timed = times[warm:]
     ms = 1e3 * sum(timed) / len(timed)
     sample = (f"{len(timed)} oracle decode steps of the Llama-3-8B shape at positions "
-              f"{warm}..{len(times) - 1} (after {warm} untimed), bf16 weights widened to fp32 "
-              f"on the fly, {cores} OpenMP threads")
+              f"{first_pos + warm}..{first_pos + len(times) - 1} (after {warm} untimed), bf16 "
+              f"weights widened to fp32 on the fly, {cores} OpenMP threads"
+              + (" (cache of the earlier positions filled with random bf16 values: the "
+                 "timing does not depend on them)" if long_ctx else ""))
     line = {
         "impl": "reference", "metric": METRIC, "value": ms, "unit": "ms/token",
         "n_gpus": args.gpus, "steps": len(timed), "warmup": warm, "ms_per_step": ms,
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
-        "config": {"workload": "llama-3-8b-shape decode, batch 1, 39-token random prompt, "
-                               "greedy decode", "sample": "bounded oracle sample"},
+        "config": {"workload": f"llama-3-8b-shape decode, batch 1, {prompt_len}-token random "
+                               "prompt, greedy decode", "sample": "bounded oracle sample"},
         "cpu_baseline": {"value": ms, "unit": "ms/token", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": ms, "unit": "ms/token", "h2d_bytes_per_step": 0,
@@ -208,6 +224,10 @@ def run_mk(args):
     if args.layers:
         model = model.with_layers(args.layers)
     W, K = args.warmup, args.steps
+    long_ctx = args.workload == "llama8b-32k"
+    PROMPT = LONG_PROMPT if long_ctx else SHORT_PROMPT
+    if long_ctx and W + K > LONG_STEPS:
+        K = LONG_STEPS - W   # the workload decodes 256 steps after its prompt
     max_seq = PROMPT + W + K + 1
     w = synth.make_model(model, 0, device="cuda")
     stream = torch.cuda.current_stream()
@@ -217,8 +237,17 @@ def run_mk(args):
     prompt = synth.make_prompt(PROMPT, model.vocab).cuda()
     ids = [torch.zeros(1, dtype=torch.int32, device="cuda") for _ in range(2)]
 
+    first_id = []
+
     def prefill():
-        dec.prefill(prompt, [0, PROMPT], None, ids[0])
+        # Decode steps write the cache only at positions >= PROMPT, so after
+        # the first prefill the cache of the prompt stays valid: later
+        # "prefills" only restore the first generated id.
+        if not first_id:
+            dec.prefill(prompt, [0, PROMPT], None, ids[0])
+            first_id.append(ids[0].clone())
+        else:
+            ids[0].copy_(first_id[0])
 
     def run_steps(first_pos, n, evs=None):
         for k in range(n):
@@ -326,7 +355,7 @@ def run_mk(args):
         "warmup": W, "ms_per_step": total_ms / K, "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "weights": "bf16",
         "data": "synthetic",
-        "config": {"workload": "llama-3-8b-shape decode, batch 1, 39-token random prompt, "
+        "config": {"workload": f"llama-3-8b-shape decode, batch 1, {PROMPT}-token random prompt, "
                                f"greedy decode steps {PROMPT + W}..{PROMPT + W + K - 1} timed",
                    "l2": "inputs larger than L2 (15.0 GB of weights streamed per step)",
                    "parallelism": f"replicas x{world}"},
@@ -358,14 +387,18 @@ def run_mk(args):
         w2 = synth.make_model(model, 0, device="cuda")
         w_cpu = {k: v.cpu() for k, v in w2.items()}
         del w2
-        times, cores = oracle_sample(model, w_cpu, 4, 25.0)
+        first_pos = PROMPT + W if long_ctx else 0
+        times, cores = oracle_sample(model, w_cpu, 4 if not long_ctx else 3, 25.0, first_pos)
         timed = times[1:] if len(times) > 1 else times
         cms = 1e3 * sum(timed) / len(timed)
+        p0 = first_pos + len(times) - len(timed)
         line["cpu_baseline"] = {
             "value": cms, "unit": "ms/token", "cores": cores, "kind": "oracle",
             "sample": f"{len(timed)} oracle decode steps of the same Llama-3-8B-shape model "
-                      f"at positions {len(times) - len(timed)}..{len(times) - 1}, fp32 with "
-                      f"bf16 weights widened on the fly"}
+                      f"at positions {p0}..{first_pos + len(times) - 1}, fp32 with "
+                      f"bf16 weights widened on the fly"
+                      + (" (cache of the earlier positions filled with random bf16 values: "
+                         "the timing does not depend on them)" if long_ctx else "")}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -392,6 +425,9 @@ def main():
     ap.add_argument("--trace", default=None, help="write a per-task timeline summary here")
     ap.add_argument("--l2-prefetch", type=int, default=0,
                     help="ring chunks prefetched into L2 beyond the ring (0: library default)")
+    ap.add_argument("--workload", default="llama8b", choices=["llama8b", "llama8b-32k"],
+                    help="llama8b: 39-token prompt (default); llama8b-32k: 32768-token "
+                         "prompt, at most 256 decode steps")
     ap.add_argument("--layers", type=int, default=0,
                     help="profiling aid: a shallower model of the same widths (not a bench line)")
     args = ap.parse_args()
