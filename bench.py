@@ -224,47 +224,61 @@ def run_mk(args):
     if args.layers:
         model = model.with_layers(args.layers)
     W, K = args.warmup, args.steps
-    long_ctx = args.workload == "llama8b-32k"
-    PROMPT = LONG_PROMPT if long_ctx else SHORT_PROMPT
-    if long_ctx and W + K > LONG_STEPS:
-        K = LONG_STEPS - W   # the workload decodes 256 steps after its prompt
-    max_seq = PROMPT + W + K + 1
+    if args.workload == "llama8b-32k":
+        lens = [LONG_PROMPT]
+    elif args.workload == "llama8b-batch8":
+        lens = list(synth.packed_batch_lengths())
+    else:
+        lens = [SHORT_PROMPT]
+    n = len(lens)
+    if args.workload != "llama8b" and W + K > LONG_STEPS:
+        K = LONG_STEPS - W   # these workloads decode 256 steps after their prompts
+    max_seq = max(lens) + W + K + 1
     w = synth.make_model(model, 0, device="cuda")
     stream = torch.cuda.current_stream()
-    dec = binding.Decoder(model, w, max_seq, stream=stream, l2_prefetch=args.l2_prefetch)
+    dec = binding.Decoder(model, w, max_seq, max_batch=n, stream=stream,
+                          l2_prefetch=args.l2_prefetch)
     del w  # mk_create copied and packed the weights
     torch.cuda.empty_cache()
-    prompt = synth.make_prompt(PROMPT, model.vocab).cuda()
-    ids = [torch.zeros(1, dtype=torch.int32, device="cuda") for _ in range(2)]
+    if n == 1:
+        prompt, offs = synth.make_prompt(lens[0], model.vocab), [0, lens[0]]
+    else:
+        prompt, offs = synth.make_packed_prompts(lens, model.vocab)
+        offs = offs.tolist()
+    prompt = prompt.to(torch.int32).cuda()
+    ids = [torch.zeros(n, dtype=torch.int32, device="cuda") for _ in range(2)]
 
     first_id = []
 
     def prefill():
-        # Decode steps write the cache only at positions >= PROMPT, so after
-        # the first prefill the cache of the prompt stays valid: later
-        # "prefills" only restore the first generated id.
+        # Decode steps write the cache only at positions past each prompt, so
+        # after the first prefill the prompts' cache stays valid: later
+        # "prefills" only restore the first generated ids.
         if not first_id:
-            dec.prefill(prompt, [0, PROMPT], None, ids[0])
+            dec.prefill(prompt, offs, None, ids[0])
             first_id.append(ids[0].clone())
         else:
             ids[0].copy_(first_id[0])
 
-    def run_steps(first_pos, n, evs=None):
-        for k in range(n):
-            dec.decode(ids[k % 2], [first_pos + k], None, ids[(k + 1) % 2])
+    def positions(step):
+        return [lens[r] + step for r in range(n)]
+
+    def run_steps(first_step, count, evs=None):
+        for k in range(count):
+            dec.decode(ids[k % 2], positions(first_step + k), None, ids[(k + 1) % 2])
             if evs is not None:
                 evs[k + 1].record(stream)
 
     # ---- device-timed region (megakernel)
     prefill()
-    run_steps(PROMPT, W)
+    run_steps(0, W)
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
     torch.cuda.synchronize()
     barrier(world)
     with ClockSampler(local) as clk:
         torch.cuda.synchronize()
         evs[0].record(stream)
-        run_steps(PROMPT + W, K, evs)
+        run_steps(W, K, evs)
         torch.cuda.synchronize()
     barrier(world)
     rc = dec.status()
@@ -274,8 +288,7 @@ def run_mk(args):
     total_ms = evs[0].elapsed_time(evs[K])
     total_ms = max_over_ranks(total_ms, world)
     value = total_ms / (K * world)
-    positions = list(range(PROMPT + W, PROMPT + W + K))
-    bytes_mean = sum(roofline.step_bytes(model, [p]) for p in positions) / K
+    bytes_mean = sum(roofline.step_bytes(model, positions(W + k)) for k in range(K)) / K
     avg_launch_s = (sum(per_step) / K) * 1e-3
     achieved = bytes_mean / avg_launch_s / 1e9
     peak, peak_src = measured_peaks()
@@ -301,47 +314,47 @@ def run_mk(args):
     for name, mode in (("per_op", binding.MODE_PER_OP), ("per_op_graph", binding.MODE_PER_OP_GRAPH)):
         dec.set_mode(mode)
         prefill()
-        run_steps(PROMPT, min(W, 4))
+        run_steps(0, min(W, 4))
         bev = [torch.cuda.Event(enable_timing=True) for _ in range(nb + 1)]
         torch.cuda.synchronize()
         bev[0].record(stream)
-        run_steps(PROMPT + min(W, 4), nb, bev)
+        run_steps(min(W, 4), nb, bev)
         torch.cuda.synchronize()
         steps_ms = [bev[k].elapsed_time(bev[k + 1]) for k in range(nb)]
-        baselines[name] = {"ms_per_token": statistics.median(steps_ms), "steps": nb,
-                           "launches_per_step": dec_stage_count(dec)}
+        baselines[name] = {"ms_per_token": statistics.median(steps_ms) / n, "steps": nb,
+                           "launches_per_step": n * dec_stage_count(dec)}
     dec.set_mode(binding.MODE_MEGAKERNEL)
     rc = dec.status()
     if rc != 0:
         raise RuntimeError(f"device status {rc}: {dec.last_error()}")
 
-    # ---- end to end through the host entry point (token in, id out, per step)
+    # ---- end to end through the host entry point (tokens in, ids out, per step)
     prefill()
     torch.cuda.synchronize()
-    tok = int(ids[0].item())
+    toks = [int(v) for v in ids[0].tolist()]
     for k in range(W):
-        tok = dec.decode_host([tok], [PROMPT + k])[0]
+        toks = dec.decode_host(toks, positions(k))
     barrier(world)
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     t0.record(stream)
     for k in range(K):
-        tok = dec.decode_host([tok], [PROMPT + W + k])[0]
+        toks = dec.decode_host(toks, positions(W + k))
     t1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(t0.elapsed_time(t1), world) / (K * world)
 
     trace_summary = None
-    if args.trace:
+    if args.trace and n == 1:
         # a few more steps with the per-task timeline on (not part of the timing)
         from persistent_megakernel_03_b200 import trace as mktrace
         plan = binding.Plan(model, max_seq, dec_num_ctas())
         tbuf = torch.zeros((plan.info.n_tasks, 8), dtype=torch.int64, device="cuda")
         prefill()
-        run_steps(PROMPT, W)
+        run_steps(0, W)
         dec.set_trace(tbuf)
-        run_steps(PROMPT + W, 1)
+        run_steps(W, 1)
         torch.cuda.synchronize()
         dec.set_trace(None)
         rows = tbuf.cpu().numpy().astype("uint64").tolist()
@@ -350,16 +363,25 @@ def run_mk(args):
             json.dump(trace_summary, f, indent=1)
 
     clocks = clk.summary()
+    if n == 1:
+        workload = (f"llama-3-8b-shape decode, batch 1, {lens[0]}-token random prompt, "
+                    f"greedy decode steps {lens[0] + W}..{lens[0] + W + K - 1} timed")
+        unit, metric = "ms/token", METRIC
+    else:
+        workload = (f"llama-3-8b-shape decode, {n} requests per step, random prompts of "
+                    f"{lens} tokens packed with offsets, greedy decode steps {W}..{W + K - 1} "
+                    "after each prompt timed; requests run in turn through the one-request "
+                    "graph (weights streamed once per request)")
+        unit, metric = "ms/step", f"decode ms/step ({n} requests, Llama-3-8B-shape)"
     line = {
-        "metric": METRIC, "value": value, "unit": "ms/token", "n_gpus": world, "steps": K,
+        "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": K,
         "warmup": W, "ms_per_step": total_ms / K, "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "weights": "bf16",
         "data": "synthetic",
-        "config": {"workload": f"llama-3-8b-shape decode, batch 1, {PROMPT}-token random prompt, "
-                               f"greedy decode steps {PROMPT + W}..{PROMPT + W + K - 1} timed",
+        "config": {"workload": workload,
                    "l2": "inputs larger than L2 (15.0 GB of weights streamed per step)",
                    "parallelism": f"replicas x{world}"},
-        "tok_per_s": 1e3 / value,
+        "tok_per_s": 1e3 * n / value,
         "step_ms": {"median": statistics.median(per_step),
                     "p10": float(np.percentile(per_step, 10)),
                     "p90": float(np.percentile(per_step, 90))},
@@ -367,14 +389,18 @@ def run_mk(args):
         "read_probe_gbs": probe_gbs, "frac_of_read_probe": achieved / probe_gbs,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": peak_src,
-                     "traffic": load_traffic(),
+                     "traffic": load_traffic() if n == 1 else None,
                      "bytes_per_launch": bytes_mean},
         "baselines": baselines,
         "clocks": clocks,
-        "e2e": {"value": e2e_ms, "unit": "ms/token", "h2d_bytes_per_step": 4,
-                "d2h_bytes_per_step": 4},
-        "gpu_launches": K,
+        "e2e": {"value": e2e_ms, "unit": unit, "h2d_bytes_per_step": 4 * n,
+                "d2h_bytes_per_step": 4 * n},
+        "gpu_launches": K * n,
     }
+    if n > 1:
+        line["roofline"]["bytes_note"] = ("algorithmic bytes: weights once per step plus every "
+                                          "request's KV; the path streams the weights once per "
+                                          "request")
     if args.layers:
         line["config"]["workload"] += f" [profiling case: {args.layers} layers]"
     if args.l2_prefetch:
@@ -387,18 +413,19 @@ def run_mk(args):
         w2 = synth.make_model(model, 0, device="cuda")
         w_cpu = {k: v.cpu() for k, v in w2.items()}
         del w2
-        first_pos = PROMPT + W if long_ctx else 0
-        times, cores = oracle_sample(model, w_cpu, 4 if not long_ctx else 3, 25.0, first_pos)
+        first_pos = lens[0] + W if n > 1 or lens[0] > SHORT_PROMPT else 0
+        times, cores = oracle_sample(model, w_cpu, 4 if first_pos == 0 else 3, 25.0, first_pos)
         timed = times[1:] if len(times) > 1 else times
-        cms = 1e3 * sum(timed) / len(timed)
+        cms = 1e3 * sum(timed) / len(timed) * n
         p0 = first_pos + len(times) - len(timed)
         line["cpu_baseline"] = {
-            "value": cms, "unit": "ms/token", "cores": cores, "kind": "oracle",
+            "value": cms, "unit": unit, "cores": cores, "kind": "oracle",
             "sample": f"{len(timed)} oracle decode steps of the same Llama-3-8B-shape model "
                       f"at positions {p0}..{first_pos + len(times) - 1}, fp32 with "
                       f"bf16 weights widened on the fly"
                       + (" (cache of the earlier positions filled with random bf16 values: "
-                         "the timing does not depend on them)" if long_ctx else "")}
+                         "the timing does not depend on them)" if first_pos else "")
+                      + (f"; x{n}: one such step per request" if n > 1 else "")}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -425,9 +452,11 @@ def main():
     ap.add_argument("--trace", default=None, help="write a per-task timeline summary here")
     ap.add_argument("--l2-prefetch", type=int, default=0,
                     help="ring chunks prefetched into L2 beyond the ring (0: library default)")
-    ap.add_argument("--workload", default="llama8b", choices=["llama8b", "llama8b-32k"],
+    ap.add_argument("--workload", default="llama8b",
+                    choices=["llama8b", "llama8b-32k", "llama8b-batch8"],
                     help="llama8b: 39-token prompt (default); llama8b-32k: 32768-token "
-                         "prompt, at most 256 decode steps")
+                         "prompt; llama8b-batch8: 8 requests with prompts of U[32, 2048] "
+                         "tokens (the last two decode at most 256 steps)")
     ap.add_argument("--layers", type=int, default=0,
                     help="profiling aid: a shallower model of the same widths (not a bench line)")
     args = ap.parse_args()

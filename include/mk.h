@@ -124,7 +124,9 @@ int mk_prefill(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t* offsets_ho
 /* One decode step: request r feeds tokens_dev[r] at position pos_host[r]
  * (positions 0..pos-1 must be in its KV cache), appends its K/V at pos, and
  * writes logits_dev[r*vocab ..] (may be NULL) and next_ids_dev[r] (may be
- * NULL).  n_req <= max_batch. */
+ * NULL).  n_req <= max_batch.  Requests run one after another through the
+ * one-request task graph, each on its own KV-cache slot (one persistent
+ * launch per request); the weights are streamed once per request. */
 int mk_decode_step(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t* pos_host, int n_req,
                    float* logits_dev, int32_t* next_ids_dev);
 
@@ -133,8 +135,9 @@ int mk_decode_step(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t* pos_ho
 int mk_decode_step_host(mk_ctx* ctx, const int32_t* tokens_host, const int32_t* pos_host,
                         int n_req, int32_t* next_ids_host);
 
-/* Copies the final residual stream of the last step (before the final norm),
- * n_req x hidden fp32, to hidden_dev (enqueued on the context's stream). */
+/* Copies the final residual stream of the last step or prefill (before the
+ * final norm), n_req x hidden fp32, to hidden_dev (enqueued on the context's
+ * stream); n_req must not exceed that call's. */
 int mk_copy_hidden(mk_ctx* ctx, float* hidden_dev, int n_req);
 
 /* Device pointer of the bf16 K (which=0) or V (which=1) cache of one request,

@@ -49,6 +49,8 @@ struct mk_ctx {
   cudaGraphExec_t graph = nullptr;
   cudaGraph_t graph_src = nullptr;
   size_t kv_bytes = 0;
+  float* hidden_all = nullptr;   // [max_batch][hidden]: residual streams of a multi-request step
+  int last_n_req = 1;
 };
 
 namespace mk {
@@ -160,8 +162,6 @@ extern "C" int mk_create(const mk_config* cfg, const mk_weights* w, const mk_opt
   *out = nullptr;
   std::string verr = validate_config(*cfg);
   if (!verr.empty()) return fail(nullptr, MK_ERR_INVALID_ARG, verr);
-  if (cfg->max_batch != 1)
-    return fail(nullptr, MK_ERR_UNSUPPORTED, "this build decodes one request per step (max_batch 1)");
   if (!w->embed || !w->layers || !w->final_norm || (!cfg->tied_embeddings && !w->lm_head))
     return fail(nullptr, MK_ERR_INVALID_ARG, "missing weight pointer");
   for (int l = 0; l < cfg->n_layers; ++l) {
@@ -309,6 +309,7 @@ extern "C" int mk_create(const mk_config* cfg, const mk_weights* w, const mk_opt
   if ((rc = dalloc(ctx, &part, (size_t)B * nkv * S * G * attn_part_stride(d) * 4))) return bail(rc);
   if ((rc = dalloc(ctx, &am, (size_t)B * plan.n_lm_slots * 8))) return bail(rc);
   CKC(cudaMemsetAsync(x, 0, (size_t)B * H * 4, st));
+  if ((rc = dalloc(ctx, &ctx->hidden_all, (size_t)B * H * 4))) return bail(rc);
   uint32_t *events = nullptr, *tickets = nullptr, *epoch = nullptr;
   int32_t* status = nullptr;
   if ((rc = dalloc(ctx, &events, (size_t)plan.n_events * 4))) return bail(rc);
@@ -346,7 +347,9 @@ extern "C" int mk_create(const mk_config* cfg, const mk_weights* w, const mk_opt
 
   ModelDev& m = ctx->md;
   m.n_layers = L; m.hidden = H; m.n_q = nq; m.n_kv = nkv; m.head_dim = d; m.ffn = F; m.vocab = V;
-  m.group = G; m.max_seq = cfg->max_seq; m.max_batch = B; m.attn_splits = S;
+  // max_batch here is the graph's request count (one; see mk_decode_step):
+  // the KV cache holds B slots, addressed through StepParams::kv_slot.
+  m.group = G; m.max_seq = cfg->max_seq; m.max_batch = 1; m.attn_splits = S;
   m.qkv_bias = cfg->qkv_bias ? 1 : 0;
   m.rms_eps = cfg->rms_eps;
   m.attn_scale = (float)(1.0 / std::sqrt((double)d));
@@ -388,17 +391,27 @@ extern "C" int mk_decode_step(mk_ctx* ctx, const int32_t* tokens_dev, const int3
   if (rc) return rc;
   if (!tokens_dev) return fail(ctx, MK_ERR_INVALID_ARG, "tokens_dev is null");
   if ((rc = check_step_args(ctx, pos_host, n_req))) return rc;
-  StepParams sp{};
-  sp.n_req = n_req;
+  // The requests run through the one-request graph in turn, each on its own
+  // KV-cache slot; with several requests the residual stream of each is kept
+  // for mk_copy_hidden.  (Every request streams the weights again: this is
+  // the plain small-batch path, not a batched GEMV.)
+  const int H = ctx->cfg.hidden, V = ctx->cfg.vocab;
   for (int r = 0; r < n_req; ++r) {
-    sp.pos[r] = pos_host[r];
-    sp.kv_slot[r] = r;
+    StepParams sp{};
+    sp.n_req = 1;
+    sp.pos[0] = pos_host[r];
+    sp.kv_slot[0] = r;
+    sp.tokens = tokens_dev + r;
+    sp.logits = logits_dev ? logits_dev + (size_t)r * V : nullptr;
+    sp.next_ids = next_ids_dev ? next_ids_dev + r : nullptr;
+    sp.want_logits = logits_dev != nullptr;
+    if ((rc = enqueue_step(ctx, sp))) return rc;
+    if (n_req > 1)
+      CK(cudaMemcpyAsync(ctx->hidden_all + (size_t)r * H, ctx->md.x, (size_t)H * 4,
+                         cudaMemcpyDeviceToDevice, ctx->stream));
   }
-  sp.tokens = tokens_dev;
-  sp.logits = logits_dev;
-  sp.next_ids = next_ids_dev;
-  sp.want_logits = logits_dev != nullptr;
-  return enqueue_step(ctx, sp);
+  ctx->last_n_req = n_req;
+  return MK_OK;
 }
 
 extern "C" int mk_decode_step_host(mk_ctx* ctx, const int32_t* tokens_host, const int32_t* pos_host,
@@ -445,7 +458,11 @@ extern "C" int mk_prefill(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t*
       sp.want_logits = sp.logits != nullptr;
       if ((rc = enqueue_step(ctx, sp))) return rc;
     }
+    if (n_req > 1)
+      CK(cudaMemcpyAsync(ctx->hidden_all + (size_t)r * ctx->cfg.hidden, ctx->md.x,
+                         (size_t)ctx->cfg.hidden * 4, cudaMemcpyDeviceToDevice, ctx->stream));
   }
+  ctx->last_n_req = n_req;
   return MK_OK;
 }
 
@@ -453,7 +470,9 @@ extern "C" int mk_copy_hidden(mk_ctx* ctx, float* hidden_dev, int n_req) {
   int rc = check_ctx(ctx);
   if (rc) return rc;
   if (!hidden_dev || n_req < 1 || n_req > ctx->cfg.max_batch) return fail(ctx, MK_ERR_INVALID_ARG, "bad argument");
-  CK(cudaMemcpyAsync(hidden_dev, ctx->md.x, (size_t)n_req * ctx->cfg.hidden * 4, cudaMemcpyDeviceToDevice,
+  if (n_req > ctx->last_n_req) return fail(ctx, MK_ERR_INVALID_ARG, "n_req exceeds the last step's");
+  const float* src = ctx->last_n_req > 1 ? ctx->hidden_all : ctx->md.x;
+  CK(cudaMemcpyAsync(hidden_dev, src, (size_t)n_req * ctx->cfg.hidden * 4, cudaMemcpyDeviceToDevice,
                      ctx->stream));
   return MK_OK;
 }

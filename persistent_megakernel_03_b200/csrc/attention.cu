@@ -39,6 +39,7 @@ __global__ void __launch_bounds__(kAttnOpWarps * 32)
                        uint8_t* __restrict__ ws, float* __restrict__ out) {
   constexpr int d = DPL * 32, PS = d + 4;
   __shared__ __align__(16) float buf[kAttnOpWarps][G][PS];
+  __shared__ __align__(16) float xb[kAttnOpWarps][kAttnXbStride];
   __shared__ int last;
   unsigned int* ticket = reinterpret_cast<unsigned int*>(ws);
   float* part = reinterpret_cast<float*>(ws + kAttnTicketBytes);
@@ -47,21 +48,31 @@ __global__ void __launch_bounds__(kAttnOpWarps * 32)
   const int k0 = min(n, split * chunk), k1 = min(n, k0 + chunk);
 
   AttnState<DPL, G> st;
+  attn_init<DPL, G>(st, q, d, scale, lane);
+  // four consecutive keys per warp at a time
+  for (int j0 = k0 + 4 * warp; j0 < k1; j0 += 4 * kAttnOpWarps) {
+    const int nj = min(4, k1 - j0);
+    {
+      float kv[4][DPL];
 #pragma unroll
-  for (int h = 0; h < G; ++h) {
+      for (int t = 0; t < 4; ++t) {
+        const int jr = attn_key_row<G>(t, lane);
+        if (jr < nj) load_kv_row_global<DPL>(K + (size_t)(j0 + jr) * d + lane * DPL, kv[t]);
+        else
 #pragma unroll
-    for (int i = 0; i < DPL; ++i) {
-      st.q[h][i] = q[h * d + lane * DPL + i] * scale;
-      st.o[h][i] = 0.f;
+          for (int i = 0; i < DPL; ++i) kv[t][i] = 0.f;
+      }
+      attn_scores4<DPL, G>(st, kv, nj, xb[warp], lane);
     }
-    st.mx[h] = -INFINITY;
-    st.l[h] = 0.f;
-  }
-  for (int j = k0 + warp; j < k1; j += kAttnOpWarps) {
-    float kv[DPL], vv[DPL];
-    load_kv_row_global<DPL>(K + (size_t)j * d + lane * DPL, kv);
-    load_kv_row_global<DPL>(V + (size_t)j * d + lane * DPL, vv);
-    attn_key<DPL, G>(st, kv, vv);
+    float vv[4][DPL];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      if (t < nj) load_kv_row_global<DPL>(V + (size_t)(j0 + t) * d + lane * DPL, vv[t]);
+      else
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) vv[t][i] = 0.f;
+    }
+    attn_update4<DPL, G>(st, vv, xb[warp]);
   }
 #pragma unroll
   for (int h = 0; h < G; ++h) {

@@ -47,6 +47,8 @@ struct __align__(128) Smem {
   int32_t flag;
   int32_t cur_qi;              // queue entry the workers are running (trace)
   unsigned long long lm_best;  // running argmax over this CTA's LM-head tasks
+  int32_t attn_last;           // this attention task merges its KV head's splits
+  __align__(16) float attn_xb[kWorkerWarps][kAttnXbStride];  // attention: per-warp softmax weights
 };
 
 constexpr uint32_t kWorkerBarrier = 1;
@@ -129,6 +131,7 @@ __device__ __forceinline__ unsigned long long argmax_key(float v, int idx) {
 
 struct AttnRange {
   int k0, k1, old_end;  // keys [k0, k1); [k0, old_end) come through the ring
+  int live;             // splits that hold keys at this position
   bool active;
 };
 
@@ -137,12 +140,15 @@ __device__ __forceinline__ AttnRange attn_range(const Task& t, const StepParams&
   AttnRange r{0, 0, 0, false};
   if (t.req >= sp.n_req) return r;
   const int pos = sp.pos[t.req];
-  const int n = pos + 1, S = m.attn_splits;
-  const int chunk = (n + S - 1) / S;
+  const int n = pos + 1;
+  const int live = attn_live_splits(n, m.attn_splits, attn_keys_per_chunk(m.head_dim));
+  if (t.row1 >= live) return r;  // a split with no keys at this position
+  const int chunk = (n + live - 1) / live;
   r.k0 = min(n, t.row1 * chunk);
   r.k1 = min(n, r.k0 + chunk);
   r.old_end = min(r.k1, pos);
   if (r.old_end < r.k0) r.old_end = r.k0;
+  r.live = live;
   r.active = true;
   return r;
 }
@@ -350,58 +356,9 @@ __device__ __forceinline__ void wait_full(Smem& s, uint32_t seq, const ModelDev&
   wait_bounded(s, &s.full[slot], ph, m, kWaitFull);
 }
 
-// Attention output for input columns [8cc, 8cc + 8) of the O projection,
-// merged from the split partials in one pass with a running maximum (online
-// softmax, "Hạt nhân là gì ...": each split's sum and output are rescaled to
-// the common maximum); four splits' loads are in flight at a time.
-struct Cols8 {
-  float2 v[4];
-};
-
-__device__ __forceinline__ Cols8 merge_attn_columns(const ModelDev& m, int cc) {
-  const int d = m.head_dim, G = m.group, S = m.attn_splits, PS = attn_part_stride(d);
-  const int col = cc * 8, h = col / d, i0 = col - h * d;
-  const float* base = m.part + ((size_t)(h / G) * S * G + (h % G)) * PS;
-  const size_t sstride = (size_t)G * PS;
-  float M = -INFINITY, den = 0.f;
-  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  for (int s0 = 0; s0 < S; s0 += 4) {
-    float2 ml[4];
-    float4 oa[4], ob[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      if (s0 + j < S) {
-        const float* ps = base + (size_t)(s0 + j) * sstride;
-        ml[j] = __ldcg(reinterpret_cast<const float2*>(ps + d));
-        oa[j] = __ldcg(reinterpret_cast<const float4*>(ps + i0));
-        ob[j] = __ldcg(reinterpret_cast<const float4*>(ps + i0) + 1);
-      } else {
-        ml[j] = make_float2(-INFINITY, 0.f);
-        oa[j] = ob[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      if (ml[j].y == 0.f) continue;  // empty split
-      const float mn = fmaxf(M, ml[j].x);
-      const float co = __expf(M - mn), cn = __expf(ml[j].x - mn);
-      den = fmaf(den, co, ml[j].y * cn);
-      const float o[8] = {oa[j].x, oa[j].y, oa[j].z, oa[j].w, ob[j].x, ob[j].y, ob[j].z, ob[j].w};
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] = fmaf(acc[e], co, cn * o[e]);
-      M = mn;
-    }
-  }
-  const float inv = 1.0f / den;
-  Cols8 r;
-#pragma unroll
-  for (int e = 0; e < 4; ++e) r.v[e] = make_float2(acc[2 * e] * inv, acc[2 * e + 1] * inv);
-  return r;
-}
-
 // Loads this thread's input columns into xr (fp32, or the bf16 embedding
-// row).  For the O projection the input is the attention output, merged from
-// the split partials (merge_attn_columns).  For operators
+// row).  For the O projection the input is the attention output, which the
+// last attention task of each KV head merged from the split partials.  For operators
 // that start with RMSNorm, xr = x * w_norm and the returned value is this
 // thread's share of sum(x^2); the 1/rms factor is applied to the dot products
 // afterwards (W (x * w * r) = r * W (x * w)), so the first ring chunk is not
@@ -429,7 +386,7 @@ __device__ __forceinline__ float gemv_load_input(const KernelArgs& a, const Task
         src32 = m.x;
       }
       break;
-    case T_OPROJ: break;
+    case T_OPROJ: src32 = m.attn; break;
     case T_GATEUP: src32 = m.x; normw = m.ffn_norm + (size_t)t.layer * m.hidden; break;
     case T_DOWN: src32 = m.act; break;
     default: src32 = m.x; normw = m.final_norm; break;  // LM head
@@ -442,14 +399,7 @@ __device__ __forceinline__ float gemv_load_input(const KernelArgs& a, const Task
 #pragma unroll
     for (int e = 0; e < 4; ++e) x2[c][e] = make_float2(0.f, 0.f);
     if (cc >= C) continue;
-    if (t.kind == T_OPROJ) {
-      // n_q * head_dim <= 8192 (checked at create) keeps CPT <= 2 here.
-      if constexpr (CPT <= 2) {
-        const Cols8 v = merge_attn_columns(m, cc);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) x2[c][e] = v.v[e];
-      }
-    } else if (src16) {
+    if (src16) {
       const uint4 v = __ldg(reinterpret_cast<const uint4*>(src16) + cc);
       x2[c][0] = make_float2(bf_lo(v.x), bf_hi(v.x));
       x2[c][1] = make_float2(bf_lo(v.y), bf_hi(v.y));
@@ -803,16 +753,7 @@ __device__ __forceinline__ void attn_task(const KernelArgs& a, Smem& s, const Ta
     load_kv_row_global<DPL>(m.kcache + off + lane * DPL, kn);
     load_kv_row_global<DPL>(m.vcache + off + lane * DPL, vn);
   }
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-#pragma unroll
-    for (int i = 0; i < DPL; ++i) {
-      st.q[h][i] = __ldcg(m.q + (size_t)(g * G + h) * d + lane * DPL + i) * m.attn_scale;
-      st.o[h][i] = 0.f;
-    }
-    st.mx[h] = -INFINITY;
-    st.l[h] = 0.f;
-  }
+  attn_init<DPL, G>(st, m.q + (size_t)g * G * d, d, m.attn_scale, lane);
   trace_mark(a, s, wtid, 2);
   const int kpc = attn_keys_per_chunk(d);
   for (int k = r.k0; k < r.old_end; k += kpc) {
@@ -822,17 +763,49 @@ __device__ __forceinline__ void attn_task(const KernelArgs& a, Smem& s, const Ta
     if (k == r.k0) trace_mark(a, s, wtid, 3);
     const uint16_t* kb = reinterpret_cast<const uint16_t*>(s.ring[slot]);
     const uint16_t* vb = reinterpret_cast<const uint16_t*>(s.ring[slot] + kSlotBytes / 2);
-    for (int j = warp; j < nk; j += kWorkerWarps) {
-      float kv[DPL], vv[DPL];
-      load_kv_row<DPL>(kb + (size_t)j * d + lane * DPL, kv);
-      load_kv_row<DPL>(vb + (size_t)j * d + lane * DPL, vv);
-      attn_key<DPL, G>(st, kv, vv);
+    // four consecutive keys per warp at a time
+    for (int j0 = 4 * warp; j0 < nk; j0 += 4 * kWorkerWarps) {
+      const int nj = min(4, nk - j0);
+      {
+        float kv[4][DPL];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int jr = attn_key_row<G>(t, lane);
+          if (jr < nj) load_kv_row<DPL>(kb + (size_t)(j0 + jr) * d + lane * DPL, kv[t]);
+          else
+#pragma unroll
+            for (int i = 0; i < DPL; ++i) kv[t][i] = 0.f;
+        }
+        attn_scores4<DPL, G>(st, kv, nj, s.attn_xb[warp], lane);
+      }
+      float vv[4][DPL];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        if (t < nj) load_kv_row<DPL>(vb + (size_t)(j0 + t) * d + lane * DPL, vv[t]);
+        else
+#pragma unroll
+          for (int i = 0; i < DPL; ++i) vv[t][i] = 0.f;
+      }
+      attn_update4<DPL, G>(st, vv, s.attn_xb[warp]);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&s.empty[slot]);
     ++seq;
   }
-  if (has_new) attn_key<DPL, G>(st, kn, vn);
+  if (has_new) {  // the newest key, as a batch of one (warp-uniform branch)
+    float kv[4][DPL], vv[4][DPL];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const bool mine = attn_key_row<G>(t, lane) == 0;
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) {
+        kv[t][i] = mine ? kn[i] : 0.f;
+        vv[t][i] = t == 0 ? vn[i] : 0.f;
+      }
+    }
+    attn_scores4<DPL, G>(st, kv, 1, s.attn_xb[warp], lane);
+    attn_update4<DPL, G>(st, vv, s.attn_xb[warp]);
+  }
   trace_mark(a, s, wtid, 4);
   // Merge the 16 warps' (max, sum, output): warps 8-15 into warps 0-7, then
   // one pass over the 8 remaining states with one output element per thread.
@@ -868,8 +841,30 @@ __device__ __forceinline__ void attn_task(const KernelArgs& a, Smem& s, const Ta
   worker_sync();
   if (warp < kHalf) attn_write_state<DPL, G>(st, buf + warp * sw, PS, d, lane);
   worker_sync();
+  const int live = r.live;
+  if (live == 1) {
+    // the only split: normalise and write the attention output directly
+    float* out = m.attn + ((size_t)b * m.n_q + (size_t)g * G) * d;
+    for (int idx = wtid; idx < G * d; idx += kWorkerThreads) {
+      const int h = idx / d, i = idx - h * d;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kHalf; ++w) M = fmaxf(M, buf[w * sw + h * PS + d]);
+      float num = 0.f, den = 0.f;
+#pragma unroll
+      for (int w = 0; w < kHalf; ++w) {
+        const float mw = buf[w * sw + h * PS + d];
+        if (mw == -INFINITY) continue;
+        const float c = __expf(mw - M);
+        num = fmaf(c, buf[w * sw + h * PS + i], num);
+        den = fmaf(c, buf[w * sw + h * PS + d + 1], den);
+      }
+      out[h * d + i] = num / den;
+    }
+    return;
+  }
   // The split's partial -- output unnormalised at the split's maximum, the
-  // maximum, the sum -- for the O projection to merge.
+  // maximum, the sum.
   float* part = m.part + ((size_t)(b * m.n_kv + g) * S_all + split) * G * PS;
   for (int idx = wtid; idx < G * (d + 2); idx += kWorkerThreads) {
     const int h = idx / (d + 2), i = idx - h * (d + 2);
@@ -888,6 +883,48 @@ __device__ __forceinline__ void attn_task(const KernelArgs& a, Smem& s, const Ta
     }
     // i < d: output dim i; i == d: the maximum; i == d + 1: the sum
     part[h * PS + i] = i == d ? M : val;
+  }
+  // The last of the `live` split tasks of this (request, KV head) to finish
+  // merges them into the attention output (online softmax, "Hạt nhân là gì
+  // ...": each split's sum and output rescaled to the common maximum), then
+  // divides by the sum.  It also puts the ticket back to zero for the next
+  // step, which reaches it only after this step's events.
+  worker_sync();
+  if (wtid == 0) {
+    uint32_t* tk = m.tickets + kAttnTicketBase + ((size_t)t.layer * m.max_batch + b) * m.n_kv + g;
+    const uint32_t old = atom_add_acq_rel_gpu(tk, 1u);  // release: this split's partial
+    const bool last = old == (uint32_t)live - 1u;
+    if (last) *tk = 0u;
+    s.attn_last = last;
+  }
+  worker_sync();
+  if (!s.attn_last) return;
+  const float* pg = m.part + (size_t)(b * m.n_kv + g) * S_all * G * PS;
+  // every split's (maximum, sum) into shared memory, then the common maxima
+  float* ml = buf;  // [live][G][2]
+  for (int idx = wtid; idx < live * G; idx += kWorkerThreads) {
+    const float2 v = __ldcg(reinterpret_cast<const float2*>(pg + (size_t)idx * PS + d));
+    ml[2 * idx] = v.x;
+    ml[2 * idx + 1] = v.y;
+  }
+  worker_sync();
+  float* out = m.attn + ((size_t)b * m.n_q + (size_t)g * G) * d;
+  for (int idx = wtid; idx < G * d; idx += kWorkerThreads) {
+    const int h = idx / d, i = idx - h * d;
+    float M = -INFINITY;
+    for (int sp_ = 0; sp_ < live; ++sp_)
+      if (ml[2 * (sp_ * G + h) + 1] != 0.f) M = fmaxf(M, ml[2 * (sp_ * G + h)]);
+    float num = 0.f, den = 0.f;
+#pragma unroll 4
+    for (int sp_ = 0; sp_ < live; ++sp_) {
+      const float ls = ml[2 * (sp_ * G + h) + 1];
+      const float o = __ldcg(pg + ((size_t)sp_ * G + h) * PS + i);
+      if (ls == 0.f) continue;  // a split without keys
+      const float c = __expf(ml[2 * (sp_ * G + h)] - M);
+      num = fmaf(c, o, num);
+      den = fmaf(c, ls, den);
+    }
+    out[h * d + i] = num / den;
   }
 }
 

@@ -96,7 +96,8 @@ struct ModelDev {
   unsigned long long* am; // [batch][n_lm_slots] packed (value, index) argmax partials
   // sync
   uint32_t* events;
-  uint32_t* tickets;       // [0]: LM-head argmax ticket
+  uint32_t* tickets;       // [0]: LM-head argmax; [kAttnTicketBase + (layer*batch + req)*n_kv + g]:
+                           // attention split-merge tickets
   uint32_t* epoch;         // completed steps
   int32_t* status;         // 0 ok, else an MK_ERR_* code
   int32_t* status_info;    // task index / detail of the first error
@@ -168,12 +169,14 @@ MK_HD int gemv_max_task_rows(int K) {
 // Attention split partial record: o[d], then m and l, padded to 16 bytes.
 MK_HD int attn_part_stride(int d) { return d + 4; }
 
-// Attention splits actually used at a position: about one split per
-// kAttnKeysPerSplit keys, at most the graph's `splits` tasks per KV head.  A
-// short context then has few partials for the O projection to merge.
-constexpr int kAttnKeysPerSplit = 256;
-MK_HD int attn_live_splits(int n_keys, int splits) {
-  int s = (n_keys + kAttnKeysPerSplit - 1) / kAttnKeysPerSplit;
+// First attention merge ticket (ticket 0 is the LM head's).
+constexpr int kAttnTicketBase = 1;
+
+// Attention splits holding keys at a context of n_keys: about one split per
+// ring chunk of keys, at most the graph's `splits` tasks per KV head.  A
+// short context then has one split (no merge) or a few partials to merge.
+MK_HD int attn_live_splits(int n_keys, int splits, int keys_per_split) {
+  int s = (n_keys + keys_per_split - 1) / keys_per_split;
   return s < 1 ? 1 : (s > splits ? splits : s);
 }
 

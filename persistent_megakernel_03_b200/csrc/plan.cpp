@@ -117,12 +117,14 @@ struct Builder {
 
   void build(int splits) {
     const int L = c.n_layers, H = c.hidden, nq = c.n_q_heads, nkv = c.n_kv_heads;
-    const int d = c.head_dim, G = nq / nkv, F = c.ffn, V = c.vocab, B = c.max_batch;
+    // The graph covers one request; a step over several requests runs it once
+    // per request (each with its own KV-cache slot).
+    const int d = c.head_dim, G = nq / nkv, F = c.ffn, V = c.vocab, B = 1;
     const int qkvR = qkv_rows(nq, nkv, d), per_group = (G + 2) * d;
     p.event_count.assign(ev.count(), 0);
     p.n_events = ev.count();
     p.attn_splits = splits;
-    p.n_tickets = 1;
+    p.n_tickets = kAttnTicketBase + L * B * nkv;
     p.lm_ticket = 0;
     p.n_stages = 5 * L + 1;
     for (int l = 0; l < L; ++l) {
@@ -236,7 +238,7 @@ std::string build_plan(const mk_config& c, int num_ctas, int attn_splits, Plan* 
   std::string err = validate_config(c);
   if (!err.empty()) return err;
   if (num_ctas <= 0) return "num_ctas must be positive";
-  int per_batch = std::max(1, num_ctas / (c.max_batch * c.n_kv_heads));
+  int per_batch = std::max(1, num_ctas / c.n_kv_heads);
   int S = attn_splits > 0 ? attn_splits
                           : std::max(1, std::min(per_batch, (c.max_seq + 63) / 64));
   if (S > 4096) return "attn_splits too large";

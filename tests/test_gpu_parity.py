@@ -71,6 +71,25 @@ def test_tiny_attention_split_counts(tiny, cuda_ok, splits):
     assert_within(compare(tr, gl, gh, gi))
 
 
+@pytest.fixture(scope="module")
+def tiny_long():
+    # 300-token prompt: the context spans several ring chunks of keys, so the
+    # attention runs on several splits whose partials are merged
+    cfg = synth.TINY
+    w = synth.make_model(cfg, 5)
+    prompt = synth.make_prompt(300, cfg.vocab, seed=6).tolist()
+    tr, _, _ = oracle_trace(cfg, w, prompt, 6, 320)
+    return cfg, w, tr
+
+
+@pytest.mark.parametrize("splits", [1, 2, 3, 7])
+def test_tiny_merged_splits(tiny_long, cuda_ok, splits):
+    cfg, w, tr = tiny_long
+    dec = binding.Decoder(cfg, {k: v.cuda() for k, v in w.items()}, 320, attn_splits=splits)
+    gl, gh, gi = run_gpu(dec, cfg, tr)
+    assert_within(compare(tr, gl, gh, gi))
+
+
 @pytest.mark.parametrize("ctas", [1, 5, 64])
 def test_tiny_fewer_ctas(tiny, cuda_ok, ctas):
     cfg, w, tr = tiny
