@@ -249,13 +249,20 @@ def run_mk(args):
     ids = [torch.zeros(n, dtype=torch.int32, device="cuda") for _ in range(2)]
 
     first_id = []
+    prefill_ms = []
 
     def prefill():
         # Decode steps write the cache only at positions past each prompt, so
         # after the first prefill the prompts' cache stays valid: later
         # "prefills" only restore the first generated ids.
         if not first_id:
+            pe0 = torch.cuda.Event(enable_timing=True)
+            pe1 = torch.cuda.Event(enable_timing=True)
+            pe0.record(stream)
             dec.prefill(prompt, offs, None, ids[0])
+            pe1.record(stream)
+            torch.cuda.synchronize()
+            prefill_ms.append(pe0.elapsed_time(pe1))
             first_id.append(ids[0].clone())
         else:
             ids[0].copy_(first_id[0])
@@ -392,6 +399,8 @@ def run_mk(args):
                      "traffic": load_traffic() if n == 1 else None,
                      "bytes_per_launch": bytes_mean},
         "baselines": baselines,
+        "prefill": {"ms": prefill_ms[0], "positions": int(sum(lens)),
+                    "path": "tensor-core GEMMs for all but each prompt's last position"},
         "clocks": clocks,
         "e2e": {"value": e2e_ms, "unit": unit, "h2d_bytes_per_step": 4 * n,
                 "d2h_bytes_per_step": 4 * n},

@@ -100,6 +100,9 @@ typedef struct {
   int l2_prefetch;   /* when a CTA's next task must wait for its event, the number
                         of 32 KB weight chunks past its shared-memory ring it
                         prefetches into L2 meanwhile; 0: default (off), < 0: off */
+  int prefill_steps; /* 1: mk_prefill runs every prompt position as a decode step;
+                        0: default, the tensor-core prefill (when every contraction
+                        length is a multiple of 64) */
 } mk_options;
 
 typedef struct mk_ctx mk_ctx;
@@ -117,7 +120,13 @@ int mk_create(const mk_config* cfg, const mk_weights* w, const mk_options* opt, 
  * ("LLM高速化勉強会資料" slides 14-16): request r owns tokens
  * [offsets_host[r], offsets_host[r+1]) of tokens_dev; 1 <= len <= max_seq.
  * Writes the last position's logits (n_req x vocab fp32, may be NULL) and
- * greedy next ids (n_req int32, may be NULL). */
+ * greedy next ids (n_req int32, may be NULL).  By default positions 0..len-2
+ * run as whole-sequence operators with the weight contractions on the tensor
+ * cores (tcgen05, bf16 weights times the fp32 activations split into two bf16
+ * parts, fp32 accumulation) and causal attention over the cache, in blocks of
+ * 2048 positions; the last position runs as a decode step.  This path
+ * allocates its scratch (~0.4 GB for the Llama-3-8B shape) at the first call
+ * and synchronises the stream before returning. */
 int mk_prefill(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t* offsets_host, int n_req,
                float* last_logits_dev, int32_t* next_ids_dev);
 

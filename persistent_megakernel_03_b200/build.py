@@ -9,8 +9,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libmk.so")
-SOURCES = ["plan.cpp", "kernel.cu", "api.cu", "attention.cu"]
-HEADERS = ["mk_internal.h", "plan.h", "ptx.cuh", "attn_math.cuh"]
+SOURCES = ["plan.cpp", "kernel.cu", "api.cu", "attention.cu", "prefill.cu"]
+HEADERS = ["mk_internal.h", "plan.h", "ptx.cuh", "attn_math.cuh", "tc.cuh", "prefill.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -1,6 +1,7 @@
 // api.cu -- the C-ABI of libmk (declared in include/mk.h).
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -10,6 +11,7 @@
 #include "../../include/mk.h"
 #include "mk_internal.h"
 #include "plan.h"
+#include "prefill.h"
 
 namespace mk {
 size_t step_kernel_smem_bytes();
@@ -51,6 +53,8 @@ struct mk_ctx {
   size_t kv_bytes = 0;
   float* hidden_all = nullptr;   // [max_batch][hidden]: residual streams of a multi-request step
   int last_n_req = 1;
+  PrefillWeights pw;             // packed weight pointers for the tensor-core prefill
+  PrefillScratch ps;             // its scratch (allocated at the first prefill)
 };
 
 namespace mk {
@@ -257,6 +261,8 @@ extern "C" int mk_create(const mk_config* cfg, const mk_weights* w, const mk_opt
     CKC(launch_pack_gateup(pg, (const uint16_t*)Lw.w_gate, (const uint16_t*)Lw.w_up, H, F, st));
     CKC(cudaMemcpyAsync(pd, Lw.w_down, sz_dn, cudaMemcpyDeviceToDevice, st));
     w_qkv[l] = pq; w_o[l] = po; w_gu[l] = pg; w_dn[l] = pd;
+    ctx->pw.qkv.push_back(pq); ctx->pw.o.push_back(po);
+    ctx->pw.gu.push_back(pg); ctx->pw.dn.push_back(pd);
   }
   uint16_t* emb = (uint16_t*)take(sz_emb);
   CKC(cudaMemcpyAsync(emb, w->embed, sz_emb, cudaMemcpyDeviceToDevice, st));
@@ -441,12 +447,27 @@ extern "C" int mk_prefill(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t*
     if (offsets_host[r] < 0 || len < 1 || len > ctx->cfg.max_seq)
       return fail(ctx, MK_ERR_POS_RANGE, "prompt length outside [1, max_seq]");
   }
-  // Each prompt position runs through the same step as decoding: position t
-  // appends its K/V and attends over 0..t.  Only the last position's logits
-  // and id are kept.
+  // Tensor-core path: every position but each prompt's last through the
+  // whole-sequence operators; the last position then runs as a decode step
+  // (its logits and greedy id).  Otherwise every position is a decode step:
+  // position t appends its K/V and attends over 0..t.
+  const bool gemm_path = ctx->opt.prefill_steps <= 0 && prefill_gemm_supported(ctx->md);
+  if (gemm_path) {
+    if (!ctx->ps.max_tokens) {
+      const int cap = std::min(kPrefillBlockTokens, ctx->cfg.max_seq * ctx->cfg.max_batch);
+      const std::string e = prefill_alloc(ctx->md, std::max(cap, 1), &ctx->ps, &ctx->allocs);
+      if (!e.empty()) return fail(ctx, MK_ERR_CUDA, e);
+    }
+    const std::string e = prefill_run(ctx->md, ctx->pw, ctx->ps, ctx->stream, tokens_dev,
+                                      offsets_host, n_req);
+    if (!e.empty()) {
+      ctx->poisoned = true;
+      return fail(ctx, MK_ERR_CUDA, e);
+    }
+  }
   for (int r = 0; r < n_req; ++r) {
     const int len = offsets_host[r + 1] - offsets_host[r];
-    for (int t = 0; t < len; ++t) {
+    for (int t = gemm_path ? len - 1 : 0; t < len; ++t) {
       StepParams sp{};
       sp.n_req = 1;
       sp.pos[0] = t;

@@ -6,7 +6,9 @@ Llama-3-8B shape's widths cut to two layers:
 
 * layer 0's cached K and V at a position depend on that position's token
   alone (RMSNorm, the K/V projections, RoPE at that position), so the oracle
-  computes sampled rows directly from the embedding;
+  computes sampled rows directly from the embedding (the prompt runs through
+  the tensor-core prefill, whose sums round differently: entries agree to a
+  bf16 step of the row's scale);
 * the oracle takes the GPU's cache for positions [0, P-1) as its own state,
   recomputes the last prompt position and decodes teacher-forced steps after
   it; logits, residual stream and greedy ids must meet the usual acceptance
@@ -72,9 +74,14 @@ def test_layer0_cache_rows_at_sampled_positions(long_ctx):
                     v = oracle.rope(v, p, cfg.rope_theta)
                 want = _bf16(v)
                 diff = np.abs(got[p] - want)
-                step = np.abs(want) * 2.0 ** -7 + 1e-30
-                assert np.mean(diff == 0) > 0.95, (g, which, p)
-                assert np.all(diff <= step * 1.01 + 1e-6), (g, which, p)
+                # one bf16 step of the value, floored at the row's rms: the
+                # prefill's tensor-core sums round differently from the
+                # oracle's sequential fp32 sums, which moves entries near a
+                # rounding boundary (and tiny entries) by a step
+                rms = float(np.sqrt(np.mean(want * want)))
+                step = np.maximum(np.abs(want), rms) * 2.0 ** -7
+                assert np.mean(diff == 0) > 0.9, (g, which, p)
+                assert np.all(diff <= step * 1.01), (g, which, p)
 
 
 def test_decode_after_long_prompt_matches_oracle(long_ctx):
