@@ -100,6 +100,8 @@ typedef struct {
   int l2_prefetch;   /* when a CTA's next task must wait for its event, the number
                         of 32 KB weight chunks past its shared-memory ring it
                         prefetches into L2 meanwhile; 0: default (off), < 0: off */
+  int batch_sequential; /* 1: a step of several requests runs them one after another
+                           through the megakernel; 0: default, one batched step */
   int prefill_steps; /* 1: mk_prefill runs every prompt position as a decode step;
                         0: default, the tensor-core prefill (when every contraction
                         length is a multiple of 64) */
@@ -133,9 +135,14 @@ int mk_prefill(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t* offsets_ho
 /* One decode step: request r feeds tokens_dev[r] at position pos_host[r]
  * (positions 0..pos-1 must be in its KV cache), appends its K/V at pos, and
  * writes logits_dev[r*vocab ..] (may be NULL) and next_ids_dev[r] (may be
- * NULL).  n_req <= max_batch.  Requests run one after another through the
- * one-request task graph, each on its own KV-cache slot (one persistent
- * launch per request); the weights are streamed once per request. */
+ * NULL).  n_req <= max_batch.  One request: one launch of the persistent
+ * megakernel.  Several requests (megakernel mode, contraction lengths
+ * multiples of 64): one batched step -- every weight matrix streamed once
+ * through tcgen05 GEMMs over the requests' columns, split-KV attention per
+ * request and KV head, greedy argmax per request -- replayed from a CUDA
+ * graph captured at the first step of that request count.  Otherwise (or
+ * with batch_sequential) the requests run one after another through the
+ * megakernel, each on its own KV-cache slot. */
 int mk_decode_step(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t* pos_host, int n_req,
                    float* logits_dev, int32_t* next_ids_dev);
 

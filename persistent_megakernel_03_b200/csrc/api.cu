@@ -55,6 +55,8 @@ struct mk_ctx {
   int last_n_req = 1;
   PrefillWeights pw;             // packed weight pointers for the tensor-core prefill
   PrefillScratch ps;             // its scratch (allocated at the first prefill)
+  BatchScratch bs;               // batched decode step (allocated at its first use)
+  bool last_batched = false;     // the last step ran the batched path (hidden in bs.x)
 };
 
 namespace mk {
@@ -90,6 +92,10 @@ static void release(mk_ctx* ctx) {
   if (!ctx) return;
   if (ctx->graph) cudaGraphExecDestroy(ctx->graph);
   if (ctx->graph_src) cudaGraphDestroy(ctx->graph_src);
+  for (int n = 0; n <= kMaxBatch; ++n) {
+    if (ctx->bs.graph[n]) cudaGraphExecDestroy(ctx->bs.graph[n]);
+    if (ctx->bs.graph_src[n]) cudaGraphDestroy(ctx->bs.graph_src[n]);
+  }
   for (void* p : ctx->allocs) cudaFree(p);
   if (ctx->h_pinned) cudaFreeHost(ctx->h_pinned);
   ctx->allocs.clear();
@@ -397,11 +403,40 @@ extern "C" int mk_decode_step(mk_ctx* ctx, const int32_t* tokens_dev, const int3
   if (rc) return rc;
   if (!tokens_dev) return fail(ctx, MK_ERR_INVALID_ARG, "tokens_dev is null");
   if ((rc = check_step_args(ctx, pos_host, n_req))) return rc;
-  // The requests run through the one-request graph in turn, each on its own
-  // KV-cache slot; with several requests the residual stream of each is kept
-  // for mk_copy_hidden.  (Every request streams the weights again: this is
-  // the plain small-batch path, not a batched GEMV.)
   const int H = ctx->cfg.hidden, V = ctx->cfg.vocab;
+  // Several requests: by default one batched step that streams every weight
+  // matrix once (tensor-core GEMMs over the requests' columns).
+  if (n_req > 1 && ctx->mode == MK_MODE_MEGAKERNEL && ctx->opt.batch_sequential <= 0 &&
+      prefill_gemm_supported(ctx->md)) {
+    if (!ctx->bs.params) {
+      const std::string e = batch_alloc(ctx->md, ctx->plan.num_ctas, &ctx->bs, &ctx->allocs);
+      if (!e.empty()) return fail(ctx, MK_ERR_CUDA, e);
+    }
+    BatchParams hp{};
+    hp.n = n_req;
+    for (int r = 0; r < n_req; ++r) {
+      hp.pos[r] = pos_host[r];
+      hp.slot[r] = r;
+      hp.src[r] = r;
+    }
+    CK(cudaMemcpyAsync(ctx->bs.tokens, tokens_dev, (size_t)n_req * 4, cudaMemcpyDeviceToDevice,
+                       ctx->stream));
+    CK(cudaMemcpyAsync(ctx->bs.params, &hp, sizeof hp, cudaMemcpyHostToDevice, ctx->stream));
+    const std::string e = batch_step(ctx->md, ctx->pw, ctx->bs, n_req, ctx->plan.num_ctas, ctx->stream);
+    if (!e.empty()) return fail(ctx, MK_ERR_CUDA, e);
+    if (logits_dev)
+      CK(cudaMemcpyAsync(logits_dev, ctx->bs.logits, (size_t)n_req * V * 4, cudaMemcpyDeviceToDevice,
+                         ctx->stream));
+    if (next_ids_dev)
+      CK(cudaMemcpyAsync(next_ids_dev, ctx->bs.ids, (size_t)n_req * 4, cudaMemcpyDeviceToDevice,
+                         ctx->stream));
+    ctx->last_n_req = n_req;
+    ctx->last_batched = true;
+    return MK_OK;
+  }
+  // Otherwise the requests run through the one-request graph in turn, each on
+  // its own KV-cache slot (every request streams the weights again); with
+  // several requests the residual stream of each is kept for mk_copy_hidden.
   for (int r = 0; r < n_req; ++r) {
     StepParams sp{};
     sp.n_req = 1;
@@ -417,6 +452,7 @@ extern "C" int mk_decode_step(mk_ctx* ctx, const int32_t* tokens_dev, const int3
                          cudaMemcpyDeviceToDevice, ctx->stream));
   }
   ctx->last_n_req = n_req;
+  ctx->last_batched = false;
   return MK_OK;
 }
 
@@ -484,6 +520,7 @@ extern "C" int mk_prefill(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t*
                          (size_t)ctx->cfg.hidden * 4, cudaMemcpyDeviceToDevice, ctx->stream));
   }
   ctx->last_n_req = n_req;
+  ctx->last_batched = false;
   return MK_OK;
 }
 
@@ -492,7 +529,7 @@ extern "C" int mk_copy_hidden(mk_ctx* ctx, float* hidden_dev, int n_req) {
   if (rc) return rc;
   if (!hidden_dev || n_req < 1 || n_req > ctx->cfg.max_batch) return fail(ctx, MK_ERR_INVALID_ARG, "bad argument");
   if (n_req > ctx->last_n_req) return fail(ctx, MK_ERR_INVALID_ARG, "n_req exceeds the last step's");
-  const float* src = ctx->last_n_req > 1 ? ctx->hidden_all : ctx->md.x;
+  const float* src = ctx->last_batched ? ctx->bs.x : (ctx->last_n_req > 1 ? ctx->hidden_all : ctx->md.x);
   CK(cudaMemcpyAsync(hidden_dev, src, (size_t)n_req * ctx->cfg.hidden * 4, cudaMemcpyDeviceToDevice,
                      ctx->stream));
   return MK_OK;
@@ -553,6 +590,13 @@ extern "C" int mk_status(mk_ctx* ctx) {
                        : st[0] == MK_ERR_TOKEN_RANGE ? "token id out of range: "
                                                      : "device error, detail ";
     return fail(ctx, st[0], std::string(what) + std::to_string(st[1]));
+  }
+  if (ctx->bs.err) {  // the batched step's GEMM pipeline waits
+    int32_t be = 0;
+    if (cudaMemcpy(&be, ctx->bs.err, 4, cudaMemcpyDeviceToHost) == cudaSuccess && be) {
+      ctx->poisoned = true;
+      return fail(ctx, MK_ERR_TIMEOUT, "batched step: a GEMM pipeline wait timed out");
+    }
   }
   return MK_OK;
 }

@@ -34,28 +34,37 @@ namespace mk {
 namespace {
 
 // ------------------------------------------------------------------ GEMM
-// One CTA per 128 weight rows x 128 tokens.  Warp 0 lane 0 issues the TMA
-// loads of a 4-stage ring (W tile 128 x 64, xh and xl tiles 128 x 64, all
-// 128-byte swizzled), warp 1 lane 0 issues the MMAs into a 128 x 128 fp32
-// accumulator in tensor memory and frees each stage with tcgen05.commit, and
-// all four warps read the accumulator back (warp w owns TMEM lanes 32w..32w+31,
-// i.e. weight rows) and store Y[token][row].
-constexpr int kGM = 128, kGN = 128, kGK = 64, kGStages = 4;
-constexpr int kGTile = 128 * kGK * 2;  // 16 KB, every operand tile
-constexpr uint32_t kGStageBytes = 3 * kGTile;
+// Y[t][r] = sum_k W[r][k] * (xh[t][k] + xl[t][k]) for 128 weight rows and BN
+// tokens per CTA, K blocks [z*nk/Z, (z+1)*nk/Z) of a Z-way split (gridDim.z;
+// split z writes its partial sums at Y + z * part_stride).  Warp 0 lane 0
+// issues the TMA loads of a STAGES-deep ring (W tile 128 x 64, xh and xl
+// tiles BN x 64, all 128-byte swizzled), warp 1 lane 0 issues the MMAs into a
+// 128 x BN fp32 accumulator in tensor memory and frees each stage with
+// tcgen05.commit, and all four warps read the accumulator back (warp w owns
+// TMEM lanes 32w..32w+31, i.e. weight rows) and store Y[token][row].
+// BN = 128 serves the prompt (many tokens); BN = 16 serves a decode step of
+// up to 8 requests, where the weights dominate and the deeper ring keeps more
+// of them in flight.
+constexpr int kGM = 128, kGK = 64;
+constexpr int kGTileA = kGM * kGK * 2;  // 16 KB
 constexpr uint64_t kGWaitNs = 2000000000ull;  // 2 s: far beyond any legal wait
 
+template <int BN, int STAGES>
 struct __align__(1024) GemmSmem {
-  uint8_t a[kGStages][kGTile];
-  uint8_t bh[kGStages][kGTile];
-  uint8_t bl[kGStages][kGTile];
-  uint64_t full[kGStages];
-  uint64_t empty[kGStages];
+  static constexpr int kTileB = BN * kGK * 2;
+  static constexpr uint32_t kStageBytes = kGTileA + 2 * kTileB;
+  static constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;
+  uint8_t a[STAGES][kGTileA];
+  uint8_t bh[STAGES][kTileB];
+  uint8_t bl[STAGES][kTileB];
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
   uint64_t done;
   uint32_t tmem;
   int32_t failed;
 };
-constexpr size_t kGemmSmemBytes = sizeof(GemmSmem) + 1024;
+template <int BN, int STAGES>
+constexpr size_t gemm_smem_bytes() { return sizeof(GemmSmem<BN, STAGES>) + 1024; }
 
 // Bounded wait on an mbarrier phase; false after kGWaitNs (the caller records
 // the failure and stops issuing work).
@@ -67,21 +76,27 @@ __device__ __forceinline__ bool gemm_wait(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
+template <int BN, int STAGES>
 __global__ void __launch_bounds__(128, 1)
     gemm_wx_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_xh,
                    const __grid_constant__ CUtensorMap tm_xl, int n_rows, int n_tok, int K,
-                   float* __restrict__ Y, int ldy, const uint16_t* __restrict__ bias,
-                   int32_t* __restrict__ err) {
+                   float* __restrict__ Y, int ldy, size_t part_stride,
+                   const uint16_t* __restrict__ bias, int32_t* __restrict__ err,
+                   const float* __restrict__ tok_ss, int norm_len, float norm_eps) {
+  using S = GemmSmem<BN, STAGES>;
   // The swizzled tiles must start on 1024-byte boundaries of the shared
   // window: round the dynamic base up (the launch adds 1 KB of slack).
   extern __shared__ __align__(16) uint8_t gsm_raw[];
   const uint32_t base = smem_u32(gsm_raw);
-  GemmSmem& s = *reinterpret_cast<GemmSmem*>(gsm_raw + (((base + 1023u) & ~1023u) - base));
+  S& s = *reinterpret_cast<S*>(gsm_raw + (((base + 1023u) & ~1023u) - base));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * kGM, n0 = blockIdx.y * kGN;
-  const int nk = K / kGK;
+  const int m0 = blockIdx.x * kGM, n0 = blockIdx.y * BN;
+  const int nk_all = K / kGK, Z = gridDim.z, z = blockIdx.z;
+  const int kb0 = (int)((long long)nk_all * z / Z), kb1 = (int)((long long)nk_all * (z + 1) / Z);
+  const int nk = kb1 - kb0;
+  Y += (size_t)z * part_stride;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kGStages; ++i) {
+    for (int i = 0; i < STAGES; ++i) {
       mbar_init(&s.full[i], 1);
       mbar_init(&s.empty[i], 1);
     }
@@ -90,37 +105,36 @@ __global__ void __launch_bounds__(128, 1)
     fence_barrier_init();
   }
   if (warp == 0) {
-    tmem_alloc(&s.tmem, kGN);
+    tmem_alloc(&s.tmem, S::kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = s.tmem;
-  // Loads issued and MMAs committed, for the teardown after a failed wait.
-  int issued = 0;
   if (warp == 0 && lane == 0) {
-    for (int kb = 0; kb < nk; ++kb) {
-      const int st = kb % kGStages;
-      if (kb >= kGStages && !gemm_wait(&s.empty[st], ((kb / kGStages) - 1) & 1)) {
+    int issued = 0;
+    for (int i = 0; i < nk; ++i) {
+      const int st = i % STAGES;
+      if (i >= STAGES && !gemm_wait(&s.empty[st], ((i / STAGES) - 1) & 1)) {
         s.failed = 1;
         break;
       }
-      mbar_arrive_expect_tx(&s.full[st], kGStageBytes);
-      tma_load_2d(s.a[st], &tm_w, kb * kGK, m0, &s.full[st]);
-      tma_load_2d(s.bh[st], &tm_xh, kb * kGK, n0, &s.full[st]);
-      tma_load_2d(s.bl[st], &tm_xl, kb * kGK, n0, &s.full[st]);
-      issued = kb + 1;
+      const int kc = (kb0 + i) * kGK;
+      mbar_arrive_expect_tx(&s.full[st], S::kStageBytes);
+      tma_load_2d(s.a[st], &tm_w, kc, m0, &s.full[st]);
+      tma_load_2d(s.bh[st], &tm_xh, kc, n0, &s.full[st]);
+      tma_load_2d(s.bl[st], &tm_xl, kc, n0, &s.full[st]);
+      issued = i + 1;
     }
     // every load must land before this CTA may exit
-    for (int kb = (issued > kGStages ? issued - kGStages : 0); kb < issued; ++kb)
-      gemm_wait(&s.full[kb % kGStages], (kb / kGStages) & 1);
+    for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
+      gemm_wait(&s.full[i % STAGES], (i / STAGES) & 1);
   } else if (warp == 1 && lane == 0) {
-    constexpr uint32_t idesc = mma_idesc_bf16_f32(kGM, kGN);
-    int kb = 0;
-    for (; kb < nk; ++kb) {
-      const int st = kb % kGStages;
-      if (!gemm_wait(&s.full[st], (kb / kGStages) & 1)) {
+    constexpr uint32_t idesc = mma_idesc_bf16_f32(kGM, BN);
+    for (int i = 0; i < nk; ++i) {
+      const int st = i % STAGES;
+      if (!gemm_wait(&s.full[st], (i / STAGES) & 1)) {
         s.failed = 1;
         break;
       }
@@ -131,7 +145,7 @@ __global__ void __launch_bounds__(128, 1)
 #pragma unroll
       for (int k = 0; k < kGK / 16; ++k) {
         // +2 in the address field = 32 bytes = 16 bf16 along K
-        tc_mma_f16(tmem, da + 2 * k, dh + 2 * k, idesc, (kb | k) != 0);
+        tc_mma_f16(tmem, da + 2 * k, dh + 2 * k, idesc, (i | k) != 0);
         tc_mma_f16(tmem, da + 2 * k, dl + 2 * k, idesc, 1u);
       }
       tc_commit(&s.empty[st]);
@@ -143,27 +157,31 @@ __global__ void __launch_bounds__(128, 1)
   const bool ok = gemm_wait(&s.done, 0);
   tc_fence_after_sync();
   __syncthreads();
-  if (ok && !s.failed) {
+  if (ok && !s.failed && nk > 0) {
     const int row = m0 + warp * 32 + lane;
     const float b = (bias && row < n_rows) ? __uint_as_float((uint32_t)bias[row] << 16) : 0.f;
 #pragma unroll 1
-    for (int c0 = 0; c0 < kGN; c0 += 16) {
+    for (int c0 = 0; c0 < BN; c0 += 16) {
       float v[16];
       tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
       if (row < n_rows) {
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const int tok = n0 + c0 + j;
-          if (tok < n_tok) Y[(size_t)tok * ldy + row] = v[j] + b;
+          if (tok < n_tok) {
+            // deferred RMSNorm: the input was x * w, its scale 1/rms applies here
+            const float sc = tok_ss ? 1.0f / sqrtf(tok_ss[tok] / (float)norm_len + norm_eps) : 1.0f;
+            Y[(size_t)tok * ldy + row] = v[j] * sc + b;
+          }
         }
       }
     }
-  } else if (threadIdx.x == 0) {
+  } else if (threadIdx.x == 0 && (!ok || s.failed)) {
     atomicExch(err, 1);
   }
   tc_fence_before_sync();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, kGN);
+  if (warp == 0) tmem_dealloc(tmem, S::kTmemCols);
 }
 
 // ------------------------------------------------------- small operators
@@ -216,16 +234,25 @@ __global__ void rmsnorm_split_kernel(const float* __restrict__ x, const uint16_t
 
 // RoPE on the packed q/k rows of each token, q to qout, K/V (bf16) into the
 // cache at the token's (slot, position).  Mirrors the decode step's epilogue.
-__global__ void rope_kv_kernel(const float* __restrict__ y, int ldy, const int32_t* __restrict__ slot,
+__global__ void rope_kv_kernel(const float* __restrict__ y, int ldy, int nparts, size_t pstride,
+                               const uint16_t* __restrict__ bias, const int32_t* __restrict__ slot,
                                const int32_t* __restrict__ pos, ModelDev m, int layer,
                                float* __restrict__ qout) {
   const int t = blockIdx.x;
   const int d = m.head_dim, G = m.group, half = d >> 1;
   const int npairs = qkv_rows(m.n_q, m.n_kv, d) >> 1;
   const int p = pos[t], sl = slot[t];
-  for (int pi = threadIdx.x; pi < npairs; pi += blockDim.x) {
+  for (int pi = blockIdx.y * blockDim.x + threadIdx.x; pi < npairs; pi += blockDim.x * gridDim.y) {
     const int r = 2 * pi;
-    float y0 = y[(size_t)t * ldy + r], y1 = y[(size_t)t * ldy + r + 1];
+    float y0 = 0.f, y1 = 0.f;
+    for (int z = 0; z < nparts; ++z) {  // split-K partial sums, in order
+      y0 += y[z * pstride + (size_t)t * ldy + r];
+      y1 += y[z * pstride + (size_t)t * ldy + r + 1];
+    }
+    if (bias) {
+      y0 += bf16_val(bias[r]);
+      y1 += bf16_val(bias[r + 1]);
+    }
     int which, head, dim0, w1, h1, dim1;
     qkv_source(r, G, d, &which, &head, &dim0);
     qkv_source(r + 1, G, d, &w1, &h1, &dim1);
@@ -328,19 +355,341 @@ __global__ void __launch_bounds__(kPAWarps * 32, 1)
   }
 }
 
-// x[t] += y[t]
-__global__ void residual_kernel(float* __restrict__ x, const float* __restrict__ y, int H, int ldy) {
+// x[t] += y[t] (the sum of nparts split-K partials, in order)
+__global__ void residual_kernel(float* __restrict__ x, const float* __restrict__ y, int H, int ldy,
+                                int nparts, size_t pstride) {
   const int t = blockIdx.x;
-  for (int i = threadIdx.x; i < H; i += blockDim.x) x[(size_t)t * H + i] += y[(size_t)t * ldy + i];
+  for (int i = threadIdx.x; i < H; i += blockDim.x) {
+    float v = 0.f;
+    for (int z = 0; z < nparts; ++z) v += y[z * pstride + (size_t)t * ldy + i];
+    x[(size_t)t * H + i] += v;
+  }
+}
+
+// x[t] += sum of the nparts partials of y[t]; then [xh, xl][t] =
+// split(x[t] * w / sqrt(mean(x[t]^2) + eps)) for the next contraction.
+__global__ void residual_rmsnorm_split_kernel(float* __restrict__ x, const float* __restrict__ y,
+                                              int H, int ldy, int nparts, size_t pstride,
+                                              const uint16_t* __restrict__ w, float eps,
+                                              uint16_t* __restrict__ xh, uint16_t* __restrict__ xl) {
+  __shared__ float red[32];
+  const int t = blockIdx.x;
+  float* xr = x + (size_t)t * H;
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < H; i += blockDim.x) {
+    float v = 0.f;
+    for (int z = 0; z < nparts; ++z) v += y[z * pstride + (size_t)t * ldy + i];
+    const float nx = xr[i] + v;
+    xr[i] = nx;
+    ss = fmaf(nx, nx, ss);
+  }
+  for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  float tot = 0.f;
+  for (int i = 0; i < (int)(blockDim.x >> 5); ++i) tot += red[i];
+  const float r = 1.0f / sqrtf(tot / (float)H + eps);
+  for (int i = threadIdx.x; i < H; i += blockDim.x)
+    split_store(xr[i] * r * bf16_val(w[i]), xh, xl, (size_t)t * H + i);
 }
 
 // [xh, xl][t][j] = split(silu(gate_j) * up_j); gate/up interleaved in y.
-__global__ void swiglu_split_kernel(const float* __restrict__ y, int ldy, int F,
-                                    uint16_t* __restrict__ xh, uint16_t* __restrict__ xl) {
+__global__ void swiglu_split_kernel(const float* __restrict__ y, int ldy, int F, int nparts,
+                                    size_t pstride, uint16_t* __restrict__ xh,
+                                    uint16_t* __restrict__ xl) {
   const int t = blockIdx.x;
   for (int j = threadIdx.x; j < F; j += blockDim.x) {
-    const float g = y[(size_t)t * ldy + 2 * j], u = y[(size_t)t * ldy + 2 * j + 1];
+    float g = 0.f, u = 0.f;
+    for (int z = 0; z < nparts; ++z) {  // split-K partial sums, in order
+      g += y[z * pstride + (size_t)t * ldy + 2 * j];
+      u += y[z * pstride + (size_t)t * ldy + 2 * j + 1];
+    }
     split_store(g / (1.0f + expf(-g)) * u, xh, xl, (size_t)t * F + j);
+  }
+}
+
+// ------------------------------------------------- batched decode step
+// Split-KV decode attention for several requests at once: CTA (split s, KV
+// head g, request r) runs keys [k0, k1) of the request's cache, 64 keys at a
+// time double-buffered through shared memory with cp.async (16-byte pieces),
+// four keys per warp with the decode step's online-softmax update, then
+// merges its 16 warps and writes one partial (output unnormalised at the
+// split's maximum, the maximum, the sum).  About one split per 256 keys
+// holds keys; the rest return at once.
+constexpr int kBAWarps = 16;
+constexpr int kBAKeys = 64;
+constexpr int kBAKeysPerSplit = 256;
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+__device__ __forceinline__ int batch_live_splits(int n_keys, int S) {
+  int l = (n_keys + kBAKeysPerSplit - 1) / kBAKeysPerSplit;
+  return l < 1 ? 1 : (l > S ? S : l);
+}
+
+template <int DPL, int G>
+__global__ void __launch_bounds__(kBAWarps * 32, 1)
+    batch_attn_kernel(const float* __restrict__ q, const BatchParams* __restrict__ bp, ModelDev m,
+                      int layer, int S, float* __restrict__ part) {
+  constexpr int d = DPL * 32, PS = d + 4;
+  constexpr int kBuf = 2 * kBAKeys * d;  // bf16 elements per buffer (K then V)
+  extern __shared__ __align__(16) uint8_t ba_raw[];
+  uint16_t* buf = reinterpret_cast<uint16_t*>(ba_raw);
+  float* xbs = reinterpret_cast<float*>(buf + 2 * kBuf);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int sp = blockIdx.x, g = blockIdx.y, r = blockIdx.z;
+  const int n_keys = bp->pos[r] + 1;
+  const int live = batch_live_splits(n_keys, S);
+  if (sp >= live) return;
+  const int chunk = (n_keys + live - 1) / live;
+  const int k0 = min(n_keys, sp * chunk), k1 = min(n_keys, k0 + chunk);
+  const int nq = m.n_q;
+  const size_t head_off =
+      (((size_t)bp->slot[r] * m.n_layers + layer) * m.n_kv + g) * (size_t)m.max_seq * d;
+  const uint16_t* K = m.kcache + head_off;
+  const uint16_t* V = m.vcache + head_off;
+  AttnState<DPL, G> st;
+  attn_init<DPL, G>(st, q + (size_t)r * nq * d + (size_t)g * G * d, d, m.attn_scale, lane);
+  float* xb = xbs + warp * kAttnXbStride;
+  const int nblk = (k1 - k0 + kBAKeys - 1) / kBAKeys;
+  auto issue = [&](int b) {
+    const int kb = k0 + b * kBAKeys, nk = min(kBAKeys, k1 - kb);
+    uint16_t* dst = buf + (b & 1) * kBuf;
+    const int pieces = nk * d / 8;  // 16-byte pieces of K (and of V)
+    for (int i = threadIdx.x; i < pieces; i += blockDim.x) {
+      cp_async16(dst + i * 8, K + (size_t)kb * d + i * 8);
+      cp_async16(dst + kBAKeys * d + i * 8, V + (size_t)kb * d + i * 8);
+    }
+  };
+  if (nblk > 0) issue(0);
+  cp_async_commit();
+  for (int b = 0; b < nblk; ++b) {
+    if (b + 1 < nblk) issue(b + 1);
+    cp_async_commit();
+    cp_async_wait<1>();
+    __syncthreads();
+    const int kb = k0 + b * kBAKeys, nk = min(kBAKeys, k1 - kb);
+    const uint16_t* ks = buf + (b & 1) * kBuf;
+    const uint16_t* vs = ks + kBAKeys * d;
+    for (int j0 = 4 * warp; j0 < nk; j0 += 4 * kBAWarps) {
+      const int nj = min(4, nk - j0);
+      {
+        float kv[4][DPL];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int jr = attn_key_row<G>(t, lane);
+          if (jr < nj) load_kv_row<DPL>(ks + (size_t)(j0 + jr) * d + lane * DPL, kv[t]);
+          else
+#pragma unroll
+            for (int i = 0; i < DPL; ++i) kv[t][i] = 0.f;
+        }
+        attn_scores4<DPL, G>(st, kv, nj, xb, lane);
+      }
+      float vv[4][DPL];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        if (t < nj) load_kv_row<DPL>(vs + (size_t)(j0 + t) * d + lane * DPL, vv[t]);
+        else
+#pragma unroll
+          for (int i = 0; i < DPL; ++i) vv[t][i] = 0.f;
+      }
+      attn_update4<DPL, G>(st, vv, xb);
+    }
+    __syncthreads();  // buffer b & 1 is refilled by block b + 2
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+  // the 16 warps' states through shared memory, then one partial
+  float* ws = reinterpret_cast<float*>(ba_raw);  // [16][G][PS], reuses the key buffers
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) ws[(warp * G + h) * PS + lane * DPL + i] = st.o[h][i];
+    if (lane == 0) {
+      ws[(warp * G + h) * PS + d] = st.mx[h];
+      ws[(warp * G + h) * PS + d + 1] = st.l[h];
+    }
+  }
+  __syncthreads();
+  float* dst = part + ((size_t)(r * m.n_kv + g) * S + sp) * G * PS;
+  for (int idx = threadIdx.x; idx < G * (d + 2); idx += blockDim.x) {
+    const int h = idx / (d + 2), i = idx - h * (d + 2);
+    float M = -INFINITY;
+    for (int w = 0; w < kBAWarps; ++w) M = fmaxf(M, ws[(w * G + h) * PS + d]);
+    float val = 0.f;
+    if (M != -INFINITY)
+      for (int w = 0; w < kBAWarps; ++w) {
+        const float mw = ws[(w * G + h) * PS + d];
+        if (mw == -INFINITY) continue;
+        const float x = i < d ? ws[(w * G + h) * PS + i] : ws[(w * G + h) * PS + d + 1];
+        val = fmaf(__expf(mw - M), x, val);
+      }
+    dst[h * PS + i] = i == d ? M : val;
+  }
+}
+
+// Merges the live splits of (KV head g, request r) and writes the attention
+// output, normalised, as the O projection's [xh, xl] input.
+__global__ void batch_attn_merge_kernel(const float* __restrict__ part, const BatchParams* __restrict__ bp,
+                                        ModelDev m, int S, uint16_t* __restrict__ xh,
+                                        uint16_t* __restrict__ xl) {
+  const int g = blockIdx.x, r = blockIdx.y;
+  const int d = m.head_dim, G = m.group, PS = d + 4, nq = m.n_q;
+  const int live = batch_live_splits(bp->pos[r] + 1, S);
+  const float* pg = part + (size_t)(r * m.n_kv + g) * S * G * PS;
+  for (int idx = threadIdx.x; idx < G * d; idx += blockDim.x) {
+    const int h = idx / d, i = idx - h * d;
+    float M = -INFINITY;
+    for (int s2 = 0; s2 < live; ++s2) {
+      const float* ps = pg + ((size_t)s2 * G + h) * PS;
+      if (ps[d + 1] != 0.f) M = fmaxf(M, ps[d]);
+    }
+    float num = 0.f, den = 0.f;
+    for (int s2 = 0; s2 < live; ++s2) {
+      const float* ps = pg + ((size_t)s2 * G + h) * PS;
+      const float ls = ps[d + 1];
+      if (ls == 0.f) continue;
+      const float c = __expf(ps[d] - M);
+      num = fmaf(c, ps[i], num);
+      den = fmaf(c, ls, den);
+    }
+    split_store(num / den, xh, xl, (size_t)r * nq * d + (size_t)(g * G + h) * d + i);
+  }
+}
+
+// The batched step's elementwise operators run over (token, 1024-element
+// slice) grids of 256 threads, four elements each.  RMSNorm is deferred: they
+// write x * w (split into xh, xl) and add this slice's sum of x^2 into
+// tok_ss[t]; the next GEMM scales its outputs by 1/sqrt(tok_ss[t]/H + eps).
+__device__ __forceinline__ void block_ss_add(float ss, float* dst) {
+  __shared__ float red[8];
+  for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float tot = 0.f;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) tot += red[i];
+    atomicAdd(dst, tot);
+  }
+}
+
+// x[t] = E[token]; xh/xl = split(x * w); tok_ss[t] += sum x^2.
+__global__ void b_embed_norm_kernel(const uint16_t* __restrict__ E, const int32_t* __restrict__ tokens,
+                                    int H, int vocab, const uint16_t* __restrict__ w,
+                                    float* __restrict__ x, uint16_t* __restrict__ xh,
+                                    uint16_t* __restrict__ xl, float* __restrict__ tok_ss,
+                                    int32_t* __restrict__ status) {
+  const int t = blockIdx.y;
+  int tok = tokens[t];
+  if (tok < 0 || tok >= vocab) {
+    if (threadIdx.x == 0 && blockIdx.x == 0 && atomicCAS(status, 0, MK_ERR_TOKEN_RANGE) == 0)
+      status[1] = tok;
+    tok = 0;
+  }
+  float ss = 0.f;
+  const int i0 = blockIdx.x * 1024 + threadIdx.x * 4;
+  for (int i = i0; i < min(H, i0 + 4); ++i) {
+    const float v = bf16_val(E[(size_t)tok * H + i]);
+    x[(size_t)t * H + i] = v;
+    ss = fmaf(v, v, ss);
+    split_store(v * bf16_val(w[i]), xh, xl, (size_t)t * H + i);
+  }
+  block_ss_add(ss, tok_ss + t);
+}
+
+// x[t] += sum of the partials of y[t]; xh/xl = split(x * w); tok_ss[t] += sum x^2.
+__global__ void b_residual_norm_kernel(float* __restrict__ x, const float* __restrict__ y, int H,
+                                       int ldy, int nparts, size_t pstride,
+                                       const uint16_t* __restrict__ w, uint16_t* __restrict__ xh,
+                                       uint16_t* __restrict__ xl, float* __restrict__ tok_ss) {
+  const int t = blockIdx.y;
+  float ss = 0.f;
+  const int i0 = blockIdx.x * 1024 + threadIdx.x * 4;
+  for (int i = i0; i < min(H, i0 + 4); ++i) {
+    float v = 0.f;
+    for (int z = 0; z < nparts; ++z) v += y[z * pstride + (size_t)t * ldy + i];
+    const float nx = x[(size_t)t * H + i] + v;
+    x[(size_t)t * H + i] = nx;
+    ss = fmaf(nx, nx, ss);
+    split_store(nx * bf16_val(w[i]), xh, xl, (size_t)t * H + i);
+  }
+  block_ss_add(ss, tok_ss + t);
+}
+
+// xh/xl[t][j] = split(silu(gate_j) * up_j), gate/up summed over the partials.
+__global__ void b_swiglu_kernel(const float* __restrict__ y, int ldy, int F, int nparts,
+                                size_t pstride, uint16_t* __restrict__ xh, uint16_t* __restrict__ xl) {
+  const int t = blockIdx.y;
+  const int j0 = blockIdx.x * 1024 + threadIdx.x * 4;
+  for (int j = j0; j < min(F, j0 + 4); ++j) {
+    float g = 0.f, u = 0.f;
+    for (int z = 0; z < nparts; ++z) {
+      g += y[z * pstride + (size_t)t * ldy + 2 * j];
+      u += y[z * pstride + (size_t)t * ldy + 2 * j + 1];
+    }
+    split_store(g / (1.0f + expf(-g)) * u, xh, xl, (size_t)t * F + j);
+  }
+}
+
+// Per-request argmax over the logits: slices of 4096 entries fold into one
+// 64-bit (ordered value, inverted index) key per request with atomicMax; the
+// lowest index wins ties.  best[] starts at zero each step.
+__global__ void b_argmax_kernel(const float* __restrict__ logits, int V,
+                                unsigned long long* __restrict__ best) {
+  __shared__ unsigned long long red[8];
+  const int r = blockIdx.y;
+  unsigned long long k = 0ull;
+  const int i1 = min(V, (int)(blockIdx.x + 1) * 4096);
+  for (int i = blockIdx.x * 4096 + threadIdx.x; i < i1; i += blockDim.x) {
+    uint32_t u = __float_as_uint(logits[(size_t)r * V + i]);
+    u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    const unsigned long long c = ((unsigned long long)u << 32) | (0xffffffffu - (uint32_t)i);
+    k = c > k ? c : k;
+  }
+  for (int o = 16; o; o >>= 1) {
+    const unsigned long long v = __shfl_xor_sync(0xffffffffu, k, o);
+    k = v > k ? v : k;
+  }
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = k;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w2 = 1; w2 < (int)(blockDim.x >> 5); ++w2) k = red[w2] > k ? red[w2] : k;
+    k = red[0] > k ? red[0] : k;
+    atomicMax(best + r, k);
+  }
+}
+
+__global__ void b_ids_kernel(const unsigned long long* __restrict__ best, int n, int32_t* __restrict__ ids) {
+  const int r = threadIdx.x;
+  if (r < n) ids[r] = (int32_t)(0xffffffffu - (uint32_t)(best[r] & 0xffffffffull));
+}
+
+// Greedy id of each request: the largest logit, the lowest index on ties.
+__global__ void argmax_rows_kernel(const float* __restrict__ logits, int V, int32_t* __restrict__ ids) {
+  __shared__ unsigned long long red[32];
+  const int r = blockIdx.x;
+  unsigned long long best = 0ull;
+  for (int i = threadIdx.x; i < V; i += blockDim.x) {
+    uint32_t u = __float_as_uint(logits[(size_t)r * V + i]);
+    u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    const unsigned long long k = ((unsigned long long)u << 32) | (0xffffffffu - (uint32_t)i);
+    best = k > best ? k : best;
+  }
+  for (int o = 16; o; o >>= 1) {
+    const unsigned long long v = __shfl_xor_sync(0xffffffffu, best, o);
+    best = v > best ? v : best;
+  }
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = best;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) best = red[w] > best ? red[w] : best;
+    best = red[0] > best ? red[0] : best;
+    ids[r] = (int32_t)(0xffffffffu - (uint32_t)(best & 0xffffffffull));
   }
 }
 
@@ -358,30 +707,39 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D bf16 tensor [rows][cols] (row-major), boxes of 64 columns x 128 rows,
-// 128-byte swizzle, zero fill outside.
-bool make_map(CUtensorMap* map, const void* base, int rows, int cols) {
+// 2-D bf16 tensor [rows][cols] (row-major), boxes of 64 columns x box_rows
+// rows, 128-byte swizzle, zero fill outside.
+bool make_map(CUtensorMap* map, const void* base, int rows, int cols, int box_rows = 128) {
   auto fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)kGK, 128u};
+  const cuuint32_t box[2] = {(cuuint32_t)kGK, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1u, 1u};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Y (+ z * n_tok * ldy for split z) = W x^T over `splits` K ranges.
+template <int BN, int STAGES>
 std::string gemm(const uint16_t* W, int n_rows, int K, const uint16_t* xh, const uint16_t* xl,
-                 int n_tok, float* Y, int ldy, const uint16_t* bias, int32_t* err, cudaStream_t st) {
+                 int n_tok, float* Y, int ldy, const uint16_t* bias, int32_t* err, cudaStream_t st,
+                 int splits = 1, const float* tok_ss = nullptr, float norm_eps = 0.f) {
   CUtensorMap mw, mh, ml;
-  if (!make_map(&mw, W, n_rows, K) || !make_map(&mh, xh, n_tok, K) || !make_map(&ml, xl, n_tok, K))
+  if (!make_map(&mw, W, n_rows, K) || !make_map(&mh, xh, n_tok, K, BN) ||
+      !make_map(&ml, xl, n_tok, K, BN))
     return "cuTensorMapEncodeTiled failed";
-  const dim3 grid((n_rows + kGM - 1) / kGM, (n_tok + kGN - 1) / kGN);
-  gemm_wx_kernel<<<grid, 128, kGemmSmemBytes, st>>>(mw, mh, ml, n_rows, n_tok, K, Y, ldy, bias, err);
+  const dim3 grid((n_rows + kGM - 1) / kGM, (n_tok + BN - 1) / BN, splits);
+  gemm_wx_kernel<BN, STAGES><<<grid, 128, gemm_smem_bytes<BN, STAGES>(), st>>>(
+      mw, mh, ml, n_rows, n_tok, K, Y, ldy, (size_t)n_tok * ldy, splits == 1 ? bias : nullptr, err,
+      tok_ss, K, norm_eps);
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? "" : std::string("GEMM launch: ") + cudaGetErrorString(e);
 }
+
+constexpr int kPBN = 128, kPStages = 4;   // prompt GEMM: 128 tokens per CTA
+constexpr int kDBN = 16, kDStages = 10;   // decode GEMM: up to 16 tokens (8 requests)
 
 template <int DPL, int G>
 std::string launch_attn(dim3 grid, cudaStream_t st, const float* q, const int32_t* tiles,
@@ -436,8 +794,8 @@ std::string prefill_alloc(const ModelDev& m, int max_tokens, PrefillScratch* sc,
     owned->push_back(*a.p);
   }
   cudaMemset(sc->err, 0, 16);
-  if (cudaFuncSetAttribute(gemm_wx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)kGemmSmemBytes) != cudaSuccess)
+  if (cudaFuncSetAttribute(gemm_wx_kernel<kPBN, kPStages>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)gemm_smem_bytes<kPBN, kPStages>()) != cudaSuccess)
     return "GEMM shared memory attribute";
   sc->max_tokens = max_tokens;
   return "";
@@ -487,16 +845,16 @@ std::string prefill_run(const ModelDev& m, const PrefillWeights& w, PrefillScrat
     for (int l = 0; l < L; ++l) {
       rmsnorm_split_kernel<<<T, 256, 0, st>>>(sc.x, m.attn_norm + (size_t)l * H, H, m.rms_eps, sc.xh, sc.xl);
       const uint16_t* bias = m.qkv_bias ? m.bqkv + (size_t)l * qkvR : nullptr;
-      if (!(e = gemm(w.qkv[l], qkvR, H, sc.xh, sc.xl, T, sc.y, ldy, bias, sc.err, st)).empty()) return e;
-      rope_kv_kernel<<<T, 256, 0, st>>>(sc.y, ldy, d_slot, d_pos, m, l, sc.q);
+      if (!(e = gemm<kPBN, kPStages>(w.qkv[l], qkvR, H, sc.xh, sc.xl, T, sc.y, ldy, bias, sc.err, st)).empty()) return e;
+      rope_kv_kernel<<<T, 256, 0, st>>>(sc.y, ldy, 1, 0, nullptr, d_slot, d_pos, m, l, sc.q);
       if (!(e = attn(dim3(ntiles, m.n_kv), st, sc.q, d_tiles, m, l, sc.xh, sc.xl)).empty()) return e;
-      if (!(e = gemm(w.o[l], H, qd, sc.xh, sc.xl, T, sc.y, ldy, nullptr, sc.err, st)).empty()) return e;
-      residual_kernel<<<T, 256, 0, st>>>(sc.x, sc.y, H, ldy);
+      if (!(e = gemm<kPBN, kPStages>(w.o[l], H, qd, sc.xh, sc.xl, T, sc.y, ldy, nullptr, sc.err, st)).empty()) return e;
+      residual_kernel<<<T, 256, 0, st>>>(sc.x, sc.y, H, ldy, 1, 0);
       rmsnorm_split_kernel<<<T, 256, 0, st>>>(sc.x, m.ffn_norm + (size_t)l * H, H, m.rms_eps, sc.xh, sc.xl);
-      if (!(e = gemm(w.gu[l], 2 * F, H, sc.xh, sc.xl, T, sc.y, ldy, nullptr, sc.err, st)).empty()) return e;
-      swiglu_split_kernel<<<T, 256, 0, st>>>(sc.y, ldy, F, sc.xh, sc.xl);
-      if (!(e = gemm(w.dn[l], H, F, sc.xh, sc.xl, T, sc.y, ldy, nullptr, sc.err, st)).empty()) return e;
-      residual_kernel<<<T, 256, 0, st>>>(sc.x, sc.y, H, ldy);
+      if (!(e = gemm<kPBN, kPStages>(w.gu[l], 2 * F, H, sc.xh, sc.xl, T, sc.y, ldy, nullptr, sc.err, st)).empty()) return e;
+      swiglu_split_kernel<<<T, 256, 0, st>>>(sc.y, ldy, F, 1, 0, sc.xh, sc.xl);
+      if (!(e = gemm<kPBN, kPStages>(w.dn[l], H, F, sc.xh, sc.xl, T, sc.y, ldy, nullptr, sc.err, st)).empty()) return e;
+      residual_kernel<<<T, 256, 0, st>>>(sc.x, sc.y, H, ldy, 1, 0);
     }
     const cudaError_t ce = cudaGetLastError();
     if (ce != cudaSuccess) return std::string("prefill launch: ") + cudaGetErrorString(ce);
@@ -508,6 +866,180 @@ std::string prefill_run(const ModelDev& m, const PrefillWeights& w, PrefillScrat
     return std::string("prefill: ") + cudaGetErrorString(cudaGetLastError());
   if (herr) return "prefill GEMM: a pipeline wait timed out";
   return "";
+}
+
+namespace {
+
+template <int DPL, int G>
+size_t batch_attn_smem() {
+  // two key/value buffers and the warps' softmax scratch; after the key loop
+  // the warps' states (16 x G x (d + 4) floats) reuse the same bytes
+  const size_t loop = (size_t)2 * 2 * kBAKeys * DPL * 32 * 2 + (size_t)kBAWarps * kAttnXbStride * 4;
+  const size_t merge = (size_t)kBAWarps * G * (DPL * 32 + 4) * 4;
+  return loop > merge ? loop : merge;
+}
+
+template <int DPL, int G>
+std::string launch_batch_attn(dim3 grid, cudaStream_t st, const float* q, const BatchParams* bp,
+                              const ModelDev& m, int layer, int S, float* part, bool set_attr) {
+  auto k = batch_attn_kernel<DPL, G>;
+  const size_t smem = batch_attn_smem<DPL, G>();
+  if (set_attr) {
+    return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) == cudaSuccess
+               ? "" : "batched attention shared memory attribute";
+  }
+  k<<<grid, kBAWarps * 32, smem, st>>>(q, bp, m, layer, S, part);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? "" : std::string("batched attention launch: ") + cudaGetErrorString(e);
+}
+
+std::string batch_attn(dim3 grid, cudaStream_t st, const float* q, const BatchParams* bp,
+                       const ModelDev& m, int layer, int S, float* part, bool set_attr = false) {
+  const int G = m.group;
+#define MK_BA(DPL_, G_) return launch_batch_attn<DPL_, G_>(grid, st, q, bp, m, layer, S, part, set_attr)
+  if (m.head_dim == 128) {
+    if (G == 1) MK_BA(4, 1);
+    if (G == 2) MK_BA(4, 2);
+    if (G == 4) MK_BA(4, 4);
+  } else {
+    if (G == 1) MK_BA(2, 1);
+    if (G == 2) MK_BA(2, 2);
+    if (G == 4) MK_BA(2, 4);
+    if (G == 7) MK_BA(2, 7);
+    if (G == 8) MK_BA(2, 8);
+  }
+#undef MK_BA
+  return "unsupported query heads per KV head";
+}
+
+// K split of a decode GEMM from a simple cost model: a CTA costs a fixed
+// ~4 us (setup, pipeline fill, epilogue) plus its share of the 128-row tile
+// at ~40 GB/s; waves of num_sms CTAs run one after another.  At least two K
+// blocks per CTA, at most kBatchMaxSplitK splits.
+int split_k(int n_rows, int K, int num_sms) {
+  const int tiles = (n_rows + kGM - 1) / kGM, nk = K / kGK;
+  const double tile_us = (double)kGM * K * 2 / 40e3;  // bytes / (40 GB/s) in us
+  int best = 1;
+  double best_t = 1e30;
+  for (int z = 1; z <= kBatchMaxSplitK && z <= std::max(1, nk / 2); ++z) {
+    const int waves = (tiles * z + num_sms - 1) / num_sms;
+    const double t = waves * (4.0 + tile_us / z);
+    if (t < best_t - 1e-9) {
+      best_t = t;
+      best = z;
+    }
+  }
+  return best;
+}
+
+std::string batch_enqueue(const ModelDev& m, const PrefillWeights& w, BatchScratch& bs, int n,
+                          int num_sms, cudaStream_t st) {
+  const int H = m.hidden, F = m.ffn, d = m.head_dim, qd = m.n_q * d, L = m.n_layers, V = m.vocab;
+  const int qkvR = qkv_rows(m.n_q, m.n_kv, d);
+  const int ldy = std::max(std::max(qkvR, 2 * F), H);
+  const size_t pstride = (size_t)n * ldy;
+  const int zq = split_k(qkvR, H, num_sms), zo = split_k(H, qd, num_sms);
+  const int zg = split_k(2 * F, H, num_sms), zd = split_k(H, F, num_sms);
+  std::string e;
+  BatchParams* bp = bs.params;
+  const int hsl = (H + 1023) / 1024, fsl = (F + 1023) / 1024;
+  const int psl = ((qkvR >> 1) + 255) / 256;
+  // per-step accumulators: the norms' sums of squares, the argmax keys
+  if (cudaMemsetAsync(bs.acc, 0, bs.acc_bytes, st) != cudaSuccess) return "batched step memset";
+  float* ss = reinterpret_cast<float*>(bs.acc);                       // [2L + 1][kMaxBatch]
+  unsigned long long* best = reinterpret_cast<unsigned long long*>(bs.acc) + (2 * L + 1) * kMaxBatch / 2 + 1;
+  b_embed_norm_kernel<<<dim3(hsl, n), 256, 0, st>>>(m.embed, bs.tokens, H, m.vocab, m.attn_norm, bs.x,
+                                                    bs.xh, bs.xl, ss, m.status);
+  for (int l = 0; l < L; ++l) {
+    float* ss_attn = ss + (size_t)(2 * l) * kMaxBatch;
+    float* ss_ffn = ss + (size_t)(2 * l + 1) * kMaxBatch;
+    float* ss_next = ss + (size_t)(2 * l + 2) * kMaxBatch;
+    const uint16_t* bias = m.qkv_bias ? m.bqkv + (size_t)l * qkvR : nullptr;
+    if (!(e = gemm<kDBN, kDStages>(w.qkv[l], qkvR, H, bs.xh, bs.xl, n, bs.y, ldy, nullptr, bs.err, st, zq,
+                                   ss_attn, m.rms_eps)).empty()) return e;
+    rope_kv_kernel<<<dim3(n, psl), 256, 0, st>>>(bs.y, ldy, zq, pstride, bias, bp->slot, bp->pos, m, l, bs.q);
+    if (!(e = batch_attn(dim3(bs.splits, m.n_kv, n), st, bs.q, bp, m, l, bs.splits, bs.part)).empty()) return e;
+    batch_attn_merge_kernel<<<dim3(m.n_kv, n), 256, 0, st>>>(bs.part, bp, m, bs.splits, bs.xh, bs.xl);
+    if (!(e = gemm<kDBN, kDStages>(w.o[l], H, qd, bs.xh, bs.xl, n, bs.y, ldy, nullptr, bs.err, st, zo)).empty()) return e;
+    b_residual_norm_kernel<<<dim3(hsl, n), 256, 0, st>>>(bs.x, bs.y, H, ldy, zo, pstride,
+                                                         m.ffn_norm + (size_t)l * H, bs.xh, bs.xl, ss_ffn);
+    if (!(e = gemm<kDBN, kDStages>(w.gu[l], 2 * F, H, bs.xh, bs.xl, n, bs.y, ldy, nullptr, bs.err, st, zg,
+                                   ss_ffn, m.rms_eps)).empty()) return e;
+    b_swiglu_kernel<<<dim3(fsl, n), 256, 0, st>>>(bs.y, ldy, F, zg, pstride, bs.xh, bs.xl);
+    if (!(e = gemm<kDBN, kDStages>(w.dn[l], H, F, bs.xh, bs.xl, n, bs.y, ldy, nullptr, bs.err, st, zd)).empty()) return e;
+    // the residual add, then the next layer's attention norm (the final norm after the last)
+    const uint16_t* next_norm = l + 1 < L ? m.attn_norm + (size_t)(l + 1) * H : m.final_norm;
+    b_residual_norm_kernel<<<dim3(hsl, n), 256, 0, st>>>(bs.x, bs.y, H, ldy, zd, pstride, next_norm,
+                                                         bs.xh, bs.xl, ss_next);
+  }
+  if (!(e = gemm<kDBN, kDStages>(m.lm_head, V, H, bs.xh, bs.xl, n, bs.logits, V, nullptr, bs.err, st, 1,
+                                 ss + (size_t)(2 * L) * kMaxBatch, m.rms_eps)).empty()) return e;
+  b_argmax_kernel<<<dim3((V + 4095) / 4096, n), 256, 0, st>>>(bs.logits, V, best);
+  b_ids_kernel<<<1, 32, 0, st>>>(best, n, bs.ids);
+  const cudaError_t ce = cudaGetLastError();
+  return ce == cudaSuccess ? "" : std::string("batched step launch: ") + cudaGetErrorString(ce);
+}
+
+}  // namespace
+
+std::string batch_alloc(const ModelDev& m, int num_sms, BatchScratch* bs, std::vector<void*>* owned) {
+  const int H = m.hidden, F = m.ffn, d = m.head_dim, qd = m.n_q * d, G = m.group;
+  const int qkvR = qkv_rows(m.n_q, m.n_kv, d);
+  const size_t B = kMaxBatch;
+  const size_t ycols = (size_t)std::max(std::max(qkvR, 2 * F), H);
+  const size_t xcols = (size_t)std::max(std::max(H, F), qd);
+  bs->splits = std::max(1, (2 * num_sms + (int)B * m.n_kv - 1) / ((int)B * m.n_kv));
+  // per step: (2 layers + 1) norms' sums of squares, then the argmax keys
+  bs->acc_bytes = ((size_t)(2 * m.n_layers + 1) * kMaxBatch + 2) * 4 + (size_t)kMaxBatch * 8 + 16;
+  struct A { void** p; size_t bytes; } allocs[] = {
+      {(void**)&bs->params, sizeof(BatchParams)},
+      {(void**)&bs->tokens, B * 4},
+      {(void**)&bs->x, B * H * 4},
+      {(void**)&bs->y, (size_t)kBatchMaxSplitK * B * ycols * 4},
+      {(void**)&bs->q, B * qd * 4},
+      {(void**)&bs->part, B * m.n_kv * bs->splits * G * (d + 4) * 4},
+      {(void**)&bs->xh, B * xcols * 2},
+      {(void**)&bs->xl, B * xcols * 2},
+      {(void**)&bs->logits, B * (size_t)m.vocab * 4},
+      {(void**)&bs->ids, B * 4},
+      {(void**)&bs->err, 16},
+      {(void**)&bs->acc, bs->acc_bytes}};
+  for (auto& a : allocs) {
+    const cudaError_t e = cudaMalloc(a.p, a.bytes);
+    if (e != cudaSuccess) return std::string("batched step scratch: ") + cudaGetErrorString(e);
+    owned->push_back(*a.p);
+  }
+  cudaMemset(bs->err, 0, 16);
+  if (cudaFuncSetAttribute(gemm_wx_kernel<kDBN, kDStages>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)gemm_smem_bytes<kDBN, kDStages>()) != cudaSuccess)
+    return "decode GEMM shared memory attribute";
+  return batch_attn(dim3(1), nullptr, nullptr, nullptr, m, 0, bs->splits, nullptr, true);
+}
+
+std::string batch_step(const ModelDev& m, const PrefillWeights& w, BatchScratch& bs, int n,
+                       int num_sms, cudaStream_t st) {
+  if (n < 2 || n > kMaxBatch) return "batched step needs 2..8 requests";
+  if (!bs.graph[n]) {
+    cudaStream_t cs;
+    if (cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) != cudaSuccess) return "capture stream";
+    cudaError_t e = cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal);
+    std::string err = e == cudaSuccess ? batch_enqueue(m, w, bs, n, num_sms, cs) : "begin capture";
+    cudaGraph_t g = nullptr;
+    const cudaError_t e2 = cudaStreamEndCapture(cs, &g);
+    cudaStreamDestroy(cs);
+    if (!err.empty()) {
+      if (g) cudaGraphDestroy(g);
+      return err;
+    }
+    if (e2 != cudaSuccess) return std::string("batched step capture: ") + cudaGetErrorString(e2);
+    if (cudaGraphInstantiate(&bs.graph[n], g, 0) != cudaSuccess) {
+      cudaGraphDestroy(g);
+      return "batched step graph instantiation";
+    }
+    bs.graph_src[n] = g;
+  }
+  const cudaError_t e = cudaGraphLaunch(bs.graph[n], st);
+  return e == cudaSuccess ? "" : std::string("batched step replay: ") + cudaGetErrorString(e);
 }
 
 }  // namespace mk

@@ -33,6 +33,36 @@ struct PrefillScratch {
   int32_t* err = nullptr;      // device error word of the GEMM kernel
 };
 
+// Device-side parameters of a batched decode step (read by the captured
+// kernels, written before each replay).
+struct BatchParams {
+  int32_t n;
+  int32_t pos[kMaxBatch];
+  int32_t slot[kMaxBatch];
+  int32_t src[kMaxBatch];   // token index of request r: r
+};
+
+// Scratch and captured graphs of the batched decode step.
+struct BatchScratch {
+  int splits = 0;              // attention splits per (request, KV head)
+  BatchParams* params = nullptr;
+  int32_t* tokens = nullptr;   // [kMaxBatch] this step's input ids
+  float* x = nullptr;          // [kMaxBatch][hidden] residual stream
+  float* y = nullptr;          // [kBatchMaxSplitK][kMaxBatch][max(qkv rows, 2 ffn, hidden)]
+  float* q = nullptr;          // [kMaxBatch][n_q * d]
+  float* part = nullptr;       // [kMaxBatch][n_kv][splits][G][d + 4] attention partials
+  uint16_t* xh = nullptr;      // [kMaxBatch][max(hidden, ffn, n_q*d)]
+  uint16_t* xl = nullptr;
+  float* logits = nullptr;     // [kMaxBatch][vocab]
+  int32_t* ids = nullptr;      // [kMaxBatch]
+  int32_t* err = nullptr;
+  void* acc = nullptr;         // per-step accumulators (zeroed by the step)
+  size_t acc_bytes = 0;
+  cudaGraphExec_t graph[kMaxBatch + 1] = {};
+  cudaGraph_t graph_src[kMaxBatch + 1] = {};
+};
+constexpr int kBatchMaxSplitK = 16;
+
 // Whether the GEMM path handles this shape (every contraction length a
 // multiple of 64).
 bool prefill_gemm_supported(const ModelDev& m);
@@ -46,5 +76,16 @@ std::string prefill_alloc(const ModelDev& m, int max_tokens, PrefillScratch* sc,
 std::string prefill_run(const ModelDev& m, const PrefillWeights& w, PrefillScratch& sc,
                         cudaStream_t st, const int32_t* tokens_dev, const int32_t* offsets_host,
                         int n_req);
+
+// Allocates the batched decode scratch (cudaMalloc).
+std::string batch_alloc(const ModelDev& m, int num_sms, BatchScratch* bs, std::vector<void*>* owned);
+
+// One decode step of n (2..8) requests with every weight matrix streamed
+// once: tcgen05 GEMMs of 16 token columns (split along K where a matrix has
+// few 128-row tiles), split-KV attention per (request, KV head), argmax per
+// request.  Reads bs.tokens and bs.params; writes bs.logits, bs.ids, bs.x.
+// Captured into a CUDA graph per n on first use, then replayed.
+std::string batch_step(const ModelDev& m, const PrefillWeights& w, BatchScratch& bs, int n,
+                       int num_sms, cudaStream_t st);
 
 }  // namespace mk

@@ -48,9 +48,18 @@ def _run_batch(model, w, lens, steps, max_seq, seed=1, **kw):
     return dec
 
 
-def test_tiny_eight_requests(cuda_ok):
+@pytest.mark.parametrize("sequential", [0, 1], ids=["batched", "sequential"])
+def test_tiny_eight_requests(cuda_ok, sequential):
+    # batched: one step streams each weight matrix once (tensor-core GEMMs over
+    # the requests); sequential: the requests run through the megakernel in turn
     w = synth.make_model(synth.TINY, 7)
-    _run_batch(synth.TINY, w, [5, 17, 9, 30, 1, 12, 23, 8], 6, 40)
+    _run_batch(synth.TINY, w, [5, 17, 9, 30, 1, 12, 23, 8], 6, 40, batch_sequential=sequential)
+
+
+def test_tiny_long_contexts_batched(cuda_ok):
+    # contexts past 256 keys: several attention splits per request and KV head
+    w = synth.make_model(synth.TINY, 9)
+    _run_batch(synth.TINY, w, [700, 40, 333, 1024], 4, 1030)
 
 
 def test_tiny_eight_requests_per_op_graph(cuda_ok):
@@ -88,4 +97,4 @@ def test_fewer_requests_than_the_batch(cuda_ok):
                          ids=lambda m: m.name)
 def test_wide_shapes_three_requests(model, cuda_ok):
     w = synth.make_model(model, 2)
-    _run_batch(model, w, [39, 7, 64], 3, 70)
+    _run_batch(model, w, [39, 7, 300], 3, 310)
