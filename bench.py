@@ -377,8 +377,8 @@ def run_mk(args):
     else:
         workload = (f"llama-3-8b-shape decode, {n} requests per step, random prompts of "
                     f"{lens} tokens packed with offsets, greedy decode steps {W}..{W + K - 1} "
-                    "after each prompt timed; requests run in turn through the one-request "
-                    "graph (weights streamed once per request)")
+                    "after each prompt timed; one batched step per token (tcgen05 GEMMs over "
+                    "the requests' columns, each weight matrix streamed once; CUDA graph)")
         unit, metric = "ms/step", f"decode ms/step ({n} requests, Llama-3-8B-shape)"
     line = {
         "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": K,
@@ -408,8 +408,8 @@ def run_mk(args):
     }
     if n > 1:
         line["roofline"]["bytes_note"] = ("algorithmic bytes: weights once per step plus every "
-                                          "request's KV; the path streams the weights once per "
-                                          "request")
+                                          "request's KV (the baselines run the requests in turn "
+                                          "through the per-operator launches)")
     if args.layers:
         line["config"]["workload"] += f" [profiling case: {args.layers} layers]"
     if args.l2_prefetch:

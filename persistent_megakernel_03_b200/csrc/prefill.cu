@@ -49,22 +49,27 @@ constexpr int kGM = 128, kGK = 64;
 constexpr int kGTileA = kGM * kGK * 2;  // 16 KB
 constexpr uint64_t kGWaitNs = 2000000000ull;  // 2 s: far beyond any legal wait
 
-template <int BN, int STAGES>
+// HL: the B operand is one BN-row tile whose first BN/2 rows are the high
+// parts and the last BN/2 rows the low parts of the same BN/2 tokens (a
+// decode step of up to 8 requests): one MMA per K step, and the epilogue adds
+// accumulator columns j and j + BN/2.
+template <int BN, int STAGES, bool HL = false>
 struct __align__(1024) GemmSmem {
   static constexpr int kTileB = BN * kGK * 2;
-  static constexpr uint32_t kStageBytes = kGTileA + 2 * kTileB;
+  static constexpr int kBTiles = HL ? 1 : 2;
+  static constexpr uint32_t kStageBytes = kGTileA + kBTiles * kTileB;
   static constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;
   uint8_t a[STAGES][kGTileA];
   uint8_t bh[STAGES][kTileB];
-  uint8_t bl[STAGES][kTileB];
+  uint8_t bl[HL ? 1 : STAGES][HL ? 16 : kTileB];
   uint64_t full[STAGES];
   uint64_t empty[STAGES];
   uint64_t done;
   uint32_t tmem;
   int32_t failed;
 };
-template <int BN, int STAGES>
-constexpr size_t gemm_smem_bytes() { return sizeof(GemmSmem<BN, STAGES>) + 1024; }
+template <int BN, int STAGES, bool HL = false>
+constexpr size_t gemm_smem_bytes() { return sizeof(GemmSmem<BN, STAGES, HL>) + 1024; }
 
 // Bounded wait on an mbarrier phase; false after kGWaitNs (the caller records
 // the failure and stops issuing work).
@@ -76,14 +81,14 @@ __device__ __forceinline__ bool gemm_wait(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool HL = false>
 __global__ void __launch_bounds__(128, 1)
     gemm_wx_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_xh,
                    const __grid_constant__ CUtensorMap tm_xl, int n_rows, int n_tok, int K,
                    float* __restrict__ Y, int ldy, size_t part_stride,
                    const uint16_t* __restrict__ bias, int32_t* __restrict__ err,
                    const float* __restrict__ tok_ss, int norm_len, float norm_eps) {
-  using S = GemmSmem<BN, STAGES>;
+  using S = GemmSmem<BN, STAGES, HL>;
   // The swizzled tiles must start on 1024-byte boundaries of the shared
   // window: round the dynamic base up (the launch adds 1 KB of slack).
   extern __shared__ __align__(16) uint8_t gsm_raw[];
@@ -112,11 +117,24 @@ __global__ void __launch_bounds__(128, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = s.tmem;
+  pdl_trigger();
   if (warp == 0 && lane == 0) {
-    int issued = 0;
-    for (int i = 0; i < nk; ++i) {
+    // The weight tiles of the first STAGES stages do not depend on the
+    // previous kernel: they are requested before waiting for it.
+    const int pre = nk < STAGES ? nk : STAGES;
+    for (int i = 0; i < pre; ++i) {
+      mbar_arrive_expect_tx(&s.full[i], S::kStageBytes);
+      tma_load_2d(s.a[i], &tm_w, (kb0 + i) * kGK, m0, &s.full[i]);
+    }
+    pdl_wait();
+    for (int i = 0; i < pre; ++i) {
+      tma_load_2d(s.bh[i], &tm_xh, (kb0 + i) * kGK, n0, &s.full[i]);
+      if constexpr (!HL) tma_load_2d(s.bl[i], &tm_xl, (kb0 + i) * kGK, n0, &s.full[i]);
+    }
+    int issued = pre;
+    for (int i = pre; i < nk; ++i) {
       const int st = i % STAGES;
-      if (i >= STAGES && !gemm_wait(&s.empty[st], ((i / STAGES) - 1) & 1)) {
+      if (!gemm_wait(&s.empty[st], ((i / STAGES) - 1) & 1)) {
         s.failed = 1;
         break;
       }
@@ -124,7 +142,7 @@ __global__ void __launch_bounds__(128, 1)
       mbar_arrive_expect_tx(&s.full[st], S::kStageBytes);
       tma_load_2d(s.a[st], &tm_w, kc, m0, &s.full[st]);
       tma_load_2d(s.bh[st], &tm_xh, kc, n0, &s.full[st]);
-      tma_load_2d(s.bl[st], &tm_xl, kc, n0, &s.full[st]);
+      if constexpr (!HL) tma_load_2d(s.bl[st], &tm_xl, kc, n0, &s.full[st]);
       issued = i + 1;
     }
     // every load must land before this CTA may exit
@@ -141,12 +159,11 @@ __global__ void __launch_bounds__(128, 1)
       tc_fence_after_sync();
       const uint64_t da = sw128_kmajor_desc(s.a[st]);
       const uint64_t dh = sw128_kmajor_desc(s.bh[st]);
-      const uint64_t dl = sw128_kmajor_desc(s.bl[st]);
 #pragma unroll
       for (int k = 0; k < kGK / 16; ++k) {
         // +2 in the address field = 32 bytes = 16 bf16 along K
         tc_mma_f16(tmem, da + 2 * k, dh + 2 * k, idesc, (i | k) != 0);
-        tc_mma_f16(tmem, da + 2 * k, dl + 2 * k, idesc, 1u);
+        if constexpr (!HL) tc_mma_f16(tmem, da + 2 * k, sw128_kmajor_desc(s.bl[st]) + 2 * k, idesc, 1u);
       }
       tc_commit(&s.empty[st]);
     }
@@ -156,22 +173,37 @@ __global__ void __launch_bounds__(128, 1)
   // Accumulator ready (or the issuing stopped): every warp waits on `done`.
   const bool ok = gemm_wait(&s.done, 0);
   tc_fence_after_sync();
+  pdl_wait();  // (returned long ago in the producer) before writing Y
   __syncthreads();
   if (ok && !s.failed && nk > 0) {
     const int row = m0 + warp * 32 + lane;
     const float b = (bias && row < n_rows) ? __uint_as_float((uint32_t)bias[row] << 16) : 0.f;
-#pragma unroll 1
-    for (int c0 = 0; c0 < BN; c0 += 16) {
+    if constexpr (HL) {
       float v[16];
-      tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
+      tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16), v);
       if (row < n_rows) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int tok = n0 + c0 + j;
-          if (tok < n_tok) {
-            // deferred RMSNorm: the input was x * w, its scale 1/rms applies here
-            const float sc = tok_ss ? 1.0f / sqrtf(tok_ss[tok] / (float)norm_len + norm_eps) : 1.0f;
-            Y[(size_t)tok * ldy + row] = v[j] * sc + b;
+        for (int j = 0; j < BN / 2; ++j) {
+          if (j < n_tok) {
+            const float sc = tok_ss ? 1.0f / sqrtf(tok_ss[j] / (float)norm_len + norm_eps) : 1.0f;
+            Y[(size_t)j * ldy + row] = (v[j] + v[j + BN / 2]) * sc + b;
+          }
+        }
+      }
+    } else {
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 16) {
+        float v[16];
+        tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
+        if (row < n_rows) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int tok = n0 + c0 + j;
+            if (tok < n_tok) {
+              // deferred RMSNorm: the input was x * w, its scale 1/rms applies here
+              const float sc = tok_ss ? 1.0f / sqrtf(tok_ss[tok] / (float)norm_len + norm_eps) : 1.0f;
+              Y[(size_t)tok * ldy + row] = v[j] * sc + b;
+            }
           }
         }
       }
@@ -238,6 +270,8 @@ __global__ void rope_kv_kernel(const float* __restrict__ y, int ldy, int nparts,
                                const uint16_t* __restrict__ bias, const int32_t* __restrict__ slot,
                                const int32_t* __restrict__ pos, ModelDev m, int layer,
                                float* __restrict__ qout) {
+  pdl_trigger();
+  pdl_wait();
   const int t = blockIdx.x;
   const int d = m.head_dim, G = m.group, half = d >> 1;
   const int npairs = qkv_rows(m.n_q, m.n_kv, d) >> 1;
@@ -436,6 +470,8 @@ template <int DPL, int G>
 __global__ void __launch_bounds__(kBAWarps * 32, 1)
     batch_attn_kernel(const float* __restrict__ q, const BatchParams* __restrict__ bp, ModelDev m,
                       int layer, int S, float* __restrict__ part) {
+  pdl_trigger();
+  pdl_wait();
   constexpr int d = DPL * 32, PS = d + 4;
   constexpr int kBuf = 2 * kBAKeys * d;  // bf16 elements per buffer (K then V)
   extern __shared__ __align__(16) uint8_t ba_raw[];
@@ -538,6 +574,8 @@ __global__ void __launch_bounds__(kBAWarps * 32, 1)
 __global__ void batch_attn_merge_kernel(const float* __restrict__ part, const BatchParams* __restrict__ bp,
                                         ModelDev m, int S, uint16_t* __restrict__ xh,
                                         uint16_t* __restrict__ xl) {
+  pdl_trigger();
+  pdl_wait();
   const int g = blockIdx.x, r = blockIdx.y;
   const int d = m.head_dim, G = m.group, PS = d + 4, nq = m.n_q;
   const int live = batch_live_splits(bp->pos[r] + 1, S);
@@ -584,6 +622,8 @@ __global__ void b_embed_norm_kernel(const uint16_t* __restrict__ E, const int32_
                                     float* __restrict__ x, uint16_t* __restrict__ xh,
                                     uint16_t* __restrict__ xl, float* __restrict__ tok_ss,
                                     int32_t* __restrict__ status) {
+  pdl_trigger();
+  pdl_wait();
   const int t = blockIdx.y;
   int tok = tokens[t];
   if (tok < 0 || tok >= vocab) {
@@ -607,6 +647,8 @@ __global__ void b_residual_norm_kernel(float* __restrict__ x, const float* __res
                                        int ldy, int nparts, size_t pstride,
                                        const uint16_t* __restrict__ w, uint16_t* __restrict__ xh,
                                        uint16_t* __restrict__ xl, float* __restrict__ tok_ss) {
+  pdl_trigger();
+  pdl_wait();
   const int t = blockIdx.y;
   float ss = 0.f;
   const int i0 = blockIdx.x * 1024 + threadIdx.x * 4;
@@ -624,6 +666,8 @@ __global__ void b_residual_norm_kernel(float* __restrict__ x, const float* __res
 // xh/xl[t][j] = split(silu(gate_j) * up_j), gate/up summed over the partials.
 __global__ void b_swiglu_kernel(const float* __restrict__ y, int ldy, int F, int nparts,
                                 size_t pstride, uint16_t* __restrict__ xh, uint16_t* __restrict__ xl) {
+  pdl_trigger();
+  pdl_wait();
   const int t = blockIdx.y;
   const int j0 = blockIdx.x * 1024 + threadIdx.x * 4;
   for (int j = j0; j < min(F, j0 + 4); ++j) {
@@ -641,6 +685,8 @@ __global__ void b_swiglu_kernel(const float* __restrict__ y, int ldy, int F, int
 // lowest index wins ties.  best[] starts at zero each step.
 __global__ void b_argmax_kernel(const float* __restrict__ logits, int V,
                                 unsigned long long* __restrict__ best) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ unsigned long long red[8];
   const int r = blockIdx.y;
   unsigned long long k = 0ull;
@@ -665,6 +711,8 @@ __global__ void b_argmax_kernel(const float* __restrict__ logits, int V,
 }
 
 __global__ void b_ids_kernel(const unsigned long long* __restrict__ best, int n, int32_t* __restrict__ ids) {
+  pdl_trigger();
+  pdl_wait();
   const int r = threadIdx.x;
   if (r < n) ids[r] = (int32_t)(0xffffffffu - (uint32_t)(best[r] & 0xffffffffull));
 }
@@ -694,6 +742,25 @@ __global__ void argmax_rows_kernel(const float* __restrict__ logits, int V, int3
 }
 
 // ------------------------------------------------------------------ host
+
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel of the stream runs; it calls pdl_wait() before reading
+// that kernel's results (the kernels above all do).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, args...);
+}
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -725,21 +792,46 @@ bool make_map(CUtensorMap* map, const void* base, int rows, int cols, int box_ro
 template <int BN, int STAGES>
 std::string gemm(const uint16_t* W, int n_rows, int K, const uint16_t* xh, const uint16_t* xl,
                  int n_tok, float* Y, int ldy, const uint16_t* bias, int32_t* err, cudaStream_t st,
-                 int splits = 1, const float* tok_ss = nullptr, float norm_eps = 0.f) {
+                 int splits = 1, const float* tok_ss = nullptr, float norm_eps = 0.f,
+                 bool pdl = false) {
   CUtensorMap mw, mh, ml;
   if (!make_map(&mw, W, n_rows, K) || !make_map(&mh, xh, n_tok, K, BN) ||
       !make_map(&ml, xl, n_tok, K, BN))
     return "cuTensorMapEncodeTiled failed";
   const dim3 grid((n_rows + kGM - 1) / kGM, (n_tok + BN - 1) / BN, splits);
-  gemm_wx_kernel<BN, STAGES><<<grid, 128, gemm_smem_bytes<BN, STAGES>(), st>>>(
-      mw, mh, ml, n_rows, n_tok, K, Y, ldy, (size_t)n_tok * ldy, splits == 1 ? bias : nullptr, err,
-      tok_ss, K, norm_eps);
+  const uint16_t* b = splits == 1 ? bias : nullptr;
+  const size_t pst = (size_t)n_tok * ldy;
+  if (pdl) {
+    const cudaError_t le = launch_pdl(gemm_wx_kernel<BN, STAGES>, grid, dim3(128),
+                                      gemm_smem_bytes<BN, STAGES>(), st, mw, mh, ml, n_rows, n_tok, K,
+                                      Y, ldy, pst, b, err, tok_ss, K, norm_eps);
+    if (le != cudaSuccess) return std::string("GEMM launch: ") + cudaGetErrorString(le);
+  } else {
+    gemm_wx_kernel<BN, STAGES><<<grid, 128, gemm_smem_bytes<BN, STAGES>(), st>>>(
+        mw, mh, ml, n_rows, n_tok, K, Y, ldy, pst, b, err, tok_ss, K, norm_eps);
+  }
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? "" : std::string("GEMM launch: ") + cudaGetErrorString(e);
 }
 
 constexpr int kPBN = 128, kPStages = 4;   // prompt GEMM: 128 tokens per CTA
-constexpr int kDBN = 16, kDStages = 10;   // decode GEMM: up to 16 tokens (8 requests)
+constexpr int kDStages = 11;              // decode GEMM: 8 requests, high and low parts packed
+
+// Y (+ z * n_tok * ldy for split z) = W x^T for n_tok <= 8 tokens whose high
+// parts are rows 0..7 and low parts rows 8..15 of xhl ([16][K] bf16).
+std::string gemm_hl(const uint16_t* W, int n_rows, int K, const uint16_t* xhl, int n_tok, float* Y,
+                    int ldy, int32_t* err, cudaStream_t st, int splits, const float* tok_ss,
+                    float norm_eps) {
+  CUtensorMap mw, mh;
+  if (!make_map(&mw, W, n_rows, K) || !make_map(&mh, xhl, 16, K, 16))
+    return "cuTensorMapEncodeTiled failed";
+  const dim3 grid((n_rows + kGM - 1) / kGM, 1, splits);
+  const cudaError_t le = launch_pdl(gemm_wx_kernel<16, kDStages, true>, grid, dim3(128),
+                                    gemm_smem_bytes<16, kDStages, true>(), st, mw, mh, mh, n_rows,
+                                    n_tok, K, Y, ldy, (size_t)n_tok * ldy, (const uint16_t*)nullptr,
+                                    err, tok_ss, K, norm_eps);
+  return le == cudaSuccess ? "" : std::string("GEMM launch: ") + cudaGetErrorString(le);
+}
 
 template <int DPL, int G>
 std::string launch_attn(dim3 grid, cudaStream_t st, const float* q, const int32_t* tiles,
@@ -888,8 +980,7 @@ std::string launch_batch_attn(dim3 grid, cudaStream_t st, const float* q, const 
     return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) == cudaSuccess
                ? "" : "batched attention shared memory attribute";
   }
-  k<<<grid, kBAWarps * 32, smem, st>>>(q, bp, m, layer, S, part);
-  const cudaError_t e = cudaGetLastError();
+  const cudaError_t e = launch_pdl(k, grid, dim3(kBAWarps * 32), smem, st, q, bp, m, layer, S, part);
   return e == cudaSuccess ? "" : std::string("batched attention launch: ") + cudaGetErrorString(e);
 }
 
@@ -942,43 +1033,56 @@ std::string batch_enqueue(const ModelDev& m, const PrefillWeights& w, BatchScrat
   const int zg = split_k(2 * F, H, num_sms), zd = split_k(H, F, num_sms);
   std::string e;
   BatchParams* bp = bs.params;
+#define CKL(call)                                                                       \
+  do {                                                                                  \
+    const cudaError_t le_ = (call);                                                     \
+    if (le_ != cudaSuccess) return std::string("batched step launch: ") + cudaGetErrorString(le_); \
+  } while (0)
   const int hsl = (H + 1023) / 1024, fsl = (F + 1023) / 1024;
   const int psl = ((qkvR >> 1) + 255) / 256;
   // per-step accumulators: the norms' sums of squares, the argmax keys
   if (cudaMemsetAsync(bs.acc, 0, bs.acc_bytes, st) != cudaSuccess) return "batched step memset";
   float* ss = reinterpret_cast<float*>(bs.acc);                       // [2L + 1][kMaxBatch]
   unsigned long long* best = reinterpret_cast<unsigned long long*>(bs.acc) + (2 * L + 1) * kMaxBatch / 2 + 1;
+  // GEMM inputs: [16][K] per contraction, rows 0..7 the high parts, 8..15 the low parts
+  uint16_t* const xhl = bs.xh;
+  auto lo = [&](int K) { return xhl + (size_t)8 * K; };
   b_embed_norm_kernel<<<dim3(hsl, n), 256, 0, st>>>(m.embed, bs.tokens, H, m.vocab, m.attn_norm, bs.x,
-                                                    bs.xh, bs.xl, ss, m.status);
+                                                    xhl, lo(H), ss, m.status);
   for (int l = 0; l < L; ++l) {
     float* ss_attn = ss + (size_t)(2 * l) * kMaxBatch;
     float* ss_ffn = ss + (size_t)(2 * l + 1) * kMaxBatch;
     float* ss_next = ss + (size_t)(2 * l + 2) * kMaxBatch;
     const uint16_t* bias = m.qkv_bias ? m.bqkv + (size_t)l * qkvR : nullptr;
-    if (!(e = gemm<kDBN, kDStages>(w.qkv[l], qkvR, H, bs.xh, bs.xl, n, bs.y, ldy, nullptr, bs.err, st, zq,
-                                   ss_attn, m.rms_eps)).empty()) return e;
-    rope_kv_kernel<<<dim3(n, psl), 256, 0, st>>>(bs.y, ldy, zq, pstride, bias, bp->slot, bp->pos, m, l, bs.q);
+    if (!(e = gemm_hl(w.qkv[l], qkvR, H, xhl, n, bs.y, ldy, bs.err, st, zq, ss_attn, m.rms_eps)).empty())
+      return e;
+    CKL(launch_pdl(rope_kv_kernel, dim3(n, psl), dim3(256), 0, st, (const float*)bs.y, ldy, zq, pstride,
+                   bias, (const int32_t*)bp->slot, (const int32_t*)bp->pos, m, l, bs.q));
     if (!(e = batch_attn(dim3(bs.splits, m.n_kv, n), st, bs.q, bp, m, l, bs.splits, bs.part)).empty()) return e;
-    batch_attn_merge_kernel<<<dim3(m.n_kv, n), 256, 0, st>>>(bs.part, bp, m, bs.splits, bs.xh, bs.xl);
-    if (!(e = gemm<kDBN, kDStages>(w.o[l], H, qd, bs.xh, bs.xl, n, bs.y, ldy, nullptr, bs.err, st, zo)).empty()) return e;
-    b_residual_norm_kernel<<<dim3(hsl, n), 256, 0, st>>>(bs.x, bs.y, H, ldy, zo, pstride,
-                                                         m.ffn_norm + (size_t)l * H, bs.xh, bs.xl, ss_ffn);
-    if (!(e = gemm<kDBN, kDStages>(w.gu[l], 2 * F, H, bs.xh, bs.xl, n, bs.y, ldy, nullptr, bs.err, st, zg,
-                                   ss_ffn, m.rms_eps)).empty()) return e;
-    b_swiglu_kernel<<<dim3(fsl, n), 256, 0, st>>>(bs.y, ldy, F, zg, pstride, bs.xh, bs.xl);
-    if (!(e = gemm<kDBN, kDStages>(w.dn[l], H, F, bs.xh, bs.xl, n, bs.y, ldy, nullptr, bs.err, st, zd)).empty()) return e;
+    CKL(launch_pdl(batch_attn_merge_kernel, dim3(m.n_kv, n), dim3(256), 0, st, (const float*)bs.part,
+                   (const BatchParams*)bp, m, bs.splits, xhl, lo(qd)));
+    if (!(e = gemm_hl(w.o[l], H, qd, xhl, n, bs.y, ldy, bs.err, st, zo, nullptr, 0.f)).empty()) return e;
+    CKL(launch_pdl(b_residual_norm_kernel, dim3(hsl, n), dim3(256), 0, st, bs.x, (const float*)bs.y, H,
+                   ldy, zo, pstride, m.ffn_norm + (size_t)l * H, xhl, lo(H), ss_ffn));
+    if (!(e = gemm_hl(w.gu[l], 2 * F, H, xhl, n, bs.y, ldy, bs.err, st, zg, ss_ffn, m.rms_eps)).empty())
+      return e;
+    CKL(launch_pdl(b_swiglu_kernel, dim3(fsl, n), dim3(256), 0, st, (const float*)bs.y, ldy, F, zg,
+                   pstride, xhl, lo(F)));
+    if (!(e = gemm_hl(w.dn[l], H, F, xhl, n, bs.y, ldy, bs.err, st, zd, nullptr, 0.f)).empty()) return e;
     // the residual add, then the next layer's attention norm (the final norm after the last)
     const uint16_t* next_norm = l + 1 < L ? m.attn_norm + (size_t)(l + 1) * H : m.final_norm;
-    b_residual_norm_kernel<<<dim3(hsl, n), 256, 0, st>>>(bs.x, bs.y, H, ldy, zd, pstride, next_norm,
-                                                         bs.xh, bs.xl, ss_next);
+    CKL(launch_pdl(b_residual_norm_kernel, dim3(hsl, n), dim3(256), 0, st, bs.x, (const float*)bs.y, H,
+                   ldy, zd, pstride, next_norm, xhl, lo(H), ss_next));
   }
-  if (!(e = gemm<kDBN, kDStages>(m.lm_head, V, H, bs.xh, bs.xl, n, bs.logits, V, nullptr, bs.err, st, 1,
-                                 ss + (size_t)(2 * L) * kMaxBatch, m.rms_eps)).empty()) return e;
-  b_argmax_kernel<<<dim3((V + 4095) / 4096, n), 256, 0, st>>>(bs.logits, V, best);
-  b_ids_kernel<<<1, 32, 0, st>>>(best, n, bs.ids);
+  if (!(e = gemm_hl(m.lm_head, V, H, xhl, n, bs.logits, V, bs.err, st, 1,
+                    ss + (size_t)(2 * L) * kMaxBatch, m.rms_eps)).empty()) return e;
+  CKL(launch_pdl(b_argmax_kernel, dim3((V + 4095) / 4096, n), dim3(256), 0, st, (const float*)bs.logits,
+                 V, best));
+  CKL(launch_pdl(b_ids_kernel, dim3(1), dim3(32), 0, st, (const unsigned long long*)best, n, bs.ids));
   const cudaError_t ce = cudaGetLastError();
   return ce == cudaSuccess ? "" : std::string("batched step launch: ") + cudaGetErrorString(ce);
 }
+#undef CKL
 
 }  // namespace
 
@@ -998,8 +1102,7 @@ std::string batch_alloc(const ModelDev& m, int num_sms, BatchScratch* bs, std::v
       {(void**)&bs->y, (size_t)kBatchMaxSplitK * B * ycols * 4},
       {(void**)&bs->q, B * qd * 4},
       {(void**)&bs->part, B * m.n_kv * bs->splits * G * (d + 4) * 4},
-      {(void**)&bs->xh, B * xcols * 2},
-      {(void**)&bs->xl, B * xcols * 2},
+      {(void**)&bs->xh, 2 * B * xcols * 2},
       {(void**)&bs->logits, B * (size_t)m.vocab * 4},
       {(void**)&bs->ids, B * 4},
       {(void**)&bs->err, 16},
@@ -1010,8 +1113,9 @@ std::string batch_alloc(const ModelDev& m, int num_sms, BatchScratch* bs, std::v
     owned->push_back(*a.p);
   }
   cudaMemset(bs->err, 0, 16);
-  if (cudaFuncSetAttribute(gemm_wx_kernel<kDBN, kDStages>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)gemm_smem_bytes<kDBN, kDStages>()) != cudaSuccess)
+  cudaMemset(bs->xh, 0, 2 * B * xcols * 2);  // rows of absent requests stay finite
+  if (cudaFuncSetAttribute(gemm_wx_kernel<16, kDStages, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)gemm_smem_bytes<16, kDStages, true>()) != cudaSuccess)
     return "decode GEMM shared memory attribute";
   return batch_attn(dim3(1), nullptr, nullptr, nullptr, m, 0, bs->splits, nullptr, true);
 }

@@ -51,8 +51,7 @@ struct BatchScratch {
   float* y = nullptr;          // [kBatchMaxSplitK][kMaxBatch][max(qkv rows, 2 ffn, hidden)]
   float* q = nullptr;          // [kMaxBatch][n_q * d]
   float* part = nullptr;       // [kMaxBatch][n_kv][splits][G][d + 4] attention partials
-  uint16_t* xh = nullptr;      // [kMaxBatch][max(hidden, ffn, n_q*d)]
-  uint16_t* xl = nullptr;
+  uint16_t* xh = nullptr;      // [2 kMaxBatch][K] GEMM input: high parts, then low parts
   float* logits = nullptr;     // [kMaxBatch][vocab]
   int32_t* ids = nullptr;      // [kMaxBatch]
   int32_t* err = nullptr;

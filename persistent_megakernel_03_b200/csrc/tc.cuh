@@ -103,4 +103,12 @@ __host__ __device__ constexpr uint32_t mma_idesc_bf16_f32(int M, int N) {
          ((uint32_t)(M >> 4) << 24);
 }
 
+// Programmatic dependent launch: let the next kernel of the stream start its
+// independent prologue now / wait until the previous kernel has completed
+// and its writes are visible.  Both are no-ops for a normal launch.
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 }  // namespace mk
