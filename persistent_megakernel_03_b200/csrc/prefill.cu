@@ -33,6 +33,19 @@ namespace mk {
 
 namespace {
 
+__device__ __forceinline__ uint16_t bf16_bits(float f) {
+  __nv_bfloat16 b = __float2bfloat16_rn(f);
+  return *reinterpret_cast<uint16_t*>(&b);
+}
+__device__ __forceinline__ float bf16_val(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
+
+// v -> (bf16(v), bf16(v - bf16(v)))
+__device__ __forceinline__ void split_store(float v, uint16_t* hi, uint16_t* lo, size_t i) {
+  const uint16_t h = bf16_bits(v);
+  hi[i] = h;
+  lo[i] = bf16_bits(v - bf16_val(h));
+}
+
 // ------------------------------------------------------------------ GEMM
 // Y[t][r] = sum_k W[r][k] * (xh[t][k] + xl[t][k]) for 128 weight rows and BN
 // tokens per CTA, K blocks [z*nk/Z, (z+1)*nk/Z) of a Z-way split (gridDim.z;
@@ -87,7 +100,8 @@ __global__ void __launch_bounds__(128, 1)
                    const __grid_constant__ CUtensorMap tm_xl, int n_rows, int n_tok, int K,
                    float* __restrict__ Y, int ldy, size_t part_stride,
                    const uint16_t* __restrict__ bias, int32_t* __restrict__ err,
-                   const float* __restrict__ tok_ss, int norm_len, float norm_eps) {
+                   const float* __restrict__ tok_ss, int norm_len, float norm_eps,
+                   uint16_t* __restrict__ act_hl, int act_ld) {
   using S = GemmSmem<BN, STAGES, HL>;
   // The swizzled tiles must start on 1024-byte boundaries of the shared
   // window: round the dynamic base up (the launch adds 1 KB of slack).
@@ -181,7 +195,20 @@ __global__ void __launch_bounds__(128, 1)
     if constexpr (HL) {
       float v[16];
       tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16), v);
-      if (row < n_rows) {
+      if (act_hl) {
+        // gate/up rows 2j, 2j+1 sit in adjacent lanes: the even lane forms
+        // silu(gate) * up and writes it as the next GEMM's split input
+#pragma unroll
+        for (int j = 0; j < BN / 2; ++j) {
+          const bool live = row < n_rows && j < n_tok;
+          const float sc = (live && tok_ss) ? 1.0f / sqrtf(tok_ss[j] / (float)norm_len + norm_eps) : 1.0f;
+          const float yv = live ? (v[j] + v[j + BN / 2]) * sc + b : 0.f;
+          const float up = __shfl_xor_sync(0xffffffffu, yv, 1);
+          if (live && !(lane & 1))
+            split_store(yv / (1.0f + expf(-yv)) * up, act_hl, act_hl + (size_t)(BN / 2) * act_ld,
+                        (size_t)j * act_ld + (row >> 1));
+        }
+      } else if (row < n_rows) {
 #pragma unroll
         for (int j = 0; j < BN / 2; ++j) {
           if (j < n_tok) {
@@ -217,19 +244,6 @@ __global__ void __launch_bounds__(128, 1)
 }
 
 // ------------------------------------------------------- small operators
-
-__device__ __forceinline__ uint16_t bf16_bits(float f) {
-  __nv_bfloat16 b = __float2bfloat16_rn(f);
-  return *reinterpret_cast<uint16_t*>(&b);
-}
-__device__ __forceinline__ float bf16_val(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
-
-// v -> (bf16(v), bf16(v - bf16(v)))
-__device__ __forceinline__ void split_store(float v, uint16_t* hi, uint16_t* lo, size_t i) {
-  const uint16_t h = bf16_bits(v);
-  hi[i] = h;
-  lo[i] = bf16_bits(v - bf16_val(h));
-}
 
 // x[t] = E[token of t] (fp32).  meta_tok: index into tokens_dev per token.
 __global__ void embed_kernel(const uint16_t* __restrict__ E, const int32_t* __restrict__ tokens,
@@ -469,7 +483,8 @@ __device__ __forceinline__ int batch_live_splits(int n_keys, int S) {
 template <int DPL, int G>
 __global__ void __launch_bounds__(kBAWarps * 32, 1)
     batch_attn_kernel(const float* __restrict__ q, const BatchParams* __restrict__ bp, ModelDev m,
-                      int layer, int S, float* __restrict__ part) {
+                      int layer, int S, float* __restrict__ part, uint32_t* __restrict__ tickets,
+                      uint16_t* __restrict__ xh, uint16_t* __restrict__ xl) {
   pdl_trigger();
   pdl_wait();
   constexpr int d = DPL * 32, PS = d + 4;
@@ -552,6 +567,25 @@ __global__ void __launch_bounds__(kBAWarps * 32, 1)
     }
   }
   __syncthreads();
+  const size_t out_row = (size_t)r * nq * d + (size_t)g * G * d;
+  if (live == 1) {
+    // the only split: normalise and write the O projection's input directly
+    for (int idx = threadIdx.x; idx < G * d; idx += blockDim.x) {
+      const int h = idx / d, i = idx - h * d;
+      float M = -INFINITY;
+      for (int w = 0; w < kBAWarps; ++w) M = fmaxf(M, ws[(w * G + h) * PS + d]);
+      float num = 0.f, den = 0.f;
+      for (int w = 0; w < kBAWarps; ++w) {
+        const float mw = ws[(w * G + h) * PS + d];
+        if (mw == -INFINITY) continue;
+        const float c = __expf(mw - M);
+        num = fmaf(c, ws[(w * G + h) * PS + i], num);
+        den = fmaf(c, ws[(w * G + h) * PS + d + 1], den);
+      }
+      split_store(num / den, xh, xl, out_row + (size_t)h * d + i);
+    }
+    return;
+  }
   float* dst = part + ((size_t)(r * m.n_kv + g) * S + sp) * G * PS;
   for (int idx = threadIdx.x; idx < G * (d + 2); idx += blockDim.x) {
     const int h = idx / (d + 2), i = idx - h * (d + 2);
@@ -567,36 +601,38 @@ __global__ void __launch_bounds__(kBAWarps * 32, 1)
       }
     dst[h * PS + i] = i == d ? M : val;
   }
-}
-
-// Merges the live splits of (KV head g, request r) and writes the attention
-// output, normalised, as the O projection's [xh, xl] input.
-__global__ void batch_attn_merge_kernel(const float* __restrict__ part, const BatchParams* __restrict__ bp,
-                                        ModelDev m, int S, uint16_t* __restrict__ xh,
-                                        uint16_t* __restrict__ xl) {
-  pdl_trigger();
-  pdl_wait();
-  const int g = blockIdx.x, r = blockIdx.y;
-  const int d = m.head_dim, G = m.group, PS = d + 4, nq = m.n_q;
-  const int live = batch_live_splits(bp->pos[r] + 1, S);
+  // The last of the live splits of (request, KV head) merges them (the
+  // ticket counts the splits of this step and is put back to zero by the
+  // last one; the next step reaches it only after this kernel completes).
+  __shared__ int is_last;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();  // this split's partial before the ticket
+    const unsigned old = atomicAdd(tickets + r * m.n_kv + g, 1u);
+    is_last = old == (unsigned)live - 1u;
+    if (is_last) tickets[r * m.n_kv + g] = 0u;
+  }
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();  // the other splits' partials, after their tickets
   const float* pg = part + (size_t)(r * m.n_kv + g) * S * G * PS;
   for (int idx = threadIdx.x; idx < G * d; idx += blockDim.x) {
     const int h = idx / d, i = idx - h * d;
     float M = -INFINITY;
     for (int s2 = 0; s2 < live; ++s2) {
       const float* ps = pg + ((size_t)s2 * G + h) * PS;
-      if (ps[d + 1] != 0.f) M = fmaxf(M, ps[d]);
+      if (__ldcg(ps + d + 1) != 0.f) M = fmaxf(M, __ldcg(ps + d));
     }
     float num = 0.f, den = 0.f;
     for (int s2 = 0; s2 < live; ++s2) {
       const float* ps = pg + ((size_t)s2 * G + h) * PS;
-      const float ls = ps[d + 1];
+      const float ls = __ldcg(ps + d + 1);
       if (ls == 0.f) continue;
-      const float c = __expf(ps[d] - M);
-      num = fmaf(c, ps[i], num);
+      const float c = __expf(__ldcg(ps + d) - M);
+      num = fmaf(c, __ldcg(ps + i), num);
       den = fmaf(c, ls, den);
     }
-    split_store(num / den, xh, xl, (size_t)r * nq * d + (size_t)(g * G + h) * d + i);
+    split_store(num / den, xh, xl, out_row + (size_t)h * d + i);
   }
 }
 
@@ -717,29 +753,6 @@ __global__ void b_ids_kernel(const unsigned long long* __restrict__ best, int n,
   if (r < n) ids[r] = (int32_t)(0xffffffffu - (uint32_t)(best[r] & 0xffffffffull));
 }
 
-// Greedy id of each request: the largest logit, the lowest index on ties.
-__global__ void argmax_rows_kernel(const float* __restrict__ logits, int V, int32_t* __restrict__ ids) {
-  __shared__ unsigned long long red[32];
-  const int r = blockIdx.x;
-  unsigned long long best = 0ull;
-  for (int i = threadIdx.x; i < V; i += blockDim.x) {
-    uint32_t u = __float_as_uint(logits[(size_t)r * V + i]);
-    u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-    const unsigned long long k = ((unsigned long long)u << 32) | (0xffffffffu - (uint32_t)i);
-    best = k > best ? k : best;
-  }
-  for (int o = 16; o; o >>= 1) {
-    const unsigned long long v = __shfl_xor_sync(0xffffffffu, best, o);
-    best = v > best ? v : best;
-  }
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = best;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) best = red[w] > best ? red[w] : best;
-    best = red[0] > best ? red[0] : best;
-    ids[r] = (int32_t)(0xffffffffu - (uint32_t)(best & 0xffffffffull));
-  }
-}
 
 // ------------------------------------------------------------------ host
 
@@ -804,11 +817,11 @@ std::string gemm(const uint16_t* W, int n_rows, int K, const uint16_t* xh, const
   if (pdl) {
     const cudaError_t le = launch_pdl(gemm_wx_kernel<BN, STAGES>, grid, dim3(128),
                                       gemm_smem_bytes<BN, STAGES>(), st, mw, mh, ml, n_rows, n_tok, K,
-                                      Y, ldy, pst, b, err, tok_ss, K, norm_eps);
+                                      Y, ldy, pst, b, err, tok_ss, K, norm_eps, (uint16_t*)nullptr, 0);
     if (le != cudaSuccess) return std::string("GEMM launch: ") + cudaGetErrorString(le);
   } else {
     gemm_wx_kernel<BN, STAGES><<<grid, 128, gemm_smem_bytes<BN, STAGES>(), st>>>(
-        mw, mh, ml, n_rows, n_tok, K, Y, ldy, pst, b, err, tok_ss, K, norm_eps);
+        mw, mh, ml, n_rows, n_tok, K, Y, ldy, pst, b, err, tok_ss, K, norm_eps, nullptr, 0);
   }
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? "" : std::string("GEMM launch: ") + cudaGetErrorString(e);
@@ -819,9 +832,11 @@ constexpr int kDStages = 11;              // decode GEMM: 8 requests, high and l
 
 // Y (+ z * n_tok * ldy for split z) = W x^T for n_tok <= 8 tokens whose high
 // parts are rows 0..7 and low parts rows 8..15 of xhl ([16][K] bf16).
+// act_hl (with splits == 1): instead of Y, write silu(gate) * up of the
+// interleaved gate/up rows as the next GEMM's [16][n_rows / 2] split input.
 std::string gemm_hl(const uint16_t* W, int n_rows, int K, const uint16_t* xhl, int n_tok, float* Y,
                     int ldy, int32_t* err, cudaStream_t st, int splits, const float* tok_ss,
-                    float norm_eps) {
+                    float norm_eps, uint16_t* act_hl = nullptr) {
   CUtensorMap mw, mh;
   if (!make_map(&mw, W, n_rows, K) || !make_map(&mh, xhl, 16, K, 16))
     return "cuTensorMapEncodeTiled failed";
@@ -829,7 +844,7 @@ std::string gemm_hl(const uint16_t* W, int n_rows, int K, const uint16_t* xhl, i
   const cudaError_t le = launch_pdl(gemm_wx_kernel<16, kDStages, true>, grid, dim3(128),
                                     gemm_smem_bytes<16, kDStages, true>(), st, mw, mh, mh, n_rows,
                                     n_tok, K, Y, ldy, (size_t)n_tok * ldy, (const uint16_t*)nullptr,
-                                    err, tok_ss, K, norm_eps);
+                                    err, tok_ss, K, norm_eps, act_hl, n_rows / 2);
   return le == cudaSuccess ? "" : std::string("GEMM launch: ") + cudaGetErrorString(le);
 }
 
@@ -973,21 +988,25 @@ size_t batch_attn_smem() {
 
 template <int DPL, int G>
 std::string launch_batch_attn(dim3 grid, cudaStream_t st, const float* q, const BatchParams* bp,
-                              const ModelDev& m, int layer, int S, float* part, bool set_attr) {
+                              const ModelDev& m, int layer, int S, float* part, bool set_attr,
+                              uint32_t* tickets, uint16_t* xh, uint16_t* xl) {
   auto k = batch_attn_kernel<DPL, G>;
   const size_t smem = batch_attn_smem<DPL, G>();
   if (set_attr) {
     return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) == cudaSuccess
                ? "" : "batched attention shared memory attribute";
   }
-  const cudaError_t e = launch_pdl(k, grid, dim3(kBAWarps * 32), smem, st, q, bp, m, layer, S, part);
+  const cudaError_t e = launch_pdl(k, grid, dim3(kBAWarps * 32), smem, st, q, bp, m, layer, S, part,
+                                   tickets, xh, xl);
   return e == cudaSuccess ? "" : std::string("batched attention launch: ") + cudaGetErrorString(e);
 }
 
 std::string batch_attn(dim3 grid, cudaStream_t st, const float* q, const BatchParams* bp,
-                       const ModelDev& m, int layer, int S, float* part, bool set_attr = false) {
+                       const ModelDev& m, int layer, int S, float* part, bool set_attr = false,
+                       uint32_t* tickets = nullptr, uint16_t* xh = nullptr, uint16_t* xl = nullptr) {
   const int G = m.group;
-#define MK_BA(DPL_, G_) return launch_batch_attn<DPL_, G_>(grid, st, q, bp, m, layer, S, part, set_attr)
+#define MK_BA(DPL_, G_) \
+  return launch_batch_attn<DPL_, G_>(grid, st, q, bp, m, layer, S, part, set_attr, tickets, xh, xl)
   if (m.head_dim == 128) {
     if (G == 1) MK_BA(4, 1);
     if (G == 2) MK_BA(4, 2);
@@ -1058,17 +1077,24 @@ std::string batch_enqueue(const ModelDev& m, const PrefillWeights& w, BatchScrat
       return e;
     CKL(launch_pdl(rope_kv_kernel, dim3(n, psl), dim3(256), 0, st, (const float*)bs.y, ldy, zq, pstride,
                    bias, (const int32_t*)bp->slot, (const int32_t*)bp->pos, m, l, bs.q));
-    if (!(e = batch_attn(dim3(bs.splits, m.n_kv, n), st, bs.q, bp, m, l, bs.splits, bs.part)).empty()) return e;
-    CKL(launch_pdl(batch_attn_merge_kernel, dim3(m.n_kv, n), dim3(256), 0, st, (const float*)bs.part,
-                   (const BatchParams*)bp, m, bs.splits, xhl, lo(qd)));
+    if (!(e = batch_attn(dim3(bs.splits, m.n_kv, n), st, bs.q, bp, m, l, bs.splits, bs.part, false,
+                         bs.tickets, xhl, lo(qd))).empty())
+      return e;
     if (!(e = gemm_hl(w.o[l], H, qd, xhl, n, bs.y, ldy, bs.err, st, zo, nullptr, 0.f)).empty()) return e;
     CKL(launch_pdl(b_residual_norm_kernel, dim3(hsl, n), dim3(256), 0, st, bs.x, (const float*)bs.y, H,
                    ldy, zo, pstride, m.ffn_norm + (size_t)l * H, xhl, lo(H), ss_ffn));
-    if (!(e = gemm_hl(w.gu[l], 2 * F, H, xhl, n, bs.y, ldy, bs.err, st, zg, ss_ffn, m.rms_eps)).empty())
-      return e;
-    CKL(launch_pdl(b_swiglu_kernel, dim3(fsl, n), dim3(256), 0, st, (const float*)bs.y, ldy, F, zg,
-                   pstride, xhl, lo(F)));
-    if (!(e = gemm_hl(w.dn[l], H, F, xhl, n, bs.y, ldy, bs.err, st, zd, nullptr, 0.f)).empty()) return e;
+    // SwiGLU output into a second buffer: the gate/up GEMM still reads xhl
+    if (zg == 1) {  // in the GEMM's epilogue
+      if (!(e = gemm_hl(w.gu[l], 2 * F, H, xhl, n, bs.y, ldy, bs.err, st, 1, ss_ffn, m.rms_eps,
+                        bs.xh2)).empty())
+        return e;
+    } else {
+      if (!(e = gemm_hl(w.gu[l], 2 * F, H, xhl, n, bs.y, ldy, bs.err, st, zg, ss_ffn, m.rms_eps)).empty())
+        return e;
+      CKL(launch_pdl(b_swiglu_kernel, dim3(fsl, n), dim3(256), 0, st, (const float*)bs.y, ldy, F, zg,
+                     pstride, bs.xh2, bs.xh2 + (size_t)8 * F));
+    }
+    if (!(e = gemm_hl(w.dn[l], H, F, bs.xh2, n, bs.y, ldy, bs.err, st, zd, nullptr, 0.f)).empty()) return e;
     // the residual add, then the next layer's attention norm (the final norm after the last)
     const uint16_t* next_norm = l + 1 < L ? m.attn_norm + (size_t)(l + 1) * H : m.final_norm;
     CKL(launch_pdl(b_residual_norm_kernel, dim3(hsl, n), dim3(256), 0, st, bs.x, (const float*)bs.y, H,
@@ -1103,6 +1129,8 @@ std::string batch_alloc(const ModelDev& m, int num_sms, BatchScratch* bs, std::v
       {(void**)&bs->q, B * qd * 4},
       {(void**)&bs->part, B * m.n_kv * bs->splits * G * (d + 4) * 4},
       {(void**)&bs->xh, 2 * B * xcols * 2},
+      {(void**)&bs->xh2, 2 * B * xcols * 2},
+      {(void**)&bs->tickets, B * m.n_kv * 4},
       {(void**)&bs->logits, B * (size_t)m.vocab * 4},
       {(void**)&bs->ids, B * 4},
       {(void**)&bs->err, 16},
@@ -1114,6 +1142,8 @@ std::string batch_alloc(const ModelDev& m, int num_sms, BatchScratch* bs, std::v
   }
   cudaMemset(bs->err, 0, 16);
   cudaMemset(bs->xh, 0, 2 * B * xcols * 2);  // rows of absent requests stay finite
+  cudaMemset(bs->xh2, 0, 2 * B * xcols * 2);
+  cudaMemset(bs->tickets, 0, B * m.n_kv * 4);
   if (cudaFuncSetAttribute(gemm_wx_kernel<16, kDStages, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)gemm_smem_bytes<16, kDStages, true>()) != cudaSuccess)
     return "decode GEMM shared memory attribute";

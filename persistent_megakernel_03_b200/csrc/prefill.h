@@ -52,6 +52,8 @@ struct BatchScratch {
   float* q = nullptr;          // [kMaxBatch][n_q * d]
   float* part = nullptr;       // [kMaxBatch][n_kv][splits][G][d + 4] attention partials
   uint16_t* xh = nullptr;      // [2 kMaxBatch][K] GEMM input: high parts, then low parts
+  uint16_t* xh2 = nullptr;     // the same for the SwiGLU output (the down projection's input)
+  uint32_t* tickets = nullptr; // [kMaxBatch][n_kv] attention split-merge tickets
   float* logits = nullptr;     // [kMaxBatch][vocab]
   int32_t* ids = nullptr;      // [kMaxBatch]
   int32_t* err = nullptr;
