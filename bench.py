@@ -220,7 +220,9 @@ def run_mk(args):
 
     rank, world, local = dist_setup(args.gpus)
     torch.cuda.set_device(local)
-    model = synth.LLAMA8B
+    model = synth.QWEN05B if args.workload == "qwen05b" else synth.LLAMA8B
+    shape = "qwen2.5-0.5b-shape" if args.workload == "qwen05b" else "llama-3-8b-shape"
+    shape_cap = "Qwen2.5-0.5B-shape" if args.workload == "qwen05b" else "Llama-3-8B-shape"
     if args.layers:
         model = model.with_layers(args.layers)
     W, K = args.warmup, args.steps
@@ -231,7 +233,7 @@ def run_mk(args):
     else:
         lens = [SHORT_PROMPT]
     n = len(lens)
-    if args.workload != "llama8b" and W + K > LONG_STEPS:
+    if args.workload in ("llama8b-32k", "llama8b-batch8") and W + K > LONG_STEPS:
         K = LONG_STEPS - W   # these workloads decode 256 steps after their prompts
     max_seq = max(lens) + W + K + 1
     w = synth.make_model(model, 0, device="cuda")
@@ -371,9 +373,11 @@ def run_mk(args):
 
     clocks = clk.summary()
     if n == 1:
-        workload = (f"llama-3-8b-shape decode, batch 1, {lens[0]}-token random prompt, "
+        workload = (f"{shape} decode, batch 1, {lens[0]}-token random prompt, "
                     f"greedy decode steps {lens[0] + W}..{lens[0] + W + K - 1} timed")
-        unit, metric = "ms/token", METRIC
+        unit = "ms/token"
+        metric = METRIC if model.name.startswith("llama") else (
+            f"decode ms/token (batch 1, {shape_cap}) & achieved HBM GB/s vs 8 TB/s peak")
     else:
         workload = (f"llama-3-8b-shape decode, {n} requests per step, random prompts of "
                     f"{lens} tokens packed with offsets, greedy decode steps {W}..{W + K - 1} "
@@ -386,7 +390,8 @@ def run_mk(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "weights": "bf16",
         "data": "synthetic",
         "config": {"workload": workload,
-                   "l2": "inputs larger than L2 (15.0 GB of weights streamed per step)",
+                   "l2": (f"inputs larger than L2 ({roofline.weight_bytes(model) / 1e9:.2f} GB of "
+                          "weights streamed per step)"),
                    "parallelism": f"replicas x{world}"},
         "tok_per_s": 1e3 * n / value,
         "step_ms": {"median": statistics.median(per_step),
@@ -429,7 +434,7 @@ def run_mk(args):
         p0 = first_pos + len(times) - len(timed)
         line["cpu_baseline"] = {
             "value": cms, "unit": unit, "cores": cores, "kind": "oracle",
-            "sample": f"{len(timed)} oracle decode steps of the same Llama-3-8B-shape model "
+            "sample": f"{len(timed)} oracle decode steps of the same {shape_cap} model "
                       f"at positions {p0}..{first_pos + len(times) - 1}, fp32 with "
                       f"bf16 weights widened on the fly"
                       + (" (cache of the earlier positions filled with random bf16 values: "
@@ -462,10 +467,11 @@ def main():
     ap.add_argument("--l2-prefetch", type=int, default=0,
                     help="ring chunks prefetched into L2 beyond the ring (0: library default)")
     ap.add_argument("--workload", default="llama8b",
-                    choices=["llama8b", "llama8b-32k", "llama8b-batch8"],
+                    choices=["llama8b", "llama8b-32k", "llama8b-batch8", "qwen05b"],
                     help="llama8b: 39-token prompt (default); llama8b-32k: 32768-token "
                          "prompt; llama8b-batch8: 8 requests with prompts of U[32, 2048] "
-                         "tokens (the last two decode at most 256 steps)")
+                         "tokens (these two decode at most 256 steps); qwen05b: the "
+                         "Qwen2.5-0.5B shape, 39-token prompt")
     ap.add_argument("--layers", type=int, default=0,
                     help="profiling aid: a shallower model of the same widths (not a bench line)")
     args = ap.parse_args()

@@ -834,17 +834,27 @@ constexpr int kDStages = 11;              // decode GEMM: 8 requests, high and l
 // parts are rows 0..7 and low parts rows 8..15 of xhl ([16][K] bf16).
 // act_hl (with splits == 1): instead of Y, write silu(gate) * up of the
 // interleaved gate/up rows as the next GEMM's [16][n_rows / 2] split input.
+// two_per_sm: 6 stages (108 KB) so that two CTAs share an SM -- for a matrix
+// whose 128-row tiles number between one and two waves of SMs, all of them
+// then start at once instead of a full wave and a partial one.
+constexpr int kDStagesPair = 6;
 std::string gemm_hl(const uint16_t* W, int n_rows, int K, const uint16_t* xhl, int n_tok, float* Y,
                     int ldy, int32_t* err, cudaStream_t st, int splits, const float* tok_ss,
-                    float norm_eps, uint16_t* act_hl = nullptr) {
+                    float norm_eps, uint16_t* act_hl = nullptr, bool two_per_sm = false) {
   CUtensorMap mw, mh;
   if (!make_map(&mw, W, n_rows, K) || !make_map(&mh, xhl, 16, K, 16))
     return "cuTensorMapEncodeTiled failed";
   const dim3 grid((n_rows + kGM - 1) / kGM, 1, splits);
-  const cudaError_t le = launch_pdl(gemm_wx_kernel<16, kDStages, true>, grid, dim3(128),
-                                    gemm_smem_bytes<16, kDStages, true>(), st, mw, mh, mh, n_rows,
-                                    n_tok, K, Y, ldy, (size_t)n_tok * ldy, (const uint16_t*)nullptr,
-                                    err, tok_ss, K, norm_eps, act_hl, n_rows / 2);
+  const cudaError_t le =
+      two_per_sm
+          ? launch_pdl(gemm_wx_kernel<16, kDStagesPair, true>, grid, dim3(128),
+                       gemm_smem_bytes<16, kDStagesPair, true>(), st, mw, mh, mh, n_rows, n_tok, K, Y,
+                       ldy, (size_t)n_tok * ldy, (const uint16_t*)nullptr, err, tok_ss, K, norm_eps,
+                       act_hl, n_rows / 2)
+          : launch_pdl(gemm_wx_kernel<16, kDStages, true>, grid, dim3(128),
+                       gemm_smem_bytes<16, kDStages, true>(), st, mw, mh, mh, n_rows, n_tok, K, Y,
+                       ldy, (size_t)n_tok * ldy, (const uint16_t*)nullptr, err, tok_ss, K, norm_eps,
+                       act_hl, n_rows / 2);
   return le == cudaSuccess ? "" : std::string("GEMM launch: ") + cudaGetErrorString(le);
 }
 
@@ -1049,6 +1059,8 @@ std::string batch_enqueue(const ModelDev& m, const PrefillWeights& w, BatchScrat
   const int ldy = std::max(std::max(qkvR, 2 * F), H);
   const size_t pstride = (size_t)n * ldy;
   const int zq = split_k(qkvR, H, num_sms), zo = split_k(H, qd, num_sms);
+  const int gu_tiles = (2 * F + kGM - 1) / kGM;
+  const bool gu_pair = gu_tiles > num_sms && gu_tiles <= 2 * num_sms;
   const int zg = split_k(2 * F, H, num_sms), zd = split_k(H, F, num_sms);
   std::string e;
   BatchParams* bp = bs.params;
@@ -1086,7 +1098,7 @@ std::string batch_enqueue(const ModelDev& m, const PrefillWeights& w, BatchScrat
     // SwiGLU output into a second buffer: the gate/up GEMM still reads xhl
     if (zg == 1) {  // in the GEMM's epilogue
       if (!(e = gemm_hl(w.gu[l], 2 * F, H, xhl, n, bs.y, ldy, bs.err, st, 1, ss_ffn, m.rms_eps,
-                        bs.xh2)).empty())
+                        bs.xh2, gu_pair)).empty())
         return e;
     } else {
       if (!(e = gemm_hl(w.gu[l], 2 * F, H, xhl, n, bs.y, ldy, bs.err, st, zg, ss_ffn, m.rms_eps)).empty())
@@ -1145,7 +1157,10 @@ std::string batch_alloc(const ModelDev& m, int num_sms, BatchScratch* bs, std::v
   cudaMemset(bs->xh2, 0, 2 * B * xcols * 2);
   cudaMemset(bs->tickets, 0, B * m.n_kv * 4);
   if (cudaFuncSetAttribute(gemm_wx_kernel<16, kDStages, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)gemm_smem_bytes<16, kDStages, true>()) != cudaSuccess)
+                           (int)gemm_smem_bytes<16, kDStages, true>()) != cudaSuccess ||
+      cudaFuncSetAttribute(gemm_wx_kernel<16, kDStagesPair, true>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)gemm_smem_bytes<16, kDStagesPair, true>()) != cudaSuccess)
     return "decode GEMM shared memory attribute";
   return batch_attn(dim3(1), nullptr, nullptr, nullptr, m, 0, bs->splits, nullptr, true);
 }
