@@ -1058,10 +1058,19 @@ std::string batch_enqueue(const ModelDev& m, const PrefillWeights& w, BatchScrat
   const int qkvR = qkv_rows(m.n_q, m.n_kv, d);
   const int ldy = std::max(std::max(qkvR, 2 * F), H);
   const size_t pstride = (size_t)n * ldy;
-  const int zq = split_k(qkvR, H, num_sms), zo = split_k(H, qd, num_sms);
+  // W_qkv, W_o, W_down have few 128-row tiles: split K so that two CTAs per
+  // SM (6 stages each) fill one wave of 2 * num_sms
+  auto pair_split = [&](int rows, int K) {
+    const int tiles = (rows + kGM - 1) / kGM, nk = K / kGK;
+    int z = (2 * num_sms) / tiles;
+    z = std::min(z, kBatchMaxSplitK);
+    z = std::min(z, std::max(1, nk / 2));
+    return std::max(z, 1);
+  };
+  const int zq = pair_split(qkvR, H), zo = pair_split(H, qd);
   const int gu_tiles = (2 * F + kGM - 1) / kGM;
   const bool gu_pair = gu_tiles > num_sms && gu_tiles <= 2 * num_sms;
-  const int zg = split_k(2 * F, H, num_sms), zd = split_k(H, F, num_sms);
+  const int zg = split_k(2 * F, H, num_sms), zd = pair_split(H, F);
   std::string e;
   BatchParams* bp = bs.params;
 #define CKL(call)                                                                       \
@@ -1085,14 +1094,16 @@ std::string batch_enqueue(const ModelDev& m, const PrefillWeights& w, BatchScrat
     float* ss_ffn = ss + (size_t)(2 * l + 1) * kMaxBatch;
     float* ss_next = ss + (size_t)(2 * l + 2) * kMaxBatch;
     const uint16_t* bias = m.qkv_bias ? m.bqkv + (size_t)l * qkvR : nullptr;
-    if (!(e = gemm_hl(w.qkv[l], qkvR, H, xhl, n, bs.y, ldy, bs.err, st, zq, ss_attn, m.rms_eps)).empty())
+    if (!(e = gemm_hl(w.qkv[l], qkvR, H, xhl, n, bs.y, ldy, bs.err, st, zq, ss_attn, m.rms_eps,
+                      nullptr, true)).empty())
       return e;
     CKL(launch_pdl(rope_kv_kernel, dim3(n, psl), dim3(256), 0, st, (const float*)bs.y, ldy, zq, pstride,
                    bias, (const int32_t*)bp->slot, (const int32_t*)bp->pos, m, l, bs.q));
     if (!(e = batch_attn(dim3(bs.splits, m.n_kv, n), st, bs.q, bp, m, l, bs.splits, bs.part, false,
                          bs.tickets, xhl, lo(qd))).empty())
       return e;
-    if (!(e = gemm_hl(w.o[l], H, qd, xhl, n, bs.y, ldy, bs.err, st, zo, nullptr, 0.f)).empty()) return e;
+    if (!(e = gemm_hl(w.o[l], H, qd, xhl, n, bs.y, ldy, bs.err, st, zo, nullptr, 0.f, nullptr, true)).empty())
+      return e;
     CKL(launch_pdl(b_residual_norm_kernel, dim3(hsl, n), dim3(256), 0, st, bs.x, (const float*)bs.y, H,
                    ldy, zo, pstride, m.ffn_norm + (size_t)l * H, xhl, lo(H), ss_ffn));
     // SwiGLU output into a second buffer: the gate/up GEMM still reads xhl
@@ -1106,7 +1117,8 @@ std::string batch_enqueue(const ModelDev& m, const PrefillWeights& w, BatchScrat
       CKL(launch_pdl(b_swiglu_kernel, dim3(fsl, n), dim3(256), 0, st, (const float*)bs.y, ldy, F, zg,
                      pstride, bs.xh2, bs.xh2 + (size_t)8 * F));
     }
-    if (!(e = gemm_hl(w.dn[l], H, F, bs.xh2, n, bs.y, ldy, bs.err, st, zd, nullptr, 0.f)).empty()) return e;
+    if (!(e = gemm_hl(w.dn[l], H, F, bs.xh2, n, bs.y, ldy, bs.err, st, zd, nullptr, 0.f, nullptr, true)).empty())
+      return e;
     // the residual add, then the next layer's attention norm (the final norm after the last)
     const uint16_t* next_norm = l + 1 < L ? m.attn_norm + (size_t)(l + 1) * H : m.final_norm;
     CKL(launch_pdl(b_residual_norm_kernel, dim3(hsl, n), dim3(256), 0, st, bs.x, (const float*)bs.y, H,
