@@ -101,8 +101,9 @@ struct ModelDev {
   uint32_t* epoch;         // completed steps
   int32_t* status;         // 0 ok, else an MK_ERR_* code
   int32_t* status_info;    // task index / detail of the first error
-  // optional per-task trace: 4 words per queue entry of the megakernel queue set
-  // (event satisfied, workers start, workers done [%globaltimer ns], cta << 32 | task)
+  // optional per-task trace: 8 words per queue entry of the megakernel queue set
+  // (%globaltimer ns at: event satisfied, workers start, input loaded, first
+  // chunk ready, last chunk consumed, epilogue done, end; then cta << 32 | task)
   unsigned long long* trace;
 };
 
