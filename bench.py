@@ -312,6 +312,23 @@ def run_mk(args):
     achieved = bytes_mean / avg_launch_s / 1e9
     peak, peak_src = measured_peaks()
 
+    # ---- the device-resident loop: the same K steps in one persistent launch
+    loop = None
+    if n == 1 and world == 1:
+        prefill()
+        run_steps(0, W)
+        seq = torch.empty(K, dtype=torch.int32, device="cuda")
+        le = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        torch.cuda.synchronize()
+        le[0].record(stream)
+        dec.decode_steps(ids[W % 2], lens[0] + W, K, seq)
+        le[1].record(stream)
+        torch.cuda.synchronize()
+        rc = dec.status()
+        if rc != 0:
+            raise RuntimeError(f"device status {rc}: {dec.last_error()}")
+        loop = {"ms_per_token": le[0].elapsed_time(le[1]) / K, "steps_per_launch": K}
+
     # ---- read-stream probe: practical read ceiling on this GPU
     probe_buf = torch.empty(4 * 2**30, dtype=torch.uint8, device="cuda")
     sink = torch.zeros(1, dtype=torch.int64, device="cuda")
@@ -414,6 +431,7 @@ def run_mk(args):
                      "traffic": load_traffic() if n == 1 else None,
                      "bytes_per_launch": bytes_mean},
         "baselines": baselines,
+        "device_loop": loop,
         "prefill": {"ms": prefill_ms[0], "positions": int(sum(lens)),
                     "path": "tensor-core GEMMs for all but each prompt's last position"},
         "clocks": clocks,

@@ -146,6 +146,19 @@ int mk_prefill(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t* offsets_ho
 int mk_decode_step(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t* pos_host, int n_req,
                    float* logits_dev, int32_t* next_ids_dev);
 
+/* n_steps greedy decode steps of request 0 in ONE persistent launch (the
+ * device-resident loop): step s runs at position pos0 + s, feeds the id step
+ * s - 1 produced (step 0 feeds token_dev[0]), appends its K/V and writes its
+ * greedy id to ids_dev[s]; only the last step writes logits (last_logits_dev,
+ * vocab fp32, may be NULL).  Inside the launch a step's first layer waits for
+ * the previous step's argmax through the device epoch, so no kernel boundary
+ * or host round trip separates the steps and the weight prefetch of a step
+ * overlaps the previous step's LM head.  Megakernel mode only
+ * (MK_ERR_UNSUPPORTED otherwise); pos0 + n_steps <= max_seq
+ * (MK_ERR_POS_RANGE).  Results equal n_steps calls of mk_decode_step. */
+int mk_decode_steps(mk_ctx* ctx, const int32_t* token_dev, int pos0, int n_steps, int32_t* ids_dev,
+                    float* last_logits_dev);
+
 /* mk_decode_step from and to HOST memory: copies the tokens in, runs the
  * step, copies the next ids out and synchronises the stream. */
 int mk_decode_step_host(mk_ctx* ctx, const int32_t* tokens_host, const int32_t* pos_host,

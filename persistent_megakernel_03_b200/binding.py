@@ -22,7 +22,8 @@ ERRORS = {-1: "MK_ERR_INVALID_ARG", -2: "MK_ERR_OOM", -3: "MK_ERR_CUDA", -4: "MK
 MODE_MEGAKERNEL, MODE_PER_OP, MODE_PER_OP_GRAPH = 0, 1, 2
 TASK_KINDS = ("QKV", "ATTN", "OPROJ", "GATEUP", "DOWN", "LMHEAD")
 
-EXPORTS = ("mk_create", "mk_prefill", "mk_decode_step", "mk_decode_step_host", "mk_copy_hidden",
+EXPORTS = ("mk_create", "mk_prefill", "mk_decode_step", "mk_decode_steps", "mk_decode_step_host",
+           "mk_copy_hidden",
            "mk_kv_pointer", "mk_copy_kv", "mk_set_mode", "mk_status", "mk_last_error",
            "mk_destroy", "mk_plan_build", "mk_plan_get_info", "mk_plan_get_tasks",
            "mk_plan_get_queue", "mk_plan_get_event_counts", "mk_plan_destroy",
@@ -98,6 +99,7 @@ def lib(build_if_missing: bool = True):
     L.mk_prefill.argtypes = [vp, vp, ip, i, vp, vp]
     L.mk_decode_step.argtypes = [vp, vp, ip, i, vp, vp]
     L.mk_decode_step_host.argtypes = [vp, ip, ip, i, ip]
+    L.mk_decode_steps.argtypes = [vp, vp, i, i, vp, vp]
     L.mk_copy_hidden.argtypes = [vp, vp, i]
     L.mk_kv_pointer.argtypes = [vp, i, i, i, i, C.POINTER(vp)]
     L.mk_copy_kv.argtypes = [vp, i, i, i, i, i, vp]
@@ -257,6 +259,13 @@ class Decoder:
         _check(lib().mk_decode_step(self.h, tokens_dev.data_ptr(), _ints(pos), len(pos),
                                     None if logits_dev is None else logits_dev.data_ptr(),
                                     None if next_ids_dev is None else next_ids_dev.data_ptr()),
+               self.h)
+
+    def decode_steps(self, token_dev, pos0: int, n_steps: int, ids_dev, last_logits_dev=None):
+        """n_steps greedy steps in one persistent launch; ids_dev[s] gets step s's id."""
+        _check(lib().mk_decode_steps(self.h, token_dev.data_ptr(), int(pos0), int(n_steps),
+                                     ids_dev.data_ptr(),
+                                     None if last_logits_dev is None else last_logits_dev.data_ptr()),
                self.h)
 
     def decode_host(self, tokens: Sequence[int], pos: Sequence[int]) -> List[int]:

@@ -112,6 +112,8 @@ static void fill_args(mk_ctx* ctx, KernelArgs& a, int set, const StepParams* sp_
   if (sp_val) a.sp_val = *sp_val; else memset(&a.sp_val, 0, sizeof(a.sp_val));
   a.sp_ptr = sp_ptr;
   a.no_wait = no_wait ? 1 : 0;
+  a.n_steps = 1;
+  a.ids_seq = nullptr;
 }
 
 // Enqueues one decode step in the context's mode.
@@ -452,6 +454,34 @@ extern "C" int mk_decode_step(mk_ctx* ctx, const int32_t* tokens_dev, const int3
                          cudaMemcpyDeviceToDevice, ctx->stream));
   }
   ctx->last_n_req = n_req;
+  ctx->last_batched = false;
+  return MK_OK;
+}
+
+extern "C" int mk_decode_steps(mk_ctx* ctx, const int32_t* token_dev, int pos0, int n_steps,
+                               int32_t* ids_dev, float* last_logits_dev) {
+  int rc = check_ctx(ctx);
+  if (rc) return rc;
+  if (ctx->mode != MK_MODE_MEGAKERNEL)
+    return fail(ctx, MK_ERR_UNSUPPORTED, "the device-resident loop runs in megakernel mode only");
+  if (!token_dev || !ids_dev || n_steps < 1) return fail(ctx, MK_ERR_INVALID_ARG, "bad argument");
+  if (pos0 < 0 || (long long)pos0 + n_steps > ctx->cfg.max_seq)
+    return fail(ctx, MK_ERR_POS_RANGE, "positions " + std::to_string(pos0) + ".." +
+                                           std::to_string(pos0 + n_steps - 1) + " outside [0, max_seq)");
+  StepParams sp{};
+  sp.n_req = 1;
+  sp.pos[0] = pos0;
+  sp.kv_slot[0] = 0;
+  sp.tokens = token_dev;
+  sp.logits = last_logits_dev;
+  sp.next_ids = ids_dev;
+  sp.want_logits = last_logits_dev != nullptr;
+  KernelArgs a;
+  fill_args(ctx, a, 0, &sp, nullptr, false);
+  a.n_steps = n_steps;
+  a.ids_seq = ids_dev;
+  CK(launch_step(a, ctx->plan.num_ctas, true, ctx->stream));
+  ctx->last_n_req = 1;
   ctx->last_batched = false;
   return MK_OK;
 }

@@ -47,6 +47,8 @@ struct __align__(128) Smem {
   int32_t flag;
   int32_t cur_qi;              // queue entry the workers are running (trace)
   unsigned long long lm_best;  // running argmax over this CTA's LM-head tasks
+  StepParams sp_work;          // the workers' current step (set by the scheduler between steps)
+  uint32_t epoch0;             // completed steps when this launch started
   int32_t attn_last;           // this attention task merges its KV head's splits
   __align__(16) float attn_xb[kWorkerWarps][kAttnXbStride];  // attention: per-warp softmax weights
 };
@@ -59,6 +61,22 @@ __device__ __forceinline__ bool aborting(Smem& s) { return *(volatile int32_t*)&
 
 __device__ __forceinline__ const StepParams& step_params(const KernelArgs& a) {
   return a.sp_ptr ? *a.sp_ptr : a.sp_val;
+}
+
+// The parameters of step `step` of this launch.  With a device-resident loop
+// (n_steps > 1) position and token advance per step: step s feeds the id step
+// s - 1 wrote, writes its own id to ids_seq[s], and only the last step writes
+// logits.
+__device__ __forceinline__ void step_at(const KernelArgs& a, int step, StepParams& out) {
+  out = step_params(a);
+  if (a.n_steps > 1) {
+    out.pos[0] += step;
+    out.tokens = step == 0 ? out.tokens : a.ids_seq + (step - 1);
+    out.next_ids = a.ids_seq + step;
+    const bool last = step == a.n_steps - 1;
+    out.logits = last ? out.logits : nullptr;
+    out.want_logits = last ? out.want_logits : 0;
+  }
 }
 
 // Per-task timeline (diagnostics, off unless a trace buffer is set): word k of
@@ -227,19 +245,38 @@ struct ChunkCursor {
 // consumption order, as fast as slots free up.
 __device__ __forceinline__ void producer(const KernelArgs& a, Smem& s, int q0, int q1) {
   const ModelDev& m = a.m;
-  const StepParams& sp = step_params(a);
   const uint64_t pol_w = l2_policy_evict_first();
   const uint64_t pol_keep = l2_policy_evict_normal();
-  ChunkCursor cc{q0, q1, -1};
   Chunk c;
   uint32_t seq = 0;
-  while (cc.next(a, sp, c)) {
-    if (!producer_acquire_slot(s, seq, m)) break;
-    const int slot = seq % kRingSlots;
-    mbar_arrive_expect_tx(&s.full[slot], c.bytes0 + c.bytes1);
-    bulk_g2s(s.ring[slot], c.src0, c.bytes0, &s.full[slot], c.kv ? pol_keep : pol_w);
-    if (c.src1) bulk_g2s(s.ring[slot] + kSlotBytes / 2, c.src1, c.bytes1, &s.full[slot], pol_keep);
-    ++seq;
+  bool stop = false;
+  for (int step = 0; step < a.n_steps && !stop; ++step) {
+    StepParams sp;
+    step_at(a, step, sp);
+    // Cached keys of a step after the first include the key the previous
+    // step wrote (another CTA, same launch): before copying any, wait until
+    // that step has completed (its last LM-head task bumps the epoch) and
+    // order those writes before this thread's bulk copies.
+    bool kv_ready = step == 0;
+    ChunkCursor cc{q0, q1, -1};
+    while (cc.next(a, sp, c)) {
+      if (c.kv && !kv_ready) {
+        const uint64_t t0 = globaltimer_ns();
+        const uint64_t limit = 2ull * (uint64_t)(m.timeout_ms > 0 ? m.timeout_ms : 1000) * 1000000ull;
+        while ((int32_t)(ld_acquire_gpu(m.epoch) - (s.epoch0 + (uint32_t)step)) < 0) {
+          if (aborting(s) || globaltimer_ns() - t0 > limit) { stop = true; break; }
+        }
+        if (stop) break;
+        fence_proxy_async_global();
+        kv_ready = true;
+      }
+      if (!producer_acquire_slot(s, seq, m)) { stop = true; break; }
+      const int slot = seq % kRingSlots;
+      mbar_arrive_expect_tx(&s.full[slot], c.bytes0 + c.bytes1);
+      bulk_g2s(s.ring[slot], c.src0, c.bytes0, &s.full[slot], c.kv ? pol_keep : pol_w);
+      if (c.src1) bulk_g2s(s.ring[slot] + kSlotBytes / 2, c.src1, c.bytes1, &s.full[slot], pol_keep);
+      ++seq;
+    }
   }
   // Before this warp may retire, every copy it issued must have landed: if
   // the workers stop early (abort) nobody else waits for them, and a bulk copy
@@ -259,16 +296,38 @@ __device__ __forceinline__ void producer(const KernelArgs& a, Smem& s, int q0, i
 
 __device__ __forceinline__ void scheduler(const KernelArgs& a, Smem& s, int q0, int q1) {
   const ModelDev& m = a.m;
-  const StepParams& sp = step_params(a);
   const uint64_t pol_keep = l2_policy_evict_normal();
-  const uint32_t epoch = s.epoch;
   const uint64_t limit = (uint64_t)(m.timeout_ms > 0 ? m.timeout_ms : 1000) * 1000000ull;
   int i = 0;
+  for (int step = 0; step < a.n_steps; ++step) {
+  StepParams sp;
+  step_at(a, step, sp);
+  const uint32_t epoch = s.epoch0 + (uint32_t)step;
+  if (step > 0) {
+    // the workers are idle (the previous task's `done` was observed)
+    s.sp_work = sp;
+    s.epoch = epoch;
+  }
   for (int qi = q0; qi < q1; ++qi, ++i) {
     const int tid = a.queue[qi];
     const Task& t = a.tasks[tid];
     bool abort = false;
-    if (t.wait_ev >= 0 && !a.no_wait) {
+    if (step > 0 && t.kind == T_QKV && t.layer == 0) {
+      // the first layer embeds the id the previous step produced
+      const uint64_t t0 = globaltimer_ns();
+      uint32_t spins = 0;
+      while ((int32_t)(ld_acquire_gpu(m.epoch) - epoch) < 0) {
+        if ((++spins & 63u) == 0) {
+          if (ld_relaxed_gpu_s32(m.status) != 0 || aborting(s)) { abort = true; break; }
+          if (globaltimer_ns() - t0 > limit) {
+            set_error(m, MK_ERR_TIMEOUT, tid);
+            abort = true;
+            break;
+          }
+        }
+      }
+    }
+    if (!abort && t.wait_ev >= 0 && !a.no_wait) {
       const uint32_t target = t.wait_count * (epoch + 1u);
       const uint32_t* ev = m.events + t.wait_ev;
       if (m.l2_prefetch_chunks > 0 && (int32_t)(ld_acquire_gpu(ev) - target) < 0) {
@@ -306,6 +365,7 @@ __device__ __forceinline__ void scheduler(const KernelArgs& a, Smem& s, int q0, 
     if (m.trace) m.trace[(size_t)qi * kTraceWords] = globaltimer_ns();
     mbar_arrive(&s.ready);
     if (!wait_bounded(s, &s.done, i & 1, m, kWaitDone)) return;
+  }
   }
 }
 
@@ -364,10 +424,10 @@ __device__ __forceinline__ void wait_full(Smem& s, uint32_t seq, const ModelDev&
 // afterwards (W (x * w * r) = r * W (x * w)), so the first ring chunk is not
 // held back by a block-wide reduction.
 template <int CPT>
-__device__ __forceinline__ float gemv_load_input(const KernelArgs& a, const Task& t, int wtid,
-                                                 int ct, int rl, float2 (&x2)[CPT][4]) {
+__device__ __forceinline__ float gemv_load_input(const KernelArgs& a, const StepParams& sp,
+                                                 const Task& t, int wtid, int ct, int rl,
+                                                 float2 (&x2)[CPT][4]) {
   const ModelDev& m = a.m;
-  const StepParams& sp = step_params(a);
   const int K = t.K, C = K >> 3;
   const float* src32 = nullptr;
   const uint16_t* src16 = nullptr;
@@ -441,7 +501,7 @@ __device__ __forceinline__ void gemv_stream(const KernelArgs& a, Smem& s, const 
   const size_t row_bytes = (size_t)K * 2;
   const int nrows = t.row1 - t.row0;
   float2 x2[CPT][4];
-  float ss = gemv_load_input<CPT>(a, t, wtid, ct, rl, x2);
+  float ss = gemv_load_input<CPT>(a, s.sp_work, t, wtid, ct, rl, x2);
   trace_mark(a, s, wtid, 2);
   const bool has_norm = t.kind == T_QKV || t.kind == T_GATEUP || t.kind == T_LMHEAD;
   if (has_norm) {
@@ -551,9 +611,9 @@ struct EpiPre {
   float c, sn, b0, b1, res;
 };
 
-__device__ __forceinline__ EpiPre epilogue_prefetch(const KernelArgs& a, const Task& t, int wtid) {
+__device__ __forceinline__ EpiPre epilogue_prefetch(const KernelArgs& a, const StepParams& sp,
+                                                    const Task& t, int wtid) {
   const ModelDev& m = a.m;
-  const StepParams& sp = step_params(a);
   EpiPre p{1.f, 0.f, 0.f, 0.f, 0.f};
   const int nrows = t.row1 - t.row0;
   if (t.kind == T_QKV) {
@@ -582,7 +642,7 @@ __device__ __forceinline__ EpiPre epilogue_prefetch(const KernelArgs& a, const T
 __device__ __forceinline__ void epilogue_qkv(const KernelArgs& a, Smem& s, const Task& t, int wtid,
                                              const EpiPre& pre) {
   const ModelDev& m = a.m;
-  const StepParams& sp = step_params(a);
+  const StepParams& sp = s.sp_work;
   const int d = m.head_dim, G = m.group, half = d >> 1;
   const int pos = sp.pos[0], slot = sp.kv_slot[0];
   const int qkvR = qkv_rows(m.n_q, m.n_kv, d);
@@ -632,7 +692,7 @@ __device__ __forceinline__ void epilogue_qkv(const KernelArgs& a, Smem& s, const
 __device__ __forceinline__ void epilogue_residual(const KernelArgs& a, Smem& s, const Task& t, int wtid,
                                                   const EpiPre& pre) {
   const ModelDev& m = a.m;
-  const StepParams& sp = step_params(a);
+  const StepParams& sp = s.sp_work;
   const int nrows = t.row1 - t.row0;
   const bool from_embed = t.kind == T_OPROJ && t.layer == 0;
   int tok = 0;
@@ -660,7 +720,7 @@ __device__ __forceinline__ void epilogue_swiglu(const KernelArgs& a, Smem& s, co
 
 __device__ __forceinline__ void epilogue_lmhead(const KernelArgs& a, Smem& s, const Task& t, int wtid) {
   const ModelDev& m = a.m;
-  const StepParams& sp = step_params(a);
+  const StepParams& sp = s.sp_work;
   const int nrows = t.row1 - t.row0;
   unsigned long long best = 0ull;
   for (int i = wtid; i < nrows; i += kWorkerThreads) {
@@ -735,7 +795,7 @@ __device__ __forceinline__ void attn_write_state(const AttnState<DPL, G>& st, fl
 template <int DPL, int G>
 __device__ __forceinline__ void attn_task(const KernelArgs& a, Smem& s, const Task& t, uint32_t& seq, int wtid) {
   const ModelDev& m = a.m;
-  const StepParams& sp = step_params(a);
+  const StepParams& sp = s.sp_work;
   const int d = m.head_dim, S_all = m.attn_splits, PS = attn_part_stride(d);
   const int warp = wtid >> 5, lane = wtid & 31;
   const int g = t.row0, split = t.row1, b = t.req;
@@ -955,12 +1015,14 @@ __device__ __forceinline__ void worker(const KernelArgs& a, Smem& s, int q0, int
   const int wtid = threadIdx.x - kFirstWorkerWarp * 32;
   uint32_t seq = 0;
   int i = 0;
+  bool stop = false;
+  for (int step = 0; step < a.n_steps && !stop; ++step)
   for (int qi = q0; qi < q1; ++qi, ++i) {
     const Task t = a.tasks[a.queue[qi]];
     const bool go = wait_bounded(s, &s.ready, i & 1, a.m, kWaitReady);
     // all workers agree: the flag was published before the ready arrival
     worker_sync();
-    if (!go || aborting(s)) break;
+    if (!go || aborting(s)) { stop = true; break; }
     if (wtid == 0) s.cur_qi = qi;  // read by this thread only (trace_mark)
     trace_mark(a, s, wtid, 1);
     switch (t.kind) {
@@ -974,7 +1036,7 @@ __device__ __forceinline__ void worker(const KernelArgs& a, Smem& s, int q0, int
         finish_task(a, s, t, wtid, false);
         break;
       default: {
-        const EpiPre pre = epilogue_prefetch(a, t, wtid);
+        const EpiPre pre = epilogue_prefetch(a, s.sp_work, t, wtid);
         gemv_core(a, s, t, seq, wtid);
         if (t.kind == T_QKV) epilogue_qkv(a, s, t, wtid, pre);
         else if (t.kind == T_GATEUP) epilogue_swiglu(a, s, t, wtid);
@@ -1006,6 +1068,8 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
     s.abort_flag = 0;
     s.flag = 0;
     s.epoch = *reinterpret_cast<volatile uint32_t*>(a.m.epoch);
+    s.epoch0 = s.epoch;
+    step_at(a, 0, s.sp_work);
     fence_barrier_init();
   }
   __syncthreads();

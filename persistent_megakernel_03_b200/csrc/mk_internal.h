@@ -114,6 +114,9 @@ struct KernelArgs {
   const int32_t* queue_off;  // [num_ctas + 1] for this launch's queue set
   StepParams sp_val;         // step inputs by value ...
   const StepParams* sp_ptr;  // ... or, when non-null, from device memory (graph replay)
+  int32_t n_steps;           // decode steps in this launch (1, or more: device-resident loop)
+  int32_t* ids_seq;          // n_steps > 1: step s writes its greedy id to ids_seq[s] and
+                             // step s + 1 embeds it (step 0 embeds sp.tokens[0])
   int32_t no_wait;           // per-operator mode: kernel boundaries order the tasks
 };
 
