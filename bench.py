@@ -247,9 +247,13 @@ def run_mk(args):
         K = LONG_STEPS - W   # these workloads decode 256 steps after their prompts
     max_seq = max(lens) + W + K + 1
     w = synth.make_model(model, 0, device="cuda")
+    fp8 = args.weights == "fp8"
+    if fp8:  # the row-quantized model (every GEMV matrix e4m3 codes x row powers of two)
+        w = synth.quantize_fp8_model(model, w)
+    wbytes = 1 if fp8 else 2
     stream = torch.cuda.current_stream()
     dec = binding.Decoder(model, w, max_seq, max_batch=n, stream=stream,
-                          l2_prefetch=args.l2_prefetch)
+                          l2_prefetch=args.l2_prefetch, weight_format=1 if fp8 else 0)
     del w  # mk_create copied and packed the weights
     torch.cuda.empty_cache()
     if n == 1:
@@ -307,7 +311,7 @@ def run_mk(args):
     total_ms = evs[0].elapsed_time(evs[K])
     total_ms = max_over_ranks(total_ms, world)
     value = per_token_ms(total_ms, K, world)
-    bytes_mean = sum(roofline.step_bytes(model, positions(W + k)) for k in range(K)) / K
+    bytes_mean = sum(roofline.step_bytes(model, positions(W + k), wbytes=wbytes) for k in range(K)) / K
     avg_launch_s = (sum(per_step) / K) * 1e-3
     achieved = bytes_mean / avg_launch_s / 1e9
     peak, peak_src = measured_peaks()
@@ -414,10 +418,11 @@ def run_mk(args):
     line = {
         "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": K,
         "warmup": W, "ms_per_step": total_ms / K, "higher_is_better": False,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "weights": "bf16",
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "weights": "fp8 e4m3, one power-of-two scale per row" if fp8 else "bf16",
         "data": "synthetic",
         "config": {"workload": workload,
-                   "l2": (f"inputs larger than L2 ({roofline.weight_bytes(model) / 1e9:.2f} GB of "
+                   "l2": (f"inputs larger than L2 ({roofline.weight_bytes(model, wbytes) / 1e9:.2f} GB of "
                           "weights streamed per step)"),
                    "parallelism": f"replicas x{world}"},
         "tok_per_s": 1e3 * n / value,
@@ -428,7 +433,7 @@ def run_mk(args):
         "read_probe_gbs": probe_gbs, "frac_of_read_probe": achieved / probe_gbs,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": peak_src,
-                     "traffic": load_traffic() if n == 1 else None,
+                     "traffic": load_traffic() if n == 1 and not fp8 else None,
                      "bytes_per_launch": bytes_mean},
         "baselines": baselines,
         "device_loop": loop,
@@ -453,6 +458,8 @@ def run_mk(args):
         dec.close()
         torch.cuda.empty_cache()
         w2 = synth.make_model(model, 0, device="cuda")
+        if fp8:
+            w2 = synth.quantize_fp8_model(model, w2)
         w_cpu = {k: v.cpu() for k, v in w2.items()}
         del w2
         first_pos = lens[0] + W if n > 1 or lens[0] > SHORT_PROMPT else 0
@@ -500,6 +507,9 @@ def main():
                          "prompt; llama8b-batch8: 8 requests with prompts of U[32, 2048] "
                          "tokens (these two decode at most 256 steps); qwen05b: the "
                          "Qwen2.5-0.5B shape, 39-token prompt")
+    ap.add_argument("--weights", default="bf16", choices=["bf16", "fp8"],
+                    help="fp8: the row-quantized e4m3 model through the fp8 decode path "
+                         "(not the headline configuration)")
     ap.add_argument("--layers", type=int, default=0,
                     help="profiling aid: a shallower model of the same widths (not a bench line)")
     args = ap.parse_args()

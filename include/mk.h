@@ -100,6 +100,13 @@ typedef struct {
   int l2_prefetch;   /* when a CTA's next task must wait for its event, the number
                         of 32 KB weight chunks past its shared-memory ring it
                         prefetches into L2 meanwhile; 0: default (off), < 0: off */
+  int weight_format; /* 0: bf16 decode weights (default); 1: fp8 e4m3 with one
+                        power-of-two scale per row for every GEMV matrix (QKV, O,
+                        gate/up, down, LM head): mk_create quantizes the given bf16
+                        weights (round to nearest) and replaces its bf16 copies by
+                        the dequantized values, which the prefill and the batched
+                        step then use -- bf16 weights that already are such values
+                        are kept exactly */
   int batch_sequential; /* 1: a step of several requests runs them one after another
                            through the megakernel; 0: default, one batched step */
   int prefill_steps; /* 1: mk_prefill runs every prompt position as a decode step;

@@ -61,8 +61,8 @@ class Weights(C.Structure):
 
 class Options(C.Structure):
     _fields_ = [("num_ctas", C.c_int), ("attn_splits", C.c_int), ("timeout_ms", C.c_int),
-                ("mode", C.c_int), ("l2_prefetch", C.c_int), ("batch_sequential", C.c_int),
-                ("prefill_steps", C.c_int)]
+                ("mode", C.c_int), ("l2_prefetch", C.c_int), ("weight_format", C.c_int),
+                ("batch_sequential", C.c_int), ("prefill_steps", C.c_int)]
 
 
 class PlanInfo(C.Structure):
@@ -150,11 +150,11 @@ class Plan:
     """The task graph mk_create would build (host only)."""
 
     def __init__(self, model, max_seq: int, num_ctas: int, max_batch: int = 1,
-                 attn_splits: int = 0):
+                 attn_splits: int = 0, weight_format: int = 0):
         L = lib()
         self.h = C.c_void_p()
         cfg = make_config(model, max_seq, max_batch)
-        opt = Options(num_ctas, attn_splits, 0, 0, 0, 0, 0)
+        opt = Options(num_ctas, attn_splits, 0, 0, 0, weight_format, 0, 0)
         rc = L.mk_plan_build(C.byref(cfg), C.byref(opt), int(num_ctas), C.byref(self.h))
         if rc != MK_OK:
             raise MkError(rc, "mk_plan_build rejected the configuration")
@@ -202,7 +202,8 @@ class Decoder:
     def __init__(self, model, weights: Dict[str, "torch.Tensor"], max_seq: int,
                  max_batch: int = 1, num_ctas: int = 0, attn_splits: int = 0,
                  timeout_ms: int = 0, mode: int = MODE_MEGAKERNEL, stream=None,
-                 l2_prefetch: int = 0, prefill_steps: int = 0, batch_sequential: int = 0):
+                 l2_prefetch: int = 0, prefill_steps: int = 0, batch_sequential: int = 0,
+                 weight_format: int = 0):
         import torch
         L = lib()
         self.model = model
@@ -224,8 +225,8 @@ class Decoder:
         w = Weights(ptr("embed"), layers, ptr("final_norm"),
                     None if model.tied_embeddings else ptr("lm_head"))
         cfg = make_config(model, max_seq, max_batch)
-        opt = Options(num_ctas, attn_splits, timeout_ms, mode, l2_prefetch, batch_sequential,
-                      prefill_steps)
+        opt = Options(num_ctas, attn_splits, timeout_ms, mode, l2_prefetch, weight_format,
+                      batch_sequential, prefill_steps)
         self.h = C.c_void_p()
         rc = L.mk_create(C.byref(cfg), C.byref(w), C.byref(opt), self.stream.cuda_stream,
                          C.byref(self.h))

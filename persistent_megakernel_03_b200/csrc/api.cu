@@ -15,7 +15,9 @@
 
 namespace mk {
 size_t step_kernel_smem_bytes();
-const void* step_kernel_ptr();
+const void* step_kernel_ptr(int wbytes);
+cudaError_t launch_quantize_fp8_rows(uint16_t* w, uint8_t* codes, float* scales, int rows, int K,
+                                     cudaStream_t st);
 cudaError_t launch_pack_qkv(uint16_t*, const uint16_t*, const uint16_t*, const uint16_t*, int, int,
                             int, int, cudaStream_t);
 cudaError_t launch_pack_qkv_bias(uint16_t*, const uint16_t*, const uint16_t*, const uint16_t*, int,
@@ -220,9 +222,18 @@ extern "C" int mk_create(const mk_config* cfg, const mk_weights* w, const mk_opt
                std::to_string(smem);
     return bail(MK_ERR_NOT_RESIDENT);
   }
-  CKC(cudaFuncSetAttribute(step_kernel_ptr(), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  if (ctx->opt.weight_format < 0 || ctx->opt.weight_format > 1) {
+    ctx->err = "weight_format must be 0 (bf16) or 1 (fp8 e4m3)";
+    return bail(MK_ERR_INVALID_ARG);
+  }
+  const int wbytes = ctx->opt.weight_format == 1 ? 1 : 2;
+  if (wbytes == 1 && (cfg->hidden % 16 || cfg->ffn % 16 || (cfg->n_q_heads * cfg->head_dim) % 16)) {
+    ctx->err = "fp8 weights need hidden, ffn and n_q_heads * head_dim multiples of 16";
+    return bail(MK_ERR_UNSUPPORTED);
+  }
+  CKC(cudaFuncSetAttribute(step_kernel_ptr(wbytes), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   int per_sm = 0;
-  CKC(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, step_kernel_ptr(), kThreads, smem));
+  CKC(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, step_kernel_ptr(wbytes), kThreads, smem));
   if (per_sm < 1) {
     ctx->err = "one CTA of the step kernel does not fit on an SM";
     return bail(MK_ERR_NOT_RESIDENT);
@@ -232,7 +243,7 @@ extern "C" int mk_create(const mk_config* cfg, const mk_weights* w, const mk_opt
     ctx->err = "num_ctas exceeds the co-resident limit";
     return bail(MK_ERR_NOT_RESIDENT);
   }
-  std::string perr = build_plan(*cfg, P, ctx->opt.attn_splits, &ctx->plan);
+  std::string perr = build_plan(*cfg, P, ctx->opt.attn_splits, &ctx->plan, wbytes);
   if (!perr.empty()) {
     ctx->err = perr;
     return bail(MK_ERR_INVALID_ARG);
@@ -295,6 +306,34 @@ extern "C" int mk_create(const mk_config* cfg, const mk_weights* w, const mk_opt
                                (const uint16_t*)w->layers[l].bk, (const uint16_t*)w->layers[l].bv, G, d,
                                qkvR, st));
   }
+  // fp8 decode weights: codes and row scales of every GEMV matrix; the bf16
+  // copies above are overwritten with the dequantized values (one model for
+  // the decode GEMVs, the tensor-core prefill and the batched step)
+  std::vector<const uint8_t*> c_qkv(L), c_o(L), c_gu(L), c_dn(L);
+  const uint8_t* c_lm = nullptr;
+  if (wbytes == 1) {
+    // one allocation per matrix: rows x K codes, then (16-byte aligned) the
+    // rows' fp32 scales -- where the kernel looks for them
+    auto quant = [&](uint16_t* wm, int rows, int K, const uint8_t** code_out) {
+      const size_t off = ((size_t)rows * K + 15) & ~(size_t)15;
+      uint8_t* codes = nullptr;
+      int r2 = dalloc(ctx, &codes, off + (size_t)rows * 4);
+      if (r2) return r2;
+      if (launch_quantize_fp8_rows(wm, codes, reinterpret_cast<float*>(codes + off), rows, K, st) !=
+          cudaSuccess)
+        return (int)MK_ERR_CUDA;
+      *code_out = codes;
+      return 0;
+    };
+    for (int l = 0; l < L; ++l) {
+      if ((rc = quant(const_cast<uint16_t*>(w_qkv[l]), qkvR, H, &c_qkv[l])) ||
+          (rc = quant(const_cast<uint16_t*>(w_o[l]), H, qd, &c_o[l])) ||
+          (rc = quant(const_cast<uint16_t*>(w_gu[l]), 2 * F, H, &c_gu[l])) ||
+          (rc = quant(const_cast<uint16_t*>(w_dn[l]), H, F, &c_dn[l])))
+        return bail(rc);
+    }
+    if ((rc = quant(lm, V, H, &c_lm))) return bail(rc);
+  }
   if ((size_t)(cur - wbuf) > total) {
     ctx->err = "internal: weight buffer overflow";
     return bail(MK_ERR_INVALID_ARG);
@@ -346,6 +385,18 @@ extern "C" int mk_create(const mk_config* cfg, const mk_weights* w, const mk_opt
       case T_LMHEAD: t.w = lm; break;
       default: t.w = nullptr; break;
     }
+    if (wbytes == 1) {  // the decode GEMVs stream the fp8 codes
+      const uint8_t* c = nullptr;
+      switch (t.kind) {
+        case T_QKV: c = c_qkv[t.layer]; break;
+        case T_OPROJ: c = c_o[t.layer]; break;
+        case T_GATEUP: c = c_gu[t.layer]; break;
+        case T_DOWN: c = c_dn[t.layer]; break;
+        case T_LMHEAD: c = c_lm; break;
+        default: break;
+      }
+      if (c) t.w = reinterpret_cast<const uint16_t*>(c);
+    }
   }
   if ((rc = dalloc(ctx, &ctx->d_tasks, tasks.size() * sizeof(Task)))) return bail(rc);
   if ((rc = dalloc(ctx, &ctx->d_queue, plan.queue.size() * 4))) return bail(rc);
@@ -369,6 +420,7 @@ extern "C" int mk_create(const mk_config* cfg, const mk_weights* w, const mk_opt
   m.attn_scale = (float)(1.0 / std::sqrt((double)d));
   m.n_lm_slots = plan.n_lm_slots;
   m.timeout_ms = ctx->opt.timeout_ms > 0 ? ctx->opt.timeout_ms : 1000;
+  m.wbytes = wbytes;
   m.l2_prefetch_chunks = ctx->opt.l2_prefetch == 0 ? kDefaultL2Prefetch
                                                   : (ctx->opt.l2_prefetch < 0 ? 0 : ctx->opt.l2_prefetch);
   m.trace = nullptr;

@@ -23,6 +23,8 @@
 //                      SwiGLU and the argmax ("Crear desde cero ..." §3.3).
 // A finished task bumps its event counters with a gpu-scope release.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <math.h>
 
 #include "../../include/mk.h"
@@ -104,6 +106,32 @@ __device__ __forceinline__ float2 dot8(const uint4 w, const float2 (&x)[4], floa
   acc = __ffma2_rn(make_float2(bf_lo(w.z), bf_hi(w.z)), x[2], acc);
   acc = __ffma2_rn(make_float2(bf_lo(w.w), bf_hi(w.w)), x[3], acc);
   return acc;
+}
+
+// Sixteen fp8 (e4m3) weights of one 16-byte piece against their inputs: pairs
+// of codes widen exactly to half and then to float.
+__device__ __forceinline__ float2 fp8x2_to_float2(uint32_t two) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)two, __NV_E4M3);
+  return __half22float2(*reinterpret_cast<const __half2*>(&h));
+}
+__device__ __forceinline__ float2 dot16_fp8(const uint4 w, const float2 (&x)[8], float2 acc) {
+  const uint32_t v[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    acc = __ffma2_rn(fp8x2_to_float2(v[q] & 0xffffu), x[2 * q], acc);
+    acc = __ffma2_rn(fp8x2_to_float2(v[q] >> 16), x[2 * q + 1], acc);
+  }
+  return acc;
+}
+
+// Row scales of a task's fp8 matrix: they follow the matrix's codes in the
+// same allocation, at the 16-byte-aligned end of its rows x K bytes.
+__device__ __forceinline__ const float* task_wscale(const ModelDev& m, const Task& t) {
+  const int rows = t.kind == T_QKV ? qkv_rows(m.n_q, m.n_kv, m.head_dim)
+                   : t.kind == T_GATEUP ? 2 * m.ffn
+                   : t.kind == T_LMHEAD ? m.vocab : m.hidden;
+  const size_t off = ((size_t)rows * t.K + 15) & ~(size_t)15;
+  return reinterpret_cast<const float*>(reinterpret_cast<const uint8_t*>(t.w) + off);
 }
 
 __device__ __forceinline__ void set_error(const ModelDev& m, int code, int info) {
@@ -225,9 +253,9 @@ struct ChunkCursor {
         const int r = off < 0 ? t.row0 : off;
         if (r < t.row1) {
           const int nr = min(t.chunk_rows, t.row1 - r);
-          c.src0 = t.w + (size_t)r * t.K;
+          c.src0 = reinterpret_cast<const uint8_t*>(t.w) + (size_t)r * t.K * m.wbytes;
           c.src1 = nullptr;
-          c.bytes0 = (uint32_t)nr * t.K * 2;
+          c.bytes0 = (uint32_t)nr * t.K * m.wbytes;
           c.bytes1 = 0;
           c.kv = false;
           off = r + nr;
@@ -423,12 +451,14 @@ __device__ __forceinline__ void wait_full(Smem& s, uint32_t seq, const ModelDev&
 // thread's share of sum(x^2); the 1/rms factor is applied to the dot products
 // afterwards (W (x * w * r) = r * W (x * w)), so the first ring chunk is not
 // held back by a block-wide reduction.
-template <int CPT>
+// PW: input pairs per 16-byte weight piece -- 4 for bf16 (8 columns), 8 for
+// fp8 (16 columns).
+template <int CPT, int PW>
 __device__ __forceinline__ float gemv_load_input(const KernelArgs& a, const StepParams& sp,
                                                  const Task& t, int wtid, int ct, int rl,
-                                                 float2 (&x2)[CPT][4]) {
+                                                 float2 (&x2)[CPT][PW]) {
   const ModelDev& m = a.m;
-  const int K = t.K, C = K >> 3;
+  const int K = t.K, C = K / (2 * PW);
   const float* src32 = nullptr;
   const uint16_t* src16 = nullptr;
   const uint16_t* normw = nullptr;
@@ -457,33 +487,38 @@ __device__ __forceinline__ float gemv_load_input(const KernelArgs& a, const Step
   for (int c = 0; c < CPT; ++c) {
     const int cc = ct + c * TPR;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) x2[c][e] = make_float2(0.f, 0.f);
+    for (int e = 0; e < PW; ++e) x2[c][e] = make_float2(0.f, 0.f);
     if (cc >= C) continue;
-    if (src16) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(src16) + cc);
-      x2[c][0] = make_float2(bf_lo(v.x), bf_hi(v.x));
-      x2[c][1] = make_float2(bf_lo(v.y), bf_hi(v.y));
-      x2[c][2] = make_float2(bf_lo(v.z), bf_hi(v.z));
-      x2[c][3] = make_float2(bf_lo(v.w), bf_hi(v.w));
-    } else {
-      const float4 u = __ldcg(reinterpret_cast<const float4*>(src32) + 2 * cc);
-      const float4 w = __ldcg(reinterpret_cast<const float4*>(src32) + 2 * cc + 1);
-      x2[c][0] = make_float2(u.x, u.y);
-      x2[c][1] = make_float2(u.z, u.w);
-      x2[c][2] = make_float2(w.x, w.y);
-      x2[c][3] = make_float2(w.z, w.w);
-    }
-    if (normw) {
-      const uint4 wv = __ldg(reinterpret_cast<const uint4*>(normw) + cc);
-      const float2 wn[4] = {make_float2(bf_lo(wv.x), bf_hi(wv.x)), make_float2(bf_lo(wv.y), bf_hi(wv.y)),
-                            make_float2(bf_lo(wv.z), bf_hi(wv.z)), make_float2(bf_lo(wv.w), bf_hi(wv.w))};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        if (rl == 0) {
-          ss = fmaf(x2[c][e].x, x2[c][e].x, ss);
-          ss = fmaf(x2[c][e].y, x2[c][e].y, ss);
+    for (int q = 0; q < PW / 4; ++q) {  // 8-column blocks of this piece
+      const int sc = cc * (PW / 4) + q;
+      float2* xq = &x2[c][4 * q];
+      if (src16) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(src16) + sc);
+        xq[0] = make_float2(bf_lo(v.x), bf_hi(v.x));
+        xq[1] = make_float2(bf_lo(v.y), bf_hi(v.y));
+        xq[2] = make_float2(bf_lo(v.z), bf_hi(v.z));
+        xq[3] = make_float2(bf_lo(v.w), bf_hi(v.w));
+      } else {
+        const float4 u = __ldcg(reinterpret_cast<const float4*>(src32) + 2 * sc);
+        const float4 w = __ldcg(reinterpret_cast<const float4*>(src32) + 2 * sc + 1);
+        xq[0] = make_float2(u.x, u.y);
+        xq[1] = make_float2(u.z, u.w);
+        xq[2] = make_float2(w.x, w.y);
+        xq[3] = make_float2(w.z, w.w);
+      }
+      if (normw) {
+        const uint4 wv = __ldg(reinterpret_cast<const uint4*>(normw) + sc);
+        const float2 wn[4] = {make_float2(bf_lo(wv.x), bf_hi(wv.x)), make_float2(bf_lo(wv.y), bf_hi(wv.y)),
+                              make_float2(bf_lo(wv.z), bf_hi(wv.z)), make_float2(bf_lo(wv.w), bf_hi(wv.w))};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if (rl == 0) {
+            ss = fmaf(xq[e].x, xq[e].x, ss);
+            ss = fmaf(xq[e].y, xq[e].y, ss);
+          }
+          xq[e] = make_float2(xq[e].x * wn[e].x, xq[e].y * wn[e].y);
         }
-        x2[c][e] = make_float2(x2[c][e].x * wn[e].x, x2[c][e].y * wn[e].y);
       }
     }
   }
@@ -491,17 +526,26 @@ __device__ __forceinline__ float gemv_load_input(const KernelArgs& a, const Step
 }
 
 // Streams the task's rows through the ring and leaves y[row] in s.ybuf.
-template <int CPT, int NR>
+template <int CPT, int NR, int PW>
 __device__ __forceinline__ void gemv_stream(const KernelArgs& a, Smem& s, const Task& t, uint32_t& seq, int wtid) {
   const int TPR = t.tpr;
   const int rl = wtid / TPR, ct = wtid % TPR;
   const int wpr = TPR >> 5, wir = ct >> 5;
   const int lane = wtid & 31;
-  const int K = t.K, C = K >> 3;
-  const size_t row_bytes = (size_t)K * 2;
+  const int K = t.K, C = K / (2 * PW);
+  const size_t row_bytes = (size_t)K * 8 / PW;
   const int nrows = t.row1 - t.row0;
-  float2 x2[CPT][4];
-  float ss = gemv_load_input<CPT>(a, s.sp_work, t, wtid, ct, rl, x2);
+  // fp8: the row scales of this thread's output rows (at most two: a task
+  // has at most kYBufFloats = 2 x 512 rows), requested with the inputs
+  static_assert(kYBufFloats <= 2 * kWorkerThreads, "two output rows per thread at most");
+  float rsc0 = 1.f, rsc1 = 1.f;
+  if constexpr (PW == 8) {
+    const float* wsc = task_wscale(a.m, t) + t.row0;
+    if (wtid < nrows) rsc0 = __ldg(wsc + wtid);
+    if (wtid + kWorkerThreads < nrows) rsc1 = __ldg(wsc + wtid + kWorkerThreads);
+  }
+  float2 x2[CPT][PW];
+  float ss = gemv_load_input<CPT, PW>(a, s.sp_work, t, wtid, ct, rl, x2);
   trace_mark(a, s, wtid, 2);
   const bool has_norm = t.kind == T_QKV || t.kind == T_GATEUP || t.kind == T_LMHEAD;
   if (has_norm) {
@@ -526,7 +570,11 @@ __device__ __forceinline__ void gemv_stream(const KernelArgs& a, Smem& s, const 
 #pragma unroll
         for (int c = 0; c < CPT; ++c) {
           const int cc = ct + c * TPR;
-          if (cc < C) a2 = dot8(*reinterpret_cast<const uint4*>(row + (size_t)cc * 16), x2[c], a2);
+          if (cc < C) {
+            const uint4 piece = *reinterpret_cast<const uint4*>(row + (size_t)cc * 16);
+            if constexpr (PW == 4) a2 = dot8(piece, x2[c], a2);
+            else a2 = dot16_fp8(piece, x2[c], a2);
+          }
         }
       }
       acc[j] = a2.x + a2.y;
@@ -561,28 +609,34 @@ __device__ __forceinline__ void gemv_stream(const KernelArgs& a, Smem& s, const 
       y3 += s.scratch[(w + 3) * nrows + i];
     }
     for (; w < wpr; ++w) y0 += s.scratch[w * nrows + i];
-    const float y = (y0 + y1) + (y2 + y3);
+    float y = (y0 + y1) + (y2 + y3);
+    if constexpr (PW == 8) y *= i < kWorkerThreads ? rsc0 : rsc1;  // fp8 row scale
     s.ybuf[i] = has_norm ? y * r : y;
   }
   worker_sync();
 }
 
-template <int CPT>
+template <int CPT, int PW>
 __device__ __forceinline__ void gemv_dispatch_nr(const KernelArgs& a, Smem& s, const Task& t, uint32_t& seq,
                                  int wtid) {
   const int nr = t.chunk_rows / (kWorkerThreads / t.tpr);
-  if (nr >= 4) gemv_stream<CPT, 4>(a, s, t, seq, wtid);
-  else if (nr == 2) gemv_stream<CPT, 2>(a, s, t, seq, wtid);
-  else gemv_stream<CPT, 1>(a, s, t, seq, wtid);
+  if constexpr (PW == 8 && CPT > 2) {
+    gemv_stream<CPT, 1, PW>(a, s, t, seq, wtid);  // (fp8 geometry never has NR > 1 here)
+  } else {
+    if (nr >= 4) gemv_stream<CPT, 4, PW>(a, s, t, seq, wtid);
+    else if (nr == 2) gemv_stream<CPT, 2, PW>(a, s, t, seq, wtid);
+    else gemv_stream<CPT, 1, PW>(a, s, t, seq, wtid);
+  }
 }
 
+template <int PW>
 __device__ __forceinline__ void gemv_core(const KernelArgs& a, Smem& s, const Task& t, uint32_t& seq, int wtid) {
-  const int cpt = (t.K / 8 + t.tpr - 1) / t.tpr;
+  const int cpt = (t.K / (2 * PW) + t.tpr - 1) / t.tpr;
   switch (cpt) {
-    case 1: gemv_dispatch_nr<1>(a, s, t, seq, wtid); break;
-    case 2: gemv_dispatch_nr<2>(a, s, t, seq, wtid); break;
-    case 3: gemv_dispatch_nr<3>(a, s, t, seq, wtid); break;
-    default: gemv_dispatch_nr<4>(a, s, t, seq, wtid); break;
+    case 1: gemv_dispatch_nr<1, PW>(a, s, t, seq, wtid); break;
+    case 2: gemv_dispatch_nr<2, PW>(a, s, t, seq, wtid); break;
+    case 3: gemv_dispatch_nr<3, PW>(a, s, t, seq, wtid); break;
+    default: gemv_dispatch_nr<4, PW>(a, s, t, seq, wtid); break;
   }
 }
 
@@ -1011,6 +1065,7 @@ __device__ __forceinline__ void attn_dispatch(const KernelArgs& a, Smem& s, cons
 
 // ------------------------------------------------------------------ worker
 
+template <int PW>
 __device__ __forceinline__ void worker(const KernelArgs& a, Smem& s, int q0, int q1) {
   const int wtid = threadIdx.x - kFirstWorkerWarp * 32;
   uint32_t seq = 0;
@@ -1031,13 +1086,13 @@ __device__ __forceinline__ void worker(const KernelArgs& a, Smem& s, int q0, int
         finish_task(a, s, t, wtid, true);
         break;
       case T_LMHEAD:
-        gemv_core(a, s, t, seq, wtid);
+        gemv_core<PW>(a, s, t, seq, wtid);
         epilogue_lmhead(a, s, t, wtid);
         finish_task(a, s, t, wtid, false);
         break;
       default: {
         const EpiPre pre = epilogue_prefetch(a, s.sp_work, t, wtid);
-        gemv_core(a, s, t, seq, wtid);
+        gemv_core<PW>(a, s, t, seq, wtid);
         if (t.kind == T_QKV) epilogue_qkv(a, s, t, wtid, pre);
         else if (t.kind == T_GATEUP) epilogue_swiglu(a, s, t, wtid);
         else epilogue_residual(a, s, t, wtid, pre);
@@ -1053,6 +1108,8 @@ __device__ __forceinline__ void worker(const KernelArgs& a, Smem& s, int q0, int
   }
 }
 
+// PW 4: bf16 weights; PW 8: fp8 e4m3 weights with row scales.
+template <int PW>
 __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_constant__ KernelArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   Smem& s = *reinterpret_cast<Smem*>(smem_raw);
@@ -1079,7 +1136,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   } else if (warp == kSchedulerWarp) {
     if (lane == 0) scheduler(a, s, q0, q1);
   } else {
-    worker(a, s, q0, q1);
+    worker<PW>(a, s, q0, q1);
   }
 }
 
@@ -1139,12 +1196,55 @@ __global__ void __launch_bounds__(512) read_probe_kernel(const uint4* __restrict
   if (acc == 0x9e3779b9u) atomicAdd(sink, 1ull);  // data-dependent, practically never taken
 }
 
+// fp8 weights (e4m3) with one power-of-two scale per row: scale = the
+// smallest 2^k with max|w| / 2^k <= 448 (the largest finite e4m3), codes =
+// e4m3(w / scale) rounded to nearest (saturating), and the bf16 matrix is
+// overwritten with the dequantized values code * scale -- exactly
+// representable in bf16 (3 significand bits times a power of two) -- so the
+// tensor-core prefill and the batched step use the same model as the fp8
+// decode GEMVs.  Weights that already are such values are reproduced exactly.
+__global__ void quantize_fp8_rows_kernel(uint16_t* __restrict__ w, uint8_t* __restrict__ codes,
+                                         float* __restrict__ scales, int K) {
+  __shared__ float red[8];
+  __shared__ float sc;
+  const int r = blockIdx.x;
+  uint16_t* row = w + (size_t)r * K;
+  float mx = 0.f;
+  for (int i = threadIdx.x; i < K; i += blockDim.x) mx = fmaxf(mx, fabsf(bf16_to_float(row[i])));
+  for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m2 = 0.f;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) m2 = fmaxf(m2, red[i]);
+    int k = 0;
+    if (m2 > 0.f) {
+      k = (int)ceilf(log2f(m2 / 448.f));
+      while (m2 / ldexpf(1.f, k) > 448.f) ++k;   // the scale must not be too small
+      while (m2 / ldexpf(1.f, k - 1) <= 448.f) --k;  // nor larger than needed
+    }
+    sc = ldexpf(1.f, k);
+    scales[r] = sc;
+  }
+  __syncthreads();
+  const float s = sc;
+  for (int i = threadIdx.x; i < K; i += blockDim.x) {
+    const __nv_fp8_storage_t c = __nv_cvt_float_to_fp8(bf16_to_float(row[i]) / s, __NV_SATFINITE, __NV_E4M3);
+    codes[(size_t)r * K + i] = c;
+    const __half_raw h = __nv_cvt_fp8_to_halfraw(c, __NV_E4M3);
+    row[i] = float_to_bf16_rne(__half2float(*reinterpret_cast<const __half*>(&h)) * s);
+  }
+}
+
 }  // namespace mk
 
 // Host-visible launch helpers (called from api.cu).
 namespace mk {
 size_t step_kernel_smem_bytes() { return sizeof(Smem); }
-const void* step_kernel_ptr() { return reinterpret_cast<const void*>(&mk_step_kernel); }
+const void* step_kernel_ptr(int wbytes) {
+  return wbytes == 1 ? reinterpret_cast<const void*>(&mk_step_kernel<8>)
+                     : reinterpret_cast<const void*>(&mk_step_kernel<4>);
+}
 
 cudaError_t launch_pack_qkv(uint16_t* dst, const uint16_t* wq, const uint16_t* wk,
                             const uint16_t* wv, int H, int G, int d, int rows, cudaStream_t st) {
@@ -1177,6 +1277,12 @@ cudaError_t launch_step(const KernelArgs& args, int grid, bool cooperative, cuda
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = cooperative ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, mk_step_kernel, args);
+  return args.m.wbytes == 1 ? cudaLaunchKernelEx(&cfg, mk_step_kernel<8>, args)
+                            : cudaLaunchKernelEx(&cfg, mk_step_kernel<4>, args);
+}
+cudaError_t launch_quantize_fp8_rows(uint16_t* w, uint8_t* codes, float* scales, int rows, int K,
+                                     cudaStream_t st) {
+  quantize_fp8_rows_kernel<<<rows, 256, 0, st>>>(w, codes, scales, K);
+  return cudaGetLastError();
 }
 }  // namespace mk

@@ -73,7 +73,8 @@ struct ModelDev {
   float rms_eps, attn_scale;
   int32_t n_lm_slots, timeout_ms;  // CTAs holding LM-head tasks (argmax slots)
   int32_t l2_prefetch_chunks;  // chunks past the ring prefetched into L2 when a task must wait (0: off)
-  int32_t pad0_;
+  int32_t wbytes;              // bytes per GEMV weight: 2 (bf16) or 1 (fp8 e4m3; a matrix's
+                               // fp32 row scales follow its codes, 16-byte aligned)
   // packed weights
   const uint16_t* embed;       // [vocab][hidden]
   const uint16_t* lm_head;     // [vocab][hidden] (== embed when tied)
@@ -81,6 +82,7 @@ struct ModelDev {
   const uint16_t* attn_norm;   // [layers][hidden]
   const uint16_t* ffn_norm;    // [layers][hidden]
   const uint16_t* bqkv;        // [layers][qkv_rows] packed order (nullable)
+
   // rope table [max_seq][head_dim/2]
   const float* rope_cos;
   const float* rope_sin;

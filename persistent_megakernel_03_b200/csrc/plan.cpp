@@ -62,8 +62,15 @@ struct Builder {
   EventMap ev;
   std::vector<std::vector<int>> per_cta;  // megakernel queues
 
-  Builder(const mk_config& c_, int P_, Plan& p_)
-      : c(c_), P(P_), p(p_), ev{c_.n_layers, c_.n_kv_heads}, per_cta(P_) {}
+  int wb = 2;  // bytes per GEMV weight
+
+  Builder(const mk_config& c_, int P_, Plan& p_, int wbytes)
+      : c(c_), P(P_), p(p_), ev{c_.n_layers, c_.n_kv_heads}, per_cta(P_), wb(wbytes) {}
+
+  // A GEMV over K columns of wb-byte weights has the geometry of a bf16 GEMV
+  // over K * wb / 2 columns (same bytes per row; a 16-byte piece then holds
+  // 16 / wb columns).
+  int kb(int K) const { return K * wb / 2; }
 
   int add(const Task& t, int cta) {
     p.tasks.push_back(t);
@@ -107,8 +114,8 @@ struct Builder {
     t.sig_ev0 = -1;
     t.n_sig = 0;
     t.K = K;
-    t.tpr = gemv_tpr(K);
-    t.chunk_rows = gemv_chunk_rows(K);
+    t.tpr = gemv_tpr(kb(K));
+    t.chunk_rows = gemv_chunk_rows(kb(K));
     t.w = nullptr;
     t.aux = -1;
     t.stage = kind == T_LMHEAD ? c.n_layers * 5 : layer * 5 + kind;
@@ -129,7 +136,7 @@ struct Builder {
     p.n_stages = 5 * L + 1;
     for (int l = 0; l < L; ++l) {
       // QKV: rows of whole RoPE pairs; signal every group the rows touch.
-      split_rows(qkvR, 2, gemv_max_task_rows(H), [&](int cta, int r0, int r1) {
+      split_rows(qkvR, 2, gemv_max_task_rows(kb(H)), [&](int cta, int r0, int r1) {
         Task t = gemv_task(T_QKV, l, H, r0, r1);
         if (l > 0) { t.wait_ev = ev.down(l - 1); }
         int g0 = r0 / per_group, g1 = (r1 - 1) / per_group;
@@ -156,21 +163,21 @@ struct Builder {
         int cta = (int)((long long)a * P / A);
         add(t, cta);
       }
-      split_rows(H, 1, gemv_max_task_rows(nq * d), [&](int cta, int r0, int r1) {
+      split_rows(H, 1, gemv_max_task_rows(kb(nq * d)), [&](int cta, int r0, int r1) {
         Task t = gemv_task(T_OPROJ, l, nq * d, r0, r1);
         t.wait_ev = ev.attn(l);
         t.sig_ev0 = ev.oproj(l);
         t.n_sig = 1;
         add(t, cta);
       });
-      split_rows(2 * F, 2, gemv_max_task_rows(H), [&](int cta, int r0, int r1) {
+      split_rows(2 * F, 2, gemv_max_task_rows(kb(H)), [&](int cta, int r0, int r1) {
         Task t = gemv_task(T_GATEUP, l, H, r0, r1);
         t.wait_ev = ev.oproj(l);
         t.sig_ev0 = ev.gateup(l);
         t.n_sig = 1;
         add(t, cta);
       });
-      split_rows(H, 1, gemv_max_task_rows(F), [&](int cta, int r0, int r1) {
+      split_rows(H, 1, gemv_max_task_rows(kb(F)), [&](int cta, int r0, int r1) {
         Task t = gemv_task(T_DOWN, l, F, r0, r1);
         t.wait_ev = ev.gateup(l);
         t.sig_ev0 = ev.down(l);
@@ -182,7 +189,7 @@ struct Builder {
     // shared memory and only the CTA's last one publishes it.
     int n_lm = 0, n_slots = 0, last_cta = -1;
     std::vector<int> lm_ids;
-    split_rows(V, 1, gemv_max_task_rows(H), [&](int cta, int r0, int r1) {
+    split_rows(V, 1, gemv_max_task_rows(kb(H)), [&](int cta, int r0, int r1) {
       Task t = gemv_task(T_LMHEAD, L, H, r0, r1);
       t.layer = L - 1;
       t.wait_ev = ev.down(L - 1);
@@ -234,7 +241,7 @@ struct Builder {
 
 }  // namespace
 
-std::string build_plan(const mk_config& c, int num_ctas, int attn_splits, Plan* out) {
+std::string build_plan(const mk_config& c, int num_ctas, int attn_splits, Plan* out, int wbytes) {
   std::string err = validate_config(c);
   if (!err.empty()) return err;
   if (num_ctas <= 0) return "num_ctas must be positive";
@@ -244,7 +251,8 @@ std::string build_plan(const mk_config& c, int num_ctas, int attn_splits, Plan* 
   if (S > 4096) return "attn_splits too large";
   *out = Plan{};
   out->num_ctas = num_ctas;
-  Builder b(c, num_ctas, *out);
+  if (wbytes != 1 && wbytes != 2) return "wbytes must be 1 or 2";
+  Builder b(c, num_ctas, *out, wbytes);
   b.build(S);
   return "";
 }
@@ -264,7 +272,8 @@ extern "C" int mk_plan_build(const mk_config* cfg, const mk_options* opt, int nu
   *out = nullptr;
   mk_plan* h = new mk_plan();
   h->cfg = *cfg;
-  std::string err = mk::build_plan(*cfg, num_ctas, opt ? opt->attn_splits : 0, &h->p);
+  std::string err = mk::build_plan(*cfg, num_ctas, opt ? opt->attn_splits : 0, &h->p,
+                                   opt && opt->weight_format == 1 ? 1 : 2);
   if (!err.empty()) {
     delete h;
     return MK_ERR_INVALID_ARG;

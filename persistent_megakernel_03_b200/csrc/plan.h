@@ -32,7 +32,9 @@ struct Plan {
 std::string validate_config(const mk_config& c);
 
 // Builds the task graph for `num_ctas` CTAs.  attn_splits <= 0: automatic.
-std::string build_plan(const mk_config& c, int num_ctas, int attn_splits, Plan* out);
+// wbytes: bytes per GEMV weight (2 bf16, 1 fp8); a task's geometry (threads
+// per row, rows per ring chunk, rows per task) follows the bytes of a row.
+std::string build_plan(const mk_config& c, int num_ctas, int attn_splits, Plan* out, int wbytes = 2);
 
 // Event indices.
 struct EventMap {

@@ -17,14 +17,14 @@ Activations (a few KB per layer, L2-resident) are not counted.
 from __future__ import annotations
 
 
-def weight_bytes(m) -> int:
+def weight_bytes(m, wbytes: int = 2) -> int:
+    """wbytes: bytes per matrix weight -- 2 for bf16, 1 for fp8 (plus one fp32
+    scale per matrix row); norms and biases stay bf16."""
     h, f, qd, kvd = m.hidden, m.ffn, m.q_dim, m.kv_dim
-    per_layer = (qd + 2 * kvd) * h + h * qd + 2 * f * h + h * f      # matrices
-    per_layer += 2 * h                                               # two norms
-    if m.qkv_bias:
-        per_layer += qd + 2 * kvd
-    total = m.n_layers * per_layer + h + m.vocab * h                 # final norm + LM head
-    return 2 * total
+    mat = m.n_layers * ((qd + 2 * kvd) * h + h * qd + 2 * f * h + h * f) + m.vocab * h
+    rows = m.n_layers * ((qd + 2 * kvd) + h + 2 * f + h) + m.vocab
+    vec = m.n_layers * (2 * h + ((qd + 2 * kvd) if m.qkv_bias else 0)) + h   # norms, biases
+    return wbytes * mat + 2 * vec + (4 * rows if wbytes == 1 else 0)
 
 
 def kv_read_bytes(m, pos: int) -> int:
@@ -35,10 +35,10 @@ def kv_write_bytes(m) -> int:
     return 2 * m.n_layers * m.kv_dim * 2
 
 
-def step_bytes(m, positions, want_logits: bool = False) -> int:
+def step_bytes(m, positions, want_logits: bool = False, wbytes: int = 2) -> int:
     """Bytes one decode step moves for requests at `positions`."""
     n = len(positions)
-    b = weight_bytes(m)
+    b = weight_bytes(m, wbytes)
     b += n * (0 if m.tied_embeddings else m.hidden * 2)   # embedding rows
     if m.tied_embeddings:
         b += 0                                             # rows come from the LM-head read
