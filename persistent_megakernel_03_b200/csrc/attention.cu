@@ -1,11 +1,13 @@
 // attention.cu -- standalone split-KV grouped-query decode attention.
 //
 // One KV head and its G query heads against n cached keys: the keys are cut
-// into `splits` contiguous blocks, one CTA each.  Every warp of a CTA keeps an
-// online softmax (running maximum, running sum, rescaled output) over its
-// keys; the CTA merges its warps and writes its block's partial (unnormalised
-// output at the block maximum, the maximum, the sum) to the workspace; the
-// last CTA to finish merges the blocks ("Hạt nhân là gì ...": the online
+// into `splits` contiguous blocks, one CTA each.  A CTA stages its keys 64 at
+// a time in shared memory (cp.async, double-buffered, so the next block
+// loads while this one is used); each warp keeps an online softmax (running
+// maximum, running sum, rescaled output) over four keys per block; the CTA
+// merges its warps and writes its block's partial (unnormalised output at
+// the block maximum, the maximum, the sum) to the workspace; the last CTA to
+// finish merges the blocks ("Hạt nhân là gì ...": the online
 // softmax gives the exact softmax up to rounding; "LLM高速化勉強会資料" slides
 // 11-13, 28; "Crear desde cero ..." §3.4).  The same math runs inside the
 // persistent decode kernel's attention tasks (attn_math.cuh).
@@ -23,7 +25,8 @@ namespace mk {
 
 void set_last_error(const char* msg);  // api.cu: the message mk_last_error(NULL) returns
 
-constexpr int kAttnOpWarps = 8;
+constexpr int kAttnOpWarps = 16;
+constexpr int kAttnOpKeys = 64;  // keys per staged block
 constexpr int kAttnOpMaxG = 8;
 constexpr size_t kAttnTicketBytes = 256;  // the merge ticket, padded
 
@@ -32,14 +35,37 @@ size_t attn_op_workspace_bytes(int G, int d, int splits) {
   return kAttnTicketBytes + (size_t)splits * G * attn_part_stride(d) * sizeof(float);
 }
 
+__device__ __forceinline__ void op_cp_async(void* dst, const void* src, bool b16) {
+  if (b16)
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                     static_cast<uint32_t>(__cvta_generic_to_shared(dst))), "l"(src) : "memory");
+  else
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(
+                     static_cast<uint32_t>(__cvta_generic_to_shared(dst))), "l"(src) : "memory");
+}
+__device__ __forceinline__ void op_cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void op_cp_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Dynamic shared memory of the op: two K/V blocks and the warps' softmax
+// scratch while streaming; afterwards the warps' states reuse the bytes.
 template <int DPL, int G>
-__global__ void __launch_bounds__(kAttnOpWarps * 32)
+constexpr size_t attn_op_smem() {
+  constexpr size_t loop = (size_t)2 * 2 * kAttnOpKeys * DPL * 32 * 2 + (size_t)kAttnOpWarps * kAttnXbStride * 4;
+  constexpr size_t merge = (size_t)kAttnOpWarps * G * (DPL * 32 + 4) * 4;
+  return loop > merge ? loop : merge;
+}
+
+template <int DPL, int G>
+__global__ void __launch_bounds__(kAttnOpWarps * 32, 1)
     attn_decode_kernel(const float* __restrict__ q, const uint16_t* __restrict__ K,
                        const uint16_t* __restrict__ V, int n, float scale, int splits,
                        uint8_t* __restrict__ ws, float* __restrict__ out) {
   constexpr int d = DPL * 32, PS = d + 4;
-  __shared__ __align__(16) float buf[kAttnOpWarps][G][PS];
-  __shared__ __align__(16) float xb[kAttnOpWarps][kAttnXbStride];
+  constexpr int kBuf = 2 * kAttnOpKeys * d;  // bf16 elements per buffer (K then V)
+  extern __shared__ __align__(16) uint8_t op_raw[];
+  uint16_t* kvbuf = reinterpret_cast<uint16_t*>(op_raw);
+  float* xbs = reinterpret_cast<float*>(kvbuf + 2 * kBuf);
   __shared__ int last;
   unsigned int* ticket = reinterpret_cast<unsigned int*>(ws);
   float* part = reinterpret_cast<float*>(ws + kAttnTicketBytes);
@@ -49,38 +75,66 @@ __global__ void __launch_bounds__(kAttnOpWarps * 32)
 
   AttnState<DPL, G> st;
   attn_init<DPL, G>(st, q, d, scale, lane);
-  // four consecutive keys per warp at a time
-  for (int j0 = k0 + 4 * warp; j0 < k1; j0 += 4 * kAttnOpWarps) {
-    const int nj = min(4, k1 - j0);
-    {
-      float kv[4][DPL];
+  float* xb = xbs + warp * kAttnXbStride;
+  const bool b16 = ((reinterpret_cast<uintptr_t>(K) | reinterpret_cast<uintptr_t>(V)) & 15u) == 0;
+  const int nblk = (k1 - k0 + kAttnOpKeys - 1) / kAttnOpKeys;
+  auto issue = [&](int b) {
+    const int kb = k0 + b * kAttnOpKeys, nk = min(kAttnOpKeys, k1 - kb);
+    uint16_t* dst = kvbuf + (b & 1) * kBuf;
+    const int per = b16 ? 8 : 4;  // bf16 elements per copy
+    const int pieces = nk * d / per;
+    for (int i = threadIdx.x; i < pieces; i += blockDim.x) {
+      op_cp_async(dst + i * per, K + (size_t)kb * d + i * per, b16);
+      op_cp_async(dst + kAttnOpKeys * d + i * per, V + (size_t)kb * d + i * per, b16);
+    }
+  };
+  if (nblk > 0) issue(0);
+  op_cp_commit();
+  for (int b = 0; b < nblk; ++b) {
+    if (b + 1 < nblk) issue(b + 1);
+    op_cp_commit();
+    op_cp_wait<1>();
+    __syncthreads();
+    const int kb = k0 + b * kAttnOpKeys, nk = min(kAttnOpKeys, k1 - kb);
+    const uint16_t* ks = kvbuf + (b & 1) * kBuf;
+    const uint16_t* vs = ks + kAttnOpKeys * d;
+    // four consecutive keys per warp
+    for (int j0 = 4 * warp; j0 < nk; j0 += 4 * kAttnOpWarps) {
+      const int nj = min(4, nk - j0);
+      {
+        float kv[4][DPL];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int jr = attn_key_row<G>(t, lane);
+          if (jr < nj) load_kv_row<DPL>(ks + (size_t)(j0 + jr) * d + lane * DPL, kv[t]);
+          else
+#pragma unroll
+            for (int i = 0; i < DPL; ++i) kv[t][i] = 0.f;
+        }
+        attn_scores4<DPL, G>(st, kv, nj, xb, lane);
+      }
+      float vv[4][DPL];
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
-        const int jr = attn_key_row<G>(t, lane);
-        if (jr < nj) load_kv_row_global<DPL>(K + (size_t)(j0 + jr) * d + lane * DPL, kv[t]);
+        if (t < nj) load_kv_row<DPL>(vs + (size_t)(j0 + t) * d + lane * DPL, vv[t]);
         else
 #pragma unroll
-          for (int i = 0; i < DPL; ++i) kv[t][i] = 0.f;
+          for (int i = 0; i < DPL; ++i) vv[t][i] = 0.f;
       }
-      attn_scores4<DPL, G>(st, kv, nj, xb[warp], lane);
+      attn_update4<DPL, G>(st, vv, xb);
     }
-    float vv[4][DPL];
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      if (t < nj) load_kv_row_global<DPL>(V + (size_t)(j0 + t) * d + lane * DPL, vv[t]);
-      else
-#pragma unroll
-        for (int i = 0; i < DPL; ++i) vv[t][i] = 0.f;
-    }
-    attn_update4<DPL, G>(st, vv, xb[warp]);
+    __syncthreads();  // buffer b & 1 is refilled by block b + 2
   }
+  op_cp_wait<0>();
+  __syncthreads();
+  float* buf = reinterpret_cast<float*>(op_raw);  // [warps][G][PS], reuses the key buffers
 #pragma unroll
   for (int h = 0; h < G; ++h) {
 #pragma unroll
-    for (int i = 0; i < DPL; ++i) buf[warp][h][lane * DPL + i] = st.o[h][i];
+    for (int i = 0; i < DPL; ++i) buf[(warp * G + h) * PS + lane * DPL + i] = st.o[h][i];
     if (lane == 0) {
-      buf[warp][h][d] = st.mx[h];
-      buf[warp][h][d + 1] = st.l[h];
+      buf[(warp * G + h) * PS + d] = st.mx[h];
+      buf[(warp * G + h) * PS + d + 1] = st.l[h];
     }
   }
   __syncthreads();
@@ -90,14 +144,14 @@ __global__ void __launch_bounds__(kAttnOpWarps * 32)
     const int h = idx / (d + 2), i = idx - h * (d + 2);
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kAttnOpWarps; ++w) M = fmaxf(M, buf[w][h][d]);
+    for (int w = 0; w < kAttnOpWarps; ++w) M = fmaxf(M, buf[(w * G + h) * PS + d]);
     float val = 0.f;
     if (M != -INFINITY) {
 #pragma unroll
       for (int w = 0; w < kAttnOpWarps; ++w) {
-        const float mw = buf[w][h][d];
+        const float mw = buf[(w * G + h) * PS + d];
         if (mw == -INFINITY) continue;
-        val = fmaf(__expf(mw - M), i < d ? buf[w][h][i] : buf[w][h][d + 1], val);
+        val = fmaf(__expf(mw - M), i < d ? buf[(w * G + h) * PS + i] : buf[(w * G + h) * PS + d + 1], val);
       }
     }
     mine[h * PS + i] = i == d ? M : val;
@@ -135,14 +189,24 @@ static cudaError_t launch_attn_g(int G, const float* q, const uint16_t* K, const
                                  int n, float scale, int splits, uint8_t* ws, float* out,
                                  cudaStream_t st) {
   const dim3 grid(splits), block(kAttnOpWarps * 32);
+#define MK_OP(G_)                                                                          \
+  {                                                                                        \
+    constexpr size_t sm = attn_op_smem<DPL, G_>();                                         \
+    cudaError_t e = cudaFuncSetAttribute(attn_decode_kernel<DPL, G_>,                      \
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm); \
+    if (e != cudaSuccess) return e;                                                        \
+    attn_decode_kernel<DPL, G_><<<grid, block, sm, st>>>(q, K, V, n, scale, splits, ws, out); \
+    break;                                                                                 \
+  }
   switch (G) {
-    case 1: attn_decode_kernel<DPL, 1><<<grid, block, 0, st>>>(q, K, V, n, scale, splits, ws, out); break;
-    case 2: attn_decode_kernel<DPL, 2><<<grid, block, 0, st>>>(q, K, V, n, scale, splits, ws, out); break;
-    case 4: attn_decode_kernel<DPL, 4><<<grid, block, 0, st>>>(q, K, V, n, scale, splits, ws, out); break;
-    case 7: attn_decode_kernel<DPL, 7><<<grid, block, 0, st>>>(q, K, V, n, scale, splits, ws, out); break;
-    case 8: attn_decode_kernel<DPL, 8><<<grid, block, 0, st>>>(q, K, V, n, scale, splits, ws, out); break;
+    case 1: MK_OP(1)
+    case 2: MK_OP(2)
+    case 4: MK_OP(4)
+    case 7: MK_OP(7)
+    case 8: MK_OP(8)
     default: return cudaErrorInvalidValue;
   }
+#undef MK_OP
   return cudaGetLastError();
 }
 
