@@ -202,6 +202,20 @@ int mk_status(mk_ctx* ctx);
 const char* mk_last_error(const mk_ctx* ctx);
 void mk_destroy(mk_ctx* ctx);
 
+/* Failure-detection hook (host-side injection, no device fault): raises the
+ * wait threshold of one task of the megakernel's task graph by one
+ * completion, so the event it waits on can never reach it.  The next
+ * megakernel step (mk_decode_step of one request, mk_decode_steps, the last
+ * prompt position of mk_prefill) stalls there until timeout_ms, records
+ * MK_ERR_TIMEOUT, and every CTA leaves the launch through its abort path;
+ * mk_status then reports MK_ERR_TIMEOUT and poisons the context, and the
+ * CUDA context stays usable.  task: index into the context's task table
+ * (0 .. tasks - 1), or < 0 for the first task in table order that waits on
+ * an event.  Synchronises the stream.  MK_ERR_INVALID_ARG when the index is
+ * out of range or the task waits on no event.  The change is permanent:
+ * destroy the context afterwards. */
+int mk_inject_stall(mk_ctx* ctx, int task);
+
 /* Split-KV grouped-query decode attention for one KV head ("Hạt nhân là gì
  * ...": online softmax, exact up to rounding; "LLM高速化勉強会資料" slides
  * 11-13 and 28).  q_dev: fp32 [n_q_per_kv][head_dim] query rows of the

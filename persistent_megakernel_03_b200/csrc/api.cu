@@ -3,6 +3,7 @@
 
 #include <algorithm>
 #include <cmath>
+#include <cstddef>
 #include <cstdio>
 #include <cstring>
 #include <string>
@@ -692,6 +693,28 @@ extern "C" void mk_destroy(mk_ctx* ctx) {
   cudaStreamSynchronize(ctx->stream);
   release(ctx);
   delete ctx;
+}
+
+extern "C" int mk_inject_stall(mk_ctx* ctx, int task) {
+  if (!ctx) return MK_ERR_INVALID_ARG;
+  if (ctx->poisoned) return MK_ERR_POISONED;
+  const std::vector<Task>& tasks = ctx->plan.tasks;
+  if (task < 0) {
+    for (size_t i = 0; i < tasks.size(); ++i)
+      if (tasks[i].wait_ev >= 0) {
+        task = (int)i;
+        break;
+      }
+  }
+  if (task < 0 || task >= (int)tasks.size() || tasks[task].wait_ev < 0)
+    return fail(ctx, MK_ERR_INVALID_ARG, "inject stall: no such task waiting on an event");
+  // one more completion than the event receives per step: never reached
+  const uint32_t raised = tasks[task].wait_count + 1u;
+  uint8_t* field = reinterpret_cast<uint8_t*>(ctx->d_tasks + task) + offsetof(Task, wait_count);
+  cudaError_t e = cudaMemcpyAsync(field, &raised, sizeof raised, cudaMemcpyHostToDevice, ctx->stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(ctx->stream);
+  if (e != cudaSuccess) return fail(ctx, MK_ERR_CUDA, std::string("inject stall: ") + cudaGetErrorString(e));
+  return MK_OK;
 }
 
 extern "C" int mk_read_probe(const void* src_dev, size_t bytes, unsigned long long* sink_dev,

@@ -46,6 +46,13 @@ def test_create_rejects_bad_config_without_gpu():
     assert b"head_dim" in L.mk_last_error(None)
 
 
+def test_null_context_calls_are_argument_errors_without_gpu():
+    L = binding.lib()
+    assert L.mk_inject_stall(None, -1) == -1
+    assert L.mk_status(None) == -1
+    assert L.mk_set_mode(None, 0) == -1
+
+
 @pytest.mark.parametrize("model,bad", [
     (synth.TINY, dict(head_dim=96)),
     (synth.TINY, dict(n_kv_heads=3)),
