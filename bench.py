@@ -204,9 +204,9 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
-def load_traffic():
+def load_traffic(workload):
     """DRAM traffic per launch from the committed ncu summary, when it was
-    taken on the current kernel sources."""
+    taken on the current kernel sources and scaled to this workload."""
     import hashlib
     p = os.path.join(ROOT, "profiles", "megakernel_traffic.json")
     if not os.path.exists(p):
@@ -217,7 +217,7 @@ def load_traffic():
     for name in ("kernel.cu", "mk_internal.h", "ptx.cuh", "attn_math.cuh"):
         with open(os.path.join(ROOT, "persistent_megakernel_03_b200", "csrc", name), "rb") as f:
             h.update(f.read())
-    if rec.get("source_sha256") != h.hexdigest():
+    if rec.get("source_sha256") != h.hexdigest() or rec.get("workload") != workload:
         return None
     return rec.get("traffic_bytes_per_launch_full")
 
@@ -433,7 +433,8 @@ def run_mk(args):
         "read_probe_gbs": probe_gbs, "frac_of_read_probe": achieved / probe_gbs,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": peak_src,
-                     "traffic": load_traffic() if n == 1 and not fp8 else None,
+                     "traffic": (load_traffic(args.workload)
+                                 if n == 1 and not fp8 and not args.layers else None),
                      "bytes_per_launch": bytes_mean},
         "baselines": baselines,
         "device_loop": loop,
