@@ -278,6 +278,20 @@ __global__ void rmsnorm_split_kernel(const float* __restrict__ x, const uint16_t
     split_store(xr[i] * r * bf16_val(w[i]), xh, xl, (size_t)t * H + i);
 }
 
+// Sum of split-K partials p[z * pstride], z = 0 .. nparts - 1, added in split
+// order (the same rounding as a plain loop) with the loads issued together.
+__device__ __forceinline__ float sum_parts(const float* __restrict__ p, int nparts, size_t pstride) {
+  float t[kBatchMaxSplitK];
+#pragma unroll
+  for (int z = 0; z < kBatchMaxSplitK; ++z) t[z] = z < nparts ? p[z * pstride] : 0.f;
+  float v = 0.f;
+#pragma unroll
+  for (int z = 0; z < kBatchMaxSplitK; ++z)
+    if (z < nparts) v += t[z];
+  for (int z = kBatchMaxSplitK; z < nparts; ++z) v += p[z * pstride];
+  return v;
+}
+
 // RoPE on the packed q/k rows of each token, q to qout, K/V (bf16) into the
 // cache at the token's (slot, position).  Mirrors the decode step's epilogue.
 __global__ void rope_kv_kernel(const float* __restrict__ y, int ldy, int nparts, size_t pstride,
@@ -292,11 +306,8 @@ __global__ void rope_kv_kernel(const float* __restrict__ y, int ldy, int nparts,
   const int p = pos[t], sl = slot[t];
   for (int pi = blockIdx.y * blockDim.x + threadIdx.x; pi < npairs; pi += blockDim.x * gridDim.y) {
     const int r = 2 * pi;
-    float y0 = 0.f, y1 = 0.f;
-    for (int z = 0; z < nparts; ++z) {  // split-K partial sums, in order
-      y0 += y[z * pstride + (size_t)t * ldy + r];
-      y1 += y[z * pstride + (size_t)t * ldy + r + 1];
-    }
+    float y0 = sum_parts(y + (size_t)t * ldy + r, nparts, pstride);
+    float y1 = sum_parts(y + (size_t)t * ldy + r + 1, nparts, pstride);
     if (bias) {
       y0 += bf16_val(bias[r]);
       y1 += bf16_val(bias[r + 1]);
@@ -408,9 +419,7 @@ __global__ void residual_kernel(float* __restrict__ x, const float* __restrict__
                                 int nparts, size_t pstride) {
   const int t = blockIdx.x;
   for (int i = threadIdx.x; i < H; i += blockDim.x) {
-    float v = 0.f;
-    for (int z = 0; z < nparts; ++z) v += y[z * pstride + (size_t)t * ldy + i];
-    x[(size_t)t * H + i] += v;
+    x[(size_t)t * H + i] += sum_parts(y + (size_t)t * ldy + i, nparts, pstride);
   }
 }
 
@@ -425,9 +434,7 @@ __global__ void residual_rmsnorm_split_kernel(float* __restrict__ x, const float
   float* xr = x + (size_t)t * H;
   float ss = 0.f;
   for (int i = threadIdx.x; i < H; i += blockDim.x) {
-    float v = 0.f;
-    for (int z = 0; z < nparts; ++z) v += y[z * pstride + (size_t)t * ldy + i];
-    const float nx = xr[i] + v;
+    const float nx = xr[i] + sum_parts(y + (size_t)t * ldy + i, nparts, pstride);
     xr[i] = nx;
     ss = fmaf(nx, nx, ss);
   }
@@ -447,11 +454,8 @@ __global__ void swiglu_split_kernel(const float* __restrict__ y, int ldy, int F,
                                     uint16_t* __restrict__ xl) {
   const int t = blockIdx.x;
   for (int j = threadIdx.x; j < F; j += blockDim.x) {
-    float g = 0.f, u = 0.f;
-    for (int z = 0; z < nparts; ++z) {  // split-K partial sums, in order
-      g += y[z * pstride + (size_t)t * ldy + 2 * j];
-      u += y[z * pstride + (size_t)t * ldy + 2 * j + 1];
-    }
+    const float g = sum_parts(y + (size_t)t * ldy + 2 * j, nparts, pstride);
+    const float u = sum_parts(y + (size_t)t * ldy + 2 * j + 1, nparts, pstride);
     split_store(g / (1.0f + expf(-g)) * u, xh, xl, (size_t)t * F + j);
   }
 }
@@ -459,14 +463,16 @@ __global__ void swiglu_split_kernel(const float* __restrict__ y, int ldy, int F,
 // ------------------------------------------------- batched decode step
 // Split-KV decode attention for several requests at once: CTA (split s, KV
 // head g, request r) runs keys [k0, k1) of the request's cache, 64 keys at a
-// time double-buffered through shared memory with cp.async (16-byte pieces),
-// four keys per warp with the decode step's online-softmax update, then
-// merges its 16 warps and writes one partial (output unnormalised at the
-// split's maximum, the maximum, the sum).  About one split per 256 keys
-// holds keys; the rest return at once.
+// time through a 3-stage cp.async pipeline in shared memory (16-byte
+// pieces), four keys per warp with the decode step's online-softmax update,
+// then merges its 16 warps and writes one partial (output unnormalised at
+// the split's maximum, the maximum, the sum).  The keys per split follow
+// from the whole step's keys, so that the splits holding keys fit in about
+// one wave of SMs; the rest return at once.
 constexpr int kBAWarps = 16;
 constexpr int kBAKeys = 64;
-constexpr int kBAKeysPerSplit = 256;
+constexpr int kBAStages = 3;
+constexpr int kBAMinKeysPerSplit = 256;
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
@@ -475,27 +481,47 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-__device__ __forceinline__ int batch_live_splits(int n_keys, int S) {
-  int l = (n_keys + kBAKeysPerSplit - 1) / kBAKeysPerSplit;
+// Keys per split of this step: the step's (request, KV head) key rows spread
+// over the SMs less one per (request, KV head) for rounding up, at least
+// kBAMinKeysPerSplit, and enough that no request needs more than S splits.
+__device__ __forceinline__ int batch_keys_per_split(const BatchParams* bp, int n_kv, int S,
+                                                    int num_sms) {
+  long long total = 0;
+  int nmax = 1;
+  for (int i = 0; i < bp->n; ++i) {
+    const int k = bp->pos[i] + 1;
+    total += k;
+    nmax = max(nmax, k);
+  }
+  const int slots = max(num_sms - bp->n * n_kv, num_sms / 2);
+  long long kps = (total * n_kv + slots - 1) / slots;
+  kps = max(kps, (long long)kBAMinKeysPerSplit);
+  kps = max(kps, (long long)((nmax + S - 1) / S));
+  return (int)kps;
+}
+
+__device__ __forceinline__ int batch_live_splits(int n_keys, int S, int kps) {
+  int l = (n_keys + kps - 1) / kps;
   return l < 1 ? 1 : (l > S ? S : l);
 }
 
 template <int DPL, int G>
 __global__ void __launch_bounds__(kBAWarps * 32, 1)
     batch_attn_kernel(const float* __restrict__ q, const BatchParams* __restrict__ bp, ModelDev m,
-                      int layer, int S, float* __restrict__ part, uint32_t* __restrict__ tickets,
-                      uint16_t* __restrict__ xh, uint16_t* __restrict__ xl) {
+                      int layer, int S, int num_sms, float* __restrict__ part,
+                      uint32_t* __restrict__ tickets, uint16_t* __restrict__ xh,
+                      uint16_t* __restrict__ xl) {
   pdl_trigger();
   pdl_wait();
   constexpr int d = DPL * 32, PS = d + 4;
   constexpr int kBuf = 2 * kBAKeys * d;  // bf16 elements per buffer (K then V)
   extern __shared__ __align__(16) uint8_t ba_raw[];
   uint16_t* buf = reinterpret_cast<uint16_t*>(ba_raw);
-  float* xbs = reinterpret_cast<float*>(buf + 2 * kBuf);
+  float* xbs = reinterpret_cast<float*>(buf + kBAStages * kBuf);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int sp = blockIdx.x, g = blockIdx.y, r = blockIdx.z;
   const int n_keys = bp->pos[r] + 1;
-  const int live = batch_live_splits(n_keys, S);
+  const int live = batch_live_splits(n_keys, S, batch_keys_per_split(bp, m.n_kv, S, num_sms));
   if (sp >= live) return;
   const int chunk = (n_keys + live - 1) / live;
   const int k0 = min(n_keys, sp * chunk), k1 = min(n_keys, k0 + chunk);
@@ -510,22 +536,27 @@ __global__ void __launch_bounds__(kBAWarps * 32, 1)
   const int nblk = (k1 - k0 + kBAKeys - 1) / kBAKeys;
   auto issue = [&](int b) {
     const int kb = k0 + b * kBAKeys, nk = min(kBAKeys, k1 - kb);
-    uint16_t* dst = buf + (b & 1) * kBuf;
+    uint16_t* dst = buf + (b % kBAStages) * kBuf;
     const int pieces = nk * d / 8;  // 16-byte pieces of K (and of V)
     for (int i = threadIdx.x; i < pieces; i += blockDim.x) {
       cp_async16(dst + i * 8, K + (size_t)kb * d + i * 8);
       cp_async16(dst + kBAKeys * d + i * 8, V + (size_t)kb * d + i * 8);
     }
   };
-  if (nblk > 0) issue(0);
-  cp_async_commit();
-  for (int b = 0; b < nblk; ++b) {
-    if (b + 1 < nblk) issue(b + 1);
+  // blocks 0 .. kBAStages - 2 in flight before the loop; block b + kBAStages - 1
+  // is requested while block b is used (one commit group per block)
+#pragma unroll
+  for (int b = 0; b < kBAStages - 1; ++b) {
+    if (b < nblk) issue(b);
     cp_async_commit();
-    cp_async_wait<1>();
+  }
+  for (int b = 0; b < nblk; ++b) {
+    if (b + kBAStages - 1 < nblk) issue(b + kBAStages - 1);
+    cp_async_commit();
+    cp_async_wait<kBAStages - 1>();
     __syncthreads();
     const int kb = k0 + b * kBAKeys, nk = min(kBAKeys, k1 - kb);
-    const uint16_t* ks = buf + (b & 1) * kBuf;
+    const uint16_t* ks = buf + (b % kBAStages) * kBuf;
     const uint16_t* vs = ks + kBAKeys * d;
     for (int j0 = 4 * warp; j0 < nk; j0 += 4 * kBAWarps) {
       const int nj = min(4, nk - j0);
@@ -551,7 +582,7 @@ __global__ void __launch_bounds__(kBAWarps * 32, 1)
       }
       attn_update4<DPL, G>(st, vv, xb);
     }
-    __syncthreads();  // buffer b & 1 is refilled by block b + 2
+    __syncthreads();  // this buffer is refilled by block b + kBAStages
   }
   cp_async_wait<0>();
   __syncthreads();
@@ -689,9 +720,7 @@ __global__ void b_residual_norm_kernel(float* __restrict__ x, const float* __res
   float ss = 0.f;
   const int i0 = blockIdx.x * 1024 + threadIdx.x * 4;
   for (int i = i0; i < min(H, i0 + 4); ++i) {
-    float v = 0.f;
-    for (int z = 0; z < nparts; ++z) v += y[z * pstride + (size_t)t * ldy + i];
-    const float nx = x[(size_t)t * H + i] + v;
+    const float nx = x[(size_t)t * H + i] + sum_parts(y + (size_t)t * ldy + i, nparts, pstride);
     x[(size_t)t * H + i] = nx;
     ss = fmaf(nx, nx, ss);
     split_store(nx * bf16_val(w[i]), xh, xl, (size_t)t * H + i);
@@ -707,11 +736,8 @@ __global__ void b_swiglu_kernel(const float* __restrict__ y, int ldy, int F, int
   const int t = blockIdx.y;
   const int j0 = blockIdx.x * 1024 + threadIdx.x * 4;
   for (int j = j0; j < min(F, j0 + 4); ++j) {
-    float g = 0.f, u = 0.f;
-    for (int z = 0; z < nparts; ++z) {
-      g += y[z * pstride + (size_t)t * ldy + 2 * j];
-      u += y[z * pstride + (size_t)t * ldy + 2 * j + 1];
-    }
+    const float g = sum_parts(y + (size_t)t * ldy + 2 * j, nparts, pstride);
+    const float u = sum_parts(y + (size_t)t * ldy + 2 * j + 1, nparts, pstride);
     split_store(g / (1.0f + expf(-g)) * u, xh, xl, (size_t)t * F + j);
   }
 }
@@ -989,16 +1015,18 @@ namespace {
 
 template <int DPL, int G>
 size_t batch_attn_smem() {
-  // two key/value buffers and the warps' softmax scratch; after the key loop
-  // the warps' states (16 x G x (d + 4) floats) reuse the same bytes
-  const size_t loop = (size_t)2 * 2 * kBAKeys * DPL * 32 * 2 + (size_t)kBAWarps * kAttnXbStride * 4;
+  // kBAStages key/value buffers and the warps' softmax scratch; after the key
+  // loop the warps' states (16 x G x (d + 4) floats) reuse the same bytes
+  const size_t loop =
+      (size_t)kBAStages * 2 * kBAKeys * DPL * 32 * 2 + (size_t)kBAWarps * kAttnXbStride * 4;
   const size_t merge = (size_t)kBAWarps * G * (DPL * 32 + 4) * 4;
   return loop > merge ? loop : merge;
 }
 
 template <int DPL, int G>
 std::string launch_batch_attn(dim3 grid, cudaStream_t st, const float* q, const BatchParams* bp,
-                              const ModelDev& m, int layer, int S, float* part, bool set_attr,
+                              const ModelDev& m, int layer, int S, int num_sms, float* part,
+                              bool set_attr,
                               uint32_t* tickets, uint16_t* xh, uint16_t* xl) {
   auto k = batch_attn_kernel<DPL, G>;
   const size_t smem = batch_attn_smem<DPL, G>();
@@ -1006,17 +1034,19 @@ std::string launch_batch_attn(dim3 grid, cudaStream_t st, const float* q, const 
     return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) == cudaSuccess
                ? "" : "batched attention shared memory attribute";
   }
-  const cudaError_t e = launch_pdl(k, grid, dim3(kBAWarps * 32), smem, st, q, bp, m, layer, S, part,
-                                   tickets, xh, xl);
+  const cudaError_t e = launch_pdl(k, grid, dim3(kBAWarps * 32), smem, st, q, bp, m, layer, S, num_sms,
+                                   part, tickets, xh, xl);
   return e == cudaSuccess ? "" : std::string("batched attention launch: ") + cudaGetErrorString(e);
 }
 
 std::string batch_attn(dim3 grid, cudaStream_t st, const float* q, const BatchParams* bp,
-                       const ModelDev& m, int layer, int S, float* part, bool set_attr = false,
+                       const ModelDev& m, int layer, int S, int num_sms, float* part,
+                       bool set_attr = false,
                        uint32_t* tickets = nullptr, uint16_t* xh = nullptr, uint16_t* xl = nullptr) {
   const int G = m.group;
 #define MK_BA(DPL_, G_) \
-  return launch_batch_attn<DPL_, G_>(grid, st, q, bp, m, layer, S, part, set_attr, tickets, xh, xl)
+  return launch_batch_attn<DPL_, G_>(grid, st, q, bp, m, layer, S, num_sms, part, set_attr, tickets, \
+                                     xh, xl)
   if (m.head_dim == 128) {
     if (G == 1) MK_BA(4, 1);
     if (G == 2) MK_BA(4, 2);
@@ -1099,7 +1129,7 @@ std::string batch_enqueue(const ModelDev& m, const PrefillWeights& w, BatchScrat
       return e;
     CKL(launch_pdl(rope_kv_kernel, dim3(n, psl), dim3(256), 0, st, (const float*)bs.y, ldy, zq, pstride,
                    bias, (const int32_t*)bp->slot, (const int32_t*)bp->pos, m, l, bs.q));
-    if (!(e = batch_attn(dim3(bs.splits, m.n_kv, n), st, bs.q, bp, m, l, bs.splits, bs.part, false,
+    if (!(e = batch_attn(dim3(bs.splits, m.n_kv, n), st, bs.q, bp, m, l, bs.splits, num_sms, bs.part, false,
                          bs.tickets, xhl, lo(qd))).empty())
       return e;
     if (!(e = gemm_hl(w.o[l], H, qd, xhl, n, bs.y, ldy, bs.err, st, zo, nullptr, 0.f, nullptr, true)).empty())
@@ -1174,7 +1204,7 @@ std::string batch_alloc(const ModelDev& m, int num_sms, BatchScratch* bs, std::v
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)gemm_smem_bytes<16, kDStagesPair, true>()) != cudaSuccess)
     return "decode GEMM shared memory attribute";
-  return batch_attn(dim3(1), nullptr, nullptr, nullptr, m, 0, bs->splits, nullptr, true);
+  return batch_attn(dim3(1), nullptr, nullptr, nullptr, m, 0, bs->splits, num_sms, nullptr, true);
 }
 
 std::string batch_step(const ModelDev& m, const PrefillWeights& w, BatchScratch& bs, int n,
