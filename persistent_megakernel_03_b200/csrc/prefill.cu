@@ -647,20 +647,28 @@ __global__ void __launch_bounds__(kBAWarps * 32, 1)
   if (!is_last) return;
   __threadfence();  // the other splits' partials, after their tickets
   const float* pg = part + (size_t)(r * m.n_kv + g) * S * G * PS;
+  // every split's (maximum, sum) into shared memory (the warps' states are
+  // no longer needed), then each output element from the splits' partials
+  float* ml = reinterpret_cast<float*>(ba_raw);  // [live][G][2]
+  for (int idx = threadIdx.x; idx < live * G; idx += blockDim.x) {
+    const float2 v = __ldcg(reinterpret_cast<const float2*>(pg + (size_t)idx * PS + d));
+    ml[2 * idx] = v.x;
+    ml[2 * idx + 1] = v.y;
+  }
+  __syncthreads();
   for (int idx = threadIdx.x; idx < G * d; idx += blockDim.x) {
     const int h = idx / d, i = idx - h * d;
     float M = -INFINITY;
-    for (int s2 = 0; s2 < live; ++s2) {
-      const float* ps = pg + ((size_t)s2 * G + h) * PS;
-      if (__ldcg(ps + d + 1) != 0.f) M = fmaxf(M, __ldcg(ps + d));
-    }
+    for (int s2 = 0; s2 < live; ++s2)
+      if (ml[2 * (s2 * G + h) + 1] != 0.f) M = fmaxf(M, ml[2 * (s2 * G + h)]);
     float num = 0.f, den = 0.f;
+#pragma unroll 4
     for (int s2 = 0; s2 < live; ++s2) {
-      const float* ps = pg + ((size_t)s2 * G + h) * PS;
-      const float ls = __ldcg(ps + d + 1);
+      const float ls = ml[2 * (s2 * G + h) + 1];
+      const float o = __ldcg(pg + ((size_t)s2 * G + h) * PS + i);
       if (ls == 0.f) continue;
-      const float c = __expf(__ldcg(ps + d) - M);
-      num = fmaf(c, __ldcg(ps + i), num);
+      const float c = __expf(ml[2 * (s2 * G + h)] - M);
+      num = fmaf(c, o, num);
       den = fmaf(c, ls, den);
     }
     split_store(num / den, xh, xl, out_row + (size_t)h * d + i);
