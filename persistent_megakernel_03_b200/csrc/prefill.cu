@@ -423,31 +423,6 @@ __global__ void residual_kernel(float* __restrict__ x, const float* __restrict__
   }
 }
 
-// x[t] += sum of the nparts partials of y[t]; then [xh, xl][t] =
-// split(x[t] * w / sqrt(mean(x[t]^2) + eps)) for the next contraction.
-__global__ void residual_rmsnorm_split_kernel(float* __restrict__ x, const float* __restrict__ y,
-                                              int H, int ldy, int nparts, size_t pstride,
-                                              const uint16_t* __restrict__ w, float eps,
-                                              uint16_t* __restrict__ xh, uint16_t* __restrict__ xl) {
-  __shared__ float red[32];
-  const int t = blockIdx.x;
-  float* xr = x + (size_t)t * H;
-  float ss = 0.f;
-  for (int i = threadIdx.x; i < H; i += blockDim.x) {
-    const float nx = xr[i] + sum_parts(y + (size_t)t * ldy + i, nparts, pstride);
-    xr[i] = nx;
-    ss = fmaf(nx, nx, ss);
-  }
-  for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
-  __syncthreads();
-  float tot = 0.f;
-  for (int i = 0; i < (int)(blockDim.x >> 5); ++i) tot += red[i];
-  const float r = 1.0f / sqrtf(tot / (float)H + eps);
-  for (int i = threadIdx.x; i < H; i += blockDim.x)
-    split_store(xr[i] * r * bf16_val(w[i]), xh, xl, (size_t)t * H + i);
-}
-
 // [xh, xl][t][j] = split(silu(gate_j) * up_j); gate/up interleaved in y.
 __global__ void swiglu_split_kernel(const float* __restrict__ y, int ldy, int F, int nparts,
                                     size_t pstride, uint16_t* __restrict__ xh,
