@@ -167,7 +167,9 @@ int mk_decode_steps(mk_ctx* ctx, const int32_t* token_dev, int pos0, int n_steps
                     float* last_logits_dev);
 
 /* mk_decode_step from and to HOST memory: copies the tokens in, runs the
- * step, copies the next ids out and synchronises the stream. */
+ * step, copies the next ids out and synchronises the stream.  Token ids
+ * outside [0, vocab) are rejected before anything is enqueued
+ * (MK_ERR_TOKEN_RANGE; the context is not poisoned). */
 int mk_decode_step_host(mk_ctx* ctx, const int32_t* tokens_host, const int32_t* pos_host,
                         int n_req, int32_t* next_ids_host);
 

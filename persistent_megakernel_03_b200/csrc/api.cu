@@ -545,6 +545,10 @@ extern "C" int mk_decode_step_host(mk_ctx* ctx, const int32_t* tokens_host, cons
   if (rc) return rc;
   if (!tokens_host || !next_ids_host) return fail(ctx, MK_ERR_INVALID_ARG, "null host buffer");
   if ((rc = check_step_args(ctx, pos_host, n_req))) return rc;
+  for (int r = 0; r < n_req; ++r)  // host tokens: checked before anything is enqueued
+    if (tokens_host[r] < 0 || tokens_host[r] >= ctx->cfg.vocab)
+      return fail(ctx, MK_ERR_TOKEN_RANGE,
+                  "token id " + std::to_string(tokens_host[r]) + " outside [0, vocab)");
   memcpy(ctx->h_pinned, tokens_host, (size_t)n_req * 4);
   CK(cudaMemcpyAsync(ctx->d_tokens, ctx->h_pinned, (size_t)n_req * 4, cudaMemcpyHostToDevice, ctx->stream));
   if ((rc = mk_decode_step(ctx, ctx->d_tokens, pos_host, n_req, nullptr, ctx->d_ids))) return rc;

@@ -151,6 +151,17 @@ def test_token_out_of_range_is_reported_not_faulted(tiny, cuda_ok):
         dec.decode(tok, [1])
 
 
+def test_host_token_out_of_range_is_rejected_before_launch(tiny, cuda_ok):
+    cfg, w, tr = tiny
+    dec = binding.Decoder(cfg, {k: v.cuda() for k, v in w.items()}, 32)
+    for bad in (cfg.vocab, -1):
+        with pytest.raises(binding.MkError, match="TOKEN_RANGE"):
+            dec.decode_host([bad], [0])
+    assert dec.status() == 0  # an argument error does not poison the context
+    out = dec.decode_host([0], [0])
+    assert 0 <= out[0] < cfg.vocab and dec.status() == 0
+
+
 WIDE = [
     synth.QWEN05B.with_layers(2),
     synth.LLAMA8B.with_layers(2),
