@@ -164,41 +164,95 @@ def oracle_sample(model, w_cpu, n_steps: int, budget_s: float, first_pos: int = 
 
 
 def run_reference(args):
+    """The oracle as it stands, timed on the host's cores on the megakernel
+    arm's workload (same metric, unit and config): W untimed and K timed
+    steps, a step decoding one token of every request at the positions the
+    megakernel arm decodes.  So that any K finishes within the time budget
+    (MK_REF_BUDGET_S, default 120 s), a step may run the oracle on the model's
+    first Ls layers (with its final norm and LM head); each request's time
+    then scales to the whole model by the ratio of the two decode steps'
+    algorithmic bytes (the oracle's GEMVs stream its weights from host
+    memory).  The cache positions before the first decoded one hold random
+    values: the timing does not depend on them."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
+    import numpy as np
     import torch
 
-    from persistent_megakernel_03_b200 import synth
-    model = synth.LLAMA8B
+    import oracle
+    from persistent_megakernel_03_b200 import roofline, synth
+    spec = workload_spec(args)
+    model, lens, n, W, K = spec.model, spec.lens, spec.n, spec.W, spec.K
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     w = synth.make_model(model, 0, device=dev)
     w_cpu = {k: v.cpu() for k, v in w.items()}
     del w
-    budget = float(os.environ.get("MK_REF_BUDGET_S", "60"))
-    n = max(2, min(args.warmup + args.steps, 64))
-    long_ctx = args.workload == "llama8b-32k"
-    prompt_len = LONG_PROMPT if long_ctx else SHORT_PROMPT
-    first_pos = prompt_len if long_ctx else 0
-    times, cores = oracle_sample(model, w_cpu, n, budget, first_pos)
-    warm = min(1, len(times) - 1)
-    timed = times[warm:]
-    ms = 1e3 * sum(timed) / len(timed)
-    sample = (f"{len(timed)} oracle decode steps of the Llama-3-8B shape at positions "
-              f"{first_pos + warm}..{first_pos + len(times) - 1} (after {warm} untimed), bf16 "
-              f"weights widened to fp32 on the fly, {cores} OpenMP threads"
-              + (" (cache of the earlier positions filled with random bf16 values: the "
-                 "timing does not depend on them)" if long_ctx else ""))
+    budget = float(os.environ.get("MK_REF_BUDGET_S", "120"))
+    rng = np.random.default_rng(0)
+
+    def states(m):
+        om = oracle.OracleModel(m, w_cpu)
+        sts = []
+        for r in range(n):
+            st = om.new_state(lens[r] + W + K + 1)
+            fill = rng.standard_normal((lens[r], m.head_dim), dtype=np.float32)
+            for l in range(m.n_layers):
+                for g in range(m.n_kv_heads):
+                    for which in (0, 1):
+                        st.set_kv(l, g, which, fill)
+            sts.append(st)
+        return om, sts
+
+    def step(om, sts, j):
+        """One step (positions lens[r] + j); per-request seconds."""
+        out = []
+        for r in range(n):
+            t0 = time.perf_counter()
+            om.decode(sts[r], 1, lens[r] + j, want_logits=False)
+            out.append(time.perf_counter() - t0)
+        return out
+
+    def nbytes(m, p):
+        return roofline.step_bytes(m, [p])
+
+    # the depth Ls whose W + K steps fit the budget, from a one-layer probe
+    m1 = model.with_layers(1)
+    om, sts = states(m1)
+    step(om, sts, 0)
+    t1 = sum(step(om, sts, 1))
+    del om, sts
+    per_step_full = t1 * nbytes(model, lens[0]) / nbytes(m1, lens[0])
+    Ls = model.n_layers
+    while Ls > 1 and (W + K) * per_step_full * nbytes(model.with_layers(Ls), lens[0]) / \
+            nbytes(model, lens[0]) > budget:
+        Ls -= 1
+    ms_ = model if Ls == model.n_layers else model.with_layers(Ls)
+    om, sts = states(ms_)
+    scaled = []
+    for j in range(W + K):
+        per_req = step(om, sts, j)
+        if j >= W:
+            scaled.append(sum(t * nbytes(model, lens[r] + j) / nbytes(ms_, lens[r] + j)
+                              for r, t in enumerate(per_req)))
+    cores = oracle.num_threads()
+    ms = 1e3 * sum(scaled) / len(scaled)
+    depth = (f"all {model.n_layers} layers" if Ls == model.n_layers else
+             f"the first {Ls} of {model.n_layers} layers with the final norm and LM head, "
+             f"scaled to the whole model by the algorithmic bytes")
+    sample = (f"{K} oracle steps ({W} untimed before them) of the {spec.shape_cap} model "
+              f"at the megakernel arm's positions, {depth}; fp32 with bf16 weights widened "
+              f"on the fly, {cores} OpenMP threads"
+              + (f"; one decode per request, {n} requests per step" if n > 1 else ""))
     line = {
-        "impl": "reference", "metric": METRIC, "value": ms, "unit": "ms/token",
-        "n_gpus": args.gpus, "steps": len(timed), "warmup": warm, "ms_per_step": ms,
+        "impl": "reference", "metric": spec.metric, "value": ms, "unit": spec.unit,
+        "n_gpus": args.gpus, "steps": K, "warmup": W, "ms_per_step": ms,
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
-        "config": {"workload": f"llama-3-8b-shape decode, batch 1, {prompt_len}-token random "
-                               "prompt, greedy decode", "sample": "bounded oracle sample"},
-        "cpu_baseline": {"value": ms, "unit": "ms/token", "cores": cores, "kind": "oracle",
+        "config": {"workload": spec.workload, "sample": "bounded oracle sample"},
+        "cpu_baseline": {"value": ms, "unit": spec.unit, "cores": cores, "kind": "oracle",
                          "sample": sample},
-        "e2e": {"value": ms, "unit": "ms/token", "h2d_bytes_per_step": 0,
+        "e2e": {"value": ms, "unit": spec.unit, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -222,17 +276,16 @@ def load_traffic(workload):
     return rec.get("traffic_bytes_per_launch_full")
 
 
-def run_mk(args):
-    import numpy as np
-    import torch
+def workload_spec(args):
+    """The model, prompt lengths, step counts, metric, unit and workload
+    description of one workload, as both arms report it."""
+    from types import SimpleNamespace
 
-    from persistent_megakernel_03_b200 import binding, roofline, synth
-
-    rank, world, local = dist_setup(args.gpus)
-    torch.cuda.set_device(local)
-    model = synth.QWEN05B if args.workload == "qwen05b" else synth.LLAMA8B
-    shape = "qwen2.5-0.5b-shape" if args.workload == "qwen05b" else "llama-3-8b-shape"
-    shape_cap = "Qwen2.5-0.5B-shape" if args.workload == "qwen05b" else "Llama-3-8B-shape"
+    from persistent_megakernel_03_b200 import synth
+    qwen = args.workload == "qwen05b"
+    model = synth.QWEN05B if qwen else synth.LLAMA8B
+    shape = "qwen2.5-0.5b-shape" if qwen else "llama-3-8b-shape"
+    shape_cap = "Qwen2.5-0.5B-shape" if qwen else "Llama-3-8B-shape"
     if args.layers:
         model = model.with_layers(args.layers)
     W, K = args.warmup, args.steps
@@ -245,6 +298,32 @@ def run_mk(args):
     n = len(lens)
     if args.workload in ("llama8b-32k", "llama8b-batch8") and W + K > LONG_STEPS:
         K = LONG_STEPS - W   # these workloads decode 256 steps after their prompts
+    if n == 1:
+        workload = (f"{shape} decode, batch 1, {lens[0]}-token random prompt, "
+                    f"greedy decode steps {lens[0] + W}..{lens[0] + W + K - 1} timed")
+        unit = "ms/token"
+        metric = METRIC if model.name.startswith("llama") else (
+            f"decode ms/token (batch 1, {shape_cap}) & achieved HBM GB/s vs 8 TB/s peak")
+    else:
+        workload = (f"llama-3-8b-shape decode, {n} requests per step, random prompts of "
+                    f"{lens} tokens packed with offsets, greedy decode steps {W}..{W + K - 1} "
+                    "after each prompt timed; one batched step per token (tcgen05 GEMMs over "
+                    "the requests' columns, each weight matrix streamed once; CUDA graph)")
+        unit, metric = "ms/step", f"decode ms/step ({n} requests, Llama-3-8B-shape)"
+    return SimpleNamespace(model=model, shape=shape, shape_cap=shape_cap, lens=lens, n=n,
+                           W=W, K=K, workload=workload, unit=unit, metric=metric)
+
+
+def run_mk(args):
+    import numpy as np
+    import torch
+
+    from persistent_megakernel_03_b200 import binding, roofline, synth
+
+    rank, world, local = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    spec = workload_spec(args)
+    model, shape_cap, lens, n, W, K = spec.model, spec.shape_cap, spec.lens, spec.n, spec.W, spec.K
     max_seq = max(lens) + W + K + 1
     w = synth.make_model(model, 0, device="cuda")
     fp8 = args.weights == "fp8"
@@ -403,18 +482,7 @@ def run_mk(args):
             json.dump(trace_summary, f, indent=1)
 
     clocks = clk.summary()
-    if n == 1:
-        workload = (f"{shape} decode, batch 1, {lens[0]}-token random prompt, "
-                    f"greedy decode steps {lens[0] + W}..{lens[0] + W + K - 1} timed")
-        unit = "ms/token"
-        metric = METRIC if model.name.startswith("llama") else (
-            f"decode ms/token (batch 1, {shape_cap}) & achieved HBM GB/s vs 8 TB/s peak")
-    else:
-        workload = (f"llama-3-8b-shape decode, {n} requests per step, random prompts of "
-                    f"{lens} tokens packed with offsets, greedy decode steps {W}..{W + K - 1} "
-                    "after each prompt timed; one batched step per token (tcgen05 GEMMs over "
-                    "the requests' columns, each weight matrix streamed once; CUDA graph)")
-        unit, metric = "ms/step", f"decode ms/step ({n} requests, Llama-3-8B-shape)"
+    workload, unit, metric = spec.workload, spec.unit, spec.metric
     line = {
         "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": K,
         "warmup": W, "ms_per_step": total_ms / K, "higher_is_better": False,
