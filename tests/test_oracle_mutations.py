@@ -27,6 +27,22 @@ MUTATIONS = {
     "oproj_residual_dropped": ("for (int i = 0; i < H; ++i) x[i] = x[i] + tmp[i];",
                                "for (int i = 0; i < H; ++i) x[i] = tmp[i];"),
     "bias_dropped": ("y[i] = y[i] + bf16_to_f32(b[i]);", "y[i] = y[i];"),
+    "ffn_norm_uses_attn_norm": ("orc_rmsnorm(x, L->ffn_norm, c->hidden, c->rms_eps, xn);",
+                                "orc_rmsnorm(x, L->attn_norm, c->hidden, c->rms_eps, xn);"),
+    "final_norm_uses_a_layer_norm": (
+        "orc_rmsnorm(x, m->final_norm, c->hidden, c->rms_eps, xn);",
+        "orc_rmsnorm(x, m->layers[c->n_layers - 1].ffn_norm, c->hidden, c->rms_eps, xn);"),
+    "lm_head_always_tied": ("m->lm_head = lm_head ? lm_head : embed;", "m->lm_head = embed;"),
+    "eps_outside_sqrt": ("float r = 1.0f / sqrtf(ss / (float)n + eps);",
+                         "float r = 1.0f / (sqrtf(ss / (float)n) + eps);"),
+    "rope_pairs_adjacent": ("float a = v[i], b = v[i + half];\n    v[i] = a * c - b * s;\n"
+                            "    v[i + half] = a * s + b * c;",
+                            "float a = v[2 * i], b = v[2 * i + 1];\n    v[2 * i] = a * c - b * s;\n"
+                            "    v[2 * i + 1] = a * s + b * c;"),
+    "v_stored_as_k": ("kv_store(s, kv_index(c, s->max_seq, l, h, 0, pos), k + (size_t)h * d, d);",
+                      "kv_store(s, kv_index(c, s->max_seq, l, h, 0, pos), v + (size_t)h * d, d);"),
+    "embedding_row": ("const uint16_t* e = m->embed + (size_t)token * H;",
+                      "const uint16_t* e = m->embed + (size_t)(token ^ 1) * H;"),
 }
 
 QWEN_MINI = synth.ModelConfig("qwen-mini", n_layers=2, hidden=128, n_q_heads=6, n_kv_heads=2,
@@ -87,10 +103,10 @@ def _pins_pass(L, hf_refs) -> bool:
 
 @pytest.fixture(scope="module")
 def hf_refs():
-    from test_oracle_pins import _hf_model
+    from test_oracle_pins import _hf_model, _random_norms
     refs = []
     for cfg in (synth.TINY, QWEN_MINI):
-        w = synth.make_model(cfg, 0)
+        w = _random_norms(synth.make_model(cfg, 0), 5)
         toks = synth.make_prompt(10, cfg.vocab).numpy()
         with torch.no_grad():
             ref = _hf_model(cfg, w)(torch.from_numpy(toks.astype(np.int64))[None]).logits[0]

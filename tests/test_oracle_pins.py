@@ -344,12 +344,27 @@ def _hf_model(cfg, w):
     return model
 
 
+def _random_norms(w, seed: int):
+    """The same weights with every RMSNorm weight drawn as 1 + 0.25 N(0, 1)
+    (bf16): the synthetic models' unit norms hide which norm a step applies."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    out = dict(w)
+    for k, t in w.items():
+        if k.endswith("norm"):
+            out[k] = (1.0 + 0.25 * torch.randn(t.shape, generator=g)).to(torch.bfloat16)
+    return out
+
+
+@pytest.mark.parametrize("norms", ["unit", "random"])
 @pytest.mark.parametrize("cfg", [synth.TINY, SMALL_QWEN], ids=lambda c: c.name)
-def test_forward_matches_transformers_library(cfg):
+def test_forward_matches_transformers_library(cfg, norms):
     """An independent implementation of the same decoder (Llama / Qwen2 in
-    transformers, fp32, no KV rounding) must give the oracle's logits."""
+    transformers, fp32, no KV rounding) must give the oracle's logits, also
+    with non-unit norm weights."""
     torch.manual_seed(0)
     w = synth.make_model(cfg, 0)
+    if norms == "random":
+        w = _random_norms(w, 3)
     hf = _hf_model(cfg, w)
     toks = synth.make_prompt(12, cfg.vocab).numpy()
     with torch.no_grad():
