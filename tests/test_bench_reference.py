@@ -36,3 +36,19 @@ def test_reference_line_matches_the_megakernel_arm_workload():
 
 def test_reference_arm_prints_on_rank_zero_only():
     assert _run({"RANK": "1"}, "--workload", "qwen05b", "--steps", "3", "--warmup", "3") == []
+
+
+def test_workload_spec_per_workload():
+    def spec(wl, steps=504, warmup=8):
+        return bench.workload_spec(SimpleNamespace(workload=wl, layers=0, steps=steps,
+                                                   warmup=warmup))
+    d = spec("llama8b")
+    assert (d.n, d.lens, d.K, d.W, d.unit, d.metric) == (1, [39], 504, 8, "ms/token", bench.METRIC)
+    assert "steps 47..550 timed" in d.workload
+    d = spec("llama8b-32k")
+    assert (d.lens, d.K, d.unit) == ([32768], 248, "ms/token")   # 256 decode steps in all
+    d = spec("llama8b-batch8")
+    assert d.n == 8 and d.K == 248 and d.unit == "ms/step" and "8 requests" in d.metric
+    assert all(32 <= n <= 2048 for n in d.lens)
+    d = spec("qwen05b", steps=10, warmup=3)
+    assert d.model.name.startswith("qwen") and "Qwen2.5-0.5B-shape" in d.metric and d.K == 10
