@@ -227,13 +227,13 @@ def run_reference(args):
     while Ls > 1 and (W + K) * per_step_full * nbytes(model.with_layers(Ls), lens[0]) / \
             nbytes(model, lens[0]) > budget:
         Ls -= 1
-    ms_ = model if Ls == model.n_layers else model.with_layers(Ls)
-    om, sts = states(ms_)
+    m_run = model if Ls == model.n_layers else model.with_layers(Ls)
+    om, sts = states(m_run)
     scaled = []
     for j in range(W + K):
         per_req = step(om, sts, j)
         if j >= W:
-            scaled.append(sum(t * nbytes(model, lens[r] + j) / nbytes(ms_, lens[r] + j)
+            scaled.append(sum(t * nbytes(model, lens[r] + j) / nbytes(m_run, lens[r] + j)
                               for r, t in enumerate(per_req)))
     cores = oracle.num_threads()
     ms = 1e3 * sum(scaled) / len(scaled)
