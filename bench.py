@@ -326,9 +326,7 @@ def run_mk(args):
     model, shape_cap, lens, n, W, K = spec.model, spec.shape_cap, spec.lens, spec.n, spec.W, spec.K
     max_seq = max(lens) + W + K + 1
     w = synth.make_model(model, 0, device="cuda")
-    fp8 = args.weights == "fp8"
-    if fp8:  # the row-quantized model (every GEMV matrix e4m3 codes x row powers of two)
-        w = synth.quantize_fp8_model(model, w)
+    fp8 = args.weights == "fp8"  # the library row-quantizes the bf16 weights at create
     wbytes = 1 if fp8 else 2
     stream = torch.cuda.current_stream()
     dec = binding.Decoder(model, w, max_seq, max_batch=n, stream=stream,
@@ -527,8 +525,6 @@ def run_mk(args):
         dec.close()
         torch.cuda.empty_cache()
         w2 = synth.make_model(model, 0, device="cuda")
-        if fp8:
-            w2 = synth.quantize_fp8_model(model, w2)
         w_cpu = {k: v.cpu() for k, v in w2.items()}
         del w2
         first_pos = lens[0] + W if n > 1 or lens[0] > SHORT_PROMPT else 0

@@ -178,6 +178,17 @@ int mk_decode_step_host(mk_ctx* ctx, const int32_t* tokens_host, const int32_t* 
  * stream); n_req must not exceed that call's. */
 int mk_copy_hidden(mk_ctx* ctx, float* hidden_dev, int n_req);
 
+/* Intermediate results of the last single-request step (not the batched
+ * step), for per-stage parity checks: which = MK_ACT_Q the rotated queries of
+ * the last layer (n_q_heads x head_dim fp32, head-major), MK_ACT_ATTN its
+ * attention output (same layout, normalised), MK_ACT_FFN its SwiGLU
+ * activation silu(W_gate xn) * (W_up xn) (ffn fp32), MK_ACT_X the residual
+ * stream after the last layer (hidden fp32).  Copies n floats from the start
+ * of that vector to dst_dev on the context's stream; n must not exceed its
+ * length.  MK_ERR_INVALID_ARG after a batched step or for a bad `which`. */
+enum { MK_ACT_Q = 0, MK_ACT_ATTN = 1, MK_ACT_FFN = 2, MK_ACT_X = 3 };
+int mk_copy_activation(mk_ctx* ctx, int which, float* dst_dev, int n);
+
 /* Device pointer of the bf16 K (which=0) or V (which=1) cache of one request,
  * layer and KV head: max_seq x head_dim elements, row-major. */
 int mk_kv_pointer(mk_ctx* ctx, int req, int layer, int kv_head, int which, void** out_dev);
@@ -243,11 +254,14 @@ int mk_attention_decode(const float* q_dev, const void* k_dev, const void* v_dev
  * packaging of the op above.  The scratch is a 270,592-byte array compiled
  * into the library, so this entry point never allocates; it serves up to 64
  * splits for 8 query heads per KV head at head_dim 128 (larger requests
- * return MK_ERR_INVALID_ARG, see mk_last_error(NULL)).  The first call on a
- * device looks up the array's device address and clears its merge ticket;
- * make that first call before any stream capture.  All calls on a device
- * share the one array, which keeps the last call's partials: calls that
- * overlap on the GPU (other streams, other threads) race. */
+ * return MK_ERR_INVALID_ARG, see mk_last_error(NULL)).  Every call looks up
+ * the array's device address in the current device's context (no cached
+ * pointer survives a context that is torn down and made again) and clears the
+ * array's merge ticket with a memset on `stream` before the op.  The first
+ * call on a device loads the library's device code there: make it before any
+ * stream capture.  All calls on a device share the one array, which keeps the
+ * last call's partials: calls that overlap on the GPU (other streams, other
+ * threads) race. */
 int mk_attention_decode_noalloc(const float* q_dev, const void* k_dev, const void* v_dev,
                                 int n_keys, int n_q_per_kv, int head_dim, int splits,
                                 float* out_dev, void* stream);

@@ -168,6 +168,54 @@ double orc_kv_cache_bytes(double batch, double layers, double seq, double head_d
   return 2.0 * batch * layers * seq * head_dim * kv_heads * bytes_per_elem;
 }
 
+/* ----------------------------------------------------------- fp8 weights */
+
+/* |v| rounded to the e4m3 grid (4 exponent bits with bias 7, 3 significand
+ * bits, no infinities: the largest finite value is 1.75 * 2^8 = 448):
+ * spacing 2^(e-3) inside the binade [2^e, 2^(e+1)) for e >= -6, spacing 2^-9
+ * below 2^-6 (subnormals); round to nearest, ties to the even multiple;
+ * anything above 448 saturates to 448.  Exact in double for any float input. */
+static double e4m3_round_abs(double a) {
+  if (a == 0.0) return 0.0;
+  int E;
+  frexp(a, &E);                 /* a = f * 2^E, f in [0.5, 1): binade e = E - 1 */
+  int e = E - 1;
+  if (e < -6) e = -6;
+  double step = ldexp(1.0, e - 3);
+  double r = rint(a / step) * step;  /* default rounding mode: nearest, ties to even */
+  return r > 448.0 ? 448.0 : r;
+}
+
+/* fp8 weights ("LLM高速化勉強会資料" slide 33: fewer bits per parameter, with
+ * block-wise scaling; "Crear desde cero ..." §4: FP8).  The block is one row:
+ * k = the smallest integer with max|row| <= 448 * 2^k (k = 0 for a row of
+ * zeros), each weight becomes e4m3(w / 2^k) * 2^k.  Writes those values as
+ * bf16 (exact: 3 significand bits times a power of two) and the row exponents
+ * k. */
+void orc_quantize_fp8_rows(const uint16_t* w, int rows, int cols, uint16_t* out, int* row_exp) {
+#pragma omp parallel for schedule(static)
+  for (int r = 0; r < rows; ++r) {
+    const uint16_t* wr = w + (size_t)r * cols;
+    double mx = 0.0;
+    for (int c = 0; c < cols; ++c) {
+      double a = fabs((double)bf16_to_f32(wr[c]));
+      if (a > mx) mx = a;
+    }
+    int k = 0;
+    if (mx > 0.0) {
+      k = (int)ceil(log2(mx / 448.0));
+      while (mx > ldexp(448.0, k)) ++k;
+      while (mx <= ldexp(448.0, k - 1)) --k;
+    }
+    if (row_exp) row_exp[r] = k;
+    for (int c = 0; c < cols; ++c) {
+      double v = (double)bf16_to_f32(wr[c]);
+      double q = e4m3_round_abs(fabs(ldexp(v, -k)));
+      out[(size_t)r * cols + c] = f32_to_bf16((float)ldexp(v < 0 ? -q : q, k));
+    }
+  }
+}
+
 int orc_num_threads(void) {
 #ifdef _OPENMP
   return omp_get_max_threads();
@@ -307,11 +355,10 @@ static int head_out(const orc_model* m, const float* x, float* xn, float* logits
   return id;
 }
 
-int orc_decode(const orc_model* m, orc_state* s, int token, int pos, float* logits,
-               float* hidden) {
-  if (!m || !s || s->m != m) return -1;
+/* The transformer blocks of one decode step: token at position pos, its K/V
+ * appended to the cache; leaves the final residual stream in x_out[hidden]. */
+static void decode_layers(const orc_model* m, orc_state* s, int token, int pos, float* x_out) {
   const orc_config* c = &m->c;
-  if (token < 0 || token >= c->vocab || pos < 0 || pos >= s->max_seq) return -1;
   const int H = c->hidden, d = c->head_dim, hq = c->n_q_heads, hkv = c->n_kv_heads;
   const int G = hq / hkv, F = c->ffn, n = pos + 1;
   float* x = (float*)malloc(sizeof(float) * (size_t)H);
@@ -358,9 +405,39 @@ int orc_decode(const orc_model* m, orc_state* s, int token, int pos, float* logi
     for (int i = 0; i < H; ++i) x[i] = x[i] + tmp[i];
     ffn_block(m, L, x, xn, g, u, tmp);
   }
-  int id = head_out(m, x, xn, logits, hidden);
+  memcpy(x_out, x, sizeof(float) * (size_t)H);
   free(x); free(xn); free(q); free(k); free(v); free(att); free(tmp); free(g); free(u);
   free(Kb); free(Vb);
+}
+
+int orc_decode(const orc_model* m, orc_state* s, int token, int pos, float* logits,
+               float* hidden) {
+  if (!m || !s || s->m != m) return -1;
+  const orc_config* c = &m->c;
+  if (token < 0 || token >= c->vocab || pos < 0 || pos >= s->max_seq) return -1;
+  float* x = (float*)malloc(sizeof(float) * (size_t)c->hidden);
+  float* xn = (float*)malloc(sizeof(float) * (size_t)c->hidden);
+  decode_layers(m, s, token, pos, x);
+  int id = head_out(m, x, xn, logits, hidden);
+  free(x); free(xn);
+  return id;
+}
+
+/* A prompt as n sequential decode steps at positions 0..n-1 ("Crear desde cero
+ * ..." §1.1: the prefill fills the KV cache); only the last position goes
+ * through the final norm and the LM head, whose output the prompt's earlier
+ * positions do not need. */
+int orc_prefill(const orc_model* m, orc_state* s, const int* tokens, int n, float* logits,
+                float* hidden) {
+  if (!m || !s || s->m != m || !tokens || n < 1 || n > s->max_seq) return -1;
+  const orc_config* c = &m->c;
+  for (int t = 0; t < n; ++t)
+    if (tokens[t] < 0 || tokens[t] >= c->vocab) return -1;
+  float* x = (float*)malloc(sizeof(float) * (size_t)c->hidden);
+  float* xn = (float*)malloc(sizeof(float) * (size_t)c->hidden);
+  for (int t = 0; t < n; ++t) decode_layers(m, s, tokens[t], t, x);
+  int id = head_out(m, x, xn, logits, hidden);
+  free(x); free(xn);
   return id;
 }
 

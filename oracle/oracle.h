@@ -71,6 +71,10 @@ float  orc_silu(float z);
 int    orc_argmax(const float* v, int n);
 double orc_kv_cache_bytes(double batch, double layers, double seq, double head_dim,
                           double kv_heads, double bytes_per_elem);
+/* fp8 (e4m3) weights with one power-of-two scale per row: out[rows*cols] =
+ * e4m3(w / 2^k) * 2^k as bf16, k per row the smallest with max|row| <= 448 * 2^k
+ * (0 for a row of zeros), written to row_exp (may be NULL). */
+void   orc_quantize_fp8_rows(const uint16_t* w, int rows, int cols, uint16_t* out, int* row_exp);
 
 /* ---- model ---- */
 orc_model* orc_create(const orc_config* cfg, const uint16_t* embed, const orc_layer* layers,
@@ -86,6 +90,12 @@ void       orc_state_destroy(orc_state* s);
  * may be NULL.  Returns the greedy next id, or -1 on bad arguments. */
 int orc_decode(const orc_model* m, orc_state* s, int token, int pos, float* logits,
                float* hidden);
+
+/* A prompt of n tokens at positions 0..n-1 into an empty state, as n decode
+ * steps; logits and hidden (either may be NULL) of the last position only.
+ * Returns the greedy next id, or -1 on bad arguments. */
+int orc_prefill(const orc_model* m, orc_state* s, const int* tokens, int n, float* logits,
+                float* hidden);
 
 /* Cached K or V of one layer and kv head, positions [0, n): out[n*head_dim]. */
 int orc_state_kv(const orc_state* s, int layer, int kv_head, int which /*0 K, 1 V*/,

@@ -86,6 +86,9 @@ def _bind(L):
     L.orc_forward_full.argtypes = [C.c_void_p, _i32p, C.c_int, C.c_void_p, C.c_void_p]
     L.orc_forward_full.restype = C.c_int
     L.orc_num_threads.restype = C.c_int
+    L.orc_quantize_fp8_rows.argtypes = [C.c_void_p, C.c_int, C.c_int, C.c_void_p, _i32p]
+    L.orc_prefill.argtypes = [C.c_void_p, C.c_void_p, _i32p, C.c_int, C.c_void_p, C.c_void_p]
+    L.orc_prefill.restype = C.c_int
     return L
 
 
@@ -202,6 +205,33 @@ def num_threads() -> int:
     return int(lib().orc_num_threads())
 
 
+def quantize_fp8_rows(W_bf16):
+    """fp8 row quantization of a bf16 [rows, cols] CPU tensor: returns (the
+    values e4m3(w / 2^k) * 2^k as bf16, the row exponents k as int32 numpy)."""
+    import torch
+    W = W_bf16.detach().to("cpu").contiguous()
+    assert W.dtype == torch.bfloat16 and W.dim() == 2
+    rows, cols = W.shape
+    out = torch.empty_like(W)
+    exps = np.empty(rows, dtype=np.int32)
+    lib().orc_quantize_fp8_rows(W.data_ptr(), rows, cols, out.data_ptr(), exps)
+    return out, exps
+
+
+def quantize_fp8_model(cfg, weights):
+    """The model the fp8 decode path computes: every matrix a decode GEMV
+    streams (q, k, v, o, gate, up, down and the LM head -- the embedding when
+    tied) row-quantized by quantize_fp8_rows; norms, biases and an untied
+    embedding unchanged.  CPU bf16 tensors."""
+    out = {k: v.detach().to("cpu") for k, v in weights.items()}
+    for l in range(cfg.n_layers):
+        for key in ("wq", "wk", "wv", "wo", "w_gate", "w_up", "w_down"):
+            out[f"layers.{l}.{key}"] = quantize_fp8_rows(out[f"layers.{l}.{key}"])[0]
+    head = "embed" if cfg.tied_embeddings else "lm_head"
+    out[head] = quantize_fp8_rows(out[head])[0]
+    return out
+
+
 # ----------------------------------------------------------------- model
 
 class OracleModel:
@@ -258,6 +288,19 @@ class OracleModel:
                                hidden.ctypes.data)
         if nid < 0:
             raise ValueError("orc_decode rejected its arguments")
+        return nid, logits, hidden
+
+    def prefill(self, state: "OracleState", tokens, want_logits: bool = True):
+        """The prompt at positions 0..n-1 into an empty state (n decode steps,
+        the LM head at the last only); returns (next_id, logits or None, hidden)."""
+        tokens = np.ascontiguousarray(np.asarray(tokens, dtype=np.int32))
+        logits = np.empty(self.cfg.vocab, dtype=np.float32) if want_logits else None
+        hidden = np.empty(self.cfg.hidden, dtype=np.float32)
+        nid = self._L.orc_prefill(self.h, state.h, tokens, tokens.size,
+                                  logits.ctypes.data if want_logits else None,
+                                  hidden.ctypes.data)
+        if nid < 0:
+            raise ValueError("orc_prefill rejected its arguments")
         return nid, logits, hidden
 
     def forward_full(self, tokens):

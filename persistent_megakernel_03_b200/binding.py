@@ -20,10 +20,11 @@ ERRORS = {-1: "MK_ERR_INVALID_ARG", -2: "MK_ERR_OOM", -3: "MK_ERR_CUDA", -4: "MK
           -5: "MK_ERR_POS_RANGE", -6: "MK_ERR_NOT_RESIDENT", -7: "MK_ERR_POISONED",
           -8: "MK_ERR_TOKEN_RANGE", -9: "MK_ERR_UNSUPPORTED"}
 MODE_MEGAKERNEL, MODE_PER_OP, MODE_PER_OP_GRAPH = 0, 1, 2
+ACT_Q, ACT_ATTN, ACT_FFN, ACT_X = 0, 1, 2, 3
 TASK_KINDS = ("QKV", "ATTN", "OPROJ", "GATEUP", "DOWN", "LMHEAD")
 
 EXPORTS = ("mk_create", "mk_prefill", "mk_decode_step", "mk_decode_steps", "mk_decode_step_host",
-           "mk_copy_hidden",
+           "mk_copy_hidden", "mk_copy_activation",
            "mk_kv_pointer", "mk_copy_kv", "mk_set_mode", "mk_status", "mk_last_error",
            "mk_destroy", "mk_plan_build", "mk_plan_get_info", "mk_plan_get_tasks",
            "mk_plan_get_queue", "mk_plan_get_event_counts", "mk_plan_destroy",
@@ -101,6 +102,7 @@ def lib(build_if_missing: bool = True):
     L.mk_decode_step_host.argtypes = [vp, ip, ip, i, ip]
     L.mk_decode_steps.argtypes = [vp, vp, i, i, vp, vp]
     L.mk_copy_hidden.argtypes = [vp, vp, i]
+    L.mk_copy_activation.argtypes = [vp, i, vp, i]
     L.mk_kv_pointer.argtypes = [vp, i, i, i, i, C.POINTER(vp)]
     L.mk_copy_kv.argtypes = [vp, i, i, i, i, i, vp]
     L.mk_set_mode.argtypes = [vp, i]
@@ -278,6 +280,12 @@ class Decoder:
 
     def copy_hidden(self, dst_dev, n_req: int = 1):
         _check(lib().mk_copy_hidden(self.h, dst_dev.data_ptr(), int(n_req)), self.h)
+
+    def copy_activation(self, which: int, dst_dev):
+        """The last single-request step's ACT_Q / ACT_ATTN / ACT_FFN / ACT_X vector
+        (see mk_copy_activation) into the fp32 CUDA tensor ``dst_dev``."""
+        _check(lib().mk_copy_activation(self.h, int(which), dst_dev.data_ptr(),
+                                        int(dst_dev.numel())), self.h)
 
     def copy_kv(self, req: int, layer: int, kv_head: int, which: int, n: int, dst_dev):
         _check(lib().mk_copy_kv(self.h, req, layer, kv_head, which, n, dst_dev.data_ptr()),

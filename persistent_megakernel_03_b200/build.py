@@ -28,21 +28,38 @@ def is_fresh() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False, extra=()) -> str:
+    """Compiles every source to an object in parallel (one nvcc per file),
+    then links the shared library; skipped when libmk.so is newer than every
+    source and header."""
     if not force and is_fresh():
         return LIB
+    from concurrent.futures import ThreadPoolExecutor
+    import tempfile
     nvcc = os.environ.get("NVCC", "nvcc")
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc, "-O3", "-std=c++17", *ARCH, "-lineinfo", "-Xcompiler", "-fPIC", "-shared",
-           "-I", os.path.join(ROOT, "include"), "-o", tmp,
-           *[os.path.join(CSRC, f) for f in SOURCES], *extra]
+    common = ["-O3", "-std=c++17", *ARCH, "-lineinfo", "-Xcompiler", "-fPIC",
+              "-I", os.path.join(ROOT, "include"), *extra]
     if verbose:
-        cmd.insert(1, "-Xptxas=-v")
-    r = subprocess.run(cmd, cwd=CSRC, capture_output=True, text=True)
-    if r.returncode != 0:
-        sys.stderr.write(r.stdout + r.stderr)
-        raise RuntimeError("nvcc failed building libmk.so")
-    if verbose:
-        sys.stderr.write(r.stderr)
+        common.insert(0, "-Xptxas=-v")
+    with tempfile.TemporaryDirectory(prefix="mk_build_") as tmpdir:
+        def compile_one(src):
+            obj = os.path.join(tmpdir, os.path.splitext(src)[0] + ".o")
+            r = subprocess.run([nvcc, *common, "-c", os.path.join(CSRC, src), "-o", obj],
+                               cwd=CSRC, capture_output=True, text=True)
+            return src, obj, r
+        with ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
+            results = list(ex.map(compile_one, SOURCES))
+        failed = [r for r in results if r[2].returncode != 0]
+        for src, _, r in results:
+            if r.returncode != 0 or verbose:
+                sys.stderr.write(f"--- {src}\n" + r.stdout + r.stderr)
+        if failed:
+            raise RuntimeError("nvcc failed building libmk.so: " + ", ".join(f[0] for f in failed))
+        tmp = LIB + f".tmp{os.getpid()}"
+        r = subprocess.run([nvcc, *ARCH, "-shared", "-o", tmp, *[o for _, o, _ in results]],
+                           cwd=CSRC, capture_output=True, text=True)
+        if r.returncode != 0:
+            sys.stderr.write(r.stdout + r.stderr)
+            raise RuntimeError("nvcc failed linking libmk.so")
     os.replace(tmp, LIB)
     return LIB
 

@@ -622,6 +622,25 @@ extern "C" int mk_copy_hidden(mk_ctx* ctx, float* hidden_dev, int n_req) {
   return MK_OK;
 }
 
+extern "C" int mk_copy_activation(mk_ctx* ctx, int which, float* dst_dev, int n) {
+  int rc = check_ctx(ctx);
+  if (rc) return rc;
+  if (ctx->last_batched) return fail(ctx, MK_ERR_INVALID_ARG, "the last step was batched");
+  const mk_config& c = ctx->cfg;
+  const float* src = nullptr;
+  int len = 0;
+  switch (which) {
+    case MK_ACT_Q: src = ctx->md.q; len = c.n_q_heads * c.head_dim; break;
+    case MK_ACT_ATTN: src = ctx->md.attn; len = c.n_q_heads * c.head_dim; break;
+    case MK_ACT_FFN: src = ctx->md.act; len = c.ffn; break;
+    case MK_ACT_X: src = ctx->md.x; len = c.hidden; break;
+    default: return fail(ctx, MK_ERR_INVALID_ARG, "bad activation selector");
+  }
+  if (!dst_dev || n < 0 || n > len) return fail(ctx, MK_ERR_INVALID_ARG, "bad copy size");
+  CK(cudaMemcpyAsync(dst_dev, src, (size_t)n * 4, cudaMemcpyDeviceToDevice, ctx->stream));
+  return MK_OK;
+}
+
 extern "C" int mk_kv_pointer(mk_ctx* ctx, int req, int layer, int kv_head, int which, void** out_dev) {
   if (!ctx || !out_dev) return MK_ERR_INVALID_ARG;
   const mk_config& c = ctx->cfg;
@@ -673,7 +692,12 @@ extern "C" int mk_status(mk_ctx* ctx) {
   }
   if (st[0] != 0) {
     ctx->poisoned = true;
-    const char* what = st[0] == MK_ERR_TIMEOUT ? "event wait timed out at task "
+    // a timeout's detail: the task index of an event wait, or (negative) which
+    // shared-memory wait gave up: -1 ring full, -2 ready, -3 done, -4 ring
+    // empty, -5 the producer's final drain of its copies
+    const char* what = st[0] == MK_ERR_TIMEOUT
+                           ? (st[1] >= 0 ? "event wait timed out at task "
+                                         : "shared-memory wait timed out, kind ")
                        : st[0] == MK_ERR_TOKEN_RANGE ? "token id out of range: "
                                                      : "device error, detail ";
     return fail(ctx, st[0], std::string(what) + std::to_string(st[1]));

@@ -14,7 +14,6 @@
 #include <cuda_runtime.h>
 #include <math.h>
 
-#include <mutex>
 #include <string>
 
 #include "../../include/mk.h"
@@ -268,10 +267,6 @@ constexpr size_t kNoAllocBytes =
 // The shared scratch: 270,592 bytes per device.
 static __device__ __align__(256) uint8_t g_attn_noalloc_scratch[kNoAllocBytes];
 
-constexpr int kMaxDevices = 128;
-std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDevices] = {};
-
 }  // namespace
 }  // namespace mk
 
@@ -289,26 +284,20 @@ extern "C" int mk_attention_decode_noalloc(const float* q_dev, const void* k_dev
     return MK_ERR_INVALID_ARG;
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MK_ERR_CUDA;
+  // The array's name in host code is only a stand-in for it: its device
+  // address in the current device's context is looked up on every call
+  // (cheap, allocates nothing), so a context that was torn down and made
+  // again never sees a stale address.  The first call on a device loads this
+  // library's device code there; make it before any stream capture.
   void* scratch = nullptr;
-  {
-    // First call on this device: look up the device address of the array
-    // (the array's name in host code is only a stand-in for it) and clear
-    // the merge ticket.  Later calls reuse the address.
-    std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
-      void* p = nullptr;
-      if (cudaGetSymbolAddress(&p, g_attn_noalloc_scratch) != cudaSuccess || !p) {
-        cudaGetLastError();
-        set_last_error("mk_attention_decode_noalloc: cudaGetSymbolAddress failed");
-        return MK_ERR_CUDA;
-      }
-      if (cudaMemsetAsync(p, 0, kAttnTicketBytes, st) != cudaSuccess) return MK_ERR_CUDA;
-      g_noalloc_ptr[dev] = p;
-    }
-    scratch = g_noalloc_ptr[dev];
+  if (cudaGetSymbolAddress(&scratch, g_attn_noalloc_scratch) != cudaSuccess || !scratch) {
+    cudaGetLastError();
+    set_last_error("mk_attention_decode_noalloc: cudaGetSymbolAddress failed");
+    return MK_ERR_CUDA;
   }
+  // The merge ticket must start at zero; the partials need no clearing (each
+  // split writes its own before the ticket lets the last one read them).
+  if (cudaMemsetAsync(scratch, 0, kAttnTicketBytes, st) != cudaSuccess) return MK_ERR_CUDA;
   cudaError_t e = launch_attn_op(q_dev, k_dev, v_dev, n_keys, n_q_per_kv, head_dim, splits,
                                  scratch, out_dev, st);
   return e == cudaSuccess ? MK_OK : MK_ERR_CUDA;

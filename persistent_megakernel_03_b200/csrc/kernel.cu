@@ -140,7 +140,7 @@ __device__ __forceinline__ void set_error(const ModelDev& m, int code, int info)
 
 // Codes stored in status_info when a shared-memory barrier wait times out
 // (event waits store the task index instead).
-constexpr int kWaitFull = -1, kWaitReady = -2, kWaitDone = -3, kWaitEmpty = -4;
+constexpr int kWaitFull = -1, kWaitReady = -2, kWaitDone = -3, kWaitEmpty = -4, kWaitDrain = -5;
 
 __device__ __forceinline__ bool aborting(Smem& s);
 
@@ -310,12 +310,18 @@ __device__ __forceinline__ void producer(const KernelArgs& a, Smem& s, int q0, i
   // the workers stop early (abort) nobody else waits for them, and a bulk copy
   // must never write into shared memory of a CTA that has exited.  Only the
   // last kRingSlots copies can still be in flight (older slots were reused).
-  // The wait is bounded: the sources are valid device memory.
+  // The drain is bounded and therefore best-effort: the sources are valid
+  // device memory, so a copy lands in microseconds; if one has not after
+  // 200 ms the launch records MK_ERR_TIMEOUT (detail kWaitDrain), which
+  // poisons the context on the host so it is never used again.
   const uint32_t first = seq > kRingSlots ? seq - kRingSlots : 0;
   for (uint32_t q = first; q < seq; ++q) {
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait(&s.full[q % kRingSlots], (q / kRingSlots) & 1u)) {
-      if (globaltimer_ns() - t0 > 200000000ull) break;
+      if (globaltimer_ns() - t0 > 200000000ull) {
+        set_error(m, MK_ERR_TIMEOUT, kWaitDrain);
+        return;
+      }
     }
   }
 }

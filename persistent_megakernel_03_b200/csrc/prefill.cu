@@ -185,7 +185,10 @@ __global__ void __launch_bounds__(128, 1)
   }
   __syncwarp();
   // Accumulator ready (or the issuing stopped): every warp waits on `done`.
-  const bool ok = gemm_wait(&s.done, 0);
+  // The issuing thread commits `done` on every path, at the latest when its
+  // own bounded waits gave up, so one more bounded wait covers that case.
+  bool ok = gemm_wait(&s.done, 0);
+  if (!ok) ok = gemm_wait(&s.done, 0);
   tc_fence_after_sync();
   pdl_wait();  // (returned long ago in the producer) before writing Y
   __syncthreads();
@@ -240,7 +243,11 @@ __global__ void __launch_bounds__(128, 1)
   }
   tc_fence_before_sync();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, S::kTmemCols);
+  // Tensor memory is released only once every MMA of this CTA retired (the
+  // `done` commit arrived); if that never happened the error word is set and
+  // the columns stay allocated rather than be handed to another CTA while
+  // MMAs may still write them.
+  if (warp == 0 && ok) tmem_dealloc(tmem, S::kTmemCols);
 }
 
 // ------------------------------------------------------- small operators

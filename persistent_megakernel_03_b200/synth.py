@@ -172,45 +172,3 @@ def make_packed_prompts(lens, vocab: int, seed: int = 1):
 
 def layer_tensor(w: Dict[str, torch.Tensor], l: int, key: str) -> Optional[torch.Tensor]:
     return w.get(f"layers.{l}.{key}")
-
-
-# ------------------------------------------------------------ fp8 weights
-
-def fp8_row_scale_exponents(x: torch.Tensor) -> torch.Tensor:
-    """Per row k: the smallest 2^k with max|row| / 2^k <= 448 (the largest
-    finite e4m3 value); rows of zeros get k = 0."""
-    mx = x.abs().amax(dim=1)
-    k = torch.zeros_like(mx)
-    nz = mx > 0
-    k[nz] = torch.ceil(torch.log2(mx[nz] / 448.0))
-    for _ in range(4):  # settle log2 rounding either way
-        big = nz & (mx / torch.exp2(k) > 448.0)
-        k[big] += 1
-        small = nz & (mx / torch.exp2(k - 1) <= 448.0)
-        k[small] -= 1
-    return k
-
-
-def quantize_fp8_rows(t: torch.Tensor) -> torch.Tensor:
-    """bf16 [rows][K] -> bf16 values e4m3(w / 2^k) * 2^k with one k per row
-    (round to nearest even).  The result is exactly representable in bf16 and
-    a fixed point of the same quantization."""
-    x = t.float()
-    s = torch.exp2(fp8_row_scale_exponents(x)).unsqueeze(1)
-    codes = (x / s).to(torch.float8_e4m3fn)
-    return (codes.float() * s).to(torch.bfloat16)
-
-
-def quantize_fp8_model(cfg: ModelConfig, w: Dict[str, torch.Tensor]) -> Dict[str, torch.Tensor]:
-    """The model whose decode GEMV matrices (q, k, v, o, gate, up, down and the
-    LM head -- the embedding when tied) are fp8 row-quantized; the weights of
-    the fp8 decode path and of the oracle."""
-    out = dict(w)
-    for l in range(cfg.n_layers):
-        for key in ("wq", "wk", "wv", "wo", "w_gate", "w_up", "w_down"):
-            out[f"layers.{l}.{key}"] = quantize_fp8_rows(w[f"layers.{l}.{key}"])
-    if cfg.tied_embeddings:
-        out["embed"] = quantize_fp8_rows(w["embed"])
-    else:
-        out["lm_head"] = quantize_fp8_rows(w["lm_head"])
-    return out

@@ -34,8 +34,8 @@ def oracle_trace(model, w_cpu, prompt, steps: int, max_seq: int, kv_bf16: bool =
     om = oracle.OracleModel(model, w_cpu, kv_bf16=kv_bf16)
     st = om.new_state(max_seq)
     tr = OracleTrace(prompt=list(prompt), feed=[])
-    for p, t in enumerate(prompt):
-        nid, lg, hid = om.decode(st, int(t), p, want_logits=(p == len(prompt) - 1))
+    # the prompt as sequential decode steps (the LM head at the last only)
+    nid, lg, hid = om.prefill(st, list(prompt))
     tr.logits.append(lg)
     tr.hidden.append(hid)
     tr.ids.append(nid)

@@ -131,3 +131,51 @@ def test_planted_mistake_is_caught(name, hf_refs, variant_dir):
     assert old in src, f"mutation anchor for {name} not found"
     so = oracle.compile_variant(src.replace(old, new), variant_dir, f"mut_{name}")
     assert not _pins_pass(oracle.load_variant(so), hf_refs), f"pins missed {name}"
+
+
+# Mistakes in the fp8 weight rule (orc_quantize_fp8_rows).
+FP8_MUTATIONS = {
+    "fp8_truncates": ("double r = rint(a / step) * step;", "double r = floor(a / step) * step;"),
+    "fp8_no_subnormal_floor": ("if (e < -6) e = -6;", "if (e < -60) e = -60;"),
+    "fp8_scale_one_too_small": ("while (mx <= ldexp(448.0, k - 1)) --k;",
+                                "while (mx <= ldexp(448.0, k)) --k;"),
+    "fp8_sign_dropped": ("ldexp(v < 0 ? -q : q, k)", "ldexp(q, k)"),
+    "fp8_four_significand_bits": ("double step = ldexp(1.0, e - 3);",
+                                  "double step = ldexp(1.0, e - 4);"),
+}
+
+
+def _fp8_pins_pass(L) -> bool:
+    def q(rows):
+        w = torch.tensor(rows, dtype=torch.bfloat16)
+        out = torch.empty_like(w)
+        k = np.empty(w.shape[0], dtype=np.int32)
+        L.orc_quantize_fp8_rows(w.data_ptr(), w.shape[0], w.shape[1], out.data_ptr(), k)
+        return out, k
+    out, k = q([[448, 1, 0.1, -17, 19, 3 * 2**-9, 2**-10, -1.5 * 2**-9]])
+    if out.float()[0].tolist() != [448, 1, 0.1015625, -16, 20, 3 * 2**-9, 0, -2**-8]:
+        return False
+    g = torch.Generator("cpu").manual_seed(0)
+    w = (torch.randn(16, 64, generator=g) * 0.02).to(torch.bfloat16)
+    out = torch.empty_like(w)
+    k = np.empty(16, dtype=np.int32)
+    L.orc_quantize_fp8_rows(w.data_ptr(), 16, 64, out.data_ptr(), k)
+    s = torch.exp2(torch.from_numpy(k).double()).unsqueeze(1)
+    want = ((w.double() / s).float().to(torch.float8_e4m3fn).double() * s).to(torch.bfloat16)
+    mx = w.double().abs().amax(dim=1)
+    return bool(torch.equal(out, want) and torch.all(mx <= 448 * s[:, 0]) and
+                torch.all(mx > 224 * s[:, 0]))
+
+
+def test_fp8_control_passes(variant_dir):
+    so = oracle.compile_variant(oracle.source_text(), variant_dir, "control_fp8")
+    assert _fp8_pins_pass(oracle.load_variant(so))
+
+
+@pytest.mark.parametrize("name", sorted(FP8_MUTATIONS))
+def test_planted_fp8_mistake_is_caught(name, variant_dir):
+    src = oracle.source_text()
+    old, new = FP8_MUTATIONS[name]
+    assert old in src, f"mutation anchor for {name} not found"
+    so = oracle.compile_variant(src.replace(old, new), variant_dir, f"mut_{name}")
+    assert not _fp8_pins_pass(oracle.load_variant(so)), f"pins missed {name}"

@@ -261,6 +261,28 @@ def test_cached_decode_equals_full_recompute_wide(cfg):
         np.testing.assert_allclose(hid, hf[p], rtol=1e-5, atol=1e-5)
 
 
+def test_prefill_equals_full_recompute_and_sequential_steps(tiny):
+    # the prompt-only entry point: the last position's logits and hidden as
+    # the uncached forward gives them, and a cache identical to the one of
+    # the same positions run as decode steps
+    cfg, w = tiny
+    m = oracle.OracleModel(cfg, w)
+    toks = synth.make_prompt(20, cfg.vocab, seed=3).numpy()
+    a = m.new_state(24)
+    nid, lg, hid = m.prefill(a, toks)
+    lf, hf = m.forward_full(toks)
+    assert np.array_equal(lg, lf[-1]) and np.array_equal(hid, hf[-1])
+    assert nid == int(np.argmax(lf[-1]))
+    b = m.new_state(24)
+    for p, t in enumerate(toks):
+        m.decode(b, int(t), p)
+    for l in range(cfg.n_layers):
+        for which in (0, 1):
+            assert np.array_equal(a.kv(l, 1, which, 20), b.kv(l, 1, which, 20))
+    with pytest.raises(ValueError):
+        m.prefill(m.new_state(8), toks)          # longer than the state
+
+
 def test_cache_holds_rotated_bf16_keys(tiny):
     cfg, w = tiny
     m = oracle.OracleModel(cfg, w)
