@@ -137,32 +137,6 @@ def per_token_ms(total_ms_max: float, steps: int, world: int) -> float:
     return total_ms_max / (steps * world)
 
 
-def oracle_sample(model, w_cpu, n_steps: int, budget_s: float, first_pos: int = 0):
-    """Times the oracle's decode step (positions first_pos..) on host cores."""
-    import numpy as np
-
-    import oracle
-    om = oracle.OracleModel(model, w_cpu)
-    st = om.new_state(first_pos + n_steps + 1)
-    if first_pos:
-        rng = np.random.default_rng(0)
-        fill = rng.standard_normal((first_pos, model.head_dim), dtype=np.float32)
-        for l in range(model.n_layers):
-            for g in range(model.n_kv_heads):
-                for which in (0, 1):
-                    st.set_kv(l, g, which, fill)
-    tok = 1
-    times = []
-    t_all = time.perf_counter()
-    for p in range(first_pos, first_pos + n_steps):
-        t0 = time.perf_counter()
-        tok, _, _ = om.decode(st, tok, p, want_logits=False)
-        times.append(time.perf_counter() - t0)
-        if time.perf_counter() - t_all > budget_s and len(times) >= 2:
-            break
-    return times, oracle.num_threads()
-
-
 def run_reference(args):
     """The oracle as it stands, timed on the host's cores on the megakernel
     arm's workload (same metric, unit and config): W untimed and K timed
@@ -310,28 +284,70 @@ def workload_spec(args):
                     "after each prompt timed; one batched step per token (tcgen05 GEMMs over "
                     "the requests' columns, each weight matrix streamed once; CUDA graph)")
         unit, metric = "ms/step", f"decode ms/step ({n} requests, Llama-3-8B-shape)"
-    return SimpleNamespace(model=model, shape=shape, shape_cap=shape_cap, lens=lens, n=n,
-                           W=W, K=K, workload=workload, unit=unit, metric=metric)
+    return SimpleNamespace(name=args.workload, model=model, shape=shape, shape_cap=shape_cap,
+                           lens=lens, n=n, W=W, K=K, workload=workload, unit=unit,
+                           metric=metric)
 
 
-def run_mk(args):
+# The other workloads the default run measures next to the headline one, each
+# as a sub-record of the same JSON line: (workload, weights).
+SUB_WORKLOADS = (("qwen05b", "bf16"), ("llama8b-batch8", "bf16"), ("llama8b-32k", "bf16"),
+                 ("llama8b", "fp8"))
+
+
+def oracle_steps(model, w_cpu, lens, first_step: int, n_steps: int, budget_s: float):
+    """The oracle's decode step timed on host cores at the positions the GPU
+    arm times (lens[r] + first_step + j for request r), one decode per request
+    per step; the cache rows before hold random values (the timing does not
+    depend on them).  Stops early once budget_s of steps ran (at least 2).
+    Returns per-step seconds (summed over requests) and the thread count."""
+    import numpy as np
+
+    import oracle
+    om = oracle.OracleModel(model, w_cpu)
+    rng = np.random.default_rng(0)
+    states = []
+    for n0 in lens:
+        p0 = n0 + first_step
+        st = om.new_state(p0 + n_steps + 1)
+        fill = rng.standard_normal((p0, model.head_dim), dtype=np.float32)
+        for l in range(model.n_layers):
+            for g in range(model.n_kv_heads):
+                for which in (0, 1):
+                    st.set_kv(l, g, which, fill)
+        states.append((st, p0))
+    times = []
+    t_all = time.perf_counter()
+    for j in range(n_steps):
+        t0 = time.perf_counter()
+        for st, p0 in states:
+            om.decode(st, 1, p0 + j, want_logits=False)
+        times.append(time.perf_counter() - t0)
+        if time.perf_counter() - t_all > budget_s and len(times) >= 2:
+            break
+    return times, oracle.num_threads()
+
+
+def measure(spec, w, fp8: bool, world: int, local: int, *, full: bool, w_cpu=None,
+            cpu_budget_s: float = 25.0, trace_path=None, l2_prefetch: int = 0,
+            layers_flag: int = 0) -> dict:
+    """One workload on one decoder: W untimed and K device-timed decode steps
+    (CUDA events on the launching stream, barrier + synchronize around them,
+    max over ranks), the same steps end to end through the host entry point,
+    the per-operator CUDA-graph baseline, clocks during the timed region and,
+    with w_cpu, the oracle on host cores at the same positions.  full adds the
+    per-operator baseline, the device-resident loop, the read probe and the
+    optional per-task trace."""
     import numpy as np
     import torch
 
     from persistent_megakernel_03_b200 import binding, roofline, synth
-
-    rank, world, local = dist_setup(args.gpus)
-    torch.cuda.set_device(local)
-    spec = workload_spec(args)
-    model, shape_cap, lens, n, W, K = spec.model, spec.shape_cap, spec.lens, spec.n, spec.W, spec.K
+    model, lens, n, W, K = spec.model, spec.lens, spec.n, spec.W, spec.K
     max_seq = max(lens) + W + K + 1
-    w = synth.make_model(model, 0, device="cuda")
-    fp8 = args.weights == "fp8"  # the library row-quantizes the bf16 weights at create
     wbytes = 1 if fp8 else 2
     stream = torch.cuda.current_stream()
     dec = binding.Decoder(model, w, max_seq, max_batch=n, stream=stream,
-                          l2_prefetch=args.l2_prefetch, weight_format=1 if fp8 else 0)
-    del w  # mk_create copied and packed the weights
+                          l2_prefetch=l2_prefetch, weight_format=1 if fp8 else 0)
     torch.cuda.empty_cache()
     if n == 1:
         prompt, offs = synth.make_prompt(lens[0], model.vocab), [0, lens[0]]
@@ -340,9 +356,7 @@ def run_mk(args):
         offs = offs.tolist()
     prompt = prompt.to(torch.int32).cuda()
     ids = [torch.zeros(n, dtype=torch.int32, device="cuda") for _ in range(2)]
-
-    first_id = []
-    prefill_ms = []
+    first_id, prefill_ms = [], []
 
     def prefill():
         # Decode steps write the cache only at positions past each prompt, so
@@ -369,7 +383,12 @@ def run_mk(args):
             if evs is not None:
                 evs[k + 1].record(stream)
 
-    # ---- device-timed region (megakernel)
+    def check():
+        rc = dec.status()
+        if rc != 0:
+            raise RuntimeError(f"device status {rc}: {dec.last_error()}")
+
+    # ---- device-timed region (megakernel, or the batched step for n > 1)
     prefill()
     run_steps(0, W)
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
@@ -381,21 +400,41 @@ def run_mk(args):
         run_steps(W, K, evs)
         torch.cuda.synchronize()
     barrier(world)
-    rc = dec.status()
-    if rc != 0:
-        raise RuntimeError(f"device status {rc}: {dec.last_error()}")
+    check()
     per_step = [evs[k].elapsed_time(evs[k + 1]) for k in range(K)]
-    total_ms = evs[0].elapsed_time(evs[K])
-    total_ms = max_over_ranks(total_ms, world)
+    total_ms = max_over_ranks(evs[0].elapsed_time(evs[K]), world)
     value = per_token_ms(total_ms, K, world)
-    bytes_mean = sum(roofline.step_bytes(model, positions(W + k), wbytes=wbytes) for k in range(K)) / K
-    avg_launch_s = (sum(per_step) / K) * 1e-3
-    achieved = bytes_mean / avg_launch_s / 1e9
+    bytes_mean = sum(roofline.step_bytes(model, positions(W + k), wbytes=wbytes)
+                     for k in range(K)) / K
+    achieved = bytes_mean / ((sum(per_step) / K) * 1e-3) / 1e9
     peak, peak_src = measured_peaks()
+    rec = {
+        "workload": spec.workload, "metric": spec.metric, "unit": spec.unit, "value": value,
+        "steps": K, "warmup": W, "ms_per_step": total_ms / K,
+        "weights": "fp8 e4m3, one power-of-two scale per row" if fp8 else "bf16",
+        "tok_per_s": 1e3 * n / value,
+        "step_ms": {"median": statistics.median(per_step),
+                    "p10": float(np.percentile(per_step, 10)),
+                    "p90": float(np.percentile(per_step, 90))},
+        "achieved_gbs": achieved, "frac_of_8tbs": achieved / NOMINAL_HBM,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": peak_src,
+                     "traffic": (load_traffic(spec.name)
+                                 if n == 1 and not fp8 and not layers_flag else None),
+                     "bytes_per_launch": bytes_mean},
+        "clocks": clk.summary(),
+        "prefill": {"ms": prefill_ms[0], "positions": int(sum(lens)),
+                    "path": "tensor-core GEMMs for all but each prompt's last position"},
+        # one persistent launch per step; the batched step's graph holds an
+        # embedding kernel, 7 kernels per layer and 3 for the LM head and argmax
+        "gpu_launches": K if n == 1 else K * (7 * model.n_layers + 4),
+    }
+    if n > 1:
+        rec["roofline"]["bytes_note"] = ("algorithmic bytes: weights once per step plus every "
+                                         "request's KV")
 
     # ---- the device-resident loop: the same K steps in one persistent launch
-    loop = None
-    if n == 1 and world == 1:
+    if full and n == 1 and world == 1:
         prefill()
         run_steps(0, W)
         seq = torch.empty(K, dtype=torch.int32, device="cuda")
@@ -405,30 +444,33 @@ def run_mk(args):
         dec.decode_steps(ids[W % 2], lens[0] + W, K, seq)
         le[1].record(stream)
         torch.cuda.synchronize()
-        rc = dec.status()
-        if rc != 0:
-            raise RuntimeError(f"device status {rc}: {dec.last_error()}")
-        loop = {"ms_per_token": le[0].elapsed_time(le[1]) / K, "steps_per_launch": K}
+        check()
+        rec["device_loop"] = {"ms_per_token": le[0].elapsed_time(le[1]) / K,
+                              "steps_per_launch": K}
 
     # ---- read-stream probe: practical read ceiling on this GPU
-    probe_buf = torch.empty(4 * 2**30, dtype=torch.uint8, device="cuda")
-    sink = torch.zeros(1, dtype=torch.int64, device="cuda")
-    for _ in range(3):
-        binding.read_probe(probe_buf, sink)
-    pe = [torch.cuda.Event(enable_timing=True) for _ in range(11)]
-    pe[0].record(stream)
-    for i in range(10):
-        binding.read_probe(probe_buf, sink)
-        pe[i + 1].record(stream)
-    torch.cuda.synchronize()
-    probe_gbs = max(probe_buf.numel() / (pe[i].elapsed_time(pe[i + 1]) * 1e-3) / 1e9
-                    for i in range(10))
-    del probe_buf
+    if full:
+        probe_buf = torch.empty(4 * 2**30, dtype=torch.uint8, device="cuda")
+        sink = torch.zeros(1, dtype=torch.int64, device="cuda")
+        for _ in range(3):
+            binding.read_probe(probe_buf, sink)
+        pe = [torch.cuda.Event(enable_timing=True) for _ in range(11)]
+        pe[0].record(stream)
+        for i in range(10):
+            binding.read_probe(probe_buf, sink)
+            pe[i + 1].record(stream)
+        torch.cuda.synchronize()
+        probe_gbs = max(probe_buf.numel() / (pe[i].elapsed_time(pe[i + 1]) * 1e-3) / 1e9
+                        for i in range(10))
+        del probe_buf
+        rec["read_probe_gbs"] = probe_gbs
+        rec["frac_of_read_probe"] = achieved / probe_gbs
 
-    # ---- baselines: the same task bodies, one launch per operator
+    # ---- baselines: the same task bodies, one launch per operator (requests in turn)
     baselines = {}
-    nb = min(K, 64)
-    for name, mode in (("per_op", binding.MODE_PER_OP), ("per_op_graph", binding.MODE_PER_OP_GRAPH)):
+    nb = min(K, 64 if full else 16)
+    modes = (("per_op", binding.MODE_PER_OP), ("per_op_graph", binding.MODE_PER_OP_GRAPH))
+    for name, mode in (modes if full else modes[1:]):
         dec.set_mode(mode)
         prefill()
         run_steps(0, min(W, 4))
@@ -439,11 +481,10 @@ def run_mk(args):
         torch.cuda.synchronize()
         steps_ms = [bev[k].elapsed_time(bev[k + 1]) for k in range(nb)]
         baselines[name] = {"ms_per_token": statistics.median(steps_ms) / n, "steps": nb,
-                           "launches_per_step": n * dec_stage_count(dec)}
+                           "launches_per_step": n * (5 * model.n_layers + 1)}
     dec.set_mode(binding.MODE_MEGAKERNEL)
-    rc = dec.status()
-    if rc != 0:
-        raise RuntimeError(f"device status {rc}: {dec.last_error()}")
+    check()
+    rec["baselines"] = baselines
 
     # ---- end to end through the host entry point (tokens in, ids out, per step)
     prefill()
@@ -461,9 +502,11 @@ def run_mk(args):
     t1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(t0.elapsed_time(t1), world) / (K * world)
+    rec["e2e"] = {"value": e2e_ms, "unit": spec.unit,
+                  "h2d_bytes_per_step": 4 * n, "d2h_bytes_per_step": 4 * n,
+                  "api": "mk_decode_step_host (pinned host buffers, one sync per step)"}
 
-    trace_summary = None
-    if args.trace and n == 1:
+    if trace_path and n == 1:
         # a few more steps with the per-task timeline on (not part of the timing)
         from persistent_megakernel_03_b200 import trace as mktrace
         plan = binding.Plan(model, max_seq, dec_num_ctas())
@@ -475,80 +518,92 @@ def run_mk(args):
         torch.cuda.synchronize()
         dec.set_trace(None)
         rows = tbuf.cpu().numpy().astype("uint64").tolist()
-        trace_summary = mktrace.summarize(rows, plan.tasks())
-        with open(args.trace, "w") as f:
-            json.dump(trace_summary, f, indent=1)
+        summary = mktrace.summarize(rows, plan.tasks())
+        with open(trace_path, "w") as f:
+            json.dump(summary, f, indent=1)
+        rec["trace"] = {k: summary[k] for k in ("step_us", "mean_cta_busy_frac")}
+    dec.close()
+    del dec
+    torch.cuda.empty_cache()
 
-    clocks = clk.summary()
-    workload, unit, metric = spec.workload, spec.unit, spec.metric
+    # ---- the oracle on the host's cores at the same positions
+    if w_cpu is not None:
+        times, cores = oracle_steps(model, w_cpu, lens, W, 3, cpu_budget_s)
+        timed = times[1:] if len(times) > 1 else times
+        cms = 1e3 * sum(timed) / len(timed)
+        j0 = W + len(times) - len(timed)
+        pos_txt = (f"{lens[0] + j0}..{lens[0] + W + len(times) - 1}" if n == 1 else
+                   f"prompt length + {j0}..{W + len(times) - 1} for each of the {n} requests")
+        rec["cpu_baseline"] = {
+            "value": cms, "unit": spec.unit, "cores": cores, "kind": "oracle",
+            "sample": f"{len(timed)} oracle decode steps of the same {spec.shape_cap} model "
+                      f"at positions {pos_txt} (the GPU arm's first timed positions; cache "
+                      "rows before them hold random values, the timing does not depend on "
+                      "them), fp32 with bf16 weights widened on the fly"
+                      + (" (for the fp8 workload the bf16 weights before quantization: the "
+                         "oracle's time does not depend on the values)" if fp8 else "")
+                      + (f"; one decode per request, {n} requests per step" if n > 1 else "")}
+    return rec
+
+
+def run_mk(args):
+    import torch
+
+    from persistent_megakernel_03_b200 import roofline, synth
+
+    rank, world, local = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    spec = workload_spec(args)
+    model = spec.model
+    fp8 = args.weights == "fp8"
+    w = synth.make_model(model, 0, device="cuda")
+    cpu = world == 1 and rank == 0 and not args.no_cpu_baseline
+    w_cpu = {k: v.cpu() for k, v in w.items()} if cpu else None
+    rec = measure(spec, w, fp8, world, local, full=True, w_cpu=w_cpu, trace_path=args.trace,
+                  l2_prefetch=args.l2_prefetch, layers_flag=args.layers)
     line = {
-        "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": K,
-        "warmup": W, "ms_per_step": total_ms / K, "higher_is_better": False,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-        "weights": "fp8 e4m3, one power-of-two scale per row" if fp8 else "bf16",
-        "data": "synthetic",
-        "config": {"workload": workload,
-                   "l2": (f"inputs larger than L2 ({roofline.weight_bytes(model, wbytes) / 1e9:.2f} GB of "
-                          "weights streamed per step)"),
+        "metric": spec.metric, "value": rec["value"], "unit": spec.unit, "n_gpus": world,
+        "steps": spec.K, "warmup": spec.W, "ms_per_step": rec["ms_per_step"],
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "weights": rec["weights"], "data": "synthetic",
+        "config": {"workload": spec.workload,
+                   "l2": (f"inputs larger than L2 ({roofline.weight_bytes(model, 1 if fp8 else 2) / 1e9:.2f} "
+                          "GB of weights streamed per step)"),
                    "parallelism": f"replicas x{world}"},
-        "tok_per_s": 1e3 * n / value,
-        "step_ms": {"median": statistics.median(per_step),
-                    "p10": float(np.percentile(per_step, 10)),
-                    "p90": float(np.percentile(per_step, 90))},
-        "achieved_gbs": achieved, "frac_of_8tbs": achieved / NOMINAL_HBM,
-        "read_probe_gbs": probe_gbs, "frac_of_read_probe": achieved / probe_gbs,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "peak_source": peak_src,
-                     "traffic": (load_traffic(args.workload)
-                                 if n == 1 and not fp8 and not args.layers else None),
-                     "bytes_per_launch": bytes_mean},
-        "baselines": baselines,
-        "device_loop": loop,
-        "prefill": {"ms": prefill_ms[0], "positions": int(sum(lens)),
-                    "path": "tensor-core GEMMs for all but each prompt's last position"},
-        "clocks": clocks,
-        "e2e": {"value": e2e_ms, "unit": unit, "h2d_bytes_per_step": 4 * n,
-                "d2h_bytes_per_step": 4 * n},
-        "gpu_launches": K * n,
     }
-    if n > 1:
-        line["roofline"]["bytes_note"] = ("algorithmic bytes: weights once per step plus every "
-                                          "request's KV (the baselines run the requests in turn "
-                                          "through the per-operator launches)")
+    for k, v in rec.items():
+        if k not in ("workload", "metric", "unit", "value", "steps", "warmup", "ms_per_step",
+                     "weights"):
+            line[k] = v
     if args.layers:
         line["config"]["workload"] += f" [profiling case: {args.layers} layers]"
     if args.l2_prefetch:
         line["config"]["l2_prefetch_chunks"] = args.l2_prefetch
-    if trace_summary:
-        line["trace"] = {k: trace_summary[k] for k in ("step_us", "mean_cta_busy_frac")}
-    if world == 1 and rank == 0 and not args.no_cpu_baseline:
-        dec.close()
-        torch.cuda.empty_cache()
-        w2 = synth.make_model(model, 0, device="cuda")
-        w_cpu = {k: v.cpu() for k, v in w2.items()}
-        del w2
-        first_pos = lens[0] + W if n > 1 or lens[0] > SHORT_PROMPT else 0
-        times, cores = oracle_sample(model, w_cpu, 4 if first_pos == 0 else 3, 25.0, first_pos)
-        timed = times[1:] if len(times) > 1 else times
-        cms = 1e3 * sum(timed) / len(timed) * n
-        p0 = first_pos + len(times) - len(timed)
-        line["cpu_baseline"] = {
-            "value": cms, "unit": unit, "cores": cores, "kind": "oracle",
-            "sample": f"{len(timed)} oracle decode steps of the same {shape_cap} model "
-                      f"at positions {p0}..{first_pos + len(times) - 1}, fp32 with "
-                      f"bf16 weights widened on the fly"
-                      + (" (cache of the earlier positions filled with random bf16 values: "
-                         "the timing does not depend on them)" if first_pos else "")
-                      + (f"; x{n}: one such step per request" if n > 1 else "")}
+    # ---- the other workloads, each a sub-record (1 GPU only; not with --layers)
+    if (world == 1 and not args.no_workloads and not args.layers and args.workload == "llama8b"
+            and not fp8):
+        subs = {}
+        k_sub = max(16, min(args.steps, 64))
+        for wl, wts in SUB_WORKLOADS:
+            sargs = argparse.Namespace(workload=wl, layers=0, steps=k_sub, warmup=args.warmup)
+            sspec = workload_spec(sargs)
+            if sspec.model is model:
+                sw, sw_cpu = w, w_cpu
+            else:
+                sw = synth.make_model(sspec.model, 0, device="cuda")
+                sw_cpu = {k: v.cpu() for k, v in sw.items()} if cpu else None
+            key = wl + ("-fp8" if wts == "fp8" else "")
+            subs[key] = measure(sspec, sw, wts == "fp8", world, local, full=False,
+                                w_cpu=sw_cpu, cpu_budget_s=12.0)
+            if sw is not w:
+                del sw, sw_cpu
+            torch.cuda.empty_cache()
+        line["workloads"] = subs
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
-
-
-def dec_stage_count(dec) -> int:
-    return 5 * dec.model.n_layers + 1
 
 
 def dec_num_ctas() -> int:
@@ -563,6 +618,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--impl", default="mk", choices=["mk", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="only the selected workload (no sub-records of the other ones)")
     ap.add_argument("--trace", default=None, help="write a per-task timeline summary here")
     ap.add_argument("--l2-prefetch", type=int, default=0,
                     help="ring chunks prefetched into L2 beyond the ring (0: library default)")

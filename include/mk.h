@@ -54,6 +54,15 @@ extern "C" {
 #define MK_ERR_POISONED -7     /* an earlier device error; destroy the context */
 #define MK_ERR_TOKEN_RANGE -8  /* a token id outside [0, vocab) reached the device */
 #define MK_ERR_UNSUPPORTED -9  /* valid request this build does not implement */
+#define MK_ERR_BOUNDS -10      /* debug-bounds build only: a task's access fell outside its
+                                  buffer and was skipped (mk_last_error names the check) */
+
+/* Build properties: bit 0 set in the debug-bounds build (libmk_debug.so, compiled
+ * with MK_DEBUG_BOUNDS), where every task checks the indices of its global and
+ * shared-memory accesses and reports a violation as MK_ERR_BOUNDS through
+ * mk_status instead of performing the access. */
+#define MK_BUILD_DEBUG_BOUNDS 1
+int mk_build_flags(void);
 
 /* Execution modes of a decode step. */
 #define MK_MODE_MEGAKERNEL 0   /* one persistent launch per step (the product) */
@@ -112,6 +121,14 @@ typedef struct {
   int prefill_steps; /* 1: mk_prefill runs every prompt position as a decode step;
                         0: default, the tensor-core prefill (when every contraction
                         length is a multiple of 64) */
+  int kv_page_tokens; /* 0: default, a contiguous KV cache (max_seq positions per
+                         request slot); > 0, a multiple of 64: the KV cache is a pool
+                         of pages of this many positions ("LLM高速化勉強会資料" slides
+                         15-17, PagedAttention), assigned to a request slot through a
+                         block table as its positions are reached and returned to the
+                         pool by mk_kv_release */
+  int kv_pool_pages; /* paged cache: pages in the pool (0: enough for every slot at
+                        max_seq, i.e. max_batch * ceil(max_seq / kv_page_tokens)) */
 } mk_options;
 
 typedef struct mk_ctx mk_ctx;
@@ -153,6 +170,37 @@ int mk_prefill(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t* offsets_ho
 int mk_decode_step(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t* pos_host, int n_req,
                    float* logits_dev, int32_t* next_ids_dev);
 
+/* Continuous batching ("LLM高速化勉強会資料" slides 14-17: requests join and
+ * leave a running batch between steps).  The same as mk_prefill and
+ * mk_decode_step, with request r on KV-cache slot slots_host[r] (distinct
+ * values in [0, max_batch)) instead of slot r: a new request is prefilled into
+ * a free slot while the other slots keep their caches, and each step decodes
+ * any set of occupied slots together (one batched step for 2-8 of them).
+ * Logits, ids and mk_copy_hidden rows stay in request order r.  With a paged
+ * cache, every page the call's positions need is assigned before the launch
+ * (MK_ERR_OOM when the pool has no free page); mk_kv_release returns a
+ * finished request's pages. */
+int mk_prefill_slots(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t* offsets_host,
+                     const int32_t* slots_host, int n_req, float* last_logits_dev,
+                     int32_t* next_ids_dev);
+int mk_decode_step_slots(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t* pos_host,
+                         const int32_t* slots_host, int n_req, float* logits_dev,
+                         int32_t* next_ids_dev);
+
+/* Paged KV cache (mk_options.kv_page_tokens > 0).  Logical page i of a slot
+ * holds positions [i * page, (i + 1) * page).  mk_kv_release returns every page
+ * of `slot` to the pool (a finished request; a no-op for a contiguous cache).
+ * mk_kv_set_pages makes pages_host[0..n_pages) (free pool pages, in any order)
+ * the slot's logical pages 0..n_pages-1, after releasing its current ones; pages
+ * beyond are assigned on demand as usual.  mk_kv_get_pages copies the slot's
+ * table row (-1: no page) and returns its length (max_seq / page rounded up).
+ * mk_kv_free_pages returns the number of free pages.  Table changes are
+ * enqueued on the context's stream. */
+int mk_kv_release(mk_ctx* ctx, int slot);
+int mk_kv_set_pages(mk_ctx* ctx, int slot, const int32_t* pages_host, int n_pages);
+int mk_kv_get_pages(mk_ctx* ctx, int slot, int32_t* pages_out, int cap);
+int mk_kv_free_pages(mk_ctx* ctx);
+
 /* n_steps greedy decode steps of request 0 in ONE persistent launch (the
  * device-resident loop): step s runs at position pos0 + s, feeds the id step
  * s - 1 produced (step 0 feeds token_dev[0]), appends its K/V and writes its
@@ -190,11 +238,13 @@ enum { MK_ACT_Q = 0, MK_ACT_ATTN = 1, MK_ACT_FFN = 2, MK_ACT_X = 3 };
 int mk_copy_activation(mk_ctx* ctx, int which, float* dst_dev, int n);
 
 /* Device pointer of the bf16 K (which=0) or V (which=1) cache of one request,
- * layer and KV head: max_seq x head_dim elements, row-major. */
+ * layer and KV head: max_seq x head_dim elements, row-major.  Contiguous cache
+ * only (MK_ERR_UNSUPPORTED when paged: use mk_copy_kv). */
 int mk_kv_pointer(mk_ctx* ctx, int req, int layer, int kv_head, int which, void** out_dev);
 
 /* Copies positions [0, n) of one K (which=0) or V (which=1) cache head, bf16
- * n x head_dim, to dst_dev (enqueued on the context's stream). */
+ * n x head_dim, to dst_dev (enqueued on the context's stream; gathered page by
+ * page when the cache is paged). */
 int mk_copy_kv(mk_ctx* ctx, int req, int layer, int kv_head, int which, int n, void* dst_dev);
 
 /* Per-task timeline of later megakernel steps (diagnostics).  trace_dev
@@ -209,7 +259,8 @@ int mk_set_trace(mk_ctx* ctx, unsigned long long* trace_dev);
 int mk_set_mode(mk_ctx* ctx, int mode);
 
 /* Synchronises the stream and reports the device status: 0, MK_ERR_TIMEOUT,
- * MK_ERR_TOKEN_RANGE or MK_ERR_CUDA.  Poisons the context on error. */
+ * MK_ERR_TOKEN_RANGE, MK_ERR_BOUNDS (debug-bounds build) or MK_ERR_CUDA.
+ * Poisons the context on error. */
 int mk_status(mk_ctx* ctx);
 
 const char* mk_last_error(const mk_ctx* ctx);

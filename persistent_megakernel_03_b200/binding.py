@@ -18,13 +18,15 @@ LIB_PATH = os.environ.get("MK_LIBRARY") or os.path.join(HERE, "libmk.so")
 MK_OK = 0
 ERRORS = {-1: "MK_ERR_INVALID_ARG", -2: "MK_ERR_OOM", -3: "MK_ERR_CUDA", -4: "MK_ERR_TIMEOUT",
           -5: "MK_ERR_POS_RANGE", -6: "MK_ERR_NOT_RESIDENT", -7: "MK_ERR_POISONED",
-          -8: "MK_ERR_TOKEN_RANGE", -9: "MK_ERR_UNSUPPORTED"}
+          -8: "MK_ERR_TOKEN_RANGE", -9: "MK_ERR_UNSUPPORTED", -10: "MK_ERR_BOUNDS"}
 MODE_MEGAKERNEL, MODE_PER_OP, MODE_PER_OP_GRAPH = 0, 1, 2
 ACT_Q, ACT_ATTN, ACT_FFN, ACT_X = 0, 1, 2, 3
 TASK_KINDS = ("QKV", "ATTN", "OPROJ", "GATEUP", "DOWN", "LMHEAD")
 
 EXPORTS = ("mk_create", "mk_prefill", "mk_decode_step", "mk_decode_steps", "mk_decode_step_host",
-           "mk_copy_hidden", "mk_copy_activation",
+           "mk_copy_hidden", "mk_copy_activation", "mk_prefill_slots", "mk_decode_step_slots",
+           "mk_kv_release", "mk_kv_set_pages", "mk_kv_get_pages", "mk_kv_free_pages",
+           "mk_build_flags",
            "mk_kv_pointer", "mk_copy_kv", "mk_set_mode", "mk_status", "mk_last_error",
            "mk_destroy", "mk_plan_build", "mk_plan_get_info", "mk_plan_get_tasks",
            "mk_plan_get_queue", "mk_plan_get_event_counts", "mk_plan_destroy",
@@ -63,7 +65,8 @@ class Weights(C.Structure):
 class Options(C.Structure):
     _fields_ = [("num_ctas", C.c_int), ("attn_splits", C.c_int), ("timeout_ms", C.c_int),
                 ("mode", C.c_int), ("l2_prefetch", C.c_int), ("weight_format", C.c_int),
-                ("batch_sequential", C.c_int), ("prefill_steps", C.c_int)]
+                ("batch_sequential", C.c_int), ("prefill_steps", C.c_int),
+                ("kv_page_tokens", C.c_int), ("kv_pool_pages", C.c_int)]
 
 
 class PlanInfo(C.Structure):
@@ -103,6 +106,14 @@ def lib(build_if_missing: bool = True):
     L.mk_decode_steps.argtypes = [vp, vp, i, i, vp, vp]
     L.mk_copy_hidden.argtypes = [vp, vp, i]
     L.mk_copy_activation.argtypes = [vp, i, vp, i]
+    L.mk_prefill_slots.argtypes = [vp, vp, ip, ip, i, vp, vp]
+    L.mk_decode_step_slots.argtypes = [vp, vp, ip, ip, i, vp, vp]
+    L.mk_kv_release.argtypes = [vp, i]
+    L.mk_kv_set_pages.argtypes = [vp, i, ip, i]
+    L.mk_kv_get_pages.argtypes = [vp, i, ip, i]
+    L.mk_kv_free_pages.argtypes = [vp]
+    L.mk_build_flags.argtypes = []
+    L.mk_build_flags.restype = i
     L.mk_kv_pointer.argtypes = [vp, i, i, i, i, C.POINTER(vp)]
     L.mk_copy_kv.argtypes = [vp, i, i, i, i, i, vp]
     L.mk_set_mode.argtypes = [vp, i]
@@ -157,7 +168,7 @@ class Plan:
         L = lib()
         self.h = C.c_void_p()
         cfg = make_config(model, max_seq, max_batch)
-        opt = Options(num_ctas, attn_splits, 0, 0, 0, weight_format, 0, 0)
+        opt = Options(num_ctas, attn_splits, 0, 0, 0, weight_format, 0, 0, 0, 0)
         rc = L.mk_plan_build(C.byref(cfg), C.byref(opt), int(num_ctas), C.byref(self.h))
         if rc != MK_OK:
             raise MkError(rc, "mk_plan_build rejected the configuration")
@@ -206,7 +217,7 @@ class Decoder:
                  max_batch: int = 1, num_ctas: int = 0, attn_splits: int = 0,
                  timeout_ms: int = 0, mode: int = MODE_MEGAKERNEL, stream=None,
                  l2_prefetch: int = 0, prefill_steps: int = 0, batch_sequential: int = 0,
-                 weight_format: int = 0):
+                 weight_format: int = 0, kv_page_tokens: int = 0, kv_pool_pages: int = 0):
         import torch
         L = lib()
         self.model = model
@@ -229,7 +240,7 @@ class Decoder:
                     None if model.tied_embeddings else ptr("lm_head"))
         cfg = make_config(model, max_seq, max_batch)
         opt = Options(num_ctas, attn_splits, timeout_ms, mode, l2_prefetch, weight_format,
-                      batch_sequential, prefill_steps)
+                      batch_sequential, prefill_steps, kv_page_tokens, kv_pool_pages)
         self.h = C.c_void_p()
         rc = L.mk_create(C.byref(cfg), C.byref(w), C.byref(opt), self.stream.cuda_stream,
                          C.byref(self.h))
@@ -264,6 +275,42 @@ class Decoder:
                                     None if logits_dev is None else logits_dev.data_ptr(),
                                     None if next_ids_dev is None else next_ids_dev.data_ptr()),
                self.h)
+
+    def prefill_slots(self, tokens_dev, offsets: Sequence[int], slots: Sequence[int],
+                      logits_dev=None, next_ids_dev=None):
+        """mk_prefill with request r on KV-cache slot slots[r]."""
+        _check(lib().mk_prefill_slots(self.h, tokens_dev.data_ptr(), _ints(offsets), _ints(slots),
+                                      len(slots),
+                                      None if logits_dev is None else logits_dev.data_ptr(),
+                                      None if next_ids_dev is None else next_ids_dev.data_ptr()),
+               self.h)
+
+    def decode_slots(self, tokens_dev, pos: Sequence[int], slots: Sequence[int], logits_dev=None,
+                     next_ids_dev=None):
+        """mk_decode_step with request r on KV-cache slot slots[r]."""
+        _check(lib().mk_decode_step_slots(self.h, tokens_dev.data_ptr(), _ints(pos), _ints(slots),
+                                          len(pos),
+                                          None if logits_dev is None else logits_dev.data_ptr(),
+                                          None if next_ids_dev is None else next_ids_dev.data_ptr()),
+               self.h)
+
+    def kv_release(self, slot: int):
+        _check(lib().mk_kv_release(self.h, int(slot)), self.h)
+
+    def kv_set_pages(self, slot: int, pages: Sequence[int]):
+        _check(lib().mk_kv_set_pages(self.h, int(slot), _ints(pages), len(pages)), self.h)
+
+    def kv_pages(self, slot: int) -> List[int]:
+        n = lib().mk_kv_get_pages(self.h, int(slot), None, 0)
+        _check(min(n, 0), self.h)
+        out = (C.c_int32 * max(n, 1))()
+        lib().mk_kv_get_pages(self.h, int(slot), out, n)
+        return list(out)[:n]
+
+    def kv_free_pages(self) -> int:
+        n = lib().mk_kv_free_pages(self.h)
+        _check(min(n, 0), self.h)
+        return int(n)
 
     def decode_steps(self, token_dev, pos0: int, n_steps: int, ids_dev, last_logits_dev=None):
         """n_steps greedy steps in one persistent launch; ids_dev[s] gets step s's id."""

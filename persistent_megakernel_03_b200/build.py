@@ -9,6 +9,9 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libmk.so")
+# The debug-bounds build: the same sources with MK_DEBUG_BOUNDS, whose tasks
+# check every access and report a violation through mk_status.
+LIB_DEBUG = os.path.join(HERE, "libmk_debug.so")
 SOURCES = ["plan.cpp", "kernel.cu", "api.cu", "attention.cu", "prefill.cu"]
 HEADERS = ["mk_internal.h", "plan.h", "ptx.cuh", "attn_math.cuh", "tc.cuh", "prefill.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -20,19 +23,23 @@ def _inputs():
     return files
 
 
-def is_fresh() -> bool:
-    if not os.path.exists(LIB):
+def is_fresh(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(f) <= t for f in _inputs())
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
+def build(force: bool = False, verbose: bool = False, extra=(), debug_bounds: bool = False) -> str:
     """Compiles every source to an object in parallel (one nvcc per file),
-    then links the shared library; skipped when libmk.so is newer than every
-    source and header."""
-    if not force and is_fresh():
-        return LIB
+    then links the shared library (libmk.so, or libmk_debug.so with
+    debug_bounds); skipped when the library is newer than every source and
+    header."""
+    out = LIB_DEBUG if debug_bounds else LIB
+    if debug_bounds:
+        extra = (*extra, "-DMK_DEBUG_BOUNDS")
+    if not force and is_fresh(out):
+        return out
     from concurrent.futures import ThreadPoolExecutor
     import tempfile
     nvcc = os.environ.get("NVCC", "nvcc")
@@ -54,15 +61,16 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
                 sys.stderr.write(f"--- {src}\n" + r.stdout + r.stderr)
         if failed:
             raise RuntimeError("nvcc failed building libmk.so: " + ", ".join(f[0] for f in failed))
-        tmp = LIB + f".tmp{os.getpid()}"
+        tmp = out + f".tmp{os.getpid()}"
         r = subprocess.run([nvcc, *ARCH, "-shared", "-o", tmp, *[o for _, o, _ in results]],
                            cwd=CSRC, capture_output=True, text=True)
         if r.returncode != 0:
             sys.stderr.write(r.stdout + r.stderr)
             raise RuntimeError("nvcc failed linking libmk.so")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, out)
+    return out
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv,
+                debug_bounds="--debug-bounds" in sys.argv))

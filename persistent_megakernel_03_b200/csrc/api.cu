@@ -27,6 +27,8 @@ cudaError_t launch_pack_gateup(uint16_t*, const uint16_t*, const uint16_t*, int,
 cudaError_t launch_step(const KernelArgs& args, int grid, bool cooperative, cudaStream_t st);
 cudaError_t launch_read_probe(const void* src, size_t bytes, unsigned long long* sink, int sms,
                               cudaStream_t st);
+cudaError_t launch_kv_table_update(int32_t* table, const int* idx, const int* val, int n,
+                                   cudaStream_t st);
 }  // namespace mk
 
 using namespace mk;
@@ -60,6 +62,13 @@ struct mk_ctx {
   PrefillScratch ps;             // its scratch (allocated at the first prefill)
   BatchScratch bs;               // batched decode step (allocated at its first use)
   bool last_batched = false;     // the last step ran the batched path (hidden in bs.x)
+  // KV pages: a contiguous cache is one max_seq page per slot (page s = slot s)
+  bool kv_paged = false;
+  int kv_page = 0, kv_pps = 1, kv_pool = 0;
+  std::vector<int32_t> kv_table_h;                // [max_batch][kv_pps], -1: no page
+  std::vector<int32_t> kv_free;                   // free physical pages (a stack)
+  std::vector<std::pair<int, int>> kv_pending;    // table entries not yet on the device
+  int32_t* kv_table_d = nullptr;
 };
 
 namespace mk {
@@ -348,7 +357,33 @@ extern "C" int mk_create(const mk_config* cfg, const mk_weights* w, const mk_opt
   if ((rc = dalloc(ctx, &rs_d, hs.size() * 4))) return bail(rc);
   CKC(cudaMemcpyAsync(rc_d, hc.data(), hc.size() * 4, cudaMemcpyHostToDevice, st));
   CKC(cudaMemcpyAsync(rs_d, hs.data(), hs.size() * 4, cudaMemcpyHostToDevice, st));
-  ctx->kv_bytes = (size_t)B * L * nkv * cfg->max_seq * d * 2;
+  // KV cache: contiguous (one max_seq page per request slot) or a pool of
+  // pages assigned to slots through a block table as positions are reached
+  // ("LLM高速化勉強会資料" slides 15-17: PagedAttention)
+  const int page = ctx->opt.kv_page_tokens;
+  if (page < 0 || (page > 0 && page % kKeyBlock)) {
+    ctx->err = "kv_page_tokens must be 0 (contiguous) or a positive multiple of 64";
+    return bail(MK_ERR_INVALID_ARG);
+  }
+  ctx->kv_paged = page > 0;
+  ctx->kv_page = ctx->kv_paged ? page : cfg->max_seq;
+  ctx->kv_pps = ctx->kv_paged ? (cfg->max_seq + page - 1) / page : 1;
+  ctx->kv_pool = ctx->kv_paged ? (ctx->opt.kv_pool_pages > 0 ? ctx->opt.kv_pool_pages : B * ctx->kv_pps)
+                               : B;
+  if (ctx->opt.kv_pool_pages < 0) {
+    ctx->err = "kv_pool_pages must be >= 0";
+    return bail(MK_ERR_INVALID_ARG);
+  }
+  ctx->kv_table_h.assign((size_t)B * ctx->kv_pps, -1);
+  if (ctx->kv_paged) {
+    for (int p = ctx->kv_pool - 1; p >= 0; --p) ctx->kv_free.push_back(p);
+  } else {
+    for (int sl = 0; sl < B; ++sl) ctx->kv_table_h[sl] = sl;
+  }
+  if ((rc = dalloc(ctx, &ctx->kv_table_d, ctx->kv_table_h.size() * 4))) return bail(rc);
+  CKC(cudaMemcpyAsync(ctx->kv_table_d, ctx->kv_table_h.data(), ctx->kv_table_h.size() * 4,
+                      cudaMemcpyHostToDevice, st));
+  ctx->kv_bytes = (size_t)ctx->kv_pool * L * nkv * ctx->kv_page * d * 2;
   uint16_t *kc = nullptr, *vc = nullptr;
   if ((rc = dalloc(ctx, &kc, ctx->kv_bytes))) return bail(rc);
   if ((rc = dalloc(ctx, &vc, ctx->kv_bytes))) return bail(rc);
@@ -427,6 +462,8 @@ extern "C" int mk_create(const mk_config* cfg, const mk_weights* w, const mk_opt
   m.trace = nullptr;
   m.embed = emb; m.lm_head = lm; m.final_norm = finaln; m.attn_norm = an; m.ffn_norm = fn;
   m.bqkv = bq; m.rope_cos = rc_d; m.rope_sin = rs_d; m.kcache = kc; m.vcache = vc;
+  m.kv_table = ctx->kv_table_d; m.kv_page = ctx->kv_page; m.kv_pps = ctx->kv_pps;
+  m.kv_pool = ctx->kv_pool; m.n_tickets = plan.n_tickets;
   m.x = x; m.q = q; m.attn = att; m.act = act; m.part = part; m.am = am;
   m.events = events; m.tickets = tickets; m.epoch = epoch; m.status = status;
   m.status_info = status + 1;
@@ -452,12 +489,80 @@ static int check_step_args(mk_ctx* ctx, const int32_t* pos_host, int n_req) {
   return MK_OK;
 }
 
+// Request slots of a call: slots_host, or 0..n_req-1 when it is NULL.  They
+// must lie in [0, max_batch) and differ from each other.
+static int resolve_slots(mk_ctx* ctx, const int32_t* slots_host, int n_req, int32_t* out) {
+  for (int r = 0; r < n_req; ++r) {
+    out[r] = slots_host ? slots_host[r] : r;
+    if (out[r] < 0 || out[r] >= ctx->cfg.max_batch)
+      return fail(ctx, MK_ERR_INVALID_ARG, "slot " + std::to_string(out[r]) + " outside [0, max_batch)");
+    for (int q = 0; q < r; ++q)
+      if (out[q] == out[r]) return fail(ctx, MK_ERR_INVALID_ARG, "a slot appears twice");
+  }
+  return MK_OK;
+}
+
+// Paged cache: assigns free pages to every logical page of `slot` that
+// positions [0, n_pos) touch and that has none yet (recorded for upload).
+static int kv_ensure(mk_ctx* ctx, int slot, int n_pos) {
+  if (!ctx->kv_paged) return MK_OK;
+  const int need = (n_pos + ctx->kv_page - 1) / ctx->kv_page;
+  for (int i = 0; i < need; ++i) {
+    int32_t& e = ctx->kv_table_h[(size_t)slot * ctx->kv_pps + i];
+    if (e >= 0) continue;
+    if (ctx->kv_free.empty()) return fail(ctx, MK_ERR_OOM, "KV page pool exhausted");
+    e = ctx->kv_free.back();
+    ctx->kv_free.pop_back();
+    ctx->kv_pending.emplace_back(slot * ctx->kv_pps + i, e);
+  }
+  return MK_OK;
+}
+
+// Enqueues the recorded table entries on the context's stream (a small kernel
+// carries them as arguments: no host buffer has to outlive the call).
+static int kv_flush(mk_ctx* ctx) {
+  constexpr int kBatch = 32;
+  for (size_t i = 0; i < ctx->kv_pending.size(); i += kBatch) {
+    int idx[kBatch], val[kBatch];
+    const int n = (int)std::min<size_t>(kBatch, ctx->kv_pending.size() - i);
+    for (int j = 0; j < n; ++j) {
+      idx[j] = ctx->kv_pending[i + j].first;
+      val[j] = ctx->kv_pending[i + j].second;
+    }
+    CK(launch_kv_table_update(ctx->kv_table_d, idx, val, n, ctx->stream));
+  }
+  ctx->kv_pending.clear();
+  return MK_OK;
+}
+
+static int decode_step_impl(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t* pos_host,
+                            const int32_t* slots_host, int n_req, float* logits_dev,
+                            int32_t* next_ids_dev);
+
 extern "C" int mk_decode_step(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t* pos_host,
                               int n_req, float* logits_dev, int32_t* next_ids_dev) {
+  return decode_step_impl(ctx, tokens_dev, pos_host, nullptr, n_req, logits_dev, next_ids_dev);
+}
+
+extern "C" int mk_decode_step_slots(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t* pos_host,
+                                    const int32_t* slots_host, int n_req, float* logits_dev,
+                                    int32_t* next_ids_dev) {
+  if (!slots_host) return fail(ctx, MK_ERR_INVALID_ARG, "slots_host is null");
+  return decode_step_impl(ctx, tokens_dev, pos_host, slots_host, n_req, logits_dev, next_ids_dev);
+}
+
+static int decode_step_impl(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t* pos_host,
+                            const int32_t* slots_host, int n_req, float* logits_dev,
+                            int32_t* next_ids_dev) {
   int rc = check_ctx(ctx);
   if (rc) return rc;
   if (!tokens_dev) return fail(ctx, MK_ERR_INVALID_ARG, "tokens_dev is null");
   if ((rc = check_step_args(ctx, pos_host, n_req))) return rc;
+  int32_t slots[kMaxBatch];
+  if ((rc = resolve_slots(ctx, slots_host, n_req, slots))) return rc;
+  for (int r = 0; r < n_req; ++r)
+    if ((rc = kv_ensure(ctx, slots[r], pos_host[r] + 1))) return rc;
+  if ((rc = kv_flush(ctx))) return rc;
   const int H = ctx->cfg.hidden, V = ctx->cfg.vocab;
   // Several requests: by default one batched step that streams every weight
   // matrix once (tensor-core GEMMs over the requests' columns).
@@ -471,7 +576,7 @@ extern "C" int mk_decode_step(mk_ctx* ctx, const int32_t* tokens_dev, const int3
     hp.n = n_req;
     for (int r = 0; r < n_req; ++r) {
       hp.pos[r] = pos_host[r];
-      hp.slot[r] = r;
+      hp.slot[r] = slots[r];
       hp.src[r] = r;
     }
     CK(cudaMemcpyAsync(ctx->bs.tokens, tokens_dev, (size_t)n_req * 4, cudaMemcpyDeviceToDevice,
@@ -496,7 +601,7 @@ extern "C" int mk_decode_step(mk_ctx* ctx, const int32_t* tokens_dev, const int3
     StepParams sp{};
     sp.n_req = 1;
     sp.pos[0] = pos_host[r];
-    sp.kv_slot[0] = r;
+    sp.kv_slot[0] = slots[r];
     sp.tokens = tokens_dev + r;
     sp.logits = logits_dev ? logits_dev + (size_t)r * V : nullptr;
     sp.next_ids = next_ids_dev ? next_ids_dev + r : nullptr;
@@ -521,6 +626,7 @@ extern "C" int mk_decode_steps(mk_ctx* ctx, const int32_t* token_dev, int pos0, 
   if (pos0 < 0 || (long long)pos0 + n_steps > ctx->cfg.max_seq)
     return fail(ctx, MK_ERR_POS_RANGE, "positions " + std::to_string(pos0) + ".." +
                                            std::to_string(pos0 + n_steps - 1) + " outside [0, max_seq)");
+  if ((rc = kv_ensure(ctx, 0, pos0 + n_steps)) || (rc = kv_flush(ctx))) return rc;
   StepParams sp{};
   sp.n_req = 1;
   sp.pos[0] = pos0;
@@ -559,8 +665,26 @@ extern "C" int mk_decode_step_host(mk_ctx* ctx, const int32_t* tokens_host, cons
   return MK_OK;
 }
 
+static int prefill_impl(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t* offsets_host,
+                        const int32_t* slots_host, int n_req, float* last_logits_dev,
+                        int32_t* next_ids_dev);
+
 extern "C" int mk_prefill(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t* offsets_host,
                           int n_req, float* last_logits_dev, int32_t* next_ids_dev) {
+  return prefill_impl(ctx, tokens_dev, offsets_host, nullptr, n_req, last_logits_dev, next_ids_dev);
+}
+
+extern "C" int mk_prefill_slots(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t* offsets_host,
+                                const int32_t* slots_host, int n_req, float* last_logits_dev,
+                                int32_t* next_ids_dev) {
+  if (!slots_host) return fail(ctx, MK_ERR_INVALID_ARG, "slots_host is null");
+  return prefill_impl(ctx, tokens_dev, offsets_host, slots_host, n_req, last_logits_dev,
+                      next_ids_dev);
+}
+
+static int prefill_impl(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t* offsets_host,
+                        const int32_t* slots_host, int n_req, float* last_logits_dev,
+                        int32_t* next_ids_dev) {
   int rc = check_ctx(ctx);
   if (rc) return rc;
   if (!tokens_dev || !offsets_host) return fail(ctx, MK_ERR_INVALID_ARG, "null argument");
@@ -570,6 +694,11 @@ extern "C" int mk_prefill(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t*
     if (offsets_host[r] < 0 || len < 1 || len > ctx->cfg.max_seq)
       return fail(ctx, MK_ERR_POS_RANGE, "prompt length outside [1, max_seq]");
   }
+  int32_t slots[kMaxBatch];
+  if ((rc = resolve_slots(ctx, slots_host, n_req, slots))) return rc;
+  for (int r = 0; r < n_req; ++r)
+    if ((rc = kv_ensure(ctx, slots[r], offsets_host[r + 1] - offsets_host[r]))) return rc;
+  if ((rc = kv_flush(ctx))) return rc;
   // Tensor-core path: every position but each prompt's last through the
   // whole-sequence operators; the last position then runs as a decode step
   // (its logits and greedy id).  Otherwise every position is a decode step:
@@ -582,7 +711,7 @@ extern "C" int mk_prefill(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t*
       if (!e.empty()) return fail(ctx, MK_ERR_CUDA, e);
     }
     const std::string e = prefill_run(ctx->md, ctx->pw, ctx->ps, ctx->stream, tokens_dev,
-                                      offsets_host, n_req);
+                                      offsets_host, slots, n_req);
     if (!e.empty()) {
       ctx->poisoned = true;
       return fail(ctx, MK_ERR_CUDA, e);
@@ -594,7 +723,7 @@ extern "C" int mk_prefill(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t*
       StepParams sp{};
       sp.n_req = 1;
       sp.pos[0] = t;
-      sp.kv_slot[0] = r;
+      sp.kv_slot[0] = slots[r];
       sp.tokens = tokens_dev + offsets_host[r] + t;
       const bool last = t == len - 1;
       sp.logits = last && last_logits_dev ? last_logits_dev + (size_t)r * ctx->cfg.vocab : nullptr;
@@ -647,6 +776,8 @@ extern "C" int mk_kv_pointer(mk_ctx* ctx, int req, int layer, int kv_head, int w
   if (req < 0 || req >= c.max_batch || layer < 0 || layer >= c.n_layers || kv_head < 0 ||
       kv_head >= c.n_kv_heads || which < 0 || which > 1)
     return fail(ctx, MK_ERR_INVALID_ARG, "bad KV index");
+  if (ctx->kv_paged)
+    return fail(ctx, MK_ERR_UNSUPPORTED, "a paged KV cache has no contiguous rows: use mk_copy_kv");
   const size_t off = (((size_t)req * c.n_layers + layer) * c.n_kv_heads + kv_head) * (size_t)c.max_seq * c.head_dim;
   *out_dev = (which ? ctx->md.vcache : ctx->md.kcache) + off;
   return MK_OK;
@@ -655,11 +786,73 @@ extern "C" int mk_kv_pointer(mk_ctx* ctx, int req, int layer, int kv_head, int w
 extern "C" int mk_copy_kv(mk_ctx* ctx, int req, int layer, int kv_head, int which, int n, void* dst_dev) {
   int rc = check_ctx(ctx);
   if (rc) return rc;
-  void* src = nullptr;
-  if ((rc = mk_kv_pointer(ctx, req, layer, kv_head, which, &src))) return rc;
-  if (!dst_dev || n < 0 || n > ctx->cfg.max_seq) return fail(ctx, MK_ERR_INVALID_ARG, "bad copy size");
-  CK(cudaMemcpyAsync(dst_dev, src, (size_t)n * ctx->cfg.head_dim * 2, cudaMemcpyDeviceToDevice, ctx->stream));
+  const mk_config& c = ctx->cfg;
+  if (req < 0 || req >= c.max_batch || layer < 0 || layer >= c.n_layers || kv_head < 0 ||
+      kv_head >= c.n_kv_heads || which < 0 || which > 1)
+    return fail(ctx, MK_ERR_INVALID_ARG, "bad KV index");
+  if (!dst_dev || n < 0 || n > c.max_seq) return fail(ctx, MK_ERR_INVALID_ARG, "bad copy size");
+  const size_t row = (size_t)c.head_dim;
+  const uint16_t* base = which ? ctx->md.vcache : ctx->md.kcache;
+  for (int p0 = 0; p0 < n; p0 += ctx->kv_page) {  // one copy per page
+    const int phys = ctx->kv_table_h[(size_t)req * ctx->kv_pps + p0 / ctx->kv_page];
+    if (phys < 0) return fail(ctx, MK_ERR_INVALID_ARG, "positions without a KV page");
+    const int rows = std::min(ctx->kv_page, n - p0);
+    const uint16_t* src =
+        base + (((size_t)phys * c.n_layers + layer) * c.n_kv_heads + kv_head) * ctx->kv_page * row;
+    CK(cudaMemcpyAsync(static_cast<uint16_t*>(dst_dev) + (size_t)p0 * row, src, rows * row * 2,
+                       cudaMemcpyDeviceToDevice, ctx->stream));
+  }
   return MK_OK;
+}
+
+extern "C" int mk_kv_release(mk_ctx* ctx, int slot) {
+  int rc = check_ctx(ctx);
+  if (rc) return rc;
+  if (slot < 0 || slot >= ctx->cfg.max_batch) return fail(ctx, MK_ERR_INVALID_ARG, "bad slot");
+  if (!ctx->kv_paged) return MK_OK;  // a contiguous slot keeps its region
+  for (int i = 0; i < ctx->kv_pps; ++i) {
+    int32_t& e = ctx->kv_table_h[(size_t)slot * ctx->kv_pps + i];
+    if (e < 0) continue;
+    ctx->kv_free.push_back(e);
+    e = -1;
+    ctx->kv_pending.emplace_back(slot * ctx->kv_pps + i, -1);
+  }
+  return kv_flush(ctx);
+}
+
+extern "C" int mk_kv_set_pages(mk_ctx* ctx, int slot, const int32_t* pages_host, int n_pages) {
+  int rc = check_ctx(ctx);
+  if (rc) return rc;
+  if (!ctx->kv_paged) return fail(ctx, MK_ERR_UNSUPPORTED, "the KV cache is not paged");
+  if (slot < 0 || slot >= ctx->cfg.max_batch || n_pages < 0 || n_pages > ctx->kv_pps ||
+      (n_pages && !pages_host))
+    return fail(ctx, MK_ERR_INVALID_ARG, "bad slot or page count");
+  if ((rc = mk_kv_release(ctx, slot))) return rc;
+  for (int i = 0; i < n_pages; ++i) {
+    auto it = std::find(ctx->kv_free.begin(), ctx->kv_free.end(), pages_host[i]);
+    if (it == ctx->kv_free.end()) {
+      mk_kv_release(ctx, slot);
+      return fail(ctx, MK_ERR_INVALID_ARG, "page " + std::to_string(pages_host[i]) +
+                                               " is out of range or already assigned");
+    }
+    ctx->kv_free.erase(it);
+    ctx->kv_table_h[(size_t)slot * ctx->kv_pps + i] = pages_host[i];
+    ctx->kv_pending.emplace_back(slot * ctx->kv_pps + i, pages_host[i]);
+  }
+  return kv_flush(ctx);
+}
+
+extern "C" int mk_kv_get_pages(mk_ctx* ctx, int slot, int32_t* pages_out, int cap) {
+  if (!ctx || slot < 0 || slot >= ctx->cfg.max_batch || cap < 0 || (cap && !pages_out))
+    return MK_ERR_INVALID_ARG;
+  for (int i = 0; i < std::min(cap, ctx->kv_pps); ++i)
+    pages_out[i] = ctx->kv_table_h[(size_t)slot * ctx->kv_pps + i];
+  return ctx->kv_pps;
+}
+
+extern "C" int mk_kv_free_pages(mk_ctx* ctx) {
+  if (!ctx) return MK_ERR_INVALID_ARG;
+  return (int)ctx->kv_free.size();
 }
 
 extern "C" int mk_set_trace(mk_ctx* ctx, unsigned long long* trace_dev) {
@@ -699,6 +892,7 @@ extern "C" int mk_status(mk_ctx* ctx) {
                            ? (st[1] >= 0 ? "event wait timed out at task "
                                          : "shared-memory wait timed out, kind ")
                        : st[0] == MK_ERR_TOKEN_RANGE ? "token id out of range: "
+                       : st[0] == MK_ERR_BOUNDS      ? "bounds check failed (debug build), check "
                                                      : "device error, detail ";
     return fail(ctx, st[0], std::string(what) + std::to_string(st[1]));
   }
@@ -710,6 +904,14 @@ extern "C" int mk_status(mk_ctx* ctx) {
     }
   }
   return MK_OK;
+}
+
+extern "C" int mk_build_flags(void) {
+#ifdef MK_DEBUG_BOUNDS
+  return MK_BUILD_DEBUG_BOUNDS;
+#else
+  return 0;
+#endif
 }
 
 extern "C" const char* mk_last_error(const mk_ctx* ctx) {

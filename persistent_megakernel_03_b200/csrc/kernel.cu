@@ -124,12 +124,17 @@ __device__ __forceinline__ float2 dot16_fp8(const uint4 w, const float2 (&x)[8],
   return acc;
 }
 
+// Rows of the matrix a GEMV task streams.
+__device__ __forceinline__ int task_matrix_rows(const ModelDev& m, const Task& t) {
+  return t.kind == T_QKV ? qkv_rows(m.n_q, m.n_kv, m.head_dim)
+         : t.kind == T_GATEUP ? 2 * m.ffn
+         : t.kind == T_LMHEAD ? m.vocab : m.hidden;
+}
+
 // Row scales of a task's fp8 matrix: they follow the matrix's codes in the
 // same allocation, at the 16-byte-aligned end of its rows x K bytes.
 __device__ __forceinline__ const float* task_wscale(const ModelDev& m, const Task& t) {
-  const int rows = t.kind == T_QKV ? qkv_rows(m.n_q, m.n_kv, m.head_dim)
-                   : t.kind == T_GATEUP ? 2 * m.ffn
-                   : t.kind == T_LMHEAD ? m.vocab : m.hidden;
+  const int rows = task_matrix_rows(m, t);
   const size_t off = ((size_t)rows * t.K + 15) & ~(size_t)15;
   return reinterpret_cast<const float*>(reinterpret_cast<const uint8_t*>(t.w) + off);
 }
@@ -189,7 +194,11 @@ __device__ __forceinline__ AttnRange attn_range(const Task& t, const StepParams&
   const int n = pos + 1;
   const int live = attn_live_splits(n, m.attn_splits, attn_keys_per_chunk(m.head_dim));
   if (t.row1 >= live) return r;  // a split with no keys at this position
-  const int chunk = (n + live - 1) / live;
+  // keys per split; with a paged cache rounded up to whole key blocks, so that
+  // split ranges start on page boundaries (a trailing split may then hold no
+  // keys: it contributes an empty partial)
+  int chunk = (n + live - 1) / live;
+  if (m.kv_page < m.max_seq) chunk = (chunk + kKeyBlock - 1) / kKeyBlock * kKeyBlock;
   r.k0 = min(n, t.row1 * chunk);
   r.k1 = min(n, r.k0 + chunk);
   r.old_end = min(r.k1, pos);
@@ -201,8 +210,15 @@ __device__ __forceinline__ AttnRange attn_range(const Task& t, const StepParams&
 
 __device__ __forceinline__ size_t kv_offset(const ModelDev& m, int slot, int layer, int g,
                                             int key) {
-  return ((((size_t)slot * m.n_layers + layer) * m.n_kv + g) * (size_t)m.max_seq + key) *
-         (size_t)m.head_dim;
+  return kv_row(m, slot, layer, g, key);
+}
+
+// Keys of the ring chunk that starts at key k of [k, end): at most one ring
+// chunk, and never across a KV page boundary (a chunk is one bulk copy of
+// consecutive rows).  The producer and the attention task use the same rule.
+__device__ __forceinline__ int attn_chunk_keys(const ModelDev& m, int k, int end) {
+  const int to_page = m.kv_page - k % m.kv_page;
+  return min(min(attn_keys_per_chunk(m.head_dim), end - k), to_page);
 }
 
 // ---------------------------------------------------------------- producer
@@ -239,7 +255,9 @@ struct ChunkCursor {
         if (r.active) {
           const int k = off < 0 ? r.k0 : off;
           if (k < r.old_end) {
-            const int nk = min(attn_keys_per_chunk(m.head_dim), r.old_end - k);
+            const int nk = attn_chunk_keys(m, k, r.old_end);
+            bounds_ok(m, nk > 0 && k + nk <= m.max_seq, kBndKvKey);
+            bounds_ok(m, (uint32_t)nk * m.head_dim * 2 <= kSlotBytes / 2, kBndChunkBytes);
             const size_t o = kv_offset(m, sp.kv_slot[t.req], t.layer, t.row0, k);
             c.src0 = m.kcache + o;
             c.src1 = m.vcache + o;
@@ -253,6 +271,12 @@ struct ChunkCursor {
         const int r = off < 0 ? t.row0 : off;
         if (r < t.row1) {
           const int nr = min(t.chunk_rows, t.row1 - r);
+          if (!bounds_ok(m, r + nr <= task_matrix_rows(m, t), kBndChunkRows) ||
+              !bounds_ok(m, (size_t)nr * t.K * m.wbytes <= kSlotBytes, kBndChunkBytes)) {
+            ++qi;  // skip the task's remaining chunks (its workers see the abort)
+            off = -1;
+            continue;
+          }
           c.src0 = reinterpret_cast<const uint8_t*>(t.w) + (size_t)r * t.K * m.wbytes;
           c.src1 = nullptr;
           c.bytes0 = (uint32_t)nr * t.K * m.wbytes;
@@ -405,39 +429,28 @@ __device__ __forceinline__ void scheduler(const KernelArgs& a, Smem& s, int q0, 
 
 // ------------------------------------------------------------ worker: GEMV
 
-template <int NR>
-__device__ __forceinline__ float warp_reduce_rows(float (&v)[NR], int lane) {
-  if constexpr (NR == 4) {
-    const bool b4 = lane & 16;
-    float a0 = b4 ? v[2] : v[0], a1 = b4 ? v[3] : v[1];
-    float s0 = b4 ? v[0] : v[2], s1 = b4 ? v[1] : v[3];
-    a0 += __shfl_xor_sync(0xffffffffu, s0, 16);
-    a1 += __shfl_xor_sync(0xffffffffu, s1, 16);
-    const bool b3 = lane & 8;
-    float k = b3 ? a1 : a0, snd = b3 ? a0 : a1;
-    k += __shfl_xor_sync(0xffffffffu, snd, 8);
-    k += __shfl_xor_sync(0xffffffffu, k, 4);
-    k += __shfl_xor_sync(0xffffffffu, k, 2);
-    k += __shfl_xor_sync(0xffffffffu, k, 1);
-    return k;  // row lane >> 3
-  } else if constexpr (NR == 2) {
-    const bool b4 = lane & 16;
-    float k = b4 ? v[1] : v[0], snd = b4 ? v[0] : v[1];
-    k += __shfl_xor_sync(0xffffffffu, snd, 16);
-    k += __shfl_xor_sync(0xffffffffu, k, 8);
-    k += __shfl_xor_sync(0xffffffffu, k, 4);
-    k += __shfl_xor_sync(0xffffffffu, k, 2);
-    k += __shfl_xor_sync(0xffffffffu, k, 1);
-    return k;  // row lane >> 4
-  } else {
-    float k = v[0];
-    k += __shfl_xor_sync(0xffffffffu, k, 16);
-    k += __shfl_xor_sync(0xffffffffu, k, 8);
-    k += __shfl_xor_sync(0xffffffffu, k, 4);
-    k += __shfl_xor_sync(0xffffffffu, k, 2);
-    k += __shfl_xor_sync(0xffffffffu, k, 1);
-    return k;
+// Sums eight per-lane values across a warp at once (a transposed butterfly:
+// at each of the first three levels a lane keeps half of its values and adds
+// its partner's copy of them), seven shuffles in all instead of five per
+// value; lane l ends with the warp's sum of value l >> 2.
+__device__ __forceinline__ float warp_reduce8(const float (&v)[8], int lane) {
+  const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+  float a[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float keep = b4 ? v[i + 4] : v[i], send = b4 ? v[i] : v[i + 4];
+    a[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
   }
+  float c[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const float keep = b3 ? a[i + 2] : a[i], send = b3 ? a[i] : a[i + 2];
+    c[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+  }
+  float k = (b2 ? c[1] : c[0]) + __shfl_xor_sync(0xffffffffu, b2 ? c[0] : c[1], 4);
+  k += __shfl_xor_sync(0xffffffffu, k, 2);
+  k += __shfl_xor_sync(0xffffffffu, k, 1);
+  return k;
 }
 
 // Waits for ring chunk `seq`.  Once the CTA is aborting the workers no longer
@@ -532,8 +545,14 @@ __device__ __forceinline__ float gemv_load_input(const KernelArgs& a, const Step
 }
 
 // Streams the task's rows through the ring and leaves y[row] in s.ybuf.
+// A ring chunk holds NR rows per row-lane; a thread multiplies its CPT pieces
+// of each with its inputs and keeps the NR partial sums, and after every
+// 8 / NR chunks the warp reduces the eight partials at once (warp_reduce8), so
+// no shuffle chain sits between a chunk's arrival and its release.  The warps
+// of a row-lane are added at the end in a fixed order.
 template <int CPT, int NR, int PW>
 __device__ __forceinline__ void gemv_stream(const KernelArgs& a, Smem& s, const Task& t, uint32_t& seq, int wtid) {
+  constexpr int kGroup = 8 / NR;  // chunks per reduction
   const int TPR = t.tpr;
   const int rl = wtid / TPR, ct = wtid % TPR;
   const int wpr = TPR >> 5, wir = ct >> 5;
@@ -541,6 +560,8 @@ __device__ __forceinline__ void gemv_stream(const KernelArgs& a, Smem& s, const 
   const int K = t.K, C = K / (2 * PW);
   const size_t row_bytes = (size_t)K * 8 / PW;
   const int nrows = t.row1 - t.row0;
+  const int crows = t.chunk_rows;
+  const int nchunks = (nrows + crows - 1) / crows;
   // fp8: the row scales of this thread's output rows (at most two: a task
   // has at most kYBufFloats = 2 x 512 rows), requested with the inputs
   static_assert(kYBufFloats <= 2 * kWorkerThreads, "two output rows per thread at most");
@@ -559,41 +580,48 @@ __device__ __forceinline__ void gemv_stream(const KernelArgs& a, Smem& s, const 
     for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     if (lane == 0) s.red[wtid >> 5] = ss;  // read after the barrier that ends the stream
   }
-  constexpr int kShift = NR == 4 ? 3 : (NR == 2 ? 4 : 5);
-  for (int r = 0; r < nrows; r += t.chunk_rows) {
-    const int rows_here = min(t.chunk_rows, nrows - r);
-    const int slot = seq % kRingSlots;
-    wait_full(s, seq, a.m);
-    if (r == 0) trace_mark(a, s, wtid, 3);
-    const uint8_t* base = s.ring[slot];
-    float acc[NR];
+  for (int q0 = 0; q0 < nchunks; q0 += kGroup) {
+    float v[8];
 #pragma unroll
-    for (int j = 0; j < NR; ++j) {
-      float2 a2 = make_float2(0.f, 0.f);
-      const int lr = rl * NR + j;
-      if (lr < rows_here) {
-        const uint8_t* row = base + (size_t)lr * row_bytes;
+    for (int j = 0; j < kGroup; ++j) {
+      const int q = q0 + j;
+      float2 a2[NR];
 #pragma unroll
-        for (int c = 0; c < CPT; ++c) {
-          const int cc = ct + c * TPR;
-          if (cc < C) {
-            const uint4 piece = *reinterpret_cast<const uint4*>(row + (size_t)cc * 16);
-            if constexpr (PW == 4) a2 = dot8(piece, x2[c], a2);
-            else a2 = dot16_fp8(piece, x2[c], a2);
+      for (int k = 0; k < NR; ++k) a2[k] = make_float2(0.f, 0.f);
+      if (q < nchunks) {  // warp-uniform
+        const int slot = seq % kRingSlots;
+        wait_full(s, seq, a.m);
+        if (q == 0) trace_mark(a, s, wtid, 3);
+        const int rows_here = min(crows, nrows - q * crows);
+#pragma unroll
+        for (int k = 0; k < NR; ++k) {
+          const int lr = rl * NR + k;
+          if (lr < rows_here && bounds_ok(a.m, (size_t)(lr + 1) * row_bytes <= kSlotBytes, kBndSlotRow)) {
+            const uint8_t* row = s.ring[slot] + (size_t)lr * row_bytes;
+#pragma unroll
+            for (int c = 0; c < CPT; ++c) {
+              const int cc = ct + c * TPR;
+              if (cc < C) {
+                const uint4 piece = *reinterpret_cast<const uint4*>(row + (size_t)cc * 16);
+                if constexpr (PW == 4) a2[k] = dot8(piece, x2[c], a2[k]);
+                else a2[k] = dot16_fp8(piece, x2[c], a2[k]);
+              }
+            }
           }
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.empty[slot]);
+        ++seq;
       }
-      acc[j] = a2.x + a2.y;
+#pragma unroll
+      for (int k = 0; k < NR; ++k) v[j * NR + k] = a2[k].x + a2[k].y;
     }
-    const float v = warp_reduce_rows<NR>(acc, lane);
-    const int jj = lane >> kShift;
-    if ((lane & ((1 << kShift) - 1)) == 0) {
-      const int lr = rl * NR + jj;
-      if (lr < rows_here) s.scratch[wir * nrows + r + lr] = v;
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&s.empty[slot]);
-    ++seq;
+    const float r8 = warp_reduce8(v, lane);
+    const int idx = lane >> 2, q = q0 + idx / NR;
+    const int row = q * crows + rl * NR + idx % NR;
+    if ((lane & 3) == 0 && q < nchunks && row < nrows &&
+        bounds_ok(a.m, (wir + 1) * nrows <= kScratchBytes / 4, kBndScratch))
+      s.scratch[wir * nrows + row] = r8;
   }
   trace_mark(a, s, wtid, 4);
   worker_sync();
@@ -617,14 +645,14 @@ __device__ __forceinline__ void gemv_stream(const KernelArgs& a, Smem& s, const 
     for (; w < wpr; ++w) y0 += s.scratch[w * nrows + i];
     float y = (y0 + y1) + (y2 + y3);
     if constexpr (PW == 8) y *= i < kWorkerThreads ? rsc0 : rsc1;  // fp8 row scale
-    s.ybuf[i] = has_norm ? y * r : y;
+    if (bounds_ok(a.m, i < kYBufFloats, kBndYbuf)) s.ybuf[i] = has_norm ? y * r : y;
   }
   worker_sync();
 }
 
 template <int CPT, int PW>
 __device__ __forceinline__ void gemv_dispatch_nr(const KernelArgs& a, Smem& s, const Task& t, uint32_t& seq,
-                                 int wtid) {
+                                                 int wtid) {
   const int nr = t.chunk_rows / (kWorkerThreads / t.tpr);
   if constexpr (PW == 8 && CPT > 2) {
     gemv_stream<CPT, 1, PW>(a, s, t, seq, wtid);  // (fp8 geometry never has NR > 1 here)
@@ -738,8 +766,10 @@ __device__ __forceinline__ void epilogue_qkv(const KernelArgs& a, Smem& s, const
     }
     if (which == 0) {
       float* q = m.q + (size_t)head * d;
-      q[dim0] = y0;
-      q[dim1] = y1;
+      if (bounds_ok(m, head < m.n_q && dim0 < d && dim1 < d, kBndQ)) {
+        q[dim0] = y0;
+        q[dim1] = y1;
+      }
     } else {
       uint16_t* cache = which == 1 ? m.kcache : m.vcache;
       const size_t off = kv_offset(m, slot, t.layer, head, pos);
@@ -762,6 +792,7 @@ __device__ __forceinline__ void epilogue_residual(const KernelArgs& a, Smem& s, 
   }
   for (int i = wtid; i < nrows; i += kWorkerThreads) {
     const int row = t.row0 + i;
+    if (!bounds_ok(m, row < m.hidden, kBndResidual)) continue;
     const float old = from_embed ? bf16_to_float(m.embed[(size_t)tok * m.hidden + row])
                       : (i == wtid ? pre.res : __ldcg(m.x + row));
     m.x[row] = old + s.ybuf[i];
@@ -774,7 +805,7 @@ __device__ __forceinline__ void epilogue_swiglu(const KernelArgs& a, Smem& s, co
   for (int pi = wtid; pi < npairs; pi += kWorkerThreads) {
     const float g = s.ybuf[2 * pi], u = s.ybuf[2 * pi + 1];
     const float silu = g / (1.0f + expf(-g));
-    m.act[(t.row0 >> 1) + pi] = silu * u;
+    if (bounds_ok(m, (t.row0 >> 1) + pi < m.ffn, kBndAct)) m.act[(t.row0 >> 1) + pi] = silu * u;
   }
 }
 
@@ -785,7 +816,7 @@ __device__ __forceinline__ void epilogue_lmhead(const KernelArgs& a, Smem& s, co
   unsigned long long best = 0ull;
   for (int i = wtid; i < nrows; i += kWorkerThreads) {
     const float y = s.ybuf[i];
-    if (sp.logits) sp.logits[t.row0 + i] = y;
+    if (sp.logits && bounds_ok(m, t.row0 + i < m.vocab, kBndLogits)) sp.logits[t.row0 + i] = y;
     const unsigned long long k = argmax_key(y, t.row0 + i);
     best = k > best ? k : best;
   }
@@ -800,7 +831,8 @@ __device__ __forceinline__ void epilogue_lmhead(const KernelArgs& a, Smem& s, co
     for (int w = 0; w < kWorkerWarps; ++w) b = s.red64[w] > b ? s.red64[w] : b;
     s.lm_best = b;
     s.flag = 0;
-    if (t.req & 2) {  // the CTA's last LM task publishes its candidate
+    if ((t.req & 2) && bounds_ok(m, t.aux >= 0 && t.aux < m.n_lm_slots, kBndArgmax)) {
+      // the CTA's last LM task publishes its candidate
       m.am[t.aux] = b;
       __threadfence();
       const uint32_t old = atom_add_acq_rel_gpu(m.tickets, 1u);
@@ -875,9 +907,8 @@ __device__ __forceinline__ void attn_task(const KernelArgs& a, Smem& s, const Ta
   }
   attn_init<DPL, G>(st, m.q + (size_t)g * G * d, d, m.attn_scale, lane);
   trace_mark(a, s, wtid, 2);
-  const int kpc = attn_keys_per_chunk(d);
-  for (int k = r.k0; k < r.old_end; k += kpc) {
-    const int nk = min(kpc, r.old_end - k);
+  for (int k = r.k0, nk = 0; k < r.old_end; k += nk) {
+    nk = attn_chunk_keys(m, k, r.old_end);
     const int slot = seq % kRingSlots;
     wait_full(s, seq, m);
     if (k == r.k0) trace_mark(a, s, wtid, 3);
@@ -962,6 +993,7 @@ __device__ __forceinline__ void attn_task(const KernelArgs& a, Smem& s, const Ta
   if (warp < kHalf) attn_write_state<DPL, G>(st, buf + warp * sw, PS, d, lane);
   worker_sync();
   const int live = r.live;
+  if (!bounds_ok(m, b == 0 && (g + 1) * G <= m.n_q, kBndAttnOut)) return;
   if (live == 1) {
     // the only split: normalise and write the attention output directly
     float* out = m.attn + ((size_t)b * m.n_q + (size_t)g * G) * d;
@@ -985,6 +1017,7 @@ __device__ __forceinline__ void attn_task(const KernelArgs& a, Smem& s, const Ta
   }
   // The split's partial -- output unnormalised at the split's maximum, the
   // maximum, the sum.
+  if (!bounds_ok(m, b == 0 && g < m.n_kv && split < S_all, kBndPart)) return;
   float* part = m.part + ((size_t)(b * m.n_kv + g) * S_all + split) * G * PS;
   for (int idx = wtid; idx < G * (d + 2); idx += kWorkerThreads) {
     const int h = idx / (d + 2), i = idx - h * (d + 2);
@@ -1011,7 +1044,8 @@ __device__ __forceinline__ void attn_task(const KernelArgs& a, Smem& s, const Ta
   // step, which reaches it only after this step's events.
   worker_sync();
   if (wtid == 0) {
-    uint32_t* tk = m.tickets + kAttnTicketBase + ((size_t)t.layer * m.max_batch + b) * m.n_kv + g;
+    const size_t ti = kAttnTicketBase + ((size_t)t.layer * m.max_batch + b) * m.n_kv + g;
+    uint32_t* tk = m.tickets + (bounds_ok(m, ti < (size_t)m.n_tickets, kBndTicket) ? ti : 0);
     const uint32_t old = atom_add_acq_rel_gpu(tk, 1u);  // release: this split's partial
     const bool last = old == (uint32_t)live - 1u;
     if (last) *tk = 0u;
@@ -1182,6 +1216,17 @@ __global__ void pack_gateup_kernel(uint16_t* dst, const uint16_t* wg, const uint
   for (int i = threadIdx.x; i < H / 8; i += blockDim.x) d4[i] = s4[i];
 }
 
+// KV page table: entries idx[i] <- val[i] (the host's changes, carried as
+// arguments so no host buffer has to outlive the launch).
+struct KvTableUpdate {
+  int32_t n;
+  int32_t idx[32];
+  int32_t val[32];
+};
+__global__ void kv_table_update_kernel(int32_t* table, const KvTableUpdate u) {
+  if ((int)threadIdx.x < u.n) table[u.idx[threadIdx.x]] = u.val[threadIdx.x];
+}
+
 // Read-only stream: grid-stride 128-bit loads, bypassing L1, evict-first in
 // L2; the XOR of everything goes to one word.
 __global__ void __launch_bounds__(512) read_probe_kernel(const uint4* __restrict__ src, size_t n16,
@@ -1265,6 +1310,17 @@ cudaError_t launch_pack_qkv_bias(uint16_t* dst, const uint16_t* bq, const uint16
 cudaError_t launch_pack_gateup(uint16_t* dst, const uint16_t* wg, const uint16_t* wu, int H, int F,
                                cudaStream_t st) {
   pack_gateup_kernel<<<2 * F, 128, 0, st>>>(dst, wg, wu, H, F);
+  return cudaGetLastError();
+}
+cudaError_t launch_kv_table_update(int32_t* table, const int* idx, const int* val, int n,
+                                   cudaStream_t st) {
+  KvTableUpdate u{};
+  u.n = n < 32 ? n : 32;
+  for (int i = 0; i < u.n; ++i) {
+    u.idx[i] = idx[i];
+    u.val[i] = val[i];
+  }
+  kv_table_update_kernel<<<1, 32, 0, st>>>(table, u);
   return cudaGetLastError();
 }
 cudaError_t launch_read_probe(const void* src, size_t bytes, unsigned long long* sink, int sms,

@@ -86,9 +86,17 @@ struct ModelDev {
   // rope table [max_seq][head_dim/2]
   const float* rope_cos;
   const float* rope_sin;
-  // KV cache [slot][layer][kv_head][max_seq][head_dim] bf16
+  // KV cache: a pool of pages [page][layer][kv_head][kv_page][head_dim] bf16, K
+  // and V separate; logical page i of request slot s (positions
+  // [i*kv_page, (i+1)*kv_page)) is physical page kv_table[s*kv_pps + i].  A
+  // contiguous cache is the case kv_page = max_seq, kv_pps = 1, page s = slot s.
   uint16_t* kcache;
   uint16_t* vcache;
+  const int32_t* kv_table;     // [max slots][kv_pps]
+  int32_t kv_page;             // positions per page (a multiple of 64, or max_seq)
+  int32_t kv_pps;              // table entries per slot
+  int32_t kv_pool;             // pages in the pool
+  int32_t n_tickets;           // entries of `tickets`
   // activations (fp32, per batch slot)
   float* x;        // [batch][hidden] residual stream
   float* q;        // [batch][n_q*head_dim] rotated queries
@@ -124,6 +132,45 @@ struct KernelArgs {
 
 // ---------------------------------------------------------------- layouts
 
+// Keys per attention block: the ring's key chunk (d = 128), and the unit in
+// which split ranges are rounded and pages are sized.
+constexpr int kKeyBlock = 64;
+
+#ifdef __CUDACC__
+// Debug-bounds build (compiled with -DMK_DEBUG_BOUNDS): every task checks the
+// indices of its global and shared-memory accesses against their buffers;
+// a failed check records MK_ERR_BOUNDS with a code naming the check in the
+// status word and the access is skipped (the launch goes on; no trap).  In
+// the normal build the checks compile to nothing.
+enum BoundsWhere : int32_t {
+  kBndChunkRows = 1, kBndChunkBytes = 2, kBndKvKey = 3, kBndKvPage = 4, kBndSlotRow = 5,
+  kBndScratch = 6, kBndYbuf = 7, kBndQ = 8, kBndResidual = 9, kBndAct = 10, kBndLogits = 11,
+  kBndArgmax = 12, kBndPart = 13, kBndAttnOut = 14, kBndTicket = 15
+};
+__device__ __forceinline__ bool bounds_ok(const ModelDev& m, bool ok, int where) {
+#ifdef MK_DEBUG_BOUNDS
+  if (!ok && atomicCAS(m.status, 0, -10 /* MK_ERR_BOUNDS */) == 0) m.status_info[0] = where;
+  return ok;
+#else
+  (void)m; (void)where;
+  return true;
+#endif
+}
+
+// Element offset of the cached K/V row of (slot, layer, KV head, position).
+// Host code guarantees every page a launch touches is assigned; an entry that
+// is not (-1) maps to page 0, so an access always stays inside the pool.
+__device__ __forceinline__ size_t kv_row(const ModelDev& m, int slot, int layer, int g, int key) {
+  const int lp = key / m.kv_page;
+  int phys = __ldg(m.kv_table + slot * m.kv_pps + lp);
+  if (!bounds_ok(m, key >= 0 && key < m.max_seq, kBndKvKey)) return 0;
+  if (!bounds_ok(m, phys >= 0 && phys < m.kv_pool, kBndKvPage)) return 0;
+  phys = phys < 0 ? 0 : phys;
+  return ((((size_t)phys * m.n_layers + layer) * m.n_kv + g) * (size_t)m.kv_page +
+          (size_t)(key - lp * m.kv_page)) * (size_t)m.head_dim;
+}
+#endif
+
 MK_HD int qkv_rows(int n_q, int n_kv, int d) { return (n_q + 2 * n_kv) * d; }
 
 // Packed fused-QKV row r -> source (which 0 q / 1 k / 2 v, head, dim).
@@ -146,9 +193,12 @@ MK_HD void qkv_source(int r, int G, int d, int* which, int* head, int* dim) {
   }
 }
 
-// GEMV geometry for an input of K columns on kWorkerThreads threads:
-// the K/8 16-byte column chunks are spread over `tpr` threads (a row-lane);
-// 512/tpr row-lanes work on different rows of the same ring chunk.
+// GEMV geometry for an input of K columns on kWorkerThreads threads: the K/8
+// 16-byte column pieces of a row are spread over `tpr` threads (a row-lane;
+// the smallest power of two >= K/8, from a warp to all 512 threads), so each
+// thread loads its inputs once and no input is loaded twice by a CTA when
+// tpr = 512; the 512/tpr row-lanes work on different rows of a ring chunk,
+// `nr` rows each (up to 4, as many as fit a 32 KB chunk).
 MK_HD int gemv_tpr(int K) {
   int C = K / 8;
   int t = 32;
@@ -164,7 +214,8 @@ MK_HD int gemv_nr(int K) {
   return nr;
 }
 MK_HD int gemv_chunk_rows(int K) { return gemv_nr(K) * (kWorkerThreads / gemv_tpr(K)); }
-// Largest number of output rows one task may own (partial-sum buffer bound).
+// Largest number of output rows one task may own (partial-sum buffer bound:
+// one fp32 per row and warp of a row-lane).
 MK_HD int gemv_max_task_rows(int K) {
   int wpr = gemv_tpr(K) / 32;
   int r = kScratchBytes / (4 * wpr);

@@ -8,10 +8,12 @@
 //     -> causal GQA attention over the cache -> [xh, xl] -> GEMM(W_o) -> x +=
 //   x -> RMSNorm -> [xh, xl] -> GEMM(W_gate/up) -> SwiGLU -> [xh, xl]
 //     -> GEMM(W_down) -> x +=
-// The GEMM computes Y[t][r] = sum_k W[r][k] * (xh[t][k] + xl[t][k]): the fp32
-// activation is split into bf16 xh = bf16(x) and xl = bf16(x - xh), so two
-// bf16 tcgen05.mma per K step reproduce the fp32 product to ~2^-16 relative,
-// well inside the decode path's tolerance against the fp32 oracle.
+// The GEMM computes Y[t][r] = sum_k W[r][k] * (xh[t][k] + xm[t][k] + xl[t][k]):
+// the fp32 activation is split into three bf16 parts xh = bf16(x),
+// xm = bf16(x - xh), xl = bf16(x - xh - xm) (each difference exact), 24
+// significand bits in all, so three bf16 tcgen05.mma per K step reproduce the
+// fp32 product to fp32 precision (a two-part split keeps only ~2^-16, which at
+// full depth visibly moves the logits).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -39,11 +41,23 @@ __device__ __forceinline__ uint16_t bf16_bits(float f) {
 }
 __device__ __forceinline__ float bf16_val(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
 
-// v -> (bf16(v), bf16(v - bf16(v)))
+// v -> (bf16(v), bf16(v - bf16(v))): the batched decode step's two parts
 __device__ __forceinline__ void split_store(float v, uint16_t* hi, uint16_t* lo, size_t i) {
   const uint16_t h = bf16_bits(v);
   hi[i] = h;
   lo[i] = bf16_bits(v - bf16_val(h));
+}
+
+// v -> (h, m, l) = (bf16(v), bf16(v - h), bf16(v - h - m)): the prompt GEMMs'
+// three parts (both differences are exact in fp32)
+__device__ __forceinline__ void split3_store(float v, uint16_t* hi, uint16_t* mid, uint16_t* lo,
+                                             size_t i) {
+  const uint16_t h = bf16_bits(v);
+  const float r1 = v - bf16_val(h);
+  const uint16_t m = bf16_bits(r1);
+  hi[i] = h;
+  mid[i] = m;
+  lo[i] = bf16_bits(r1 - bf16_val(m));
 }
 
 // ------------------------------------------------------------------ GEMM
@@ -69,11 +83,12 @@ constexpr uint64_t kGWaitNs = 2000000000ull;  // 2 s: far beyond any legal wait
 template <int BN, int STAGES, bool HL = false>
 struct __align__(1024) GemmSmem {
   static constexpr int kTileB = BN * kGK * 2;
-  static constexpr int kBTiles = HL ? 1 : 2;
+  static constexpr int kBTiles = HL ? 1 : 3;
   static constexpr uint32_t kStageBytes = kGTileA + kBTiles * kTileB;
   static constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;
   uint8_t a[STAGES][kGTileA];
   uint8_t bh[STAGES][kTileB];
+  uint8_t bm[HL ? 1 : STAGES][HL ? 16 : kTileB];
   uint8_t bl[HL ? 1 : STAGES][HL ? 16 : kTileB];
   uint64_t full[STAGES];
   uint64_t empty[STAGES];
@@ -97,7 +112,8 @@ __device__ __forceinline__ bool gemm_wait(uint64_t* bar, uint32_t parity) {
 template <int BN, int STAGES, bool HL = false>
 __global__ void __launch_bounds__(128, 1)
     gemm_wx_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_xh,
-                   const __grid_constant__ CUtensorMap tm_xl, int n_rows, int n_tok, int K,
+                   const __grid_constant__ CUtensorMap tm_xm, const __grid_constant__ CUtensorMap tm_xl,
+                   int n_rows, int n_tok, int K,
                    float* __restrict__ Y, int ldy, size_t part_stride,
                    const uint16_t* __restrict__ bias, int32_t* __restrict__ err,
                    const float* __restrict__ tok_ss, int norm_len, float norm_eps,
@@ -143,7 +159,10 @@ __global__ void __launch_bounds__(128, 1)
     pdl_wait();
     for (int i = 0; i < pre; ++i) {
       tma_load_2d(s.bh[i], &tm_xh, (kb0 + i) * kGK, n0, &s.full[i]);
-      if constexpr (!HL) tma_load_2d(s.bl[i], &tm_xl, (kb0 + i) * kGK, n0, &s.full[i]);
+      if constexpr (!HL) {
+        tma_load_2d(s.bm[i], &tm_xm, (kb0 + i) * kGK, n0, &s.full[i]);
+        tma_load_2d(s.bl[i], &tm_xl, (kb0 + i) * kGK, n0, &s.full[i]);
+      }
     }
     int issued = pre;
     for (int i = pre; i < nk; ++i) {
@@ -156,7 +175,10 @@ __global__ void __launch_bounds__(128, 1)
       mbar_arrive_expect_tx(&s.full[st], S::kStageBytes);
       tma_load_2d(s.a[st], &tm_w, kc, m0, &s.full[st]);
       tma_load_2d(s.bh[st], &tm_xh, kc, n0, &s.full[st]);
-      if constexpr (!HL) tma_load_2d(s.bl[st], &tm_xl, kc, n0, &s.full[st]);
+      if constexpr (!HL) {
+        tma_load_2d(s.bm[st], &tm_xm, kc, n0, &s.full[st]);
+        tma_load_2d(s.bl[st], &tm_xl, kc, n0, &s.full[st]);
+      }
       issued = i + 1;
     }
     // every load must land before this CTA may exit
@@ -177,7 +199,10 @@ __global__ void __launch_bounds__(128, 1)
       for (int k = 0; k < kGK / 16; ++k) {
         // +2 in the address field = 32 bytes = 16 bf16 along K
         tc_mma_f16(tmem, da + 2 * k, dh + 2 * k, idesc, (i | k) != 0);
-        if constexpr (!HL) tc_mma_f16(tmem, da + 2 * k, sw128_kmajor_desc(s.bl[st]) + 2 * k, idesc, 1u);
+        if constexpr (!HL) {
+          tc_mma_f16(tmem, da + 2 * k, sw128_kmajor_desc(s.bm[st]) + 2 * k, idesc, 1u);
+          tc_mma_f16(tmem, da + 2 * k, sw128_kmajor_desc(s.bl[st]) + 2 * k, idesc, 1u);
+        }
       }
       tc_commit(&s.empty[st]);
     }
@@ -266,10 +291,10 @@ __global__ void embed_kernel(const uint16_t* __restrict__ E, const int32_t* __re
     x[(size_t)t * H + i] = bf16_val(E[(size_t)tok * H + i]);
 }
 
-// [xh, xl][t] = split(x[t] * w / sqrt(mean(x[t]^2) + eps))
+// [xh, xm, xl][t] = split3(x[t] * w / sqrt(mean(x[t]^2) + eps))
 __global__ void rmsnorm_split_kernel(const float* __restrict__ x, const uint16_t* __restrict__ w,
                                      int H, float eps, uint16_t* __restrict__ xh,
-                                     uint16_t* __restrict__ xl) {
+                                     uint16_t* __restrict__ xm, uint16_t* __restrict__ xl) {
   __shared__ float red[32];
   const int t = blockIdx.x;
   const float* xr = x + (size_t)t * H;
@@ -282,7 +307,7 @@ __global__ void rmsnorm_split_kernel(const float* __restrict__ x, const uint16_t
   for (int i = 0; i < (int)(blockDim.x >> 5); ++i) tot += red[i];
   const float r = 1.0f / sqrtf(tot / (float)H + eps);
   for (int i = threadIdx.x; i < H; i += blockDim.x)
-    split_store(xr[i] * r * bf16_val(w[i]), xh, xl, (size_t)t * H + i);
+    split3_store(xr[i] * r * bf16_val(w[i]), xh, xm, xl, (size_t)t * H + i);
 }
 
 // Sum of split-K partials p[z * pstride], z = 0 .. nparts - 1, added in split
@@ -335,8 +360,7 @@ __global__ void rope_kv_kernel(const float* __restrict__ y, int ldy, int nparts,
       q[dim1] = y1;
     } else {
       uint16_t* cache = which == 1 ? m.kcache : m.vcache;
-      const size_t off =
-          ((((size_t)sl * m.n_layers + layer) * m.n_kv + head) * (size_t)m.max_seq + p) * (size_t)d;
+      const size_t off = kv_row(m, sl, layer, head, p);
       cache[off + dim0] = bf16_bits(y0);
       cache[off + dim1] = bf16_bits(y1);
     }
@@ -354,7 +378,8 @@ constexpr int kPAKeys = 64;
 template <int DPL, int G>
 __global__ void __launch_bounds__(kPAWarps * 32, 1)
     prefill_attn_kernel(const float* __restrict__ q, const int32_t* __restrict__ tiles, ModelDev m,
-                        int layer, uint16_t* __restrict__ xh, uint16_t* __restrict__ xl) {
+                        int layer, uint16_t* __restrict__ xh, uint16_t* __restrict__ xm,
+                        uint16_t* __restrict__ xl) {
   constexpr int d = DPL * 32;
   extern __shared__ __align__(16) uint8_t pa_raw[];
   uint16_t* ks = reinterpret_cast<uint16_t*>(pa_raw);
@@ -370,18 +395,20 @@ __global__ void __launch_bounds__(kPAWarps * 32, 1)
   AttnState<DPL, G> st;
   if (mine) attn_init<DPL, G>(st, q + (size_t)(t0 + warp) * nq * d + (size_t)g * G * d, d,
                               m.attn_scale, lane);
-  const size_t head_off = (((size_t)sl * m.n_layers + layer) * m.n_kv + g) * (size_t)m.max_seq * d;
-  const uint16_t* K = m.kcache + head_off;
-  const uint16_t* V = m.vcache + head_off;
   const int n_keys = p0 + nt;  // keys 0 .. last position of the tile
   float* xb = xbs + warp * kAttnXbStride;
   for (int kb = 0; kb < n_keys; kb += kPAKeys) {
     const int nk = min(kPAKeys, n_keys - kb);
+    // a block of kPAKeys keys starting at a multiple of kPAKeys lies in one
+    // KV page (pages hold a multiple of 64 positions), so its rows are contiguous
+    const size_t off = kv_row(m, sl, layer, g, kb);
+    const uint16_t* K = m.kcache + off;
+    const uint16_t* V = m.vcache + off;
     __syncthreads();
     const int vec = nk * d / 8;  // 16-byte pieces
     for (int i = threadIdx.x; i < vec; i += blockDim.x) {
-      reinterpret_cast<uint4*>(ks)[i] = __ldcg(reinterpret_cast<const uint4*>(K + (size_t)kb * d) + i);
-      reinterpret_cast<uint4*>(vs)[i] = __ldcg(reinterpret_cast<const uint4*>(V + (size_t)kb * d) + i);
+      reinterpret_cast<uint4*>(ks)[i] = __ldcg(reinterpret_cast<const uint4*>(K) + i);
+      reinterpret_cast<uint4*>(vs)[i] = __ldcg(reinterpret_cast<const uint4*>(V) + i);
     }
     __syncthreads();
     if (!mine) continue;
@@ -417,7 +444,8 @@ __global__ void __launch_bounds__(kPAWarps * 32, 1)
   for (int h = 0; h < G; ++h) {
     const float inv = 1.0f / st.l[h];
 #pragma unroll
-    for (int i = 0; i < DPL; ++i) split_store(st.o[h][i] * inv, xh, xl, row + (size_t)h * d + lane * DPL + i);
+    for (int i = 0; i < DPL; ++i)
+      split3_store(st.o[h][i] * inv, xh, xm, xl, row + (size_t)h * d + lane * DPL + i);
   }
 }
 
@@ -430,15 +458,15 @@ __global__ void residual_kernel(float* __restrict__ x, const float* __restrict__
   }
 }
 
-// [xh, xl][t][j] = split(silu(gate_j) * up_j); gate/up interleaved in y.
+// [xh, xm, xl][t][j] = split3(silu(gate_j) * up_j); gate/up interleaved in y.
 __global__ void swiglu_split_kernel(const float* __restrict__ y, int ldy, int F, int nparts,
                                     size_t pstride, uint16_t* __restrict__ xh,
-                                    uint16_t* __restrict__ xl) {
+                                    uint16_t* __restrict__ xm, uint16_t* __restrict__ xl) {
   const int t = blockIdx.x;
   for (int j = threadIdx.x; j < F; j += blockDim.x) {
     const float g = sum_parts(y + (size_t)t * ldy + 2 * j, nparts, pstride);
     const float u = sum_parts(y + (size_t)t * ldy + 2 * j + 1, nparts, pstride);
-    split_store(g / (1.0f + expf(-g)) * u, xh, xl, (size_t)t * F + j);
+    split3_store(g / (1.0f + expf(-g)) * u, xh, xm, xl, (size_t)t * F + j);
   }
 }
 
@@ -505,13 +533,11 @@ __global__ void __launch_bounds__(kBAWarps * 32, 1)
   const int n_keys = bp->pos[r] + 1;
   const int live = batch_live_splits(n_keys, S, batch_keys_per_split(bp, m.n_kv, S, num_sms));
   if (sp >= live) return;
-  const int chunk = (n_keys + live - 1) / live;
+  // keys per split in whole blocks of kBAKeys: every block then lies in one KV
+  // page (a trailing split may hold no keys and contributes an empty partial)
+  const int chunk = ((n_keys + live - 1) / live + kBAKeys - 1) / kBAKeys * kBAKeys;
   const int k0 = min(n_keys, sp * chunk), k1 = min(n_keys, k0 + chunk);
-  const int nq = m.n_q;
-  const size_t head_off =
-      (((size_t)bp->slot[r] * m.n_layers + layer) * m.n_kv + g) * (size_t)m.max_seq * d;
-  const uint16_t* K = m.kcache + head_off;
-  const uint16_t* V = m.vcache + head_off;
+  const int nq = m.n_q, slot = bp->slot[r];
   AttnState<DPL, G> st;
   attn_init<DPL, G>(st, q + (size_t)r * nq * d + (size_t)g * G * d, d, m.attn_scale, lane);
   float* xb = xbs + warp * kAttnXbStride;
@@ -519,10 +545,13 @@ __global__ void __launch_bounds__(kBAWarps * 32, 1)
   auto issue = [&](int b) {
     const int kb = k0 + b * kBAKeys, nk = min(kBAKeys, k1 - kb);
     uint16_t* dst = buf + (b % kBAStages) * kBuf;
+    const size_t off = kv_row(m, slot, layer, g, kb);
+    const uint16_t* K = m.kcache + off;
+    const uint16_t* V = m.vcache + off;
     const int pieces = nk * d / 8;  // 16-byte pieces of K (and of V)
     for (int i = threadIdx.x; i < pieces; i += blockDim.x) {
-      cp_async16(dst + i * 8, K + (size_t)kb * d + i * 8);
-      cp_async16(dst + kBAKeys * d + i * 8, V + (size_t)kb * d + i * 8);
+      cp_async16(dst + i * 8, K + i * 8);
+      cp_async16(dst + kBAKeys * d + i * 8, V + i * 8);
     }
   };
   // blocks 0 .. kBAStages - 2 in flight before the loop; block b + kBAStages - 1
@@ -819,31 +848,31 @@ bool make_map(CUtensorMap* map, const void* base, int rows, int cols, int box_ro
 
 // Y (+ z * n_tok * ldy for split z) = W x^T over `splits` K ranges.
 template <int BN, int STAGES>
-std::string gemm(const uint16_t* W, int n_rows, int K, const uint16_t* xh, const uint16_t* xl,
-                 int n_tok, float* Y, int ldy, const uint16_t* bias, int32_t* err, cudaStream_t st,
-                 int splits = 1, const float* tok_ss = nullptr, float norm_eps = 0.f,
-                 bool pdl = false) {
-  CUtensorMap mw, mh, ml;
+std::string gemm(const uint16_t* W, int n_rows, int K, const uint16_t* xh, const uint16_t* xm,
+                 const uint16_t* xl, int n_tok, float* Y, int ldy, const uint16_t* bias,
+                 int32_t* err, cudaStream_t st, int splits = 1, const float* tok_ss = nullptr,
+                 float norm_eps = 0.f, bool pdl = false) {
+  CUtensorMap mw, mh, mm, ml;
   if (!make_map(&mw, W, n_rows, K) || !make_map(&mh, xh, n_tok, K, BN) ||
-      !make_map(&ml, xl, n_tok, K, BN))
+      !make_map(&mm, xm, n_tok, K, BN) || !make_map(&ml, xl, n_tok, K, BN))
     return "cuTensorMapEncodeTiled failed";
   const dim3 grid((n_rows + kGM - 1) / kGM, (n_tok + BN - 1) / BN, splits);
   const uint16_t* b = splits == 1 ? bias : nullptr;
   const size_t pst = (size_t)n_tok * ldy;
   if (pdl) {
     const cudaError_t le = launch_pdl(gemm_wx_kernel<BN, STAGES>, grid, dim3(128),
-                                      gemm_smem_bytes<BN, STAGES>(), st, mw, mh, ml, n_rows, n_tok, K,
+                                      gemm_smem_bytes<BN, STAGES>(), st, mw, mh, mm, ml, n_rows, n_tok, K,
                                       Y, ldy, pst, b, err, tok_ss, K, norm_eps, (uint16_t*)nullptr, 0);
     if (le != cudaSuccess) return std::string("GEMM launch: ") + cudaGetErrorString(le);
   } else {
     gemm_wx_kernel<BN, STAGES><<<grid, 128, gemm_smem_bytes<BN, STAGES>(), st>>>(
-        mw, mh, ml, n_rows, n_tok, K, Y, ldy, pst, b, err, tok_ss, K, norm_eps, nullptr, 0);
+        mw, mh, mm, ml, n_rows, n_tok, K, Y, ldy, pst, b, err, tok_ss, K, norm_eps, nullptr, 0);
   }
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? "" : std::string("GEMM launch: ") + cudaGetErrorString(e);
 }
 
-constexpr int kPBN = 128, kPStages = 4;   // prompt GEMM: 128 tokens per CTA
+constexpr int kPBN = 128, kPStages = 3;   // prompt GEMM: 128 tokens per CTA, 64 KB per stage
 constexpr int kDStages = 11;              // decode GEMM: 8 requests, high and low parts packed
 
 // Y (+ z * n_tok * ldy for split z) = W x^T for n_tok <= 8 tokens whose high
@@ -864,11 +893,11 @@ std::string gemm_hl(const uint16_t* W, int n_rows, int K, const uint16_t* xhl, i
   const cudaError_t le =
       two_per_sm
           ? launch_pdl(gemm_wx_kernel<16, kDStagesPair, true>, grid, dim3(128),
-                       gemm_smem_bytes<16, kDStagesPair, true>(), st, mw, mh, mh, n_rows, n_tok, K, Y,
+                       gemm_smem_bytes<16, kDStagesPair, true>(), st, mw, mh, mh, mh, n_rows, n_tok, K, Y,
                        ldy, (size_t)n_tok * ldy, (const uint16_t*)nullptr, err, tok_ss, K, norm_eps,
                        act_hl, n_rows / 2)
           : launch_pdl(gemm_wx_kernel<16, kDStages, true>, grid, dim3(128),
-                       gemm_smem_bytes<16, kDStages, true>(), st, mw, mh, mh, n_rows, n_tok, K, Y,
+                       gemm_smem_bytes<16, kDStages, true>(), st, mw, mh, mh, mh, n_rows, n_tok, K, Y,
                        ldy, (size_t)n_tok * ldy, (const uint16_t*)nullptr, err, tok_ss, K, norm_eps,
                        act_hl, n_rows / 2);
   return le == cudaSuccess ? "" : std::string("GEMM launch: ") + cudaGetErrorString(le);
@@ -876,28 +905,28 @@ std::string gemm_hl(const uint16_t* W, int n_rows, int K, const uint16_t* xhl, i
 
 template <int DPL, int G>
 std::string launch_attn(dim3 grid, cudaStream_t st, const float* q, const int32_t* tiles,
-                        const ModelDev& m, int layer, uint16_t* xh, uint16_t* xl) {
+                        const ModelDev& m, int layer, uint16_t* xh, uint16_t* xm, uint16_t* xl) {
   const size_t smem = (size_t)2 * kPAKeys * DPL * 32 * 2 + (size_t)kPAWarps * kAttnXbStride * 4;
   auto k = prefill_attn_kernel<DPL, G>;
   cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  k<<<grid, kPAWarps * 32, smem, st>>>(q, tiles, m, layer, xh, xl);
+  k<<<grid, kPAWarps * 32, smem, st>>>(q, tiles, m, layer, xh, xm, xl);
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? "" : std::string("attention launch: ") + cudaGetErrorString(e);
 }
 
 std::string attn(dim3 grid, cudaStream_t st, const float* q, const int32_t* tiles, const ModelDev& m,
-                 int layer, uint16_t* xh, uint16_t* xl) {
+                 int layer, uint16_t* xh, uint16_t* xm, uint16_t* xl) {
   const int G = m.group;
   if (m.head_dim == 128) {
-    if (G == 1) return launch_attn<4, 1>(grid, st, q, tiles, m, layer, xh, xl);
-    if (G == 2) return launch_attn<4, 2>(grid, st, q, tiles, m, layer, xh, xl);
-    if (G == 4) return launch_attn<4, 4>(grid, st, q, tiles, m, layer, xh, xl);
+    if (G == 1) return launch_attn<4, 1>(grid, st, q, tiles, m, layer, xh, xm, xl);
+    if (G == 2) return launch_attn<4, 2>(grid, st, q, tiles, m, layer, xh, xm, xl);
+    if (G == 4) return launch_attn<4, 4>(grid, st, q, tiles, m, layer, xh, xm, xl);
   } else {
-    if (G == 1) return launch_attn<2, 1>(grid, st, q, tiles, m, layer, xh, xl);
-    if (G == 2) return launch_attn<2, 2>(grid, st, q, tiles, m, layer, xh, xl);
-    if (G == 4) return launch_attn<2, 4>(grid, st, q, tiles, m, layer, xh, xl);
-    if (G == 7) return launch_attn<2, 7>(grid, st, q, tiles, m, layer, xh, xl);
-    if (G == 8) return launch_attn<2, 8>(grid, st, q, tiles, m, layer, xh, xl);
+    if (G == 1) return launch_attn<2, 1>(grid, st, q, tiles, m, layer, xh, xm, xl);
+    if (G == 2) return launch_attn<2, 2>(grid, st, q, tiles, m, layer, xh, xm, xl);
+    if (G == 4) return launch_attn<2, 4>(grid, st, q, tiles, m, layer, xh, xm, xl);
+    if (G == 7) return launch_attn<2, 7>(grid, st, q, tiles, m, layer, xh, xm, xl);
+    if (G == 8) return launch_attn<2, 8>(grid, st, q, tiles, m, layer, xh, xm, xl);
   }
   return "unsupported query heads per KV head";
 }
@@ -919,7 +948,8 @@ std::string prefill_alloc(const ModelDev& m, int max_tokens, PrefillScratch* sc,
   struct A { void** p; size_t bytes; } allocs[] = {
       {(void**)&sc->x, T * H * 4},          {(void**)&sc->y, T * ycols * 4},
       {(void**)&sc->q, T * qd * 4},         {(void**)&sc->xh, T * xcols * 2},
-      {(void**)&sc->xl, T * xcols * 2},     {(void**)&sc->meta, (3 * T + 4 * T + 16) * 4},
+      {(void**)&sc->xl, T * xcols * 2},     {(void**)&sc->xm, T * xcols * 2},
+      {(void**)&sc->meta, (3 * T + 4 * T + 16) * 4},
       {(void**)&sc->err, 16}};
   for (auto& a : allocs) {
     const cudaError_t e = cudaMalloc(a.p, a.bytes);
@@ -936,7 +966,7 @@ std::string prefill_alloc(const ModelDev& m, int max_tokens, PrefillScratch* sc,
 
 std::string prefill_run(const ModelDev& m, const PrefillWeights& w, PrefillScratch& sc,
                         cudaStream_t st, const int32_t* tokens_dev, const int32_t* offsets_host,
-                        int n_req) {
+                        const int32_t* slots_host, int n_req) {
   const int H = m.hidden, F = m.ffn, d = m.head_dim, qd = m.n_q * d, L = m.n_layers;
   const int qkvR = qkv_rows(m.n_q, m.n_kv, d);
   const int ldy = std::max(std::max(qkvR, 2 * F), H);
@@ -945,7 +975,7 @@ std::string prefill_run(const ModelDev& m, const PrefillWeights& w, PrefillScrat
   for (int r = 0; r < n_req; ++r)
     for (int p = 0; p + 1 < offsets_host[r + 1] - offsets_host[r]; ++p) {
       tok_src.push_back(offsets_host[r] + p);
-      slot.push_back(r);
+      slot.push_back(slots_host[r]);
       pos.push_back(p);
     }
   const int total = (int)tok_src.size();
@@ -976,17 +1006,17 @@ std::string prefill_run(const ModelDev& m, const PrefillWeights& w, PrefillScrat
       return "prefill metadata upload";
     embed_kernel<<<T, 256, 0, st>>>(m.embed, tokens_dev, d_src, H, m.vocab, sc.x, m.status);
     for (int l = 0; l < L; ++l) {
-      rmsnorm_split_kernel<<<T, 256, 0, st>>>(sc.x, m.attn_norm + (size_t)l * H, H, m.rms_eps, sc.xh, sc.xl);
+      rmsnorm_split_kernel<<<T, 256, 0, st>>>(sc.x, m.attn_norm + (size_t)l * H, H, m.rms_eps, sc.xh, sc.xm, sc.xl);
       const uint16_t* bias = m.qkv_bias ? m.bqkv + (size_t)l * qkvR : nullptr;
-      if (!(e = gemm<kPBN, kPStages>(w.qkv[l], qkvR, H, sc.xh, sc.xl, T, sc.y, ldy, bias, sc.err, st)).empty()) return e;
+      if (!(e = gemm<kPBN, kPStages>(w.qkv[l], qkvR, H, sc.xh, sc.xm, sc.xl, T, sc.y, ldy, bias, sc.err, st)).empty()) return e;
       rope_kv_kernel<<<T, 256, 0, st>>>(sc.y, ldy, 1, 0, nullptr, d_slot, d_pos, m, l, sc.q);
-      if (!(e = attn(dim3(ntiles, m.n_kv), st, sc.q, d_tiles, m, l, sc.xh, sc.xl)).empty()) return e;
-      if (!(e = gemm<kPBN, kPStages>(w.o[l], H, qd, sc.xh, sc.xl, T, sc.y, ldy, nullptr, sc.err, st)).empty()) return e;
+      if (!(e = attn(dim3(ntiles, m.n_kv), st, sc.q, d_tiles, m, l, sc.xh, sc.xm, sc.xl)).empty()) return e;
+      if (!(e = gemm<kPBN, kPStages>(w.o[l], H, qd, sc.xh, sc.xm, sc.xl, T, sc.y, ldy, nullptr, sc.err, st)).empty()) return e;
       residual_kernel<<<T, 256, 0, st>>>(sc.x, sc.y, H, ldy, 1, 0);
-      rmsnorm_split_kernel<<<T, 256, 0, st>>>(sc.x, m.ffn_norm + (size_t)l * H, H, m.rms_eps, sc.xh, sc.xl);
-      if (!(e = gemm<kPBN, kPStages>(w.gu[l], 2 * F, H, sc.xh, sc.xl, T, sc.y, ldy, nullptr, sc.err, st)).empty()) return e;
-      swiglu_split_kernel<<<T, 256, 0, st>>>(sc.y, ldy, F, 1, 0, sc.xh, sc.xl);
-      if (!(e = gemm<kPBN, kPStages>(w.dn[l], H, F, sc.xh, sc.xl, T, sc.y, ldy, nullptr, sc.err, st)).empty()) return e;
+      rmsnorm_split_kernel<<<T, 256, 0, st>>>(sc.x, m.ffn_norm + (size_t)l * H, H, m.rms_eps, sc.xh, sc.xm, sc.xl);
+      if (!(e = gemm<kPBN, kPStages>(w.gu[l], 2 * F, H, sc.xh, sc.xm, sc.xl, T, sc.y, ldy, nullptr, sc.err, st)).empty()) return e;
+      swiglu_split_kernel<<<T, 256, 0, st>>>(sc.y, ldy, F, 1, 0, sc.xh, sc.xm, sc.xl);
+      if (!(e = gemm<kPBN, kPStages>(w.dn[l], H, F, sc.xh, sc.xm, sc.xl, T, sc.y, ldy, nullptr, sc.err, st)).empty()) return e;
       residual_kernel<<<T, 256, 0, st>>>(sc.x, sc.y, H, ldy, 1, 0);
     }
     const cudaError_t ce = cudaGetLastError();

@@ -2,7 +2,7 @@
 //
 // Positions [0, len-1) of every prompt run as whole-sequence operators: the
 // five weight contractions of a layer as tcgen05 GEMMs (bf16 weights, fp32
-// activations split into a bf16 high and low part, fp32 accumulation),
+// activations split into three bf16 parts, fp32 accumulation),
 // RMSNorm / RoPE / KV append / SwiGLU / residual as small kernels, and causal
 // GQA attention over the cache.  The last prompt position then runs through
 // the decode step, which produces its logits and greedy id.
@@ -28,6 +28,7 @@ struct PrefillScratch {
   float* y = nullptr;          // [T][max(qkv rows, 2 ffn, hidden)] GEMM output
   float* q = nullptr;          // [T][n_q * d] rotated queries
   uint16_t* xh = nullptr;      // [T][max(hidden, ffn, n_q*d)] GEMM input, bf16 high part
+  uint16_t* xm = nullptr;      //   ... middle part
   uint16_t* xl = nullptr;      //   ... and low part
   int32_t* meta = nullptr;     // per-token and per-tile arrays (see prefill.cu)
   int32_t* err = nullptr;      // device error word of the GEMM kernel
@@ -73,10 +74,11 @@ std::string prefill_alloc(const ModelDev& m, int max_tokens, PrefillScratch* sc,
                           std::vector<void*>* owned);
 
 // Runs positions [0, len_r - 1) of each request r (tokens_dev packed with
-// offsets_host) through the layers, filling the KV cache.  Enqueued on `st`.
+// offsets_host) through the layers, filling the KV cache of request slot
+// slots_host[r].  Enqueued on `st`.
 std::string prefill_run(const ModelDev& m, const PrefillWeights& w, PrefillScratch& sc,
                         cudaStream_t st, const int32_t* tokens_dev, const int32_t* offsets_host,
-                        int n_req);
+                        const int32_t* slots_host, int n_req);
 
 // Allocates the batched decode scratch (cudaMalloc).
 std::string batch_alloc(const ModelDev& m, int num_sms, BatchScratch* bs, std::vector<void*>* owned);
