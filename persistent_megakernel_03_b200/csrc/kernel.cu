@@ -293,9 +293,12 @@ struct ChunkCursor {
   }
 };
 
-// Streams every chunk of the CTA's queue into the ring, in the workers'
-// consumption order, as fast as slots free up.
-__device__ __forceinline__ void producer(const KernelArgs& a, Smem& s, int q0, int q1) {
+// Streams the chunks of the CTA's queue into the ring, in the workers'
+// consumption order, as fast as slots free up.  Producer `pid` of
+// kProducerWarps issues chunks seq with seq % kProducerWarps == pid (every
+// producer walks the whole chunk list; a slot is always filled by the same
+// producer, and each waits only for its own slots to be released).
+__device__ __forceinline__ void producer(const KernelArgs& a, Smem& s, int q0, int q1, int pid) {
   const ModelDev& m = a.m;
   const uint64_t pol_w = l2_policy_evict_first();
   const uint64_t pol_keep = l2_policy_evict_normal();
@@ -322,11 +325,13 @@ __device__ __forceinline__ void producer(const KernelArgs& a, Smem& s, int q0, i
         fence_proxy_async_global();
         kv_ready = true;
       }
-      if (!producer_acquire_slot(s, seq, m)) { stop = true; break; }
-      const int slot = seq % kRingSlots;
-      mbar_arrive_expect_tx(&s.full[slot], c.bytes0 + c.bytes1);
-      bulk_g2s(s.ring[slot], c.src0, c.bytes0, &s.full[slot], c.kv ? pol_keep : pol_w);
-      if (c.src1) bulk_g2s(s.ring[slot] + kSlotBytes / 2, c.src1, c.bytes1, &s.full[slot], pol_keep);
+      if ((int)(seq % kProducerWarps) == pid) {
+        if (!producer_acquire_slot(s, seq, m)) { stop = true; break; }
+        const int slot = seq % kRingSlots;
+        mbar_arrive_expect_tx(&s.full[slot], c.bytes0 + c.bytes1);
+        bulk_g2s(s.ring[slot], c.src0, c.bytes0, &s.full[slot], c.kv ? pol_keep : pol_w);
+        if (c.src1) bulk_g2s(s.ring[slot] + kSlotBytes / 2, c.src1, c.bytes1, &s.full[slot], pol_keep);
+      }
       ++seq;
     }
   }
@@ -340,6 +345,7 @@ __device__ __forceinline__ void producer(const KernelArgs& a, Smem& s, int q0, i
   // poisons the context on the host so it is never used again.
   const uint32_t first = seq > kRingSlots ? seq - kRingSlots : 0;
   for (uint32_t q = first; q < seq; ++q) {
+    if ((int)(q % kProducerWarps) != pid) continue;  // the other producer's copy
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait(&s.full[q % kRingSlots], (q / kRingSlots) & 1u)) {
       if (globaltimer_ns() - t0 > 200000000ull) {
@@ -1171,8 +1177,8 @@ __global__ void __launch_bounds__(kThreads, 1) mk_step_kernel(const __grid_const
   }
   __syncthreads();
   if (q0 == q1) return;
-  if (warp == kProducerWarp) {
-    if (lane == 0) producer(a, s, q0, q1);
+  if (warp < kProducerWarps) {
+    if (lane == 0) producer(a, s, q0, q1, warp);
   } else if (warp == kSchedulerWarp) {
     if (lane == 0) scheduler(a, s, q0, q1);
   } else {

@@ -24,12 +24,18 @@ enum TaskKind : int32_t { T_QKV = 0, T_ATTN = 1, T_OPROJ = 2, T_GATEUP = 3, T_DO
 constexpr int kMaxBatch = 8;
 constexpr int kWorkerWarps = 16;                  // compute warps per CTA
 constexpr int kWorkerThreads = kWorkerWarps * 32; // 512
-constexpr int kProducerWarp = 0;                  // bulk-copy (TMA) issue
-constexpr int kSchedulerWarp = 1;                 // event waits
-constexpr int kFirstWorkerWarp = 2;
-constexpr int kThreads = (kFirstWorkerWarp + kWorkerWarps) * 32; // 576
+// Bulk copies issued by one thread run one after another (each ~0.4 us
+// whatever its size up to 32 KB, measured), which caps a single issuer at
+// ~70-80 GB/s per SM -- barely above an SM's share of HBM.  Copies from
+// different issuing warps overlap, so the ring is filled by two producer
+// warps, each owning every other chunk (and so every other slot).
+constexpr int kProducerWarps = 2;                 // bulk-copy (TMA) issue, warps 0 .. 1
+constexpr int kSchedulerWarp = kProducerWarps;    // event waits
+constexpr int kFirstWorkerWarp = kProducerWarps + 1;
+constexpr int kThreads = (kFirstWorkerWarp + kWorkerWarps) * 32; // 608
 constexpr int kSlotBytes = 32768;                 // one weight-ring stage
 constexpr int kRingSlots = 6;                     // 192 KB of weights in flight / buffered
+static_assert(kRingSlots % 2 == 0, "each producer warp owns every other slot");
 constexpr int kScratchBytes = 20480;              // GEMV partial sums / attention merge
 constexpr int kYBufFloats = 1024;                 // reduced GEMV outputs of one task
 constexpr int kMaxTaskRowsCap = 1024;

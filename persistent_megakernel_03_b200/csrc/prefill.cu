@@ -85,7 +85,12 @@ struct __align__(1024) GemmSmem {
   static constexpr int kTileB = BN * kGK * 2;
   static constexpr int kBTiles = HL ? 1 : 3;
   static constexpr uint32_t kStageBytes = kGTileA + kBTiles * kTileB;
-  static constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;
+  // accumulators: one (HL), or three -- the high part's even and odd K blocks
+  // and the middle + low parts -- so no single fp32 accumulator takes every
+  // MMA of the contraction; the epilogue adds them
+  static constexpr int kAcc = HL ? 1 : 3;
+  static constexpr uint32_t kTmemCols = kAcc * BN <= 32 ? 32 : kAcc * BN <= 64 ? 64
+                                      : kAcc * BN <= 128 ? 128 : kAcc * BN <= 256 ? 256 : 512;
   uint8_t a[STAGES][kGTileA];
   uint8_t bh[STAGES][kTileB];
   uint8_t bm[HL ? 1 : STAGES][HL ? 16 : kTileB];
@@ -148,24 +153,32 @@ __global__ void __launch_bounds__(128, 1)
   tc_fence_after_sync();
   const uint32_t tmem = s.tmem;
   pdl_trigger();
-  if (warp == 0 && lane == 0) {
-    // The weight tiles of the first STAGES stages do not depend on the
-    // previous kernel: they are requested before waiting for it.
-    const int pre = nk < STAGES ? nk : STAGES;
-    for (int i = 0; i < pre; ++i) {
-      mbar_arrive_expect_tx(&s.full[i], S::kStageBytes);
-      tma_load_2d(s.a[i], &tm_w, (kb0 + i) * kGK, m0, &s.full[i]);
-    }
-    pdl_wait();
-    for (int i = 0; i < pre; ++i) {
-      tma_load_2d(s.bh[i], &tm_xh, (kb0 + i) * kGK, n0, &s.full[i]);
-      if constexpr (!HL) {
-        tma_load_2d(s.bm[i], &tm_xm, (kb0 + i) * kGK, n0, &s.full[i]);
-        tma_load_2d(s.bl[i], &tm_xl, (kb0 + i) * kGK, n0, &s.full[i]);
+  // TMA loads issued by one thread run one after another, so two producer
+  // threads (lane 0 of warps 0 and 2) issue the stages past the first ring's
+  // worth alternately; warp 0 alone issues the first STAGES stages.
+  const int pre = nk < STAGES ? nk : STAGES;
+  if ((warp == 0 || warp == 2) && lane == 0) {
+    const int pid = warp >> 1;
+    if (pid == 0) {
+      // The weight tiles of the first STAGES stages do not depend on the
+      // previous kernel: they are requested before waiting for it.
+      for (int i = 0; i < pre; ++i) {
+        mbar_arrive_expect_tx(&s.full[i], S::kStageBytes);
+        tma_load_2d(s.a[i], &tm_w, (kb0 + i) * kGK, m0, &s.full[i]);
       }
     }
-    int issued = pre;
-    for (int i = pre; i < nk; ++i) {
+    pdl_wait();
+    if (pid == 0) {
+      for (int i = 0; i < pre; ++i) {
+        tma_load_2d(s.bh[i], &tm_xh, (kb0 + i) * kGK, n0, &s.full[i]);
+        if constexpr (!HL) {
+          tma_load_2d(s.bm[i], &tm_xm, (kb0 + i) * kGK, n0, &s.full[i]);
+          tma_load_2d(s.bl[i], &tm_xl, (kb0 + i) * kGK, n0, &s.full[i]);
+        }
+      }
+    }
+    int issued = pid == 0 ? pre : 0;  // one past this producer's last issued stage
+    for (int i = pre + pid; i < nk; i += 2) {
       const int st = i % STAGES;
       if (!gemm_wait(&s.empty[st], ((i / STAGES) - 1) & 1)) {
         s.failed = 1;
@@ -181,9 +194,12 @@ __global__ void __launch_bounds__(128, 1)
       }
       issued = i + 1;
     }
-    // every load must land before this CTA may exit
-    for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
-      gemm_wait(&s.full[i % STAGES], (i / STAGES) & 1);
+    // every load this thread issued must land before the CTA may exit (the
+    // last STAGES stages are the only ones that can still be in flight)
+    for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i) {
+      const bool mine = i < pre ? pid == 0 : ((i - pre) & 1) == pid;
+      if (mine) gemm_wait(&s.full[i % STAGES], (i / STAGES) & 1);
+    }
   } else if (warp == 1 && lane == 0) {
     constexpr uint32_t idesc = mma_idesc_bf16_f32(kGM, BN);
     for (int i = 0; i < nk; ++i) {
@@ -198,10 +214,14 @@ __global__ void __launch_bounds__(128, 1)
 #pragma unroll
       for (int k = 0; k < kGK / 16; ++k) {
         // +2 in the address field = 32 bytes = 16 bf16 along K
-        tc_mma_f16(tmem, da + 2 * k, dh + 2 * k, idesc, (i | k) != 0);
-        if constexpr (!HL) {
-          tc_mma_f16(tmem, da + 2 * k, sw128_kmajor_desc(s.bm[st]) + 2 * k, idesc, 1u);
-          tc_mma_f16(tmem, da + 2 * k, sw128_kmajor_desc(s.bl[st]) + 2 * k, idesc, 1u);
+        if constexpr (HL) {
+          tc_mma_f16(tmem, da + 2 * k, dh + 2 * k, idesc, (i | k) != 0);
+        } else {
+          const uint32_t acc_h = tmem + ((i & 1) ? 2u * BN : 0u);
+          const uint32_t acc_ml = tmem + (uint32_t)BN;
+          tc_mma_f16(acc_h, da + 2 * k, dh + 2 * k, idesc, (i > 1 || k > 0) ? 1u : 0u);
+          tc_mma_f16(acc_ml, da + 2 * k, sw128_kmajor_desc(s.bm[st]) + 2 * k, idesc, (i | k) != 0);
+          tc_mma_f16(acc_ml, da + 2 * k, sw128_kmajor_desc(s.bl[st]) + 2 * k, idesc, 1u);
         }
       }
       tc_commit(&s.empty[st]);
@@ -246,10 +266,16 @@ __global__ void __launch_bounds__(128, 1)
         }
       }
     } else {
+      const bool odd_blocks = nk > 1;  // the second high-part accumulator was written
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 16) {
-        float v[16];
-        tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
+        float v[16], ml[16], v2[16];
+        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0;
+        tmem_ld16(lane_base, v);
+        tmem_ld16(lane_base + (uint32_t)BN, ml);
+        if (odd_blocks) tmem_ld16(lane_base + 2u * BN, v2);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = (v[j] + (odd_blocks ? v2[j] : 0.f)) + ml[j];
         if (row < n_rows) {
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
