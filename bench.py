@@ -242,7 +242,8 @@ def load_traffic(workload):
     with open(p) as f:
         rec = json.load(f)
     h = hashlib.sha256()
-    for name in ("kernel.cu", "mk_internal.h", "ptx.cuh", "attn_math.cuh"):
+    for name in ("step_kernel.cuh", "step_bf16_d128.cu", "mk_internal.h", "ptx.cuh",
+                 "attn_math.cuh"):
         with open(os.path.join(ROOT, "persistent_megakernel_03_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     if rec.get("source_sha256") != h.hexdigest() or rec.get("workload") != workload:

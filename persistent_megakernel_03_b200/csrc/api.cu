@@ -16,7 +16,7 @@
 
 namespace mk {
 size_t step_kernel_smem_bytes();
-const void* step_kernel_ptr(int wbytes);
+const void* step_kernel_ptr(int wbytes, int head_dim, int G);
 cudaError_t launch_quantize_fp8_rows(uint16_t* w, uint8_t* codes, float* scales, int rows, int K,
                                      cudaStream_t st);
 cudaError_t launch_pack_qkv(uint16_t*, const uint16_t*, const uint16_t*, const uint16_t*, int, int,
@@ -241,9 +241,14 @@ extern "C" int mk_create(const mk_config* cfg, const mk_weights* w, const mk_opt
     ctx->err = "fp8 weights need hidden, ffn and n_q_heads * head_dim multiples of 16";
     return bail(MK_ERR_UNSUPPORTED);
   }
-  CKC(cudaFuncSetAttribute(step_kernel_ptr(wbytes), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  const void* step_k = step_kernel_ptr(wbytes, cfg->head_dim, G);
+  if (!step_k) {
+    ctx->err = "no step kernel for this head_dim and query heads per KV head";
+    return bail(MK_ERR_UNSUPPORTED);
+  }
+  CKC(cudaFuncSetAttribute(step_k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   int per_sm = 0;
-  CKC(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, step_kernel_ptr(wbytes), kThreads, smem));
+  CKC(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, step_k, kThreads, smem));
   if (per_sm < 1) {
     ctx->err = "one CTA of the step kernel does not fit on an SM";
     return bail(MK_ERR_NOT_RESIDENT);

@@ -254,6 +254,16 @@ std::string build_plan(const mk_config& c, int num_ctas, int attn_splits, Plan* 
   if (wbytes != 1 && wbytes != 2) return "wbytes must be 1 or 2";
   Builder b(c, num_ctas, *out, wbytes);
   b.build(S);
+  // every GEMV task must have a geometry the kernel instantiates: (pieces per
+  // thread, rows per chunk) = (1, 4), (2, 2), (3, 1) or (4, 1) (fp8: the first two)
+  for (const Task& t : out->tasks) {
+    if (t.kind == T_ATTN) continue;
+    const int pieces = t.K * wbytes / 16;
+    const int cpt = (pieces + t.tpr - 1) / t.tpr, nr = t.chunk_rows / (kWorkerThreads / t.tpr);
+    const bool ok = (cpt == 1 && nr == 4) || (cpt == 2 && nr == 2) ||
+                    (wbytes == 2 && ((cpt == 3 && nr == 1) || (cpt == 4 && nr == 1)));
+    if (!ok) return "internal: a GEMV geometry the kernel does not implement";
+  }
   return "";
 }
 
