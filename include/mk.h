@@ -129,6 +129,14 @@ typedef struct {
                          pool by mk_kv_release */
   int kv_pool_pages; /* paged cache: pages in the pool (0: enough for every slot at
                         max_seq, i.e. max_batch * ceil(max_seq / kv_page_tokens)) */
+  int prefill_megakernel; /* tensor-core prefill only.  1: each block of <= 2048
+                             prompt positions runs as ONE persistent kernel (every
+                             operator of every layer a task; tasks of different
+                             128-position tiles overlap across operator and layer
+                             boundaries, dependencies per tile through event
+                             counters; the GEMMs as tcgen05 tiles); 0: default, one
+                             launch per operator and layer.  Both give the same
+                             result up to the order of the fp32 additions. */
 } mk_options;
 
 typedef struct mk_ctx mk_ctx;

@@ -66,7 +66,8 @@ class Options(C.Structure):
     _fields_ = [("num_ctas", C.c_int), ("attn_splits", C.c_int), ("timeout_ms", C.c_int),
                 ("mode", C.c_int), ("l2_prefetch", C.c_int), ("weight_format", C.c_int),
                 ("batch_sequential", C.c_int), ("prefill_steps", C.c_int),
-                ("kv_page_tokens", C.c_int), ("kv_pool_pages", C.c_int)]
+                ("kv_page_tokens", C.c_int), ("kv_pool_pages", C.c_int),
+                ("prefill_megakernel", C.c_int)]
 
 
 class PlanInfo(C.Structure):
@@ -168,7 +169,7 @@ class Plan:
         L = lib()
         self.h = C.c_void_p()
         cfg = make_config(model, max_seq, max_batch)
-        opt = Options(num_ctas, attn_splits, 0, 0, 0, weight_format, 0, 0, 0, 0)
+        opt = Options(num_ctas, attn_splits, 0, 0, 0, weight_format, 0, 0, 0, 0, 0)
         rc = L.mk_plan_build(C.byref(cfg), C.byref(opt), int(num_ctas), C.byref(self.h))
         if rc != MK_OK:
             raise MkError(rc, "mk_plan_build rejected the configuration")
@@ -217,7 +218,8 @@ class Decoder:
                  max_batch: int = 1, num_ctas: int = 0, attn_splits: int = 0,
                  timeout_ms: int = 0, mode: int = MODE_MEGAKERNEL, stream=None,
                  l2_prefetch: int = 0, prefill_steps: int = 0, batch_sequential: int = 0,
-                 weight_format: int = 0, kv_page_tokens: int = 0, kv_pool_pages: int = 0):
+                 weight_format: int = 0, kv_page_tokens: int = 0, kv_pool_pages: int = 0,
+                 prefill_megakernel: int = 0):
         import torch
         L = lib()
         self.model = model
@@ -240,7 +242,8 @@ class Decoder:
                     None if model.tied_embeddings else ptr("lm_head"))
         cfg = make_config(model, max_seq, max_batch)
         opt = Options(num_ctas, attn_splits, timeout_ms, mode, l2_prefetch, weight_format,
-                      batch_sequential, prefill_steps, kv_page_tokens, kv_pool_pages)
+                      batch_sequential, prefill_steps, kv_page_tokens, kv_pool_pages,
+                      prefill_megakernel)
         self.h = C.c_void_p()
         rc = L.mk_create(C.byref(cfg), C.byref(w), C.byref(opt), self.stream.cuda_stream,
                          C.byref(self.h))

@@ -715,8 +715,12 @@ static int prefill_impl(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t* o
       const std::string e = prefill_alloc(ctx->md, std::max(cap, 1), &ctx->ps, &ctx->allocs);
       if (!e.empty()) return fail(ctx, MK_ERR_CUDA, e);
     }
-    const std::string e = prefill_run(ctx->md, ctx->pw, ctx->ps, ctx->stream, tokens_dev,
-                                      offsets_host, slots, n_req);
+    const std::string e =
+        ctx->opt.prefill_megakernel > 0
+            ? prefill_mk_run(ctx->md, ctx->pw, ctx->ps, ctx->stream, tokens_dev, offsets_host, slots,
+                             n_req, ctx->plan.num_ctas, &ctx->allocs)
+            : prefill_run(ctx->md, ctx->pw, ctx->ps, ctx->stream, tokens_dev, offsets_host, slots,
+                          n_req);
     if (!e.empty()) {
       ctx->poisoned = true;
       return fail(ctx, MK_ERR_CUDA, e);

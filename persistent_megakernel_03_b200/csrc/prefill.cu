@@ -959,6 +959,8 @@ std::string attn(dim3 grid, cudaStream_t st, const float* q, const int32_t* tile
 
 }  // namespace
 
+PFN_cuTensorMapEncodeTiled_v12000 prefill_encode_fn() { return encode_fn(); }
+
 bool prefill_gemm_supported(const ModelDev& m) {
   const int qd = m.n_q * m.head_dim;
   return m.hidden % kGK == 0 && m.ffn % kGK == 0 && qd % kGK == 0 && encode_fn() != nullptr;

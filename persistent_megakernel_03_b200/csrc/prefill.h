@@ -22,6 +22,18 @@ struct PrefillWeights {
   std::vector<const uint16_t*> qkv, o, gu, dn;  // packed, per layer
 };
 
+// Device buffers of the persistent prefill (prefill_mk.cu), grown on demand.
+struct PfBuffers {
+  bool configured = false;
+  uint8_t* maps = nullptr;     // tensor maps (global memory, 256-byte aligned)
+  uint8_t* tasks = nullptr;
+  int32_t* queue = nullptr;
+  int32_t* queue_off = nullptr;
+  uint32_t* events = nullptr;
+  int32_t* err = nullptr;
+  size_t maps_cap = 0, tasks_cap = 0, queue_cap = 0, queue_off_cap = 0, events_cap = 0, err_cap = 0;
+};
+
 struct PrefillScratch {
   int max_tokens = 0;          // tokens per block
   float* x = nullptr;          // [T][hidden] residual stream
@@ -32,6 +44,7 @@ struct PrefillScratch {
   uint16_t* xl = nullptr;      //   ... and low part
   int32_t* meta = nullptr;     // per-token and per-tile arrays (see prefill.cu)
   int32_t* err = nullptr;      // device error word of the GEMM kernel
+  PfBuffers pf;                // the persistent prefill's task graph and maps
 };
 
 // Device-side parameters of a batched decode step (read by the captured
@@ -79,6 +92,14 @@ std::string prefill_alloc(const ModelDev& m, int max_tokens, PrefillScratch* sc,
 std::string prefill_run(const ModelDev& m, const PrefillWeights& w, PrefillScratch& sc,
                         cudaStream_t st, const int32_t* tokens_dev, const int32_t* offsets_host,
                         const int32_t* slots_host, int n_req);
+
+// The same prefill as ONE persistent kernel per block (prefill_mk.cu): every
+// operator of every layer a task, dependencies per (layer, stage, token tile)
+// through event counters, the GEMMs as tcgen05 tiles.  Synchronises `st`.
+std::string prefill_mk_run(const ModelDev& m, const PrefillWeights& w, PrefillScratch& sc,
+                           cudaStream_t st, const int32_t* tokens_dev, const int32_t* offsets_host,
+                           const int32_t* slots_host, int n_req, int num_sms,
+                           std::vector<void*>* owned);
 
 // Allocates the batched decode scratch (cudaMalloc).
 std::string batch_alloc(const ModelDev& m, int num_sms, BatchScratch* bs, std::vector<void*>* owned);

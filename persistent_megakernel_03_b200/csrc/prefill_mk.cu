@@ -1,0 +1,777 @@
+// prefill_mk.cu -- the tensor-core prompt prefill as ONE persistent kernel per
+// block of prompt positions: every operator of every layer is a task of a
+// task graph ("LLMs in einen MegaKernel kompilieren ...", "Part 1. Compiler":
+// operators refined into SM-sized tasks linked by events, dependencies that
+// follow data tiles rather than kernel boundaries; "MPK: A Compiler and
+// Runtime ..." idea 3: a graph that depends on the data -- here the prompt
+// lengths -- is built when the call arrives).
+//
+// The block's positions are cut into token tiles of 128.  Per layer and token
+// tile n the tasks are
+//   NORM    (layer 0 only) x = E[token]; the attention RMSNorm as three bf16 parts
+//   QKV     one per 128-row tile m of W_qkv: a tcgen05 GEMM tile (128 rows x
+//           the tile's tokens), waits for the norm of tile n only
+//   ROPE    RoPE q, K/V into the cache, for tile n; waits for every QKV tile of n
+//   ATTN    causal GQA attention, per (run of <= 16 positions, KV head); waits
+//           for the ROPE of every token tile up to its own (the keys it reads)
+//   OPROJ   GEMM tiles of W_o; wait for the ATTN tasks of tile n
+//   RES1    x += W_o attn, the FFN RMSNorm as three parts; waits for OPROJ of n
+//   GATEUP  GEMM tiles of W_gate/up; wait for RES1 of n
+//   SWIGLU  silu(gate) * up as three parts; waits for GATEUP of n
+//   DOWN    GEMM tiles of W_down; wait for SWIGLU of n
+//   RES2    x += W_down act and the next layer's attention RMSNorm; waits for
+//           DOWN of n
+// so a token tile runs ahead through the layer while other tiles are still in
+// earlier stages.  Every CTA walks its ahead-of-time queue in this order (all
+// CTAs co-resident, cooperative launch), which keeps the earliest unfinished
+// task runnable: no deadlock.  Every wait is bounded and recorded.
+//
+// The GEMM tile is the prefill GEMM of prefill.cu run inside the loop: the
+// weights and the three activation parts arrive by 2-D TMA (tensor maps in
+// global memory) in a 3-stage ring issued by two threads, lane 0 of warp 1
+// issues tcgen05.mma into three tensor-memory accumulators (allocated once
+// per CTA), warps 0-3 read them back.  The ring's and the accumulators'
+// phases run on across tiles.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <string>
+#include <vector>
+
+#include "../../include/mk.h"
+#include "attn_math.cuh"
+#include "mk_internal.h"
+#include "prefill.h"
+#include "ptx.cuh"
+#include "tc.cuh"
+
+namespace mk {
+
+PFN_cuTensorMapEncodeTiled_v12000 prefill_encode_fn();  // prefill.cu
+
+namespace {
+
+constexpr int kPfThreads = 512;
+constexpr int kPfWarps = kPfThreads / 32;
+constexpr int kPfTokTile = 128;      // tokens per token tile (the GEMM's N)
+constexpr int kPfRows = 128;         // weight rows per GEMM tile (the MMA's M)
+constexpr int kPfK = 64;             // K per stage
+constexpr int kPfStages = 3;
+constexpr int kPfAttnPos = 16;       // positions per attention task (one warp each)
+constexpr int kPfAttnKeys = 64;      // keys staged per block
+constexpr uint64_t kPfWaitNs = 2000000000ull;
+
+enum PfKind : int32_t {
+  PF_NORM = 0, PF_GEMM = 1, PF_ROPE = 2, PF_ATTN = 3, PF_RES1 = 4, PF_SWIGLU = 5, PF_RES2 = 6
+};
+enum PfMat : int32_t { PF_QKV = 0, PF_O = 1, PF_GU = 2, PF_DN = 3 };
+
+struct PfTask {
+  int32_t kind, layer;
+  int32_t n;          // token tile
+  int32_t a, b;       // GEMM: matrix (PfMat), row tile; ATTN: attention tile, KV head
+  int32_t wait_ev;    // -1: none
+  uint32_t wait_count;
+  int32_t sig_ev0, n_sig;
+  int32_t pad_[3];
+};
+static_assert(sizeof(PfTask) == 48, "PfTask layout");
+
+struct PfArgs {
+  ModelDev m;
+  const PfTask* tasks;
+  const int32_t* queue;
+  const int32_t* queue_off;       // [grid + 1]
+  const CUtensorMap* maps;        // [4 L] weight tiles, then [3 parts][3 K kinds] activations
+  uint32_t* events;
+  int32_t* err;                   // [0]: first error code, [1]: detail
+  const int32_t* tokens;          // the prompt tokens (device)
+  const int32_t* tok_src;         // [T] index into tokens of block token t
+  const int32_t* slot;            // [T] KV slot of token t
+  const int32_t* pos;             // [T] position of token t
+  const int32_t* attn_tiles;      // [n_attn][4]: first token, count, slot, first position
+  float* x;                       // [T][H]
+  float* y;                       // [T][ldy]
+  float* q;                       // [T][n_q d]
+  uint16_t* xh;                   // [T][ldx] three bf16 parts of the GEMM input (the
+  uint16_t* xm;                   // first K columns of a row; one row stride for every
+  uint16_t* xl;                   // stage, since token tiles sit in different stages)
+  int32_t T, ldy, ldx;
+};
+
+// maps[] index of an activation part (0 high, 1 middle, 2 low) for a GEMM over
+// K = hidden (0), n_q d (1) or ffn (2)
+__host__ __device__ __forceinline__ int pf_xmap(int L, int part, int kk) { return 4 * L + 3 * part + kk; }
+
+struct __align__(1024) PfSmem {
+  // GEMM stages (the attention tasks reuse these bytes)
+  uint8_t a[kPfStages][kPfRows * kPfK * 2];
+  uint8_t bh[kPfStages][kPfTokTile * kPfK * 2];
+  uint8_t bm[kPfStages][kPfTokTile * kPfK * 2];
+  uint8_t bl[kPfStages][kPfTokTile * kPfK * 2];
+  uint64_t full[kPfStages];
+  uint64_t empty[kPfStages];
+  uint64_t done;
+  uint32_t tmem;
+  int32_t abort_flag;
+  int32_t tmem_ok;   // cleared when an accumulator wait gave up (MMAs may be in flight)
+  uint32_t armed[kPfStages];  // the last ring position whose loads went to each stage
+};
+constexpr uint32_t kPfStageBytes = kPfRows * kPfK * 2 + 3 * kPfTokTile * kPfK * 2;
+constexpr uint32_t kPfTmemCols = 512;  // three 128-column accumulators
+
+__device__ __forceinline__ uint16_t pf_bf16(float f) {
+  __nv_bfloat16 b = __float2bfloat16_rn(f);
+  return *reinterpret_cast<uint16_t*>(&b);
+}
+__device__ __forceinline__ float pf_val(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
+
+// v -> three bf16 parts whose sum is v
+__device__ __forceinline__ void pf_split3(float v, uint16_t* hi, uint16_t* mid, uint16_t* lo, size_t i) {
+  const uint16_t h = pf_bf16(v);
+  const float r1 = v - pf_val(h);
+  const uint16_t md = pf_bf16(r1);
+  hi[i] = h;
+  mid[i] = md;
+  lo[i] = pf_bf16(r1 - pf_val(md));
+}
+
+__device__ __forceinline__ void pf_fail(const PfArgs& p, PfSmem& s, int code, int detail) {
+  if (atomicCAS(p.err, 0, code) == 0) p.err[1] = detail;
+  *(volatile int32_t*)&s.abort_flag = 1;
+}
+
+__device__ __forceinline__ bool pf_wait(const PfArgs& p, PfSmem& s, uint64_t* bar, uint32_t parity,
+                                        int where) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*(volatile int32_t*)&s.abort_flag) return false;
+    if (globaltimer_ns() - t0 > kPfWaitNs) {
+      pf_fail(p, s, MK_ERR_TIMEOUT, where);
+      return false;
+    }
+  }
+  return true;
+}
+
+// Wait without regard to the abort flag, bounded (the abort path's drain).
+__device__ __forceinline__ bool pf_drain(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer_ns() - t0 > 200000000ull) return false;
+  return true;
+}
+
+// Sum of squares of x[t] over the block (all threads), then the three parts of
+// x[t] * w / rms.
+__device__ __forceinline__ void pf_norm_rows(const PfArgs& p, PfSmem& s, int t0, int t1,
+                                             const uint16_t* w) {
+  const int H = p.m.hidden;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // one warp per token
+  for (int t = t0 + warp; t < t1; t += kPfWarps) {
+    const float* xr = p.x + (size_t)t * H;
+    float ss = 0.f;
+    for (int i = lane; i < H; i += 32) {
+      const float v = __ldcg(xr + i);
+      ss = fmaf(v, v, ss);
+    }
+    for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float r = 1.0f / sqrtf(ss / (float)H + p.m.rms_eps);
+    for (int i = lane; i < H; i += 32)
+      pf_split3(__ldcg(xr + i) * r * pf_val(w[i]), p.xh, p.xm, p.xl, (size_t)t * p.ldx + i);
+  }
+}
+
+// ----------------------------------------------------------------- GEMM tile
+
+struct PfGemmState {
+  uint32_t kb;      // k blocks issued / consumed by this CTA so far (ring position)
+  uint32_t tiles;   // GEMM tiles finished by this CTA so far (accumulator phase)
+};
+
+// Y[t][r] = sum_k W[r][k] (xh + xm + xl)[t][k] for rows [m0, m0 + 128) and the
+// tokens of tile n; bias added when given.
+__device__ __forceinline__ void pf_gemm_tile(const PfArgs& p, PfSmem& s, PfGemmState& gs,
+                                             const CUtensorMap* tm_w, int kk, int K, int n_rows,
+                                             int m0, int n, const uint16_t* bias) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nk = K / kPfK;
+  const int L = p.m.n_layers;
+  const CUtensorMap* th = p.maps + pf_xmap(L, 0, kk);
+  const CUtensorMap* tmm = p.maps + pf_xmap(L, 1, kk);
+  const CUtensorMap* tl = p.maps + pf_xmap(L, 2, kk);
+  const int n0 = n * kPfTokTile;
+  if ((warp == 0 || warp == 2) && lane == 0) {
+    // two issuing threads, alternate k blocks (one thread's TMA loads run one
+    // after another).  The stage memory may have been written by an attention
+    // task's generic stores: order them before the async-proxy writes.
+    fence_proxy_async_shared();
+    fence_proxy_async_global();
+    const int pid = warp >> 1;
+    for (int i = pid; i < nk; i += 2) {
+      const uint32_t g = gs.kb + i;
+      const int st = g % kPfStages;
+      if (g >= kPfStages && !pf_wait(p, s, &s.empty[st], ((g / kPfStages) - 1) & 1, -21)) break;
+      mbar_arrive_expect_tx(&s.full[st], kPfStageBytes);
+      s.armed[st] = g;
+      tma_load_2d(s.a[st], tm_w, i * kPfK, m0, &s.full[st]);
+      tma_load_2d(s.bh[st], th, i * kPfK, n0, &s.full[st]);
+      tma_load_2d(s.bm[st], tmm, i * kPfK, n0, &s.full[st]);
+      tma_load_2d(s.bl[st], tl, i * kPfK, n0, &s.full[st]);
+    }
+  } else if (warp == 1 && lane == 0) {
+    constexpr uint32_t idesc = mma_idesc_bf16_f32(kPfRows, kPfTokTile);
+    tc_fence_after_sync();
+    for (int i = 0; i < nk; ++i) {
+      const uint32_t g = gs.kb + i;
+      const int st = g % kPfStages;
+      if (!pf_wait(p, s, &s.full[st], (g / kPfStages) & 1, -22)) break;
+      tc_fence_after_sync();
+      const uint64_t da = sw128_kmajor_desc(s.a[st]);
+      const uint64_t dh = sw128_kmajor_desc(s.bh[st]);
+      const uint64_t dm = sw128_kmajor_desc(s.bm[st]);
+      const uint64_t dl = sw128_kmajor_desc(s.bl[st]);
+      const uint32_t acc_h = s.tmem + ((i & 1) ? 2u * kPfTokTile : 0u);
+      const uint32_t acc_ml = s.tmem + (uint32_t)kPfTokTile;
+#pragma unroll
+      for (int k = 0; k < kPfK / 16; ++k) {
+        tc_mma_f16(acc_h, da + 2 * k, dh + 2 * k, idesc, (i > 1 || k > 0) ? 1u : 0u);
+        tc_mma_f16(acc_ml, da + 2 * k, dm + 2 * k, idesc, (i | k) != 0);
+        tc_mma_f16(acc_ml, da + 2 * k, dl + 2 * k, idesc, 1u);
+      }
+      tc_commit(&s.empty[st]);
+    }
+    tc_commit(&s.done);  // also when stopped early: retires what was issued
+  }
+  __syncwarp();
+  gs.kb += nk;
+  // accumulators ready: warps 0-3 (tensor-memory lanes 32 w ..) read them
+  const uint32_t ph = gs.tiles & 1u;
+  gs.tiles += 1;
+  if (warp < 4) {
+    const bool ok = pf_wait(p, s, &s.done, ph, -23);
+    if (!ok) s.tmem_ok = 0;
+    tc_fence_after_sync();
+    if (ok) {
+      const int row = m0 + warp * 32 + lane;
+      const float b = (bias && row < n_rows) ? pf_val(bias[row]) : 0.f;
+      const bool odd = nk > 1;
+#pragma unroll 1
+      for (int c0 = 0; c0 < kPfTokTile; c0 += 16) {
+        float v[16], ml[16], v2[16];
+        const uint32_t base = s.tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0;
+        tmem_ld16(base, v);
+        tmem_ld16(base + (uint32_t)kPfTokTile, ml);
+        if (odd) tmem_ld16(base + 2u * kPfTokTile, v2);
+        if (row < n_rows) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int tok = n0 + c0 + j;
+            if (tok < p.T) p.y[(size_t)tok * p.ldy + row] = (v[j] + (odd ? v2[j] : 0.f)) + ml[j] + b;
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before_sync();
+}
+
+// --------------------------------------------------------- other task bodies
+
+// RoPE on the packed q/k rows, q to p.q, K/V (bf16) into the cache, for the
+// tokens of tile n (the decode step's QKV epilogue, over many tokens).
+__device__ __forceinline__ void pf_rope(const PfArgs& p, int layer, int t0, int t1) {
+  const ModelDev& m = p.m;
+  const int d = m.head_dim, G = m.group, half = d >> 1;
+  const int npairs = qkv_rows(m.n_q, m.n_kv, d) >> 1;
+  const uint16_t* bias = m.qkv_bias ? m.bqkv + (size_t)layer * qkv_rows(m.n_q, m.n_kv, d) : nullptr;
+  const int total = (t1 - t0) * npairs;
+  for (int idx = threadIdx.x; idx < total; idx += kPfThreads) {
+    const int t = t0 + idx / npairs, pi = idx - (idx / npairs) * npairs;
+    const int r = 2 * pi, ps = p.pos[t], sl = p.slot[t];
+    float y0 = __ldcg(p.y + (size_t)t * p.ldy + r), y1 = __ldcg(p.y + (size_t)t * p.ldy + r + 1);
+    if (bias) {
+      y0 += pf_val(bias[r]);
+      y1 += pf_val(bias[r + 1]);
+    }
+    int which, head, dim0, w1, h1, dim1;
+    qkv_source(r, G, d, &which, &head, &dim0);
+    qkv_source(r + 1, G, d, &w1, &h1, &dim1);
+    if (which < 2) {
+      const float c = m.rope_cos[(size_t)ps * half + dim0], sn = m.rope_sin[(size_t)ps * half + dim0];
+      const float o0 = y0 * c - y1 * sn, o1 = y0 * sn + y1 * c;
+      y0 = o0;
+      y1 = o1;
+    }
+    if (which == 0) {
+      float* qq = p.q + (size_t)t * m.n_q * d + (size_t)head * d;
+      qq[dim0] = y0;
+      qq[dim1] = y1;
+    } else {
+      uint16_t* cache = which == 1 ? m.kcache : m.vcache;
+      const size_t off = kv_row(m, sl, layer, head, ps);
+      cache[off + dim0] = pf_bf16(y0);
+      cache[off + dim1] = pf_bf16(y1);
+    }
+  }
+}
+
+// Causal GQA attention of up to 16 consecutive positions of one request
+// against its cache, one warp per position, 64 keys staged at a time in
+// shared memory (the decode step's four-key online-softmax update); output as
+// the O projection's three parts.
+template <int DPL, int G>
+__device__ __forceinline__ void pf_attn(const PfArgs& p, PfSmem& s, int layer, const int* tl, int g) {
+  constexpr int d = DPL * 32;
+  uint16_t* ks = reinterpret_cast<uint16_t*>(&s.a[0][0]);
+  uint16_t* vs = ks + kPfAttnKeys * d;
+  float* xbs = reinterpret_cast<float*>(vs + kPfAttnKeys * d);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t0 = tl[0], nt = tl[1], sl = tl[2], p0 = tl[3];
+  const ModelDev& m = p.m;
+  const int nq = m.n_q;
+  const bool mine = warp < nt;
+  const int ps = p0 + warp;
+  AttnState<DPL, G> st;
+  if (mine) attn_init<DPL, G>(st, p.q + (size_t)(t0 + warp) * nq * d + (size_t)g * G * d, d, m.attn_scale, lane);
+  const int n_keys = p0 + nt;
+  float* xb = xbs + warp * kAttnXbStride;
+  for (int kb = 0; kb < n_keys; kb += kPfAttnKeys) {
+    const int nk = min(kPfAttnKeys, n_keys - kb);
+    const size_t off = kv_row(m, sl, layer, g, kb);  // a 64-key block lies in one page
+    const uint16_t* K = m.kcache + off;
+    const uint16_t* V = m.vcache + off;
+    __syncthreads();
+    const int vec = nk * d / 8;
+    for (int i = threadIdx.x; i < vec; i += kPfThreads) {
+      reinterpret_cast<uint4*>(ks)[i] = __ldcg(reinterpret_cast<const uint4*>(K) + i);
+      reinterpret_cast<uint4*>(vs)[i] = __ldcg(reinterpret_cast<const uint4*>(V) + i);
+    }
+    __syncthreads();
+    if (!mine) continue;
+    const int lim = min(nk, ps + 1 - kb);  // causal: keys <= the position
+    for (int j0 = 0; j0 < lim; j0 += 4) {
+      const int nj = min(4, lim - j0);
+      {
+        float kv[4][DPL];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int jr = attn_key_row<G>(t, lane);
+          if (jr < nj) load_kv_row<DPL>(ks + (size_t)(j0 + jr) * d + lane * DPL, kv[t]);
+          else
+#pragma unroll
+            for (int i = 0; i < DPL; ++i) kv[t][i] = 0.f;
+        }
+        attn_scores4<DPL, G>(st, kv, nj, xb, lane);
+      }
+      float vv[4][DPL];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        if (t < nj) load_kv_row<DPL>(vs + (size_t)(j0 + t) * d + lane * DPL, vv[t]);
+        else
+#pragma unroll
+          for (int i = 0; i < DPL; ++i) vv[t][i] = 0.f;
+      }
+      attn_update4<DPL, G>(st, vv, xb);
+    }
+  }
+  if (!mine) return;
+  const size_t row = (size_t)(t0 + warp) * p.ldx + (size_t)g * G * d;
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    const float inv = 1.0f / st.l[h];
+#pragma unroll
+    for (int i = 0; i < DPL; ++i)
+      pf_split3(st.o[h][i] * inv, p.xh, p.xm, p.xl, row + (size_t)h * d + lane * DPL + i);
+  }
+}
+
+template <int DPL>
+__device__ __forceinline__ void pf_attn_g(const PfArgs& p, PfSmem& s, int layer, const int* tl, int g) {
+  switch (p.m.group) {
+    case 1: pf_attn<DPL, 1>(p, s, layer, tl, g); break;
+    case 2: pf_attn<DPL, 2>(p, s, layer, tl, g); break;
+    case 4: pf_attn<DPL, 4>(p, s, layer, tl, g); break;
+    case 7: if constexpr (DPL == 2) pf_attn<DPL, 7>(p, s, layer, tl, g); break;
+    case 8: if constexpr (DPL == 2) pf_attn<DPL, 8>(p, s, layer, tl, g); break;
+    default: break;
+  }
+}
+
+// ----------------------------------------------------------------- the kernel
+
+__global__ void __launch_bounds__(kPfThreads, 1) prefill_mk_kernel(const __grid_constant__ PfArgs p) {
+  extern __shared__ __align__(16) uint8_t pf_raw[];
+  const uint32_t base = smem_u32(pf_raw);
+  PfSmem& s = *reinterpret_cast<PfSmem*>(pf_raw + (((base + 1023u) & ~1023u) - base));
+  const int warp = threadIdx.x >> 5;
+  const ModelDev& m = p.m;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kPfStages; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.empty[i], 1);
+    }
+    mbar_init(&s.done, 1);
+    for (int i = 0; i < kPfStages; ++i) s.armed[i] = 0xffffffffu;
+    s.abort_flag = 0;
+    s.tmem_ok = 1;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&s.tmem, kPfTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  PfGemmState gs{0u, 0u};
+  const int q0 = p.queue_off[blockIdx.x], q1 = p.queue_off[blockIdx.x + 1];
+  const int H = m.hidden, F = m.ffn, L = m.n_layers, qd = m.n_q * m.head_dim;
+  const int qkvR = qkv_rows(m.n_q, m.n_kv, m.head_dim);
+  __shared__ int s_go;
+  for (int qi = q0; qi < q1; ++qi) {
+    const PfTask t = p.tasks[p.queue[qi]];
+    if (threadIdx.x == 0) {
+      int go = *(volatile int32_t*)&s.abort_flag == 0;
+      if (go && t.wait_ev >= 0) {
+        const uint64_t t0 = globaltimer_ns();
+        uint32_t spins = 0;
+        while (ld_acquire_gpu(p.events + t.wait_ev) < t.wait_count) {
+          if ((++spins & 63u) == 0) {
+            if (ld_relaxed_gpu_s32(p.err) != 0) { go = 0; break; }
+            if (globaltimer_ns() - t0 > kPfWaitNs) {
+              pf_fail(p, s, MK_ERR_TIMEOUT, qi);
+              go = 0;
+              break;
+            }
+          }
+        }
+        // the inputs were written by generic stores of other CTAs; the GEMM
+        // tiles read them through the async proxy (TMA)
+        fence_proxy_async_global();
+      }
+      s_go = go;
+    }
+    __syncthreads();
+    if (!s_go) break;
+    const int n = t.n, t0 = n * kPfTokTile, t1 = min(p.T, t0 + kPfTokTile);
+    const int l = t.layer;
+    switch (t.kind) {
+      case PF_NORM: {
+        const int HH = H;
+        for (int i = threadIdx.x; i < (t1 - t0) * HH; i += kPfThreads) {
+          const int tt = t0 + i / HH, c = i - (i / HH) * HH;
+          int tok = p.tokens[p.tok_src[tt]];
+          if (tok < 0 || tok >= m.vocab) {
+            if (atomicCAS(m.status, 0, MK_ERR_TOKEN_RANGE) == 0) m.status_info[0] = tok;
+            tok = 0;
+          }
+          p.x[(size_t)tt * H + c] = pf_val(m.embed[(size_t)tok * H + c]);
+        }
+        __syncthreads();
+        pf_norm_rows(p, s, t0, t1, m.attn_norm);
+        break;
+      }
+      case PF_GEMM: {
+        const int mat = t.a, m0 = t.b * kPfRows;
+        const CUtensorMap* tm_w = p.maps + 4 * l + mat;
+        if (mat == PF_QKV)  // (the bias is added with RoPE)
+          pf_gemm_tile(p, s, gs, tm_w, 0, H, qkvR, m0, n, nullptr);
+        else if (mat == PF_O)
+          pf_gemm_tile(p, s, gs, tm_w, 1, qd, H, m0, n, nullptr);
+        else if (mat == PF_GU)
+          pf_gemm_tile(p, s, gs, tm_w, 0, H, 2 * F, m0, n, nullptr);
+        else
+          pf_gemm_tile(p, s, gs, tm_w, 2, F, H, m0, n, nullptr);
+        break;
+      }
+      case PF_ROPE:
+        pf_rope(p, l, t0, t1);
+        break;
+      case PF_ATTN:
+        if (m.head_dim == 128) pf_attn_g<4>(p, s, l, p.attn_tiles + 4 * t.a, t.b);
+        else pf_attn_g<2>(p, s, l, p.attn_tiles + 4 * t.a, t.b);
+        break;
+      case PF_RES1:
+      case PF_RES2: {
+        for (int i = threadIdx.x; i < (t1 - t0) * H; i += kPfThreads) {
+          const int tt = t0 + i / H, c = i - (i / H) * H;
+          float* xv = p.x + (size_t)tt * H + c;
+          *xv = __ldcg(xv) + __ldcg(p.y + (size_t)tt * p.ldy + c);
+        }
+        __syncthreads();
+        if (t.kind == PF_RES1) pf_norm_rows(p, s, t0, t1, m.ffn_norm + (size_t)l * H);
+        else if (l + 1 < L) pf_norm_rows(p, s, t0, t1, m.attn_norm + (size_t)(l + 1) * H);
+        break;
+      }
+      case PF_SWIGLU: {
+        for (int i = threadIdx.x; i < (t1 - t0) * F; i += kPfThreads) {
+          const int tt = t0 + i / F, j = i - (i / F) * F;
+          const float g = __ldcg(p.y + (size_t)tt * p.ldy + 2 * j);
+          const float u = __ldcg(p.y + (size_t)tt * p.ldy + 2 * j + 1);
+          pf_split3(g / (1.0f + expf(-g)) * u, p.xh, p.xm, p.xl, (size_t)tt * p.ldx + j);
+        }
+        break;
+      }
+      default:
+        break;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && t.n_sig > 0) {
+      fence_acq_rel_gpu();
+      for (int e = 0; e < t.n_sig; ++e) red_relaxed_gpu_add(p.events + t.sig_ev0 + e, 1u);
+    }
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (*(volatile int32_t*)&s.abort_flag && threadIdx.x == 0) {
+    // stopped inside a GEMM tile: let the loads still in flight land (each
+    // stage's last armed position) and the issued MMAs retire before exit
+    for (int i = 0; i < kPfStages; ++i)
+      if (s.armed[i] != 0xffffffffu) pf_drain(&s.full[i], (s.armed[i] / kPfStages) & 1);
+    if (!s.tmem_ok && gs.tiles > 0 && pf_drain(&s.done, (gs.tiles - 1) & 1)) s.tmem_ok = 1;
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  // tensor memory is released once every MMA retired; otherwise the error word
+  // is set and the columns stay allocated rather than be handed out while MMAs
+  // may still write them
+  if (warp == 0 && s.tmem_ok) tmem_dealloc(s.tmem, kPfTmemCols);
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ host side
+
+namespace {
+
+bool pf_make_map(CUtensorMap* map, const void* base, int rows, int cols, size_t row_stride_elems) {
+  auto fn = prefill_encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)row_stride_elems * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)kPfK, (cuuint32_t)kPfRows};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct PfGraph {
+  std::vector<PfTask> tasks;
+  std::vector<int32_t> queue, queue_off;
+  int n_events = 0;
+};
+
+// The task graph of one block (T tokens, attention tiles as built for it) on P
+// CTAs.  Events per (layer, stage, token tile); a task's wait count is the
+// number of producer tasks it needs.
+void pf_build(const ModelDev& m, int T, const std::vector<int32_t>& attn_tiles, int P, PfGraph& g) {
+  const int L = m.n_layers, H = m.hidden, F = m.ffn, nkv = m.n_kv;
+  const int qkvR = qkv_rows(m.n_q, m.n_kv, m.head_dim);
+  const int NT = (T + kPfTokTile - 1) / kPfTokTile;
+  const int mt_qkv = (qkvR + kPfRows - 1) / kPfRows, mt_h = (H + kPfRows - 1) / kPfRows;
+  const int mt_gu = (2 * F + kPfRows - 1) / kPfRows;
+  // event index: ((l * kStages + stage) * NT + n)
+  enum { E_NORM, E_QKV, E_ROPE, E_ATTN, E_O, E_RES1, E_GU, E_SW, E_DN, kStages };
+  auto ev = [&](int l, int st, int n) { return (l * kStages + st) * NT + n; };
+  g.n_events = (L + 1) * kStages * NT;
+  std::vector<int> attn_per_tile(NT, 0);
+  const int n_attn = (int)attn_tiles.size() / 4;
+  for (int a = 0; a < n_attn; ++a) attn_per_tile[attn_tiles[4 * a] / kPfTokTile] += 1;
+  g.tasks.clear();
+  auto add = [&](int kind, int l, int n, int a, int b, int wait_ev, int wait_count, int sig0,
+                 int nsig) {
+    PfTask t{};
+    t.kind = kind; t.layer = l; t.n = n; t.a = a; t.b = b;
+    t.wait_ev = wait_ev; t.wait_count = (uint32_t)wait_count; t.sig_ev0 = sig0; t.n_sig = nsig;
+    g.tasks.push_back(t);
+  };
+  for (int l = 0; l < L; ++l) {
+    if (l == 0)
+      for (int n = 0; n < NT; ++n) add(PF_NORM, 0, n, 0, 0, -1, 0, ev(0, E_NORM, n), 1);
+    for (int n = 0; n < NT; ++n)
+      for (int mt = 0; mt < mt_qkv; ++mt)
+        add(PF_GEMM, l, n, PF_QKV, mt, ev(l, E_NORM, n), 1, ev(l, E_QKV, n), 1);
+    // RoPE of tile n counts toward every later tile's "keys ready" event
+    for (int n = 0; n < NT; ++n)
+      add(PF_ROPE, l, n, 0, 0, ev(l, E_QKV, n), mt_qkv, ev(l, E_ROPE, n), NT - n);
+    for (int a = 0; a < n_attn; ++a) {
+      const int n = attn_tiles[4 * a] / kPfTokTile;
+      for (int kv = 0; kv < nkv; ++kv)
+        add(PF_ATTN, l, n, a, kv, ev(l, E_ROPE, n), n + 1, ev(l, E_ATTN, n), 1);
+    }
+    for (int n = 0; n < NT; ++n)
+      for (int mt = 0; mt < mt_h; ++mt)
+        add(PF_GEMM, l, n, PF_O, mt, ev(l, E_ATTN, n), attn_per_tile[n] * nkv, ev(l, E_O, n), 1);
+    for (int n = 0; n < NT; ++n) add(PF_RES1, l, n, 0, 0, ev(l, E_O, n), mt_h, ev(l, E_RES1, n), 1);
+    for (int n = 0; n < NT; ++n)
+      for (int mt = 0; mt < mt_gu; ++mt)
+        add(PF_GEMM, l, n, PF_GU, mt, ev(l, E_RES1, n), 1, ev(l, E_GU, n), 1);
+    for (int n = 0; n < NT; ++n) add(PF_SWIGLU, l, n, 0, 0, ev(l, E_GU, n), mt_gu, ev(l, E_SW, n), 1);
+    for (int n = 0; n < NT; ++n)
+      for (int mt = 0; mt < mt_h; ++mt)
+        add(PF_GEMM, l, n, PF_DN, mt, ev(l, E_SW, n), 1, ev(l, E_DN, n), 1);
+    // the residual, then the next layer's attention norm: its E_NORM event
+    for (int n = 0; n < NT; ++n)
+      add(PF_RES2, l, n, 0, 0, ev(l, E_DN, n), mt_h, ev(l + 1, E_NORM, n), 1);
+  }
+  // queues: the tasks in this (topological) order, dealt round-robin
+  std::vector<std::vector<int32_t>> per(P);
+  for (size_t i = 0; i < g.tasks.size(); ++i) per[i % P].push_back((int32_t)i);
+  g.queue.clear();
+  g.queue_off.assign(P + 1, 0);
+  for (int c = 0; c < P; ++c) {
+    g.queue_off[c] = (int32_t)g.queue.size();
+    g.queue.insert(g.queue.end(), per[c].begin(), per[c].end());
+  }
+  g.queue_off[P] = (int32_t)g.queue.size();
+}
+
+template <class T>
+std::string pf_grow(T** p, size_t* cap, size_t need, std::vector<void*>* owned) {
+  if (*cap >= need) return "";
+  void* v = nullptr;
+  if (cudaMalloc(&v, need) != cudaSuccess) return "prefill megakernel scratch: cudaMalloc";
+  owned->push_back(v);  // freed with the context
+  *p = static_cast<T*>(v);
+  *cap = need;
+  return "";
+}
+
+}  // namespace
+
+size_t prefill_mk_smem_bytes() { return sizeof(PfSmem) + 1024; }
+
+std::string prefill_mk_run(const ModelDev& m, const PrefillWeights& w, PrefillScratch& sc,
+                           cudaStream_t st, const int32_t* tokens_dev, const int32_t* offsets_host,
+                           const int32_t* slots_host, int n_req, int num_sms,
+                           std::vector<void*>* owned) {
+  const int H = m.hidden, F = m.ffn, d = m.head_dim, qd = m.n_q * d, L = m.n_layers;
+  const int qkvR = qkv_rows(m.n_q, m.n_kv, d);
+  const int ldy = std::max(std::max(qkvR, 2 * F), H);
+  const int ldx = std::max(std::max(H, F), qd);
+  PfBuffers& b = sc.pf;
+  if (!b.configured) {
+    if (cudaFuncSetAttribute(prefill_mk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)prefill_mk_smem_bytes()) != cudaSuccess)
+      return "prefill megakernel: shared memory attribute";
+    b.configured = true;
+  }
+  if (!b.maps) {
+    // tensor maps, written once per context: the weights of every layer, then
+    // the activation parts for K = hidden, n_q d, ffn over all max_tokens rows
+    // (token columns past a block's end are computed from stale rows and never
+    // stored)
+    std::vector<CUtensorMap> maps((size_t)4 * L + 9);
+    for (int l = 0; l < L; ++l) {
+      if (!pf_make_map(&maps[4 * l + PF_QKV], w.qkv[l], qkvR, H, H) ||
+          !pf_make_map(&maps[4 * l + PF_O], w.o[l], H, qd, qd) ||
+          !pf_make_map(&maps[4 * l + PF_GU], w.gu[l], 2 * F, H, H) ||
+          !pf_make_map(&maps[4 * l + PF_DN], w.dn[l], H, F, F))
+        return "prefill megakernel: weight tensor map";
+    }
+    const uint16_t* parts[3] = {sc.xh, sc.xm, sc.xl};
+    const int kdim[3] = {H, qd, F};
+    for (int part = 0; part < 3; ++part)
+      for (int kk = 0; kk < 3; ++kk)
+        if (!pf_make_map(&maps[pf_xmap(L, part, kk)], parts[part], sc.max_tokens, kdim[kk], ldx))
+          return "prefill megakernel: activation tensor map";
+    std::string e0 = pf_grow(&b.maps, &b.maps_cap, maps.size() * sizeof(CUtensorMap), owned);
+    if (!e0.empty()) return e0;
+    if (cudaMemcpy(b.maps, maps.data(), maps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice) != cudaSuccess)
+      return "prefill megakernel: tensor map upload";
+  }
+  // every position but each prompt's last, as (request, position) in order
+  std::vector<int> tok_src, slot, pos;
+  for (int r = 0; r < n_req; ++r)
+    for (int p = 0; p + 1 < offsets_host[r + 1] - offsets_host[r]; ++p) {
+      tok_src.push_back(offsets_host[r] + p);
+      slot.push_back(slots_host[r]);
+      pos.push_back(p);
+    }
+  const int total = (int)tok_src.size();
+  std::string e;
+  for (int b0 = 0; b0 < total; b0 += sc.max_tokens) {
+    const int T = std::min(sc.max_tokens, total - b0);
+    std::vector<int32_t> meta(3 * (size_t)T), tiles;
+    for (int t = 0; t < T; ++t) {
+      meta[t] = tok_src[b0 + t];
+      meta[T + t] = slot[b0 + t];
+      meta[2 * T + t] = pos[b0 + t];
+    }
+    // attention tiles: runs of <= 16 positions of one request inside one token tile
+    for (int t = 0; t < T;) {
+      int n = 1;
+      while (t + n < T && n < kPfAttnPos && slot[b0 + t + n] == slot[b0 + t] &&
+             (t + n) % kPfTokTile != 0)
+        ++n;
+      tiles.insert(tiles.end(), {t, n, slot[b0 + t], pos[b0 + t]});
+      t += n;
+    }
+    PfGraph gr;
+    pf_build(m, T, tiles, num_sms, gr);
+    if (!(e = pf_grow(&b.tasks, &b.tasks_cap, gr.tasks.size() * sizeof(PfTask), owned)).empty() ||
+        !(e = pf_grow(&b.queue, &b.queue_cap, gr.queue.size() * 4, owned)).empty() ||
+        !(e = pf_grow(&b.queue_off, &b.queue_off_cap, gr.queue_off.size() * 4, owned)).empty() ||
+        !(e = pf_grow(&b.events, &b.events_cap, (size_t)gr.n_events * 4, owned)).empty() ||
+        !(e = pf_grow(&b.err, &b.err_cap, 16, owned)).empty())
+      return e;
+    int32_t* d_src = sc.meta;
+    int32_t* d_slot = sc.meta + T;
+    int32_t* d_pos = sc.meta + 2 * T;
+    int32_t* d_tiles = sc.meta + 3 * (size_t)sc.max_tokens;
+    if (cudaMemcpyAsync(sc.meta, meta.data(), meta.size() * 4, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(d_tiles, tiles.data(), tiles.size() * 4, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(b.tasks, gr.tasks.data(), gr.tasks.size() * sizeof(PfTask), cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(b.queue, gr.queue.data(), gr.queue.size() * 4, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(b.queue_off, gr.queue_off.data(), gr.queue_off.size() * 4, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemsetAsync(b.events, 0, (size_t)gr.n_events * 4, st) != cudaSuccess ||
+        cudaMemsetAsync(b.err, 0, 16, st) != cudaSuccess)
+      return "prefill megakernel: upload";
+    PfArgs a{};
+    a.m = m;
+    a.tasks = reinterpret_cast<const PfTask*>(b.tasks);
+    a.queue = b.queue;
+    a.queue_off = b.queue_off;
+    a.maps = reinterpret_cast<const CUtensorMap*>(b.maps);
+    a.events = b.events;
+    a.err = b.err;
+    a.tokens = tokens_dev;
+    a.tok_src = d_src;
+    a.slot = d_slot;
+    a.pos = d_pos;
+    a.attn_tiles = d_tiles;
+    a.x = sc.x; a.y = sc.y; a.q = sc.q;
+    a.xh = sc.xh; a.xm = sc.xm; a.xl = sc.xl;
+    a.T = T; a.ldy = ldy; a.ldx = ldx;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(num_sms);
+    cfg.blockDim = dim3(kPfThreads);
+    cfg.dynamicSmemBytes = prefill_mk_smem_bytes();
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t le = cudaLaunchKernelEx(&cfg, prefill_mk_kernel, a);
+    if (le != cudaSuccess) return std::string("prefill megakernel launch: ") + cudaGetErrorString(le);
+    // the host vectors above are staged by the (pageable) copies before they return
+    int32_t herr[2] = {0, 0};
+    if (cudaMemcpyAsync(herr, b.err, 8, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+      return std::string("prefill megakernel: ") + cudaGetErrorString(cudaGetLastError());
+    if (herr[0]) return "prefill megakernel: a wait timed out (detail " + std::to_string(herr[1]) + ")";
+  }
+  return "";
+}
+
+}  // namespace mk

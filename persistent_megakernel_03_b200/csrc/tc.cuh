@@ -12,6 +12,13 @@ namespace mk {
 
 // One box of a 2-D tensor map into shared memory; completes on `bar` with the
 // box's byte count.  c0 is the inner (contiguous) coordinate in elements.
+// Orders this thread's earlier generic-proxy accesses of shared memory
+// before its later async-proxy operations on it (TMA copies into bytes that
+// generic stores used before).
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1,
                                             uint64_t* bar) {
   asm volatile(
