@@ -137,6 +137,11 @@ typedef struct {
                              counters; the GEMMs as tcgen05 tiles); 0: default, one
                              launch per operator and layer.  Both give the same
                              result up to the order of the fp32 additions. */
+  int prefill_attention; /* tensor-core prefill only.  0: default, the causal
+                            attention on the tensor cores (tcgen05: 128 positions x
+                            64 keys per step, online softmax, the fp32 queries and
+                            probabilities as two bf16 parts each); 1: on CUDA cores
+                            (one warp per position, fp32 throughout). */
 } mk_options;
 
 typedef struct mk_ctx mk_ctx;

@@ -67,7 +67,7 @@ class Options(C.Structure):
                 ("mode", C.c_int), ("l2_prefetch", C.c_int), ("weight_format", C.c_int),
                 ("batch_sequential", C.c_int), ("prefill_steps", C.c_int),
                 ("kv_page_tokens", C.c_int), ("kv_pool_pages", C.c_int),
-                ("prefill_megakernel", C.c_int)]
+                ("prefill_megakernel", C.c_int), ("prefill_attention", C.c_int)]
 
 
 class PlanInfo(C.Structure):
@@ -169,7 +169,7 @@ class Plan:
         L = lib()
         self.h = C.c_void_p()
         cfg = make_config(model, max_seq, max_batch)
-        opt = Options(num_ctas, attn_splits, 0, 0, 0, weight_format, 0, 0, 0, 0, 0)
+        opt = Options(num_ctas, attn_splits, 0, 0, 0, weight_format, 0, 0, 0, 0, 0, 0)
         rc = L.mk_plan_build(C.byref(cfg), C.byref(opt), int(num_ctas), C.byref(self.h))
         if rc != MK_OK:
             raise MkError(rc, "mk_plan_build rejected the configuration")
@@ -219,7 +219,7 @@ class Decoder:
                  timeout_ms: int = 0, mode: int = MODE_MEGAKERNEL, stream=None,
                  l2_prefetch: int = 0, prefill_steps: int = 0, batch_sequential: int = 0,
                  weight_format: int = 0, kv_page_tokens: int = 0, kv_pool_pages: int = 0,
-                 prefill_megakernel: int = 0):
+                 prefill_megakernel: int = 0, prefill_attention: int = 0):
         import torch
         L = lib()
         self.model = model
@@ -243,7 +243,7 @@ class Decoder:
         cfg = make_config(model, max_seq, max_batch)
         opt = Options(num_ctas, attn_splits, timeout_ms, mode, l2_prefetch, weight_format,
                       batch_sequential, prefill_steps, kv_page_tokens, kv_pool_pages,
-                      prefill_megakernel)
+                      prefill_megakernel, prefill_attention)
         self.h = C.c_void_p()
         rc = L.mk_create(C.byref(cfg), C.byref(w), C.byref(opt), self.stream.cuda_stream,
                          C.byref(self.h))

@@ -14,7 +14,7 @@ LIB = os.path.join(HERE, "libmk.so")
 LIB_DEBUG = os.path.join(HERE, "libmk_debug.so")
 SOURCES = ["plan.cpp", "kernel.cu", "step_bf16_d128.cu", "step_bf16_d64.cu", "step_fp8_d128.cu",
            "step_fp8_d64.cu", "api.cu", "attention.cu", "prefill.cu",
-           "prefill_mk.cu"]
+           "prefill_mk.cu", "flash_attn.cu"]
 HEADERS = ["mk_internal.h", "plan.h", "ptx.cuh", "attn_math.cuh", "tc.cuh", "prefill.h",
            "step_kernel.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -720,7 +720,7 @@ static int prefill_impl(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t* o
             ? prefill_mk_run(ctx->md, ctx->pw, ctx->ps, ctx->stream, tokens_dev, offsets_host, slots,
                              n_req, ctx->plan.num_ctas, &ctx->allocs)
             : prefill_run(ctx->md, ctx->pw, ctx->ps, ctx->stream, tokens_dev, offsets_host, slots,
-                          n_req);
+                          n_req, ctx->opt.prefill_attention != 1);
     if (!e.empty()) {
       ctx->poisoned = true;
       return fail(ctx, MK_ERR_CUDA, e);

@@ -20,6 +20,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <array>
 #include <cmath>
 #include <string>
 #include <vector>
@@ -994,10 +995,15 @@ std::string prefill_alloc(const ModelDev& m, int max_tokens, PrefillScratch* sc,
 
 std::string prefill_run(const ModelDev& m, const PrefillWeights& w, PrefillScratch& sc,
                         cudaStream_t st, const int32_t* tokens_dev, const int32_t* offsets_host,
-                        const int32_t* slots_host, int n_req) {
+                        const int32_t* slots_host, int n_req, bool tc_attn) {
   const int H = m.hidden, F = m.ffn, d = m.head_dim, qd = m.n_q * d, L = m.n_layers;
   const int qkvR = qkv_rows(m.n_q, m.n_kv, d);
   const int ldy = std::max(std::max(qkvR, 2 * F), H);
+  const bool use_fa = tc_attn;
+  if (use_fa) {
+    const std::string fe = flash_attn_prepare(m, &sc.fa);
+    if (!fe.empty()) return fe;
+  }
   // every position but each prompt's last, as (request, position) in order
   std::vector<int> tok_src, slot, pos;
   for (int r = 0; r < n_req; ++r)
@@ -1024,7 +1030,25 @@ std::string prefill_run(const ModelDev& m, const PrefillWeights& w, PrefillScrat
       tiles.insert(tiles.end(), {t, n, slot[b0 + t], pos[b0 + t]});
       t += n;
     }
-    const int ntiles = (int)tiles.size() / 4;
+    int ntiles = (int)tiles.size() / 4;
+    if (use_fa) {
+      // tensor-core attention: runs of <= 128 positions of one request, the
+      // longest key ranges first (the causal work is uneven)
+      std::vector<std::array<int32_t, 4>> ft;
+      for (int t = 0; t < T;) {
+        int n = 1;
+        while (t + n < T && n < kFaTileRows && slot[b0 + t + n] == slot[b0 + t]) ++n;
+        ft.push_back({t, n, slot[b0 + t], pos[b0 + t]});
+        t += n;
+      }
+      std::stable_sort(ft.begin(), ft.end(), [](const std::array<int32_t, 4>& a,
+                                                const std::array<int32_t, 4>& b) {
+        return a[1] + a[3] > b[1] + b[3];
+      });
+      tiles.clear();
+      for (const auto& f : ft) tiles.insert(tiles.end(), f.begin(), f.end());
+      ntiles = (int)ft.size();
+    }
     int32_t* d_src = sc.meta;
     int32_t* d_slot = sc.meta + T;
     int32_t* d_pos = sc.meta + 2 * T;
@@ -1038,7 +1062,10 @@ std::string prefill_run(const ModelDev& m, const PrefillWeights& w, PrefillScrat
       const uint16_t* bias = m.qkv_bias ? m.bqkv + (size_t)l * qkvR : nullptr;
       if (!(e = gemm<kPBN, kPStages>(w.qkv[l], qkvR, H, sc.xh, sc.xm, sc.xl, T, sc.y, ldy, bias, sc.err, st)).empty()) return e;
       rope_kv_kernel<<<T, 256, 0, st>>>(sc.y, ldy, 1, 0, nullptr, d_slot, d_pos, m, l, sc.q);
-      if (!(e = attn(dim3(ntiles, m.n_kv), st, sc.q, d_tiles, m, l, sc.xh, sc.xm, sc.xl)).empty()) return e;
+      e = use_fa ? flash_attn_launch(m, sc.fa, d_tiles, ntiles, l, sc.q, qd, sc.xh, sc.xm, sc.xl, qd,
+                                     sc.err, st)
+                 : attn(dim3(ntiles, m.n_kv), st, sc.q, d_tiles, m, l, sc.xh, sc.xm, sc.xl);
+      if (!e.empty()) return e;
       if (!(e = gemm<kPBN, kPStages>(w.o[l], H, qd, sc.xh, sc.xm, sc.xl, T, sc.y, ldy, nullptr, sc.err, st)).empty()) return e;
       residual_kernel<<<T, 256, 0, st>>>(sc.x, sc.y, H, ldy, 1, 0);
       rmsnorm_split_kernel<<<T, 256, 0, st>>>(sc.x, m.ffn_norm + (size_t)l * H, H, m.rms_eps, sc.xh, sc.xm, sc.xl);
@@ -1055,7 +1082,7 @@ std::string prefill_run(const ModelDev& m, const PrefillWeights& w, PrefillScrat
   if (cudaMemcpyAsync(&herr, sc.err, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
       cudaStreamSynchronize(st) != cudaSuccess)
     return std::string("prefill: ") + cudaGetErrorString(cudaGetLastError());
-  if (herr) return "prefill GEMM: a pipeline wait timed out";
+  if (herr) return "prefill: a pipeline wait timed out (GEMM or attention)";
   return "";
 }
 

@@ -7,6 +7,7 @@
 // GQA attention over the cache.  The last prompt position then runs through
 // the decode step, which produces its logits and greedy id.
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <string>
@@ -34,6 +35,14 @@ struct PfBuffers {
   size_t maps_cap = 0, tasks_cap = 0, queue_cap = 0, queue_off_cap = 0, events_cap = 0, err_cap = 0;
 };
 
+// Tensor maps of the KV cache for the tensor-core attention (flash_attn.cu):
+// rows of head_dim bf16, boxes of 64 keys x 64 dims, K and V, first and
+// second 64-dim half.
+struct FaMaps {
+  CUtensorMap k0, k1, v0, v1;
+  bool ready = false;
+};
+
 struct PrefillScratch {
   int max_tokens = 0;          // tokens per block
   float* x = nullptr;          // [T][hidden] residual stream
@@ -45,7 +54,19 @@ struct PrefillScratch {
   int32_t* meta = nullptr;     // per-token and per-tile arrays (see prefill.cu)
   int32_t* err = nullptr;      // device error word of the GEMM kernel
   PfBuffers pf;                // the persistent prefill's task graph and maps
+  FaMaps fa;                   // the KV cache as tensor maps (tensor-core attention)
 };
+
+// Causal GQA attention of runs of <= 128 consecutive prompt positions of one
+// request on the tensor cores (flash_attn.cu).  tiles_dev: [n_tiles][4] = first
+// block token, rows, KV slot, first position; q: [T][ldq] rotated fp32
+// queries; output [T][ldo] as three bf16 parts.  Waits that run out set
+// err[0] = MK_ERR_TIMEOUT.
+constexpr int kFaTileRows = 128;
+std::string flash_attn_prepare(const ModelDev& m, FaMaps* fm);
+std::string flash_attn_launch(const ModelDev& m, const FaMaps& fm, const int32_t* tiles_dev,
+                              int n_tiles, int layer, const float* q, int ldq, uint16_t* oh,
+                              uint16_t* om, uint16_t* ol, int ldo, int32_t* err, cudaStream_t st);
 
 // Device-side parameters of a batched decode step (read by the captured
 // kernels, written before each replay).
@@ -91,7 +112,8 @@ std::string prefill_alloc(const ModelDev& m, int max_tokens, PrefillScratch* sc,
 // slots_host[r].  Enqueued on `st`.
 std::string prefill_run(const ModelDev& m, const PrefillWeights& w, PrefillScratch& sc,
                         cudaStream_t st, const int32_t* tokens_dev, const int32_t* offsets_host,
-                        const int32_t* slots_host, int n_req);
+                        const int32_t* slots_host, int n_req,
+                        bool tc_attn);
 
 // The same prefill as ONE persistent kernel per block (prefill_mk.cu): every
 // operator of every layer a task, dependencies per (layer, stage, token tile)

@@ -10,15 +10,16 @@
 
 namespace mk {
 
-// One box of a 2-D tensor map into shared memory; completes on `bar` with the
-// box's byte count.  c0 is the inner (contiguous) coordinate in elements.
 // Orders this thread's earlier generic-proxy accesses of shared memory
 // before its later async-proxy operations on it (TMA copies into bytes that
-// generic stores used before).
+// generic stores used before, tcgen05.mma reading operands that generic
+// stores wrote).
 __device__ __forceinline__ void fence_proxy_async_shared() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// One box of a 2-D tensor map into shared memory; completes on `bar` with the
+// box's byte count.  c0 is the inner (contiguous) coordinate in elements.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1,
                                             uint64_t* bar) {
   asm volatile(
@@ -85,6 +86,22 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 16 consecutive fp32 columns of this thread's TMEM lane from registers; the
+// store has completed on return.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15]))
+      : "memory");
+}
+
 // Shared-memory matrix descriptor of a K-major tile written by TMA with the
 // 128-byte swizzle: rows of 64 bf16 (128 B), groups of 8 rows 1024 B apart.
 // Fields: start address >> 4 [0,14), leading-byte offset >> 4 [16,30) (not
@@ -97,6 +114,21 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(const void* tile) {
   uint64_t d = (uint64_t)((a & 0x3FFFFu) >> 4);
   d |= (uint64_t)1 << 16;
   d |= (uint64_t)(1024 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+// Descriptor of an MN-major operand in the 128-byte swizzled layout: rows of
+// 128 B hold 64 consecutive M/N elements, consecutive rows are consecutive K;
+// `lbo` = bytes between 64-element blocks along M/N, `sbo` = bytes between
+// groups of 8 K rows (1024 for densely stacked rows).  A K step of 16 is a
+// start-address advance of 2 * sbo.
+__device__ __forceinline__ uint64_t sw128_mnmajor_desc(const void* tile, uint32_t lbo, uint32_t sbo) {
+  const uint32_t a = smem_u32(tile);
+  uint64_t d = (uint64_t)((a & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
   d |= (uint64_t)1 << 46;
   d |= (uint64_t)2 << 61;
   return d;

@@ -76,3 +76,32 @@ def test_tensor_core_prefill_then_decode_matches_oracle(cuda_ok):
     dec = binding.Decoder(model, {k: v.cuda() for k, v in w.items()}, 340)
     gl, gh, gi = run_gpu(dec, model, tr)
     assert_within(compare(tr, gl, gh, gi))
+
+
+@pytest.mark.parametrize("model,lens", [
+    (synth.TINY, [300, 1, 129, 2100]),
+    (synth.QWEN05B.with_layers(2), [200, 77, 130]),
+    (synth.LLAMA8B.with_layers(2), [260, 5, 64, 129]),
+], ids=["tiny", "qwen-2l", "llama-2l"])
+def test_tensor_core_attention_matches_cuda_core_attention(cuda_ok, model, lens):
+    # the prefill's attention on the tensor cores (queries and probabilities as
+    # two bf16 parts, fp32 accumulation) against the fp32 CUDA-core attention:
+    # the caches they leave differ by the accumulation order only
+    w = {k: v.cuda() for k, v in synth.make_model(model, 5).items()}
+    a, la, _ = _prefill_opt(model, w, lens, prefill_attention=0)
+    b, lb, _ = _prefill_opt(model, w, lens, prefill_attention=1)
+    for x, y in zip(_cache(a, model, lens), _cache(b, model, lens)):
+        assert np.linalg.norm(x - y) <= 2e-3 * np.linalg.norm(y)
+        assert np.abs(x - y).max() <= 0.02 * np.abs(y).max()
+    np.testing.assert_allclose(la, lb, atol=5e-3, rtol=0)
+
+
+def _prefill_opt(model, w, lens, **kw):
+    toks, offs = synth.make_packed_prompts(lens, model.vocab, seed=11)
+    dec = binding.Decoder(model, w, max(lens) + 2, max_batch=len(lens), **kw)
+    logits = torch.empty(len(lens), model.vocab, device="cuda")
+    ids = torch.empty(len(lens), dtype=torch.int32, device="cuda")
+    dec.prefill(toks.to(torch.int32).cuda(), offs.tolist(), logits, ids)
+    torch.cuda.synchronize()
+    assert dec.status() == 0, dec.last_error()
+    return dec, logits.cpu().numpy(), ids.cpu().numpy()
