@@ -129,19 +129,21 @@ typedef struct {
                          pool by mk_kv_release */
   int kv_pool_pages; /* paged cache: pages in the pool (0: enough for every slot at
                         max_seq, i.e. max_batch * ceil(max_seq / kv_page_tokens)) */
-  int prefill_megakernel; /* tensor-core prefill only.  1: each block of <= 2048
-                             prompt positions runs as ONE persistent kernel (every
-                             operator of every layer a task; tasks of different
-                             128-position tiles overlap across operator and layer
-                             boundaries, dependencies per tile through event
-                             counters; the GEMMs as tcgen05 tiles); 0: default, one
-                             launch per operator and layer.  Both give the same
-                             result up to the order of the fp32 additions. */
+  int prefill_per_operator; /* tensor-core prefill only.  0: default, each block of
+                               <= 2048 prompt positions runs as ONE persistent
+                               kernel (every operator of every layer a task; tasks
+                               of different 128-position tiles overlap across
+                               operator and layer boundaries, dependencies per
+                               tile through event counters; tcgen05 GEMM and
+                               attention tasks); 1: one launch per operator and
+                               layer.  Both give the same result up to the order
+                               of the fp32 additions. */
   int prefill_attention; /* tensor-core prefill only.  0: default, the causal
                             attention on the tensor cores (tcgen05: 128 positions x
                             64 keys per step, online softmax, the fp32 queries and
                             probabilities as two bf16 parts each); 1: on CUDA cores
-                            (one warp per position, fp32 throughout). */
+                            (one warp per position, fp32 throughout; implies
+                            prefill_per_operator). */
 } mk_options;
 
 typedef struct mk_ctx mk_ctx;
@@ -267,6 +269,19 @@ int mk_copy_kv(mk_ctx* ctx, int req, int layer, int kv_head, int which, int n, v
  * consumed, 5 epilogue done, 6 finished; 7 holds (cta << 32 | task).
  * NULL turns tracing off.  The buffer must outlive the traced steps. */
 int mk_set_trace(mk_ctx* ctx, unsigned long long* trace_dev);
+
+/* Per-task timeline of the persistent prefill (the default tensor-core prefill)
+ * (diagnostics).  For the tasks of the FIRST block of a later prefill call, in
+ * the order the kernel's host graph lists them (at most `capacity` tasks),
+ * trace_dev receives 4 uint64 per task, %globaltimer ns: 0 the CTA began
+ * waiting for the task's dependencies, 1 they were satisfied, 2 the task
+ * finished (its completion signalled); word 3 describes the task: bits 0-15
+ * the CTA, 16-19 the kind (0 embedding + norm, 1 GEMM tile, 2 RoPE + KV
+ * append, 3 attention, 4 O residual + norm, 5 SwiGLU, 6 down residual +
+ * norm), 20-23 the GEMM's matrix (0 QKV, 1 O, 2 gate/up, 3 down), 24-31 the
+ * layer, 32-47 the 128-position tile, 48-63 the row tile / query head.
+ * NULL turns tracing off.  The buffer must outlive the traced call. */
+int mk_set_prefill_trace(mk_ctx* ctx, unsigned long long* trace_dev, int capacity);
 
 /* Selects the execution mode of later steps (MK_MODE_*). */
 int mk_set_mode(mk_ctx* ctx, int mode);

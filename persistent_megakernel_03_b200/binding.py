@@ -30,7 +30,7 @@ EXPORTS = ("mk_create", "mk_prefill", "mk_decode_step", "mk_decode_steps", "mk_d
            "mk_kv_pointer", "mk_copy_kv", "mk_set_mode", "mk_status", "mk_last_error",
            "mk_destroy", "mk_plan_build", "mk_plan_get_info", "mk_plan_get_tasks",
            "mk_plan_get_queue", "mk_plan_get_event_counts", "mk_plan_destroy",
-           "mk_qkv_row_source", "mk_read_probe", "mk_set_trace",
+           "mk_qkv_row_source", "mk_read_probe", "mk_set_trace", "mk_set_prefill_trace",
            "mk_attention_workspace_bytes", "mk_attention_decode",
            "mk_attention_decode_noalloc", "mk_inject_stall")
 
@@ -67,7 +67,7 @@ class Options(C.Structure):
                 ("mode", C.c_int), ("l2_prefetch", C.c_int), ("weight_format", C.c_int),
                 ("batch_sequential", C.c_int), ("prefill_steps", C.c_int),
                 ("kv_page_tokens", C.c_int), ("kv_pool_pages", C.c_int),
-                ("prefill_megakernel", C.c_int), ("prefill_attention", C.c_int)]
+                ("prefill_per_operator", C.c_int), ("prefill_attention", C.c_int)]
 
 
 class PlanInfo(C.Structure):
@@ -134,6 +134,7 @@ def lib(build_if_missing: bool = True):
     L.mk_qkv_row_source.argtypes = [C.POINTER(Config), i, ip, ip, ip]
     L.mk_read_probe.argtypes = [vp, C.c_size_t, vp, vp]
     L.mk_set_trace.argtypes = [vp, vp]
+    L.mk_set_prefill_trace.argtypes = [vp, vp, C.c_int]
     L.mk_attention_workspace_bytes.argtypes = [i, i, i]
     L.mk_attention_workspace_bytes.restype = C.c_size_t
     L.mk_attention_decode.argtypes = [vp, vp, vp, i, i, i, i, vp, vp, vp]
@@ -219,7 +220,7 @@ class Decoder:
                  timeout_ms: int = 0, mode: int = MODE_MEGAKERNEL, stream=None,
                  l2_prefetch: int = 0, prefill_steps: int = 0, batch_sequential: int = 0,
                  weight_format: int = 0, kv_page_tokens: int = 0, kv_pool_pages: int = 0,
-                 prefill_megakernel: int = 0, prefill_attention: int = 0):
+                 prefill_per_operator: int = 0, prefill_attention: int = 0):
         import torch
         L = lib()
         self.model = model
@@ -243,7 +244,7 @@ class Decoder:
         cfg = make_config(model, max_seq, max_batch)
         opt = Options(num_ctas, attn_splits, timeout_ms, mode, l2_prefetch, weight_format,
                       batch_sequential, prefill_steps, kv_page_tokens, kv_pool_pages,
-                      prefill_megakernel, prefill_attention)
+                      prefill_per_operator, prefill_attention)
         self.h = C.c_void_p()
         rc = L.mk_create(C.byref(cfg), C.byref(w), C.byref(opt), self.stream.cuda_stream,
                          C.byref(self.h))
@@ -346,6 +347,13 @@ class Decoder:
         (int64 CUDA tensor, 8 words per task); None turns it off."""
         _check(lib().mk_set_trace(self.h, None if trace_dev is None else trace_dev.data_ptr()),
                self.h)
+
+    def set_prefill_trace(self, trace_dev=None):
+        """Per-task timeline of the persistent prefill's first block into
+        ``trace_dev`` (int64 CUDA tensor, 4 words per task); None turns it off."""
+        cap = 0 if trace_dev is None else trace_dev.numel() // 4
+        _check(lib().mk_set_prefill_trace(self.h, None if trace_dev is None else trace_dev.data_ptr(),
+                                          cap), self.h)
 
     def status(self) -> int:
         return int(lib().mk_status(self.h))

@@ -716,7 +716,7 @@ static int prefill_impl(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t* o
       if (!e.empty()) return fail(ctx, MK_ERR_CUDA, e);
     }
     const std::string e =
-        ctx->opt.prefill_megakernel > 0
+        ctx->opt.prefill_per_operator <= 0 && ctx->opt.prefill_attention != 1
             ? prefill_mk_run(ctx->md, ctx->pw, ctx->ps, ctx->stream, tokens_dev, offsets_host, slots,
                              n_req, ctx->plan.num_ctas, &ctx->allocs)
             : prefill_run(ctx->md, ctx->pw, ctx->ps, ctx->stream, tokens_dev, offsets_host, slots,
@@ -862,6 +862,15 @@ extern "C" int mk_kv_get_pages(mk_ctx* ctx, int slot, int32_t* pages_out, int ca
 extern "C" int mk_kv_free_pages(mk_ctx* ctx) {
   if (!ctx) return MK_ERR_INVALID_ARG;
   return (int)ctx->kv_free.size();
+}
+
+extern "C" int mk_set_prefill_trace(mk_ctx* ctx, unsigned long long* trace_dev, int capacity) {
+  int rc = check_ctx(ctx);
+  if (rc) return rc;
+  if (trace_dev && capacity <= 0) return fail(ctx, MK_ERR_INVALID_ARG, "trace capacity must be > 0");
+  ctx->ps.pf.trace = reinterpret_cast<uint64_t*>(trace_dev);
+  ctx->ps.pf.trace_cap = trace_dev ? capacity : 0;
+  return MK_OK;
 }
 
 extern "C" int mk_set_trace(mk_ctx* ctx, unsigned long long* trace_dev) {

@@ -33,6 +33,8 @@ struct PfBuffers {
   uint32_t* events = nullptr;
   int32_t* err = nullptr;
   size_t maps_cap = 0, tasks_cap = 0, queue_cap = 0, queue_off_cap = 0, events_cap = 0, err_cap = 0;
+  uint64_t* trace = nullptr;   // per-task timeline of the first block (mk_set_prefill_trace)
+  int trace_cap = 0;
 };
 
 // Tensor maps of the KV cache for the tensor-core attention (flash_attn.cu):

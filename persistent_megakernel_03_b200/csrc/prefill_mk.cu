@@ -7,13 +7,16 @@
 // lengths -- is built when the call arrives).
 //
 // The block's positions are cut into token tiles of 128.  Per layer and token
-// tile n the tasks are
+// tile n the tasks are (the elementwise ones -- NORM, ROPE, RES1, SWIGLU,
+// RES2 -- split into 16 tasks of 8 positions, so that many SMs share them)
 //   NORM    (layer 0 only) x = E[token]; the attention RMSNorm as three bf16 parts
 //   QKV     one per 128-row tile m of W_qkv: a tcgen05 GEMM tile (128 rows x
-//           the tile's tokens), waits for the norm of tile n only
-//   ROPE    RoPE q, K/V into the cache, for tile n; waits for every QKV tile of n
-//   ATTN    causal GQA attention, per (run of <= 16 positions, KV head); waits
-//           for the ROPE of every token tile up to its own (the keys it reads)
+//           the tile's tokens), waits for the norms of tile n only
+//   ROPE    RoPE q, K/V into the cache; waits for every QKV tile of n
+//   ATTN    causal GQA attention on the tensor cores (fa_tile, flash_attn.cuh),
+//           per (run of one request's positions inside tile n, query head);
+//           waits for the ROPE of every token tile up to its own (the keys it
+//           reads)
 //   OPROJ   GEMM tiles of W_o; wait for the ATTN tasks of tile n
 //   RES1    x += W_o attn, the FFN RMSNorm as three parts; waits for OPROJ of n
 //   GATEUP  GEMM tiles of W_gate/up; wait for RES1 of n
@@ -43,7 +46,7 @@
 #include <vector>
 
 #include "../../include/mk.h"
-#include "attn_math.cuh"
+#include "flash_attn.cuh"
 #include "mk_internal.h"
 #include "prefill.h"
 #include "ptx.cuh"
@@ -56,13 +59,12 @@ PFN_cuTensorMapEncodeTiled_v12000 prefill_encode_fn();  // prefill.cu
 namespace {
 
 constexpr int kPfThreads = 512;
-constexpr int kPfWarps = kPfThreads / 32;
 constexpr int kPfTokTile = 128;      // tokens per token tile (the GEMM's N)
 constexpr int kPfRows = 128;         // weight rows per GEMM tile (the MMA's M)
 constexpr int kPfK = 64;             // K per stage
 constexpr int kPfStages = 3;
-constexpr int kPfAttnPos = 16;       // positions per attention task (one warp each)
-constexpr int kPfAttnKeys = 64;      // keys staged per block
+constexpr int kPfEwTok = 8;          // positions per elementwise task (norm, RoPE, residual, SwiGLU)
+constexpr int kPfEwSub = kPfTokTile / kPfEwTok;  // elementwise tasks per token tile
 constexpr uint64_t kPfWaitNs = 2000000000ull;
 
 enum PfKind : int32_t {
@@ -86,7 +88,8 @@ struct PfArgs {
   const PfTask* tasks;
   const int32_t* queue;
   const int32_t* queue_off;       // [grid + 1]
-  const CUtensorMap* maps;        // [4 L] weight tiles, then [3 parts][3 K kinds] activations
+  const CUtensorMap* maps;        // [4 L] weight tiles, [3 parts][3 K kinds] activations, then
+                                  // the KV cache (K, K second half, V, V second half)
   uint32_t* events;
   int32_t* err;                   // [0]: first error code, [1]: detail
   const int32_t* tokens;          // the prompt tokens (device)
@@ -94,6 +97,7 @@ struct PfArgs {
   const int32_t* slot;            // [T] KV slot of token t
   const int32_t* pos;             // [T] position of token t
   const int32_t* attn_tiles;      // [n_attn][4]: first token, count, slot, first position
+  float qscale;                   // attention scale * log2(e)
   float* x;                       // [T][H]
   float* y;                       // [T][ldy]
   float* q;                       // [T][n_q d]
@@ -101,14 +105,19 @@ struct PfArgs {
   uint16_t* xm;                   // first K columns of a row; one row stride for every
   uint16_t* xl;                   // stage, since token tiles sit in different stages)
   int32_t T, ldy, ldx;
+  uint64_t* trace;                // per-task timeline (4 words per task index) or null
+  int32_t trace_cap;
 };
 
 // maps[] index of an activation part (0 high, 1 middle, 2 low) for a GEMM over
 // K = hidden (0), n_q d (1) or ffn (2)
 __host__ __device__ __forceinline__ int pf_xmap(int L, int part, int kk) { return 4 * L + 3 * part + kk; }
+// maps[] index of the KV-cache maps (K first half, K second half, V, V second half)
+__host__ __device__ __forceinline__ int pf_kvmap(int L, int i) { return 4 * L + 9 + i; }
+constexpr int kPfMapsExtra = 13;  // maps past the 4 L weight maps
 
 struct __align__(1024) PfSmem {
-  // GEMM stages (the attention tasks reuse these bytes)
+  // GEMM stages (the attention tasks use the same 192 KB as FaBuffers)
   uint8_t a[kPfStages][kPfRows * kPfK * 2];
   uint8_t bh[kPfStages][kPfTokTile * kPfK * 2];
   uint8_t bm[kPfStages][kPfTokTile * kPfK * 2];
@@ -120,7 +129,11 @@ struct __align__(1024) PfSmem {
   int32_t abort_flag;
   int32_t tmem_ok;   // cleared when an accumulator wait gave up (MMAs may be in flight)
   uint32_t armed[kPfStages];  // the last ring position whose loads went to each stage
+  FaBarriers fab;             // the attention tasks' barriers
+  float ew_red[16];           // per-warp sums of squares of the residual/norm tasks
 };
+static_assert(offsetof(PfSmem, a) == 0 && kPfStages * 4 * kPfRows * kPfK * 2 == sizeof(FaBuffers),
+              "the attention buffers alias the GEMM stages");
 constexpr uint32_t kPfStageBytes = kPfRows * kPfK * 2 + 3 * kPfTokTile * kPfK * 2;
 constexpr uint32_t kPfTmemCols = 512;  // three 128-column accumulators
 
@@ -167,24 +180,62 @@ __device__ __forceinline__ bool pf_drain(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
-// Sum of squares of x[t] over the block (all threads), then the three parts of
-// x[t] * w / rms.
-__device__ __forceinline__ void pf_norm_rows(const PfArgs& p, PfSmem& s, int t0, int t1,
-                                             const uint16_t* w) {
-  const int H = p.m.hidden;
+// Rows [e0, e1) (at most kPfEwTok) of the residual stream: x (+)= src, then
+// the RMSNorm of the new x times w as the next GEMM's three bf16 parts.  Two
+// warps per row (each half of the columns), 16-byte accesses; `src` is the
+// GEMM output y (add = true) or the embedding rows (add = false).
+__device__ __forceinline__ void pf_residual_norm(const PfArgs& p, PfSmem& s, int e0, int e1, bool add,
+                                                 const uint16_t* w) {
+  const ModelDev& m = p.m;
+  const int H = m.hidden, Hh = H >> 1;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // one warp per token
-  for (int t = t0 + warp; t < t1; t += kPfWarps) {
-    const float* xr = p.x + (size_t)t * H;
-    float ss = 0.f;
-    for (int i = lane; i < H; i += 32) {
-      const float v = __ldcg(xr + i);
-      ss = fmaf(v, v, ss);
+  const int t = e0 + (warp & 7), c0 = (warp >> 3) * Hh;
+  const bool live = warp < 16 && t < e1;
+  float ss = 0.f;
+  if (live) {
+    float* xr = p.x + (size_t)t * H;
+    const uint16_t* er = nullptr;
+    if (!add) {
+      int tok = __ldg(p.tokens + __ldg(p.tok_src + t));
+      if (tok < 0 || tok >= m.vocab) {
+        if (atomicCAS(m.status, 0, MK_ERR_TOKEN_RANGE) == 0) m.status_info[0] = tok;
+        tok = 0;
+      }
+      er = m.embed + (size_t)tok * H;
+    }
+    for (int i = c0 + lane * 4; i < c0 + Hh; i += 128) {
+      float4 v;
+      if (add) {
+        const float4 a = __ldcg(reinterpret_cast<const float4*>(xr + i));
+        const float4 b = __ldcg(reinterpret_cast<const float4*>(p.y + (size_t)t * p.ldy + i));
+        v = make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+      } else {
+        const uint2 e = __ldg(reinterpret_cast<const uint2*>(er + i));
+        v = make_float4(__uint_as_float(e.x << 16), __uint_as_float(e.x & 0xFFFF0000u),
+                        __uint_as_float(e.y << 16), __uint_as_float(e.y & 0xFFFF0000u));
+      }
+      *reinterpret_cast<float4*>(xr + i) = v;
+      ss = fmaf(v.x, v.x, ss);
+      ss = fmaf(v.y, v.y, ss);
+      ss = fmaf(v.z, v.z, ss);
+      ss = fmaf(v.w, v.w, ss);
     }
     for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    const float r = 1.0f / sqrtf(ss / (float)H + p.m.rms_eps);
-    for (int i = lane; i < H; i += 32)
-      pf_split3(__ldcg(xr + i) * r * pf_val(w[i]), p.xh, p.xm, p.xl, (size_t)t * p.ldx + i);
+  }
+  if (lane == 0 && warp < 16) s.ew_red[warp] = ss;
+  __syncthreads();
+  if (!live || !w) return;
+  const float tot = s.ew_red[warp & 7] + s.ew_red[(warp & 7) + 8];
+  const float r = 1.0f / sqrtf(tot / (float)H + m.rms_eps);
+  const float* xr = p.x + (size_t)t * H;
+  for (int i = c0 + lane * 4; i < c0 + Hh; i += 128) {
+    const float4 v = *reinterpret_cast<const float4*>(xr + i);  // this thread's own stores
+    const uint2 wv = __ldg(reinterpret_cast<const uint2*>(w + i));
+    const size_t o = (size_t)t * p.ldx + i;
+    pf_split3(v.x * r * pf_val((uint16_t)(wv.x & 0xFFFFu)), p.xh, p.xm, p.xl, o);
+    pf_split3(v.y * r * pf_val((uint16_t)(wv.x >> 16)), p.xh, p.xm, p.xl, o + 1);
+    pf_split3(v.z * r * pf_val((uint16_t)(wv.y & 0xFFFFu)), p.xh, p.xm, p.xl, o + 2);
+    pf_split3(v.w * r * pf_val((uint16_t)(wv.y >> 16)), p.xh, p.xm, p.xl, o + 3);
   }
 }
 
@@ -322,88 +373,6 @@ __device__ __forceinline__ void pf_rope(const PfArgs& p, int layer, int t0, int 
   }
 }
 
-// Causal GQA attention of up to 16 consecutive positions of one request
-// against its cache, one warp per position, 64 keys staged at a time in
-// shared memory (the decode step's four-key online-softmax update); output as
-// the O projection's three parts.
-template <int DPL, int G>
-__device__ __forceinline__ void pf_attn(const PfArgs& p, PfSmem& s, int layer, const int* tl, int g) {
-  constexpr int d = DPL * 32;
-  uint16_t* ks = reinterpret_cast<uint16_t*>(&s.a[0][0]);
-  uint16_t* vs = ks + kPfAttnKeys * d;
-  float* xbs = reinterpret_cast<float*>(vs + kPfAttnKeys * d);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t0 = tl[0], nt = tl[1], sl = tl[2], p0 = tl[3];
-  const ModelDev& m = p.m;
-  const int nq = m.n_q;
-  const bool mine = warp < nt;
-  const int ps = p0 + warp;
-  AttnState<DPL, G> st;
-  if (mine) attn_init<DPL, G>(st, p.q + (size_t)(t0 + warp) * nq * d + (size_t)g * G * d, d, m.attn_scale, lane);
-  const int n_keys = p0 + nt;
-  float* xb = xbs + warp * kAttnXbStride;
-  for (int kb = 0; kb < n_keys; kb += kPfAttnKeys) {
-    const int nk = min(kPfAttnKeys, n_keys - kb);
-    const size_t off = kv_row(m, sl, layer, g, kb);  // a 64-key block lies in one page
-    const uint16_t* K = m.kcache + off;
-    const uint16_t* V = m.vcache + off;
-    __syncthreads();
-    const int vec = nk * d / 8;
-    for (int i = threadIdx.x; i < vec; i += kPfThreads) {
-      reinterpret_cast<uint4*>(ks)[i] = __ldcg(reinterpret_cast<const uint4*>(K) + i);
-      reinterpret_cast<uint4*>(vs)[i] = __ldcg(reinterpret_cast<const uint4*>(V) + i);
-    }
-    __syncthreads();
-    if (!mine) continue;
-    const int lim = min(nk, ps + 1 - kb);  // causal: keys <= the position
-    for (int j0 = 0; j0 < lim; j0 += 4) {
-      const int nj = min(4, lim - j0);
-      {
-        float kv[4][DPL];
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const int jr = attn_key_row<G>(t, lane);
-          if (jr < nj) load_kv_row<DPL>(ks + (size_t)(j0 + jr) * d + lane * DPL, kv[t]);
-          else
-#pragma unroll
-            for (int i = 0; i < DPL; ++i) kv[t][i] = 0.f;
-        }
-        attn_scores4<DPL, G>(st, kv, nj, xb, lane);
-      }
-      float vv[4][DPL];
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        if (t < nj) load_kv_row<DPL>(vs + (size_t)(j0 + t) * d + lane * DPL, vv[t]);
-        else
-#pragma unroll
-          for (int i = 0; i < DPL; ++i) vv[t][i] = 0.f;
-      }
-      attn_update4<DPL, G>(st, vv, xb);
-    }
-  }
-  if (!mine) return;
-  const size_t row = (size_t)(t0 + warp) * p.ldx + (size_t)g * G * d;
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-    const float inv = 1.0f / st.l[h];
-#pragma unroll
-    for (int i = 0; i < DPL; ++i)
-      pf_split3(st.o[h][i] * inv, p.xh, p.xm, p.xl, row + (size_t)h * d + lane * DPL + i);
-  }
-}
-
-template <int DPL>
-__device__ __forceinline__ void pf_attn_g(const PfArgs& p, PfSmem& s, int layer, const int* tl, int g) {
-  switch (p.m.group) {
-    case 1: pf_attn<DPL, 1>(p, s, layer, tl, g); break;
-    case 2: pf_attn<DPL, 2>(p, s, layer, tl, g); break;
-    case 4: pf_attn<DPL, 4>(p, s, layer, tl, g); break;
-    case 7: if constexpr (DPL == 2) pf_attn<DPL, 7>(p, s, layer, tl, g); break;
-    case 8: if constexpr (DPL == 2) pf_attn<DPL, 8>(p, s, layer, tl, g); break;
-    default: break;
-  }
-}
-
 // ----------------------------------------------------------------- the kernel
 
 __global__ void __launch_bounds__(kPfThreads, 1) prefill_mk_kernel(const __grid_constant__ PfArgs p) {
@@ -419,6 +388,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_mk_kernel(const __grid_
     }
     mbar_init(&s.done, 1);
     for (int i = 0; i < kPfStages; ++i) s.armed[i] = 0xffffffffu;
+    fa_init_barriers(s.fab);
     s.abort_flag = 0;
     s.tmem_ok = 1;
     fence_barrier_init();
@@ -431,13 +401,19 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_mk_kernel(const __grid_
   __syncthreads();
   tc_fence_after_sync();
   PfGemmState gs{0u, 0u};
+  uint32_t fa_tiles = 0, fa_calls = 0;  // key tiles / attention tasks run through s.fab
+  FaBuffers& fab_buf = *reinterpret_cast<FaBuffers*>(&s.a[0][0]);
+  auto fwait = [&](uint64_t* bar, uint32_t parity, int where) { return pf_wait(p, s, bar, parity, where); };
   const int q0 = p.queue_off[blockIdx.x], q1 = p.queue_off[blockIdx.x + 1];
   const int H = m.hidden, F = m.ffn, L = m.n_layers, qd = m.n_q * m.head_dim;
   const int qkvR = qkv_rows(m.n_q, m.n_kv, m.head_dim);
   __shared__ int s_go;
   for (int qi = q0; qi < q1; ++qi) {
-    const PfTask t = p.tasks[p.queue[qi]];
+    const int ti = p.queue[qi];
+    const PfTask t = p.tasks[ti];
+    uint64_t tw0 = 0, tw1 = 0;
     if (threadIdx.x == 0) {
+      if (p.trace) tw0 = globaltimer_ns();
       int go = *(volatile int32_t*)&s.abort_flag == 0;
       if (go && t.wait_ev >= 0) {
         const uint64_t t0 = globaltimer_ns();
@@ -456,28 +432,19 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_mk_kernel(const __grid_
         // tiles read them through the async proxy (TMA)
         fence_proxy_async_global();
       }
+      if (p.trace) tw1 = globaltimer_ns();
       s_go = go;
     }
     __syncthreads();
     if (!s_go) break;
-    const int n = t.n, t0 = n * kPfTokTile, t1 = min(p.T, t0 + kPfTokTile);
+    const int n = t.n, t0 = n * kPfTokTile;
+    // elementwise tasks: positions [e0, e1) of the tile
+    const int e0 = t0 + t.b * kPfEwTok, e1 = min(p.T, e0 + kPfEwTok);
     const int l = t.layer;
     switch (t.kind) {
-      case PF_NORM: {
-        const int HH = H;
-        for (int i = threadIdx.x; i < (t1 - t0) * HH; i += kPfThreads) {
-          const int tt = t0 + i / HH, c = i - (i / HH) * HH;
-          int tok = p.tokens[p.tok_src[tt]];
-          if (tok < 0 || tok >= m.vocab) {
-            if (atomicCAS(m.status, 0, MK_ERR_TOKEN_RANGE) == 0) m.status_info[0] = tok;
-            tok = 0;
-          }
-          p.x[(size_t)tt * H + c] = pf_val(m.embed[(size_t)tok * H + c]);
-        }
-        __syncthreads();
-        pf_norm_rows(p, s, t0, t1, m.attn_norm);
+      case PF_NORM:
+        pf_residual_norm(p, s, e0, e1, false, m.attn_norm);
         break;
-      }
       case PF_GEMM: {
         const int mat = t.a, m0 = t.b * kPfRows;
         const CUtensorMap* tm_w = p.maps + 4 * l + mat;
@@ -492,30 +459,45 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_mk_kernel(const __grid_
         break;
       }
       case PF_ROPE:
-        pf_rope(p, l, t0, t1);
+        pf_rope(p, l, e0, e1);
         break;
-      case PF_ATTN:
-        if (m.head_dim == 128) pf_attn_g<4>(p, s, l, p.attn_tiles + 4 * t.a, t.b);
-        else pf_attn_g<2>(p, s, l, p.attn_tiles + 4 * t.a, t.b);
-        break;
-      case PF_RES1:
-      case PF_RES2: {
-        for (int i = threadIdx.x; i < (t1 - t0) * H; i += kPfThreads) {
-          const int tt = t0 + i / H, c = i - (i / H) * H;
-          float* xv = p.x + (size_t)tt * H + c;
-          *xv = __ldcg(xv) + __ldcg(p.y + (size_t)tt * p.ldy + c);
-        }
-        __syncthreads();
-        if (t.kind == PF_RES1) pf_norm_rows(p, s, t0, t1, m.ffn_norm + (size_t)l * H);
-        else if (l + 1 < L) pf_norm_rows(p, s, t0, t1, m.attn_norm + (size_t)(l + 1) * H);
+      case PF_ATTN: {
+        const int* tl = p.attn_tiles + 4 * t.a;
+        FaJob j;
+        j.mk0 = p.maps + pf_kvmap(L, 0);
+        j.mk1 = p.maps + pf_kvmap(L, 1);
+        j.mv0 = p.maps + pf_kvmap(L, 2);
+        j.mv1 = p.maps + pf_kvmap(L, 3);
+        j.q = p.q;
+        j.ldq = qd;
+        j.oh = p.xh; j.om = p.xm; j.ol = p.xl;
+        j.ldo = p.ldx;
+        j.layer = l;
+        j.qscale = p.qscale;
+        j.t0 = tl[0]; j.nrows = tl[1]; j.slot = tl[2]; j.p0 = tl[3]; j.h = t.b;
+        bool ok;
+        if (m.head_dim == 128) ok = fa_tile<128>(m, j, fab_buf, s.fab, s.tmem, fa_tiles, fwait);
+        else ok = fa_tile<64>(m, j, fab_buf, s.fab, s.tmem, fa_tiles, fwait);
+        if (!ok) *(volatile int32_t*)&s.abort_flag = 1;
+        fa_tiles += (uint32_t)fa_key_tiles(j.p0, j.nrows);
+        fa_calls += 1;
         break;
       }
+      case PF_RES1:
+        pf_residual_norm(p, s, e0, e1, true, m.ffn_norm + (size_t)l * H);
+        break;
+      case PF_RES2:
+        pf_residual_norm(p, s, e0, e1, true, l + 1 < L ? m.attn_norm + (size_t)(l + 1) * H : nullptr);
+        break;
       case PF_SWIGLU: {
-        for (int i = threadIdx.x; i < (t1 - t0) * F; i += kPfThreads) {
-          const int tt = t0 + i / F, j = i - (i / F) * F;
-          const float g = __ldcg(p.y + (size_t)tt * p.ldy + 2 * j);
-          const float u = __ldcg(p.y + (size_t)tt * p.ldy + 2 * j + 1);
-          pf_split3(g / (1.0f + expf(-g)) * u, p.xh, p.xm, p.xl, (size_t)tt * p.ldx + j);
+        // rows [e0, e1): gate/up interleaved in y, two outputs per thread and step
+        const int F2 = F >> 1;
+        for (int i = threadIdx.x; i < (e1 - e0) * F2; i += kPfThreads) {
+          const int tt = e0 + i / F2, j = 2 * (i - (i / F2) * F2);
+          const float4 gu = __ldcg(reinterpret_cast<const float4*>(p.y + (size_t)tt * p.ldy + 2 * j));
+          const size_t o = (size_t)tt * p.ldx + j;
+          pf_split3(gu.x / (1.0f + expf(-gu.x)) * gu.y, p.xh, p.xm, p.xl, o);
+          pf_split3(gu.z / (1.0f + expf(-gu.z)) * gu.w, p.xh, p.xm, p.xl, o + 1);
         }
         break;
       }
@@ -527,6 +509,15 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_mk_kernel(const __grid_
       fence_acq_rel_gpu();
       for (int e = 0; e < t.n_sig; ++e) red_relaxed_gpu_add(p.events + t.sig_ev0 + e, 1u);
     }
+    if (threadIdx.x == 0 && p.trace && ti < p.trace_cap) {
+      uint64_t* tr = p.trace + 4 * (size_t)ti;
+      tr[0] = tw0;
+      tr[1] = tw1;
+      tr[2] = globaltimer_ns();
+      tr[3] = (uint64_t)blockIdx.x | ((uint64_t)(t.kind & 15) << 16) |
+              ((uint64_t)((t.kind == PF_GEMM ? t.a : 0) & 15) << 20) | ((uint64_t)(t.layer & 255) << 24) |
+              ((uint64_t)(t.n & 0xFFFF) << 32) | ((uint64_t)(t.b & 0xFFFF) << 48);
+    }
   }
   tc_fence_before_sync();
   __syncthreads();
@@ -536,6 +527,10 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_mk_kernel(const __grid_
     for (int i = 0; i < kPfStages; ++i)
       if (s.armed[i] != 0xffffffffu) pf_drain(&s.full[i], (s.armed[i] / kPfStages) & 1);
     if (!s.tmem_ok && gs.tiles > 0 && pf_drain(&s.done, (gs.tiles - 1) & 1)) s.tmem_ok = 1;
+    // the attention tasks' loads and MMAs
+    for (int i = 0; i < 2; ++i)
+      if (s.fab.armed[i] != 0xffffffffu) pf_drain(&s.fab.kv_full[i], (s.fab.armed[i] >> 1) & 1);
+    if (fa_calls > 0 && !pf_drain(&s.fab.fin, (fa_calls - 1) & 1)) s.tmem_ok = 0;
   }
   tc_fence_before_sync();
   __syncthreads();
@@ -574,7 +569,7 @@ struct PfGraph {
 // CTAs.  Events per (layer, stage, token tile); a task's wait count is the
 // number of producer tasks it needs.
 void pf_build(const ModelDev& m, int T, const std::vector<int32_t>& attn_tiles, int P, PfGraph& g) {
-  const int L = m.n_layers, H = m.hidden, F = m.ffn, nkv = m.n_kv;
+  const int L = m.n_layers, H = m.hidden, F = m.ffn, nq = m.n_q;
   const int qkvR = qkv_rows(m.n_q, m.n_kv, m.head_dim);
   const int NT = (T + kPfTokTile - 1) / kPfTokTile;
   const int mt_qkv = (qkvR + kPfRows - 1) / kPfRows, mt_h = (H + kPfRows - 1) / kPfRows;
@@ -586,6 +581,11 @@ void pf_build(const ModelDev& m, int T, const std::vector<int32_t>& attn_tiles, 
   std::vector<int> attn_per_tile(NT, 0);
   const int n_attn = (int)attn_tiles.size() / 4;
   for (int a = 0; a < n_attn; ++a) attn_per_tile[attn_tiles[4 * a] / kPfTokTile] += 1;
+  std::vector<int> attn_order(n_attn);
+  for (int a = 0; a < n_attn; ++a) attn_order[a] = a;
+  std::stable_sort(attn_order.begin(), attn_order.end(), [&](int x, int y) {
+    return attn_tiles[4 * x + 1] + attn_tiles[4 * x + 3] > attn_tiles[4 * y + 1] + attn_tiles[4 * y + 3];
+  });
   g.tasks.clear();
   auto add = [&](int kind, int l, int n, int a, int b, int wait_ev, int wait_count, int sig0,
                  int nsig) {
@@ -595,33 +595,43 @@ void pf_build(const ModelDev& m, int T, const std::vector<int32_t>& attn_tiles, 
     g.tasks.push_back(t);
   };
   for (int l = 0; l < L; ++l) {
+    // elementwise stages: kPfEwSub tasks of kPfEwTok positions per token tile
     if (l == 0)
-      for (int n = 0; n < NT; ++n) add(PF_NORM, 0, n, 0, 0, -1, 0, ev(0, E_NORM, n), 1);
+      for (int n = 0; n < NT; ++n)
+        for (int b = 0; b < kPfEwSub; ++b) add(PF_NORM, 0, n, 0, b, -1, 0, ev(0, E_NORM, n), 1);
     for (int n = 0; n < NT; ++n)
       for (int mt = 0; mt < mt_qkv; ++mt)
-        add(PF_GEMM, l, n, PF_QKV, mt, ev(l, E_NORM, n), 1, ev(l, E_QKV, n), 1);
+        add(PF_GEMM, l, n, PF_QKV, mt, ev(l, E_NORM, n), kPfEwSub, ev(l, E_QKV, n), 1);
     // RoPE of tile n counts toward every later tile's "keys ready" event
     for (int n = 0; n < NT; ++n)
-      add(PF_ROPE, l, n, 0, 0, ev(l, E_QKV, n), mt_qkv, ev(l, E_ROPE, n), NT - n);
-    for (int a = 0; a < n_attn; ++a) {
+      for (int b = 0; b < kPfEwSub; ++b)
+        add(PF_ROPE, l, n, 0, b, ev(l, E_QKV, n), mt_qkv, ev(l, E_ROPE, n), NT - n);
+    // per (run, query head); the runs with the most keys first (every task of
+    // the stage depends only on earlier stages, so any order is topological)
+    for (int a : attn_order) {
       const int n = attn_tiles[4 * a] / kPfTokTile;
-      for (int kv = 0; kv < nkv; ++kv)
-        add(PF_ATTN, l, n, a, kv, ev(l, E_ROPE, n), n + 1, ev(l, E_ATTN, n), 1);
+      for (int h = 0; h < nq; ++h)
+        add(PF_ATTN, l, n, a, h, ev(l, E_ROPE, n), kPfEwSub * (n + 1), ev(l, E_ATTN, n), 1);
     }
     for (int n = 0; n < NT; ++n)
       for (int mt = 0; mt < mt_h; ++mt)
-        add(PF_GEMM, l, n, PF_O, mt, ev(l, E_ATTN, n), attn_per_tile[n] * nkv, ev(l, E_O, n), 1);
-    for (int n = 0; n < NT; ++n) add(PF_RES1, l, n, 0, 0, ev(l, E_O, n), mt_h, ev(l, E_RES1, n), 1);
+        add(PF_GEMM, l, n, PF_O, mt, ev(l, E_ATTN, n), attn_per_tile[n] * nq, ev(l, E_O, n), 1);
+    for (int n = 0; n < NT; ++n)
+      for (int b = 0; b < kPfEwSub; ++b)
+        add(PF_RES1, l, n, 0, b, ev(l, E_O, n), mt_h, ev(l, E_RES1, n), 1);
     for (int n = 0; n < NT; ++n)
       for (int mt = 0; mt < mt_gu; ++mt)
-        add(PF_GEMM, l, n, PF_GU, mt, ev(l, E_RES1, n), 1, ev(l, E_GU, n), 1);
-    for (int n = 0; n < NT; ++n) add(PF_SWIGLU, l, n, 0, 0, ev(l, E_GU, n), mt_gu, ev(l, E_SW, n), 1);
+        add(PF_GEMM, l, n, PF_GU, mt, ev(l, E_RES1, n), kPfEwSub, ev(l, E_GU, n), 1);
+    for (int n = 0; n < NT; ++n)
+      for (int b = 0; b < kPfEwSub; ++b)
+        add(PF_SWIGLU, l, n, 0, b, ev(l, E_GU, n), mt_gu, ev(l, E_SW, n), 1);
     for (int n = 0; n < NT; ++n)
       for (int mt = 0; mt < mt_h; ++mt)
-        add(PF_GEMM, l, n, PF_DN, mt, ev(l, E_SW, n), 1, ev(l, E_DN, n), 1);
+        add(PF_GEMM, l, n, PF_DN, mt, ev(l, E_SW, n), kPfEwSub, ev(l, E_DN, n), 1);
     // the residual, then the next layer's attention norm: its E_NORM event
     for (int n = 0; n < NT; ++n)
-      add(PF_RES2, l, n, 0, 0, ev(l, E_DN, n), mt_h, ev(l + 1, E_NORM, n), 1);
+      for (int b = 0; b < kPfEwSub; ++b)
+        add(PF_RES2, l, n, 0, b, ev(l, E_DN, n), mt_h, ev(l + 1, E_NORM, n), 1);
   }
   // queues: the tasks in this (topological) order, dealt round-robin
   std::vector<std::vector<int32_t>> per(P);
@@ -670,7 +680,7 @@ std::string prefill_mk_run(const ModelDev& m, const PrefillWeights& w, PrefillSc
     // the activation parts for K = hidden, n_q d, ffn over all max_tokens rows
     // (token columns past a block's end are computed from stale rows and never
     // stored)
-    std::vector<CUtensorMap> maps((size_t)4 * L + 9);
+    std::vector<CUtensorMap> maps((size_t)4 * L + kPfMapsExtra);
     for (int l = 0; l < L; ++l) {
       if (!pf_make_map(&maps[4 * l + PF_QKV], w.qkv[l], qkvR, H, H) ||
           !pf_make_map(&maps[4 * l + PF_O], w.o[l], H, qd, qd) ||
@@ -684,6 +694,13 @@ std::string prefill_mk_run(const ModelDev& m, const PrefillWeights& w, PrefillSc
       for (int kk = 0; kk < 3; ++kk)
         if (!pf_make_map(&maps[pf_xmap(L, part, kk)], parts[part], sc.max_tokens, kdim[kk], ldx))
           return "prefill megakernel: activation tensor map";
+    // the KV cache for the attention tasks (the same maps as the standalone kernel)
+    std::string fe = flash_attn_prepare(m, &sc.fa);
+    if (!fe.empty()) return fe;
+    maps[pf_kvmap(L, 0)] = sc.fa.k0;
+    maps[pf_kvmap(L, 1)] = sc.fa.k1;
+    maps[pf_kvmap(L, 2)] = sc.fa.v0;
+    maps[pf_kvmap(L, 3)] = sc.fa.v1;
     std::string e0 = pf_grow(&b.maps, &b.maps_cap, maps.size() * sizeof(CUtensorMap), owned);
     if (!e0.empty()) return e0;
     if (cudaMemcpy(b.maps, maps.data(), maps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice) != cudaSuccess)
@@ -707,12 +724,10 @@ std::string prefill_mk_run(const ModelDev& m, const PrefillWeights& w, PrefillSc
       meta[T + t] = slot[b0 + t];
       meta[2 * T + t] = pos[b0 + t];
     }
-    // attention tiles: runs of <= 16 positions of one request inside one token tile
+    // attention tiles: the positions of one request inside one token tile
     for (int t = 0; t < T;) {
       int n = 1;
-      while (t + n < T && n < kPfAttnPos && slot[b0 + t + n] == slot[b0 + t] &&
-             (t + n) % kPfTokTile != 0)
-        ++n;
+      while (t + n < T && slot[b0 + t + n] == slot[b0 + t] && (t + n) % kPfTokTile != 0) ++n;
       tiles.insert(tiles.end(), {t, n, slot[b0 + t], pos[b0 + t]});
       t += n;
     }
@@ -752,6 +767,9 @@ std::string prefill_mk_run(const ModelDev& m, const PrefillWeights& w, PrefillSc
     a.x = sc.x; a.y = sc.y; a.q = sc.q;
     a.xh = sc.xh; a.xm = sc.xm; a.xl = sc.xl;
     a.T = T; a.ldy = ldy; a.ldx = ldx;
+    a.qscale = m.attn_scale * 1.4426950408889634f;
+    a.trace = b0 == 0 ? b.trace : nullptr;
+    a.trace_cap = b.trace_cap;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(num_sms);
     cfg.blockDim = dim3(kPfThreads);

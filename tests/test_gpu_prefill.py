@@ -2,7 +2,8 @@
 
 mk_prefill runs positions 0..len-2 of each prompt as whole-sequence
 operators (tcgen05 GEMMs on bf16 weights and the fp32 activations split into
-two bf16 parts, causal attention over the cache) and the last position as a
+three bf16 parts, causal attention over the cache on the tensor cores; by
+default all of it one persistent kernel per block) and the last position as a
 decode step.  The cache it leaves must be the decode-step prefill's up to the
 tensor cores' accumulation rounding: per cache head a relative L2 difference
 of a few 1e-4 (bf16 entries equal or a step or two apart), and what follows
@@ -88,8 +89,8 @@ def test_tensor_core_attention_matches_cuda_core_attention(cuda_ok, model, lens)
     # two bf16 parts, fp32 accumulation) against the fp32 CUDA-core attention:
     # the caches they leave differ by the accumulation order only
     w = {k: v.cuda() for k, v in synth.make_model(model, 5).items()}
-    a, la, _ = _prefill_opt(model, w, lens, prefill_attention=0)
-    b, lb, _ = _prefill_opt(model, w, lens, prefill_attention=1)
+    a, la, _ = _prefill_opt(model, w, lens, prefill_per_operator=1, prefill_attention=0)
+    b, lb, _ = _prefill_opt(model, w, lens, prefill_per_operator=1, prefill_attention=1)
     for x, y in zip(_cache(a, model, lens), _cache(b, model, lens)):
         assert np.linalg.norm(x - y) <= 2e-3 * np.linalg.norm(y)
         assert np.abs(x - y).max() <= 0.02 * np.abs(y).max()

@@ -1,4 +1,4 @@
-"""The prefill as one persistent kernel (mk_options.prefill_megakernel = 1).
+"""The prefill as one persistent kernel (the default tensor-core prefill).
 
 Every operator of every layer of a block of prompt positions is a task of one
 launch ("LLMs in einen MegaKernel kompilieren ...", "Part 1. Compiler":
@@ -43,8 +43,8 @@ def _prefill(model, w, lens, **kw):
 ], ids=["tiny", "qwen-2l", "llama-2l"])
 def test_persistent_prefill_matches_per_operator_prefill(cuda_ok, model, lens):
     w = {k: v.cuda() for k, v in synth.make_model(model, 4).items()}
-    a, la, _ = _prefill(model, w, lens, prefill_megakernel=1)
-    b, lb, _ = _prefill(model, w, lens)
+    a, la, _ = _prefill(model, w, lens)
+    b, lb, _ = _prefill(model, w, lens, prefill_per_operator=1)
     for x, y in zip(_cache(a, model, lens), _cache(b, model, lens)):
         assert np.linalg.norm(x - y) <= CACHE_REL_L2 * np.linalg.norm(y)
         assert np.abs(x - y).max() <= 0.02 * np.abs(y).max()
@@ -56,7 +56,7 @@ def test_persistent_prefill_then_decode_matches_oracle(cuda_ok):
     w = synth.make_model(model, 6)
     prompt = synth.make_prompt(333, model.vocab, seed=8).tolist()
     tr, _, _ = oracle_trace(model, w, prompt, 4, 340)
-    dec = binding.Decoder(model, {k: v.cuda() for k, v in w.items()}, 340, prefill_megakernel=1)
+    dec = binding.Decoder(model, {k: v.cuda() for k, v in w.items()}, 340)
     gl, gh, gi = run_gpu(dec, model, tr)
     assert_within(compare(tr, gl, gh, gi))
 
@@ -68,7 +68,7 @@ def test_persistent_prefill_past_one_block_against_the_oracles_prefill(cuda_ok):
     P, steps = 2100, 3
     prompt = synth.make_prompt(P, model.vocab, seed=5).tolist()
     tr, om, st = oracle_trace(model, w_cpu, prompt, steps, P + steps)
-    dec = binding.Decoder(model, w, P + steps, prefill_megakernel=1)
+    dec = binding.Decoder(model, w, P + steps)
     gl, gh, gi = run_gpu(dec, model, tr)
     assert_within(compare(tr, gl, gh, gi))
     for positions in (np.arange(0, 130), np.arange(2040, 2056), np.arange(2056, P)):
@@ -89,10 +89,52 @@ def test_persistent_prefill_several_requests_paged(cuda_ok):
     # at 128-position tiles), the cache in 64-position pages
     w = synth.make_model(synth.TINY, 7)
     _run_batch(synth.TINY, w, [5, 170, 9, 300, 1, 129, 23, 64], 4, 310,
-               prefill_megakernel=1, kv_page_tokens=64)
+               kv_page_tokens=64)
 
 
 def test_persistent_prefill_eight_requests_at_llama_widths(cuda_ok):
     model = synth.LLAMA8B.with_layers(2)
     w = synth.make_model(model, 4)
-    _run_batch(model, w, [40, 700, 129, 1, 256, 333, 90, 517], 3, 705, prefill_megakernel=1)
+    _run_batch(model, w, [40, 700, 129, 1, 256, 333, 90, 517], 3, 705)
+
+
+def test_prefill_timeline_records_every_task_in_dependency_order(cuda_ok):
+    # mk_set_prefill_trace: one record per task of the first block, the
+    # timestamps of a task in order, every tile and layer present, sixteen
+    # elementwise tasks per tile and stage, attention after its keys' RoPE
+    model = synth.LLAMA8B.with_layers(2)
+    w = {k: v.cuda() for k, v in synth.make_model(model, 2).items()}
+    P = 300
+    dec = binding.Decoder(model, w, P + 2)
+    tr = torch.zeros(4 * 100000, dtype=torch.int64, device="cuda")
+    dec.set_prefill_trace(tr)
+    toks = synth.make_prompt(P, model.vocab, seed=3).to(torch.int32).cuda()
+    dec.prefill(toks, [0, P], None, None)
+    torch.cuda.synchronize()
+    assert dec.status() == 0, dec.last_error()
+    dec.set_prefill_trace(None)
+    a = tr.view(-1, 4).cpu().numpy().astype(np.uint64)
+    a = a[a[:, 2] != 0]
+    assert len(a) > 0
+    assert np.all(a[:, 0] <= a[:, 1]) and np.all(a[:, 1] <= a[:, 2])
+    d = a[:, 3]
+    kind = (d >> 16) & 15
+    layer = (d >> 24) & 255
+    tile = (d >> 32) & 0xFFFF
+    cta = d & 0xFFFF
+    assert int(cta.max()) < torch.cuda.get_device_properties(0).multi_processor_count
+    n_tiles = (P - 1 + 127) // 128
+    assert set(int(t) for t in tile) == set(range(n_tiles))
+    assert set(int(x) for x in layer) == set(range(model.n_layers))
+    # per layer: 16 tasks per tile for each elementwise stage present
+    for l in range(model.n_layers):
+        for k, stages in ((2, 1), (4, 1), (5, 1), (6, 1)):
+            assert int(np.sum((kind == k) & (layer == l))) == 16 * n_tiles * stages
+    # an attention task of tile n starts only after every RoPE task of tiles
+    # <= n has started (it waits for their completion signals)
+    for l in range(model.n_layers):
+        rope_start = {n: a[(kind == 2) & (layer == l) & (tile == n), 1].max() for n in range(n_tiles)}
+        for n in range(n_tiles):
+            att = a[(kind == 3) & (layer == l) & (tile == n)]
+            assert len(att) > 0
+            assert att[:, 1].min() >= max(rope_start[m] for m in range(n + 1))
