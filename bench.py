@@ -427,8 +427,8 @@ def measure(spec, w, fp8: bool, world: int, local: int, *, full: bool, w_cpu=Non
         "prefill": {"ms": prefill_ms[0], "positions": int(sum(lens)),
                     "positions_per_s": float(sum(lens)) / (prefill_ms[0] * 1e-3),
                     "path": ("one persistent kernel per block of <= 2048 positions (tcgen05 GEMM "
-                             "and attention tasks) for all but each prompt's last position, "
-                             "which runs as a decode step; first call, setup included")},
+                             "and attention tasks), each prompt's last position with its LM head "
+                             "and greedy id inside the kernel; first call, setup included")},
         # one persistent launch per step; the batched step's graph holds an
         # embedding kernel, 7 kernels per layer and 3 for the LM head and argmax
         "gpu_launches": K if n == 1 else K * (7 * model.n_layers + 4),

@@ -161,13 +161,16 @@ int mk_create(const mk_config* cfg, const mk_weights* w, const mk_options* opt, 
  * ("LLM高速化勉強会資料" slides 14-16): request r owns tokens
  * [offsets_host[r], offsets_host[r+1]) of tokens_dev; 1 <= len <= max_seq.
  * Writes the last position's logits (n_req x vocab fp32, may be NULL) and
- * greedy next ids (n_req int32, may be NULL).  By default positions 0..len-2
- * run as whole-sequence operators with the weight contractions on the tensor
- * cores (tcgen05, bf16 weights times the fp32 activations split into two bf16
- * parts, fp32 accumulation) and causal attention over the cache, in blocks of
- * 2048 positions; the last position runs as a decode step.  This path
- * allocates its scratch (~0.4 GB for the Llama-3-8B shape) at the first call
- * and synchronises the stream before returning. */
+ * greedy next ids (n_req int32, may be NULL).  By default every position runs
+ * inside one persistent kernel per block of 2048 positions (the weight
+ * contractions and the causal attention on the tensor cores: tcgen05, bf16
+ * weights times the fp32 activations split into three bf16 parts, fp32
+ * accumulation), the last position's final norm, LM head and greedy id
+ * included; a prompt of one position runs as a decode step.  With
+ * prefill_per_operator = 1 positions 0..len-2 run one launch per operator and
+ * the last as a decode step.  This path allocates its scratch (~0.4 GB for
+ * the Llama-3-8B shape) at the first call and synchronises the stream before
+ * returning. */
 int mk_prefill(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t* offsets_host, int n_req,
                float* last_logits_dev, int32_t* next_ids_dev);
 
@@ -307,6 +310,14 @@ void mk_destroy(mk_ctx* ctx);
  * out of range or the task waits on no event.  The change is permanent:
  * destroy the context afterwards. */
 int mk_inject_stall(mk_ctx* ctx, int task);
+
+/* The same for the persistent prefill: the next mk_prefill[_slots] call
+ * raises by one the wait count of task `task` of its first block's graph (in
+ * the order the mk_set_prefill_trace records list the tasks; -1: the last
+ * task that waits on an event), so that its event never reaches it.  The
+ * prefill's waits are bounded (2 x mk_options.timeout_ms): the call returns
+ * MK_ERR_TIMEOUT and poisons the context.  Testing aid; no GPU fault. */
+int mk_inject_prefill_stall(mk_ctx* ctx, int task);
 
 /* Split-KV grouped-query decode attention for one KV head ("Hạt nhân là gì
  * ...": online softmax, exact up to rounding; "LLM高速化勉強会資料" slides

@@ -30,7 +30,7 @@ EXPORTS = ("mk_create", "mk_prefill", "mk_decode_step", "mk_decode_steps", "mk_d
            "mk_kv_pointer", "mk_copy_kv", "mk_set_mode", "mk_status", "mk_last_error",
            "mk_destroy", "mk_plan_build", "mk_plan_get_info", "mk_plan_get_tasks",
            "mk_plan_get_queue", "mk_plan_get_event_counts", "mk_plan_destroy",
-           "mk_qkv_row_source", "mk_read_probe", "mk_set_trace", "mk_set_prefill_trace",
+           "mk_qkv_row_source", "mk_read_probe", "mk_set_trace", "mk_set_prefill_trace", "mk_inject_prefill_stall",
            "mk_attention_workspace_bytes", "mk_attention_decode",
            "mk_attention_decode_noalloc", "mk_inject_stall")
 
@@ -124,6 +124,7 @@ def lib(build_if_missing: bool = True):
     L.mk_destroy.argtypes = [vp]
     L.mk_destroy.restype = None
     L.mk_inject_stall.argtypes = [vp, i]
+    L.mk_inject_prefill_stall.argtypes = [vp, i]
     L.mk_plan_build.argtypes = [C.POINTER(Config), C.POINTER(Options), i, C.POINTER(vp)]
     L.mk_plan_get_info.argtypes = [vp, C.POINTER(PlanInfo)]
     L.mk_plan_get_tasks.argtypes = [vp, C.POINTER(PlanTask), i]
@@ -362,6 +363,11 @@ class Decoder:
         """Makes one task's event wait unreachable (failure-detection test hook):
         the next megakernel step ends with MK_ERR_TIMEOUT after timeout_ms."""
         _check(lib().mk_inject_stall(self.h, int(task)), self.h)
+
+    def inject_prefill_stall(self, task: int = -1):
+        """The same for the persistent prefill: the next prefill call ends with
+        MK_ERR_TIMEOUT after 2 x timeout_ms."""
+        _check(lib().mk_inject_prefill_stall(self.h, int(task)), self.h)
 
     def last_error(self) -> str:
         return lib().mk_last_error(self.h).decode(errors="replace")

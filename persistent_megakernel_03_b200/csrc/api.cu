@@ -709,24 +709,35 @@ static int prefill_impl(mk_ctx* ctx, const int32_t* tokens_dev, const int32_t* o
   // (its logits and greedy id).  Otherwise every position is a decode step:
   // position t appends its K/V and attends over 0..t.
   const bool gemm_path = ctx->opt.prefill_steps <= 0 && prefill_gemm_supported(ctx->md);
+  PfOutputs out;
   if (gemm_path) {
     if (!ctx->ps.max_tokens) {
       const int cap = std::min(kPrefillBlockTokens, ctx->cfg.max_seq * ctx->cfg.max_batch);
       const std::string e = prefill_alloc(ctx->md, std::max(cap, 1), &ctx->ps, &ctx->allocs);
       if (!e.empty()) return fail(ctx, MK_ERR_CUDA, e);
     }
-    const std::string e =
-        ctx->opt.prefill_per_operator <= 0 && ctx->opt.prefill_attention != 1
-            ? prefill_mk_run(ctx->md, ctx->pw, ctx->ps, ctx->stream, tokens_dev, offsets_host, slots,
-                             n_req, ctx->plan.num_ctas, &ctx->allocs)
-            : prefill_run(ctx->md, ctx->pw, ctx->ps, ctx->stream, tokens_dev, offsets_host, slots,
-                          n_req, ctx->opt.prefill_attention != 1);
+    bool timed_out = false;
+    const bool persistent = ctx->opt.prefill_per_operator <= 0 && ctx->opt.prefill_attention != 1;
+    std::string e;
+    if (persistent) {
+      // the persistent prefill also runs the last positions (LM head, id)
+      out.logits = last_logits_dev;
+      out.ids = next_ids_dev;
+      for (int r = 0; r < n_req; ++r)
+        out.hidden[r] = n_req > 1 ? ctx->hidden_all + (size_t)r * ctx->cfg.hidden : ctx->md.x;
+      e = prefill_mk_run(ctx->md, ctx->pw, ctx->ps, ctx->stream, tokens_dev, offsets_host, slots,
+                         n_req, ctx->plan.num_ctas, &ctx->allocs, &timed_out, &out);
+    } else {
+      e = prefill_run(ctx->md, ctx->pw, ctx->ps, ctx->stream, tokens_dev, offsets_host, slots,
+                      n_req, ctx->opt.prefill_attention != 1, &timed_out);
+    }
     if (!e.empty()) {
       ctx->poisoned = true;
-      return fail(ctx, MK_ERR_CUDA, e);
+      return fail(ctx, timed_out ? MK_ERR_TIMEOUT : MK_ERR_CUDA, e);
     }
   }
   for (int r = 0; r < n_req; ++r) {
+    if (out.folded[r]) continue;  // done inside the persistent prefill
     const int len = offsets_host[r + 1] - offsets_host[r];
     for (int t = gemm_path ? len - 1 : 0; t < len; ++t) {
       StepParams sp{};
@@ -962,6 +973,14 @@ extern "C" int mk_inject_stall(mk_ctx* ctx, int task) {
   cudaError_t e = cudaMemcpyAsync(field, &raised, sizeof raised, cudaMemcpyHostToDevice, ctx->stream);
   if (e == cudaSuccess) e = cudaStreamSynchronize(ctx->stream);
   if (e != cudaSuccess) return fail(ctx, MK_ERR_CUDA, std::string("inject stall: ") + cudaGetErrorString(e));
+  return MK_OK;
+}
+
+extern "C" int mk_inject_prefill_stall(mk_ctx* ctx, int task) {
+  int rc = check_ctx(ctx);
+  if (rc) return rc;
+  if (task < -1) return fail(ctx, MK_ERR_INVALID_ARG, "inject prefill stall: task must be >= -1");
+  ctx->ps.pf.stall_task = task;
   return MK_OK;
 }
 

@@ -978,7 +978,7 @@ std::string prefill_alloc(const ModelDev& m, int max_tokens, PrefillScratch* sc,
       {(void**)&sc->x, T * H * 4},          {(void**)&sc->y, T * ycols * 4},
       {(void**)&sc->q, T * qd * 4},         {(void**)&sc->xh, T * xcols * 2},
       {(void**)&sc->xl, T * xcols * 2},     {(void**)&sc->xm, T * xcols * 2},
-      {(void**)&sc->meta, (3 * T + 4 * T + 16) * 4},
+      {(void**)&sc->meta, (3 * T + 4 * T + T + 16) * 4},
       {(void**)&sc->err, 16}};
   for (auto& a : allocs) {
     const cudaError_t e = cudaMalloc(a.p, a.bytes);
@@ -995,7 +995,8 @@ std::string prefill_alloc(const ModelDev& m, int max_tokens, PrefillScratch* sc,
 
 std::string prefill_run(const ModelDev& m, const PrefillWeights& w, PrefillScratch& sc,
                         cudaStream_t st, const int32_t* tokens_dev, const int32_t* offsets_host,
-                        const int32_t* slots_host, int n_req, bool tc_attn) {
+                        const int32_t* slots_host, int n_req, bool tc_attn, bool* timed_out) {
+  *timed_out = false;
   const int H = m.hidden, F = m.ffn, d = m.head_dim, qd = m.n_q * d, L = m.n_layers;
   const int qkvR = qkv_rows(m.n_q, m.n_kv, d);
   const int ldy = std::max(std::max(qkvR, 2 * F), H);
@@ -1082,7 +1083,10 @@ std::string prefill_run(const ModelDev& m, const PrefillWeights& w, PrefillScrat
   if (cudaMemcpyAsync(&herr, sc.err, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
       cudaStreamSynchronize(st) != cudaSuccess)
     return std::string("prefill: ") + cudaGetErrorString(cudaGetLastError());
-  if (herr) return "prefill: a pipeline wait timed out (GEMM or attention)";
+  if (herr) {
+    *timed_out = true;
+    return "prefill: a pipeline wait timed out (GEMM or attention)";
+  }
   return "";
 }
 

@@ -35,6 +35,18 @@ struct PfBuffers {
   size_t maps_cap = 0, tasks_cap = 0, queue_cap = 0, queue_off_cap = 0, events_cap = 0, err_cap = 0;
   uint64_t* trace = nullptr;   // per-task timeline of the first block (mk_set_prefill_trace)
   int trace_cap = 0;
+  int stall_task = -2;         // mk_inject_prefill_stall: task index, -1 the last waiting, -2 none
+  unsigned long long* lm_keys = nullptr;  // per request: argmax key of its last position
+  size_t lm_keys_cap = 0;
+};
+
+// Where the persistent prefill puts the results of the prompts' last
+// positions (prompts of two or more positions; `folded` reports which).
+struct PfOutputs {
+  float* logits = nullptr;               // [n_req][vocab] or null
+  int32_t* ids = nullptr;                // [n_req] greedy ids or null
+  float* hidden[kMaxBatch] = {};         // per request: its residual stream (hidden) or null
+  bool folded[kMaxBatch] = {};           // out: the request's last position was handled
 };
 
 // Tensor maps of the KV cache for the tensor-core attention (flash_attn.cu):
@@ -115,15 +127,18 @@ std::string prefill_alloc(const ModelDev& m, int max_tokens, PrefillScratch* sc,
 std::string prefill_run(const ModelDev& m, const PrefillWeights& w, PrefillScratch& sc,
                         cudaStream_t st, const int32_t* tokens_dev, const int32_t* offsets_host,
                         const int32_t* slots_host, int n_req,
-                        bool tc_attn);
+                        bool tc_attn, bool* timed_out);
 
 // The same prefill as ONE persistent kernel per block (prefill_mk.cu): every
 // operator of every layer a task, dependencies per (layer, stage, token tile)
-// through event counters, the GEMMs as tcgen05 tiles.  Synchronises `st`.
+// through event counters, the GEMMs as tcgen05 tiles.  Unlike prefill_run it
+// also runs each prompt's LAST position (prompts of two or more positions):
+// the final norm, the LM head and the greedy id, results per `out`.
+// Synchronises `st`.
 std::string prefill_mk_run(const ModelDev& m, const PrefillWeights& w, PrefillScratch& sc,
                            cudaStream_t st, const int32_t* tokens_dev, const int32_t* offsets_host,
                            const int32_t* slots_host, int n_req, int num_sms,
-                           std::vector<void*>* owned);
+                           std::vector<void*>* owned, bool* timed_out, PfOutputs* out);
 
 // Allocates the batched decode scratch (cudaMalloc).
 std::string batch_alloc(const ModelDev& m, int num_sms, BatchScratch* bs, std::vector<void*>* owned);

@@ -22,8 +22,12 @@
 //   GATEUP  GEMM tiles of W_gate/up; wait for RES1 of n
 //   SWIGLU  silu(gate) * up as three parts; waits for GATEUP of n
 //   DOWN    GEMM tiles of W_down; wait for SWIGLU of n
-//   RES2    x += W_down act and the next layer's attention RMSNorm; waits for
-//           DOWN of n
+//   RES2    x += W_down act and the next layer's attention RMSNorm (after the
+//           last layer the final norm); waits for DOWN of n
+//   LM      (tiles holding a prompt's last position) a GEMM tile of 128 rows
+//           of the LM head; writes those positions' logits and folds the
+//           rows' maximum into each request's argmax key; waits for the final
+//           norms of tile n
 // so a token tile runs ahead through the layer while other tiles are still in
 // earlier stages.  Every CTA walks its ahead-of-time queue in this order (all
 // CTAs co-resident, cooperative launch), which keeps the earliest unfinished
@@ -65,12 +69,11 @@ constexpr int kPfK = 64;             // K per stage
 constexpr int kPfStages = 3;
 constexpr int kPfEwTok = 8;          // positions per elementwise task (norm, RoPE, residual, SwiGLU)
 constexpr int kPfEwSub = kPfTokTile / kPfEwTok;  // elementwise tasks per token tile
-constexpr uint64_t kPfWaitNs = 2000000000ull;
 
 enum PfKind : int32_t {
   PF_NORM = 0, PF_GEMM = 1, PF_ROPE = 2, PF_ATTN = 3, PF_RES1 = 4, PF_SWIGLU = 5, PF_RES2 = 6
 };
-enum PfMat : int32_t { PF_QKV = 0, PF_O = 1, PF_GU = 2, PF_DN = 3 };
+enum PfMat : int32_t { PF_QKV = 0, PF_O = 1, PF_GU = 2, PF_DN = 3, PF_LM = 4 };
 
 struct PfTask {
   int32_t kind, layer;
@@ -107,14 +110,29 @@ struct PfArgs {
   int32_t T, ldy, ldx;
   uint64_t* trace;                // per-task timeline (4 words per task index) or null
   int32_t trace_cap;
+  uint64_t wait_ns;               // limit of every wait
+  // the prompts' last positions: LM head and greedy id inside the kernel
+  const int32_t* lm_req;          // [T] request whose last position token t is, or -1
+  unsigned long long* lm_keys;    // [requests] argmax keys (larger value, then lower index)
+  float* logits;                  // [requests][vocab] or null
 };
+
+// Orderable key of (logit, vocabulary index): larger value first, then the
+// lower index (the greedy id's tie rule).
+__device__ __forceinline__ unsigned long long pf_argmax_key(float v, int idx) {
+  uint32_t u = __float_as_uint(v);
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return ((unsigned long long)u << 32) | (0xffffffffu - (uint32_t)idx);
+}
 
 // maps[] index of an activation part (0 high, 1 middle, 2 low) for a GEMM over
 // K = hidden (0), n_q d (1) or ffn (2)
 __host__ __device__ __forceinline__ int pf_xmap(int L, int part, int kk) { return 4 * L + 3 * part + kk; }
 // maps[] index of the KV-cache maps (K first half, K second half, V, V second half)
 __host__ __device__ __forceinline__ int pf_kvmap(int L, int i) { return 4 * L + 9 + i; }
-constexpr int kPfMapsExtra = 13;  // maps past the 4 L weight maps
+// maps[] index of the LM head
+__host__ __device__ __forceinline__ int pf_lmmap(int L) { return 4 * L + 13; }
+constexpr int kPfMapsExtra = 14;  // maps past the 4 L weight maps
 
 struct __align__(1024) PfSmem {
   // GEMM stages (the attention tasks use the same 192 KB as FaBuffers)
@@ -164,7 +182,7 @@ __device__ __forceinline__ bool pf_wait(const PfArgs& p, PfSmem& s, uint64_t* ba
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity)) {
     if (*(volatile int32_t*)&s.abort_flag) return false;
-    if (globaltimer_ns() - t0 > kPfWaitNs) {
+    if (globaltimer_ns() - t0 > p.wait_ns) {
       pf_fail(p, s, MK_ERR_TIMEOUT, where);
       return false;
     }
@@ -250,7 +268,7 @@ struct PfGemmState {
 // tokens of tile n; bias added when given.
 __device__ __forceinline__ void pf_gemm_tile(const PfArgs& p, PfSmem& s, PfGemmState& gs,
                                              const CUtensorMap* tm_w, int kk, int K, int n_rows,
-                                             int m0, int n, const uint16_t* bias) {
+                                             int m0, int n, const uint16_t* bias, bool lm) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nk = K / kPfK;
   const int L = p.m.n_layers;
@@ -320,7 +338,25 @@ __device__ __forceinline__ void pf_gemm_tile(const PfArgs& p, PfSmem& s, PfGemmS
         tmem_ld16(base, v);
         tmem_ld16(base + (uint32_t)kPfTokTile, ml);
         if (odd) tmem_ld16(base + 2u * kPfTokTile, v2);
-        if (row < n_rows) {
+        if (lm) {
+          // LM head: the prompts' last positions only -- their logits, and the
+          // warp's best (logit, row) per request folded into the request's key
+#pragma unroll 1
+          for (int j = 0; j < 16; ++j) {
+            const int tok = n0 + c0 + j;
+            const int req = tok < p.T ? __ldg(p.lm_req + tok) : -1;  // warp-uniform
+            if (req < 0) continue;
+            const float val = (v[j] + (odd ? v2[j] : 0.f)) + ml[j];
+            if (row < n_rows && p.logits) p.logits[(size_t)req * n_rows + row] = val;
+            unsigned long long key = row < n_rows ? pf_argmax_key(val, row) : 0ull;
+#pragma unroll
+            for (int o = 16; o; o >>= 1) {
+              const unsigned long long other = __shfl_xor_sync(0xffffffffu, key, o);
+              key = other > key ? other : key;
+            }
+            if (lane == 0) atomicMax(p.lm_keys + req, key);
+          }
+        } else if (row < n_rows) {
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int tok = n0 + c0 + j;
@@ -421,7 +457,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_mk_kernel(const __grid_
         while (ld_acquire_gpu(p.events + t.wait_ev) < t.wait_count) {
           if ((++spins & 63u) == 0) {
             if (ld_relaxed_gpu_s32(p.err) != 0) { go = 0; break; }
-            if (globaltimer_ns() - t0 > kPfWaitNs) {
+            if (globaltimer_ns() - t0 > p.wait_ns) {
               pf_fail(p, s, MK_ERR_TIMEOUT, qi);
               go = 0;
               break;
@@ -447,15 +483,17 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_mk_kernel(const __grid_
         break;
       case PF_GEMM: {
         const int mat = t.a, m0 = t.b * kPfRows;
-        const CUtensorMap* tm_w = p.maps + 4 * l + mat;
+        const CUtensorMap* tm_w = mat == PF_LM ? p.maps + pf_lmmap(L) : p.maps + 4 * l + mat;
         if (mat == PF_QKV)  // (the bias is added with RoPE)
-          pf_gemm_tile(p, s, gs, tm_w, 0, H, qkvR, m0, n, nullptr);
+          pf_gemm_tile(p, s, gs, tm_w, 0, H, qkvR, m0, n, nullptr, false);
         else if (mat == PF_O)
-          pf_gemm_tile(p, s, gs, tm_w, 1, qd, H, m0, n, nullptr);
+          pf_gemm_tile(p, s, gs, tm_w, 1, qd, H, m0, n, nullptr, false);
         else if (mat == PF_GU)
-          pf_gemm_tile(p, s, gs, tm_w, 0, H, 2 * F, m0, n, nullptr);
-        else
-          pf_gemm_tile(p, s, gs, tm_w, 2, F, H, m0, n, nullptr);
+          pf_gemm_tile(p, s, gs, tm_w, 0, H, 2 * F, m0, n, nullptr, false);
+        else if (mat == PF_DN)
+          pf_gemm_tile(p, s, gs, tm_w, 2, F, H, m0, n, nullptr, false);
+        else  // LM head over the final norm of the tile (the last layer's RES2)
+          pf_gemm_tile(p, s, gs, tm_w, 0, H, m.vocab, m0, n, nullptr, true);
         break;
       }
       case PF_ROPE:
@@ -487,7 +525,10 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_mk_kernel(const __grid_
         pf_residual_norm(p, s, e0, e1, true, m.ffn_norm + (size_t)l * H);
         break;
       case PF_RES2:
-        pf_residual_norm(p, s, e0, e1, true, l + 1 < L ? m.attn_norm + (size_t)(l + 1) * H : nullptr);
+        // the next layer's attention norm, after the last layer the final norm
+        // (the LM head's input)
+        pf_residual_norm(p, s, e0, e1, true,
+                         l + 1 < L ? m.attn_norm + (size_t)(l + 1) * H : m.final_norm);
         break;
       case PF_SWIGLU: {
         // rows [e0, e1): gate/up interleaved in y, two outputs per thread and step
@@ -547,6 +588,13 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_mk_kernel(const __grid_
 
 namespace {
 
+// Greedy ids from the argmax keys of the requests whose last position the
+// kernel handled (mask bit r).
+__global__ void pf_ids_kernel(const unsigned long long* keys, int32_t* ids, uint32_t mask, int n) {
+  const int r = threadIdx.x;
+  if (r < n && ((mask >> r) & 1u)) ids[r] = (int32_t)(0xffffffffu - (uint32_t)(keys[r] & 0xffffffffull));
+}
+
 bool pf_make_map(CUtensorMap* map, const void* base, int rows, int cols, size_t row_stride_elems) {
   auto fn = prefill_encode_fn();
   if (!fn) return false;
@@ -568,7 +616,8 @@ struct PfGraph {
 // The task graph of one block (T tokens, attention tiles as built for it) on P
 // CTAs.  Events per (layer, stage, token tile); a task's wait count is the
 // number of producer tasks it needs.
-void pf_build(const ModelDev& m, int T, const std::vector<int32_t>& attn_tiles, int P, PfGraph& g) {
+void pf_build(const ModelDev& m, int T, const std::vector<int32_t>& attn_tiles,
+              const std::vector<int32_t>& lm_req, int P, PfGraph& g) {
   const int L = m.n_layers, H = m.hidden, F = m.ffn, nq = m.n_q;
   const int qkvR = qkv_rows(m.n_q, m.n_kv, m.head_dim);
   const int NT = (T + kPfTokTile - 1) / kPfTokTile;
@@ -633,6 +682,15 @@ void pf_build(const ModelDev& m, int T, const std::vector<int32_t>& attn_tiles, 
       for (int b = 0; b < kPfEwSub; ++b)
         add(PF_RES2, l, n, 0, b, ev(l, E_DN, n), mt_h, ev(l + 1, E_NORM, n), 1);
   }
+  // the LM head for the tiles holding a prompt's last position: 128 vocabulary
+  // rows per task, after the tile's final norm (the last layer's RES2)
+  const int mt_lm = (m.vocab + kPfRows - 1) / kPfRows;
+  for (int n = 0; n < NT; ++n) {
+    bool any = false;
+    for (int t = n * kPfTokTile; t < std::min(T, (n + 1) * kPfTokTile); ++t) any = any || lm_req[t] >= 0;
+    if (!any) continue;
+    for (int mt = 0; mt < mt_lm; ++mt) add(PF_GEMM, L, n, PF_LM, mt, ev(L, E_NORM, n), kPfEwSub, -1, 0);
+  }
   // queues: the tasks in this (topological) order, dealt round-robin
   std::vector<std::vector<int32_t>> per(P);
   for (size_t i = 0; i < g.tasks.size(); ++i) per[i % P].push_back((int32_t)i);
@@ -663,7 +721,9 @@ size_t prefill_mk_smem_bytes() { return sizeof(PfSmem) + 1024; }
 std::string prefill_mk_run(const ModelDev& m, const PrefillWeights& w, PrefillScratch& sc,
                            cudaStream_t st, const int32_t* tokens_dev, const int32_t* offsets_host,
                            const int32_t* slots_host, int n_req, int num_sms,
-                           std::vector<void*>* owned) {
+                           std::vector<void*>* owned, bool* timed_out, PfOutputs* out) {
+  *timed_out = false;
+  for (int r = 0; r < n_req; ++r) out->folded[r] = false;
   const int H = m.hidden, F = m.ffn, d = m.head_dim, qd = m.n_q * d, L = m.n_layers;
   const int qkvR = qkv_rows(m.n_q, m.n_kv, d);
   const int ldy = std::max(std::max(qkvR, 2 * F), H);
@@ -701,24 +761,38 @@ std::string prefill_mk_run(const ModelDev& m, const PrefillWeights& w, PrefillSc
     maps[pf_kvmap(L, 1)] = sc.fa.k1;
     maps[pf_kvmap(L, 2)] = sc.fa.v0;
     maps[pf_kvmap(L, 3)] = sc.fa.v1;
+    if (!pf_make_map(&maps[pf_lmmap(L)], m.lm_head, m.vocab, H, H))
+      return "prefill megakernel: LM head tensor map";
     std::string e0 = pf_grow(&b.maps, &b.maps_cap, maps.size() * sizeof(CUtensorMap), owned);
     if (!e0.empty()) return e0;
     if (cudaMemcpy(b.maps, maps.data(), maps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice) != cudaSuccess)
       return "prefill megakernel: tensor map upload";
   }
-  // every position but each prompt's last, as (request, position) in order
-  std::vector<int> tok_src, slot, pos;
-  for (int r = 0; r < n_req; ++r)
-    for (int p = 0; p + 1 < offsets_host[r + 1] - offsets_host[r]; ++p) {
+  // every position of each prompt of two or more positions, as (request,
+  // position) in order; a prompt's last position also gets the LM head and
+  // the greedy id here (a one-position prompt is left to the decode step)
+  std::vector<int> tok_src, slot, pos, lmr;
+  for (int r = 0; r < n_req; ++r) {
+    const int len = offsets_host[r + 1] - offsets_host[r];
+    if (len < 2) continue;
+    out->folded[r] = true;
+    for (int p = 0; p < len; ++p) {
       tok_src.push_back(offsets_host[r] + p);
       slot.push_back(slots_host[r]);
       pos.push_back(p);
+      lmr.push_back(p == len - 1 ? r : -1);
     }
+  }
   const int total = (int)tok_src.size();
   std::string e;
+  if (total > 0) {
+    if (!(e = pf_grow(&b.lm_keys, &b.lm_keys_cap, (size_t)kMaxBatch * 8, owned)).empty()) return e;
+    if (cudaMemsetAsync(b.lm_keys, 0, (size_t)kMaxBatch * 8, st) != cudaSuccess)
+      return "prefill megakernel: key reset";
+  }
   for (int b0 = 0; b0 < total; b0 += sc.max_tokens) {
     const int T = std::min(sc.max_tokens, total - b0);
-    std::vector<int32_t> meta(3 * (size_t)T), tiles;
+    std::vector<int32_t> meta(3 * (size_t)T), tiles, lm_req(lmr.begin() + b0, lmr.begin() + b0 + T);
     for (int t = 0; t < T; ++t) {
       meta[t] = tok_src[b0 + t];
       meta[T + t] = slot[b0 + t];
@@ -732,7 +806,17 @@ std::string prefill_mk_run(const ModelDev& m, const PrefillWeights& w, PrefillSc
       t += n;
     }
     PfGraph gr;
-    pf_build(m, T, tiles, num_sms, gr);
+    pf_build(m, T, tiles, lm_req, num_sms, gr);
+    if (b0 == 0 && b.stall_task >= -1) {
+      // failure injection: one more completion than the event will receive
+      int ti = b.stall_task;
+      if (ti == -1)
+        for (int i = (int)gr.tasks.size() - 1; i >= 0 && ti == -1; --i)
+          if (gr.tasks[i].wait_ev >= 0) ti = i;
+      if (ti < 0 || ti >= (int)gr.tasks.size() || gr.tasks[ti].wait_ev < 0)
+        return "inject prefill stall: no such task waiting on an event";
+      gr.tasks[ti].wait_count += 1u;
+    }
     if (!(e = pf_grow(&b.tasks, &b.tasks_cap, gr.tasks.size() * sizeof(PfTask), owned)).empty() ||
         !(e = pf_grow(&b.queue, &b.queue_cap, gr.queue.size() * 4, owned)).empty() ||
         !(e = pf_grow(&b.queue_off, &b.queue_off_cap, gr.queue_off.size() * 4, owned)).empty() ||
@@ -743,8 +827,10 @@ std::string prefill_mk_run(const ModelDev& m, const PrefillWeights& w, PrefillSc
     int32_t* d_slot = sc.meta + T;
     int32_t* d_pos = sc.meta + 2 * T;
     int32_t* d_tiles = sc.meta + 3 * (size_t)sc.max_tokens;
+    int32_t* d_lm_req = sc.meta + 7 * (size_t)sc.max_tokens;
     if (cudaMemcpyAsync(sc.meta, meta.data(), meta.size() * 4, cudaMemcpyHostToDevice, st) != cudaSuccess ||
         cudaMemcpyAsync(d_tiles, tiles.data(), tiles.size() * 4, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(d_lm_req, lm_req.data(), lm_req.size() * 4, cudaMemcpyHostToDevice, st) != cudaSuccess ||
         cudaMemcpyAsync(b.tasks, gr.tasks.data(), gr.tasks.size() * sizeof(PfTask), cudaMemcpyHostToDevice, st) != cudaSuccess ||
         cudaMemcpyAsync(b.queue, gr.queue.data(), gr.queue.size() * 4, cudaMemcpyHostToDevice, st) != cudaSuccess ||
         cudaMemcpyAsync(b.queue_off, gr.queue_off.data(), gr.queue_off.size() * 4, cudaMemcpyHostToDevice, st) != cudaSuccess ||
@@ -769,6 +855,10 @@ std::string prefill_mk_run(const ModelDev& m, const PrefillWeights& w, PrefillSc
     a.T = T; a.ldy = ldy; a.ldx = ldx;
     a.qscale = m.attn_scale * 1.4426950408889634f;
     a.trace = b0 == 0 ? b.trace : nullptr;
+    a.wait_ns = 2ull * (uint64_t)(m.timeout_ms > 0 ? m.timeout_ms : 1000) * 1000000ull;
+    a.lm_req = d_lm_req;
+    a.lm_keys = b.lm_keys;
+    a.logits = out->logits;
     a.trace_cap = b.trace_cap;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(num_sms);
@@ -787,7 +877,24 @@ std::string prefill_mk_run(const ModelDev& m, const PrefillWeights& w, PrefillSc
     if (cudaMemcpyAsync(herr, b.err, 8, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
         cudaStreamSynchronize(st) != cudaSuccess)
       return std::string("prefill megakernel: ") + cudaGetErrorString(cudaGetLastError());
-    if (herr[0]) return "prefill megakernel: a wait timed out (detail " + std::to_string(herr[1]) + ")";
+    if (herr[0]) {
+      *timed_out = herr[0] == MK_ERR_TIMEOUT;
+      return "prefill megakernel: a wait timed out (detail " + std::to_string(herr[1]) + ")";
+    }
+    // the last positions' residual streams (the hidden state after the prompt)
+    for (int t = 0; t < T; ++t) {
+      const int r = lm_req[t];
+      if (r >= 0 && out->hidden[r] &&
+          cudaMemcpyAsync(out->hidden[r], sc.x + (size_t)t * H, (size_t)H * 4, cudaMemcpyDeviceToDevice,
+                          st) != cudaSuccess)
+        return "prefill megakernel: hidden state copy";
+    }
+  }
+  if (total > 0 && out->ids) {
+    uint32_t mask = 0;
+    for (int r = 0; r < n_req; ++r) mask |= out->folded[r] ? 1u << r : 0u;
+    pf_ids_kernel<<<1, 32, 0, st>>>(b.lm_keys, out->ids, mask, n_req);
+    if (cudaGetLastError() != cudaSuccess) return "prefill megakernel: greedy id launch";
   }
   return "";
 }

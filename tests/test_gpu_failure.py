@@ -89,3 +89,44 @@ def dec_plan_tasks(cfg):
     (the same plan mk_create builds)."""
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     return binding.Plan(cfg, 32, sms).tasks()
+
+
+@pytest.mark.parametrize("task", [-1, 0, 500])
+def test_stalled_prefill_task_times_out_and_poisons(cuda_ok, task):
+    # the persistent prefill: one task of the first block's graph can never
+    # see its event; every CTA's bounded wait must end the launch, the call
+    # must return MK_ERR_TIMEOUT within the limit, and the device must stay
+    # usable.  Task -1 is the last waiting task (layer L-1), task 0 the first
+    # elementwise task (no wait: refused), 500 a GEMM tile of layer 0.
+    cfg = synth.LLAMA8B.with_layers(2)
+    w = {k: v.cuda() for k, v in synth.make_model(cfg, 1).items()}
+    prompt = synth.make_prompt(300, cfg.vocab, seed=4)
+    toks = prompt.to(torch.int32).cuda()
+    ids = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ref = binding.Decoder(cfg, w, 310, timeout_ms=TIMEOUT_MS)
+    ref.prefill(toks, [0, 300], None, ids)
+    assert ref.status() == 0, ref.last_error()
+    want = int(ids[0])
+    ref.close()
+    dec = binding.Decoder(cfg, w, 310, timeout_ms=TIMEOUT_MS)
+    dec.inject_prefill_stall(task)
+    t0 = time.monotonic()
+    with pytest.raises(binding.MkError) as err:
+        dec.prefill(toks, [0, 300], None, ids)
+    elapsed = time.monotonic() - t0
+    if task == 0:
+        assert err.value.code == MK_ERR_INVALID_ARG or "no such task" in str(err.value)
+    else:
+        assert err.value.code == MK_ERR_TIMEOUT, str(err.value)
+        assert "timed out" in str(err.value)
+        assert elapsed < 5.0  # 2 x 100 ms per wait
+    with pytest.raises(binding.MkError):  # poisoned
+        dec.prefill(toks, [0, 300], None, ids)
+    dec.close()
+    torch.cuda.synchronize()
+    again = binding.Decoder(cfg, w, 310, timeout_ms=TIMEOUT_MS)
+    ids.zero_()
+    again.prefill(toks, [0, 300], None, ids)
+    assert again.status() == 0, again.last_error()
+    assert int(ids[0]) == want
+    again.close()

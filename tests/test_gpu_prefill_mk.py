@@ -123,9 +123,13 @@ def test_prefill_timeline_records_every_task_in_dependency_order(cuda_ok):
     tile = (d >> 32) & 0xFFFF
     cta = d & 0xFFFF
     assert int(cta.max()) < torch.cuda.get_device_properties(0).multi_processor_count
-    n_tiles = (P - 1 + 127) // 128
+    n_tiles = (P + 127) // 128  # every position, the last one included
     assert set(int(t) for t in tile) == set(range(n_tiles))
-    assert set(int(x) for x in layer) == set(range(model.n_layers))
+    # the layers, then the LM head (layer index n_layers) of the last position's tile
+    assert set(int(x) for x in layer) == set(range(model.n_layers + 1))
+    lm = (kind == 1) & (layer == model.n_layers)
+    assert int(np.sum(lm)) == (model.vocab + 127) // 128
+    assert set(int(t) for t in tile[lm]) == {(P - 1) // 128}
     # per layer: 16 tasks per tile for each elementwise stage present
     for l in range(model.n_layers):
         for k, stages in ((2, 1), (4, 1), (5, 1), (6, 1)):
