@@ -768,19 +768,33 @@ std::string prefill_mk_run(const ModelDev& m, const PrefillWeights& w, PrefillSc
     if (cudaMemcpy(b.maps, maps.data(), maps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice) != cudaSuccess)
       return "prefill megakernel: tensor map upload";
   }
-  // every position of each prompt of two or more positions, as (request,
-  // position) in order; a prompt's last position also gets the LM head and
-  // the greedy id here (a one-position prompt is left to the decode step)
+  // every position but each prompt's last, as (request, position) in order;
+  // then as many last positions (with the LM head and greedy id) as the final
+  // block's last 128-position tile has room for: there they cost next to
+  // nothing, while a tile or block of their own would cost more than the
+  // decode steps the rest get (a tile's GEMMs take ~50 us each whatever the
+  // number of positions in it, a one-tile block ~12 ms for the 8B shape)
   std::vector<int> tok_src, slot, pos, lmr;
-  for (int r = 0; r < n_req; ++r) {
-    const int len = offsets_host[r + 1] - offsets_host[r];
-    if (len < 2) continue;
-    out->folded[r] = true;
-    for (int p = 0; p < len; ++p) {
+  for (int r = 0; r < n_req; ++r)
+    for (int p = 0; p + 1 < offsets_host[r + 1] - offsets_host[r]; ++p) {
       tok_src.push_back(offsets_host[r] + p);
       slot.push_back(slots_host[r]);
       pos.push_back(p);
-      lmr.push_back(p == len - 1 ? r : -1);
+      lmr.push_back(-1);
+    }
+  if (!tok_src.empty()) {
+    const int tn = (int)tok_src.size();
+    const int t_final = tn - ((tn - 1) / sc.max_tokens) * sc.max_tokens;  // tokens of the final block
+    int room = std::min((t_final + kPfTokTile - 1) / kPfTokTile * kPfTokTile, sc.max_tokens) - t_final;
+    for (int r = 0; r < n_req && room > 0; ++r) {
+      const int len = offsets_host[r + 1] - offsets_host[r];
+      if (len < 2) continue;  // a one-position prompt is left to the decode step
+      out->folded[r] = true;
+      tok_src.push_back(offsets_host[r] + len - 1);
+      slot.push_back(slots_host[r]);
+      pos.push_back(len - 1);
+      lmr.push_back(r);
+      --room;
     }
   }
   const int total = (int)tok_src.size();
