@@ -4,8 +4,8 @@
 // chip, an online softmax, key tiles past a query's position skipped).
 //
 // One CTA per (run of <= 128 consecutive prompt positions of one request, query
-// head); the tile itself is fa_tile (flash_attn.cuh).  192 threads: the four
-// softmax warps, the TMA warp, the MMA warp.  Every wait is bounded (2 s); a
+// head); the tile itself is fa_tile (flash_attn.cuh).  320 threads: eight
+// softmax warps (two per row), the TMA warp, the MMA warp.  Every wait is bounded (2 s); a
 // timeout sets the error word, and the CTA releases its tensor memory only
 // once every MMA it issued has retired.
 #include <cuda.h>
@@ -29,7 +29,7 @@ PFN_cuTensorMapEncodeTiled_v12000 prefill_encode_fn();  // prefill.cu
 
 namespace {
 
-constexpr int kFaThreads = 192;
+constexpr int kFaThreads = kFaMinThreads;  // 8 softmax warps, the TMA warp, the MMA warp
 constexpr uint64_t kFaWaitNs = 2000000000ull;
 static_assert(kFaRows == kFaTileRows, "tile rows");
 
@@ -114,8 +114,10 @@ __global__ void __launch_bounds__(kFaThreads, 1)
     // loads still in flight land before the CTA exits
     s.tmem_ok = fa_drain(&s.bar.fin, 0) ? 1 : 0;
     if (*(volatile int32_t*)&s.abort_flag)
-      for (int i = 0; i < 2; ++i)
-        if (s.bar.armed[i] != 0xffffffffu) fa_drain(&s.bar.kv_full[i], (s.bar.armed[i] >> 1) & 1);
+      for (int i = 0; i < 2; ++i) {
+        if (s.bar.armed_k[i] != 0xffffffffu) fa_drain(&s.bar.k_full[i], (s.bar.armed_k[i] >> 1) & 1);
+        if (s.bar.armed_v[i] != 0xffffffffu) fa_drain(&s.bar.v_full[i], (s.bar.armed_v[i] >> 1) & 1);
+      }
   }
   __syncthreads();
   tc_fence_after_sync();

@@ -437,7 +437,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_mk_kernel(const __grid_
   __syncthreads();
   tc_fence_after_sync();
   PfGemmState gs{0u, 0u};
-  uint32_t fa_tiles = 0, fa_calls = 0;  // key tiles / attention tasks run through s.fab
+  uint32_t fa_calls = 0;  // attention tasks run by this CTA
   FaBuffers& fab_buf = *reinterpret_cast<FaBuffers*>(&s.a[0][0]);
   auto fwait = [&](uint64_t* bar, uint32_t parity, int where) { return pf_wait(p, s, bar, parity, where); };
   const int q0 = p.queue_off[blockIdx.x], q1 = p.queue_off[blockIdx.x + 1];
@@ -513,11 +513,20 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_mk_kernel(const __grid_
         j.layer = l;
         j.qscale = p.qscale;
         j.t0 = tl[0]; j.nrows = tl[1]; j.slot = tl[2]; j.p0 = tl[3]; j.h = t.b;
+        // fresh barriers for every attention task: the previous task's last
+        // commit (`fin`) has arrived once its products retired, so no
+        // arrival is pending when they are initialised again
+        if (threadIdx.x == 0) {
+          if (fa_calls > 0 && !pf_wait(p, s, &s.fab.fin, 0, -50))
+            *(volatile int32_t*)&s.abort_flag = 1;
+          fa_init_barriers(s.fab);
+          fence_barrier_init();
+        }
+        __syncthreads();
         bool ok;
-        if (m.head_dim == 128) ok = fa_tile<128>(m, j, fab_buf, s.fab, s.tmem, fa_tiles, fwait);
-        else ok = fa_tile<64>(m, j, fab_buf, s.fab, s.tmem, fa_tiles, fwait);
+        if (m.head_dim == 128) ok = fa_tile<128>(m, j, fab_buf, s.fab, s.tmem, 0u, fwait);
+        else ok = fa_tile<64>(m, j, fab_buf, s.fab, s.tmem, 0u, fwait);
         if (!ok) *(volatile int32_t*)&s.abort_flag = 1;
-        fa_tiles += (uint32_t)fa_key_tiles(j.p0, j.nrows);
         fa_calls += 1;
         break;
       }
@@ -569,9 +578,11 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_mk_kernel(const __grid_
       if (s.armed[i] != 0xffffffffu) pf_drain(&s.full[i], (s.armed[i] / kPfStages) & 1);
     if (!s.tmem_ok && gs.tiles > 0 && pf_drain(&s.done, (gs.tiles - 1) & 1)) s.tmem_ok = 1;
     // the attention tasks' loads and MMAs
-    for (int i = 0; i < 2; ++i)
-      if (s.fab.armed[i] != 0xffffffffu) pf_drain(&s.fab.kv_full[i], (s.fab.armed[i] >> 1) & 1);
-    if (fa_calls > 0 && !pf_drain(&s.fab.fin, (fa_calls - 1) & 1)) s.tmem_ok = 0;
+    for (int i = 0; i < 2; ++i) {
+      if (s.fab.armed_k[i] != 0xffffffffu) pf_drain(&s.fab.k_full[i], (s.fab.armed_k[i] >> 1) & 1);
+      if (s.fab.armed_v[i] != 0xffffffffu) pf_drain(&s.fab.v_full[i], (s.fab.armed_v[i] >> 1) & 1);
+    }
+    if (fa_calls > 0 && !pf_drain(&s.fab.fin, 0)) s.tmem_ok = 0;  // re-initialised per task
   }
   tc_fence_before_sync();
   __syncthreads();
