@@ -91,8 +91,8 @@ struct PfArgs {
   const PfTask* tasks;
   const int32_t* queue;
   const int32_t* queue_off;       // [grid + 1]
-  const CUtensorMap* maps;        // [4 L] weight tiles, [3 parts][3 K kinds] activations, then
-                                  // the KV cache (K, K second half, V, V second half)
+  const CUtensorMap* maps;        // [4 L] weight tiles, [3 parts][3 K kinds] activations, the
+                                  // KV cache (K, K second half, V, V second half), the LM head
   uint32_t* events;
   int32_t* err;                   // [0]: first error code, [1]: detail
   const int32_t* tokens;          // the prompt tokens (device)
