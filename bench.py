@@ -364,13 +364,16 @@ def measure(spec, w, fp8: bool, world: int, local: int, *, full: bool, w_cpu=Non
         # after the first prefill the prompts' cache stays valid: later
         # "prefills" only restore the first generated ids.
         if not first_id:
-            pe0 = torch.cuda.Event(enable_timing=True)
-            pe1 = torch.cuda.Event(enable_timing=True)
-            pe0.record(stream)
-            dec.prefill(prompt, offs, None, ids[0])
-            pe1.record(stream)
-            torch.cuda.synchronize()
-            prefill_ms.append(pe0.elapsed_time(pe1))
+            # twice: the first call includes one-time setup (scratch, tensor
+            # maps, module loading); the second rewrites the same cache rows
+            for _ in range(2):
+                pe0 = torch.cuda.Event(enable_timing=True)
+                pe1 = torch.cuda.Event(enable_timing=True)
+                pe0.record(stream)
+                dec.prefill(prompt, offs, None, ids[0])
+                pe1.record(stream)
+                torch.cuda.synchronize()
+                prefill_ms.append(pe0.elapsed_time(pe1))
             first_id.append(ids[0].clone())
         else:
             ids[0].copy_(first_id[0])
@@ -424,11 +427,13 @@ def measure(spec, w, fp8: bool, world: int, local: int, *, full: bool, w_cpu=Non
                                  if n == 1 and not fp8 and not layers_flag else None),
                      "bytes_per_launch": bytes_mean},
         "clocks": clk.summary(),
-        "prefill": {"ms": prefill_ms[0], "positions": int(sum(lens)),
-                    "positions_per_s": float(sum(lens)) / (prefill_ms[0] * 1e-3),
+        "prefill": {"ms": prefill_ms[1], "first_call_ms": prefill_ms[0],
+                    "positions": int(sum(lens)),
+                    "positions_per_s": float(sum(lens)) / (prefill_ms[1] * 1e-3),
                     "path": ("one persistent kernel per block of <= 2048 positions (tcgen05 GEMM "
                              "and attention tasks), each prompt's last position with its LM head "
-                             "and greedy id inside the kernel; first call, setup included")},
+                             "and greedy id inside the kernel when its tile has room; ms: a second "
+                             "call, first_call_ms: the first, setup included")},
         # one persistent launch per step; the batched step's graph holds an
         # embedding kernel, 7 kernels per layer and 3 for the LM head and argmax
         "gpu_launches": K if n == 1 else K * (7 * model.n_layers + 4),
