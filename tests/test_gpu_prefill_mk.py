@@ -142,3 +142,37 @@ def test_prefill_timeline_records_every_task_in_dependency_order(cuda_ok):
             att = a[(kind == 3) & (layer == l) & (tile == n)]
             assert len(att) > 0
             assert att[:, 1].min() >= max(rope_start[m] for m in range(n + 1))
+
+
+@pytest.mark.parametrize("P,folded", [(129, False), (130, True), (39, True)])
+def test_last_position_folds_only_into_room_in_the_final_tile(cuda_ok, P, folded):
+    # a prompt whose other positions fill the final 128-position tile exactly
+    # (P - 1 = 128) leaves its last position to the decode step: no LM-head
+    # tasks in the kernel; one more position (or a short prompt) folds it in.
+    # Either way the greedy id and logits are the per-operator path's.
+    model = synth.LLAMA8B.with_layers(2)
+    w = {k: v.cuda() for k, v in synth.make_model(model, 2).items()}
+    toks = synth.make_prompt(P, model.vocab, seed=9).to(torch.int32).cuda()
+    dec = binding.Decoder(model, w, P + 2)
+    tr = torch.zeros(4 * 60000, dtype=torch.int64, device="cuda")
+    dec.set_prefill_trace(tr)
+    lg = torch.empty(1, model.vocab, device="cuda")
+    ids = torch.empty(1, dtype=torch.int32, device="cuda")
+    dec.prefill(toks, [0, P], lg, ids)
+    torch.cuda.synchronize()
+    assert dec.status() == 0, dec.last_error()
+    a = tr.view(-1, 4).cpu().numpy().astype(np.uint64)
+    a = a[a[:, 2] != 0]
+    layer = (a[:, 3] >> 24) & 255
+    kind = (a[:, 3] >> 16) & 15
+    assert bool(np.any((kind == 1) & (layer == model.n_layers))) == folded
+    ref = binding.Decoder(model, w, P + 2, prefill_per_operator=1)
+    lg2 = torch.empty(1, model.vocab, device="cuda")
+    ids2 = torch.empty(1, dtype=torch.int32, device="cuda")
+    ref.prefill(toks, [0, P], lg2, ids2)
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(lg.cpu().numpy(), lg2.cpu().numpy(), atol=5e-3, rtol=0)
+    l0 = lg2.cpu().numpy()[0]
+    top = np.sort(l0)[-2:]
+    if top[1] - top[0] >= 0.1:
+        assert int(ids[0]) == int(ids2[0])
