@@ -331,7 +331,7 @@ def oracle_steps(model, w_cpu, lens, first_step: int, n_steps: int, budget_s: fl
 
 def measure(spec, w, fp8: bool, world: int, local: int, *, full: bool, w_cpu=None,
             cpu_budget_s: float = 25.0, trace_path=None, l2_prefetch: int = 0,
-            layers_flag: int = 0) -> dict:
+            layers_flag: int = 0, prefill_per_operator: int = 0) -> dict:
     """One workload on one decoder: W untimed and K device-timed decode steps
     (CUDA events on the launching stream, barrier + synchronize around them,
     max over ranks), the same steps end to end through the host entry point,
@@ -348,6 +348,7 @@ def measure(spec, w, fp8: bool, world: int, local: int, *, full: bool, w_cpu=Non
     wbytes = 1 if fp8 else 2
     stream = torch.cuda.current_stream()
     dec = binding.Decoder(model, w, max_seq, max_batch=n, stream=stream,
+                          prefill_per_operator=prefill_per_operator,
                           l2_prefetch=l2_prefetch, weight_format=1 if fp8 else 0)
     torch.cuda.empty_cache()
     if n == 1:
@@ -569,7 +570,8 @@ def run_mk(args):
     cpu = world == 1 and rank == 0 and not args.no_cpu_baseline
     w_cpu = {k: v.cpu() for k, v in w.items()} if cpu else None
     rec = measure(spec, w, fp8, world, local, full=True, w_cpu=w_cpu, trace_path=args.trace,
-                  l2_prefetch=args.l2_prefetch, layers_flag=args.layers)
+                  l2_prefetch=args.l2_prefetch, layers_flag=args.layers,
+                  prefill_per_operator=1 if args.prefill_per_operator else 0)
     line = {
         "metric": spec.metric, "value": rec["value"], "unit": spec.unit, "n_gpus": world,
         "steps": spec.K, "warmup": spec.W, "ms_per_step": rec["ms_per_step"],
@@ -588,6 +590,8 @@ def run_mk(args):
         line["config"]["workload"] += f" [profiling case: {args.layers} layers]"
     if args.l2_prefetch:
         line["config"]["l2_prefetch_chunks"] = args.l2_prefetch
+    if args.prefill_per_operator:
+        line["config"]["prefill"] = "one launch per operator (profiling aid)"
     # ---- the other workloads, each a sub-record (1 GPU only; not with --layers)
     if (world == 1 and not args.no_workloads and not args.layers and args.workload == "llama8b"
             and not fp8):
@@ -643,6 +647,9 @@ def main():
                          "(not the headline configuration)")
     ap.add_argument("--layers", type=int, default=0,
                     help="profiling aid: a shallower model of the same widths (not a bench line)")
+    ap.add_argument("--prefill-per-operator", action="store_true",
+                    help="profiling aid: the prefill as one launch per operator (its kernels "
+                         "become launches of their own), not the persistent prefill kernel")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
