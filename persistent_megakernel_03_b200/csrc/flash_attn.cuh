@@ -281,11 +281,9 @@ __device__ __forceinline__ bool fa_tile(const ModelDev& m, const FaJob& j, FaBuf
       ok = ok && wait(&bar.s_full[bf], (gi >> 1) & 1, -44);
       if (!fa_softmax_sync_and(ok)) { ok = false; break; }
       tc_fence_after_sync();
+      static_assert(kC == 32, "one 32-column load per half row");
       float sv[kC];
-#pragma unroll
-      for (int c = 0; c < kC; c += 16)
-        tmem_ld16(tS + lane_base + (uint32_t)(bf * kFaKeys + half * kC + c),
-                  *reinterpret_cast<float(*)[16]>(sv + c));
+      tmem_ld32(tS + lane_base + (uint32_t)(bf * kFaKeys + half * kC), sv);
       // causal mask: key k0 + c is visible to this row when k0 + c <= its position
       const int k0 = i * kFaKeys + half * kC;
       float mt = -INFINITY;
