@@ -398,6 +398,25 @@ int mk_plan_get_queue(const mk_plan* p, int cta, int* out, int cap);
 int mk_plan_get_event_counts(const mk_plan* p, int* out, int cap);
 void mk_plan_destroy(mk_plan* p);
 
+/* Host-only inspection of the persistent prefill's task graph (CPU tests):
+ * the graph of ONE block of T prompt positions whose attention runs are
+ * tiles_host [n_tiles][4] (first block position, count, KV slot, first
+ * position: one request's positions inside one 128-position tile) and whose
+ * prompts' last positions are marked in lm_req_host [T] (request index, or
+ * -1), dealt to num_ctas CTAs -- the graph mk_prefill builds for such a block.
+ * Writes min(cap_tasks, n) tasks as 9 int32 each (kind as in
+ * mk_set_prefill_trace, layer (n_layers for the LM head), 128-position tile,
+ * a (GEMM: matrix 0 QKV, 1 O, 2 gate/up, 3 down, 4 LM head; attention: run
+ * index), b (GEMM: 128-row tile; attention: query head; elementwise: 8-position
+ * slice), wait event or -1, wait count, first signalled event, number of
+ * consecutive events signalled), the queue offsets [num_ctas + 1] and the
+ * queues (task indices in run order, at most cap_queue), and the task and
+ * event counts.  MK_ERR_INVALID_ARG on a bad argument. */
+int mk_prefill_graph(const mk_config* cfg, int T, const int32_t* tiles_host, int n_tiles,
+                     const int32_t* lm_req_host, int num_ctas, int32_t* tasks_out, int cap_tasks,
+                     int32_t* queue_off_out, int32_t* queue_out, int cap_queue, int* n_tasks,
+                     int* n_events);
+
 /* Packed-row layout of the fused QKV matrix: the source of packed row r as
  * (which: 0 q, 1 k, 2 v; head; dim).  Rows are grouped per KV head (its G
  * query heads, then its K head, then its V head); inside a q or k head the

@@ -30,7 +30,7 @@ EXPORTS = ("mk_create", "mk_prefill", "mk_decode_step", "mk_decode_steps", "mk_d
            "mk_kv_pointer", "mk_copy_kv", "mk_set_mode", "mk_status", "mk_last_error",
            "mk_destroy", "mk_plan_build", "mk_plan_get_info", "mk_plan_get_tasks",
            "mk_plan_get_queue", "mk_plan_get_event_counts", "mk_plan_destroy",
-           "mk_qkv_row_source", "mk_read_probe", "mk_set_trace", "mk_set_prefill_trace", "mk_inject_prefill_stall",
+           "mk_qkv_row_source", "mk_read_probe", "mk_set_trace", "mk_set_prefill_trace", "mk_inject_prefill_stall", "mk_prefill_graph",
            "mk_attention_workspace_bytes", "mk_attention_decode",
            "mk_attention_decode_noalloc", "mk_inject_stall")
 
@@ -125,6 +125,7 @@ def lib(build_if_missing: bool = True):
     L.mk_destroy.restype = None
     L.mk_inject_stall.argtypes = [vp, i]
     L.mk_inject_prefill_stall.argtypes = [vp, i]
+    L.mk_prefill_graph.argtypes = [vp, i, vp, i, vp, i, vp, i, vp, vp, i, vp, vp]
     L.mk_plan_build.argtypes = [C.POINTER(Config), C.POINTER(Options), i, C.POINTER(vp)]
     L.mk_plan_get_info.argtypes = [vp, C.POINTER(PlanInfo)]
     L.mk_plan_get_tasks.argtypes = [vp, C.POINTER(PlanTask), i]
@@ -162,6 +163,30 @@ def _check(rc: int, h=None):
 
 
 # ------------------------------------------------------------------ plan
+
+def prefill_graph(model, T: int, tiles, lm_req, num_ctas: int):
+    """The persistent prefill's task graph of one block (host only, see
+    mk_prefill_graph): (tasks as rows of 9 ints, queue offsets, queues, number
+    of events)."""
+    L = lib()
+    cfg = make_config(model, max(T, 1), 1)
+    flat = [int(v) for t in tiles for v in t]
+    tiles_c = (C.c_int32 * len(flat))(*flat)
+    lm_c = (C.c_int32 * T)(*[int(v) for v in lm_req])
+    n_tasks, n_events = C.c_int(0), C.c_int(0)
+    rc = L.mk_prefill_graph(C.byref(cfg), T, tiles_c, len(tiles), lm_c, num_ctas, None, 0, None,
+                            None, 0, C.byref(n_tasks), C.byref(n_events))
+    if rc != MK_OK:
+        raise MkError(rc, "mk_prefill_graph rejected the block")
+    n = n_tasks.value
+    tasks = (C.c_int32 * (9 * n))()
+    qoff = (C.c_int32 * (num_ctas + 1))()
+    queue = (C.c_int32 * n)()
+    _check(L.mk_prefill_graph(C.byref(cfg), T, tiles_c, len(tiles), lm_c, num_ctas, tasks, n, qoff,
+                              queue, n, C.byref(n_tasks), C.byref(n_events)))
+    rows = [list(tasks[9 * i:9 * i + 9]) for i in range(n)]
+    return rows, list(qoff), list(queue), n_events.value
+
 
 class Plan:
     """The task graph mk_create would build (host only)."""

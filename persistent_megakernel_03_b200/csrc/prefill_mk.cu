@@ -925,3 +925,42 @@ std::string prefill_mk_run(const ModelDev& m, const PrefillWeights& w, PrefillSc
 }
 
 }  // namespace mk
+
+extern "C" int mk_prefill_graph(const mk_config* cfg, int T, const int32_t* tiles_host, int n_tiles,
+                                const int32_t* lm_req_host, int num_ctas, int32_t* tasks_out,
+                                int cap_tasks, int32_t* queue_off_out, int32_t* queue_out,
+                                int cap_queue, int* n_tasks, int* n_events) {
+  if (!cfg || T <= 0 || !tiles_host || n_tiles <= 0 || !lm_req_host || num_ctas <= 0 ||
+      !n_tasks || !n_events || cfg->n_kv_heads <= 0 || cfg->n_q_heads % cfg->n_kv_heads)
+    return MK_ERR_INVALID_ARG;
+  for (int a = 0; a < n_tiles; ++a) {
+    const int32_t* t = tiles_host + 4 * a;
+    if (t[0] < 0 || t[1] < 1 || t[0] + t[1] > T || t[0] / 128 != (t[0] + t[1] - 1) / 128)
+      return MK_ERR_INVALID_ARG;
+  }
+  mk::ModelDev m{};  // sizes only: the graph depends on nothing else
+  m.n_layers = cfg->n_layers;
+  m.hidden = cfg->hidden;
+  m.ffn = cfg->ffn;
+  m.n_q = cfg->n_q_heads;
+  m.n_kv = cfg->n_kv_heads;
+  m.head_dim = cfg->head_dim;
+  m.group = cfg->n_q_heads / cfg->n_kv_heads;
+  m.vocab = cfg->vocab;
+  const std::vector<int32_t> tiles(tiles_host, tiles_host + 4 * (size_t)n_tiles);
+  const std::vector<int32_t> lm(lm_req_host, lm_req_host + T);
+  mk::PfGraph g;
+  mk::pf_build(m, T, tiles, lm, num_ctas, g);
+  *n_tasks = (int)g.tasks.size();
+  *n_events = g.n_events;
+  for (int i = 0; tasks_out && i < std::min(cap_tasks, *n_tasks); ++i) {
+    const mk::PfTask& t = g.tasks[i];
+    const int32_t v[9] = {t.kind, t.layer, t.n, t.a, t.b, t.wait_ev, (int32_t)t.wait_count,
+                          t.sig_ev0, t.n_sig};
+    for (int k = 0; k < 9; ++k) tasks_out[9 * (size_t)i + k] = v[k];
+  }
+  if (queue_off_out)
+    for (int c = 0; c <= num_ctas; ++c) queue_off_out[c] = g.queue_off[c];
+  for (int i = 0; queue_out && i < std::min(cap_queue, (int)g.queue.size()); ++i) queue_out[i] = g.queue[i];
+  return MK_OK;
+}
