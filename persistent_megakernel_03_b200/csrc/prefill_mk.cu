@@ -276,6 +276,9 @@ __device__ __forceinline__ void pf_gemm_tile(const PfArgs& p, PfSmem& s, PfGemmS
   const CUtensorMap* tmm = p.maps + pf_xmap(L, 1, kk);
   const CUtensorMap* tl = p.maps + pf_xmap(L, 2, kk);
   const int n0 = n * kPfTokTile;
+  // the tile's positions that exist (a block's last tile may be short): the
+  // MMAs' N covers them rounded up to 16, the columns past them are not read
+  const int nmma = (max(1, min(kPfTokTile, p.T - n0)) + 15) & ~15;
   if ((warp == 0 || warp == 2) && lane == 0) {
     // two issuing threads, alternate k blocks (one thread's TMA loads run one
     // after another).  The stage memory may have been written by an attention
@@ -295,7 +298,7 @@ __device__ __forceinline__ void pf_gemm_tile(const PfArgs& p, PfSmem& s, PfGemmS
       tma_load_2d(s.bl[st], tl, i * kPfK, n0, &s.full[st]);
     }
   } else if (warp == 1 && lane == 0) {
-    constexpr uint32_t idesc = mma_idesc_bf16_f32(kPfRows, kPfTokTile);
+    const uint32_t idesc = mma_idesc_bf16_f32(kPfRows, nmma);
     tc_fence_after_sync();
     for (int i = 0; i < nk; ++i) {
       const uint32_t g = gs.kb + i;
@@ -332,7 +335,7 @@ __device__ __forceinline__ void pf_gemm_tile(const PfArgs& p, PfSmem& s, PfGemmS
       const float b = (bias && row < n_rows) ? pf_val(bias[row]) : 0.f;
       const bool odd = nk > 1;
 #pragma unroll 1
-      for (int c0 = 0; c0 < kPfTokTile; c0 += 16) {
+      for (int c0 = 0; c0 < nmma; c0 += 16) {
         float v[16], ml[16], v2[16];
         const uint32_t base = s.tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0;
         tmem_ld16(base, v);
