@@ -46,6 +46,59 @@ def test_create_rejects_bad_config_without_gpu():
     assert b"head_dim" in L.mk_last_error(None)
 
 
+def _fake_weights(model, **override):
+    """Weight structs whose pointers are 16-byte-aligned addresses that are
+    never dereferenced: mk_create checks them before any CUDA call."""
+    import ctypes as C
+    layers = (binding.LayerWeights * model.n_layers)()
+    addr = 0x100000
+    for l in range(model.n_layers):
+        for k in binding.LAYER_FIELDS:
+            setattr(layers[l], k, addr)
+            addr += 0x1000
+    for (l, k), v in override.get("layer", {}).items():
+        setattr(layers[l], k, v)
+    w = binding.Weights(override.get("embed", 0x10000), layers, override.get("final_norm", 0x20000),
+                        override.get("lm_head", 0x30000))
+    return w, layers
+
+
+@pytest.mark.parametrize("case,want_rc,want_msg", [
+    ("no embedding", -1, b"missing weight pointer"),
+    ("no final norm", -1, b"missing weight pointer"),
+    ("no LM head, untied", -1, b"missing weight pointer"),
+    ("null down projection", -1, b"16-byte aligned"),
+    ("misaligned O projection", -1, b"16-byte aligned"),
+    ("bias flag without a bias", -1, b"bias pointer is null"),
+    ("three query heads per KV head", -9, b"query heads per KV head"),
+])
+def test_create_rejects_weights_and_shapes_before_any_launch(case, want_rc, want_msg):
+    # argument errors come back before mk_create touches the device, so these
+    # run without a GPU
+    import ctypes as C
+    import dataclasses
+    L = binding.lib()
+    model = dataclasses.replace(synth.TINY, tied_embeddings=False)
+    override = {
+        "no embedding": {"embed": None},
+        "no final norm": {"final_norm": None},
+        "no LM head, untied": {"lm_head": None},
+        "null down projection": {"layer": {(1, "w_down"): None}},
+        "misaligned O projection": {"layer": {(0, "wo"): 0x100008}},
+    }.get(case, {})
+    if case == "bias flag without a bias":
+        model = dataclasses.replace(model, qkv_bias=True)
+        override = {"layer": {(1, "bk"): None}}
+    if case == "three query heads per KV head":
+        model = dataclasses.replace(model, n_q_heads=6, n_kv_heads=2)
+    w, keep = _fake_weights(model, **override)
+    cfg = binding.make_config(model, 32)
+    h = C.c_void_p()
+    assert L.mk_create(C.byref(cfg), C.byref(w), None, None, C.byref(h)) == want_rc
+    assert want_msg in L.mk_last_error(None)
+    assert not h.value
+
+
 def test_null_context_calls_are_argument_errors_without_gpu():
     L = binding.lib()
     assert L.mk_inject_stall(None, -1) == -1

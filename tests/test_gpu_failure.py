@@ -11,7 +11,7 @@ from persistent_megakernel_03_b200 import binding, synth
 
 pytestmark = pytest.mark.gpu
 
-MK_ERR_INVALID_ARG, MK_ERR_TIMEOUT = -1, -4
+MK_ERR_INVALID_ARG, MK_ERR_TIMEOUT, MK_ERR_NOT_RESIDENT = -1, -4, -6
 TIMEOUT_MS = 100
 
 
@@ -130,3 +130,19 @@ def test_stalled_prefill_task_times_out_and_poisons(cuda_ok, task):
     assert again.status() == 0, again.last_error()
     assert int(ids[0]) == want
     again.close()
+
+
+def test_more_ctas_than_can_be_co_resident_is_refused_before_any_launch(tiny, cuda_ok):
+    # the persistent kernel needs every CTA resident at once: a request for
+    # more CTAs than the device holds is refused by mk_create (no launch), and
+    # the device stays usable
+    cfg, w, prompt = tiny
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    with pytest.raises(binding.MkError) as e:
+        binding.Decoder(cfg, w, 32, num_ctas=4 * sms)
+    assert e.value.code == MK_ERR_NOT_RESIDENT
+    assert "co-resident" in str(e.value)
+    dec, ids = _prefilled(cfg, w, prompt)
+    dec.decode(ids, [len(prompt)])
+    assert dec.status() == 0, dec.last_error()
+    dec.close()
