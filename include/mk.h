@@ -398,6 +398,24 @@ int mk_plan_get_queue(const mk_plan* p, int cta, int* out, int cap);
 int mk_plan_get_event_counts(const mk_plan* p, int* out, int cap);
 void mk_plan_destroy(mk_plan* p);
 
+/* Host-only inspection of how mk_prefill lays out a call's prompt positions
+ * for the persistent prefill (CPU tests).  offsets_host [n_req + 1] as for
+ * mk_prefill (non-decreasing), slots_host [n_req] the requests' KV slots,
+ * max_tokens the block size (positions per launch).  The positions are every
+ * prompt position but each prompt's last, in request order, then the last
+ * positions of prompts of two or more positions, in request order, as many as
+ * the final block's last 128-position tile has room for (those requests'
+ * logits and greedy ids come from the same launch; folded_out [n_req] marks
+ * them).  Writes min(cap_positions, n) positions as 4 int32 each (token index
+ * into the call's tokens, KV slot, position, request for a last position or
+ * -1) and min(cap_runs, m) attention runs as 5 int32 each (block, first
+ * position inside the block, count, KV slot, first position: one request's
+ * positions inside one 128-position tile of a block), and the counts.
+ * MK_ERR_INVALID_ARG on a bad argument. */
+int mk_prefill_layout(const int32_t* offsets_host, const int32_t* slots_host, int n_req,
+                      int max_tokens, int32_t* positions_out, int cap_positions, int32_t* runs_out,
+                      int cap_runs, int* n_positions, int* n_runs, int32_t* folded_out);
+
 /* Host-only inspection of the persistent prefill's task graph (CPU tests):
  * the graph of ONE block of T prompt positions whose attention runs are
  * tiles_host [n_tiles][4] (first block position, count, KV slot, first

@@ -31,6 +31,7 @@ EXPORTS = ("mk_create", "mk_prefill", "mk_decode_step", "mk_decode_steps", "mk_d
            "mk_destroy", "mk_plan_build", "mk_plan_get_info", "mk_plan_get_tasks",
            "mk_plan_get_queue", "mk_plan_get_event_counts", "mk_plan_destroy",
            "mk_qkv_row_source", "mk_read_probe", "mk_set_trace", "mk_set_prefill_trace", "mk_inject_prefill_stall", "mk_prefill_graph",
+           "mk_prefill_layout",
            "mk_attention_workspace_bytes", "mk_attention_decode",
            "mk_attention_decode_noalloc", "mk_inject_stall")
 
@@ -126,6 +127,7 @@ def lib(build_if_missing: bool = True):
     L.mk_inject_stall.argtypes = [vp, i]
     L.mk_inject_prefill_stall.argtypes = [vp, i]
     L.mk_prefill_graph.argtypes = [vp, i, vp, i, vp, i, vp, i, vp, vp, i, vp, vp]
+    L.mk_prefill_layout.argtypes = [vp, vp, i, i, vp, i, vp, i, vp, vp, vp]
     L.mk_plan_build.argtypes = [C.POINTER(Config), C.POINTER(Options), i, C.POINTER(vp)]
     L.mk_plan_get_info.argtypes = [vp, C.POINTER(PlanInfo)]
     L.mk_plan_get_tasks.argtypes = [vp, C.POINTER(PlanTask), i]
@@ -163,6 +165,30 @@ def _check(rc: int, h=None):
 
 
 # ------------------------------------------------------------------ plan
+
+def prefill_layout(offsets, slots, max_tokens: int):
+    """How mk_prefill lays out a call's positions for the persistent prefill
+    (host only, see mk_prefill_layout): (positions as rows of (token index,
+    slot, position, request or -1), attention runs as rows of (block, first
+    block position, count, slot, first position), folded flag per request)."""
+    L = lib()
+    n_req = len(offsets) - 1
+    off_c = (C.c_int32 * len(offsets))(*[int(v) for v in offsets])
+    sl_c = (C.c_int32 * n_req)(*[int(v) for v in slots])
+    n_pos, n_runs = C.c_int(0), C.c_int(0)
+    rc = L.mk_prefill_layout(off_c, sl_c, n_req, max_tokens, None, 0, None, 0, C.byref(n_pos),
+                             C.byref(n_runs), None)
+    if rc != MK_OK:
+        raise MkError(rc, "mk_prefill_layout rejected the call")
+    pos_c = (C.c_int32 * (4 * n_pos.value))()
+    runs_c = (C.c_int32 * (5 * n_runs.value))()
+    fold_c = (C.c_int32 * n_req)()
+    _check(L.mk_prefill_layout(off_c, sl_c, n_req, max_tokens, pos_c, n_pos.value, runs_c,
+                               n_runs.value, C.byref(n_pos), C.byref(n_runs), fold_c))
+    positions = [tuple(pos_c[4 * t:4 * t + 4]) for t in range(n_pos.value)]
+    runs = [tuple(runs_c[5 * i:5 * i + 5]) for i in range(n_runs.value)]
+    return positions, runs, [bool(v) for v in fold_c]
+
 
 def prefill_graph(model, T: int, tiles, lm_req, num_ctas: int):
     """The persistent prefill's task graph of one block (host only, see

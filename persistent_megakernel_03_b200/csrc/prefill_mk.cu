@@ -728,6 +728,55 @@ std::string pf_grow(T** p, size_t* cap, size_t need, std::vector<void*>* owned) 
   return "";
 }
 
+// The positions of one prefill call in the order the kernel takes them: every
+// position but each prompt's last, as (request, position) in request order;
+// then as many last positions (with the LM head and greedy id) as the final
+// block's last 128-position tile has room for: there they cost next to
+// nothing, while a tile or block of their own would cost more than the
+// decode steps the rest get (a tile's GEMMs take ~50 us each whatever the
+// number of positions in it, a one-tile block ~12 ms for the 8B shape).
+struct PfLayout {
+  std::vector<int> tok_src, slot, pos, lmr;  // per position: token index, KV slot, position, request or -1
+  bool folded[kMaxBatch] = {};               // the request's last position is among them
+};
+
+void pf_layout(const int32_t* offsets_host, const int32_t* slots_host, int n_req, int max_tokens,
+               PfLayout* lay) {
+  for (int r = 0; r < n_req; ++r)
+    for (int p = 0; p + 1 < offsets_host[r + 1] - offsets_host[r]; ++p) {
+      lay->tok_src.push_back(offsets_host[r] + p);
+      lay->slot.push_back(slots_host[r]);
+      lay->pos.push_back(p);
+      lay->lmr.push_back(-1);
+    }
+  if (lay->tok_src.empty()) return;
+  const int tn = (int)lay->tok_src.size();
+  const int t_final = tn - ((tn - 1) / max_tokens) * max_tokens;  // positions of the final block
+  int room = std::min((t_final + kPfTokTile - 1) / kPfTokTile * kPfTokTile, max_tokens) - t_final;
+  for (int r = 0; r < n_req && room > 0; ++r) {
+    const int len = offsets_host[r + 1] - offsets_host[r];
+    if (len < 2) continue;  // a one-position prompt is left to the decode step
+    lay->folded[r] = true;
+    lay->tok_src.push_back(offsets_host[r] + len - 1);
+    lay->slot.push_back(slots_host[r]);
+    lay->pos.push_back(len - 1);
+    lay->lmr.push_back(r);
+    --room;
+  }
+}
+
+// Attention runs of the block of positions [b0, b0 + T): the positions of one
+// request inside one token tile, as (first block position, count, KV slot,
+// first position).
+void pf_runs(const PfLayout& lay, int b0, int T, std::vector<int32_t>* tiles) {
+  for (int t = 0; t < T;) {
+    int n = 1;
+    while (t + n < T && lay.slot[b0 + t + n] == lay.slot[b0 + t] && (t + n) % kPfTokTile != 0) ++n;
+    tiles->insert(tiles->end(), {t, n, lay.slot[b0 + t], lay.pos[b0 + t]});
+    t += n;
+  }
+}
+
 }  // namespace
 
 size_t prefill_mk_smem_bytes() { return sizeof(PfSmem) + 1024; }
@@ -782,36 +831,10 @@ std::string prefill_mk_run(const ModelDev& m, const PrefillWeights& w, PrefillSc
     if (cudaMemcpy(b.maps, maps.data(), maps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice) != cudaSuccess)
       return "prefill megakernel: tensor map upload";
   }
-  // every position but each prompt's last, as (request, position) in order;
-  // then as many last positions (with the LM head and greedy id) as the final
-  // block's last 128-position tile has room for: there they cost next to
-  // nothing, while a tile or block of their own would cost more than the
-  // decode steps the rest get (a tile's GEMMs take ~50 us each whatever the
-  // number of positions in it, a one-tile block ~12 ms for the 8B shape)
-  std::vector<int> tok_src, slot, pos, lmr;
-  for (int r = 0; r < n_req; ++r)
-    for (int p = 0; p + 1 < offsets_host[r + 1] - offsets_host[r]; ++p) {
-      tok_src.push_back(offsets_host[r] + p);
-      slot.push_back(slots_host[r]);
-      pos.push_back(p);
-      lmr.push_back(-1);
-    }
-  if (!tok_src.empty()) {
-    const int tn = (int)tok_src.size();
-    const int t_final = tn - ((tn - 1) / sc.max_tokens) * sc.max_tokens;  // tokens of the final block
-    int room = std::min((t_final + kPfTokTile - 1) / kPfTokTile * kPfTokTile, sc.max_tokens) - t_final;
-    for (int r = 0; r < n_req && room > 0; ++r) {
-      const int len = offsets_host[r + 1] - offsets_host[r];
-      if (len < 2) continue;  // a one-position prompt is left to the decode step
-      out->folded[r] = true;
-      tok_src.push_back(offsets_host[r] + len - 1);
-      slot.push_back(slots_host[r]);
-      pos.push_back(len - 1);
-      lmr.push_back(r);
-      --room;
-    }
-  }
-  const int total = (int)tok_src.size();
+  PfLayout lay;
+  pf_layout(offsets_host, slots_host, n_req, sc.max_tokens, &lay);
+  for (int r = 0; r < n_req; ++r) out->folded[r] = lay.folded[r];
+  const int total = (int)lay.tok_src.size();
   std::string e;
   if (total > 0) {
     if (!(e = pf_grow(&b.lm_keys, &b.lm_keys_cap, (size_t)kMaxBatch * 8, owned)).empty()) return e;
@@ -820,19 +843,14 @@ std::string prefill_mk_run(const ModelDev& m, const PrefillWeights& w, PrefillSc
   }
   for (int b0 = 0; b0 < total; b0 += sc.max_tokens) {
     const int T = std::min(sc.max_tokens, total - b0);
-    std::vector<int32_t> meta(3 * (size_t)T), tiles, lm_req(lmr.begin() + b0, lmr.begin() + b0 + T);
+    std::vector<int32_t> meta(3 * (size_t)T), tiles;
+    std::vector<int32_t> lm_req(lay.lmr.begin() + b0, lay.lmr.begin() + b0 + T);
     for (int t = 0; t < T; ++t) {
-      meta[t] = tok_src[b0 + t];
-      meta[T + t] = slot[b0 + t];
-      meta[2 * T + t] = pos[b0 + t];
+      meta[t] = lay.tok_src[b0 + t];
+      meta[T + t] = lay.slot[b0 + t];
+      meta[2 * T + t] = lay.pos[b0 + t];
     }
-    // attention tiles: the positions of one request inside one token tile
-    for (int t = 0; t < T;) {
-      int n = 1;
-      while (t + n < T && slot[b0 + t + n] == slot[b0 + t] && (t + n) % kPfTokTile != 0) ++n;
-      tiles.insert(tiles.end(), {t, n, slot[b0 + t], pos[b0 + t]});
-      t += n;
-    }
+    pf_runs(lay, b0, T, &tiles);
     PfGraph gr;
     pf_build(m, T, tiles, lm_req, num_sms, gr);
     if (b0 == 0 && b.stall_task >= -1) {
@@ -965,5 +983,38 @@ extern "C" int mk_prefill_graph(const mk_config* cfg, int T, const int32_t* tile
   if (queue_off_out)
     for (int c = 0; c <= num_ctas; ++c) queue_off_out[c] = g.queue_off[c];
   for (int i = 0; queue_out && i < std::min(cap_queue, (int)g.queue.size()); ++i) queue_out[i] = g.queue[i];
+  return MK_OK;
+}
+
+extern "C" int mk_prefill_layout(const int32_t* offsets_host, const int32_t* slots_host, int n_req,
+                                 int max_tokens, int32_t* positions_out, int cap_positions,
+                                 int32_t* runs_out, int cap_runs, int* n_positions, int* n_runs,
+                                 int32_t* folded_out) {
+  if (!offsets_host || !slots_host || n_req < 1 || n_req > mk::kMaxBatch || max_tokens < 1 ||
+      !n_positions || !n_runs || offsets_host[0] < 0)
+    return MK_ERR_INVALID_ARG;
+  for (int r = 0; r < n_req; ++r)
+    if (offsets_host[r + 1] < offsets_host[r]) return MK_ERR_INVALID_ARG;
+  mk::PfLayout lay;
+  mk::pf_layout(offsets_host, slots_host, n_req, max_tokens, &lay);
+  const int total = (int)lay.tok_src.size();
+  std::vector<int32_t> runs;
+  for (int b0 = 0; b0 < total; b0 += max_tokens) {
+    std::vector<int32_t> tiles;
+    mk::pf_runs(lay, b0, std::min(max_tokens, total - b0), &tiles);
+    for (size_t i = 0; i < tiles.size(); i += 4)
+      runs.insert(runs.end(), {b0 / max_tokens, tiles[i], tiles[i + 1], tiles[i + 2], tiles[i + 3]});
+  }
+  *n_positions = total;
+  *n_runs = (int)(runs.size() / 5);
+  for (int t = 0; positions_out && t < std::min(cap_positions, total); ++t) {
+    positions_out[4 * (size_t)t] = lay.tok_src[t];
+    positions_out[4 * (size_t)t + 1] = lay.slot[t];
+    positions_out[4 * (size_t)t + 2] = lay.pos[t];
+    positions_out[4 * (size_t)t + 3] = lay.lmr[t];
+  }
+  for (int i = 0; runs_out && i < std::min(cap_runs, *n_runs); ++i)
+    for (int k = 0; k < 5; ++k) runs_out[5 * (size_t)i + k] = runs[5 * (size_t)i + k];
+  for (int r = 0; folded_out && r < n_req; ++r) folded_out[r] = lay.folded[r] ? 1 : 0;
   return MK_OK;
 }

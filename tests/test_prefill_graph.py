@@ -1,6 +1,10 @@
-"""The persistent prefill's task graph, on the host (no GPU).
+"""The persistent prefill's layout and task graph, on the host (no GPU).
 
-mk_prefill_graph returns the graph one block of a prompt gets: its tasks
+mk_prefill_layout returns the order in which a call's prompt positions go
+through the kernel (every position but each prompt's last, then the last
+positions that fit the final block's last 128-position tile) and the
+attention runs of each block; mk_prefill_graph returns the graph one block
+gets: its tasks
 (kind, layer, 128-position tile, a, b, wait event, wait count, signalled
 events) and the per-CTA queues.  The kernel runs each CTA's queue in order,
 a task starting once its event reached its wait count ("LLMs in einen
@@ -22,32 +26,18 @@ MAT_QKV, MAT_O, MAT_GU, MAT_DN, MAT_LM = range(5)
 TILE = 128
 
 
-def _block(lens, fold=True):
-    """One block's positions as the library lays them out: every position but
-    each prompt's last, in request order, then the last positions that fit the
-    final tile's room; attention runs of one request inside one tile."""
-    slot, pos, lm = [], [], []
-    for r, n in enumerate(lens):
-        for p in range(n - 1):
-            slot.append(r)
-            pos.append(p)
-            lm.append(-1)
-    room = (-len(slot)) % TILE if slot else 0
-    for r, n in enumerate(lens):
-        if fold and n >= 2 and room > 0:
-            slot.append(r)
-            pos.append(n - 1)
-            lm.append(r)
-            room -= 1
-    T = len(slot)
-    tiles, t = [], 0
-    while t < T:
-        k = 1
-        while t + k < T and slot[t + k] == slot[t] and pos[t + k] == pos[t] + k and (t + k) % TILE:
-            k += 1
-        tiles.append((t, k, slot[t], pos[t]))
-        t += k
-    return T, tiles, lm
+def _block(lens, max_tokens=2048, block=0):
+    """Block `block` of a call with these prompt lengths, as the library lays
+    it out (mk_prefill_layout): (positions T, attention runs, request per
+    position or -1)."""
+    offs = [0]
+    for n in lens:
+        offs.append(offs[-1] + n)
+    positions, runs, _ = binding.prefill_layout(offs, list(range(len(lens))), max_tokens)
+    b0 = block * max_tokens
+    blk = positions[b0:b0 + max_tokens]
+    tiles = [r[1:] for r in runs if r[0] == block]
+    return len(blk), tiles, [p[3] for p in blk]
 
 
 def _simulate(rows, qoff, queue, n_events, rng):
@@ -148,3 +138,83 @@ def test_no_lm_head_without_a_folded_position():
 def test_rejects_a_run_across_tiles():
     with pytest.raises(binding.MkError):
         binding.prefill_graph(synth.TINY, 200, [(100, 60, 0, 100)], [-1] * 200, 4)
+
+
+def _random_call(rng):
+    n_req = rng.randint(1, 8)
+    lens = [rng.choice([1, 2, rng.randint(1, 40), rng.randint(100, 700), rng.randint(1000, 3000)])
+            for _ in range(n_req)]
+    slots = rng.sample(range(16), n_req)
+    return lens, slots, rng.choice([2048, 2048, 1000, 302, 128])
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_layout_takes_every_position_once_and_folds_only_into_room(seed):
+    rng = random.Random(seed)
+    lens, slots, B = _random_call(rng)
+    offs = [0]
+    for n in lens:
+        offs.append(offs[-1] + n)
+    positions, runs, folded = binding.prefill_layout(offs, slots, B)
+    # every position but each prompt's last, in request order
+    body = [(offs[r] + p, slots[r], p, -1) for r in range(len(lens)) for p in range(lens[r] - 1)]
+    N = len(body)
+    assert positions[:N] == body
+    # then last positions of prompts of two or more positions, in request order
+    tail = positions[N:]
+    eligible = [r for r in range(len(lens)) if lens[r] >= 2]
+    assert [p[3] for p in tail] == eligible[:len(tail)]
+    for tok, slot, pos, r in tail:
+        assert (tok, slot, pos) == (offs[r + 1] - 1, slots[r], lens[r] - 1)
+    assert folded == [r in {p[3] for p in tail} for r in range(len(lens))]
+    if N == 0:
+        assert not tail
+        assert not runs
+        return
+    total = len(positions)
+    # folding adds neither a block nor a 128-position tile, and stops only
+    # when every eligible prompt is in or the final tile is full
+    blocks = lambda n: (n + B - 1) // B
+    assert blocks(total) == blocks(N)
+    last_n, last_t = N - (blocks(N) - 1) * B, total - (blocks(N) - 1) * B
+    assert (last_t + 127) // 128 == (last_n + 127) // 128
+    assert len(tail) == len(eligible) or last_t % 128 == 0 or last_t == B
+    # attention runs: cover each block in order, one request and consecutive
+    # positions inside one 128-position tile, a new run only where the tile or
+    # the request changes
+    for b in range(blocks(total)):
+        T = min(B, total - b * B)
+        rs = [r for r in runs if r[0] == b]
+        t = 0
+        for k, (_, first, count, slot, p0) in enumerate(rs):
+            assert first == t and count >= 1
+            assert first // 128 == (first + count - 1) // 128
+            for i in range(count):
+                _, s_, p_, _ = positions[b * B + first + i]
+                assert (s_, p_) == (slot, p0 + i)
+            if k > 0:
+                prev = rs[k - 1]
+                assert first % 128 == 0 or prev[3] != slot
+            t += count
+        assert t == T
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_graphs_of_random_calls_finish(seed):
+    # layout and graph together, as mk_prefill launches them: every block of a
+    # random call, 148 CTAs
+    rng = random.Random(100 + seed)
+    lens, _, B = _random_call(rng)
+    n_blocks = (sum(max(n - 1, 0) for n in lens) + B - 1) // B
+    for block in range(n_blocks):
+        T, tiles, lm = _block(lens, B, block)
+        rows, qoff, queue, n_events = binding.prefill_graph(synth.TINY, T, tiles, lm, 148)
+        events, waiters, order, stuck = _simulate(rows, qoff, queue, n_events, rng)
+        assert not stuck
+        for e, counts in waiters.items():
+            assert counts == {events[e]}
+
+
+def test_layout_rejects_decreasing_offsets():
+    with pytest.raises(binding.MkError):
+        binding.prefill_layout([0, 10, 5], [0, 1], 2048)
