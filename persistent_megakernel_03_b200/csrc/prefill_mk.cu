@@ -52,6 +52,7 @@
 #include "../../include/mk.h"
 #include "flash_attn.cuh"
 #include "mk_internal.h"
+#include "plan.h"
 #include "prefill.h"
 #include "ptx.cuh"
 #include "tc.cuh"
@@ -952,7 +953,7 @@ extern "C" int mk_prefill_graph(const mk_config* cfg, int T, const int32_t* tile
                                 int cap_tasks, int32_t* queue_off_out, int32_t* queue_out,
                                 int cap_queue, int* n_tasks, int* n_events) {
   if (!cfg || T <= 0 || !tiles_host || n_tiles <= 0 || !lm_req_host || num_ctas <= 0 ||
-      !n_tasks || !n_events || cfg->n_kv_heads <= 0 || cfg->n_q_heads % cfg->n_kv_heads)
+      !n_tasks || !n_events || !mk::validate_config(*cfg).empty())
     return MK_ERR_INVALID_ARG;
   for (int a = 0; a < n_tiles; ++a) {
     const int32_t* t = tiles_host + 4 * a;

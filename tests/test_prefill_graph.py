@@ -218,3 +218,10 @@ def test_graphs_of_random_calls_finish(seed):
 def test_layout_rejects_decreasing_offsets():
     with pytest.raises(binding.MkError):
         binding.prefill_layout([0, 10, 5], [0, 1], 2048)
+
+
+def test_graph_rejects_an_invalid_shape():
+    import dataclasses
+    bad = dataclasses.replace(synth.TINY, head_dim=96)
+    with pytest.raises(binding.MkError):
+        binding.prefill_graph(bad, 10, [(0, 10, 0, 0)], [-1] * 10, 4)
